@@ -1,0 +1,394 @@
+"""Benchmark of the MoE-layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+A step is one pass of the whole layer (router, top-k, histogram/scan, permute, grouped
+gate/up GEMM + SwiGLU, grouped down GEMM x gate, combine, router statistics) over one
+batch of synthetic tokens of the handbook-scale workload (T=8192, d=2048, E=64, k=8,
+F=1024, bf16, fp32 router).  Inputs are resident in HBM; L2 is flushed (256 MB write)
+before every step and each step is timed with CUDA events on the launching stream.
+With N > 1 (torchrun) every rank runs an independent replica on its own token batch
+(the layer has no data-path collective); the timing is the max over ranks.
+
+Prints one JSON line (rank 0).  `--impl reference` times the CPU oracle instead, on a
+bounded token sample of the same workload, on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer fwd tokens/s on 1 B200; grouped-GEMM TFLOP/s; route/permute GB/s"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# DRAM traffic of the dominant kernel (moe_expert_gate_up) per launch, from an ncu capture of
+# the same kernel build (see profiles/); None when the kernel changed since the capture.
+GATE_UP_TRAFFIC = {}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def env_rank():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)), int(os.environ.get("WORLD_SIZE", 1))
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            import tempfile
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.idx), "-lms", "100"], stdout=open(self.path, "w"),
+                                         stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def layer_roofline_ms(cfg, A, pk):
+    """Sum over steps of max(compute, memory) time at the measured peaks (algorithmic bytes / flops)."""
+    T, d, E, k, F = cfg.T, cfg.d, cfg.E, cfg.k, cfg.F
+    hbm = pk["hbm_gbs"] * 1e9
+    tc = pk["bf16_tflops"] * 1e12
+    fp32 = 148 * 128 * 2 * pk.get("sm_max_mhz", 1965.0) * 1e6      # FMA lanes x 2 x clock
+    b = 2
+    steps = {
+        "route": max(2 * T * d * E / fp32, (T * d * b + d * E * 4 + T * E * 4 + T * k * 8) / hbm),
+        "histogram_scan": (T * k * 4 * 3 + A * 8) / hbm,
+        "permute": (T * d * b + A * d * b) / hbm,
+        "gate_up": max(4 * A * d * F / tc, (A * d * b + E * 2 * F * d * b + A * F * b) / hbm),
+        "down": max(2 * A * F * d / tc, (A * F * b + E * d * F * b + A * d * b) / hbm),
+        "combine": (A * d * b + T * d * b) / hbm,
+        "stats": (T * E * 4) / hbm,
+    }
+    return sum(steps.values()) * 1e3, {k_: v * 1e3 for k_, v in steps.items()}
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from routing_dispatch_expert_moe_b200 import inputs as I
+    from routing_dispatch_expert_moe_b200 import moe as M
+    from routing_dispatch_expert_moe_b200.layer import MoELayer, MoEWeights
+
+    rank, local_rank, world = env_rank()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    cfg = I.CONFIGS[args.workload]
+    dt = torch.float32 if cfg.act == "f32" else torch.bfloat16
+    x_np = I.gen_x(cfg, seed=rank)                      # each replica has its own token batch
+    Wg, off, bias = I.gen_router(cfg, 0)
+    W_gu, W_dn = I.gen_experts_torch(cfg, 0)
+    sh = I.gen_shared(cfg, 0)
+    w = MoEWeights(Wg=torch.from_numpy(Wg).to(dev), W_gu=W_gu.to(dev), W_dn=W_dn.to(dev),
+                   logit_offset=None if off is None else torch.from_numpy(off).to(dev),
+                   select_bias=None if bias is None else torch.from_numpy(bias).to(dev),
+                   W_gu_s=None if sh is None else torch.from_numpy(sh[0]).to(dt).unsqueeze(0).to(dev),
+                   W_dn_s=None if sh is None else torch.from_numpy(sh[1]).to(dt).unsqueeze(0).to(dev))
+    del W_gu, W_dn
+    cap = M.moe_capacity(cfg.T, cfg.E, cfg.k, cfg.capacity_factor, True)
+    layer = MoELayer(w, cfg.k, cfg.T, cfg.score, cfg.renormalize, cfg.scale, cap)
+    x = torch.from_numpy(x_np).to(dt).to(dev)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    stage_names = ["route", "histogram_scan", "permute", "gate_up", "down", "shared", "combine", "stats"]
+
+    def step(evs=None):
+        T = cfg.T
+        rec = (lambda i: evs[i].record(stream)) if evs is not None else (lambda i: None)
+        rec(0)
+        layer.route(x)
+        rec(1)
+        layer.histogram_scan(T)
+        rec(2)
+        layer.permute(x)
+        rec(3)
+        layer.gate_up()
+        rec(4)
+        layer.down()
+        rec(5)
+        if layer.has_shared:
+            layer.shared(x)
+        rec(6)
+        layer.combine(T)
+        rec(7)
+        layer.stats(T)
+        rec(8)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    assert M.moe_get_device_error() == 0
+    A = int(layer.offsets[-1].item())
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(9)] for _ in range(args.steps)]
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        step(evs[i])
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    per_step = np.array([evs[i][0].elapsed_time(evs[i][8]) for i in range(args.steps)])   # ms
+    stage_ms = {n: float(np.mean([evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps)]))
+                for j, n in enumerate(stage_names)}
+    total_ms = float(per_step.sum())
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = cfg.T * world * args.steps / (total_ms / 1e3)
+
+    # end to end through the public API with host buffers (pinned), copies inside the timing
+    x_host = torch.from_numpy(x_np).to(dt).pin_memory()
+    y_host = torch.empty((cfg.T, cfg.d), dtype=dt).pin_memory()
+    e2e_steps = max(3, min(args.steps, 50))
+    for _ in range(2):
+        x.copy_(x_host, non_blocking=True)
+        layer.forward(x)
+        y_host.copy_(layer.y, non_blocking=True)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        x.copy_(x_host, non_blocking=True)
+        layer.forward(x)
+        y_host.copy_(layer.y, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = cfg.T * world * e2e_steps / (e2e_ms / 1e3)
+    nbytes = cfg.T * cfg.d * (2 if dt == torch.bfloat16 else 4)
+
+    pk, pk_src = peaks()
+    gate_up_ms = stage_ms["gate_up"]
+    flops = 4.0 * A * cfg.d * cfg.F
+    achieved = flops / (gate_up_ms * 1e-3) / 1e12
+    peak = pk["bf16_tflops"]
+    roof_ms, roof_steps = layer_roofline_ms(cfg, A, pk)
+    traffic = GATE_UP_TRAFFIC.get(args.workload)
+
+    out = None
+    if rank == 0:
+        cpu = cpu_baseline(cfg, budget_s=args.cpu_budget) if (world == 1 and not args.no_cpu_baseline) else None
+        out = {
+            "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if dt == torch.bfloat16 else "f32",
+            "data": "synthetic (seeded; integer-grid router inputs, N(0,0.02) bf16 expert weights)",
+            "config": {"workload": args.workload, "T": cfg.T, "d": cfg.d, "E": cfg.E, "k": cfg.k, "F": cfg.F,
+                       "F_shared": cfg.F_s, "score": cfg.score, "capacity": cap, "rows": A,
+                       "parallelism": f"replicas x{world} (independent token batches, no collective)",
+                       "l2": "flushed before every step (256 MB write)"},
+            "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": nbytes,
+                    "d2h_bytes_per_step": nbytes, "steps": e2e_steps},
+            "gpu_launches": args.steps * layer.launches_per_forward(True),
+            "roofline": {"bound": "tensor", "kernel": "moe_expert_gate_up (tcgen05 grouped GEMM + SwiGLU)",
+                         "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+                         "frac": round(achieved / peak, 4), "traffic": traffic,
+                         "peak_source": f"{pk_src} bf16_tflops (burst)"},
+            "layer_roofline": {"ms": round(roof_ms, 4), "frac": round(roof_ms / ms_per_step, 4),
+                               "tokens_per_s": round(cfg.T / (roof_ms / 1e3), 1)},
+            "stages_ms": {k_: round(v, 4) for k_, v in stage_ms.items()},
+            "stage_roofline_ms": {k_: round(v, 4) for k_, v in roof_steps.items()},
+            "stage_throughput": {
+                "down_tflops": round(2.0 * A * cfg.F * cfg.d / (stage_ms["down"] * 1e-3) / 1e12, 1),
+                "permute_gbs": round((cfg.T * cfg.d * 2 + A * cfg.d * 2) / (stage_ms["permute"] * 1e-3) / 1e9, 1),
+                "combine_gbs": round((A * cfg.d * 2 + cfg.T * cfg.d * 2) / (stage_ms["combine"] * 1e-3) / 1e9, 1),
+                "route_gbs": round((cfg.T * cfg.d * 2 + cfg.T * cfg.E * 8 + cfg.T * cfg.k * 8) /
+                                   (stage_ms["route"] * 1e-3) / 1e9, 1),
+            },
+            "clocks": clk,
+            "cpu_baseline": cpu,
+        }
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return out
+
+
+def _oracle_step(cfg, x_np, Wg, off, bias, gu, dn, sh, tokens):
+    """One oracle pass over a token sample: routing, dispatch plan, expert FFN, combine."""
+    from oracle import moe_oracle as O
+    c = dict(T=len(tokens), E=cfg.E, k=cfg.k, score=cfg.score, renormalize=cfg.renormalize, scale=cfg.scale,
+             capacity_factor=cfg.capacity_factor)
+    xs = x_np[tokens]
+    r = O.layer_routing(c, xs, Wg, off, bias)
+    out = O.layer_outputs_for_tokens(np.arange(len(tokens)), xs, r, gu, dn, cfg.act == "bf16", shared=sh)
+    return out["y"]
+
+
+def _oracle_setup(cfg):
+    from routing_dispatch_expert_moe_b200 import inputs as I
+    x_np = I.gen_x(cfg, 0)
+    Wg, off, bias = I.gen_router(cfg, 0)
+    W_gu, W_dn = I.gen_experts_torch(cfg, 0)
+    gu = {e: W_gu[e].double().numpy() for e in range(cfg.E)}      # model weights as the oracle reads them
+    dn = {e: W_dn[e].double().numpy() for e in range(cfg.E)}
+    sh = I.gen_shared(cfg, 0)
+    return x_np, Wg, off, bias, (lambda e: gu[e]), (lambda e: dn[e]), sh
+
+
+def _threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info()]
+        return max(n) if n else (os.cpu_count() or 1)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(cfg, budget_s=15.0):
+    """The oracle on a bounded token sample of the same workload, timed on the host cores."""
+    setup = _oracle_setup(cfg)
+    rng = np.random.default_rng(1)
+    n = 64
+    tokens = rng.choice(cfg.T, size=n, replace=False)
+    t0 = time.perf_counter()
+    _oracle_step(cfg, *setup, tokens)
+    dt1 = time.perf_counter() - t0
+    n = int(min(cfg.T, max(64, n * budget_s / max(dt1, 1e-3))))
+    tokens = rng.choice(cfg.T, size=n, replace=False)
+    t0 = time.perf_counter()
+    _oracle_step(cfg, *setup, tokens)
+    dt2 = time.perf_counter() - t0
+    return {"value": round(n / dt2, 2), "unit": UNIT, "cores": _threads(), "kind": "oracle",
+            "sample": f"{n} of {cfg.T} tokens (random), full layer per token: routing, dispatch plan, "
+                      f"SwiGLU experts (float64 numpy), combine; {dt2:.1f} s",
+            "host_cpu": _cpu_model(), "nproc": os.cpu_count()}
+
+
+def _cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    return None
+
+
+def run_reference(args):
+    rank, _, world = env_rank()
+    if rank != 0:
+        return None
+    from routing_dispatch_expert_moe_b200 import inputs as I
+    cfg = I.CONFIGS[args.workload]
+    setup = _oracle_setup(cfg)
+    rng = np.random.default_rng(2)
+    n = args.ref_tokens
+    for _ in range(args.warmup):
+        _oracle_step(cfg, *setup, rng.choice(cfg.T, size=n, replace=False))
+    times = []
+    for _ in range(args.steps):
+        tok = rng.choice(cfg.T, size=n, replace=False)
+        t0 = time.perf_counter()
+        _oracle_step(cfg, *setup, tok)
+        times.append(time.perf_counter() - t0)
+    total = float(np.sum(times))
+    value = n * args.steps / total
+    sample = f"{n} of {cfg.T} tokens per step (random), full layer per token, float64 numpy oracle"
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total / args.steps * 1e3, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded)",
+            "config": {"workload": args.workload, "T": cfg.T, "d": cfg.d, "E": cfg.E, "k": cfg.k, "F": cfg.F},
+            "cpu_baseline": {"value": round(value, 2), "unit": UNIT, "cores": _threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 2), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="c2_handbook")
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-tokens", type=int, default=48, help="tokens per reference-arm step")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    out = run_reference(args) if args.impl == "reference" else run_ours(args)
+    if out is not None:
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

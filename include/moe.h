@@ -1,0 +1,257 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) MoE-layer forward library (libmoe_b200.so).
+ *
+ * The library computes the forward pass of a token-choice top-k Mixture-of-Experts
+ * layer on one GPU, one stream-ordered step per call:
+ *
+ *   moe_route            router logits (fp32), scoring, optional selection-only bias,
+ *                        top-k, renormalised and scaled gates
+ *   moe_histogram_scan   per-expert counts, capacity clamp, token-order ranks,
+ *                        expert-contiguous row offsets and the row maps
+ *   moe_permute          gather tokens into expert-contiguous rows
+ *   moe_expert_gate_up   grouped GEMM  H = silu(X Wg^T) * (X Wu^T)       (per expert)
+ *   moe_expert_down      grouped GEMM  Y = gate_of_row * (H Wd^T)       (per expert)
+ *   moe_grouped_ffn      the two GEMMs above back to back
+ *   moe_combine          gate-weighted sum of each token's rows (+ shared expert)
+ *   moe_router_stats     per-expert load, aux loss, z-loss, drops, imbalance
+ *
+ * Sources (web pages on Mixture-of-Experts, cited by title and section):
+ *   [MoE-Explained]  "Hugging Face 图解 Mixture of Experts（MoE）原理、训练与推理权衡"
+ *                    (Chinese rendering of Hugging Face's "Mixture of Experts Explained")
+ *   [Handbook-News]  "Hugging Face 团队投入 ~80 万 GPU 小时…「终极 MoE 训练手册」" (hub.geekagi.cn)
+ *   [Handbook-Digest] "Hugging Face 发布 3 万词免费 MoE 训练手册" (agihunt.info)
+ *   [Handbook-Article] "Hugging Face开源MoE训练手册：基于80万GH200卡时沉淀Megatron-LM实战" (zicq.com)
+ *
+ * Conventions for every call
+ *   - Pointers marked (device) must point to device memory owned by the caller;
+ *     the library allocates nothing and keeps no state except one device error word.
+ *   - All launches are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream).  No call synchronises the host, except moe_get_device_error.
+ *   - Layouts are dense row-major (C order) with the leading dimension equal to the
+ *     row length.  bf16 = IEEE bfloat16 stored in 2 bytes.
+ *   - Arguments are validated on the host before any launch; a failed check returns
+ *     MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED / MOE_ERR_WORKSPACE and launches nothing.
+ *     A launch error returns MOE_ERR_CUDA (moe_last_cuda_error() names it).
+ *   - Corrupt device data (an expert id outside [0,E), a token naming one expert twice,
+ *     a bounded wait that gave up) never traps: the kernel records a MOE_DEVERR_* code
+ *     in the device error word, skips the bad access and finishes; read it with
+ *     moe_get_device_error.
+ *   - Supported sizes: 1 <= E <= 1024, 1 <= k <= min(E, 32), 0 <= T < 2^24,
+ *     d % 8 == 0, F % 8 == 0 (16-byte row strides), device pointers 16-byte aligned.
+ *
+ * Numerical contract
+ *   - Router logits are fp32 sums of fp32(x) * Wg (bf16 x is widened exactly).
+ *   - Top-k selects by the logit (no selection bias) or by score + bias evaluated in
+ *     fp64 (with a selection bias); ties go to the lower expert index; outputs are
+ *     ordered by key descending, then index ascending.
+ *   - Routing indices, counts, offsets and row maps are exact integers and
+ *     deterministic run to run.
+ *   - Expert GEMMs take bf16 operands with fp32 accumulation; H and the gated expert
+ *     rows are rounded to bf16 (round to nearest even); the combine sums in fp32 in
+ *     slot order j = 0..k-1, then adds the shared expert, then rounds.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,  /* null pointer, negative size, k > E, unknown enum, ...   */
+  MOE_ERR_UNSUPPORTED = 2,  /* valid but outside the supported sizes / alignments      */
+  MOE_ERR_WORKSPACE = 3,    /* workspace pointer null or smaller than the query result */
+  MOE_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed                       */
+  MOE_ERR_DEVICE = 5        /* moe_get_device_error found a recorded device error      */
+} moe_status;
+
+typedef enum {
+  MOE_SCORE_SOFTMAX = 0,        /* softmax over experts                 */
+  MOE_SCORE_SIGMOID = 1,        /* 1 / (1 + e^-l) per expert            */
+  MOE_SCORE_SQRT_SOFTPLUS = 2   /* sqrt(log(1 + e^l)) per expert        */
+} moe_score;
+
+typedef enum { MOE_BF16 = 0, MOE_F32 = 1 } moe_dtype;
+
+/* Device error codes recorded by kernels (first one wins until read). */
+#define MOE_DEVERR_NONE 0
+#define MOE_DEVERR_EXPERT_ID 1      /* a topk_idx entry outside [0, E)                   */
+#define MOE_DEVERR_DUP_EXPERT 2     /* one token lists the same expert twice             */
+#define MOE_DEVERR_ROW 3            /* a row index outside its buffer                    */
+#define MOE_DEVERR_SCAN_TIMEOUT 4   /* scan look-back wait gave up (bounded spin)        */
+#define MOE_DEVERR_PIPE_TIMEOUT 5   /* GEMM pipeline barrier wait gave up (bounded spin) */
+
+/* ------------------------------------------------------------------------------------
+ * moe_capacity -- expert capacity in slots.
+ * [MoE-Explained] section "Switch Transformer", eq. Expert Capacity =
+ * (tokens per batch / number of experts) x capacity factor; the overflow rule is in
+ * section "MoE 与 Transformer".
+ *   per_assignment != 0: ceil(cf * T * k / E)   (tokens per batch counted as T*k)
+ *   per_assignment == 0: ceil(cf * T / E)       (the literal top-1 form)
+ * Evaluated in double.  Returns -1 (no dropping) when cf <= 0, and -2 for T < 0,
+ * E < 1 or k < 1.
+ * ---------------------------------------------------------------------------------- */
+MOE_API int32_t moe_capacity(int32_t T, int32_t E, int32_t k, double capacity_factor,
+                     int32_t per_assignment);
+
+/* Rows the permuted buffers must hold: T*k when capacity < 0, else min(T*k, E*capacity). */
+MOE_API int64_t moe_rows_max(int32_t T, int32_t E, int32_t k, int32_t capacity);
+
+/* ------------------------------------------------------------------------------------
+ * moe_route -- router, scoring, top-k and gates.
+ * [MoE-Explained] section "什么是稀疏性？": G_sigma(x) = Softmax(x . W_g),
+ * KeepTopK(v, k), G(x) = Softmax(KeepTopK(H(x), k)); section "Switch Transformer"
+ * (router kept in full precision); [Handbook-News] "真正难在三个环节" item 1 (FP32
+ * routing) and item 2 (loss-free bias), tweet (softmax / sigmoid / sqrt(softplus));
+ * [Handbook-Digest] "已确认" (sqrt(softplus) scoring, scale factor near sqrt(k)).
+ *
+ *   x            (device) [T, d], x_dtype (MOE_BF16 or MOE_F32)
+ *   Wg           (device) [d, E] fp32
+ *   logit_offset (device) [E] fp32 or NULL: added to every logit (enters selection and gates)
+ *   select_bias  (device) [E] fp32 or NULL: added to the score for selection only
+ *   score        moe_score;  renormalize 0/1;  scale multiplies the final gates
+ *   logits       (device) [T, E] fp32 out: x . Wg + logit_offset
+ *   topk_idx     (device) [T, k] int32 out
+ *   topk_gate    (device) [T, k] fp32 out
+ *   workspace    (device) >= moe_route_workspace_bytes(T, d, E) bytes (may be NULL if 0)
+ * Gates: softmax + renormalize -> softmax over the k kept logits; softmax without
+ * renormalize -> the full softmax probability; sigmoid / sqrt(softplus) -> kept scores
+ * over their sum (renormalize) or the scores; all then times scale.
+ * ---------------------------------------------------------------------------------- */
+MOE_API size_t moe_route_workspace_bytes(int32_t T, int32_t d, int32_t E);
+MOE_API moe_status moe_route(const void* x, int32_t x_dtype, const float* Wg,
+                     const float* logit_offset, const float* select_bias,
+                     int32_t T, int32_t d, int32_t E, int32_t k,
+                     int32_t score, int32_t renormalize, float scale,
+                     float* logits, int32_t* topk_idx, float* topk_gate,
+                     void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------------------
+ * moe_histogram_scan -- counts, capacity, token-order ranks, offsets, row maps.
+ * [MoE-Explained] section "MoE 与 Transformer" (an expert takes at most `capacity`
+ * tokens; overflow leaves through the residual or is dropped) and section
+ * "更多关于高效训练的内容" (uneven groups, no padding); [Handbook-Article] (capacity
+ * limit, overflow tokens dropped).
+ *
+ *   topk_idx, topk_gate (device) [T, k]: a token's k experts must be distinct
+ *   capacity     slots per expert, or -1 for no dropping
+ *   counts       (device) [E] int32 out: assignments per expert before dropping
+ *   kept         (device) [E] int32 out: min(counts, capacity)
+ *   offsets      (device) [E+1] int32 out: exclusive scan of kept; offsets[E] = rows used
+ *   row_of       (device) [T, k] int32 out: row of assignment (t, j), or -1 if dropped
+ *   token_of_row (device) [rows_max] int32 out: token of each used row
+ *   gate_of_row  (device) [rows_max] fp32 out: gate of each used row
+ *   workspace    (device) >= moe_histogram_scan_workspace_bytes(T, k, E) bytes; the
+ *                call clears what it needs (one memset node on `stream`).
+ * rank(t, j) = number of tokens t' < t whose top-k holds expert idx[t, j]; the
+ * assignment is kept iff rank < capacity; row_of = offsets[e] + rank.  Rows inside an
+ * expert are in token order.  Entries of token_of_row / gate_of_row at rows >=
+ * offsets[E] are left untouched.
+ * ---------------------------------------------------------------------------------- */
+MOE_API size_t moe_histogram_scan_workspace_bytes(int32_t T, int32_t k, int32_t E);
+MOE_API moe_status moe_histogram_scan(const int32_t* topk_idx, const float* topk_gate,
+                              int32_t T, int32_t k, int32_t E, int32_t capacity,
+                              int32_t* counts, int32_t* kept, int32_t* offsets,
+                              int32_t* row_of, int32_t* token_of_row, float* gate_of_row,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------------------
+ * moe_permute -- x_perm[row_of[t, j]] = x[t] for every kept assignment.
+ * "Send each token to its experts" ([Handbook-News] "MoE 到底省了什么";
+ * [Handbook-Article] dispatch as the real bottleneck).
+ *   x       (device) [T, d] dtype;   row_of (device) [T, k]
+ *   x_perm  (device) [rows_max, d] dtype out (rows >= offsets[E] untouched)
+ *   A row index >= rows_max is skipped and recorded as MOE_DEVERR_ROW.
+ * ---------------------------------------------------------------------------------- */
+MOE_API moe_status moe_permute(const void* x, int32_t dtype, int32_t T, int32_t d, int32_t k,
+                       const int32_t* row_of, int64_t rows_max, void* x_perm, void* stream);
+
+/* ------------------------------------------------------------------------------------
+ * Expert FFN, SwiGLU per expert over expert-contiguous rows.
+ * [MoE-Explained] section "什么是混合专家模型": each expert is an FFN; section
+ * "更多关于高效训练的内容": uneven token counts per expert handled without padding.
+ *
+ *   x_rows   (device) [rows_max, d] dtype: rows [offsets[e], offsets[e+1]) belong to e
+ *   offsets  (device) [E+1] int32 (non-decreasing, offsets[0] = 0, offsets[E] <= rows_max)
+ *   W_gu     (device) [E, 2F, d] dtype: rows 0..F-1 = W_gate[e], rows F..2F-1 = W_up[e]
+ *   W_dn     (device) [E, d, F] dtype
+ *   h        (device) [rows_max, F] dtype: H = silu(x W_gate^T) * (x W_up^T)
+ *   gate_of_row (device) [rows_max] fp32 or NULL (NULL = weight 1, e.g. a shared expert)
+ *   y_rows   (device) [rows_max, d] dtype out: gate_of_row * (H W_dn^T)
+ * bf16 uses the tcgen05 tensor-core path; fp32 uses an fp32 SIMT path.  Rows at or
+ * beyond offsets[E] are neither read into results nor written.
+ * A shared expert is the call with E = 1, offsets = {0, T} and x_rows = x.
+ * ---------------------------------------------------------------------------------- */
+MOE_API moe_status moe_expert_gate_up(const void* x_rows, int32_t dtype, const int32_t* offsets,
+                              int32_t E, int32_t d, int32_t F, int64_t rows_max,
+                              const void* W_gu, void* h, void* stream);
+MOE_API moe_status moe_expert_down(const void* h, int32_t dtype, const int32_t* offsets,
+                           int32_t E, int32_t d, int32_t F, int64_t rows_max,
+                           const void* W_dn, const float* gate_of_row, void* y_rows,
+                           void* stream);
+MOE_API moe_status moe_grouped_ffn(const void* x_rows, int32_t dtype, const int32_t* offsets,
+                           int32_t E, int32_t d, int32_t F, int64_t rows_max,
+                           const void* W_gu, const void* W_dn, const float* gate_of_row,
+                           void* h, void* y_rows, void* stream);
+
+/* ------------------------------------------------------------------------------------
+ * moe_combine -- y[t] = sum_j g_j * y_rows[row_of[t, j]]  (+ shared_y[t]).
+ * [MoE-Explained] section "什么是稀疏性？", eq. y = sum_i G(x)_i E_i(x).
+ *   y_rows    (device) [rows_max, d] dtype
+ *   row_of    (device) [T, k]: -1 slots are skipped (a dropped assignment adds 0)
+ *   topk_gate (device) [T, k] fp32, or NULL when y_rows already carry their gate
+ *   shared_y  (device) [T, d] dtype or NULL: added with weight 1
+ *   y         (device) [T, d] dtype out
+ *   A row index >= rows_max is skipped (adds 0) and recorded as MOE_DEVERR_ROW.
+ * ---------------------------------------------------------------------------------- */
+MOE_API moe_status moe_combine(const void* y_rows, const int32_t* row_of, const float* topk_gate,
+                       const void* shared_y, int32_t dtype, int32_t T, int32_t d, int32_t k,
+                       int64_t rows_max, void* y, void* stream);
+
+/* ------------------------------------------------------------------------------------
+ * moe_router_stats -- load-balance and stability statistics of one routing.
+ * [MoE-Explained] auxiliary load-balancing loss (sections on token load balancing and
+ * "Switch Transformer"), router z-loss (section "使用路由器 Z-loss 稳定训练");
+ * [Handbook-Article] monitoring of max/mean load and drop rate.
+ *   logits (device) [T, E] fp32; counts, kept (device) [E] int32 (from moe_histogram_scan)
+ *   load   (device) [E] fp32 out: f_e = counts[e] / (T k)
+ *   stats5 (device) [5] fp32 out: { aux = E sum_e f_e P_e,  z = mean_t lse_t^2,
+ *          dropped = T k - sum kept,  max_over_mean = max counts / (T k / E),
+ *          cv = std(counts) / mean(counts) }
+ *   P_e is the token-mean of softmax(l) (softmax scoring) or of s / sum_e s.
+ *   workspace (device) >= moe_router_stats_workspace_bytes(T, E) bytes.
+ * ---------------------------------------------------------------------------------- */
+MOE_API size_t moe_router_stats_workspace_bytes(int32_t T, int32_t E);
+MOE_API moe_status moe_router_stats(const float* logits, const int32_t* counts, const int32_t* kept,
+                            int32_t T, int32_t E, int32_t k, int32_t score,
+                            float* load, float* stats5,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+/* Largest workspace any of the calls above needs for these sizes. */
+MOE_API size_t moe_workspace_bytes(int32_t T, int32_t d, int32_t E, int32_t k);
+
+/* Reads and clears the current device's error word (synchronises `stream`).
+ * *code = MOE_DEVERR_*; returns MOE_ERR_DEVICE when *code != 0, else MOE_OK. */
+MOE_API moe_status moe_get_device_error(int32_t* code, void* stream);
+
+/* Human-readable names. */
+MOE_API const char* moe_status_str(int32_t status);
+MOE_API const char* moe_last_cuda_error(void);
+
+/* Library version (major * 10000 + minor * 100 + patch). */
+MOE_API int32_t moe_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_B200_H */

@@ -345,27 +345,26 @@ def layer_outputs_for_tokens(tokens, x, routing: dict, W_gu_of, W_dn_of, bf16: b
     so evaluating a subset gives exactly the rows the full layer would.
     shared: (W_gu_s, W_dn_s) or None.
     """
-    x = np.asarray(x, np.float64)
-    idx, row_of, g = routing["topk_idx"], routing["row_of"], routing["topk_gate"]
-    k = idx.shape[1]
     tokens = np.asarray(tokens, np.int64)
-    d = x.shape[1]
-    y = np.zeros((len(tokens), d), np.float64)
-    slot_rows = np.zeros((len(tokens), k, d), np.float64)
-    for i, t in enumerate(tokens):
-        acc = np.zeros(d, np.float64)
-        for j in range(k):
-            if row_of[t, j] < 0:
-                continue
-            e = int(idx[t, j])
-            o = swiglu_expert(x[t:t + 1], _get(W_gu_of, e), _get(W_dn_of, e), bf16)[0]
-            o = o * g[t, j]
-            o = bf16_round(o) if bf16 else o
-            slot_rows[i, j] = o
-            acc += o
-        if shared is not None:
-            acc += shared_expert(x[t:t + 1], shared[0], shared[1], bf16)[0]
-        y[i] = bf16_round(acc) if bf16 else acc
+    xs = np.asarray(np.asarray(x)[tokens], np.float64)          # the listed tokens only
+    idx = routing["topk_idx"][tokens]
+    row_of = routing["row_of"][tokens]
+    g = np.asarray(routing["topk_gate"], np.float64)[tokens]
+    n, k = idx.shape
+    d = xs.shape[1]
+    slot_rows = np.zeros((n, k, d), np.float64)
+    kept = row_of >= 0
+    for e in np.unique(idx[kept]):                  # every kept (token, slot) of expert e at once
+        ii, jj = np.nonzero((idx == e) & kept)
+        o = swiglu_expert(xs[ii], _get(W_gu_of, int(e)), _get(W_dn_of, int(e)), bf16)
+        o = o * g[ii, jj][:, None]
+        slot_rows[ii, jj] = bf16_round(o) if bf16 else o
+    acc = np.zeros((n, d), np.float64)
+    for j in range(k):                              # slot order; dropped slots are zero rows
+        acc += slot_rows[:, j]
+    if shared is not None:
+        acc += shared_expert(xs, shared[0], shared[1], bf16)
+    y = bf16_round(acc) if bf16 else acc
     return {"y": y, "slot_rows": slot_rows}
 
 

@@ -1,0 +1,248 @@
+// extern "C" entry points of libmoe_b200.so: argument validation, workspace queries,
+// the device error word, and dispatch to the kernel launchers.  See include/moe.h for
+// the contract of every call.
+#include <math.h>
+#include <string.h>
+
+#include "common.cuh"
+
+// The one piece of library state: a per-device error word written by kernels.
+__device__ int g_moe_device_error = 0;
+
+namespace moe {
+
+static thread_local cudaError_t g_last_cuda = cudaSuccess;
+cudaError_t& last_cuda_error_ref() { return g_last_cuda; }
+
+int* err_ptr() {
+  static int* cached[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!cached[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_moe_device_error) == cudaSuccess) cached[dev] = static_cast<int*>(p);
+  }
+  return cached[dev];
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+namespace {
+
+constexpr int kMaxE = 1024;
+constexpr int kMaxK = 32;
+constexpr long long kMaxT = 1LL << 24;
+
+inline cudaStream_t S(void* s) { return static_cast<cudaStream_t>(s); }
+
+bool dtype_ok(int32_t dt) { return dt == MOE_BF16 || dt == MOE_F32; }
+int esize(int32_t dt) { return dt == MOE_F32 ? 4 : 2; }
+
+moe_status check_dims(int32_t T, int32_t E, int32_t k) {
+  if (T < 0 || E < 1 || k < 1 || k > E) return MOE_ERR_INVALID_ARG;
+  if (E > kMaxE || k > kMaxK || (long long)T >= kMaxT) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+moe_status check_d(int32_t d) {
+  if (d < 1) return MOE_ERR_INVALID_ARG;
+  if (d % 8 != 0) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t moe_version(void) { return 10000; }
+
+const char* moe_status_str(int32_t s) {
+  switch (s) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_DEVICE: return "MOE_ERR_DEVICE";
+    default: return "MOE_ERR_UNKNOWN";
+  }
+}
+
+const char* moe_last_cuda_error(void) { return cudaGetErrorString(g_last_cuda); }
+
+int32_t moe_capacity(int32_t T, int32_t E, int32_t k, double capacity_factor, int32_t per_assignment) {
+  if (T < 0 || E < 1 || k < 1) return -2;
+  if (!(capacity_factor > 0.0)) return -1;
+  const double tokens = per_assignment ? (double)T * (double)k : (double)T;
+  const double c = ceil(capacity_factor * tokens / (double)E);
+  if (c > 2147483647.0) return 2147483647;
+  return (int32_t)c;
+}
+
+int64_t moe_rows_max(int32_t T, int32_t E, int32_t k, int32_t capacity) {
+  if (T < 0 || E < 1 || k < 1) return -1;
+  const int64_t A = (int64_t)T * k;
+  if (capacity < 0) return A;
+  const int64_t c = (int64_t)E * capacity;
+  return c < A ? c : A;
+}
+
+size_t moe_route_workspace_bytes(int32_t T, int32_t d, int32_t E) {
+  if (T < 0 || d < 1 || E < 1) return 0;
+  return route_workspace_bytes(T, d, E);
+}
+
+moe_status moe_route(const void* x, int32_t x_dtype, const float* Wg, const float* logit_offset,
+                     const float* select_bias, int32_t T, int32_t d, int32_t E, int32_t k, int32_t score,
+                     int32_t renormalize, float scale, float* logits, int32_t* topk_idx, float* topk_gate,
+                     void* workspace, size_t workspace_bytes, void* stream) {
+  moe_status st = check_dims(T, E, k);
+  if (st != MOE_OK) return st;
+  if ((st = check_d(d)) != MOE_OK) return st;
+  if (!dtype_ok(x_dtype) || score < MOE_SCORE_SOFTMAX || score > MOE_SCORE_SQRT_SOFTPLUS ||
+      (renormalize != 0 && renormalize != 1) || !isfinite(scale))
+    return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x || !Wg || !logits || !topk_idx || !topk_gate) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x)) return MOE_ERR_UNSUPPORTED;
+  const size_t need = route_workspace_bytes(T, d, E);
+  if (need > 0 && (!workspace || workspace_bytes < need)) return MOE_ERR_WORKSPACE;
+  return launch_route(x, x_dtype, Wg, logit_offset, select_bias, T, d, E, k, score, renormalize, scale, logits,
+                      topk_idx, topk_gate, workspace, S(stream));
+}
+
+size_t moe_histogram_scan_workspace_bytes(int32_t T, int32_t k, int32_t E) {
+  if (T < 0 || k < 1 || E < 1) return 0;
+  return histogram_scan_workspace_bytes(T, k, E);
+}
+
+moe_status moe_histogram_scan(const int32_t* topk_idx, const float* topk_gate, int32_t T, int32_t k, int32_t E,
+                              int32_t capacity, int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* row_of,
+                              int32_t* token_of_row, float* gate_of_row, void* workspace, size_t workspace_bytes,
+                              void* stream) {
+  moe_status st = check_dims(T, E, k);
+  if (st != MOE_OK) return st;
+  if (capacity < -1) return MOE_ERR_INVALID_ARG;
+  if (!counts || !kept || !offsets) return MOE_ERR_INVALID_ARG;
+  if (T > 0 && (!topk_idx || !topk_gate || !row_of || !token_of_row || !gate_of_row)) return MOE_ERR_INVALID_ARG;
+  const size_t need = histogram_scan_workspace_bytes(T, k, E);
+  if (need > 0 && (!workspace || workspace_bytes < need)) return MOE_ERR_WORKSPACE;
+  const long long rows_max = moe_rows_max(T, E, k, capacity);
+  return launch_histogram_scan(topk_idx, topk_gate, T, k, E, capacity, counts, kept, offsets, row_of, token_of_row,
+                               gate_of_row, rows_max, workspace, S(stream));
+}
+
+moe_status moe_permute(const void* x, int32_t dtype, int32_t T, int32_t d, int32_t k, const int32_t* row_of,
+                       int64_t rows_max, void* x_perm, void* stream) {
+  if (T < 0 || k < 1 || rows_max < 0) return MOE_ERR_INVALID_ARG;
+  if (k > kMaxK || (long long)T >= kMaxT) return MOE_ERR_UNSUPPORTED;
+  moe_status st = check_d(d);
+  if (st != MOE_OK) return st;
+  if (!dtype_ok(dtype)) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x || !row_of || (rows_max > 0 && !x_perm)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(x_perm)) return MOE_ERR_UNSUPPORTED;
+  return launch_permute(x, dtype, T, d, k, row_of, rows_max, x_perm, S(stream));
+}
+
+static moe_status check_ffn(const void* a, int32_t dtype, const int32_t* offsets, int32_t E, int32_t d, int32_t F,
+                            int64_t rows_max, const void* W, const void* out) {
+  if (E < 1 || d < 1 || F < 1 || rows_max < 0) return MOE_ERR_INVALID_ARG;
+  if (E > kMaxE) return MOE_ERR_UNSUPPORTED;
+  if (d % 8 != 0 || F % 8 != 0) return MOE_ERR_UNSUPPORTED;
+  if (rows_max >= (1LL << 31)) return MOE_ERR_UNSUPPORTED;
+  if (!dtype_ok(dtype)) return MOE_ERR_INVALID_ARG;
+  if (!offsets || !W) return MOE_ERR_INVALID_ARG;
+  if (rows_max > 0 && (!a || !out)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(a) || !aligned16(W) || !aligned16(out)) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+moe_status moe_expert_gate_up(const void* x_rows, int32_t dtype, const int32_t* offsets, int32_t E, int32_t d,
+                              int32_t F, int64_t rows_max, const void* W_gu, void* h, void* stream) {
+  moe_status st = check_ffn(x_rows, dtype, offsets, E, d, F, rows_max, W_gu, h);
+  if (st != MOE_OK || rows_max == 0) return st;
+  if (dtype == MOE_BF16) {
+    st = launch_gate_up_tc(x_rows, offsets, E, d, F, rows_max, W_gu, h, S(stream));
+    if (st != MOE_ERR_UNSUPPORTED) return st;
+  }
+  return launch_gate_up_simt(x_rows, dtype, offsets, E, d, F, rows_max, W_gu, h, S(stream));
+}
+
+moe_status moe_expert_down(const void* h, int32_t dtype, const int32_t* offsets, int32_t E, int32_t d, int32_t F,
+                           int64_t rows_max, const void* W_dn, const float* gate_of_row, void* y_rows, void* stream) {
+  moe_status st = check_ffn(h, dtype, offsets, E, d, F, rows_max, W_dn, y_rows);
+  if (st != MOE_OK || rows_max == 0) return st;
+  if (dtype == MOE_BF16) {
+    st = launch_down_tc(h, offsets, E, d, F, rows_max, W_dn, gate_of_row, y_rows, S(stream));
+    if (st != MOE_ERR_UNSUPPORTED) return st;
+  }
+  return launch_down_simt(h, dtype, offsets, E, d, F, rows_max, W_dn, gate_of_row, y_rows, S(stream));
+}
+
+moe_status moe_grouped_ffn(const void* x_rows, int32_t dtype, const int32_t* offsets, int32_t E, int32_t d, int32_t F,
+                           int64_t rows_max, const void* W_gu, const void* W_dn, const float* gate_of_row, void* h,
+                           void* y_rows, void* stream) {
+  moe_status st = moe_expert_gate_up(x_rows, dtype, offsets, E, d, F, rows_max, W_gu, h, stream);
+  if (st != MOE_OK) return st;
+  return moe_expert_down(h, dtype, offsets, E, d, F, rows_max, W_dn, gate_of_row, y_rows, stream);
+}
+
+moe_status moe_combine(const void* y_rows, const int32_t* row_of, const float* topk_gate, const void* shared_y,
+                       int32_t dtype, int32_t T, int32_t d, int32_t k, int64_t rows_max, void* y, void* stream) {
+  if (T < 0 || k < 1 || rows_max < 0) return MOE_ERR_INVALID_ARG;
+  if (k > kMaxK || (long long)T >= kMaxT) return MOE_ERR_UNSUPPORTED;
+  moe_status st = check_d(d);
+  if (st != MOE_OK) return st;
+  if (!dtype_ok(dtype)) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!row_of || !y || (rows_max > 0 && !y_rows)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(y_rows) || !aligned16(shared_y) || !aligned16(y)) return MOE_ERR_UNSUPPORTED;
+  return launch_combine(y_rows, row_of, topk_gate, shared_y, dtype, T, d, k, rows_max, y, S(stream));
+}
+
+size_t moe_router_stats_workspace_bytes(int32_t T, int32_t E) {
+  if (T < 0 || E < 1) return 0;
+  return router_stats_workspace_bytes(T, E);
+}
+
+moe_status moe_router_stats(const float* logits, const int32_t* counts, const int32_t* kept, int32_t T, int32_t E,
+                            int32_t k, int32_t score, float* load, float* stats5, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  moe_status st = check_dims(T, E, k);
+  if (st != MOE_OK) return st;
+  if (score < MOE_SCORE_SOFTMAX || score > MOE_SCORE_SQRT_SOFTPLUS) return MOE_ERR_INVALID_ARG;
+  if (!counts || !kept || !load || !stats5 || (T > 0 && !logits)) return MOE_ERR_INVALID_ARG;
+  const size_t need = router_stats_workspace_bytes(T, E);
+  if (T > 0 && (!workspace || workspace_bytes < need)) return MOE_ERR_WORKSPACE;
+  return launch_router_stats(logits, counts, kept, T, E, k, score, load, stats5, workspace, S(stream));
+}
+
+size_t moe_workspace_bytes(int32_t T, int32_t d, int32_t E, int32_t k) {
+  size_t a = moe_route_workspace_bytes(T, d, E);
+  size_t b = moe_histogram_scan_workspace_bytes(T, k, E);
+  size_t c = moe_router_stats_workspace_bytes(T, E);
+  size_t m = a > b ? a : b;
+  return m > c ? m : c;
+}
+
+moe_status moe_get_device_error(int32_t* code, void* stream) {
+  if (!code) return MOE_ERR_INVALID_ARG;
+  *code = 0;
+  int host = 0;
+  cudaError_t e = cudaMemcpyFromSymbolAsync(&host, g_moe_device_error, sizeof(int), 0, cudaMemcpyDeviceToHost, S(stream));
+  if (e == cudaSuccess) e = cudaStreamSynchronize(S(stream));
+  if (e != cudaSuccess) { g_last_cuda = e; return MOE_ERR_CUDA; }
+  if (host != 0) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbolAsync(g_moe_device_error, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, S(stream));
+    if (e == cudaSuccess) e = cudaStreamSynchronize(S(stream));
+    if (e != cudaSuccess) { g_last_cuda = e; return MOE_ERR_CUDA; }
+  }
+  *code = host;
+  return host ? MOE_ERR_DEVICE : MOE_OK;
+}
+
+}  // extern "C"

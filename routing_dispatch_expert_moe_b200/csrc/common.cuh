@@ -1,0 +1,137 @@
+// Internal helpers shared by the MoE-layer kernels (sm_100a).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "moe.h"
+
+namespace moe {
+
+constexpr int kWarp = 32;
+
+// ---- device error word (address of the library's __device__ int, per device) ----
+int* err_ptr();                       // host: current device's error word address (or null)
+cudaError_t& last_cuda_error_ref();   // host: last CUDA error seen by a call
+
+__device__ __forceinline__ void record_error(int* err, int code) {
+  if (err) atomicCAS(err, 0, code);
+}
+
+// ---- bf16 helpers ----
+__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
+
+// Round-to-nearest-even float -> bf16 pair packed as (lo | hi << 16).
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&p);
+}
+
+// 8 values from one 16-byte vector of bf16.
+__device__ __forceinline__ void unpack8(const uint4& v, float* f) {
+  f[0] = bf16_lo(v.x); f[1] = bf16_hi(v.x);
+  f[2] = bf16_lo(v.y); f[3] = bf16_hi(v.y);
+  f[4] = bf16_lo(v.z); f[5] = bf16_hi(v.z);
+  f[6] = bf16_lo(v.w); f[7] = bf16_hi(v.w);
+}
+
+__device__ __forceinline__ uint4 pack8(const float* f) {
+  uint4 v;
+  v.x = pack_bf16x2(f[0], f[1]);
+  v.y = pack_bf16x2(f[2], f[3]);
+  v.z = pack_bf16x2(f[4], f[5]);
+  v.w = pack_bf16x2(f[6], f[7]);
+  return v;
+}
+
+// Streaming (evict-first) 16-byte global accesses.
+__device__ __forceinline__ uint4 ld_stream(const uint4* p) {
+  uint4 v;
+  asm volatile("ld.global.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ unsigned lane_id() {
+  unsigned r;
+  asm volatile("mov.u32 %0, %%laneid;" : "=r"(r));
+  return r;
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+inline int num_sms() {
+  static int cached[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (!cached[dev]) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cached[dev] = n > 0 ? n : 148;
+  }
+  return cached[dev];
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline moe_status check_launch() {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    last_cuda_error_ref() = e;
+    return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
+inline moe_status cuda_status(cudaError_t e) {
+  if (e != cudaSuccess) {
+    last_cuda_error_ref() = e;
+    return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
+// ---- launchers implemented in the kernel files (arguments already validated) ----
+moe_status launch_route(const void* x, int x_dtype, const float* Wg, const float* logit_offset,
+                        const float* select_bias, int T, int d, int E, int k, int score,
+                        int renormalize, float scale, float* logits, int32_t* topk_idx,
+                        float* topk_gate, void* ws, cudaStream_t s);
+size_t route_workspace_bytes(int T, int d, int E);
+
+moe_status launch_histogram_scan(const int32_t* topk_idx, const float* topk_gate, int T, int k,
+                                 int E, int capacity, int32_t* counts, int32_t* kept,
+                                 int32_t* offsets, int32_t* row_of, int32_t* token_of_row,
+                                 float* gate_of_row, long long rows_max, void* ws, cudaStream_t s);
+size_t histogram_scan_workspace_bytes(int T, int k, int E);
+
+moe_status launch_permute(const void* x, int dtype, int T, int d, int k, const int32_t* row_of,
+                          long long rows_max, void* x_perm, cudaStream_t s);
+moe_status launch_combine(const void* y_rows, const int32_t* row_of, const float* topk_gate,
+                          const void* shared_y, int dtype, int T, int d, int k, long long rows_max,
+                          void* y, cudaStream_t s);
+
+moe_status launch_router_stats(const float* logits, const int32_t* counts, const int32_t* kept,
+                               int T, int E, int k, int score, float* load, float* stats5,
+                               void* ws, cudaStream_t s);
+size_t router_stats_workspace_bytes(int T, int E);
+
+moe_status launch_gate_up_simt(const void* x_rows, int dtype, const int32_t* offsets, int E, int d,
+                               int F, long long rows_max, const void* W_gu, void* h,
+                               cudaStream_t s);
+moe_status launch_down_simt(const void* h, int dtype, const int32_t* offsets, int E, int d, int F,
+                            long long rows_max, const void* W_dn, const float* gate_of_row,
+                            void* y_rows, cudaStream_t s);
+moe_status launch_gate_up_tc(const void* x_rows, const int32_t* offsets, int E, int d, int F,
+                             long long rows_max, const void* W_gu, void* h, cudaStream_t s);
+moe_status launch_down_tc(const void* h, const int32_t* offsets, int E, int d, int F,
+                          long long rows_max, const void* W_dn, const float* gate_of_row,
+                          void* y_rows, cudaStream_t s);
+
+}  // namespace moe

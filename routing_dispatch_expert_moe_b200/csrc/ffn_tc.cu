@@ -1,0 +1,452 @@
+// Grouped SwiGLU expert GEMMs on the 5th-generation tensor cores (sm_100a).
+//
+// Expert FFN: "Hugging Face 图解 Mixture of Experts（MoE）原理、训练与推理权衡", section
+// "什么是混合专家模型" (each expert is an FFN) and section "更多关于高效训练的内容"
+// (experts receive uneven numbers of tokens; handle them without padding or drops).
+// SwiGLU form: H = silu(X Wg^T) * (X Wu^T), Y = gate * (H Wd^T), no biases.
+//
+// One persistent kernel template, two epilogues:
+//   MODE 0 (gate_up): A = X [rows, d], B = W_gu[e] ([2F, d], gate rows then up rows).
+//       A 256-wide B tile holds 128 gate rows and the matching 128 up rows, so one
+//       128x256 accumulator carries g (columns 0..127) and u (128..255) for the same
+//       128 features; the epilogue writes H = silu(g) * u as bf16.
+//   MODE 1 (down): A = H [rows, F], B = W_dn[e] ([d, F]); the epilogue scales each row
+//       by gate_of_row and writes bf16.
+//
+// Per CTA (1 per SM, 192 threads):
+//   warp 0   TMA producer: 128x64 A tile + 256x64 B tile per stage (128-byte swizzle),
+//            4-stage ring of mbarriers (full: TMA bytes landed, empty: MMAs done).
+//   warp 1   allocates 512 TMEM columns; one thread issues tcgen05.mma
+//            (kind::f16, bf16 x bf16 -> fp32, M=128, N=256, K=16) and tcgen05.commit.
+//   warps 2-5 epilogue: tcgen05.ld 32x32b (thread = accumulator row), fused SwiGLU or
+//            gate scaling, bf16 rounding, masked 16-byte stores.  Two 256-column TMEM
+//            accumulators let the epilogue of tile i overlap the mainloop of tile i+1.
+// Tiles come from the device-side schedule built from the offsets array; a tile never
+// writes a row outside its expert's range or a column outside the output width.
+// Every barrier wait is bounded (MOE_DEVERR_PIPE_TIMEOUT, then an orderly exit: MMAs
+// drained, outstanding TMA loads awaited, TMEM freed).
+#include <cuda.h>
+
+#include "common.cuh"
+#include "tile_sched.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4, UMMA_K = 16;
+constexpr int kThreadsTC = 192;
+constexpr int A_STAGE = BM * BK * 2;   // 16 KB
+constexpr int B_STAGE = BN * BK * 2;   // 32 KB
+constexpr int kMaxE = 1024;
+constexpr uint32_t kTmemCols = 512;
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s per barrier wait
+
+struct L {
+  static constexpr int a = 0;
+  static constexpr int b = STAGES * A_STAGE;
+  static constexpr int bars = b + STAGES * B_STAGE;
+  static constexpr int nbars = 2 * STAGES + 4 + 1;          // full, empty, tfull[2], tempty[2], fin
+  static constexpr int misc = bars + nbars * 8;              // tmem slot, abort flag
+  static constexpr int tiles = misc + 16;                    // int tile_start[kMaxE + 1]
+  static constexpr int sh32 = tiles + (kMaxE + 1) * 4;      // int[32]
+  static constexpr int end = sh32 + 32 * 4;
+};
+constexpr size_t kSmemBytes = L::end + 1024;                 // + alignment slack
+
+// instruction descriptor: D fp32, A bf16, B bf16, both K-major, N = 256, M = 128
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                            ((uint32_t)(BM >> 4) << 24);
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait.  Returns false when the limit passes (records the error, raises the
+// CTA's abort flag) or when another role has already aborted.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 63u) == 0u) {
+      if (*abort_flag) return false;
+      if (global_timer_ns() - t0 > kWaitLimitNs) {
+        record_error(err, MOE_DEVERR_PIPE_TIMEOUT);
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+// Bounded wait that ignores the abort flag (used to drain in-flight work on exit).
+__device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity, int* err) {
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t i = 0;; ++i) {
+    if (mbar_try_wait(bar, parity)) return;
+    if ((i & 63u) == 63u && global_timer_ns() - t0 > kWaitLimitNs) {
+      record_error(err, MOE_DEVERR_PIPE_TIMEOUT);
+      return;
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+// K-major operand in the canonical 128-byte-swizzle layout written by TMA:
+// rows of 128 bytes (64 bf16), 8-row atoms of 1024 bytes stacked densely.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);   // start address >> 4
+  d |= (uint64_t)1 << 16;                            // leading byte offset (unused when swizzled)
+  d |= (uint64_t)(1024 >> 4) << 32;                  // stride byte offset: one 8-row atom
+  d |= (uint64_t)1 << 46;                            // descriptor version for sm_100
+  d |= (uint64_t)2 << 61;                            // 128-byte swizzle
+  return d;
+}
+
+#define MOE_R32(r) \
+  "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), \
+  "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), \
+  "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), \
+  "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+#define MOE_RW32(r) \
+  "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]), \
+  "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), \
+  "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), \
+  "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+
+// 32 consecutive fp32 accumulator columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : MOE_R32(r)
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// Ties the loaded registers to the preceding wait so no use is scheduled above it.
+__device__ __forceinline__ void tmem_regs_ready(uint32_t (&r)[32]) { asm volatile("" : MOE_RW32(r)); }
+
+template <int MODE>
+__global__ void __launch_bounds__(kThreadsTC, 1)
+grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                       const int32_t* __restrict__ offsets, int E, int K, int N_out, int F,
+                       long long rows_max, const float* __restrict__ gate_of_row,
+                       __nv_bfloat16* __restrict__ out, int* err) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int* tile_start = reinterpret_cast<int*>(smem + L::tiles);
+  int* sh32 = reinterpret_cast<int*>(smem + L::sh32);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::misc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::misc + 4);
+
+  // MODE 0: 128 H columns per tile (128 gate + 128 up accumulator columns)
+  const int n_tiles = MODE == 0 ? (F + 127) / 128 : (N_out + BN - 1) / BN;
+  build_tile_starts(offsets, E, BM, n_tiles, rows_max, tile_start, sh32, err);
+  const int total = tile_start[E];
+  if ((int)blockIdx.x >= total) return;   // uniform: nothing allocated yet
+
+  const uint32_t bar_full = sb + L::bars;
+  const uint32_t bar_empty = bar_full + 8 * STAGES;
+  const uint32_t bar_tfull = bar_empty + 8 * STAGES;
+  const uint32_t bar_tempty = bar_tfull + 16;
+  const uint32_t bar_fin = bar_tempty + 16;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_empty + 8 * s, 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(bar_tfull + 8 * a, 1);
+      mbar_init(bar_tempty + 8 * a, 128);
+    }
+    mbar_init(bar_fin, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int KB = (K + BK - 1) / BK;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int last_phase[STAGES];
+#pragma unroll
+      for (int s = 0; s < STAGES; ++s) last_phase[s] = -1;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+        const TileCoord tc = tile_coord(tile_start, offsets, E, BM, tile);
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1u, abort_flag, err)) { ok = false; break; }
+          const uint32_t full = bar_full + 8 * stage;
+          mbar_expect_tx(full, A_STAGE + B_STAGE);
+          const uint32_t a_dst = sb + L::a + stage * A_STAGE;
+          const uint32_t b_dst = sb + L::b + stage * B_STAGE;
+          tma_load_2d(a_dst, &tmA, full, kb * BK, tc.row0);
+          if (MODE == 0) {
+            const int g_row = tc.e * 2 * F + tc.n_tile * 128;
+            tma_load_2d(b_dst, &tmB, full, kb * BK, g_row);
+            tma_load_2d(b_dst + B_STAGE / 2, &tmB, full, kb * BK, g_row + F);
+          } else {
+            tma_load_2d(b_dst, &tmB, full, kb * BK, tc.e * N_out + tc.n_tile * BN);
+          }
+          last_phase[stage] = (int)phase;
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) {
+        // let every issued copy land before the CTA can exit
+        for (int s = 0; s < STAGES; ++s)
+          if (last_phase[s] >= 0) mbar_wait_drain(bar_full + 8 * s, (uint32_t)last_phase[s], err);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x, ++it) {
+        const int acc = it & 1;
+        const uint32_t acc_phase = (uint32_t)(it >> 1) & 1u;
+        if (!mbar_wait(bar_tempty + 8 * acc, acc_phase ^ 1u, abort_flag, err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag, err)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t adesc = sw128_desc(sb + L::a + stage * A_STAGE);
+          const uint64_t bdesc = sw128_desc(sb + L::b + stage * B_STAGE);
+#pragma unroll
+          for (int kk = 0; kk < BK / UMMA_K; ++kk)   // +32 bytes along K per step (>> 4 = 2)
+            umma_bf16(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, (kb | kk) != 0 ? 1u : 0u);
+          umma_commit(bar_empty + 8 * stage);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma_commit(bar_tfull + 8 * acc);
+      }
+      // all issued MMAs complete before TMEM can be released
+      umma_commit(bar_fin);
+      mbar_wait_drain(bar_fin, 0, err);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 2..5)
+    const int q = warp & 3;                 // TMEM lane quarter this warp may access
+    const int r_in = q * 32 + lane;         // accumulator row == tile row
+    int it = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
+      const TileCoord tc = tile_coord(tile_start, offsets, E, BM, tile);
+      const int acc = it & 1;
+      const uint32_t acc_phase = (uint32_t)(it >> 1) & 1u;
+      const bool got = mbar_wait(bar_tfull + 8 * acc, acc_phase, abort_flag, err);
+      // tcgen05.ld is .sync.aligned: the whole warp goes on, or the whole warp stops
+      if (!__all_sync(0xffffffffu, got)) break;
+      __syncwarp();
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+      const bool valid = r_in < tc.rows;
+      const long long row = (long long)tc.row0 + r_in;
+      if (MODE == 0) {
+        const int f0 = tc.n_tile * 128;
+        __nv_bfloat16* orow = out + row * F;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t g[32], u[32];
+          tmem_ld32(taddr + c * 32, g);
+          tmem_ld32(taddr + 128 + c * 32, u);
+          tmem_wait_ld();
+          tmem_regs_ready(g);
+          tmem_regs_ready(u);
+          if (valid) {
+            const int col = f0 + c * 32;
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
+              const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
+              const float h0 = g0 / (1.f + __expf(-g0)) * u0;
+              const float h1 = g1 / (1.f + __expf(-g1)) * u1;
+              pk[i] = pack_bf16x2(h0, h1);
+            }
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              if (col + 8 * v + 8 <= F)
+                *reinterpret_cast<uint4*>(orow + col + 8 * v) =
+                    make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          }
+        }
+      } else {
+        const int n0 = tc.n_tile * BN;
+        const float gs = (valid && gate_of_row) ? __ldg(gate_of_row + row) : 1.f;
+        __nv_bfloat16* orow = out + row * N_out;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t v32[32];
+          tmem_ld32(taddr + c * 32, v32);
+          tmem_wait_ld();
+          tmem_regs_ready(v32);
+          if (valid) {
+            const int col = n0 + c * 32;
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              pk[i] = pack_bf16x2(__uint_as_float(v32[2 * i]) * gs, __uint_as_float(v32[2 * i + 1]) * gs);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              if (col + 8 * v + 8 <= N_out)
+                *reinterpret_cast<uint4*>(orow + col + 8 * v) =
+                    make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar_tempty + 8 * acc);
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols) : "memory");
+  }
+}
+
+// ---------------------------------------------------------------- host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2D bf16 tensor [rows, cols] row-major; box = box_rows x 64 columns, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* ptr, unsigned long long rows, unsigned long long cols, unsigned box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int MODE>
+moe_status launch_tc(const CUtensorMap& ma, const CUtensorMap& mb, const int32_t* offsets, int E, int K, int N_out,
+                     int F, long long rows_max, const float* gate_of_row, void* out, cudaStream_t s) {
+  static int configured[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (!configured[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_tc_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kSmemBytes);
+    if (e != cudaSuccess) return cuda_status(e);
+    configured[dev] = 1;
+  }
+  const int n_tiles = MODE == 0 ? (F + 127) / 128 : (N_out + BN - 1) / BN;
+  const long long max_tiles = ((rows_max + BM - 1) / BM + E) * (long long)n_tiles;
+  int grid = num_sms();
+  if (max_tiles < grid) grid = (int)max_tiles;
+  if (grid < 1) grid = 1;
+  grouped_gemm_tc_kernel<MODE><<<grid, kThreadsTC, kSmemBytes, s>>>(
+      ma, mb, offsets, E, K, N_out, F, rows_max, gate_of_row, static_cast<__nv_bfloat16*>(out), err_ptr());
+  return check_launch();
+}
+
+}  // namespace
+
+// Returns MOE_ERR_UNSUPPORTED when a tensor map cannot be encoded (caller falls back).
+moe_status launch_gate_up_tc(const void* x_rows, const int32_t* offsets, int E, int d, int F, long long rows_max,
+                             const void* W_gu, void* h, cudaStream_t s) {
+  if (rows_max == 0) return MOE_OK;
+  if (d < BK || F < 8) return MOE_ERR_UNSUPPORTED;
+  CUtensorMap ma, mb;
+  if (!make_map(&ma, x_rows, (unsigned long long)rows_max, d, BM)) return MOE_ERR_UNSUPPORTED;
+  if (!make_map(&mb, W_gu, (unsigned long long)E * 2 * F, d, 128)) return MOE_ERR_UNSUPPORTED;
+  return launch_tc<0>(ma, mb, offsets, E, d, F, F, rows_max, nullptr, h, s);
+}
+
+moe_status launch_down_tc(const void* h, const int32_t* offsets, int E, int d, int F, long long rows_max,
+                          const void* W_dn, const float* gate_of_row, void* y_rows, cudaStream_t s) {
+  if (rows_max == 0) return MOE_OK;
+  if (F < BK || d < 8) return MOE_ERR_UNSUPPORTED;
+  CUtensorMap ma, mb;
+  if (!make_map(&ma, h, (unsigned long long)rows_max, F, BM)) return MOE_ERR_UNSUPPORTED;
+  if (!make_map(&mb, W_dn, (unsigned long long)E * d, F, BN)) return MOE_ERR_UNSUPPORTED;
+  return launch_tc<1>(ma, mb, offsets, E, F, d, F, rows_max, gate_of_row, y_rows, s);
+}
+
+}  // namespace moe

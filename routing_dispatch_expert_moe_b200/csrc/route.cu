@@ -1,0 +1,457 @@
+// Router: fp32 logits, scoring, selection-only bias, top-k, gates.
+//
+// Sources: "Hugging Face 图解 Mixture of Experts（MoE）原理、训练与推理权衡" (Chinese
+// rendering of "Mixture of Experts Explained"), section "什么是稀疏性？":
+//   G_sigma(x) = Softmax(x . W_g);  KeepTopK(v, k);  G(x) = Softmax(KeepTopK(H(x), k));
+// section "Switch Transformer": the router is computed in full precision because of
+// its exponential.  Handbook news post (hub.geekagi.cn), "真正难在三个环节" item 1
+// (routing in FP32) and item 2 (loss-free balancing bias); the quoted tweet lists
+// softmax, sigmoid and sqrt(softplus) routers.  Handbook digest (agihunt.info):
+// routing scale factor near sqrt(k).
+//
+// Two kernels:
+//   logits_kernel  tiled SIMT GEMM  l = x . Wg (+ offset), fp32 FMA; W_g and x staged
+//                  through shared memory, 8 experts x TM tokens per thread, optional
+//                  split over d (partials summed in a fixed order by the next kernel).
+//   topk_kernel    one warp per token: lanes own experts lane, lane+32, ...; k rounds of
+//                  a shuffle arg-max on (key desc, index asc); gates in fp32.
+#include "common.cuh"
+
+#include <float.h>
+
+namespace moe {
+namespace {
+
+constexpr int kLogitThreads = 256;
+constexpr int kKC = 32;  // d-chunk staged per iteration
+
+template <typename XT>
+struct XLoad;
+template <>
+struct XLoad<__nv_bfloat16> {
+  static constexpr int kPerVec = 8;
+  __device__ static void load(const void* base, long long elem, bool ok, float* f) {
+    if (ok) {
+      uint4 v = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(base) + elem));
+      unpack8(v, f);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) f[i] = 0.f;
+    }
+  }
+};
+template <>
+struct XLoad<float> {
+  static constexpr int kPerVec = 4;
+  __device__ static void load(const void* base, long long elem, bool ok, float* f) {
+    if (ok) {
+      float4 v = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(base) + elem));
+      f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
+    } else {
+      f[0] = f[1] = f[2] = f[3] = 0.f;
+    }
+  }
+};
+
+// Tile: BT tokens x BE experts; thread micro-tile TM tokens x 8 experts.
+template <typename XT, int BE, int TM>
+__global__ void __launch_bounds__(kLogitThreads)
+logits_kernel(const void* __restrict__ x, const float* __restrict__ Wg,
+              const float* __restrict__ logit_offset, int T, int d, int E,
+              int chunks_per_split, float* __restrict__ out, long long split_stride) {
+  constexpr int TN = 8;
+  constexpr int EG = BE / TN;                 // expert groups
+  constexpr int TG = kLogitThreads / EG;      // token groups
+  constexpr int BT = TG * TM;                 // tokens per CTA
+  constexpr int PV = XLoad<XT>::kPerVec;      // x values per 16-byte vector
+  constexpr int XV = BT * kKC / PV;           // x vectors per chunk
+  constexpr int XV_PER_T = (XV + kLogitThreads - 1) / kLogitThreads;
+  constexpr int WV = kKC * BE;                // W scalars per chunk
+  constexpr int WV_PER_T = (WV + kLogitThreads - 1) / kLogitThreads;
+
+  extern __shared__ __align__(16) float smem[];
+  float* xs = smem;                 // [kKC][BT]
+  float* wsm = smem + kKC * BT;     // [kKC][BE]
+
+  const int tid = threadIdx.x;
+  const int eg = tid % EG, tg = tid / EG;
+  const int t0 = blockIdx.x * BT;
+  const int e0 = blockIdx.y * BE;
+  const int nchunks = (d + kKC - 1) / kKC;
+  const int c_begin = blockIdx.z * chunks_per_split;
+  const int c_end = min(nchunks, c_begin + chunks_per_split);
+
+  float acc[TM][TN];
+#pragma unroll
+  for (int i = 0; i < TM; ++i)
+#pragma unroll
+    for (int j = 0; j < TN; ++j) acc[i][j] = 0.f;
+
+  float xr[XV_PER_T][PV];
+  float wr[WV_PER_T];
+
+  auto gload = [&](int c) {
+    const int kk0 = c * kKC;
+#pragma unroll
+    for (int r = 0; r < XV_PER_T; ++r) {
+      const int v = tid + r * kLogitThreads;
+      const int q = v / BT, t = v % BT;          // q-major: a warp covers 32 tokens
+      const int col = kk0 + q * PV;
+      const bool ok = (v < XV) && (t0 + t < T) && (col < d);
+      XLoad<XT>::load(x, (long long)(t0 + t) * d + col, ok, xr[r]);
+    }
+#pragma unroll
+    for (int r = 0; r < WV_PER_T; ++r) {
+      const int v = tid + r * kLogitThreads;
+      const int kk = v / BE, e = v % BE;
+      const bool ok = (v < WV) && (kk0 + kk < d) && (e0 + e < E);
+      wr[r] = ok ? __ldg(Wg + (long long)(kk0 + kk) * E + e0 + e) : 0.f;
+    }
+  };
+  auto sstore = [&]() {
+#pragma unroll
+    for (int r = 0; r < XV_PER_T; ++r) {
+      const int v = tid + r * kLogitThreads;
+      if (v < XV) {
+        const int q = v / BT, t = v % BT;
+#pragma unroll
+        for (int i = 0; i < PV; ++i) xs[(q * PV + i) * BT + t] = xr[r][i];
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < WV_PER_T; ++r) {
+      const int v = tid + r * kLogitThreads;
+      if (v < WV) wsm[v] = wr[r];   // [kk][e] layout == v
+    }
+  };
+
+  if (c_begin < c_end) gload(c_begin);
+  for (int c = c_begin; c < c_end; ++c) {
+    __syncthreads();
+    sstore();
+    __syncthreads();
+    if (c + 1 < c_end) gload(c + 1);
+#pragma unroll 8
+    for (int kk = 0; kk < kKC; ++kk) {
+      float xv[TM], wv[TN];
+      if constexpr (TM == 4) {
+        float4 a = *reinterpret_cast<const float4*>(&xs[kk * BT + tg * TM]);
+        xv[0] = a.x; xv[1] = a.y; xv[2] = a.z; xv[3] = a.w;
+      } else {
+        float2 a = *reinterpret_cast<const float2*>(&xs[kk * BT + tg * TM]);
+        xv[0] = a.x; xv[1] = a.y;
+      }
+      // experts {eg*4 .. +3} and {BE/2 + eg*4 .. +3}: a phase of 8 lanes reads 128
+      // contiguous bytes per vector, free of bank conflicts
+      float4 b0 = *reinterpret_cast<const float4*>(&wsm[kk * BE + eg * 4]);
+      float4 b1 = *reinterpret_cast<const float4*>(&wsm[kk * BE + BE / 2 + eg * 4]);
+      wv[0] = b0.x; wv[1] = b0.y; wv[2] = b0.z; wv[3] = b0.w;
+      wv[4] = b1.x; wv[5] = b1.y; wv[6] = b1.z; wv[7] = b1.w;
+#pragma unroll
+      for (int i = 0; i < TM; ++i)
+#pragma unroll
+        for (int j = 0; j < TN; ++j) acc[i][j] = fmaf(xv[i], wv[j], acc[i][j]);
+    }
+  }
+
+  float* dst = out + blockIdx.z * split_stride;
+  const bool add_off = (logit_offset != nullptr) && (gridDim.z == 1);
+#pragma unroll
+  for (int i = 0; i < TM; ++i) {
+    const int t = t0 + tg * TM + i;
+    if (t >= T) continue;
+#pragma unroll
+    for (int j = 0; j < TN; ++j) {
+      const int e = e0 + (j < 4 ? eg * 4 + j : BE / 2 + eg * 4 + (j - 4));
+      if (e < E) dst[(long long)t * E + e] = acc[i][j] + (add_off ? __ldg(logit_offset + e) : 0.f);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------------
+// top-k + gates: one warp per token.
+// ---------------------------------------------------------------------------------
+struct Cand {
+  float kf;     // key when no selection bias (the logit)
+  double kd;    // key with a selection bias (score + bias, fp64)
+  int idx;
+  float logit;
+};
+
+template <bool BIAS>
+__device__ __forceinline__ bool better(const Cand& a, const Cand& b) {
+  if (BIAS) {
+    if (a.kd != b.kd) return a.kd > b.kd;
+  } else {
+    if (a.kf != b.kf) return a.kf > b.kf;
+  }
+  return a.idx < b.idx;
+}
+
+__device__ __forceinline__ double score_d(double l, int score) {
+  if (score == MOE_SCORE_SIGMOID) return 1.0 / (1.0 + exp(-l));
+  // MOE_SCORE_SQRT_SOFTPLUS
+  return sqrt(fmax(l, 0.0) + log1p(exp(-fabs(l))));
+}
+
+__device__ __forceinline__ float score_f(float l, int score) {
+  if (score == MOE_SCORE_SIGMOID) return 1.f / (1.f + expf(-l));
+  return sqrtf(fmaxf(l, 0.f) + log1pf(expf(-fabsf(l))));
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+template <int EPL, bool BIAS>
+__global__ void __launch_bounds__(256)
+topk_kernel(const float* __restrict__ partial, int nsplit, long long split_stride,
+            const float* __restrict__ logit_offset, const float* __restrict__ select_bias,
+            int T, int E, int k, int score, int renorm, float scale,
+            float* __restrict__ logits, int write_logits,
+            int32_t* __restrict__ topk_idx, float* __restrict__ topk_gate) {
+  const unsigned lane = threadIdx.x & 31;
+  const int warps = blockDim.x >> 5;
+  const long long gw = (long long)blockIdx.x * warps + (threadIdx.x >> 5);
+  const long long nw = (long long)gridDim.x * warps;
+
+  for (long long t = gw; t < T; t += nw) {
+    float l[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      const int e = lane + 32 * i;
+      float v = -INFINITY;
+      if (e < E) {
+        float s = 0.f;
+        for (int p = 0; p < nsplit; ++p) s += partial[p * split_stride + t * E + e];
+        if (nsplit > 1 && logit_offset) s += __ldg(logit_offset + e);
+        v = s;
+        if (write_logits) logits[t * E + e] = v;
+      }
+      l[i] = v;
+    }
+
+    // selection keys
+    float kf[EPL];
+    double kd[EPL];
+    if (BIAS) {
+      double m = 0.0, z = 1.0;
+      if (score == MOE_SCORE_SOFTMAX) {
+        float mf = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) mf = fmaxf(mf, l[i]);
+        m = (double)warp_max(mf);
+        double zs = 0.0;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i)
+          if (lane + 32 * i < (unsigned)E) zs += exp((double)l[i] - m);
+        z = warp_sum_d(zs);
+      }
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) {
+        const int e = lane + 32 * i;
+        if (e < E) {
+          const double sc = (score == MOE_SCORE_SOFTMAX) ? exp((double)l[i] - m) / z
+                                                         : score_d((double)l[i], score);
+          double key = sc + (double)__ldg(select_bias + e);
+          kd[i] = (key != key) ? -INFINITY : key;
+        } else {
+          kd[i] = -INFINITY;
+        }
+        kf[i] = 0.f;
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) {
+        kf[i] = (l[i] != l[i]) ? -INFINITY : l[i];
+        kd[i] = 0.0;
+      }
+    }
+
+    // local best among untaken (ties: lower index == lower i on this lane)
+    uint32_t taken = 0;
+    auto local_best = [&]() {
+      Cand b;
+      b.kf = -INFINITY; b.kd = -INFINITY; b.idx = 0x7fffffff; b.logit = 0.f;
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) {
+        const int e = lane + 32 * i;
+        if (e < E && !((taken >> i) & 1u)) {
+          Cand c;
+          c.kf = kf[i]; c.kd = kd[i]; c.idx = e; c.logit = l[i];
+          if (better<BIAS>(c, b)) b = c;
+        }
+      }
+      return b;
+    };
+    Cand mine = local_best();
+    int sel_idx = 0;
+    float sel_logit = 0.f;
+    for (int j = 0; j < k; ++j) {
+      Cand w = mine;
+#pragma unroll
+      for (int o = 16; o; o >>= 1) {
+        Cand c;
+        if constexpr (BIAS) {
+          c.kd = __shfl_xor_sync(0xffffffffu, w.kd, o);
+          c.kf = 0.f;
+        } else {
+          c.kf = __shfl_xor_sync(0xffffffffu, w.kf, o);
+          c.kd = 0.0;
+        }
+        c.idx = __shfl_xor_sync(0xffffffffu, w.idx, o);
+        c.logit = __shfl_xor_sync(0xffffffffu, w.logit, o);
+        if (better<BIAS>(c, w)) w = c;
+      }
+      if (lane == (unsigned)j) { sel_idx = w.idx; sel_logit = w.logit; }
+      if (w.idx >= 0 && w.idx < E && (unsigned)(w.idx & 31) == lane) {
+        taken |= 1u << (w.idx >> 5);
+        mine = local_best();
+      }
+    }
+
+    // gates (fp32)
+    const bool act = lane < (unsigned)k;
+    float g;
+    if (score == MOE_SCORE_SOFTMAX) {
+      if (renorm) {
+        const float m = warp_max(act ? sel_logit : -INFINITY);
+        const float ex = act ? expf(sel_logit - m) : 0.f;
+        g = ex / warp_sum(ex);
+      } else {
+        float mf = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) mf = fmaxf(mf, l[i]);
+        const float M = warp_max(mf);
+        float zs = 0.f;
+#pragma unroll
+        for (int i = 0; i < EPL; ++i)
+          if (lane + 32 * i < (unsigned)E) zs += expf(l[i] - M);
+        const float Z = warp_sum(zs);
+        g = expf(sel_logit - M) / Z;
+      }
+    } else {
+      const float s = act ? score_f(sel_logit, score) : 0.f;
+      g = renorm ? s / warp_sum(s) : s;
+    }
+    g *= scale;
+    if (act) {
+      topk_idx[t * k + lane] = sel_idx;
+      topk_gate[t * k + lane] = g;
+    }
+  }
+}
+
+struct LogitsPlan {
+  int BE, TM, BT, nsplit, chunks_per_split;
+  size_t smem;
+};
+
+LogitsPlan plan_logits(int T, int d, int E) {
+  LogitsPlan p;
+  p.BE = E > 32 ? 64 : (E > 16 ? 32 : (E > 8 ? 16 : 8));
+  p.TM = p.BE >= 32 ? 4 : 2;
+  const int EG = p.BE / 8, TG = kLogitThreads / EG;
+  p.BT = TG * p.TM;
+  p.smem = (size_t)(kKC * p.BT + kKC * p.BE) * sizeof(float);
+  const int nchunks = (d + kKC - 1) / kKC;
+  const long long ctas = (long long)((T + p.BT - 1) / p.BT) * ((E + p.BE - 1) / p.BE);
+  int s = 1;
+  const long long target = 2LL * num_sms();
+  while (ctas * s < target && nchunks / (2 * s) >= 4) s *= 2;
+  p.nsplit = s;
+  p.chunks_per_split = (nchunks + s - 1) / s;
+  return p;
+}
+
+template <typename XT, int BE, int TM>
+moe_status run_logits(const void* x, const float* Wg, const float* off, int T, int d, int E,
+                      const LogitsPlan& p, float* out, long long split_stride, cudaStream_t s) {
+  auto kern = logits_kernel<XT, BE, TM>;
+  if (p.smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
+    if (e != cudaSuccess) return cuda_status(e);
+  }
+  dim3 grid((T + p.BT - 1) / p.BT, (E + BE - 1) / BE, p.nsplit);
+  kern<<<grid, kLogitThreads, p.smem, s>>>(x, Wg, off, T, d, E, p.chunks_per_split, out, split_stride);
+  return check_launch();
+}
+
+template <typename XT>
+moe_status dispatch_logits(const void* x, const float* Wg, const float* off, int T, int d, int E,
+                           const LogitsPlan& p, float* out, long long split_stride, cudaStream_t s) {
+  switch (p.BE) {
+    case 64: return run_logits<XT, 64, 4>(x, Wg, off, T, d, E, p, out, split_stride, s);
+    case 32: return run_logits<XT, 32, 4>(x, Wg, off, T, d, E, p, out, split_stride, s);
+    case 16: return run_logits<XT, 16, 2>(x, Wg, off, T, d, E, p, out, split_stride, s);
+    default: return run_logits<XT, 8, 2>(x, Wg, off, T, d, E, p, out, split_stride, s);
+  }
+}
+
+template <int EPL>
+moe_status run_topk(bool bias, const float* partial, int nsplit, long long split_stride,
+                    const float* off, const float* sel_bias, int T, int E, int k, int score,
+                    int renorm, float scale, float* logits, int write_logits, int32_t* idx,
+                    float* gate, cudaStream_t s) {
+  const int threads = 256;
+  const long long warps_needed = T;
+  long long blocks = (warps_needed + 7) / 8;
+  const long long cap = (long long)num_sms() * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  if (bias)
+    topk_kernel<EPL, true><<<(unsigned)blocks, threads, 0, s>>>(partial, nsplit, split_stride, off, sel_bias, T, E, k,
+                                                       score, renorm, scale, logits, write_logits, idx, gate);
+  else
+    topk_kernel<EPL, false><<<(unsigned)blocks, threads, 0, s>>>(partial, nsplit, split_stride, off, sel_bias, T, E, k,
+                                                        score, renorm, scale, logits, write_logits, idx, gate);
+  return check_launch();
+}
+
+}  // namespace
+
+size_t route_workspace_bytes(int T, int d, int E) {
+  if (T <= 0 || E <= 0 || d <= 0) return 0;
+  LogitsPlan p = plan_logits(T, d, E);
+  return p.nsplit > 1 ? (size_t)p.nsplit * T * E * sizeof(float) : 0;
+}
+
+moe_status launch_route(const void* x, int x_dtype, const float* Wg, const float* logit_offset,
+                        const float* select_bias, int T, int d, int E, int k, int score,
+                        int renormalize, float scale, float* logits, int32_t* topk_idx,
+                        float* topk_gate, void* ws, cudaStream_t s) {
+  if (T == 0) return MOE_OK;
+  LogitsPlan p = plan_logits(T, d, E);
+  float* partial = p.nsplit > 1 ? static_cast<float*>(ws) : logits;
+  const long long split_stride = (long long)T * E;
+  moe_status st = x_dtype == MOE_F32
+                      ? dispatch_logits<float>(x, Wg, logit_offset, T, d, E, p, partial, split_stride, s)
+                      : dispatch_logits<__nv_bfloat16>(x, Wg, logit_offset, T, d, E, p, partial, split_stride, s);
+  if (st != MOE_OK) return st;
+  const int write = p.nsplit > 1 ? 1 : 0;
+  const int epl = (E + 31) / 32;
+  const bool bias = select_bias != nullptr;
+#define MOE_TOPK(N) return run_topk<N>(bias, partial, p.nsplit, split_stride, logit_offset, select_bias, T, E, k, \
+                                       score, renormalize, scale, logits, write, topk_idx, topk_gate, s)
+  if (epl <= 1) MOE_TOPK(1);
+  if (epl <= 2) MOE_TOPK(2);
+  if (epl <= 4) MOE_TOPK(4);
+  if (epl <= 8) MOE_TOPK(8);
+  if (epl <= 16) MOE_TOPK(16);
+  MOE_TOPK(32);
+#undef MOE_TOPK
+}
+
+}  // namespace moe

@@ -1,0 +1,206 @@
+// Router statistics: per-expert load, aux load-balancing loss, router z-loss, drops,
+// max/mean load, coefficient of variation.
+//
+// Sources: "Hugging Face 图解 Mixture of Experts（MoE）原理、训练与推理权衡", the
+// auxiliary loss that pushes all experts toward equal importance (token load
+// balancing; simplified in section "Switch Transformer") and the router z-loss that
+// penalises large logits entering the gate (section "使用路由器 Z-loss 稳定训练").  The
+// pages print neither formula; the forms used are
+//   aux = E * sum_e f_e * P_e,  f_e = counts[e] / (T k),  P_e = mean_t p[t, e]
+//         (p = softmax(l) for softmax scoring, s / sum_e s otherwise),
+//   z   = mean_t (logsumexp_e l[t, e])^2.
+// Handbook article (zicq.com) "Router 与负载均衡为何决定训练成败": monitor the max
+// per-expert load ratio and the drop rate.
+//
+// Deterministic: stage 1 reduces each CTA's tokens into per-CTA partials in a fixed
+// order (fp64); stage 2 sums the partials in CTA order.
+#include "common.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kStatsThreads = 256;
+
+__device__ __forceinline__ float warp_max_f(float v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ double warp_sum_dd(double v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+template <int EPL>
+__global__ void __launch_bounds__(kStatsThreads)
+stats_partial_kernel(const float* __restrict__ logits, int T, int E, int score, int tokens_per_cta,
+                     double* __restrict__ partP, double* __restrict__ partZ) {
+  __shared__ double red[32 * EPL];            // running sum over warps, warp order
+  __shared__ double redz[kStatsThreads / 32];
+  const unsigned lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int nwarps = kStatsThreads / 32;
+  const long long t_begin = (long long)blockIdx.x * tokens_per_cta;
+  const long long t_end = min((long long)T, t_begin + tokens_per_cta);
+
+  double P[EPL];
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) P[i] = 0.0;
+  double z2 = 0.0;
+  for (long long t = t_begin + warp; t < t_end; t += nwarps) {
+    float l[EPL];
+    float mf = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      const int e = lane + 32 * i;
+      l[i] = e < E ? __ldg(logits + t * E + e) : -INFINITY;
+      mf = fmaxf(mf, l[i]);
+    }
+    const double m = (double)warp_max_f(mf);
+    double se = 0.0, ss = 0.0;
+    double sc[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+      const bool ok = lane + 32 * i < (unsigned)E;
+      const double ex = ok ? exp((double)l[i] - m) : 0.0;
+      se += ex;
+      double s = 0.0;
+      if (ok) {
+        if (score == MOE_SCORE_SOFTMAX) s = ex;
+        else if (score == MOE_SCORE_SIGMOID) s = 1.0 / (1.0 + exp(-(double)l[i]));
+        else s = sqrt(fmax((double)l[i], 0.0) + log1p(exp(-fabs((double)l[i]))));
+      }
+      sc[i] = s;
+      ss += s;
+    }
+    se = warp_sum_dd(se);
+    ss = warp_sum_dd(ss);
+    const double inv = 1.0 / ss;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) P[i] += sc[i] * inv;
+    const double lse = m + log(se);
+    z2 += lse * lse;
+  }
+  for (int w = 0; w < nwarps; ++w) {
+    if (warp == w) {
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) red[lane + 32 * i] = (w == 0 ? 0.0 : red[lane + 32 * i]) + P[i];
+    }
+    __syncthreads();
+  }
+  if (lane == 0) redz[warp] = z2;
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += kStatsThreads) partP[(long long)blockIdx.x * E + e] = red[e];
+  if (threadIdx.x == 0) {
+    double acc = 0.0;
+    for (int w = 0; w < nwarps; ++w) acc += redz[w];
+    partZ[blockIdx.x] = acc;
+  }
+}
+
+__device__ double block_sum_d(double v, double* sh) {
+  const unsigned lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  v = warp_sum_dd(v);
+  __syncthreads();
+  if (lane == 0) sh[warp] = v;
+  __syncthreads();
+  double r = 0.0;
+  const int nw = (blockDim.x + 31) >> 5;
+  for (int w = 0; w < nw; ++w) r += sh[w];
+  return r;
+}
+
+__global__ void __launch_bounds__(1024)
+stats_final_kernel(const double* __restrict__ partP, const double* __restrict__ partZ, int nparts,
+                   const int32_t* __restrict__ counts, const int32_t* __restrict__ kept, int T, int E,
+                   int k, float* __restrict__ load, float* __restrict__ stats5) {
+  __shared__ double sh[32];
+  const double TK = (double)T * k;
+  const double mean = TK / E;
+  double aux = 0.0, kept_sum = 0.0, var = 0.0, cmax = 0.0;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    double P = 0.0;
+    for (int b = 0; b < nparts; ++b) P += partP[(long long)b * E + e];
+    P /= (double)T;
+    const double c = (double)counts[e];
+    const double f = c / TK;
+    load[e] = (float)f;
+    aux += f * P;
+    kept_sum += (double)kept[e];
+    var += (c - mean) * (c - mean);
+    cmax = fmax(cmax, c);
+  }
+  aux = block_sum_d(aux, sh);
+  kept_sum = block_sum_d(kept_sum, sh);
+  var = block_sum_d(var, sh);
+  // block max
+  {
+    double v = cmax;
+#pragma unroll
+    for (int o = 16; o; o >>= 1) v = fmax(v, __shfl_xor_sync(0xffffffffu, v, o));
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0) sh[threadIdx.x >> 5] = v;
+    __syncthreads();
+    double r = 0.0;
+    for (int w = 0; w < (int)((blockDim.x + 31) >> 5); ++w) r = fmax(r, sh[w]);
+    cmax = r;
+  }
+  if (threadIdx.x == 0) {
+    double z = 0.0;
+    for (int b = 0; b < nparts; ++b) z += partZ[b];
+    stats5[0] = (float)(E * aux);
+    stats5[1] = (float)(z / (double)T);
+    stats5[2] = (float)(TK - kept_sum);
+    stats5[3] = (float)(cmax / mean);
+    stats5[4] = (float)(sqrt(var / E) / mean);
+  }
+}
+
+int stats_parts(int T) {
+  const int want = 2 * num_sms();
+  int parts = (T + 31) / 32;           // at least 32 tokens per CTA
+  return parts < want ? (parts < 1 ? 1 : parts) : want;
+}
+
+template <int EPL>
+moe_status run_partial(const float* logits, int T, int E, int score, int parts, double* pP, double* pZ,
+                       cudaStream_t s) {
+  const int tpc = (T + parts - 1) / parts;
+  stats_partial_kernel<EPL><<<parts, kStatsThreads, 0, s>>>(logits, T, E, score, tpc, pP, pZ);
+  return check_launch();
+}
+
+}  // namespace
+
+size_t router_stats_workspace_bytes(int T, int E) {
+  const int parts = stats_parts(T > 0 ? T : 1);
+  return ((size_t)parts * E + parts) * sizeof(double);
+}
+
+moe_status launch_router_stats(const float* logits, const int32_t* counts, const int32_t* kept,
+                               int T, int E, int k, int score, float* load, float* stats5,
+                               void* ws, cudaStream_t s) {
+  if (T == 0) {
+    moe_status st = cuda_status(cudaMemsetAsync(load, 0, (size_t)E * 4, s));
+    if (st == MOE_OK) st = cuda_status(cudaMemsetAsync(stats5, 0, 5 * 4, s));
+    return st;
+  }
+  const int parts = stats_parts(T);
+  double* pP = static_cast<double*>(ws);
+  double* pZ = pP + (size_t)parts * E;
+  const int epl = (E + 31) / 32;
+  moe_status st;
+  if (epl <= 1) st = run_partial<1>(logits, T, E, score, parts, pP, pZ, s);
+  else if (epl <= 2) st = run_partial<2>(logits, T, E, score, parts, pP, pZ, s);
+  else if (epl <= 4) st = run_partial<4>(logits, T, E, score, parts, pP, pZ, s);
+  else if (epl <= 8) st = run_partial<8>(logits, T, E, score, parts, pP, pZ, s);
+  else if (epl <= 16) st = run_partial<16>(logits, T, E, score, parts, pP, pZ, s);
+  else st = run_partial<32>(logits, T, E, score, parts, pP, pZ, s);
+  if (st != MOE_OK) return st;
+  stats_final_kernel<<<1, 1024, 0, s>>>(pP, pZ, parts, counts, kept, T, E, k, load, stats5);
+  return check_launch();
+}
+
+}  // namespace moe

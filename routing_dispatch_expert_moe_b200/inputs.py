@@ -167,6 +167,25 @@ def gen_experts(cfg: MoEConfig, seed: int = 0, threads: Optional[int] = None):
     return W_gu, W_dn
 
 
+def gen_experts_torch(cfg: MoEConfig, seed: int = 0, threads: Optional[int] = None):
+    """All experts as host torch tensors in the storage dtype (bf16 or fp32):
+    W_gu [E, 2F, d], W_dn [E, d, F].  Same values as gen_expert(cfg, e, seed)."""
+    import torch
+    dt = torch.float32 if cfg.act == "f32" else torch.bfloat16
+    W_gu = torch.empty((cfg.E, 2 * cfg.F, cfg.d), dtype=dt)
+    W_dn = torch.empty((cfg.E, cfg.d, cfg.F), dtype=dt)
+
+    def one(e):
+        a, b = gen_expert(cfg, e, seed)
+        W_gu[e].copy_(torch.from_numpy(a))      # values are already exact in dt
+        W_dn[e].copy_(torch.from_numpy(b))
+
+    threads = threads or min(16, os.cpu_count() or 1)
+    with ThreadPoolExecutor(threads) as ex:
+        list(ex.map(one, range(cfg.E)))
+    return W_gu, W_dn
+
+
 def small_config(name: str = "small", **kw) -> MoEConfig:
     """A small bf16 configuration for quick tests (overridable)."""
     base = dict(name=name, T=300, d=128, E=16, k=4, F=128, score="softmax")

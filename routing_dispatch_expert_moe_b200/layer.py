@@ -1,0 +1,131 @@
+"""MoE-layer forward as a sequence of the library's C-ABI calls.
+
+MoELayer owns preallocated device buffers for a maximum token count and runs, on one
+stream with no host synchronisation:
+
+    moe_route -> moe_histogram_scan -> moe_permute -> moe_expert_gate_up
+      -> moe_expert_down (gate fused) [-> shared expert: gate_up/down with E = 1]
+      -> moe_combine [-> moe_router_stats]
+
+Orchestration only: every step runs in the library's CUDA kernels.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+from . import moe as M
+
+
+@dataclass
+class MoEWeights:
+    Wg: torch.Tensor                          # [d, E] f32
+    W_gu: torch.Tensor                        # [E, 2F, d] act dtype (gate rows, then up rows)
+    W_dn: torch.Tensor                        # [E, d, F] act dtype
+    logit_offset: Optional[torch.Tensor] = None   # [E] f32
+    select_bias: Optional[torch.Tensor] = None    # [E] f32
+    W_gu_s: Optional[torch.Tensor] = None     # [1, 2F_s, d] shared expert
+    W_dn_s: Optional[torch.Tensor] = None     # [1, d, F_s]
+
+
+class MoELayer:
+    def __init__(self, weights: MoEWeights, k: int, T_max: int, score: str = "softmax",
+                 renormalize: bool = True, scale: float = 1.0, capacity: int = -1):
+        w = weights
+        self.w = w
+        self.d, self.E = w.Wg.shape
+        self.F = w.W_dn.shape[2]
+        self.k, self.T_max = k, T_max
+        self.score, self.renormalize, self.scale, self.capacity = score, renormalize, scale, capacity
+        self.dtype = w.W_gu.dtype
+        dev = w.Wg.device
+        self.device = dev
+        E, d, F = self.E, self.d, self.F
+        self.rows_max = M.moe_rows_max(T_max, E, k, capacity)
+        R = max(self.rows_max, 1)
+        f32, i32 = torch.float32, torch.int32
+        self.logits = torch.empty((T_max, E), dtype=f32, device=dev)
+        self.topk_idx = torch.empty((T_max, k), dtype=i32, device=dev)
+        self.topk_gate = torch.empty((T_max, k), dtype=f32, device=dev)
+        self.counts = torch.empty(E, dtype=i32, device=dev)
+        self.kept = torch.empty(E, dtype=i32, device=dev)
+        self.offsets = torch.empty(E + 1, dtype=i32, device=dev)
+        self.row_of = torch.empty((T_max, k), dtype=i32, device=dev)
+        self.token_of_row = torch.empty(R, dtype=i32, device=dev)
+        self.gate_of_row = torch.empty(R, dtype=f32, device=dev)
+        self.x_perm = torch.empty((R, d), dtype=self.dtype, device=dev)
+        self.h = torch.empty((R, F), dtype=self.dtype, device=dev)
+        self.y_perm = torch.empty((R, d), dtype=self.dtype, device=dev)
+        self.y = torch.empty((T_max, d), dtype=self.dtype, device=dev)
+        self.load = torch.empty(E, dtype=f32, device=dev)
+        self.stats5 = torch.empty(5, dtype=f32, device=dev)
+        self.ws = torch.empty(max(M.moe_workspace_bytes(T_max, d, E, k), 16), dtype=torch.uint8, device=dev)
+        self.has_shared = w.W_gu_s is not None
+        if self.has_shared:
+            self.F_s = w.W_dn_s.shape[2]
+            self.shared_offsets = torch.tensor([0, T_max], dtype=i32, device=dev)
+            self.h_s = torch.empty((T_max, self.F_s), dtype=self.dtype, device=dev)
+            self.y_s = torch.empty((T_max, d), dtype=self.dtype, device=dev)
+
+    # individual steps (so that a caller can time them one by one)
+    def route(self, x, stream=None):
+        M.moe_route(x, self.w.Wg, self.k, self.score, self.renormalize, self.scale, self.w.logit_offset,
+                    self.w.select_bias, self.logits[:x.shape[0]], self.topk_idx[:x.shape[0]],
+                    self.topk_gate[:x.shape[0]], self.ws, stream)
+
+    def histogram_scan(self, T, stream=None):
+        M.moe_histogram_scan(self.topk_idx[:T], self.topk_gate[:T], self.E, self.capacity, self.counts, self.kept,
+                             self.offsets, self.row_of[:T], self.token_of_row, self.gate_of_row, self.ws, stream)
+
+    def permute(self, x, stream=None):
+        M.moe_permute(x, self.row_of[:x.shape[0]], self.rows_max, self.x_perm, stream)
+
+    def gate_up(self, stream=None):
+        M.moe_expert_gate_up(self.x_perm, self.offsets, self.w.W_gu, self.rows_max, self.h, stream)
+
+    def down(self, stream=None):
+        M.moe_expert_down(self.h, self.offsets, self.w.W_dn, self.rows_max, self.gate_of_row, self.y_perm, stream)
+
+    def shared(self, x, stream=None):
+        T = x.shape[0]
+        if T != self.T_max:
+            self.shared_offsets[1].fill_(T)
+        M.moe_expert_gate_up(x, self.shared_offsets, self.w.W_gu_s, T, self.h_s[:T], stream)
+        M.moe_expert_down(self.h_s[:T], self.shared_offsets, self.w.W_dn_s, T, None, self.y_s[:T], stream)
+
+    def combine(self, T, stream=None):
+        M.moe_combine(self.y_perm, self.row_of[:T], T, self.rows_max, None,
+                      self.y_s[:T] if self.has_shared else None, self.y[:T], stream)
+
+    def stats(self, T, stream=None):
+        M.moe_router_stats(self.logits[:T], self.counts, self.kept, self.k, self.score, self.load, self.stats5,
+                           self.ws, stream)
+
+    def forward(self, x: torch.Tensor, stream=None, with_stats: bool = True) -> torch.Tensor:
+        T = x.shape[0]
+        if T > self.T_max:
+            raise ValueError(f"T={T} exceeds T_max={self.T_max}")
+        if x.dtype != self.dtype and not (self.dtype == torch.float32 and x.dtype == torch.float32):
+            raise ValueError(f"x must be {self.dtype}")
+        self.route(x, stream)
+        self.histogram_scan(T, stream)
+        self.permute(x, stream)
+        self.gate_up(stream)
+        self.down(stream)
+        if self.has_shared:
+            self.shared(x, stream)
+        self.combine(T, stream)
+        if with_stats:
+            self.stats(T, stream)
+        return self.y[:T]
+
+    # library kernels launched by one forward (the scan's workspace memset is not a kernel)
+    def launches_per_forward(self, with_stats: bool = True) -> int:
+        n = 2 + 2 + 1 + 1 + 1 + 1          # route(2) scan(2) permute gate_up down combine
+        if self.has_shared:
+            n += 2
+        if with_stats:
+            n += 2
+        return n

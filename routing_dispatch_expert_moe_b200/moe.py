@@ -1,0 +1,292 @@
+"""Python binding of libmoe_b200.so (include/moe.h): argument marshalling only.
+
+Every function here has the name of the C entry point it calls.  Tensors are torch
+CUDA tensors (torch supplies device memory and the current stream); outputs that are
+not passed in are allocated with torch.empty.  All arithmetic runs in the library's
+CUDA kernels -- there is no CPU or PyTorch fallback: if the shared library is missing
+or fails to load, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.environ.get("MOE_B200_LIB", os.path.join(_HERE, "libmoe_b200.so"))
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_DEVICE = range(6)
+SCORE = {"softmax": 0, "sigmoid": 1, "sqrt_softplus": 2}
+DTYPE = {torch.bfloat16: 0, torch.float32: 1}
+DEVERR = {0: "none", 1: "expert id out of range", 2: "duplicate expert in a token", 3: "row index out of range",
+          4: "scan look-back timeout", 5: "GEMM pipeline timeout"}
+
+_c_void_p, _i32, _i64, _f32, _f64, _size = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float,
+                                             ctypes.c_double, ctypes.c_size_t)
+
+# name -> (restype, argtypes), mirroring include/moe.h
+_SIGNATURES = {
+    "moe_version": (_i32, []),
+    "moe_status_str": (ctypes.c_char_p, [_i32]),
+    "moe_last_cuda_error": (ctypes.c_char_p, []),
+    "moe_capacity": (_i32, [_i32, _i32, _i32, _f64, _i32]),
+    "moe_rows_max": (_i64, [_i32, _i32, _i32, _i32]),
+    "moe_route_workspace_bytes": (_size, [_i32, _i32, _i32]),
+    "moe_route": (_i32, [_c_void_p, _i32, _c_void_p, _c_void_p, _c_void_p, _i32, _i32, _i32, _i32, _i32, _i32,
+                         _f32, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _size, _c_void_p]),
+    "moe_histogram_scan_workspace_bytes": (_size, [_i32, _i32, _i32]),
+    "moe_histogram_scan": (_i32, [_c_void_p, _c_void_p, _i32, _i32, _i32, _i32, _c_void_p, _c_void_p, _c_void_p,
+                                  _c_void_p, _c_void_p, _c_void_p, _c_void_p, _size, _c_void_p]),
+    "moe_permute": (_i32, [_c_void_p, _i32, _i32, _i32, _i32, _c_void_p, _i64, _c_void_p, _c_void_p]),
+    "moe_expert_gate_up": (_i32, [_c_void_p, _i32, _c_void_p, _i32, _i32, _i32, _i64, _c_void_p, _c_void_p,
+                                  _c_void_p]),
+    "moe_expert_down": (_i32, [_c_void_p, _i32, _c_void_p, _i32, _i32, _i32, _i64, _c_void_p, _c_void_p,
+                               _c_void_p, _c_void_p]),
+    "moe_grouped_ffn": (_i32, [_c_void_p, _i32, _c_void_p, _i32, _i32, _i32, _i64, _c_void_p, _c_void_p,
+                               _c_void_p, _c_void_p, _c_void_p, _c_void_p]),
+    "moe_combine": (_i32, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _i32, _i32, _i32, _i32, _i64, _c_void_p,
+                           _c_void_p]),
+    "moe_router_stats_workspace_bytes": (_size, [_i32, _i32]),
+    "moe_router_stats": (_i32, [_c_void_p, _c_void_p, _c_void_p, _i32, _i32, _i32, _i32, _c_void_p, _c_void_p,
+                                _c_void_p, _size, _c_void_p]),
+    "moe_workspace_bytes": (_size, [_i32, _i32, _i32, _i32]),
+    "moe_get_device_error": (_i32, [ctypes.POINTER(_i32), _c_void_p]),
+}
+
+_lib = None
+
+
+class MoEError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        name = lib().moe_status_str(status).decode()
+        extra = ""
+        if status == MOE_ERR_CUDA:
+            extra = ": " + lib().moe_last_cuda_error().decode()
+        super().__init__(f"{fn} failed with {name}{extra}")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library (raises if it is missing: no fallback exists)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} not found; build it with "
+                               "`python -m routing_dispatch_expert_moe_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGNATURES.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def exported_symbols():
+    return sorted(_SIGNATURES)
+
+
+# ---------------------------------------------------------------- helpers
+def _p(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t: torch.Tensor, name: str, dtype=None, shape=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype not in DTYPE:
+        raise ValueError(f"unsupported dtype {t.dtype} (bf16 or fp32)")
+    return DTYPE[t.dtype]
+
+
+def _check(fn: str, status: int):
+    if status != MOE_OK:
+        raise MoEError(fn, status)
+
+
+def _ws(nbytes: int, device, given: Optional[torch.Tensor]) -> Optional[torch.Tensor]:
+    if nbytes == 0:
+        return given
+    if given is not None and given.numel() * given.element_size() >= nbytes:
+        return given
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+# ---------------------------------------------------------------- sizes
+def moe_capacity(T: int, E: int, k: int, capacity_factor: Optional[float], per_assignment: bool = True) -> int:
+    return int(lib().moe_capacity(T, E, k, float(capacity_factor or 0.0), 1 if per_assignment else 0))
+
+
+def moe_rows_max(T: int, E: int, k: int, capacity: int) -> int:
+    return int(lib().moe_rows_max(T, E, k, capacity))
+
+
+def moe_workspace_bytes(T: int, d: int, E: int, k: int) -> int:
+    return int(lib().moe_workspace_bytes(T, d, E, k))
+
+
+# ---------------------------------------------------------------- the calls
+def moe_route(x, Wg, k: int, score: str = "softmax", renormalize: bool = True, scale: float = 1.0,
+              logit_offset=None, select_bias=None, logits=None, topk_idx=None, topk_gate=None,
+              workspace=None, stream=None):
+    """Router logits, top-k and gates.  Returns (logits [T,E] f32, topk_idx [T,k] i32, topk_gate [T,k] f32)."""
+    T, d = x.shape
+    E = Wg.shape[1]
+    _need(x, "x")
+    _need(Wg, "Wg", torch.float32, (d, E))
+    for t, n in ((logit_offset, "logit_offset"), (select_bias, "select_bias")):
+        if t is not None:
+            _need(t, n, torch.float32, (E,))
+    dev = x.device
+    logits = torch.empty((T, E), dtype=torch.float32, device=dev) if logits is None else \
+        _need(logits, "logits", torch.float32, (T, E))
+    topk_idx = torch.empty((T, k), dtype=torch.int32, device=dev) if topk_idx is None else \
+        _need(topk_idx, "topk_idx", torch.int32, (T, k))
+    topk_gate = torch.empty((T, k), dtype=torch.float32, device=dev) if topk_gate is None else \
+        _need(topk_gate, "topk_gate", torch.float32, (T, k))
+    nb = int(lib().moe_route_workspace_bytes(T, d, E))
+    ws = _ws(nb, dev, workspace)
+    _check("moe_route", lib().moe_route(_p(x), _dt(x), _p(Wg), _p(logit_offset), _p(select_bias), T, d, E, k,
+                                        SCORE[score], 1 if renormalize else 0, float(scale), _p(logits),
+                                        _p(topk_idx), _p(topk_gate), _p(ws), nb, _stream(stream)))
+    return logits, topk_idx, topk_gate
+
+
+def moe_histogram_scan(topk_idx, topk_gate, E: int, capacity: int = -1, counts=None, kept=None, offsets=None,
+                       row_of=None, token_of_row=None, gate_of_row=None, workspace=None, stream=None):
+    """Returns dict(counts, kept, offsets, row_of, token_of_row, gate_of_row, rows_max)."""
+    T, k = topk_idx.shape
+    _need(topk_idx, "topk_idx", torch.int32)
+    _need(topk_gate, "topk_gate", torch.float32, (T, k))
+    dev = topk_idx.device
+    rows_max = moe_rows_max(T, E, k, capacity)
+    mk = lambda t, shape, dt, n: torch.empty(shape, dtype=dt, device=dev) if t is None else _need(t, n, dt)
+    counts = mk(counts, (E,), torch.int32, "counts")
+    kept = mk(kept, (E,), torch.int32, "kept")
+    offsets = mk(offsets, (E + 1,), torch.int32, "offsets")
+    row_of = mk(row_of, (T, k), torch.int32, "row_of")
+    token_of_row = mk(token_of_row, (max(rows_max, 1),), torch.int32, "token_of_row")
+    gate_of_row = mk(gate_of_row, (max(rows_max, 1),), torch.float32, "gate_of_row")
+    nb = int(lib().moe_histogram_scan_workspace_bytes(T, k, E))
+    ws = _ws(nb, dev, workspace)
+    _check("moe_histogram_scan", lib().moe_histogram_scan(
+        _p(topk_idx), _p(topk_gate), T, k, E, capacity, _p(counts), _p(kept), _p(offsets), _p(row_of),
+        _p(token_of_row), _p(gate_of_row), _p(ws), nb, _stream(stream)))
+    return {"counts": counts, "kept": kept, "offsets": offsets, "row_of": row_of, "token_of_row": token_of_row,
+            "gate_of_row": gate_of_row, "rows_max": rows_max}
+
+
+def moe_permute(x, row_of, rows_max: int, x_perm=None, stream=None):
+    T, d = x.shape
+    k = row_of.shape[1]
+    _need(x, "x")
+    _need(row_of, "row_of", torch.int32, (T, k))
+    x_perm = torch.empty((max(rows_max, 1), d), dtype=x.dtype, device=x.device) if x_perm is None else \
+        _need(x_perm, "x_perm", x.dtype)
+    _check("moe_permute", lib().moe_permute(_p(x), _dt(x), T, d, k, _p(row_of), rows_max, _p(x_perm),
+                                            _stream(stream)))
+    return x_perm
+
+
+def moe_expert_gate_up(x_rows, offsets, W_gu, rows_max: int, h=None, stream=None):
+    E, F2, d = W_gu.shape
+    F = F2 // 2
+    _need(x_rows, "x_rows")
+    _need(offsets, "offsets", torch.int32, (E + 1,))
+    _need(W_gu, "W_gu", x_rows.dtype)
+    h = torch.empty((max(rows_max, 1), F), dtype=x_rows.dtype, device=x_rows.device) if h is None else \
+        _need(h, "h", x_rows.dtype)
+    _check("moe_expert_gate_up", lib().moe_expert_gate_up(_p(x_rows), _dt(x_rows), _p(offsets), E, d, F, rows_max,
+                                                          _p(W_gu), _p(h), _stream(stream)))
+    return h
+
+
+def moe_expert_down(h, offsets, W_dn, rows_max: int, gate_of_row=None, y_rows=None, stream=None):
+    E, d, F = W_dn.shape
+    _need(h, "h")
+    _need(offsets, "offsets", torch.int32, (E + 1,))
+    _need(W_dn, "W_dn", h.dtype)
+    if gate_of_row is not None:
+        _need(gate_of_row, "gate_of_row", torch.float32)
+    y_rows = torch.empty((max(rows_max, 1), d), dtype=h.dtype, device=h.device) if y_rows is None else \
+        _need(y_rows, "y_rows", h.dtype)
+    _check("moe_expert_down", lib().moe_expert_down(_p(h), _dt(h), _p(offsets), E, d, F, rows_max, _p(W_dn),
+                                                    _p(gate_of_row), _p(y_rows), _stream(stream)))
+    return y_rows
+
+
+def moe_grouped_ffn(x_rows, offsets, W_gu, W_dn, rows_max: int, gate_of_row=None, h=None, y_rows=None,
+                    stream=None):
+    E, F2, d = W_gu.shape
+    F = F2 // 2
+    _need(x_rows, "x_rows")
+    _need(offsets, "offsets", torch.int32, (E + 1,))
+    _need(W_gu, "W_gu", x_rows.dtype)
+    _need(W_dn, "W_dn", x_rows.dtype, (E, d, F))
+    dev = x_rows.device
+    h = torch.empty((max(rows_max, 1), F), dtype=x_rows.dtype, device=dev) if h is None else _need(h, "h")
+    y_rows = torch.empty((max(rows_max, 1), d), dtype=x_rows.dtype, device=dev) if y_rows is None else \
+        _need(y_rows, "y_rows")
+    _check("moe_grouped_ffn", lib().moe_grouped_ffn(_p(x_rows), _dt(x_rows), _p(offsets), E, d, F, rows_max,
+                                                    _p(W_gu), _p(W_dn), _p(gate_of_row), _p(h), _p(y_rows),
+                                                    _stream(stream)))
+    return y_rows
+
+
+def moe_combine(y_rows, row_of, T: int, rows_max: int, topk_gate=None, shared_y=None, y=None, stream=None):
+    d = y_rows.shape[1]
+    k = row_of.shape[1]
+    _need(y_rows, "y_rows")
+    _need(row_of, "row_of", torch.int32, (T, k))
+    if shared_y is not None:
+        _need(shared_y, "shared_y", y_rows.dtype, (T, d))
+    if topk_gate is not None:
+        _need(topk_gate, "topk_gate", torch.float32, (T, k))
+    y = torch.empty((T, d), dtype=y_rows.dtype, device=y_rows.device) if y is None else _need(y, "y", y_rows.dtype)
+    _check("moe_combine", lib().moe_combine(_p(y_rows), _p(row_of), _p(topk_gate), _p(shared_y), _dt(y_rows), T, d,
+                                            k, rows_max, _p(y), _stream(stream)))
+    return y
+
+
+def moe_router_stats(logits, counts, kept, k: int, score: str = "softmax", load=None, stats5=None, workspace=None,
+                     stream=None):
+    """Returns (load [E] f32, stats5 [5] f32 = aux, z, dropped, max_over_mean, cv)."""
+    T, E = logits.shape
+    _need(logits, "logits", torch.float32)
+    _need(counts, "counts", torch.int32, (E,))
+    _need(kept, "kept", torch.int32, (E,))
+    dev = logits.device
+    load = torch.empty(E, dtype=torch.float32, device=dev) if load is None else _need(load, "load", torch.float32)
+    stats5 = torch.empty(5, dtype=torch.float32, device=dev) if stats5 is None else \
+        _need(stats5, "stats5", torch.float32)
+    nb = int(lib().moe_router_stats_workspace_bytes(T, E))
+    ws = _ws(nb, dev, workspace)
+    _check("moe_router_stats", lib().moe_router_stats(_p(logits), _p(counts), _p(kept), T, E, k, SCORE[score],
+                                                      _p(load), _p(stats5), _p(ws), nb, _stream(stream)))
+    return load, stats5
+
+
+def moe_get_device_error(stream=None) -> int:
+    """Reads and clears the device error word (synchronises the stream); returns the code."""
+    code = _i32(0)
+    st = lib().moe_get_device_error(ctypes.byref(code), _stream(stream))
+    if st not in (MOE_OK, MOE_ERR_DEVICE):
+        raise MoEError("moe_get_device_error", st)
+    return int(code.value)

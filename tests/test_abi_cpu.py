@@ -1,0 +1,159 @@
+"""C-ABI checks that need no GPU: the library builds and loads, exports every entry point
+include/moe.h declares, and its host-side logic (capacity, sizes, validation) behaves.
+
+Every validation case below is rejected on the host before any launch, so none of
+them touches device memory even on a machine that has a GPU.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from tests._closed_form import load
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from routing_dispatch_expert_moe_b200 import build
+    build.build()
+    from routing_dispatch_expert_moe_b200 import moe
+    return moe.lib()
+
+
+def declared_symbols():
+    txt = open(os.path.join(ROOT, "include", "moe.h")).read()
+    return sorted(set(re.findall(r"^MOE_API [^(]*?\b(moe_\w+)\(", txt, flags=re.M)))
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_symbols()
+    assert len(names) >= 17
+    for n in names:
+        assert hasattr(L, n), n
+    from routing_dispatch_expert_moe_b200 import moe
+    assert sorted(moe.exported_symbols()) == names      # binding covers the whole header
+
+
+def test_status_strings(L):
+    assert L.moe_status_str(0) == b"MOE_OK"
+    assert L.moe_status_str(3) == b"MOE_ERR_WORKSPACE"
+    assert L.moe_version() >= 10000
+
+
+def test_capacity_matches_closed_forms(L, golden_dir):
+    g = load(golden_dir, "capacity.json")
+    for c in g["cases"]:
+        assert L.moe_capacity(c["T"], c["E"], c["k"], c["cf"], 1) == c["per_assignment"], c
+        assert L.moe_capacity(c["T"], c["E"], c["k"], c["cf"], 0) == c["literal"], c
+    assert L.moe_capacity(10, 4, 2, 0.0, 1) == -1
+    assert L.moe_capacity(10, 0, 2, 1.0, 1) == -2
+
+
+def test_rows_max(L):
+    assert L.moe_rows_max(100, 8, 2, -1) == 200
+    assert L.moe_rows_max(100, 8, 2, 10) == 80
+    assert L.moe_rows_max(100, 8, 2, 1000) == 200
+    assert L.moe_rows_max(0, 8, 2, -1) == 0
+
+
+def test_workspace_queries(L):
+    assert L.moe_histogram_scan_workspace_bytes(8192, 8, 64) >= 8192 * 8 * 4
+    assert L.moe_router_stats_workspace_bytes(8192, 64) > 0
+    w = L.moe_workspace_bytes(8192, 2048, 64, 8)
+    assert w >= L.moe_histogram_scan_workspace_bytes(8192, 8, 64)
+    assert L.moe_histogram_scan_workspace_bytes(0, 8, 64) == 0
+
+
+FAKE = ctypes.c_void_p(4096)   # non-null, aligned; never dereferenced (host checks fail first)
+NUL = None
+
+
+def _route(L, **kw):
+    a = dict(x=FAKE, dt=0, Wg=FAKE, off=NUL, bias=NUL, T=64, d=128, E=16, k=4, score=0, renorm=1, scale=1.0,
+             logits=FAKE, idx=FAKE, gate=FAKE, ws=FAKE, wsb=1 << 30, s=NUL)
+    a.update(kw)
+    return L.moe_route(a["x"], a["dt"], a["Wg"], a["off"], a["bias"], a["T"], a["d"], a["E"], a["k"], a["score"],
+                       a["renorm"], a["scale"], a["logits"], a["idx"], a["gate"], a["ws"], a["wsb"], a["s"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(x=NUL), 1), (dict(Wg=NUL), 1), (dict(logits=NUL), 1), (dict(k=17), 1), (dict(k=0), 1),
+    (dict(E=0), 1), (dict(T=-1), 1), (dict(score=3), 1), (dict(dt=7), 1), (dict(renorm=2), 1),
+    (dict(scale=float("nan")), 1), (dict(E=1025, k=4), 2), (dict(k=33, E=64), 2), (dict(d=100), 2),
+    (dict(x=ctypes.c_void_p(4104)), 2),
+])
+def test_route_host_validation(L, kw, status):
+    assert _route(L, **kw) == status
+
+
+def test_route_workspace_check(L):
+    need = L.moe_route_workspace_bytes(64, 4096, 16)
+    if need:
+        assert _route(L, d=4096, wsb=need - 1) == 3
+        assert _route(L, d=4096, ws=NUL) == 3
+
+
+def test_route_empty_batch_is_ok_without_launch(L):
+    assert _route(L, T=0, x=NUL, logits=NUL, idx=NUL, gate=NUL) == 0
+
+
+def test_histogram_scan_host_validation(L):
+    f = L.moe_histogram_scan
+    ok = dict(idx=FAKE, g=FAKE, T=64, k=4, E=16, cap=-1, c=FAKE, kp=FAKE, o=FAKE, r=FAKE, t=FAKE, gr=FAKE,
+              ws=FAKE, wsb=1 << 30)
+
+    def call(**kw):
+        a = dict(ok)
+        a.update(kw)
+        return f(a["idx"], a["g"], a["T"], a["k"], a["E"], a["cap"], a["c"], a["kp"], a["o"], a["r"], a["t"],
+                 a["gr"], a["ws"], a["wsb"], NUL)
+
+    assert call(cap=-2) == 1
+    assert call(c=NUL) == 1
+    assert call(idx=NUL) == 1
+    assert call(wsb=16) == 3
+    assert call(ws=NUL) == 3
+    assert call(k=20) == 1
+    assert call(E=2000, k=4) == 2
+
+
+def test_ffn_host_validation(L):
+    f = L.moe_expert_gate_up
+    assert f(FAKE, 0, FAKE, 4, 100, 64, 128, FAKE, FAKE, NUL) == 2        # d % 8
+    assert f(FAKE, 0, FAKE, 4, 128, 60, 128, FAKE, FAKE, NUL) == 2        # F % 8
+    assert f(FAKE, 0, NUL, 4, 128, 64, 128, FAKE, FAKE, NUL) == 1         # offsets
+    assert f(FAKE, 0, FAKE, 0, 128, 64, 128, FAKE, FAKE, NUL) == 1        # E
+    assert f(FAKE, 9, FAKE, 4, 128, 64, 128, FAKE, FAKE, NUL) == 1        # dtype
+    assert f(ctypes.c_void_p(4100), 0, FAKE, 4, 128, 64, 128, FAKE, FAKE, NUL) == 2   # alignment
+    assert f(FAKE, 0, FAKE, 4, 128, 64, 0, FAKE, FAKE, NUL) == 0          # no rows: nothing to do
+    g = L.moe_expert_down
+    assert g(FAKE, 0, FAKE, 4, 128, 64, -1, FAKE, NUL, FAKE, NUL) == 1
+
+
+def test_permute_combine_host_validation(L):
+    assert L.moe_permute(FAKE, 0, 64, 100, 4, FAKE, 256, FAKE, NUL) == 2
+    assert L.moe_permute(NUL, 0, 64, 128, 4, FAKE, 256, FAKE, NUL) == 1
+    assert L.moe_permute(FAKE, 0, 64, 128, 40, FAKE, 256, FAKE, NUL) == 2
+    assert L.moe_permute(FAKE, 0, 0, 128, 4, FAKE, 0, FAKE, NUL) == 0
+    assert L.moe_combine(FAKE, NUL, NUL, NUL, 0, 64, 128, 4, 256, FAKE, NUL) == 1
+    assert L.moe_combine(FAKE, FAKE, NUL, ctypes.c_void_p(4097), 0, 64, 128, 4, 256, FAKE, NUL) == 2
+
+
+def test_router_stats_host_validation(L):
+    f = L.moe_router_stats
+    assert f(FAKE, FAKE, FAKE, 64, 16, 4, 5, FAKE, FAKE, FAKE, 1 << 30, NUL) == 1
+    assert f(FAKE, FAKE, FAKE, 64, 16, 4, 0, FAKE, FAKE, FAKE, 8, NUL) == 3
+    assert f(FAKE, NUL, FAKE, 64, 16, 4, 0, FAKE, FAKE, FAKE, 1 << 30, NUL) == 1
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    import importlib
+    import routing_dispatch_expert_moe_b200.moe as m
+    monkeypatch.setattr(m, "_lib", None)
+    monkeypatch.setattr(m, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError):
+        m.lib()
+    importlib.reload(m)

@@ -1,0 +1,200 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the same seeded
+inputs, element by element.  Small shapes compare every output of every step; the
+full-size workloads compare routing in full and expert outputs on a stratified token
+sample (each token's output depends only on its own row, routing and the weights).
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import moe_oracle as O
+from routing_dispatch_expert_moe_b200 import inputs as I
+from tests import gpu_util as U
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from routing_dispatch_expert_moe_b200 import moe
+    moe.lib()
+    yield
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+
+def full_check(cfg, seed=0, per_assignment=True, check_stats=True):
+    host, dev = U.make_inputs(cfg, seed)
+    cap = O.capacity(cfg.T, cfg.E, cfg.k, cfg.capacity_factor, per_assignment)
+    from routing_dispatch_expert_moe_b200 import moe as M
+    assert M.moe_capacity(cfg.T, cfg.E, cfg.k, cfg.capacity_factor, per_assignment) == cap
+    layer, g = U.gpu_forward(cfg, dev, cap)
+    gu, dn = U.expert_getters(host)
+    bf16 = cfg.act == "bf16"
+    c = U.cfg_dict(cfg)
+    o = O.layer_routing(c, host["x"], host["Wg"], host["off"], host["bias"], per_assignment)
+    assert o["capacity"] == cap
+    if host["bias"] is not None:
+        assert (O.decision_margin(o["keys"], cfg.k) > 1e-9).all(), "near-tie in the biased keys"
+    U.assert_routing_equal(g, o)
+    # permuted rows: exact copies
+    n = g["n_rows"]
+    xp = layer.x_perm[:n].float().cpu().numpy().astype(np.float64)
+    assert np.array_equal(xp, np.asarray(host["x"], np.float64)[o["token_of_row"]])
+    # expert outputs
+    xperm = O.permute(host["x"], o["row_of"], n)
+    yp_o = O.grouped_ffn(xperm, o["offsets"], gu, dn, o["gate_of_row"], bf16)
+    yp_g = layer.y_perm[:n].float().cpu().numpy().astype(np.float64)
+    if n:
+        U.assert_y_close(yp_g, yp_o, "y_perm")
+    sh = host["shared"]
+    ys = O.shared_expert(host["x"], sh[0], sh[1], bf16) if sh is not None else None
+    y_o = O.combine(yp_o, o["row_of"], ys, bf16)
+    if np.any(y_o):
+        U.assert_y_close(g["y"], y_o, "y")
+    else:
+        assert not np.any(g["y"])
+    if check_stats:
+        st = O.router_stats(o["logits"], o["counts"], o["kept"], cfg.k, cfg.score)
+        U.assert_stats_close(g, st)
+    return g, o
+
+
+SMALL = [
+    I.small_config("softmax_bf16", T=300, d=128, E=16, k=4, F=128),
+    I.small_config("sigmoid_bias_shared", T=257, d=256, E=32, k=8, F=192, F_s=256, score="sigmoid", scale=2.5,
+                   logit_offset="normal0.5", select_bias="uniform0.1"),
+    I.small_config("sqrt_softplus_capacity_zipf", T=1000, d=128, E=64, k=6, F=64, score="sqrt_softplus",
+                   capacity_factor=1.0, logit_offset="zipf1.2"),
+    I.small_config("softmax_no_renorm", T=200, d=64, E=12, k=3, F=64, renormalize=False),
+    I.small_config("ragged_multitile", T=2000, d=512, E=8, k=2, F=384),
+    I.small_config("dense_k_eq_E", T=64, d=64, E=4, k=4, F=64),
+    I.small_config("fp32_small", T=200, d=64, E=8, k=2, F=64, act="f32", capacity_factor=1.25),
+    I.small_config("bf16_d_below_tile", T=100, d=32, E=4, k=2, F=32),
+    I.small_config("sigmoid_nobias_E_odd", T=333, d=96, E=37, k=5, F=40, score="sigmoid"),
+]
+
+
+@pytest.mark.parametrize("cfg", SMALL, ids=lambda c: c.name)
+def test_small_full_parity(cfg):
+    full_check(cfg)
+
+
+def test_c1_tiny_both_capacity_readings():
+    cfg = I.CONFIGS["c1_tiny"]
+    g, o = full_check(cfg, per_assignment=True)
+    assert o["capacity"] == 80
+    g2, o2 = full_check(cfg, per_assignment=False)
+    assert o2["capacity"] == 40 and (o2["row_of"] < 0).any()
+
+
+def test_switch_top1_literal_capacity():
+    cfg = I.small_config("switch_top1", T=500, d=64, E=8, k=1, F=64, capacity_factor=1.25)
+    g, o = full_check(cfg, per_assignment=False)
+    assert o["capacity"] == O.capacity(500, 8, 1, 1.25, True)   # k = 1: both readings agree
+
+
+def test_capacity_zero_drops_everything():
+    cfg = I.small_config("cap0", T=64, d=64, E=4, k=2, F=64, F_s=64)
+    host, dev = U.make_inputs(cfg)
+    layer, g = U.gpu_forward(cfg, dev, 0)
+    assert (g["row_of"] == -1).all() and (g["kept"] == 0).all() and g["n_rows"] == 0
+    ys = O.shared_expert(host["x"], host["shared"][0], host["shared"][1], True)
+    U.assert_y_close(g["y"], ys, "y (shared only)")
+
+
+def test_single_token():
+    cfg = I.small_config("one_token", T=1, d=128, E=8, k=8, F=128)
+    full_check(cfg)
+
+
+def test_all_logits_tied_goes_to_lowest_experts():
+    cfg = I.small_config("ties", T=128, d=64, E=16, k=3, F=64)
+    host, dev = U.make_inputs(cfg)
+    dev["Wg"].zero_()
+    layer, g = U.gpu_forward(cfg, dev, -1)
+    assert (g["topk_idx"] == np.array([0, 1, 2])).all()
+    assert (g["counts"][:3] == 128).all() and (g["counts"][3:] == 0).all()
+    np.testing.assert_allclose(g["topk_gate"], 1.0 / 3, rtol=1e-6)
+
+
+def test_deterministic_run_to_run():
+    cfg = I.small_config("det", T=700, d=128, E=32, k=4, F=128, capacity_factor=1.0)
+    host, dev = U.make_inputs(cfg)
+    cap = O.capacity(cfg.T, cfg.E, cfg.k, 1.0)
+    _, a = U.gpu_forward(cfg, dev, cap)
+    _, b = U.gpu_forward(cfg, dev, cap)
+    for key in ("topk_idx", "topk_gate", "row_of", "offsets", "token_of_row", "y", "stats5"):
+        assert np.array_equal(a[key], b[key]), key
+
+
+def test_corrupt_expert_id_is_reported_not_trapped():
+    from routing_dispatch_expert_moe_b200 import moe as M
+    T, k, E = 64, 2, 8
+    idx = torch.randint(0, E, (T, k), dtype=torch.int32, device="cuda")
+    idx[:, 1] = (idx[:, 0] + 1) % E
+    idx[5, 0] = 99                                          # out of range
+    gate = torch.ones((T, k), dtype=torch.float32, device="cuda")
+    M.moe_get_device_error()
+    r = M.moe_histogram_scan(idx, gate, E, -1)
+    code = M.moe_get_device_error()
+    assert code == 1
+    assert int(r["row_of"][5, 0].item()) == -1
+    idx[5, 0] = idx[5, 1]                                   # duplicate expert in one token
+    M.moe_histogram_scan(idx, gate, E, -1)
+    assert M.moe_get_device_error() == 2
+
+
+# ---------------------------------------------------------------- full-size workloads
+def full_size_check(name, per_assignment=True, n_sample_random=700):
+    cfg = I.CONFIGS[name]
+    host, dev = U.make_inputs(cfg)
+    cap = O.capacity(cfg.T, cfg.E, cfg.k, cfg.capacity_factor, per_assignment)
+    layer, g = U.gpu_forward(cfg, dev, cap)
+    c = U.cfg_dict(cfg)
+    o = O.layer_routing(c, host["x"], host["Wg"], host["off"], host["bias"], per_assignment)
+    if host["bias"] is not None:
+        assert (O.decision_margin(o["keys"], cfg.k) > 1e-9).all(), "near-tie in the biased keys"
+    U.assert_routing_equal(g, o)
+    st = O.router_stats(o["logits"], o["counts"], o["kept"], cfg.k, cfg.score)
+    U.assert_stats_close(g, st)
+    toks = U.stratified_tokens(o, cap, n_random=n_sample_random)
+    assert len(toks) >= 1024
+    gu, dn = U.expert_getters(host)
+    sub = O.layer_outputs_for_tokens(toks, host["x"], o, gu, dn, True, shared=host["shared"])
+    # gated expert rows of the sampled tokens
+    rows = o["row_of"][toks]
+    kept = rows >= 0
+    yp_g = layer.y_perm[torch.from_numpy(rows[kept]).long().cuda()].float().cpu().numpy().astype(np.float64)
+    U.assert_y_close(yp_g, sub["slot_rows"][kept], "y_perm (sampled)")
+    ma, me = U.assert_y_close(g["y"][toks], sub["y"], "y (sampled)")
+    del layer, dev
+    torch.cuda.empty_cache()
+    return ma, me
+
+
+@pytest.mark.slow
+def test_c2_handbook_full_size():
+    full_size_check("c2_handbook")
+
+
+@pytest.mark.slow
+def test_c3_fine_grained_full_size():
+    full_size_check("c3_fine_grained")
+
+
+@pytest.mark.slow
+def test_c4_coarse_full_size():
+    full_size_check("c4_coarse")
+
+
+@pytest.mark.slow
+def test_c5_stress_full_size_per_assignment_capacity():
+    full_size_check("c5_stress", per_assignment=True)
+
+
+@pytest.mark.slow
+def test_c5_stress_full_size_literal_capacity():
+    full_size_check("c5_stress", per_assignment=False)
