@@ -98,8 +98,9 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
-def layer_roofline_ms(cfg, A, pk):
-    """Sum over steps of max(compute, memory) time at the measured peaks (algorithmic bytes / flops)."""
+def layer_roofline_ms(cfg, A, pk, rb=4, ob=4):
+    """Sum over steps of max(compute, memory) time at the measured peaks (algorithmic bytes / flops).
+    rb / ob: bytes per element of the gated rows / of the layer output."""
     T, d, E, k, F = cfg.T, cfg.d, cfg.E, cfg.k, cfg.F
     hbm = pk["hbm_gbs"] * 1e9
     tc = pk["bf16_tflops"] * 1e12
@@ -110,8 +111,8 @@ def layer_roofline_ms(cfg, A, pk):
         "histogram_scan": (T * k * 4 * 3 + A * 8) / hbm,
         "permute": (T * d * b + A * d * b) / hbm,
         "gate_up": max(4 * A * d * F / tc, (A * d * b + E * 2 * F * d * b + A * F * b) / hbm),
-        "down": max(2 * A * F * d / tc, (A * F * b + E * d * F * b + A * d * b) / hbm),
-        "combine": (A * d * b + T * d * b) / hbm,
+        "down": max(2 * A * F * d / tc, (A * F * b + E * d * F * b + A * d * rb) / hbm),
+        "combine": (A * d * rb + T * d * ob) / hbm,
         "stats": (T * E * 4) / hbm,
     }
     return sum(steps.values()) * 1e3, {k_: v * 1e3 for k_, v in steps.items()}
@@ -207,7 +208,7 @@ def run_ours(args):
 
     # end to end through the public API with host buffers (pinned), copies inside the timing
     x_host = torch.from_numpy(x_np).to(dt).pin_memory()
-    y_host = torch.empty((cfg.T, cfg.d), dtype=dt).pin_memory()
+    y_host = torch.empty((cfg.T, cfg.d), dtype=layer.out_dtype).pin_memory()
     e2e_steps = max(3, min(args.steps, 50))
     for _ in range(2):
         x.copy_(x_host, non_blocking=True)
@@ -231,14 +232,16 @@ def run_ours(args):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         e2e_ms = float(t.item())
     e2e_value = cfg.T * world * e2e_steps / (e2e_ms / 1e3)
-    nbytes = cfg.T * cfg.d * (2 if dt == torch.bfloat16 else 4)
+    h2d_bytes = x_host.numel() * x_host.element_size()
+    d2h_bytes = y_host.numel() * y_host.element_size()
 
     pk, pk_src = peaks()
     gate_up_ms = stage_ms["gate_up"]
     flops = 4.0 * A * cfg.d * cfg.F
     achieved = flops / (gate_up_ms * 1e-3) / 1e12
     peak = pk["bf16_tflops"]
-    roof_ms, roof_steps = layer_roofline_ms(cfg, A, pk)
+    rb, ob = layer.y_perm.element_size(), layer.y.element_size()
+    roof_ms, roof_steps = layer_roofline_ms(cfg, A, pk, rb, ob)
     traffic = GATE_UP_TRAFFIC.get(args.workload)
 
     out = None
@@ -253,8 +256,8 @@ def run_ours(args):
                        "F_shared": cfg.F_s, "score": cfg.score, "capacity": cap, "rows": A,
                        "parallelism": f"replicas x{world} (independent token batches, no collective)",
                        "l2": "flushed before every step (256 MB write)"},
-            "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": nbytes,
-                    "d2h_bytes_per_step": nbytes, "steps": e2e_steps},
+            "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d_bytes,
+                    "d2h_bytes_per_step": d2h_bytes, "steps": e2e_steps},
             "gpu_launches": args.steps * layer.launches_per_forward(True),
             "roofline": {"bound": "tensor", "kernel": "moe_expert_gate_up (tcgen05 grouped GEMM + SwiGLU)",
                          "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
@@ -267,7 +270,7 @@ def run_ours(args):
             "stage_throughput": {
                 "down_tflops": round(2.0 * A * cfg.F * cfg.d / (stage_ms["down"] * 1e-3) / 1e12, 1),
                 "permute_gbs": round((cfg.T * cfg.d * 2 + A * cfg.d * 2) / (stage_ms["permute"] * 1e-3) / 1e9, 1),
-                "combine_gbs": round((A * cfg.d * 2 + cfg.T * cfg.d * 2) / (stage_ms["combine"] * 1e-3) / 1e9, 1),
+                "combine_gbs": round((A * cfg.d * rb + cfg.T * cfg.d * ob) / (stage_ms["combine"] * 1e-3) / 1e9, 1),
                 "route_gbs": round((cfg.T * cfg.d * 2 + cfg.T * cfg.E * 8 + cfg.T * cfg.k * 8) /
                                    (stage_ms["route"] * 1e-3) / 1e9, 1),
             },

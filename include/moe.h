@@ -46,9 +46,12 @@
  *     ordered by key descending, then index ascending.
  *   - Routing indices, counts, offsets and row maps are exact integers and
  *     deterministic run to run.
- *   - Expert GEMMs take bf16 operands with fp32 accumulation; H and the gated expert
- *     rows are rounded to bf16 (round to nearest even); the combine sums in fp32 in
- *     slot order j = 0..k-1, then adds the shared expert, then rounds.
+ *   - Expert GEMMs take bf16 operands with fp32 accumulation; H is rounded to bf16
+ *     (round to nearest even) because it is the down GEMM's tensor-core operand.  The
+ *     gated expert rows and the layer output are written in the dtype the caller picks
+ *     (fp32 keeps H as the only rounding inside the layer; bf16 rounds each row and the
+ *     output once more).  The combine sums in fp32 in slot order j = 0..k-1, then adds
+ *     the shared expert, then converts to the output dtype.
  */
 #ifndef MOE_B200_H
 #define MOE_B200_H
@@ -187,7 +190,8 @@ MOE_API moe_status moe_permute(const void* x, int32_t dtype, int32_t T, int32_t 
  *   W_dn     (device) [E, d, F] dtype
  *   h        (device) [rows_max, F] dtype: H = silu(x W_gate^T) * (x W_up^T)
  *   gate_of_row (device) [rows_max] fp32 or NULL (NULL = weight 1, e.g. a shared expert)
- *   y_rows   (device) [rows_max, d] dtype out: gate_of_row * (H W_dn^T)
+ *   y_dtype  dtype of y_rows (MOE_F32 or MOE_BF16; any dtype may be paired with any y_dtype)
+ *   y_rows   (device) [rows_max, d] y_dtype out: gate_of_row * (H W_dn^T)
  * bf16 uses the tcgen05 tensor-core path; fp32 uses an fp32 SIMT path.  Rows at or
  * beyond offsets[E] are neither read into results nor written.
  * A shared expert is the call with E = 1, offsets = {0, T} and x_rows = x.
@@ -197,26 +201,26 @@ MOE_API moe_status moe_expert_gate_up(const void* x_rows, int32_t dtype, const i
                               const void* W_gu, void* h, void* stream);
 MOE_API moe_status moe_expert_down(const void* h, int32_t dtype, const int32_t* offsets,
                            int32_t E, int32_t d, int32_t F, int64_t rows_max,
-                           const void* W_dn, const float* gate_of_row, void* y_rows,
-                           void* stream);
+                           const void* W_dn, const float* gate_of_row, int32_t y_dtype,
+                           void* y_rows, void* stream);
 MOE_API moe_status moe_grouped_ffn(const void* x_rows, int32_t dtype, const int32_t* offsets,
                            int32_t E, int32_t d, int32_t F, int64_t rows_max,
                            const void* W_gu, const void* W_dn, const float* gate_of_row,
-                           void* h, void* y_rows, void* stream);
+                           void* h, int32_t y_dtype, void* y_rows, void* stream);
 
 /* ------------------------------------------------------------------------------------
  * moe_combine -- y[t] = sum_j g_j * y_rows[row_of[t, j]]  (+ shared_y[t]).
  * [MoE-Explained] section "什么是稀疏性？", eq. y = sum_i G(x)_i E_i(x).
- *   y_rows    (device) [rows_max, d] dtype
+ *   y_rows    (device) [rows_max, d] rows_dtype
  *   row_of    (device) [T, k]: -1 slots are skipped (a dropped assignment adds 0)
  *   topk_gate (device) [T, k] fp32, or NULL when y_rows already carry their gate
- *   shared_y  (device) [T, d] dtype or NULL: added with weight 1
- *   y         (device) [T, d] dtype out
+ *   shared_y  (device) [T, d] rows_dtype or NULL: added with weight 1
+ *   y         (device) [T, d] y_dtype out
  *   A row index >= rows_max is skipped (adds 0) and recorded as MOE_DEVERR_ROW.
  * ---------------------------------------------------------------------------------- */
-MOE_API moe_status moe_combine(const void* y_rows, const int32_t* row_of, const float* topk_gate,
-                       const void* shared_y, int32_t dtype, int32_t T, int32_t d, int32_t k,
-                       int64_t rows_max, void* y, void* stream);
+MOE_API moe_status moe_combine(const void* y_rows, int32_t rows_dtype, const int32_t* row_of,
+                       const float* topk_gate, const void* shared_y, int32_t T, int32_t d,
+                       int32_t k, int64_t rows_max, int32_t y_dtype, void* y, void* stream);
 
 /* ------------------------------------------------------------------------------------
  * moe_router_stats -- load-balance and stability statistics of one routing.

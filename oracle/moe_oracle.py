@@ -41,8 +41,10 @@ Readings taken where the pages are silent (each listed again in the design notes
   R8 the routing scale factor multiplies the gates after renormalisation.
   R9 expert FFN = SwiGLU: silu(x W_gate^T) * (x W_up^T), then W_down, no biases.
   R10 the shared expert is ungated (weight 1) and added after the routed sum.
-  R11 bf16 workloads round H, each gated expert output row, the shared output
-     and y to bf16 (round to nearest even); sums accumulate in float64 here.
+  R11 bf16 workloads round H to bf16 (round to nearest even): it is the operand of the
+     down projection, and the pages keep expert matmuls in bf16.  Gated expert rows,
+     the shared output and y stay unrounded unless a bf16 output is asked for
+     (round_rows / round_out); sums accumulate in float64 here.
   R12 router input: bf16 x upcast exactly; W_g and the logits in fp32 (exact on
      the generator's grids, so float64 here gives the same numbers).
   R13 an additive per-expert logit offset o[e] enters both selection and gates;
@@ -249,11 +251,11 @@ def silu(z):
     return z / (1.0 + np.exp(-z))
 
 
-def swiglu_expert(x_rows, W_gu, W_dn, bf16: bool) -> np.ndarray:
-    """One expert on a block of rows: (silu(x Wg^T) * (x Wu^T)) Wd^T, float64 accumulate.
+def expert_hidden(x_rows, W_gu, bf16: bool) -> np.ndarray:
+    """H = silu(x W_gate^T) * (x W_up^T) for one expert, float64 accumulate.
 
-    W_gu [2F, d]: rows 0..F-1 are W_gate, rows F..2F-1 are W_up;  W_dn [d, F].
-    bf16: H is rounded to bf16 before the down projection (R11).
+    W_gu [2F, d]: rows 0..F-1 are W_gate, rows F..2F-1 are W_up.
+    bf16: H is rounded to bf16, as it is before the down projection (R11).
     """
     x = np.asarray(x_rows, np.float64)
     W_gu = np.asarray(W_gu, np.float64)
@@ -261,16 +263,20 @@ def swiglu_expert(x_rows, W_gu, W_dn, bf16: bool) -> np.ndarray:
     g = x @ W_gu[:F].T
     u = x @ W_gu[F:].T
     h = silu(g) * u
-    if bf16:
-        h = bf16_round(h)
-    return h @ np.asarray(W_dn, np.float64).T
+    return bf16_round(h) if bf16 else h
 
 
-def grouped_ffn(x_perm, offsets, W_gu_of, W_dn_of, gate_of_row, bf16: bool) -> np.ndarray:
+def swiglu_expert(x_rows, W_gu, W_dn, bf16: bool) -> np.ndarray:
+    """One expert on a block of rows: H W_dn^T with H from expert_hidden; W_dn [d, F]."""
+    return expert_hidden(x_rows, W_gu, bf16) @ np.asarray(W_dn, np.float64).T
+
+
+def grouped_ffn(x_perm, offsets, W_gu_of, W_dn_of, gate_of_row, bf16: bool,
+                round_rows: bool = False) -> np.ndarray:
     """y_perm[r] = gate_of_row[r] * expert_e(x_perm[r]) for r in [offsets[e], offsets[e+1]).
 
     W_gu_of(e) / W_dn_of(e) return expert e's weights (arrays or callables).
-    bf16: each gated output row is rounded to bf16 (R11).
+    bf16: H is rounded to bf16; round_rows: each gated row is rounded to bf16 too (R11).
     """
     x_perm = np.asarray(x_perm, np.float64)
     E = len(offsets) - 1
@@ -282,7 +288,7 @@ def grouped_ffn(x_perm, offsets, W_gu_of, W_dn_of, gate_of_row, bf16: bool) -> n
             continue
         o = swiglu_expert(x_perm[a:b], _get(W_gu_of, e), _get(W_dn_of, e), bf16)
         o = o * (1.0 if gate_of_row is None else np.asarray(gate_of_row, np.float64)[a:b, None])
-        y[a:b] = bf16_round(o) if bf16 else o
+        y[a:b] = bf16_round(o) if round_rows else o
     return y
 
 
@@ -290,20 +296,21 @@ def _get(W, e):
     return W(e) if callable(W) else W[e]
 
 
-def shared_expert(x, W_gu_s, W_dn_s, bf16: bool) -> np.ndarray:
+def shared_expert(x, W_gu_s, W_dn_s, bf16: bool, round_out: bool = False) -> np.ndarray:
     """Always-on expert with weight 1 (R10; [Handbook-Digest] shared experts)."""
     y = swiglu_expert(x, W_gu_s, W_dn_s, bf16)
-    return bf16_round(y) if bf16 else y
+    return bf16_round(y) if round_out else y
 
 
 # ---------------------------------------------------------------------------
 # Combine  ([MoE-Explained] eq. y = sum_i G(x)_i E_i(x); R4, R10, R11)
 # ---------------------------------------------------------------------------
-def combine(y_perm, row_of: np.ndarray, shared_y=None, bf16: bool = True,
+def combine(y_perm, row_of: np.ndarray, shared_y=None, round_out: bool = False,
             topk_gate=None) -> np.ndarray:
     """y[t] = sum_j y_perm[row_of[t, j]] (dropped slots skipped) + shared_y[t].
 
     topk_gate given: rows are multiplied by their gate here (rows not gated yet).
+    round_out: y is rounded to bf16 (R11).
     """
     y_perm = np.asarray(y_perm, np.float64)
     T, k = row_of.shape
@@ -316,7 +323,7 @@ def combine(y_perm, row_of: np.ndarray, shared_y=None, bf16: bool = True,
         y[m] += rows
     if shared_y is not None:
         y += np.asarray(shared_y, np.float64)
-    return bf16_round(y) if bf16 else y
+    return bf16_round(y) if round_out else y
 
 
 # ---------------------------------------------------------------------------
@@ -338,12 +345,12 @@ def layer_routing(cfg_like: dict, x, Wg, logit_offset=None, select_bias=None,
 
 
 def layer_outputs_for_tokens(tokens, x, routing: dict, W_gu_of, W_dn_of, bf16: bool,
-                             shared=None) -> dict:
+                             shared=None, round_rows: bool = False, round_out: bool = False) -> dict:
     """y[t] (and each kept slot's gated expert row) for the listed tokens only.
 
     A token's output depends only on its own row, its routing and the weights,
     so evaluating a subset gives exactly the rows the full layer would.
-    shared: (W_gu_s, W_dn_s) or None.
+    shared: (W_gu_s, W_dn_s) or None.  Rounding flags as in grouped_ffn / combine.
     """
     tokens = np.asarray(tokens, np.int64)
     xs = np.asarray(np.asarray(x)[tokens], np.float64)          # the listed tokens only
@@ -358,25 +365,26 @@ def layer_outputs_for_tokens(tokens, x, routing: dict, W_gu_of, W_dn_of, bf16: b
         ii, jj = np.nonzero((idx == e) & kept)
         o = swiglu_expert(xs[ii], _get(W_gu_of, int(e)), _get(W_dn_of, int(e)), bf16)
         o = o * g[ii, jj][:, None]
-        slot_rows[ii, jj] = bf16_round(o) if bf16 else o
+        slot_rows[ii, jj] = bf16_round(o) if round_rows else o
     acc = np.zeros((n, d), np.float64)
     for j in range(k):                              # slot order; dropped slots are zero rows
         acc += slot_rows[:, j]
     if shared is not None:
-        acc += shared_expert(xs, shared[0], shared[1], bf16)
-    y = bf16_round(acc) if bf16 else acc
+        acc += shared_expert(xs, shared[0], shared[1], bf16, round_rows)
+    y = bf16_round(acc) if round_out else acc
     return {"y": y, "slot_rows": slot_rows}
 
 
 def layer_forward(cfg_like: dict, x, Wg, W_gu, W_dn, logit_offset=None, select_bias=None,
-                  shared=None, bf16: bool = True, per_assignment_capacity: bool = True) -> dict:
+                  shared=None, bf16: bool = True, per_assignment_capacity: bool = True,
+                  round_rows: bool = False, round_out: bool = False) -> dict:
     """The whole layer for all tokens (small sizes): routing, permute, grouped FFN, combine."""
     r = layer_routing(cfg_like, x, Wg, logit_offset, select_bias, per_assignment_capacity)
     n_rows = int(r["offsets"][-1])
     x_perm = permute(x, r["row_of"], n_rows)
-    y_perm = grouped_ffn(x_perm, r["offsets"], W_gu, W_dn, r["gate_of_row"], bf16)
-    ys = shared_expert(x, shared[0], shared[1], bf16) if shared is not None else None
-    y = combine(y_perm, r["row_of"], ys, bf16)
+    y_perm = grouped_ffn(x_perm, r["offsets"], W_gu, W_dn, r["gate_of_row"], bf16, round_rows)
+    ys = shared_expert(x, shared[0], shared[1], bf16, round_rows) if shared is not None else None
+    y = combine(y_perm, r["row_of"], ys, round_out)
     r.update({"x_perm": x_perm, "y_perm": y_perm, "shared_y": ys, "y": y})
     return r
 

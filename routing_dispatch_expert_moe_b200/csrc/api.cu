@@ -172,35 +172,40 @@ moe_status moe_expert_gate_up(const void* x_rows, int32_t dtype, const int32_t* 
 }
 
 moe_status moe_expert_down(const void* h, int32_t dtype, const int32_t* offsets, int32_t E, int32_t d, int32_t F,
-                           int64_t rows_max, const void* W_dn, const float* gate_of_row, void* y_rows, void* stream) {
+                           int64_t rows_max, const void* W_dn, const float* gate_of_row, int32_t y_dtype,
+                           void* y_rows, void* stream) {
   moe_status st = check_ffn(h, dtype, offsets, E, d, F, rows_max, W_dn, y_rows);
-  if (st != MOE_OK || rows_max == 0) return st;
+  if (st != MOE_OK) return st;
+  if (!dtype_ok(y_dtype)) return MOE_ERR_INVALID_ARG;
+  if (rows_max == 0) return MOE_OK;
   if (dtype == MOE_BF16) {
-    st = launch_down_tc(h, offsets, E, d, F, rows_max, W_dn, gate_of_row, y_rows, S(stream));
+    st = launch_down_tc(h, offsets, E, d, F, rows_max, W_dn, gate_of_row, y_dtype, y_rows, S(stream));
     if (st != MOE_ERR_UNSUPPORTED) return st;
   }
-  return launch_down_simt(h, dtype, offsets, E, d, F, rows_max, W_dn, gate_of_row, y_rows, S(stream));
+  return launch_down_simt(h, dtype, offsets, E, d, F, rows_max, W_dn, gate_of_row, y_dtype, y_rows, S(stream));
 }
 
 moe_status moe_grouped_ffn(const void* x_rows, int32_t dtype, const int32_t* offsets, int32_t E, int32_t d, int32_t F,
                            int64_t rows_max, const void* W_gu, const void* W_dn, const float* gate_of_row, void* h,
-                           void* y_rows, void* stream) {
+                           int32_t y_dtype, void* y_rows, void* stream) {
+  if (!dtype_ok(y_dtype)) return MOE_ERR_INVALID_ARG;
   moe_status st = moe_expert_gate_up(x_rows, dtype, offsets, E, d, F, rows_max, W_gu, h, stream);
   if (st != MOE_OK) return st;
-  return moe_expert_down(h, dtype, offsets, E, d, F, rows_max, W_dn, gate_of_row, y_rows, stream);
+  return moe_expert_down(h, dtype, offsets, E, d, F, rows_max, W_dn, gate_of_row, y_dtype, y_rows, stream);
 }
 
-moe_status moe_combine(const void* y_rows, const int32_t* row_of, const float* topk_gate, const void* shared_y,
-                       int32_t dtype, int32_t T, int32_t d, int32_t k, int64_t rows_max, void* y, void* stream) {
+moe_status moe_combine(const void* y_rows, int32_t rows_dtype, const int32_t* row_of, const float* topk_gate,
+                       const void* shared_y, int32_t T, int32_t d, int32_t k, int64_t rows_max, int32_t y_dtype,
+                       void* y, void* stream) {
   if (T < 0 || k < 1 || rows_max < 0) return MOE_ERR_INVALID_ARG;
   if (k > kMaxK || (long long)T >= kMaxT) return MOE_ERR_UNSUPPORTED;
   moe_status st = check_d(d);
   if (st != MOE_OK) return st;
-  if (!dtype_ok(dtype)) return MOE_ERR_INVALID_ARG;
+  if (!dtype_ok(rows_dtype) || !dtype_ok(y_dtype)) return MOE_ERR_INVALID_ARG;
   if (T == 0) return MOE_OK;
   if (!row_of || !y || (rows_max > 0 && !y_rows)) return MOE_ERR_INVALID_ARG;
   if (!aligned16(y_rows) || !aligned16(shared_y) || !aligned16(y)) return MOE_ERR_UNSUPPORTED;
-  return launch_combine(y_rows, row_of, topk_gate, shared_y, dtype, T, d, k, rows_max, y, S(stream));
+  return launch_combine(y_rows, rows_dtype, row_of, topk_gate, shared_y, T, d, k, rows_max, y_dtype, y, S(stream));
 }
 
 size_t moe_router_stats_workspace_bytes(int32_t T, int32_t E) {

@@ -113,8 +113,8 @@ size_t histogram_scan_workspace_bytes(int T, int k, int E);
 
 moe_status launch_permute(const void* x, int dtype, int T, int d, int k, const int32_t* row_of,
                           long long rows_max, void* x_perm, cudaStream_t s);
-moe_status launch_combine(const void* y_rows, const int32_t* row_of, const float* topk_gate,
-                          const void* shared_y, int dtype, int T, int d, int k, long long rows_max,
+moe_status launch_combine(const void* y_rows, int rows_dtype, const int32_t* row_of, const float* topk_gate,
+                          const void* shared_y, int T, int d, int k, long long rows_max, int y_dtype,
                           void* y, cudaStream_t s);
 
 moe_status launch_router_stats(const float* logits, const int32_t* counts, const int32_t* kept,
@@ -127,11 +127,11 @@ moe_status launch_gate_up_simt(const void* x_rows, int dtype, const int32_t* off
                                cudaStream_t s);
 moe_status launch_down_simt(const void* h, int dtype, const int32_t* offsets, int E, int d, int F,
                             long long rows_max, const void* W_dn, const float* gate_of_row,
-                            void* y_rows, cudaStream_t s);
+                            int y_dtype, void* y_rows, cudaStream_t s);
 moe_status launch_gate_up_tc(const void* x_rows, const int32_t* offsets, int E, int d, int F,
                              long long rows_max, const void* W_gu, void* h, cudaStream_t s);
 moe_status launch_down_tc(const void* h, const int32_t* offsets, int E, int d, int F,
                           long long rows_max, const void* W_dn, const float* gate_of_row,
-                          void* y_rows, cudaStream_t s);
+                          int y_dtype, void* y_rows, cudaStream_t s);
 
 }  // namespace moe

@@ -39,11 +39,13 @@ __device__ __forceinline__ void st_elem<__nv_bfloat16>(__nv_bfloat16* p, float v
 
 // MODE 0: gate_up (A = x_rows [*, d], B = W_gu [E][2F][d], out = H [*, F])
 // MODE 1: down    (A = H [*, F], B = W_dn [E][d][F], out = Y [*, d], scaled by gate_of_row)
-template <typename DT, int MODE>
+// OT: output element type (MODE 0 writes H in the activation dtype; MODE 1 writes the
+// gated rows in the caller's choice of bf16 or fp32).
+template <typename DT, int MODE, typename OT>
 __global__ void __launch_bounds__(kThreads)
 grouped_simt_kernel(const DT* __restrict__ A, const DT* __restrict__ B, const int32_t* __restrict__ offsets,
                     int E, int K, int N, int F, long long rows_max, const float* __restrict__ gate_of_row,
-                    DT* __restrict__ out, int* err) {
+                    OT* __restrict__ out, int* err) {
   __shared__ int tile_start[kMaxE + 1];
   __shared__ int sh32[32];
   __shared__ __align__(16) float As[kBK][kBM + 4];
@@ -122,19 +124,19 @@ grouped_simt_kernel(const DT* __restrict__ A, const DT* __restrict__ B, const in
         } else {
           v = acc[i][j] * gsc;
         }
-        st_elem(out + row * N + n, v);
+        st_elem<OT>(out + row * N + n, v);
       }
     }
   }
 }
 
-template <typename DT, int MODE>
+template <typename DT, int MODE, typename OT>
 moe_status run_simt(const void* A, const void* B, const int32_t* offsets, int E, int K, int N, int F,
                     long long rows_max, const float* gate_of_row, void* out, cudaStream_t s) {
   const int grid = 2 * num_sms();
-  grouped_simt_kernel<DT, MODE><<<grid, kThreads, 0, s>>>(
+  grouped_simt_kernel<DT, MODE, OT><<<grid, kThreads, 0, s>>>(
       static_cast<const DT*>(A), static_cast<const DT*>(B), offsets, E, K, N, F, rows_max, gate_of_row,
-      static_cast<DT*>(out), err_ptr());
+      static_cast<OT*>(out), err_ptr());
   return check_launch();
 }
 
@@ -144,17 +146,21 @@ moe_status launch_gate_up_simt(const void* x_rows, int dtype, const int32_t* off
                                int F, long long rows_max, const void* W_gu, void* h, cudaStream_t s) {
   if (rows_max == 0) return MOE_OK;
   if (dtype == MOE_F32)
-    return run_simt<float, 0>(x_rows, W_gu, offsets, E, d, F, F, rows_max, nullptr, h, s);
-  return run_simt<__nv_bfloat16, 0>(x_rows, W_gu, offsets, E, d, F, F, rows_max, nullptr, h, s);
+    return run_simt<float, 0, float>(x_rows, W_gu, offsets, E, d, F, F, rows_max, nullptr, h, s);
+  return run_simt<__nv_bfloat16, 0, __nv_bfloat16>(x_rows, W_gu, offsets, E, d, F, F, rows_max, nullptr, h, s);
 }
 
 moe_status launch_down_simt(const void* h, int dtype, const int32_t* offsets, int E, int d, int F,
                             long long rows_max, const void* W_dn, const float* gate_of_row,
-                            void* y_rows, cudaStream_t s) {
+                            int y_dtype, void* y_rows, cudaStream_t s) {
   if (rows_max == 0) return MOE_OK;
+  const bool f32out = y_dtype == MOE_F32;
   if (dtype == MOE_F32)
-    return run_simt<float, 1>(h, W_dn, offsets, E, F, d, F, rows_max, gate_of_row, y_rows, s);
-  return run_simt<__nv_bfloat16, 1>(h, W_dn, offsets, E, F, d, F, rows_max, gate_of_row, y_rows, s);
+    return f32out ? run_simt<float, 1, float>(h, W_dn, offsets, E, F, d, F, rows_max, gate_of_row, y_rows, s)
+                  : run_simt<float, 1, __nv_bfloat16>(h, W_dn, offsets, E, F, d, F, rows_max, gate_of_row, y_rows, s);
+  return f32out ? run_simt<__nv_bfloat16, 1, float>(h, W_dn, offsets, E, F, d, F, rows_max, gate_of_row, y_rows, s)
+                : run_simt<__nv_bfloat16, 1, __nv_bfloat16>(h, W_dn, offsets, E, F, d, F, rows_max, gate_of_row,
+                                                            y_rows, s);
 }
 
 }  // namespace moe

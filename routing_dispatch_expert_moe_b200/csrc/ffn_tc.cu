@@ -171,12 +171,14 @@ __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.
 // Ties the loaded registers to the preceding wait so no use is scheduled above it.
 __device__ __forceinline__ void tmem_regs_ready(uint32_t (&r)[32]) { asm volatile("" : MOE_RW32(r)); }
 
-template <int MODE>
+// OutT: element type of the output rows (MODE 0 always writes bf16 H; MODE 1 writes
+// bf16 or fp32 gated rows).
+template <int MODE, typename OutT>
 __global__ void __launch_bounds__(kThreadsTC, 1)
 grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                        const int32_t* __restrict__ offsets, int E, int K, int N_out, int F,
                        long long rows_max, const float* __restrict__ gate_of_row,
-                       __nv_bfloat16* __restrict__ out, int* err) {
+                       OutT* __restrict__ out, int* err) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
@@ -306,9 +308,9 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
       const bool valid = r_in < tc.rows;
       const long long row = (long long)tc.row0 + r_in;
-      if (MODE == 0) {
+      if constexpr (MODE == 0) {
         const int f0 = tc.n_tile * 128;
-        __nv_bfloat16* orow = out + row * F;
+        OutT* orow = out + row * F;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t g[32], u[32];
@@ -324,8 +326,8 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
             for (int i = 0; i < 16; ++i) {
               const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
               const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
-              const float h0 = g0 / (1.f + __expf(-g0)) * u0;
-              const float h1 = g1 / (1.f + __expf(-g1)) * u1;
+              const float h0 = g0 / (1.f + expf(-g0)) * u0;
+              const float h1 = g1 / (1.f + expf(-g1)) * u1;
               pk[i] = pack_bf16x2(h0, h1);
             }
 #pragma unroll
@@ -338,7 +340,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
       } else {
         const int n0 = tc.n_tile * BN;
         const float gs = (valid && gate_of_row) ? __ldg(gate_of_row + row) : 1.f;
-        __nv_bfloat16* orow = out + row * N_out;
+        OutT* orow = out + row * N_out;
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
           uint32_t v32[32];
@@ -347,15 +349,24 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
           tmem_regs_ready(v32);
           if (valid) {
             const int col = n0 + c * 32;
-            uint32_t pk[16];
+            if constexpr (sizeof(OutT) == 2) {
+              uint32_t pk[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-              pk[i] = pack_bf16x2(__uint_as_float(v32[2 * i]) * gs, __uint_as_float(v32[2 * i + 1]) * gs);
+              for (int i = 0; i < 16; ++i)
+                pk[i] = pack_bf16x2(__uint_as_float(v32[2 * i]) * gs, __uint_as_float(v32[2 * i + 1]) * gs);
 #pragma unroll
-            for (int v = 0; v < 4; ++v)
-              if (col + 8 * v + 8 <= N_out)
-                *reinterpret_cast<uint4*>(orow + col + 8 * v) =
-                    make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+              for (int v = 0; v < 4; ++v)
+                if (col + 8 * v + 8 <= N_out)
+                  *reinterpret_cast<uint4*>(orow + col + 8 * v) =
+                      make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+            } else {
+#pragma unroll
+              for (int v = 0; v < 8; ++v)
+                if (col + 4 * v + 4 <= N_out)
+                  *reinterpret_cast<float4*>(orow + col + 4 * v) =
+                      make_float4(__uint_as_float(v32[4 * v]) * gs, __uint_as_float(v32[4 * v + 1]) * gs,
+                                  __uint_as_float(v32[4 * v + 2]) * gs, __uint_as_float(v32[4 * v + 3]) * gs);
+            }
           }
         }
       }
@@ -403,7 +414,7 @@ bool make_map(CUtensorMap* m, const void* ptr, unsigned long long rows, unsigned
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int MODE>
+template <int MODE, typename OutT>
 moe_status launch_tc(const CUtensorMap& ma, const CUtensorMap& mb, const int32_t* offsets, int E, int K, int N_out,
                      int F, long long rows_max, const float* gate_of_row, void* out, cudaStream_t s) {
   static int configured[64] = {0};
@@ -411,7 +422,7 @@ moe_status launch_tc(const CUtensorMap& ma, const CUtensorMap& mb, const int32_t
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) dev = 0;
   if (!configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_tc_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_tc_kernel<MODE, OutT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemBytes);
     if (e != cudaSuccess) return cuda_status(e);
     configured[dev] = 1;
@@ -421,8 +432,8 @@ moe_status launch_tc(const CUtensorMap& ma, const CUtensorMap& mb, const int32_t
   int grid = num_sms();
   if (max_tiles < grid) grid = (int)max_tiles;
   if (grid < 1) grid = 1;
-  grouped_gemm_tc_kernel<MODE><<<grid, kThreadsTC, kSmemBytes, s>>>(
-      ma, mb, offsets, E, K, N_out, F, rows_max, gate_of_row, static_cast<__nv_bfloat16*>(out), err_ptr());
+  grouped_gemm_tc_kernel<MODE, OutT><<<grid, kThreadsTC, kSmemBytes, s>>>(
+      ma, mb, offsets, E, K, N_out, F, rows_max, gate_of_row, static_cast<OutT*>(out), err_ptr());
   return check_launch();
 }
 
@@ -436,17 +447,18 @@ moe_status launch_gate_up_tc(const void* x_rows, const int32_t* offsets, int E, 
   CUtensorMap ma, mb;
   if (!make_map(&ma, x_rows, (unsigned long long)rows_max, d, BM)) return MOE_ERR_UNSUPPORTED;
   if (!make_map(&mb, W_gu, (unsigned long long)E * 2 * F, d, 128)) return MOE_ERR_UNSUPPORTED;
-  return launch_tc<0>(ma, mb, offsets, E, d, F, F, rows_max, nullptr, h, s);
+  return launch_tc<0, __nv_bfloat16>(ma, mb, offsets, E, d, F, F, rows_max, nullptr, h, s);
 }
 
 moe_status launch_down_tc(const void* h, const int32_t* offsets, int E, int d, int F, long long rows_max,
-                          const void* W_dn, const float* gate_of_row, void* y_rows, cudaStream_t s) {
+                          const void* W_dn, const float* gate_of_row, int y_dtype, void* y_rows, cudaStream_t s) {
   if (rows_max == 0) return MOE_OK;
   if (F < BK || d < 8) return MOE_ERR_UNSUPPORTED;
   CUtensorMap ma, mb;
   if (!make_map(&ma, h, (unsigned long long)rows_max, F, BM)) return MOE_ERR_UNSUPPORTED;
   if (!make_map(&mb, W_dn, (unsigned long long)E * d, F, BN)) return MOE_ERR_UNSUPPORTED;
-  return launch_tc<1>(ma, mb, offsets, E, F, d, F, rows_max, gate_of_row, y_rows, s);
+  if (y_dtype == MOE_F32) return launch_tc<1, float>(ma, mb, offsets, E, F, d, F, rows_max, gate_of_row, y_rows, s);
+  return launch_tc<1, __nv_bfloat16>(ma, mb, offsets, E, F, d, F, rows_max, gate_of_row, y_rows, s);
 }
 
 }  // namespace moe

@@ -55,37 +55,63 @@ permute_kernel(const uint4* __restrict__ x, int T, int nvec, int k, const int32_
   }
 }
 
+// Eight consecutive elements of a row, in the row's storage type.
 template <typename T>
-struct Vec;
+struct Row8;
 template <>
-struct Vec<__nv_bfloat16> {
-  static constexpr int N = 8;
-  __device__ static void unpack(const uint4& v, float* f) { unpack8(v, f); }
-  __device__ static uint4 pack(const float* f) { return pack8(f); }
+struct Row8<__nv_bfloat16> {
+  uint4 a;
+  __device__ __forceinline__ void load(const void* base, long long e) {
+    a = ld_stream(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(base) + e));
+  }
+  __device__ __forceinline__ void add(float* acc, float g, bool scale) const {
+    float f[8];
+    unpack8(a, f);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = scale ? fmaf(g, f[i], acc[i]) : acc[i] + f[i];
+  }
 };
 template <>
-struct Vec<float> {
-  static constexpr int N = 4;
-  __device__ static void unpack(const uint4& v, float* f) {
-    f[0] = __uint_as_float(v.x); f[1] = __uint_as_float(v.y);
-    f[2] = __uint_as_float(v.z); f[3] = __uint_as_float(v.w);
+struct Row8<float> {
+  uint4 a, b;
+  __device__ __forceinline__ void load(const void* base, long long e) {
+    const uint4* p = reinterpret_cast<const uint4*>(static_cast<const float*>(base) + e);
+    a = ld_stream(p);
+    b = ld_stream(p + 1);
   }
-  __device__ static uint4 pack(const float* f) {
-    return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
-                      __float_as_uint(f[3]));
+  __device__ __forceinline__ void add(float* acc, float g, bool scale) const {
+    const float f[8] = {__uint_as_float(a.x), __uint_as_float(a.y), __uint_as_float(a.z), __uint_as_float(a.w),
+                        __uint_as_float(b.x), __uint_as_float(b.y), __uint_as_float(b.z), __uint_as_float(b.w)};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = scale ? fmaf(g, f[i], acc[i]) : acc[i] + f[i];
   }
 };
 
-// KMAX: compile-time bound on k (all k rows of a token are held in registers).
-template <typename DT, int KMAX>
+template <typename T>
+__device__ __forceinline__ void store8(void* base, long long e, const float* f);
+template <>
+__device__ __forceinline__ void store8<__nv_bfloat16>(void* base, long long e, const float* f) {
+  *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(base) + e) = pack8(f);
+}
+template <>
+__device__ __forceinline__ void store8<float>(void* base, long long e, const float* f) {
+  float4* p = reinterpret_cast<float4*>(static_cast<float*>(base) + e);
+  p[0] = make_float4(f[0], f[1], f[2], f[3]);
+  p[1] = make_float4(f[4], f[5], f[6], f[7]);
+}
+
+// KMAX: compile-time bound on k (multiple of 8); a token's rows are loaded 8 slots at a
+// time (8 independent loads in flight per lane) and added in slot order.
+template <typename InT, typename OutT, int KMAX>
 __global__ void __launch_bounds__(256)
-combine_kernel(const uint4* __restrict__ y_rows, const int32_t* __restrict__ row_of,
-               const float* __restrict__ topk_gate, const uint4* __restrict__ shared_y, int T,
-               int nvec, int k, long long rows_max, uint4* __restrict__ y, int* err) {
-  constexpr int N = Vec<DT>::N;
+combine_kernel(const void* __restrict__ y_rows, const int32_t* __restrict__ row_of,
+               const float* __restrict__ topk_gate, const void* __restrict__ shared_y, int T, int d, int k,
+               long long rows_max, void* __restrict__ y, int* err) {
   const unsigned lane = threadIdx.x & 31;
   const int warps = blockDim.x >> 5;
   const long long nw = (long long)gridDim.x * warps;
+  const bool scale = topk_gate != nullptr;
+  const int n8 = d >> 3;
   for (long long t = (long long)blockIdx.x * warps + (threadIdx.x >> 5); t < T; t += nw) {
     int my_row = -1;
     float my_gate = 1.f;
@@ -93,46 +119,35 @@ combine_kernel(const uint4* __restrict__ y_rows, const int32_t* __restrict__ row
       my_row = __ldg(row_of + t * k + lane);
       if (my_row >= rows_max) { record_error(err, MOE_DEVERR_ROW); my_row = -1; }
       if (my_row < -1) my_row = -1;
-      if (topk_gate) my_gate = __ldg(topk_gate + t * k + lane);
+      if (scale) my_gate = __ldg(topk_gate + t * k + lane);
     }
     int rows[KMAX];
     float gates[KMAX];
 #pragma unroll
     for (int j = 0; j < KMAX; ++j) {
-      rows[j] = __shfl_sync(0xffffffffu, my_row, j);
-      gates[j] = __shfl_sync(0xffffffffu, my_gate, j);
+      rows[j] = __shfl_sync(0xffffffffu, my_row, j & 31);
+      gates[j] = __shfl_sync(0xffffffffu, my_gate, j & 31);
     }
-    for (int v = lane; v < nvec; v += 32) {
-      uint4 buf[KMAX];
+    for (int v = lane; v < n8; v += 32) {
+      float acc[8];
 #pragma unroll
-      for (int j = 0; j < KMAX; ++j)
-        if (j < k && rows[j] >= 0) buf[j] = ld_stream(y_rows + (long long)rows[j] * nvec + v);
-      uint4 sv;
-      if (shared_y) sv = ld_stream(shared_y + t * nvec + v);
-      float acc[N];
+      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
 #pragma unroll
-      for (int i = 0; i < N; ++i) acc[i] = 0.f;
+      for (int j0 = 0; j0 < KMAX; j0 += 8) {
+        Row8<InT> buf[8];
 #pragma unroll
-      for (int j = 0; j < KMAX; ++j) {
-        if (j < k && rows[j] >= 0) {
-          float f[N];
-          Vec<DT>::unpack(buf[j], f);
-          if (topk_gate) {
+        for (int jj = 0; jj < 8; ++jj)
+          if (rows[j0 + jj] >= 0) buf[jj].load(y_rows, (long long)rows[j0 + jj] * d + v * 8);
 #pragma unroll
-            for (int i = 0; i < N; ++i) acc[i] = fmaf(gates[j], f[i], acc[i]);
-          } else {
-#pragma unroll
-            for (int i = 0; i < N; ++i) acc[i] += f[i];
-          }
-        }
+        for (int jj = 0; jj < 8; ++jj)
+          if (rows[j0 + jj] >= 0) buf[jj].add(acc, gates[j0 + jj], scale);
       }
       if (shared_y) {
-        float f[N];
-        Vec<DT>::unpack(sv, f);
-#pragma unroll
-        for (int i = 0; i < N; ++i) acc[i] += f[i];
+        Row8<InT> sv;
+        sv.load(shared_y, t * d + v * 8);
+        sv.add(acc, 1.f, false);
       }
-      y[t * nvec + v] = Vec<DT>::pack(acc);
+      store8<OutT>(y, t * d + v * 8, acc);
     }
   }
 }
@@ -145,26 +160,20 @@ unsigned grid_for_warps(long long warps_needed) {
   return (unsigned)blocks;
 }
 
-template <typename DT, int KMAX>
-moe_status run_combine(const void* y_rows, const int32_t* row_of, const float* topk_gate,
-                       const void* shared_y, int T, int nvec, int k, long long rows_max, void* y,
-                       cudaStream_t s) {
-  combine_kernel<DT, KMAX><<<grid_for_warps(T), 256, 0, s>>>(
-      static_cast<const uint4*>(y_rows), row_of, topk_gate, static_cast<const uint4*>(shared_y), T, nvec, k,
-      rows_max, static_cast<uint4*>(y), err_ptr());
+template <typename InT, typename OutT, int KMAX>
+moe_status run_combine(const void* y_rows, const int32_t* row_of, const float* topk_gate, const void* shared_y,
+                       int T, int d, int k, long long rows_max, void* y, cudaStream_t s) {
+  combine_kernel<InT, OutT, KMAX><<<grid_for_warps(T), 256, 0, s>>>(y_rows, row_of, topk_gate, shared_y, T, d, k,
+                                                                   rows_max, y, err_ptr());
   return check_launch();
 }
 
-template <typename DT>
-moe_status combine_k(const void* y_rows, const int32_t* row_of, const float* topk_gate,
-                     const void* shared_y, int T, int nvec, int k, long long rows_max, void* y,
-                     cudaStream_t s) {
-  if (k <= 1) return run_combine<DT, 1>(y_rows, row_of, topk_gate, shared_y, T, nvec, k, rows_max, y, s);
-  if (k <= 2) return run_combine<DT, 2>(y_rows, row_of, topk_gate, shared_y, T, nvec, k, rows_max, y, s);
-  if (k <= 4) return run_combine<DT, 4>(y_rows, row_of, topk_gate, shared_y, T, nvec, k, rows_max, y, s);
-  if (k <= 8) return run_combine<DT, 8>(y_rows, row_of, topk_gate, shared_y, T, nvec, k, rows_max, y, s);
-  if (k <= 16) return run_combine<DT, 16>(y_rows, row_of, topk_gate, shared_y, T, nvec, k, rows_max, y, s);
-  return run_combine<DT, 32>(y_rows, row_of, topk_gate, shared_y, T, nvec, k, rows_max, y, s);
+template <typename InT, typename OutT>
+moe_status combine_k(const void* y_rows, const int32_t* row_of, const float* topk_gate, const void* shared_y,
+                     int T, int d, int k, long long rows_max, void* y, cudaStream_t s) {
+  if (k <= 8) return run_combine<InT, OutT, 8>(y_rows, row_of, topk_gate, shared_y, T, d, k, rows_max, y, s);
+  if (k <= 16) return run_combine<InT, OutT, 16>(y_rows, row_of, topk_gate, shared_y, T, d, k, rows_max, y, s);
+  return run_combine<InT, OutT, 32>(y_rows, row_of, topk_gate, shared_y, T, d, k, rows_max, y, s);
 }
 
 }  // namespace
@@ -179,14 +188,15 @@ moe_status launch_permute(const void* x, int dtype, int T, int d, int k, const i
   return check_launch();
 }
 
-moe_status launch_combine(const void* y_rows, const int32_t* row_of, const float* topk_gate,
-                          const void* shared_y, int dtype, int T, int d, int k, long long rows_max,
+moe_status launch_combine(const void* y_rows, int rows_dtype, const int32_t* row_of, const float* topk_gate,
+                          const void* shared_y, int T, int d, int k, long long rows_max, int y_dtype,
                           void* y, cudaStream_t s) {
   if (T == 0) return MOE_OK;
-  const int esz = dtype == MOE_F32 ? 4 : 2;
-  const int nvec = d * esz / 16;
-  if (dtype == MOE_F32) return combine_k<float>(y_rows, row_of, topk_gate, shared_y, T, nvec, k, rows_max, y, s);
-  return combine_k<__nv_bfloat16>(y_rows, row_of, topk_gate, shared_y, T, nvec, k, rows_max, y, s);
+  const bool in32 = rows_dtype == MOE_F32, out32 = y_dtype == MOE_F32;
+  if (in32 && out32) return combine_k<float, float>(y_rows, row_of, topk_gate, shared_y, T, d, k, rows_max, y, s);
+  if (in32) return combine_k<float, __nv_bfloat16>(y_rows, row_of, topk_gate, shared_y, T, d, k, rows_max, y, s);
+  if (out32) return combine_k<__nv_bfloat16, float>(y_rows, row_of, topk_gate, shared_y, T, d, k, rows_max, y, s);
+  return combine_k<__nv_bfloat16, __nv_bfloat16>(y_rows, row_of, topk_gate, shared_y, T, d, k, rows_max, y, s);
 }
 
 }  // namespace moe

@@ -32,7 +32,10 @@ class MoEWeights:
 
 class MoELayer:
     def __init__(self, weights: MoEWeights, k: int, T_max: int, score: str = "softmax",
-                 renormalize: bool = True, scale: float = 1.0, capacity: int = -1):
+                 renormalize: bool = True, scale: float = 1.0, capacity: int = -1,
+                 rows_dtype: torch.dtype = torch.float32, out_dtype: torch.dtype = torch.float32):
+        """rows_dtype: gated expert rows (and the shared expert's output); out_dtype: y.
+        fp32 (the default) leaves H as the only bf16 rounding inside the layer."""
         w = weights
         self.w = w
         self.d, self.E = w.Wg.shape
@@ -40,6 +43,7 @@ class MoELayer:
         self.k, self.T_max = k, T_max
         self.score, self.renormalize, self.scale, self.capacity = score, renormalize, scale, capacity
         self.dtype = w.W_gu.dtype
+        self.rows_dtype, self.out_dtype = rows_dtype, out_dtype
         dev = w.Wg.device
         self.device = dev
         E, d, F = self.E, self.d, self.F
@@ -57,8 +61,8 @@ class MoELayer:
         self.gate_of_row = torch.empty(R, dtype=f32, device=dev)
         self.x_perm = torch.empty((R, d), dtype=self.dtype, device=dev)
         self.h = torch.empty((R, F), dtype=self.dtype, device=dev)
-        self.y_perm = torch.empty((R, d), dtype=self.dtype, device=dev)
-        self.y = torch.empty((T_max, d), dtype=self.dtype, device=dev)
+        self.y_perm = torch.empty((R, d), dtype=rows_dtype, device=dev)
+        self.y = torch.empty((T_max, d), dtype=out_dtype, device=dev)
         self.load = torch.empty(E, dtype=f32, device=dev)
         self.stats5 = torch.empty(5, dtype=f32, device=dev)
         self.ws = torch.empty(max(M.moe_workspace_bytes(T_max, d, E, k), 16), dtype=torch.uint8, device=dev)
@@ -67,7 +71,7 @@ class MoELayer:
             self.F_s = w.W_dn_s.shape[2]
             self.shared_offsets = torch.tensor([0, T_max], dtype=i32, device=dev)
             self.h_s = torch.empty((T_max, self.F_s), dtype=self.dtype, device=dev)
-            self.y_s = torch.empty((T_max, d), dtype=self.dtype, device=dev)
+            self.y_s = torch.empty((T_max, d), dtype=rows_dtype, device=dev)
 
     # individual steps (so that a caller can time them one by one)
     def route(self, x, stream=None):
@@ -86,18 +90,19 @@ class MoELayer:
         M.moe_expert_gate_up(self.x_perm, self.offsets, self.w.W_gu, self.rows_max, self.h, stream)
 
     def down(self, stream=None):
-        M.moe_expert_down(self.h, self.offsets, self.w.W_dn, self.rows_max, self.gate_of_row, self.y_perm, stream)
+        M.moe_expert_down(self.h, self.offsets, self.w.W_dn, self.rows_max, self.gate_of_row, self.y_perm,
+                          stream=stream)
 
     def shared(self, x, stream=None):
         T = x.shape[0]
         if T != self.T_max:
             self.shared_offsets[1].fill_(T)
         M.moe_expert_gate_up(x, self.shared_offsets, self.w.W_gu_s, T, self.h_s[:T], stream)
-        M.moe_expert_down(self.h_s[:T], self.shared_offsets, self.w.W_dn_s, T, None, self.y_s[:T], stream)
+        M.moe_expert_down(self.h_s[:T], self.shared_offsets, self.w.W_dn_s, T, None, self.y_s[:T], stream=stream)
 
     def combine(self, T, stream=None):
         M.moe_combine(self.y_perm, self.row_of[:T], T, self.rows_max, None,
-                      self.y_s[:T] if self.has_shared else None, self.y[:T], stream)
+                      self.y_s[:T] if self.has_shared else None, self.y[:T], stream=stream)
 
     def stats(self, T, stream=None):
         M.moe_router_stats(self.logits[:T], self.counts, self.kept, self.k, self.score, self.load, self.stats5,
@@ -107,7 +112,7 @@ class MoELayer:
         T = x.shape[0]
         if T > self.T_max:
             raise ValueError(f"T={T} exceeds T_max={self.T_max}")
-        if x.dtype != self.dtype and not (self.dtype == torch.float32 and x.dtype == torch.float32):
+        if x.dtype != self.dtype:
             raise ValueError(f"x must be {self.dtype}")
         self.route(x, stream)
         self.histogram_scan(T, stream)

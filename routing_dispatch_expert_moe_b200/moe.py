@@ -43,11 +43,11 @@ _SIGNATURES = {
     "moe_expert_gate_up": (_i32, [_c_void_p, _i32, _c_void_p, _i32, _i32, _i32, _i64, _c_void_p, _c_void_p,
                                   _c_void_p]),
     "moe_expert_down": (_i32, [_c_void_p, _i32, _c_void_p, _i32, _i32, _i32, _i64, _c_void_p, _c_void_p,
-                               _c_void_p, _c_void_p]),
+                               _i32, _c_void_p, _c_void_p]),
     "moe_grouped_ffn": (_i32, [_c_void_p, _i32, _c_void_p, _i32, _i32, _i32, _i64, _c_void_p, _c_void_p,
-                               _c_void_p, _c_void_p, _c_void_p, _c_void_p]),
-    "moe_combine": (_i32, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _i32, _i32, _i32, _i32, _i64, _c_void_p,
-                           _c_void_p]),
+                               _c_void_p, _c_void_p, _i32, _c_void_p, _c_void_p]),
+    "moe_combine": (_i32, [_c_void_p, _i32, _c_void_p, _c_void_p, _c_void_p, _i32, _i32, _i32, _i64, _i32,
+                           _c_void_p, _c_void_p]),
     "moe_router_stats_workspace_bytes": (_size, [_i32, _i32]),
     "moe_router_stats": (_i32, [_c_void_p, _c_void_p, _c_void_p, _i32, _i32, _i32, _i32, _c_void_p, _c_void_p,
                                 _c_void_p, _size, _c_void_p]),
@@ -218,22 +218,24 @@ def moe_expert_gate_up(x_rows, offsets, W_gu, rows_max: int, h=None, stream=None
     return h
 
 
-def moe_expert_down(h, offsets, W_dn, rows_max: int, gate_of_row=None, y_rows=None, stream=None):
+def moe_expert_down(h, offsets, W_dn, rows_max: int, gate_of_row=None, y_rows=None, y_dtype=None, stream=None):
+    """Gated rows y_rows = gate_of_row * (H W_dn^T) in y_dtype (default: y_rows' dtype, else fp32)."""
     E, d, F = W_dn.shape
     _need(h, "h")
     _need(offsets, "offsets", torch.int32, (E + 1,))
     _need(W_dn, "W_dn", h.dtype)
     if gate_of_row is not None:
         _need(gate_of_row, "gate_of_row", torch.float32)
-    y_rows = torch.empty((max(rows_max, 1), d), dtype=h.dtype, device=h.device) if y_rows is None else \
-        _need(y_rows, "y_rows", h.dtype)
+    y_dtype = y_rows.dtype if y_rows is not None else (y_dtype or torch.float32)
+    y_rows = torch.empty((max(rows_max, 1), d), dtype=y_dtype, device=h.device) if y_rows is None else \
+        _need(y_rows, "y_rows")
     _check("moe_expert_down", lib().moe_expert_down(_p(h), _dt(h), _p(offsets), E, d, F, rows_max, _p(W_dn),
-                                                    _p(gate_of_row), _p(y_rows), _stream(stream)))
+                                                    _p(gate_of_row), _dt(y_rows), _p(y_rows), _stream(stream)))
     return y_rows
 
 
 def moe_grouped_ffn(x_rows, offsets, W_gu, W_dn, rows_max: int, gate_of_row=None, h=None, y_rows=None,
-                    stream=None):
+                    y_dtype=None, stream=None):
     E, F2, d = W_gu.shape
     F = F2 // 2
     _need(x_rows, "x_rows")
@@ -242,15 +244,18 @@ def moe_grouped_ffn(x_rows, offsets, W_gu, W_dn, rows_max: int, gate_of_row=None
     _need(W_dn, "W_dn", x_rows.dtype, (E, d, F))
     dev = x_rows.device
     h = torch.empty((max(rows_max, 1), F), dtype=x_rows.dtype, device=dev) if h is None else _need(h, "h")
-    y_rows = torch.empty((max(rows_max, 1), d), dtype=x_rows.dtype, device=dev) if y_rows is None else \
+    y_dtype = y_rows.dtype if y_rows is not None else (y_dtype or torch.float32)
+    y_rows = torch.empty((max(rows_max, 1), d), dtype=y_dtype, device=dev) if y_rows is None else \
         _need(y_rows, "y_rows")
     _check("moe_grouped_ffn", lib().moe_grouped_ffn(_p(x_rows), _dt(x_rows), _p(offsets), E, d, F, rows_max,
-                                                    _p(W_gu), _p(W_dn), _p(gate_of_row), _p(h), _p(y_rows),
-                                                    _stream(stream)))
+                                                    _p(W_gu), _p(W_dn), _p(gate_of_row), _p(h), _dt(y_rows),
+                                                    _p(y_rows), _stream(stream)))
     return y_rows
 
 
-def moe_combine(y_rows, row_of, T: int, rows_max: int, topk_gate=None, shared_y=None, y=None, stream=None):
+def moe_combine(y_rows, row_of, T: int, rows_max: int, topk_gate=None, shared_y=None, y=None, y_dtype=None,
+                stream=None):
+    """y[t] = sum_j (g_j) y_rows[row_of[t, j]] (+ shared_y[t]) in y_dtype (default fp32)."""
     d = y_rows.shape[1]
     k = row_of.shape[1]
     _need(y_rows, "y_rows")
@@ -259,9 +264,10 @@ def moe_combine(y_rows, row_of, T: int, rows_max: int, topk_gate=None, shared_y=
         _need(shared_y, "shared_y", y_rows.dtype, (T, d))
     if topk_gate is not None:
         _need(topk_gate, "topk_gate", torch.float32, (T, k))
-    y = torch.empty((T, d), dtype=y_rows.dtype, device=y_rows.device) if y is None else _need(y, "y", y_rows.dtype)
-    _check("moe_combine", lib().moe_combine(_p(y_rows), _p(row_of), _p(topk_gate), _p(shared_y), _dt(y_rows), T, d,
-                                            k, rows_max, _p(y), _stream(stream)))
+    y_dtype = y.dtype if y is not None else (y_dtype or torch.float32)
+    y = torch.empty((T, d), dtype=y_dtype, device=y_rows.device) if y is None else _need(y, "y")
+    _check("moe_combine", lib().moe_combine(_p(y_rows), _dt(y_rows), _p(row_of), _p(topk_gate), _p(shared_y), T, d,
+                                            k, rows_max, _dt(y), _p(y), _stream(stream)))
     return y
 
 

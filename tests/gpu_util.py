@@ -5,8 +5,11 @@ Bars (from the layer's acceptance criteria):
   routing indices, counts, kept, offsets, row maps, permuted rows: bit-exact;
   logits: bit-exact (the generator's grids make fp32 sums exact);
   gates: |err| <= 1e-6 * |gate|;
-  expert outputs y (and each gated expert row): max|err| <= 2e-2 * rms(y) and
+  layer output y (fp32 rows and output, the default): max|err| <= 2e-2 * rms(y) and
   mean|err| <= 2e-3 * rms(y).
+Derived bars (where a result passes through extra bf16 roundings; see each helper):
+  gated expert rows: componentwise bound from H's bf16 rounding;
+  bf16 rows + bf16 output: componentwise bound from every rounding point.
 """
 from __future__ import annotations
 
@@ -68,17 +71,17 @@ def expert_getters(host):
     return gu, dn
 
 
-def build_layer(cfg, dev, capacity):
+def build_layer(cfg, dev, capacity, rows_dtype=torch.float32, out_dtype=torch.float32):
     from routing_dispatch_expert_moe_b200.layer import MoELayer, MoEWeights
     w = MoEWeights(Wg=dev["Wg"], W_gu=dev["W_gu"], W_dn=dev["W_dn"], logit_offset=dev["off"],
                    select_bias=dev["bias"], W_gu_s=dev["W_gu_s"], W_dn_s=dev["W_dn_s"])
-    return MoELayer(w, cfg.k, cfg.T, cfg.score, cfg.renormalize, cfg.scale, capacity)
+    return MoELayer(w, cfg.k, cfg.T, cfg.score, cfg.renormalize, cfg.scale, capacity, rows_dtype, out_dtype)
 
 
-def gpu_forward(cfg, dev, capacity):
+def gpu_forward(cfg, dev, capacity, rows_dtype=torch.float32, out_dtype=torch.float32):
     """Runs the layer through the C ABI; returns the layer object and host copies of every output."""
     from routing_dispatch_expert_moe_b200 import moe as M
-    layer = build_layer(cfg, dev, capacity)
+    layer = build_layer(cfg, dev, capacity, rows_dtype, out_dtype)
     y = layer.forward(dev["x"])
     torch.cuda.synchronize()
     code = M.moe_get_device_error()
@@ -121,6 +124,49 @@ def assert_routing_equal(g, o, exact_logits=True):
     assert (ge <= GATE_RTOL * np.abs(o["gate_of_row"][:n]) + 1e-30).all()
 
 
+def bf16_step(v):
+    """Spacing of bf16 values at |v| (8 significant bits): 2^(floor(log2|v|) - 7)."""
+    a = np.abs(np.asarray(v, np.float64))
+    e = np.floor(np.log2(np.maximum(a, 2.0 ** -126)))
+    return np.ldexp(1.0, (e - 7).astype(np.int64))
+
+
+def row_bounds(x, tokens, experts, gates, gu, dn, bf16=True):
+    """Componentwise bound on how far a correct gated row may sit from the oracle's.
+
+    Both sides round H to bf16 from values that differ only by accumulation order, so any
+    H element may land one bf16 step (<= 2^-8 |h|) away; that moves output n by at most
+    2^-8 * gate * sum_f |h_f| |W_dn[n, f]|.  Returns that bound per row (float64).
+    """
+    x = np.asarray(x)
+    out = np.zeros((len(tokens), dn(int(experts[0])).shape[0] if len(tokens) else 0), np.float64)
+    if not bf16:                      # fp32 activations: H is not rounded on either side
+        return out
+    for e in np.unique(experts):
+        i = np.nonzero(experts == e)[0]
+        h = O.expert_hidden(np.asarray(x[tokens[i]], np.float64), gu(int(e)), bf16)
+        out[i] = 2.0 ** -8 * np.abs(np.asarray(gates, np.float64)[i])[:, None] * (np.abs(h) @ np.abs(dn(int(e))).T)
+    return out
+
+
+def assert_rows_close(gy, oy, hbound, what="y_perm", rows_bf16=False):
+    """Gated expert rows: each element within the H-rounding bound plus fp32 accumulation
+    slack (1e-5 relative, 1e-6 of the rms), and one bf16 step of its magnitude when the
+    rows themselves are stored in bf16; mean error within 2e-3 * rms."""
+    gy = np.asarray(gy, np.float64)
+    oy = np.asarray(oy, np.float64)
+    rms = float(np.sqrt(np.mean(oy ** 2)))
+    err = np.abs(gy - oy)
+    bound = hbound + 1e-5 * np.abs(oy) + 1e-6 * rms
+    if rows_bf16:
+        bound = bound + bf16_step(np.maximum(np.abs(gy), np.abs(oy)))
+    bad = err > bound
+    assert not bad.any(), (f"{what}: {int(bad.sum())} elements beyond the bound; worst err "
+                           f"{float(err[bad].max()):.4g} at |ref| {float(np.abs(oy[bad]).max()):.4g}, rms {rms:.4g}")
+    assert float(err.mean()) <= Y_MEAN_REL * rms, f"{what}: mean|err| {float(err.mean()):.4g} > {Y_MEAN_REL} * rms"
+    return float(err.max()) / rms, float(err.mean()) / rms
+
+
 def y_errors(gy, oy):
     rms = float(np.sqrt(np.mean(oy ** 2)))
     err = np.abs(gy - oy)
@@ -135,6 +181,29 @@ def assert_y_close(gy, oy, what="y"):
     return mx / rms, mean / rms
 
 
+def assert_y_close_bf16(gy, oy, slot_rows, slot_hbound, shared_y=None):
+    """bf16 rows and bf16 output: componentwise bound derived from the rounding points.
+
+    y[t] = bf16(sum_j row_j + shared); each row_j may differ by its own bound (one bf16
+    step of the row element plus the H-rounding bound), the shared row by one step, and
+    the final rounding by one bf16 step of y.  Mean error obeys the 2e-3 * rms bar.
+    slot_rows / slot_hbound: [T, k, d] oracle rows and their H bounds (zeros where dropped).
+    """
+    gy = np.asarray(gy, np.float64)
+    oy = np.asarray(oy, np.float64)
+    b = bf16_step(np.maximum(np.abs(gy), np.abs(oy)))
+    rows = np.asarray(slot_rows, np.float64)
+    b = b + (np.where(rows != 0, bf16_step(rows), 0.0) + slot_hbound).sum(axis=1)
+    if shared_y is not None:
+        b = b + bf16_step(shared_y)
+    rms = float(np.sqrt(np.mean(oy ** 2)))
+    err = np.abs(gy - oy)
+    bad = err > b + 1e-6 * rms
+    assert not bad.any(), f"y (bf16): {int(bad.sum())} elements beyond the bound, worst {float(err.max()):.4g}"
+    assert float(err.mean()) <= Y_MEAN_REL * rms
+    return float(err.max()) / rms, float(err.mean()) / rms
+
+
 def assert_stats_close(g, o_stats, dropped_exact=True):
     np.testing.assert_allclose(g["load"], o_stats["load"], rtol=1e-6, atol=0)
     s = g["stats5"].astype(np.float64)
@@ -145,7 +214,7 @@ def assert_stats_close(g, o_stats, dropped_exact=True):
     assert abs(s[4] - o_stats["cv"]) <= 1e-5 * o_stats["cv"] + 1e-7
 
 
-def stratified_tokens(o, cap, n_random=700, seed=0, limit=1200):
+def stratified_tokens(o, cap, n_random=1100, seed=0):
     """Hottest / coldest non-empty expert's tokens, capacity-boundary and fully dropped
     tokens, plus random ones (each token's output depends only on its own row)."""
     idx, row_of, rank = o["topk_idx"], o["row_of"], o["rank"]
@@ -169,4 +238,4 @@ def stratified_tokens(o, cap, n_random=700, seed=0, limit=1200):
     picks += list(rng.choice(T, size=min(n_random, T), replace=False))
     picks += [0, T - 1]
     out = np.unique(np.array(picks, np.int64))
-    return out[:limit] if len(out) > limit else out
+    return out

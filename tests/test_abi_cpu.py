@@ -130,7 +130,8 @@ def test_ffn_host_validation(L):
     assert f(ctypes.c_void_p(4100), 0, FAKE, 4, 128, 64, 128, FAKE, FAKE, NUL) == 2   # alignment
     assert f(FAKE, 0, FAKE, 4, 128, 64, 0, FAKE, FAKE, NUL) == 0          # no rows: nothing to do
     g = L.moe_expert_down
-    assert g(FAKE, 0, FAKE, 4, 128, 64, -1, FAKE, NUL, FAKE, NUL) == 1
+    assert g(FAKE, 0, FAKE, 4, 128, 64, -1, FAKE, NUL, 1, FAKE, NUL) == 1
+    assert g(FAKE, 0, FAKE, 4, 128, 64, 128, FAKE, NUL, 7, FAKE, NUL) == 1        # y dtype
 
 
 def test_permute_combine_host_validation(L):
@@ -138,8 +139,9 @@ def test_permute_combine_host_validation(L):
     assert L.moe_permute(NUL, 0, 64, 128, 4, FAKE, 256, FAKE, NUL) == 1
     assert L.moe_permute(FAKE, 0, 64, 128, 40, FAKE, 256, FAKE, NUL) == 2
     assert L.moe_permute(FAKE, 0, 0, 128, 4, FAKE, 0, FAKE, NUL) == 0
-    assert L.moe_combine(FAKE, NUL, NUL, NUL, 0, 64, 128, 4, 256, FAKE, NUL) == 1
-    assert L.moe_combine(FAKE, FAKE, NUL, ctypes.c_void_p(4097), 0, 64, 128, 4, 256, FAKE, NUL) == 2
+    assert L.moe_combine(FAKE, 0, NUL, NUL, NUL, 64, 128, 4, 256, 1, FAKE, NUL) == 1
+    assert L.moe_combine(FAKE, 0, FAKE, NUL, ctypes.c_void_p(4097), 64, 128, 4, 256, 1, FAKE, NUL) == 2
+    assert L.moe_combine(FAKE, 0, FAKE, NUL, NUL, 64, 128, 4, 256, 5, FAKE, NUL) == 1     # y dtype
 
 
 def test_router_stats_host_validation(L):

@@ -48,10 +48,12 @@ def full_check(cfg, seed=0, per_assignment=True, check_stats=True):
     yp_o = O.grouped_ffn(xperm, o["offsets"], gu, dn, o["gate_of_row"], bf16)
     yp_g = layer.y_perm[:n].float().cpu().numpy().astype(np.float64)
     if n:
-        U.assert_y_close(yp_g, yp_o, "y_perm")
+        experts = np.repeat(np.arange(cfg.E), o["kept"])
+        hb = U.row_bounds(host["x"], o["token_of_row"][:n], experts, o["gate_of_row"][:n], gu, dn, bf16)
+        U.assert_rows_close(yp_g, yp_o, hb, "y_perm")
     sh = host["shared"]
     ys = O.shared_expert(host["x"], sh[0], sh[1], bf16) if sh is not None else None
-    y_o = O.combine(yp_o, o["row_of"], ys, bf16)
+    y_o = O.combine(yp_o, o["row_of"], ys)
     if np.any(y_o):
         U.assert_y_close(g["y"], y_o, "y")
     else:
@@ -80,6 +82,31 @@ SMALL = [
 @pytest.mark.parametrize("cfg", SMALL, ids=lambda c: c.name)
 def test_small_full_parity(cfg):
     full_check(cfg)
+
+
+@pytest.mark.parametrize("cfg", [SMALL[0], SMALL[1], SMALL[4]], ids=lambda c: c.name)
+def test_bf16_rows_and_bf16_output(cfg):
+    """The bandwidth-saving variant: gated rows and y stored in bf16 (two more roundings)."""
+    host, dev = U.make_inputs(cfg)
+    cap = O.capacity(cfg.T, cfg.E, cfg.k, cfg.capacity_factor)
+    layer, g = U.gpu_forward(cfg, dev, cap, torch.bfloat16, torch.bfloat16)
+    o = O.layer_routing(U.cfg_dict(cfg), host["x"], host["Wg"], host["off"], host["bias"])
+    U.assert_routing_equal(g, o)
+    gu, dn = U.expert_getters(host)
+    toks = np.arange(cfg.T)
+    sub = O.layer_outputs_for_tokens(toks, host["x"], o, gu, dn, True, shared=host["shared"], round_rows=True,
+                                     round_out=True)
+    kept = o["row_of"] >= 0
+    ii, jj = np.nonzero(kept)
+    hb = U.row_bounds(host["x"], ii, o["topk_idx"][ii, jj], o["topk_gate"][ii, jj], gu, dn)
+    yp_g = layer.y_perm[torch.from_numpy(o["row_of"][kept]).long().cuda()].float().cpu().numpy()
+    U.assert_rows_close(yp_g, sub["slot_rows"][kept], hb, "y_perm (bf16)", rows_bf16=True)
+    slot_hb = np.zeros_like(sub["slot_rows"])
+    slot_hb[ii, jj] = hb
+    ys = None
+    if host["shared"] is not None:
+        ys = O.shared_expert(host["x"], host["shared"][0], host["shared"][1], True, round_out=True)
+    U.assert_y_close_bf16(g["y"], sub["y"], sub["slot_rows"], slot_hb, ys)
 
 
 def test_c1_tiny_both_capacity_readings():
@@ -148,7 +175,7 @@ def test_corrupt_expert_id_is_reported_not_trapped():
 
 
 # ---------------------------------------------------------------- full-size workloads
-def full_size_check(name, per_assignment=True, n_sample_random=700):
+def full_size_check(name, per_assignment=True, n_sample_random=1100):
     cfg = I.CONFIGS[name]
     host, dev = U.make_inputs(cfg)
     cap = O.capacity(cfg.T, cfg.E, cfg.k, cfg.capacity_factor, per_assignment)
@@ -168,7 +195,9 @@ def full_size_check(name, per_assignment=True, n_sample_random=700):
     rows = o["row_of"][toks]
     kept = rows >= 0
     yp_g = layer.y_perm[torch.from_numpy(rows[kept]).long().cuda()].float().cpu().numpy().astype(np.float64)
-    U.assert_y_close(yp_g, sub["slot_rows"][kept], "y_perm (sampled)")
+    ii, jj = np.nonzero(kept)
+    hb = U.row_bounds(host["x"], toks[ii], o["topk_idx"][toks][ii, jj], o["topk_gate"][toks][ii, jj], gu, dn)
+    U.assert_rows_close(yp_g, sub["slot_rows"][kept], hb, "y_perm (sampled)")
     ma, me = U.assert_y_close(g["y"][toks], sub["y"], "y (sampled)")
     del layer, dev
     torch.cuda.empty_cache()

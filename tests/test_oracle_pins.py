@@ -276,7 +276,7 @@ def test_permute_then_combine_is_identity(k):
     xp = O.permute(x, r["row_of"], n)
     # identity expert, gate 1/k on every row (k a power of two: exact)
     yp = xp * (1.0 / k)
-    y = O.combine(yp, r["row_of"], None, bf16=True)
+    y = O.combine(yp, r["row_of"], None, round_out=True)
     assert np.array_equal(y, x.astype(np.float64))
     # and the permuted rows really are the tokens
     assert np.array_equal(xp, x.astype(np.float64)[r["token_of_row"]])
@@ -287,7 +287,7 @@ def test_combine_applies_topk_gate_when_not_fused():
     yp = rng.standard_normal((6, 3))
     row_of = np.array([[0, 3], [1, -1], [5, 2]])
     g = rng.random((3, 2))
-    y = O.combine(yp, row_of, None, bf16=False, topk_gate=g)
+    y = O.combine(yp, row_of, None, round_out=False, topk_gate=g)
     np.testing.assert_allclose(y[1], yp[1] * g[1, 0])
     np.testing.assert_allclose(y[2], yp[5] * g[2, 0] + yp[2] * g[2, 1])
 
@@ -333,11 +333,15 @@ def test_subset_evaluation_matches_full_layer():
     bias = np.linspace(-0.1, 0.1, cfg.E)
     W_gu, W_dn = I.gen_experts(cfg)
     sh = I.gen_shared(cfg)
-    full = O.layer_forward(cfg.__dict__, x, Wg, W_gu, W_dn, select_bias=bias, shared=sh, bf16=True)
-    assert (full["row_of"] < 0).any()              # some drops exercised
-    toks = [0, 5, 17, 63]
-    sub = O.layer_outputs_for_tokens(toks, x, full, W_gu, W_dn, True, shared=sh)
-    assert np.array_equal(sub["y"], full["y"][toks])
+    for rr, ro in ((False, False), (True, True), (True, False)):
+        full = O.layer_forward(cfg.__dict__, x, Wg, W_gu, W_dn, select_bias=bias, shared=sh, bf16=True,
+                               round_rows=rr, round_out=ro)
+        assert (full["row_of"] < 0).any()              # some drops exercised
+        toks = [0, 5, 17, 63]
+        sub = O.layer_outputs_for_tokens(toks, x, full, W_gu, W_dn, True, shared=sh, round_rows=rr, round_out=ro)
+        np.testing.assert_allclose(sub["y"], full["y"][toks], rtol=1e-14, atol=1e-16)
+        if ro:
+            assert np.array_equal(O.bf16_round(sub["y"]), sub["y"])
 
 
 # ---------------------------------------------------------------- router stats
