@@ -169,6 +169,35 @@ MOE_API moe_status moe_histogram_scan(const int32_t* topk_idx, const float* topk
                               void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------------------
+ * moe_histogram_scan_noalloc -- moe_histogram_scan for callers that cannot allocate.
+ * (No counterpart on the pages: this is a deployment convenience, not part of the method.)
+ *
+ * Some callers may not allocate device memory once they run: a serving runtime that
+ * reserves all of its memory at start-up and forbids later cudaMalloc, a plugin hosted
+ * by another framework that hands it no workspace, or a latency-critical loop that
+ * cannot afford cudaMalloc's implicit device synchronisation.  This entry point takes
+ * the same arguments as moe_histogram_scan minus the workspace, and uses instead a
+ * scratch array that the library itself holds in device memory: 4 MiB, a static
+ * __device__ array that every GPU using the library keeps until the process exits.
+ *
+ *   - Limit: moe_histogram_scan_workspace_bytes(T, k, E) must be <= 4 MiB (4194304);
+ *     larger sizes return MOE_ERR_WORKSPACE without launching anything.  The handbook
+ *     workload (T=8192, k=8, E=64) needs about 0.3 MiB, T=32768 k=16 E=896 about 2.5 MiB.
+ *   - The first call on a device looks up the array's device address (once per device,
+ *     with that device current); make that first call before any stream capture.
+ *   - The call allocates nothing: it clears the part of the array that must start at
+ *     zero with one memset node on `stream`, then launches the same kernels.
+ *   - Every call shares the one array, which keeps the previous call's contents.  Calls
+ *     that overlap on the GPU (on different streams, or from several threads without
+ *     ordering) race on it and produce wrong results; order them on one stream.
+ * ---------------------------------------------------------------------------------- */
+MOE_API moe_status moe_histogram_scan_noalloc(const int32_t* topk_idx, const float* topk_gate,
+                              int32_t T, int32_t k, int32_t E, int32_t capacity,
+                              int32_t* counts, int32_t* kept, int32_t* offsets,
+                              int32_t* row_of, int32_t* token_of_row, float* gate_of_row,
+                              void* stream);
+
+/* ------------------------------------------------------------------------------------
  * moe_permute -- x_perm[row_of[t, j]] = x[t] for every kept assignment.
  * "Send each token to its experts" ([Handbook-News] "MoE 到底省了什么";
  * [Handbook-Article] dispatch as the real bottleneck).

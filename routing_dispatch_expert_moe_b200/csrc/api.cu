@@ -134,6 +134,19 @@ moe_status moe_histogram_scan(const int32_t* topk_idx, const float* topk_gate, i
                                gate_of_row, rows_max, workspace, S(stream));
 }
 
+moe_status moe_histogram_scan_noalloc(const int32_t* topk_idx, const float* topk_gate, int32_t T, int32_t k,
+                                      int32_t E, int32_t capacity, int32_t* counts, int32_t* kept, int32_t* offsets,
+                                      int32_t* row_of, int32_t* token_of_row, float* gate_of_row, void* stream) {
+  moe_status st = check_dims(T, E, k);
+  if (st != MOE_OK) return st;
+  if (capacity < -1) return MOE_ERR_INVALID_ARG;
+  if (!counts || !kept || !offsets) return MOE_ERR_INVALID_ARG;
+  if (T > 0 && (!topk_idx || !topk_gate || !row_of || !token_of_row || !gate_of_row)) return MOE_ERR_INVALID_ARG;
+  const long long rows_max = moe_rows_max(T, E, k, capacity);
+  return launch_histogram_scan_noalloc(topk_idx, topk_gate, T, k, E, capacity, counts, kept, offsets, row_of,
+                                       token_of_row, gate_of_row, rows_max, S(stream));
+}
+
 moe_status moe_permute(const void* x, int32_t dtype, int32_t T, int32_t d, int32_t k, const int32_t* row_of,
                        int64_t rows_max, void* x_perm, void* stream) {
   if (T < 0 || k < 1 || rows_max < 0) return MOE_ERR_INVALID_ARG;

@@ -110,6 +110,10 @@ moe_status launch_histogram_scan(const int32_t* topk_idx, const float* topk_gate
                                  int32_t* offsets, int32_t* row_of, int32_t* token_of_row,
                                  float* gate_of_row, long long rows_max, void* ws, cudaStream_t s);
 size_t histogram_scan_workspace_bytes(int T, int k, int E);
+moe_status launch_histogram_scan_noalloc(const int32_t* topk_idx, const float* topk_gate, int T, int k, int E,
+                                         int capacity, int32_t* counts, int32_t* kept, int32_t* offsets,
+                                         int32_t* row_of, int32_t* token_of_row, float* gate_of_row,
+                                         long long rows_max, cudaStream_t s);
 
 moe_status launch_permute(const void* x, int dtype, int T, int d, int k, const int32_t* row_of,
                           long long rows_max, void* x_perm, cudaStream_t s);

@@ -230,6 +230,46 @@ size_t rank_smem_bytes(int k, int E) {
 
 }  // namespace
 
+// ---------------------------------------------------------------------------------
+// Scratch for callers that cannot allocate (moe_histogram_scan_noalloc): a fixed 4 MiB
+// array in device memory, held by every GPU that loads the library until exit.  The
+// name is only a host-side handle: host code must look up its device address.
+// ---------------------------------------------------------------------------------
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
+static __device__ __align__(256) unsigned char g_scan_scratch[kNoAllocScratchBytes];
+
+// Device address of g_scan_scratch on the current device, looked up once per device.
+static moe_status noalloc_scratch(void** out) {
+  static void* cached[64] = {nullptr};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_status(e);
+  if (dev < 0 || dev >= 64) return MOE_ERR_UNSUPPORTED;
+  if (!cached[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_scan_scratch);
+    if (e != cudaSuccess) return cuda_status(e);
+    cached[dev] = p;
+  }
+  *out = cached[dev];
+  return MOE_OK;
+}
+
+moe_status launch_histogram_scan_noalloc(const int32_t* topk_idx, const float* topk_gate, int T, int k, int E,
+                                         int capacity, int32_t* counts, int32_t* kept, int32_t* offsets,
+                                         int32_t* row_of, int32_t* token_of_row, float* gate_of_row,
+                                         long long rows_max, cudaStream_t s) {
+  if (histogram_scan_workspace_bytes(T, k, E) > kNoAllocScratchBytes) return MOE_ERR_WORKSPACE;
+  void* ws = nullptr;
+  if (T > 0) {
+    moe_status st = noalloc_scratch(&ws);
+    if (st != MOE_OK) return st;
+  }
+  // the launcher clears the ticket and look-back words before the kernels run
+  return launch_histogram_scan(topk_idx, topk_gate, T, k, E, capacity, counts, kept, offsets, row_of, token_of_row,
+                               gate_of_row, rows_max, ws, s);
+}
+
 size_t histogram_scan_workspace_bytes(int T, int k, int E) {
   if (T <= 0) return 0;
   const int C = (T + kChunk - 1) / kChunk;

@@ -39,6 +39,8 @@ _SIGNATURES = {
     "moe_histogram_scan_workspace_bytes": (_size, [_i32, _i32, _i32]),
     "moe_histogram_scan": (_i32, [_c_void_p, _c_void_p, _i32, _i32, _i32, _i32, _c_void_p, _c_void_p, _c_void_p,
                                   _c_void_p, _c_void_p, _c_void_p, _c_void_p, _size, _c_void_p]),
+    "moe_histogram_scan_noalloc": (_i32, [_c_void_p, _c_void_p, _i32, _i32, _i32, _i32, _c_void_p, _c_void_p,
+                                          _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p]),
     "moe_permute": (_i32, [_c_void_p, _i32, _i32, _i32, _i32, _c_void_p, _i64, _c_void_p, _c_void_p]),
     "moe_expert_gate_up": (_i32, [_c_void_p, _i32, _c_void_p, _i32, _i32, _i32, _i64, _c_void_p, _c_void_p,
                                   _c_void_p]),
@@ -191,6 +193,24 @@ def moe_histogram_scan(topk_idx, topk_gate, E: int, capacity: int = -1, counts=N
         _p(token_of_row), _p(gate_of_row), _p(ws), nb, _stream(stream)))
     return {"counts": counts, "kept": kept, "offsets": offsets, "row_of": row_of, "token_of_row": token_of_row,
             "gate_of_row": gate_of_row, "rows_max": rows_max}
+
+
+def moe_histogram_scan_noalloc(topk_idx, topk_gate, E: int, capacity: int, counts, kept, offsets, row_of,
+                               token_of_row, gate_of_row, stream=None):
+    """moe_histogram_scan without a workspace, for callers that cannot allocate device memory:
+    the library's own 4 MiB scratch array is used instead.  Every output buffer must be
+    passed in (this wrapper allocates nothing either).  Calls that overlap on the GPU race
+    on the shared scratch; the first call on a device must come before any stream capture."""
+    T, k = topk_idx.shape
+    _need(topk_idx, "topk_idx", torch.int32)
+    _need(topk_gate, "topk_gate", torch.float32, (T, k))
+    for t, n, dt in ((counts, "counts", torch.int32), (kept, "kept", torch.int32), (offsets, "offsets", torch.int32),
+                     (row_of, "row_of", torch.int32), (token_of_row, "token_of_row", torch.int32),
+                     (gate_of_row, "gate_of_row", torch.float32)):
+        _need(t, n, dt)
+    _check("moe_histogram_scan_noalloc", lib().moe_histogram_scan_noalloc(
+        _p(topk_idx), _p(topk_gate), T, k, E, capacity, _p(counts), _p(kept), _p(offsets), _p(row_of),
+        _p(token_of_row), _p(gate_of_row), _stream(stream)))
 
 
 def moe_permute(x, row_of, rows_max: int, x_perm=None, stream=None):
