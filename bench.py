@@ -134,6 +134,8 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
     cfg = I.CONFIGS[args.workload]
+    if args.tokens:
+        cfg = cfg.with_(T=args.tokens)
     dt = torch.float32 if cfg.act == "f32" else torch.bfloat16
     x_np = I.gen_x(cfg, seed=rank)                      # each replica has its own token batch
     Wg, off, bias = I.gen_router(cfg, 0)
@@ -153,51 +155,70 @@ def run_ours(args):
 
     stage_names = ["route", "histogram_scan", "permute", "gate_up", "down", "shared", "combine", "stats"]
 
-    def step(evs=None):
+    def step(s, evs=None):
+        """One layer forward on stream s; evs: 9 timing events recorded between the stages."""
         T = cfg.T
-        rec = (lambda i: evs[i].record(stream)) if evs is not None else (lambda i: None)
+        rec = (lambda i: evs[i].record(s)) if evs is not None else (lambda i: None)
         rec(0)
-        layer.route(x)
+        layer.route(x, s)
         rec(1)
-        layer.histogram_scan(T)
+        layer.histogram_scan(T, s)
         rec(2)
-        layer.permute(x)
+        layer.permute(x, s)
         rec(3)
-        layer.gate_up()
+        layer.gate_up(s)
         rec(4)
-        layer.down()
+        layer.down(s)
         rec(5)
         if layer.has_shared:
-            layer.shared(x)
+            layer.shared(x, s)
         rec(6)
-        layer.combine(T)
+        layer.combine(T, s)
         rec(7)
-        layer.stats(T)
+        layer.stats(T, s)
         rec(8)
 
     for _ in range(args.warmup):
         flush.zero_()
-        step()
+        step(stream)
     torch.cuda.synchronize()
     assert M.moe_get_device_error() == 0
     A = int(layer.offsets[-1].item())
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(9)] for _ in range(args.steps)]
+    # The step runs as one CUDA graph (no host work between the library's launches); the
+    # timing events are nodes inside the graph, on the stream the kernels run on.
+    evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(9)]
+    graph = torch.cuda.CUDAGraph()
+    cap_stream = torch.cuda.Stream()
+    cap_stream.wait_stream(stream)
+    with torch.cuda.stream(cap_stream):
+        with torch.cuda.graph(graph, stream=cap_stream):
+            step(cap_stream, evs)
+    stream.wait_stream(cap_stream)
+    for _ in range(3):
+        flush.zero_()
+        graph.replay()
+    torch.cuda.synchronize()
+    assert M.moe_get_device_error() == 0
+
     clocks = ClockSampler(local_rank)
     clocks.start()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
+    per_step = np.zeros(args.steps)
+    stage_acc = np.zeros(len(stage_names))
     for i in range(args.steps):
-        flush.zero_()
-        step(evs[i])
+        flush.zero_()                      # L2 flush outside the step
+        graph.replay()
+        torch.cuda.synchronize()           # read this step's in-graph events
+        per_step[i] = evs[0].elapsed_time(evs[8])
+        stage_acc += [evs[j].elapsed_time(evs[j + 1]) for j in range(len(stage_names))]
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     clk = clocks.stop()
-    per_step = np.array([evs[i][0].elapsed_time(evs[i][8]) for i in range(args.steps)])   # ms
-    stage_ms = {n: float(np.mean([evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps)]))
-                for j, n in enumerate(stage_names)}
+    stage_ms = {n: float(stage_acc[j] / args.steps) for j, n in enumerate(stage_names)}
     total_ms = float(per_step.sum())
     if world > 1:
         t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
@@ -209,10 +230,11 @@ def run_ours(args):
     # end to end through the public API with host buffers (pinned), copies inside the timing
     x_host = torch.from_numpy(x_np).to(dt).pin_memory()
     y_host = torch.empty((cfg.T, cfg.d), dtype=layer.out_dtype).pin_memory()
-    e2e_steps = max(3, min(args.steps, 50))
+    e2e_steps = max(3, args.e2e_steps)
+    layer.capture(x)                       # the layer's public graph API: capture once, replay per batch
     for _ in range(2):
         x.copy_(x_host, non_blocking=True)
-        layer.forward(x)
+        layer.replay()
         y_host.copy_(layer.y, non_blocking=True)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -222,7 +244,7 @@ def run_ours(args):
     e0.record(stream)
     for _ in range(e2e_steps):
         x.copy_(x_host, non_blocking=True)
-        layer.forward(x)
+        layer.replay()
         y_host.copy_(layer.y, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
@@ -385,6 +407,9 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-tokens", type=int, default=48, help="tokens per reference-arm step")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override T (smaller cases of the same kernels, e.g. for profiler captures)")
+    ap.add_argument("--e2e-steps", type=int, default=50, help="steps timed through host buffers")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -49,7 +49,8 @@ struct L {
   static constexpr int misc = bars + nbars * 8;              // tmem slot, abort flag
   static constexpr int tiles = misc + 16;                    // int tile_start[kMaxE + 1]
   static constexpr int sh32 = tiles + (kMaxE + 1) * 4;      // int[32]
-  static constexpr int end = sh32 + 32 * 4;
+  static constexpr int stage = (sh32 + 32 * 4 + 15) / 16 * 16;   // 4 epilogue warps x 32 x 144 B
+  static constexpr int end = stage + 4 * 32 * (32 * 4 + 16);
 };
 constexpr size_t kSmemBytes = L::end + 1024;                 // + alignment slack
 
@@ -171,6 +172,49 @@ __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.
 // Ties the loaded registers to the preceding wait so no use is scheduled above it.
 __device__ __forceinline__ void tmem_regs_ready(uint32_t (&r)[32]) { asm volatile("" : MOE_RW32(r)); }
 
+// Epilogue staging: each epilogue warp turns its 32 rows x 32 columns (one value per
+// lane-row from tcgen05.ld) around in shared memory, so that every global store
+// instruction writes whole 128-byte lines of 4 (fp32) or 8 (bf16) rows instead of 32
+// half-filled sectors.  Row pitch padded by 16 bytes: conflict-free 16-byte accesses.
+constexpr int kStagePitchF32 = 32 * 4 + 16;
+constexpr int kStagePitchB16 = 32 * 2 + 16;
+constexpr int kStageWarpBytes = 32 * kStagePitchF32;
+
+template <typename OutT>
+__device__ __forceinline__ void stage_store32(uint8_t* stage, const float (&v)[32], int lane, OutT* out,
+                                              long long row0, int rows_valid, long long ld, int col, int ncols) {
+  if constexpr (sizeof(OutT) == 4) {
+    float4* dst = reinterpret_cast<float4*>(stage + lane * kStagePitchF32);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+    __syncwarp();
+    const int rs = lane >> 3, cv = lane & 7;       // 4 rows per pass, 8 x 16 B per row
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int r = i * 4 + rs;
+      const float4 x = *reinterpret_cast<const float4*>(stage + r * kStagePitchF32 + cv * 16);
+      if (r < rows_valid && col + cv * 4 + 4 <= ncols)
+        *reinterpret_cast<float4*>(out + (row0 + r) * ld + col + cv * 4) = x;
+    }
+  } else {
+    uint4* dst = reinterpret_cast<uint4*>(stage + lane * kStagePitchB16);
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      dst[q] = make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                          pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+    __syncwarp();
+    const int rs = lane >> 2, cv = lane & 3;       // 8 rows per pass, 4 x 16 B per row
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = i * 8 + rs;
+      const uint4 x = *reinterpret_cast<const uint4*>(stage + r * kStagePitchB16 + cv * 16);
+      if (r < rows_valid && col + cv * 8 + 8 <= ncols)
+        *reinterpret_cast<uint4*>(out + (row0 + r) * ld + col + cv * 8) = x;
+    }
+  }
+  __syncwarp();
+}
+
 // OutT: element type of the output rows (MODE 0 always writes bf16 H; MODE 1 writes
 // bf16 or fp32 gated rows).
 template <int MODE, typename OutT>
@@ -189,7 +233,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::misc + 4);
 
   // MODE 0: 128 H columns per tile (128 gate + 128 up accumulator columns)
-  const int n_tiles = MODE == 0 ? (F + 127) / 128 : (N_out + BN - 1) / BN;
+  const int n_tiles = MODE == 0 ? (F + 127) / 128 : (MODE == 1 ? (N_out + BN - 1) / BN : (N_out + 63) / 64);
   build_tile_starts(offsets, E, BM, n_tiles, rows_max, tile_start, sh32, err);
   const int total = tile_start[E];
   if ((int)blockIdx.x >= total) return;   // uniform: nothing allocated yet
@@ -247,8 +291,10 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
             const int g_row = tc.e * 2 * F + tc.n_tile * 128;
             tma_load_2d(b_dst, &tmB, full, kb * BK, g_row);
             tma_load_2d(b_dst + B_STAGE / 2, &tmB, full, kb * BK, g_row + F);
-          } else {
+          } else if (MODE == 1) {
             tma_load_2d(b_dst, &tmB, full, kb * BK, tc.e * N_out + tc.n_tile * BN);
+          } else {
+            tma_load_2d(b_dst, &tmB, full, kb * BK, tc.n_tile * BN);   // router: 256 rows per n-tile
           }
           last_phase[stage] = (int)phase;
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -295,6 +341,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
     // ------------------------------------------------------------ epilogue (warps 2..5)
     const int q = warp & 3;                 // TMEM lane quarter this warp may access
     const int r_in = q * 32 + lane;         // accumulator row == tile row
+    uint8_t* stage = smem + L::stage + (warp - 2) * kStageWarpBytes;
     int it = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
       const TileCoord tc = tile_coord(tile_start, offsets, E, BM, tile);
@@ -308,9 +355,10 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
       const bool valid = r_in < tc.rows;
       const long long row = (long long)tc.row0 + r_in;
+      const long long wrow0 = (long long)tc.row0 + q * 32;          // first row of this warp
+      const int wrows = min(32, max(0, tc.rows - q * 32));          // valid rows of this warp
       if constexpr (MODE == 0) {
         const int f0 = tc.n_tile * 128;
-        OutT* orow = out + row * F;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t g[32], u[32];
@@ -319,55 +367,50 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
           tmem_wait_ld();
           tmem_regs_ready(g);
           tmem_regs_ready(u);
-          if (valid) {
-            const int col = f0 + c * 32;
-            uint32_t pk[16];
+          float h[32];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
-              const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
-              const float h0 = g0 / (1.f + expf(-g0)) * u0;
-              const float h1 = g1 / (1.f + expf(-g1)) * u1;
-              pk[i] = pack_bf16x2(h0, h1);
-            }
-#pragma unroll
-            for (int v = 0; v < 4; ++v)
-              if (col + 8 * v + 8 <= F)
-                *reinterpret_cast<uint4*>(orow + col + 8 * v) =
-                    make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          for (int i = 0; i < 32; ++i) {
+            const float gi = __uint_as_float(g[i]);
+            h[i] = gi / (1.f + expf(-gi)) * __uint_as_float(u[i]);
           }
+          stage_store32<OutT>(stage, h, lane, out, wrow0, wrows, F, f0 + c * 32, F);
         }
-      } else {
+      } else if constexpr (MODE == 1) {
         const int n0 = tc.n_tile * BN;
         const float gs = (valid && gate_of_row) ? __ldg(gate_of_row + row) : 1.f;
-        OutT* orow = out + row * N_out;
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
           uint32_t v32[32];
           tmem_ld32(taddr + c * 32, v32);
           tmem_wait_ld();
           tmem_regs_ready(v32);
-          if (valid) {
-            const int col = n0 + c * 32;
-            if constexpr (sizeof(OutT) == 2) {
-              uint32_t pk[16];
+          float y[32];
 #pragma unroll
-              for (int i = 0; i < 16; ++i)
-                pk[i] = pack_bf16x2(__uint_as_float(v32[2 * i]) * gs, __uint_as_float(v32[2 * i + 1]) * gs);
+          for (int i = 0; i < 32; ++i) y[i] = __uint_as_float(v32[i]) * gs;
+          stage_store32<OutT>(stage, y, lane, out, wrow0, wrows, N_out, n0 + c * 32, N_out);
+        }
+      } else {
+        // MODE 2, router logits: columns [0,64) x.hi, [64,128) x.mid, [128,192) x.lo for
+        // experts e0..e0+63; logit = (hi + mid) + lo + offset (gate_of_row carries the offset)
+        const int e0 = tc.n_tile * 64;
+#pragma unroll 1
+        for (int c = 0; c < 2; ++c) {
+          uint32_t a[32], b[32], l3[32];
+          tmem_ld32(taddr + c * 32, a);
+          tmem_ld32(taddr + 64 + c * 32, b);
+          tmem_ld32(taddr + 128 + c * 32, l3);
+          tmem_wait_ld();
+          tmem_regs_ready(a);
+          tmem_regs_ready(b);
+          tmem_regs_ready(l3);
+          float lv[32];
 #pragma unroll
-              for (int v = 0; v < 4; ++v)
-                if (col + 8 * v + 8 <= N_out)
-                  *reinterpret_cast<uint4*>(orow + col + 8 * v) =
-                      make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
-            } else {
-#pragma unroll
-              for (int v = 0; v < 8; ++v)
-                if (col + 4 * v + 4 <= N_out)
-                  *reinterpret_cast<float4*>(orow + col + 4 * v) =
-                      make_float4(__uint_as_float(v32[4 * v]) * gs, __uint_as_float(v32[4 * v + 1]) * gs,
-                                  __uint_as_float(v32[4 * v + 2]) * gs, __uint_as_float(v32[4 * v + 3]) * gs);
-            }
+          for (int i = 0; i < 32; ++i) {
+            const int e = e0 + c * 32 + i;
+            const float off = (gate_of_row && e < N_out) ? __ldg(gate_of_row + e) : 0.f;
+            lv[i] = ((__uint_as_float(a[i]) + __uint_as_float(b[i])) + __uint_as_float(l3[i])) + off;
           }
+          stage_store32<OutT>(stage, lv, lane, out, wrow0, wrows, N_out, e0 + c * 32, N_out);
         }
       }
       tc_fence_before();
@@ -427,7 +470,7 @@ moe_status launch_tc(const CUtensorMap& ma, const CUtensorMap& mb, const int32_t
     if (e != cudaSuccess) return cuda_status(e);
     configured[dev] = 1;
   }
-  const int n_tiles = MODE == 0 ? (F + 127) / 128 : (N_out + BN - 1) / BN;
+  const int n_tiles = MODE == 0 ? (F + 127) / 128 : (MODE == 1 ? (N_out + BN - 1) / BN : (N_out + 63) / 64);
   const long long max_tiles = ((rows_max + BM - 1) / BM + E) * (long long)n_tiles;
   int grid = num_sms();
   if (max_tiles < grid) grid = (int)max_tiles;
@@ -440,6 +483,19 @@ moe_status launch_tc(const CUtensorMap& ma, const CUtensorMap& mb, const int32_t
 }  // namespace
 
 // Returns MOE_ERR_UNSUPPORTED when a tensor map cannot be encoded (caller falls back).
+// Router logits on the tensor cores: A = x [T, d] bf16 (one group, offs2 = {0, T}),
+// B = the split weight W3 [ceil(E/64) * 256, d]; writes logits [T, E] fp32 (+ offset).
+moe_status launch_router_logits_tc(const void* x, const int32_t* offs2, int T, int d, int E, const void* W3,
+                                   const float* logit_offset, float* logits, cudaStream_t s) {
+  if (T == 0) return MOE_OK;
+  if (d < BK || d % 8 != 0 || E % 4 != 0) return MOE_ERR_UNSUPPORTED;
+  const int nt = (E + 63) / 64;
+  CUtensorMap ma, mb;
+  if (!make_map(&ma, x, (unsigned long long)T, d, BM)) return MOE_ERR_UNSUPPORTED;
+  if (!make_map(&mb, W3, (unsigned long long)nt * 256, d, BN)) return MOE_ERR_UNSUPPORTED;
+  return launch_tc<2, float>(ma, mb, offs2, 1, d, E, 0, T, logit_offset, logits, s);
+}
+
 moe_status launch_gate_up_tc(const void* x_rows, const int32_t* offsets, int E, int d, int F, long long rows_max,
                              const void* W_gu, void* h, cudaStream_t s) {
   if (rows_max == 0) return MOE_OK;

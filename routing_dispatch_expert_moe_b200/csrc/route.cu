@@ -354,6 +354,46 @@ topk_kernel(const float* __restrict__ partial, int nsplit, long long split_strid
   }
 }
 
+// ---------------------------------------------------------------------------------
+// Tensor-core router operand: W_g [d, E] fp32 split into three bf16 terms
+//   hi = bf16(w), mid = bf16(w - hi), lo = bf16(w - hi - mid)
+// (each subtraction is exact in fp32; hi + mid + lo carries w to about 24 bits, and x is
+// bf16, so every product x * term is exact in fp32).  Layout W3 [n_tiles * 256, d] bf16,
+// K-major: n-tile j holds experts 64j..64j+63 as rows [0,64) hi, [64,128) mid,
+// [128,192) lo, [192,256) zero.  One 32 x 32 shared-memory transpose per block.
+// ---------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+split_router_weight_kernel(const float* __restrict__ Wg, int d, int E, __nv_bfloat16* __restrict__ W3,
+                           int32_t* __restrict__ offs2, int T) {
+  __shared__ float tile[32][33];
+  const int c0 = blockIdx.x * 32, e0 = blockIdx.y * 32;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;   // 32 x 8
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int c = c0 + ty + 8 * i, e = e0 + tx;
+    tile[ty + 8 * i][tx] = (c < d && e < E) ? __ldg(Wg + (long long)c * E + e) : 0.f;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int e = e0 + ty + 8 * i, c = c0 + tx;
+    if (e >= E || c >= d) continue;
+    const float w = tile[tx][ty + 8 * i];
+    const __nv_bfloat16 hi = __float2bfloat16_rn(w);
+    const float r1 = w - __bfloat162float(hi);
+    const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
+    const long long base = (long long)(e >> 6) * 256 + (e & 63);
+    W3[(base + 0) * d + c] = hi;
+    W3[(base + 64) * d + c] = mid;
+    W3[(base + 128) * d + c] = lo;
+  }
+  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
+    offs2[0] = 0;
+    offs2[1] = T;
+  }
+}
+
 struct LogitsPlan {
   int BE, TM, BT, nsplit, chunks_per_split;
   size_t smem;
@@ -380,9 +420,16 @@ template <typename XT, int BE, int TM>
 moe_status run_logits(const void* x, const float* Wg, const float* off, int T, int d, int E,
                       const LogitsPlan& p, float* out, long long split_stride, cudaStream_t s) {
   auto kern = logits_kernel<XT, BE, TM>;
-  if (p.smem > 48 * 1024) {
+  // the shared-memory size is fixed per instantiation: raise the limit once per device,
+  // never inside a launch sequence that may be captured into a CUDA graph
+  static int configured[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  dev &= 63;
+  if (p.smem > 48 * 1024 && !configured[dev]) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
     if (e != cudaSuccess) return cuda_status(e);
+    configured[dev] = 1;
   }
   dim3 grid((T + p.BT - 1) / p.BT, (E + BE - 1) / BE, p.nsplit);
   kern<<<grid, kLogitThreads, p.smem, s>>>(x, Wg, off, T, d, E, p.chunks_per_split, out, split_stride);
@@ -422,10 +469,17 @@ moe_status run_topk(bool bias, const float* partial, int nsplit, long long split
 
 }  // namespace
 
+// The tensor-core router takes bf16 x with d >= 64 and E a multiple of 4 (16-byte logit
+// rows); anything else runs the fp32 SIMT router.
+static bool tc_router_ok(int x_dtype, int d, int E) { return x_dtype == MOE_BF16 && d >= 64 && E % 4 == 0; }
+static size_t tc_router_w3_bytes(int d, int E) { return (size_t)((E + 63) / 64) * 256 * d * 2; }
+
 size_t route_workspace_bytes(int T, int d, int E) {
   if (T <= 0 || E <= 0 || d <= 0) return 0;
   LogitsPlan p = plan_logits(T, d, E);
-  return p.nsplit > 1 ? (size_t)p.nsplit * T * E * sizeof(float) : 0;
+  const size_t simt = p.nsplit > 1 ? (size_t)p.nsplit * T * E * sizeof(float) : 0;
+  const size_t tc = (E % 4 == 0 && d >= 64) ? 256 + tc_router_w3_bytes(d, E) : 0;
+  return simt > tc ? simt : tc;
 }
 
 moe_status launch_route(const void* x, int x_dtype, const float* Wg, const float* logit_offset,
@@ -434,11 +488,29 @@ moe_status launch_route(const void* x, int x_dtype, const float* Wg, const float
                         float* topk_gate, void* ws, cudaStream_t s) {
   if (T == 0) return MOE_OK;
   LogitsPlan p = plan_logits(T, d, E);
-  float* partial = p.nsplit > 1 ? static_cast<float*>(ws) : logits;
+  float* partial = logits;
   const long long split_stride = (long long)T * E;
-  moe_status st = x_dtype == MOE_F32
-                      ? dispatch_logits<float>(x, Wg, logit_offset, T, d, E, p, partial, split_stride, s)
-                      : dispatch_logits<__nv_bfloat16>(x, Wg, logit_offset, T, d, E, p, partial, split_stride, s);
+  moe_status st = MOE_ERR_UNSUPPORTED;
+  if (tc_router_ok(x_dtype, d, E)) {
+    // split W_g into three bf16 terms, then one tcgen05 GEMM writes logits (+ offset)
+    int32_t* offs2 = static_cast<int32_t*>(ws);
+    __nv_bfloat16* W3 = reinterpret_cast<__nv_bfloat16*>(static_cast<char*>(ws) + 256);
+    st = cuda_status(cudaMemsetAsync(W3, 0, tc_router_w3_bytes(d, E), s));
+    if (st != MOE_OK) return st;
+    dim3 g((d + 31) / 32, (E + 31) / 32);
+    split_router_weight_kernel<<<g, 256, 0, s>>>(Wg, d, E, W3, offs2, T);
+    st = check_launch();
+    if (st != MOE_OK) return st;
+    st = launch_router_logits_tc(x, offs2, T, d, E, W3, logit_offset, logits, s);
+    if (st != MOE_OK && st != MOE_ERR_UNSUPPORTED) return st;
+    if (st == MOE_OK) p.nsplit = 1;
+  }
+  if (st == MOE_ERR_UNSUPPORTED) {
+    partial = p.nsplit > 1 ? static_cast<float*>(ws) : logits;
+    st = x_dtype == MOE_F32
+             ? dispatch_logits<float>(x, Wg, logit_offset, T, d, E, p, partial, split_stride, s)
+             : dispatch_logits<__nv_bfloat16>(x, Wg, logit_offset, T, d, E, p, partial, split_stride, s);
+  }
   if (st != MOE_OK) return st;
   const int write = p.nsplit > 1 ? 1 : 0;
   const int epl = (E + 31) / 32;

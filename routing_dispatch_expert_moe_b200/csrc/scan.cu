@@ -291,9 +291,17 @@ moe_status launch_histogram_scan(const int32_t* topk_idx, const float* topk_gate
   if (st != MOE_OK) return st;
   const int nchunks = (T + kChunk - 1) / kChunk;
   const size_t smem = rank_smem_bytes(k, E);
-  if (smem > 48 * 1024) {
-    st = cuda_status(cudaFuncSetAttribute(rank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  // raise the limit once per device to the largest size any supported (k, E) needs, so
+  // that no attribute call happens inside a launch sequence captured into a CUDA graph
+  static int configured[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  dev &= 63;
+  if (!configured[dev]) {
+    st = cuda_status(cudaFuncSetAttribute(rank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          (int)rank_smem_bytes(32, 1024)));
     if (st != MOE_OK) return st;
+    configured[dev] = 1;
   }
   int* err = err_ptr();
   rank_kernel<<<nchunks, kRankThreads, smem, s>>>(topk_idx, T, k, E, capacity, nchunks, w.ticket, w.status,

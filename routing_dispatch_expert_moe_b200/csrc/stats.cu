@@ -117,13 +117,25 @@ stats_final_kernel(const double* __restrict__ partP, const double* __restrict__ 
                    const int32_t* __restrict__ counts, const int32_t* __restrict__ kept, int T, int E,
                    int k, float* __restrict__ load, float* __restrict__ stats5) {
   __shared__ double sh[32];
+  __shared__ double Ps[1024];
   const double TK = (double)T * k;
   const double mean = TK / E;
+  // P_e: one warp per expert, lanes take the partials in a fixed strided order, then a
+  // fixed butterfly -- many loads in flight, same result every run
+  {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    for (int e = warp; e < E; e += nw) {
+      double p = 0.0;
+      for (int b = lane; b < nparts; b += 32) p += partP[(long long)b * E + e];
+#pragma unroll
+      for (int o = 16; o; o >>= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
+      if (lane == 0) Ps[e] = p;
+    }
+    __syncthreads();
+  }
   double aux = 0.0, kept_sum = 0.0, var = 0.0, cmax = 0.0;
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    double P = 0.0;
-    for (int b = 0; b < nparts; ++b) P += partP[(long long)b * E + e];
-    P /= (double)T;
+    const double P = Ps[e] / (double)T;
     const double c = (double)counts[e];
     const double f = c / TK;
     load[e] = (float)f;
@@ -147,9 +159,13 @@ stats_final_kernel(const double* __restrict__ partP, const double* __restrict__ 
     for (int w = 0; w < (int)((blockDim.x + 31) >> 5); ++w) r = fmax(r, sh[w]);
     cmax = r;
   }
+  double z = 0.0;
+  if (threadIdx.x < 32) {
+    for (int b = threadIdx.x; b < nparts; b += 32) z += partZ[b];
+#pragma unroll
+    for (int o = 16; o; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+  }
   if (threadIdx.x == 0) {
-    double z = 0.0;
-    for (int b = 0; b < nparts; ++b) z += partZ[b];
     stats5[0] = (float)(E * aux);
     stats5[1] = (float)(z / (double)T);
     stats5[2] = (float)(TK - kept_sum);

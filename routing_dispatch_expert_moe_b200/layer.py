@@ -126,6 +126,30 @@ class MoELayer:
             self.stats(T, stream)
         return self.y[:T]
 
+    # ---------------------------------------------------------------- CUDA graph
+    def capture(self, x_static: torch.Tensor, with_stats: bool = True) -> None:
+        """Records one forward over the fixed input buffer x_static into a CUDA graph.
+
+        Replaying it (replay()) runs the same library kernels with no host work per
+        step.  Write the next batch into x_static before each replay.  One eager forward
+        runs first so that every per-device lookup happens outside the capture.
+        """
+        self.x_static = x_static
+        self.forward(x_static, with_stats=with_stats)
+        torch.cuda.synchronize()
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(s):
+            with torch.cuda.graph(self.graph, stream=s):
+                self.forward(x_static, stream=s, with_stats=with_stats)
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+
+    def replay(self) -> torch.Tensor:
+        self.graph.replay()
+        return self.y[:self.x_static.shape[0]]
+
     # library kernels launched by one forward (the scan's workspace memset is not a kernel)
     def launches_per_forward(self, with_stats: bool = True) -> int:
         n = 2 + 2 + 1 + 1 + 1 + 1          # route(2) scan(2) permute gate_up down combine

@@ -157,6 +157,29 @@ def test_deterministic_run_to_run():
         assert np.array_equal(a[key], b[key]), key
 
 
+def test_cuda_graph_replay_matches_eager_forward():
+    cfg = I.small_config("graph", T=640, d=256, E=32, k=4, F=128, F_s=128, score="sigmoid", scale=2.5,
+                         capacity_factor=1.0, select_bias="uniform0.1")
+    host, dev = U.make_inputs(cfg)
+    cap = O.capacity(cfg.T, cfg.E, cfg.k, cfg.capacity_factor)
+    layer = U.build_layer(cfg, dev, cap)
+    y_eager = layer.forward(dev["x"]).clone()
+    idx_eager = layer.topk_idx.clone()
+    x_static = dev["x"].clone()
+    layer.capture(x_static)
+    x_static.copy_(torch.flip(dev["x"], dims=[0]))        # a different batch through the same graph
+    layer.replay()
+    y_flip = layer.y.clone()
+    x_static.copy_(dev["x"])
+    layer.replay()
+    torch.cuda.synchronize()
+    from routing_dispatch_expert_moe_b200 import moe as M
+    assert M.moe_get_device_error() == 0
+    assert torch.equal(layer.topk_idx, idx_eager)
+    assert torch.equal(layer.y, y_eager)
+    assert not torch.equal(y_flip, y_eager)
+
+
 def test_corrupt_expert_id_is_reported_not_trapped():
     from routing_dispatch_expert_moe_b200 import moe as M
     T, k, E = 64, 2, 8
