@@ -137,6 +137,57 @@ __device__ __forceinline__ void umma_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
 }
 
+// ---- CTA-pair (cta_group::2) forms: an M=256 MMA issued by the pair's even CTA over
+// both CTAs' shared memory, accumulating into both CTAs' TMEM ----
+constexpr uint32_t kIdesc2 = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                             ((uint32_t)((2 * BM) >> 4) << 24);
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// The same shared-memory object in CTA `rank` of the cluster (shared::cluster address).
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+// TMA load into this CTA's shared memory whose completion is counted on an mbarrier that
+// may live in the peer CTA (the pair's even CTA); no multicast.
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar_cluster, int x,
+                                                 int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+      "[%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar_cluster)
+      : "memory");
+}
+__device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(kIdesc2), "r"(accumulate)
+      : "memory");
+}
+// Completion of the pair's MMAs arrives on the barrier at this offset in both CTAs.
+__device__ __forceinline__ void umma_commit_pair_both(uint32_t bar) {
+  const uint16_t both = 0x3;
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+               ::"r"(bar), "h"(both)
+               : "memory");
+}
+__device__ __forceinline__ void umma_commit_pair(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
 // K-major operand in the canonical 128-byte-swizzle layout written by TMA:
 // rows of 128 bytes (64 bf16), 8-row atoms of 1024 bytes stacked densely.
 __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
@@ -217,6 +268,73 @@ __device__ __forceinline__ void stage_store32(uint8_t* stage, const float (&v)[3
 
 // OutT: element type of the output rows (MODE 0 always writes bf16 H; MODE 1 writes
 // bf16 or fp32 gated rows).
+// One tile's epilogue for one warp: its 32 accumulator rows (TMEM lanes at taddr) become
+// output rows wrow0 .. wrow0 + wrows - 1.  The whole warp must call it (tcgen05.ld is
+// .sync.aligned); rows past wrows are read but not stored.
+//   MODE 0: columns [0,128) gate, [128,256) up -> H = silu(g) * u for features n_tile*128 + ...
+//   MODE 1: 256 columns -> gate_of_row[row] * acc for outputs n_tile*256 + ...
+//   MODE 2: [0,64) x.hi, [64,128) x.mid, [128,192) x.lo of experts n_tile*64 + ... ->
+//           logit = (hi + mid) + lo + offset (gate_of_row carries the logit offset)
+template <int MODE, typename OutT>
+__device__ __forceinline__ void epilogue_tile(uint32_t taddr, uint8_t* stage, int lane, long long wrow0, int wrows,
+                                              int n_tile, int F, int N_out, const float* __restrict__ gate_of_row,
+                                              OutT* __restrict__ out) {
+  if constexpr (MODE == 0) {
+    const int f0 = n_tile * 128;
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      uint32_t g[32], u[32];
+      tmem_ld32(taddr + c * 32, g);
+      tmem_ld32(taddr + 128 + c * 32, u);
+      tmem_wait_ld();
+      tmem_regs_ready(g);
+      tmem_regs_ready(u);
+      float h[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float gi = __uint_as_float(g[i]);
+        h[i] = gi / (1.f + expf(-gi)) * __uint_as_float(u[i]);
+      }
+      stage_store32<OutT>(stage, h, lane, out, wrow0, wrows, F, f0 + c * 32, F);
+    }
+  } else if constexpr (MODE == 1) {
+    const int n0 = n_tile * BN;
+    const float gs = (lane < wrows && gate_of_row) ? __ldg(gate_of_row + wrow0 + lane) : 1.f;
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+      uint32_t v32[32];
+      tmem_ld32(taddr + c * 32, v32);
+      tmem_wait_ld();
+      tmem_regs_ready(v32);
+      float y[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) y[i] = __uint_as_float(v32[i]) * gs;
+      stage_store32<OutT>(stage, y, lane, out, wrow0, wrows, N_out, n0 + c * 32, N_out);
+    }
+  } else {
+    const int e0 = n_tile * 64;
+#pragma unroll 1
+    for (int c = 0; c < 2; ++c) {
+      uint32_t a[32], b[32], l3[32];
+      tmem_ld32(taddr + c * 32, a);
+      tmem_ld32(taddr + 64 + c * 32, b);
+      tmem_ld32(taddr + 128 + c * 32, l3);
+      tmem_wait_ld();
+      tmem_regs_ready(a);
+      tmem_regs_ready(b);
+      tmem_regs_ready(l3);
+      float lv[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int e = e0 + c * 32 + i;
+        const float off = (gate_of_row && e < N_out) ? __ldg(gate_of_row + e) : 0.f;
+        lv[i] = ((__uint_as_float(a[i]) + __uint_as_float(b[i])) + __uint_as_float(l3[i])) + off;
+      }
+      stage_store32<OutT>(stage, lv, lane, out, wrow0, wrows, N_out, e0 + c * 32, N_out);
+    }
+  }
+}
+
 template <int MODE, typename OutT>
 __global__ void __launch_bounds__(kThreadsTC, 1)
 grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -353,66 +471,10 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
       __syncwarp();
       tc_fence_after();
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-      const bool valid = r_in < tc.rows;
-      const long long row = (long long)tc.row0 + r_in;
       const long long wrow0 = (long long)tc.row0 + q * 32;          // first row of this warp
       const int wrows = min(32, max(0, tc.rows - q * 32));          // valid rows of this warp
-      if constexpr (MODE == 0) {
-        const int f0 = tc.n_tile * 128;
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t g[32], u[32];
-          tmem_ld32(taddr + c * 32, g);
-          tmem_ld32(taddr + 128 + c * 32, u);
-          tmem_wait_ld();
-          tmem_regs_ready(g);
-          tmem_regs_ready(u);
-          float h[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float gi = __uint_as_float(g[i]);
-            h[i] = gi / (1.f + expf(-gi)) * __uint_as_float(u[i]);
-          }
-          stage_store32<OutT>(stage, h, lane, out, wrow0, wrows, F, f0 + c * 32, F);
-        }
-      } else if constexpr (MODE == 1) {
-        const int n0 = tc.n_tile * BN;
-        const float gs = (valid && gate_of_row) ? __ldg(gate_of_row + row) : 1.f;
-#pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          uint32_t v32[32];
-          tmem_ld32(taddr + c * 32, v32);
-          tmem_wait_ld();
-          tmem_regs_ready(v32);
-          float y[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) y[i] = __uint_as_float(v32[i]) * gs;
-          stage_store32<OutT>(stage, y, lane, out, wrow0, wrows, N_out, n0 + c * 32, N_out);
-        }
-      } else {
-        // MODE 2, router logits: columns [0,64) x.hi, [64,128) x.mid, [128,192) x.lo for
-        // experts e0..e0+63; logit = (hi + mid) + lo + offset (gate_of_row carries the offset)
-        const int e0 = tc.n_tile * 64;
-#pragma unroll 1
-        for (int c = 0; c < 2; ++c) {
-          uint32_t a[32], b[32], l3[32];
-          tmem_ld32(taddr + c * 32, a);
-          tmem_ld32(taddr + 64 + c * 32, b);
-          tmem_ld32(taddr + 128 + c * 32, l3);
-          tmem_wait_ld();
-          tmem_regs_ready(a);
-          tmem_regs_ready(b);
-          tmem_regs_ready(l3);
-          float lv[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int e = e0 + c * 32 + i;
-            const float off = (gate_of_row && e < N_out) ? __ldg(gate_of_row + e) : 0.f;
-            lv[i] = ((__uint_as_float(a[i]) + __uint_as_float(b[i])) + __uint_as_float(l3[i])) + off;
-          }
-          stage_store32<OutT>(stage, lv, lane, out, wrow0, wrows, N_out, e0 + c * 32, N_out);
-        }
-      }
+      (void)r_in;
+      epilogue_tile<MODE, OutT>(taddr, stage, lane, wrow0, wrows, tc.n_tile, F, N_out, gate_of_row, out);
       tc_fence_before();
       mbar_arrive(bar_tempty + 8 * acc);
     }
@@ -422,6 +484,180 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
   if (warp == 1) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols) : "memory");
+  }
+}
+
+// =====================================================================================
+// CTA-pair version: a cluster of 2 CTAs computes a 256 x 256 tile.  Each CTA stages its
+// own 128 rows of A and half (128 rows) of B per k-block -- 32 KB instead of 48 KB, so a
+// 6-stage ring fits -- and the even CTA issues cta_group::2 MMAs that read both CTAs'
+// stages and accumulate each CTA's 128 rows in that CTA's TMEM.
+//   full[s]   (even CTA only) : even CTA's expect_tx + both CTAs' TMA bytes
+//   empty[s]  (both CTAs)     : MMA completion, multicast commit
+//   tfull[a]  (both CTAs)     : accumulator ready, multicast commit
+//   tempty[a] (even CTA only) : 256 epilogue threads of both CTAs
+// Cluster barriers after set-up and before teardown; every wait bounded.
+// =====================================================================================
+constexpr int STAGES2 = 6;
+constexpr int B2_STAGE = BM * BK * 2;                        // 128 B-rows per CTA: 16 KB
+
+struct L2 {
+  static constexpr int a = 0;
+  static constexpr int b = STAGES2 * A_STAGE;
+  static constexpr int bars = b + STAGES2 * B2_STAGE;
+  static constexpr int nbars = 2 * STAGES2 + 4 + 1;
+  static constexpr int misc = bars + nbars * 8;
+  static constexpr int tiles = misc + 16;
+  static constexpr int sh32 = tiles + (kMaxE + 1) * 4;
+  static constexpr int stage = (sh32 + 32 * 4 + 15) / 16 * 16;
+  static constexpr int end = stage + 4 * 32 * (32 * 4 + 16);
+};
+constexpr size_t kSmemBytes2 = L2::end + 1024;
+
+template <int MODE, typename OutT>
+__global__ void __launch_bounds__(kThreadsTC, 1)
+grouped_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                        const int32_t* __restrict__ offsets, int E, int K, int N_out, int F,
+                        long long rows_max, const float* __restrict__ gate_of_row,
+                        OutT* __restrict__ out, int* err) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int* tile_start = reinterpret_cast<int*>(smem + L2::tiles);
+  int* sh32 = reinterpret_cast<int*>(smem + L2::sh32);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L2::misc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L2::misc + 4);
+  const uint32_t rank = cluster_ctarank();                   // 0 = even CTA (MMA issuer)
+  const int cid = (int)(blockIdx.x >> 1), ncl = (int)(gridDim.x >> 1);
+  constexpr int PM = 2 * BM;                                 // rows per pair tile
+
+  const int n_tiles = MODE == 0 ? (F + 127) / 128 : (MODE == 1 ? (N_out + BN - 1) / BN : (N_out + 63) / 64);
+  build_tile_starts(offsets, E, PM, n_tiles, rows_max, tile_start, sh32, err);
+  const int total = tile_start[E];
+  if (cid >= total) return;   // both CTAs of the pair see the same cid: uniform, nothing allocated
+
+  const uint32_t bar_full = sb + L2::bars;
+  const uint32_t bar_empty = bar_full + 8 * STAGES2;
+  const uint32_t bar_tfull = bar_empty + 8 * STAGES2;
+  const uint32_t bar_tempty = bar_tfull + 16;
+  const uint32_t bar_fin = bar_tempty + 16;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES2; ++s) {
+      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_empty + 8 * s, 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(bar_tfull + 8 * a, 1);
+      mbar_init(bar_tempty + 8 * a, 2 * 128);
+    }
+    mbar_init(bar_fin, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();                                           // peer barriers initialised
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int KB = (K + BK - 1) / BK;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer (both CTAs)
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int last_phase[STAGES2];
+#pragma unroll
+      for (int s = 0; s < STAGES2; ++s) last_phase[s] = -1;
+      bool ok = true;
+      for (int tile = cid; ok && tile < total; tile += ncl) {
+        const TileCoord tc = tile_coord(tile_start, offsets, E, PM, tile);
+        const int a_row = tc.row0 + (int)rank * BM;
+        int b_row;
+        if (MODE == 0) b_row = tc.e * 2 * F + (rank ? F : 0) + tc.n_tile * 128;   // even: gate, odd: up
+        else if (MODE == 1) b_row = tc.e * N_out + tc.n_tile * BN + (int)rank * BM;
+        else b_row = tc.n_tile * BN + (int)rank * BM;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1u, abort_flag, err)) { ok = false; break; }
+          if (rank == 0) mbar_expect_tx(bar_full + 8 * stage, 2 * (A_STAGE + B2_STAGE));
+          const uint32_t full_c = map_to_rank(bar_full + 8 * stage, 0);
+          tma_load_2d_pair(sb + L2::a + stage * A_STAGE, &tmA, full_c, kb * BK, a_row);
+          tma_load_2d_pair(sb + L2::b + stage * B2_STAGE, &tmB, full_c, kb * BK, b_row);
+          last_phase[stage] = (int)phase;
+          if (++stage == STAGES2) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok && rank == 0) {
+        for (int s = 0; s < STAGES2; ++s)
+          if (last_phase[s] >= 0) mbar_wait_drain(bar_full + 8 * s, (uint32_t)last_phase[s], err);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (even CTA)
+    if (lane == 0 && rank == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      for (int tile = cid; ok && tile < total; tile += ncl, ++it) {
+        const int acc = it & 1;
+        const uint32_t acc_phase = (uint32_t)(it >> 1) & 1u;
+        if (!mbar_wait(bar_tempty + 8 * acc, acc_phase ^ 1u, abort_flag, err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag, err)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t adesc = sw128_desc(sb + L2::a + stage * A_STAGE);
+          const uint64_t bdesc = sw128_desc(sb + L2::b + stage * B2_STAGE);
+#pragma unroll
+          for (int kk = 0; kk < BK / UMMA_K; ++kk)
+            umma_bf16_pair(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, (kb | kk) != 0 ? 1u : 0u);
+          umma_commit_pair_both(bar_empty + 8 * stage);
+          if (++stage == STAGES2) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma_commit_pair_both(bar_tfull + 8 * acc);
+      }
+      umma_commit_pair(bar_fin);
+      mbar_wait_drain(bar_fin, 0, err);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int q = warp & 3;
+    uint8_t* stage = smem + L2::stage + (warp - 2) * kStageWarpBytes;
+    int it = 0;
+    for (int tile = cid; tile < total; tile += ncl, ++it) {
+      const TileCoord tc = tile_coord(tile_start, offsets, E, PM, tile);
+      const int acc = it & 1;
+      const uint32_t acc_phase = (uint32_t)(it >> 1) & 1u;
+      const bool got = mbar_wait(bar_tfull + 8 * acc, acc_phase, abort_flag, err);
+      if (!__all_sync(0xffffffffu, got)) break;
+      __syncwarp();
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+      const int cta_rows = min(BM, max(0, tc.rows - (int)rank * BM));
+      const long long wrow0 = (long long)tc.row0 + (int)rank * BM + q * 32;
+      const int wrows = min(32, max(0, cta_rows - q * 32));
+      epilogue_tile<MODE, OutT>(taddr, stage, lane, wrow0, wrows, tc.n_tile, F, N_out, gate_of_row, out);
+      tc_fence_before();
+      mbar_arrive_cluster(map_to_rank(bar_tempty + 8 * acc, 0));
+    }
+  }
+
+  __syncthreads();
+  cluster_sync();                                           // no remote arrive after a CTA exits
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols) : "memory");
   }
 }
 
@@ -485,14 +721,54 @@ moe_status launch_tc(const CUtensorMap& ma, const CUtensorMap& mb, const int32_t
 // Returns MOE_ERR_UNSUPPORTED when a tensor map cannot be encoded (caller falls back).
 // Router logits on the tensor cores: A = x [T, d] bf16 (one group, offs2 = {0, T}),
 // B = the split weight W3 [ceil(E/64) * 256, d]; writes logits [T, E] fp32 (+ offset).
+// CTA pairs pay off when groups average at least one full 256-row pair tile; smaller
+// groups keep the single-CTA kernel (less padding in ragged groups).
+static bool use_pairs(long long rows_max, int groups) { return groups > 0 && rows_max / groups >= 2 * BM; }
+
+template <int MODE, typename OutT>
+moe_status launch_tc2(const CUtensorMap& ma, const CUtensorMap& mb, const int32_t* offsets, int E, int K, int N_out,
+                      int F, long long rows_max, const float* gate_of_row, void* out, cudaStream_t s) {
+  static int configured[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  dev &= 63;
+  if (!configured[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_tc2_kernel<MODE, OutT>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes2);
+    if (e != cudaSuccess) return cuda_status(e);
+    configured[dev] = 1;
+  }
+  const int n_tiles = MODE == 0 ? (F + 127) / 128 : (MODE == 1 ? (N_out + BN - 1) / BN : (N_out + 63) / 64);
+  const long long max_tiles = ((rows_max + 2 * BM - 1) / (2 * BM) + E) * (long long)n_tiles;
+  int pairs = num_sms() / 2;
+  if (max_tiles < pairs) pairs = (int)max_tiles;
+  if (pairs < 1) pairs = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cfg.blockDim = dim3(kThreadsTC, 1, 1);
+  cfg.dynamicSmemBytes = kSmemBytes2;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cuda_status(cudaLaunchKernelEx(&cfg, grouped_gemm_tc2_kernel<MODE, OutT>, ma, mb, offsets, E, K, N_out, F,
+                                        rows_max, gate_of_row, static_cast<OutT*>(out), err_ptr()));
+}
+
 moe_status launch_router_logits_tc(const void* x, const int32_t* offs2, int T, int d, int E, const void* W3,
                                    const float* logit_offset, float* logits, cudaStream_t s) {
   if (T == 0) return MOE_OK;
   if (d < BK || d % 8 != 0 || E % 4 != 0) return MOE_ERR_UNSUPPORTED;
   const int nt = (E + 63) / 64;
+  const bool pair = use_pairs(T, 1);
   CUtensorMap ma, mb;
   if (!make_map(&ma, x, (unsigned long long)T, d, BM)) return MOE_ERR_UNSUPPORTED;
-  if (!make_map(&mb, W3, (unsigned long long)nt * 256, d, BN)) return MOE_ERR_UNSUPPORTED;
+  if (!make_map(&mb, W3, (unsigned long long)nt * 256, d, pair ? BM : BN)) return MOE_ERR_UNSUPPORTED;
+  if (pair) return launch_tc2<2, float>(ma, mb, offs2, 1, d, E, 0, T, logit_offset, logits, s);
   return launch_tc<2, float>(ma, mb, offs2, 1, d, E, 0, T, logit_offset, logits, s);
 }
 
@@ -503,6 +779,8 @@ moe_status launch_gate_up_tc(const void* x_rows, const int32_t* offsets, int E, 
   CUtensorMap ma, mb;
   if (!make_map(&ma, x_rows, (unsigned long long)rows_max, d, BM)) return MOE_ERR_UNSUPPORTED;
   if (!make_map(&mb, W_gu, (unsigned long long)E * 2 * F, d, 128)) return MOE_ERR_UNSUPPORTED;
+  if (use_pairs(rows_max, E))
+    return launch_tc2<0, __nv_bfloat16>(ma, mb, offsets, E, d, F, F, rows_max, nullptr, h, s);
   return launch_tc<0, __nv_bfloat16>(ma, mb, offsets, E, d, F, F, rows_max, nullptr, h, s);
 }
 
@@ -510,9 +788,15 @@ moe_status launch_down_tc(const void* h, const int32_t* offsets, int E, int d, i
                           const void* W_dn, const float* gate_of_row, int y_dtype, void* y_rows, cudaStream_t s) {
   if (rows_max == 0) return MOE_OK;
   if (F < BK || d < 8) return MOE_ERR_UNSUPPORTED;
+  const bool pair = use_pairs(rows_max, E);
   CUtensorMap ma, mb;
   if (!make_map(&ma, h, (unsigned long long)rows_max, F, BM)) return MOE_ERR_UNSUPPORTED;
-  if (!make_map(&mb, W_dn, (unsigned long long)E * d, F, BN)) return MOE_ERR_UNSUPPORTED;
+  if (!make_map(&mb, W_dn, (unsigned long long)E * d, F, pair ? BM : BN)) return MOE_ERR_UNSUPPORTED;
+  if (pair) {
+    if (y_dtype == MOE_F32)
+      return launch_tc2<1, float>(ma, mb, offsets, E, F, d, F, rows_max, gate_of_row, y_rows, s);
+    return launch_tc2<1, __nv_bfloat16>(ma, mb, offsets, E, F, d, F, rows_max, gate_of_row, y_rows, s);
+  }
   if (y_dtype == MOE_F32) return launch_tc<1, float>(ma, mb, offsets, E, F, d, F, rows_max, gate_of_row, y_rows, s);
   return launch_tc<1, __nv_bfloat16>(ma, mb, offsets, E, F, d, F, rows_max, gate_of_row, y_rows, s);
 }
