@@ -296,10 +296,49 @@ topk_kernel(const float* __restrict__ partial, int nsplit, long long split_strid
       }
       return b;
     };
-    Cand mine = local_best();
     int sel_idx = 0;
     float sel_logit = 0.f;
-    for (int j = 0; j < k; ++j) {
+    if constexpr (!BIAS) {
+      // One 64-bit key per candidate: order-preserving bits of the logit above the
+      // bit-inverted expert index, so an unsigned max picks the larger logit and, on
+      // equal logits, the lower index.  0 marks an empty or already-taken slot (no finite
+      // or infinite float maps to 0).
+      uint64_t key[EPL];
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) {
+        const int e = lane + 32 * i;
+        const uint32_t u = __float_as_uint(kf[i] + 0.0f);     // -0 and +0 compare equal as floats
+        const uint32_t ord = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+        key[i] = e < E ? ((uint64_t)ord << 32) | (uint32_t)(~(uint32_t)e) : 0ull;
+      }
+      uint64_t best = 0;
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) best = key[i] > best ? key[i] : best;
+      for (int j = 0; j < k; ++j) {
+        uint64_t w = best;
+#pragma unroll
+        for (int o = 16; o; o >>= 1) {
+          const uint64_t c = __shfl_xor_sync(0xffffffffu, w, o);
+          w = c > w ? c : w;
+        }
+        const int e = (int)(~(uint32_t)w);
+        if (lane == (unsigned)j) {
+          const uint32_t ord = (uint32_t)(w >> 32);
+          sel_idx = e;
+          sel_logit = __uint_as_float((ord & 0x80000000u) ? (ord & 0x7fffffffu) : ~ord);
+        }
+        if ((unsigned)(e & 31) == lane) {          // the owner drops it and refreshes its best
+          best = 0;
+#pragma unroll
+          for (int i = 0; i < EPL; ++i) {
+            if (i == (e >> 5)) key[i] = 0ull;
+            best = key[i] > best ? key[i] : best;
+          }
+        }
+      }
+    }
+    Cand mine = local_best();
+    for (int j = 0; BIAS && j < k; ++j) {
       Cand w = mine;
 #pragma unroll
       for (int o = 16; o; o >>= 1) {

@@ -13,7 +13,8 @@
 // per-expert load ratio and the drop rate.
 //
 // Deterministic: stage 1 reduces each CTA's tokens into per-CTA partials in a fixed
-// order (fp64); stage 2 sums the partials in CTA order.
+// order (fp64); stage 2 sums the partials in a fixed lane-strided order followed by a
+// fixed butterfly, so the result does not depend on scheduling.
 #include "common.cuh"
 
 namespace moe {
@@ -99,80 +100,89 @@ stats_partial_kernel(const float* __restrict__ logits, int T, int E, int score, 
   }
 }
 
-__device__ double block_sum_d(double v, double* sh) {
-  const unsigned lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
-  v = warp_sum_dd(v);
-  __syncthreads();
-  if (lane == 0) sh[warp] = v;
-  __syncthreads();
-  double r = 0.0;
-  const int nw = (blockDim.x + 31) >> 5;
-  for (int w = 0; w < nw; ++w) r += sh[w];
-  return r;
-}
-
+// Stage 2: one CTA of 1024 threads.  P_e: one warp per expert, lanes take the partials
+// in a fixed strided order (8 loads in flight), then a fixed butterfly.  The four
+// per-expert sums (aux, kept, variance, max) are reduced together in one pass.
 __global__ void __launch_bounds__(1024)
 stats_final_kernel(const double* __restrict__ partP, const double* __restrict__ partZ, int nparts,
                    const int32_t* __restrict__ counts, const int32_t* __restrict__ kept, int T, int E,
                    int k, float* __restrict__ load, float* __restrict__ stats5) {
-  __shared__ double sh[32];
   __shared__ double Ps[1024];
-  const double TK = (double)T * k;
-  const double mean = TK / E;
-  // P_e: one warp per expert, lanes take the partials in a fixed strided order, then a
-  // fixed butterfly -- many loads in flight, same result every run
-  {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-    for (int e = warp; e < E; e += nw) {
-      double p = 0.0;
-      for (int b = lane; b < nparts; b += 32) p += partP[(long long)b * E + e];
+  __shared__ double red[4][32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  for (int e = warp; e < E; e += nw) {
+    double p = 0.0;
+    int b = lane;
+    for (; b + 32 * 7 < nparts; b += 32 * 8) {
+      double v[8];
 #pragma unroll
-      for (int o = 16; o; o >>= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
-      if (lane == 0) Ps[e] = p;
+      for (int u = 0; u < 8; ++u) v[u] = __ldg(partP + (long long)(b + 32 * u) * E + e);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) p += v[u];
     }
-    __syncthreads();
-  }
-  double aux = 0.0, kept_sum = 0.0, var = 0.0, cmax = 0.0;
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    const double P = Ps[e] / (double)T;
-    const double c = (double)counts[e];
-    const double f = c / TK;
-    load[e] = (float)f;
-    aux += f * P;
-    kept_sum += (double)kept[e];
-    var += (c - mean) * (c - mean);
-    cmax = fmax(cmax, c);
-  }
-  aux = block_sum_d(aux, sh);
-  kept_sum = block_sum_d(kept_sum, sh);
-  var = block_sum_d(var, sh);
-  // block max
-  {
-    double v = cmax;
+    for (; b < nparts; b += 32) p += __ldg(partP + (long long)b * E + e);
 #pragma unroll
-    for (int o = 16; o; o >>= 1) v = fmax(v, __shfl_xor_sync(0xffffffffu, v, o));
-    __syncthreads();
-    if ((threadIdx.x & 31) == 0) sh[threadIdx.x >> 5] = v;
-    __syncthreads();
-    double r = 0.0;
-    for (int w = 0; w < (int)((blockDim.x + 31) >> 5); ++w) r = fmax(r, sh[w]);
-    cmax = r;
+    for (int o = 16; o; o >>= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
+    if (lane == 0) Ps[e] = p;
   }
   double z = 0.0;
-  if (threadIdx.x < 32) {
-    for (int b = threadIdx.x; b < nparts; b += 32) z += partZ[b];
+  if (warp == nw - 1) {                       // the z partials, on the last warp
+    int b = lane;
+    for (; b + 32 * 7 < nparts; b += 32 * 8) {
+      double v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = __ldg(partZ + b + 32 * u);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) z += v[u];
+    }
+    for (; b < nparts; b += 32) z += __ldg(partZ + b);
 #pragma unroll
     for (int o = 16; o; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
   }
-  if (threadIdx.x == 0) {
-    stats5[0] = (float)(E * aux);
-    stats5[1] = (float)(z / (double)T);
-    stats5[2] = (float)(TK - kept_sum);
-    stats5[3] = (float)(cmax / mean);
-    stats5[4] = (float)(sqrt(var / E) / mean);
+  __syncthreads();
+  const double TK = (double)T * k;
+  const double mean = TK / E;
+  double s[4] = {0.0, 0.0, 0.0, 0.0};          // aux, kept, variance, max count
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const double c = (double)counts[e];
+    const double f = c / TK;
+    load[e] = (float)f;
+    s[0] += f * (Ps[e] / (double)T);
+    s[1] += (double)kept[e];
+    s[2] += (c - mean) * (c - mean);
+    s[3] = fmax(s[3], c);
   }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+#pragma unroll
+    for (int q = 0; q < 3; ++q) s[q] += __shfl_xor_sync(0xffffffffu, s[q], o);
+    s[3] = fmax(s[3], __shfl_xor_sync(0xffffffffu, s[3], o));
+  }
+  if (lane == 0) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) red[q][warp] = s[q];
+  }
+  __syncthreads();
+  if (warp == 0) {
+    double t[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) t[q] = lane < nw ? red[q][lane] : 0.0;
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+#pragma unroll
+      for (int q = 0; q < 3; ++q) t[q] += __shfl_xor_sync(0xffffffffu, t[q], o);
+      t[3] = fmax(t[3], __shfl_xor_sync(0xffffffffu, t[3], o));
+    }
+    if (lane == 0) {
+      stats5[0] = (float)(E * t[0]);
+      stats5[2] = (float)(TK - t[1]);
+      stats5[3] = (float)(t[3] / mean);
+      stats5[4] = (float)(sqrt(t[2] / E) / mean);
+    }
+  }
+  if (warp == nw - 1 && lane == 0) stats5[1] = (float)(z / (double)T);
 }
+
 
 int stats_parts(int T) {
   const int want = 2 * num_sms();
