@@ -98,9 +98,10 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
-def layer_roofline_ms(cfg, A, pk, rb=4, ob=4):
+def layer_roofline_ms(cfg, A, pk, rb=4, ob=4, fused=False):
     """Sum over steps of max(compute, memory) time at the measured peaks (algorithmic bytes / flops).
-    rb / ob: bytes per element of the gated rows / of the layer output."""
+    rb / ob: bytes per element of the gated rows / of the layer output.  fused: the combine runs
+    inside the down GEMM, whose algorithmic bytes are then H, W_dn and y (zero fill + result)."""
     T, d, E, k, F = cfg.T, cfg.d, cfg.E, cfg.k, cfg.F
     hbm = pk["hbm_gbs"] * 1e9
     tc = pk["bf16_tflops"] * 1e12
@@ -111,10 +112,16 @@ def layer_roofline_ms(cfg, A, pk, rb=4, ob=4):
         "histogram_scan": (T * k * 4 * 3 + A * 8) / hbm,
         "permute": (T * d * b + A * d * b) / hbm,
         "gate_up": max(4 * A * d * F / tc, (A * d * b + E * 2 * F * d * b + A * F * b) / hbm),
-        "down": max(2 * A * F * d / tc, (A * F * b + E * d * F * b + A * d * rb) / hbm),
-        "combine": (A * d * rb + T * d * ob) / hbm,
         "stats": (T * E * 4) / hbm,
     }
+    if fused:
+        steps["down_combine"] = max(2 * A * F * d / tc, (A * F * b + E * d * F * b + 2 * T * d * 4) / hbm)
+    else:
+        steps["down"] = max(2 * A * F * d / tc, (A * F * b + E * d * F * b + A * d * rb) / hbm)
+        steps["combine"] = (A * d * rb + T * d * ob) / hbm
+    if cfg.F_s:
+        Fs = cfg.F_s
+        steps["shared"] = max(6 * T * d * Fs / tc, (T * d * b + 3 * d * Fs * b + T * Fs * b + T * d * rb) / hbm)
     return sum(steps.values()) * 1e3, {k_: v * 1e3 for k_, v in steps.items()}
 
 
@@ -148,84 +155,94 @@ def run_ours(args):
                    W_dn_s=None if sh is None else torch.from_numpy(sh[1]).to(dt).unsqueeze(0).to(dev))
     del W_gu, W_dn
     cap = M.moe_capacity(cfg.T, cfg.E, cfg.k, cfg.capacity_factor, True)
-    layer = MoELayer(w, cfg.k, cfg.T, cfg.score, cfg.renormalize, cfg.scale, cap)
     x = torch.from_numpy(x_np).to(dt).to(dev)
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
 
-    stage_names = ["route", "histogram_scan", "permute", "gate_up", "down", "shared", "combine", "stats"]
+    def make_layer(mode):
+        return MoELayer(w, cfg.k, cfg.T, cfg.score, cfg.renormalize, cfg.scale, cap, combine=mode)
 
-    def step(s, evs=None):
-        """One layer forward on stream s; evs: 9 timing events recorded between the stages."""
-        T = cfg.T
-        rec = (lambda i: evs[i].record(s)) if evs is not None else (lambda i: None)
-        rec(0)
-        layer.route(x, s)
-        rec(1)
-        layer.histogram_scan(T, s)
-        rec(2)
-        layer.permute(x, s)
-        rec(3)
-        layer.gate_up(s)
-        rec(4)
-        layer.down(s)
-        rec(5)
-        if layer.has_shared:
-            layer.shared(x, s)
-        rec(6)
-        layer.combine(T, s)
-        rec(7)
-        layer.stats(T, s)
-        rec(8)
+    def time_layer(layer, steps, clocks=None):
+        """Warm-up, then `steps` replays of one forward captured as a CUDA graph whose timing
+        events are nodes inside the graph, on the stream the kernels run on.  L2 is flushed
+        (256 MB write) before every step, outside the timed span.  Returns per-step ms,
+        mean ms per stage, the rows processed and the clock record."""
+        stages = layer.stages(x)
+        names = [n for n, _ in stages]
 
-    for _ in range(args.warmup):
-        flush.zero_()
-        step(stream)
-    torch.cuda.synchronize()
-    assert M.moe_get_device_error() == 0
-    A = int(layer.offsets[-1].item())
+        def step(s, evs=None):
+            for i, (_, fn) in enumerate(stages):
+                if evs is not None:
+                    evs[i].record(s)
+                fn(s)
+            if evs is not None:
+                evs[len(stages)].record(s)
 
-    # The step runs as one CUDA graph (no host work between the library's launches); the
-    # timing events are nodes inside the graph, on the stream the kernels run on.
-    evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(9)]
-    graph = torch.cuda.CUDAGraph()
-    cap_stream = torch.cuda.Stream()
-    cap_stream.wait_stream(stream)
-    with torch.cuda.stream(cap_stream):
-        with torch.cuda.graph(graph, stream=cap_stream):
-            step(cap_stream, evs)
-    stream.wait_stream(cap_stream)
-    for _ in range(3):
-        flush.zero_()
-        graph.replay()
-    torch.cuda.synchronize()
-    assert M.moe_get_device_error() == 0
+        for _ in range(args.warmup):
+            flush.zero_()
+            step(stream)
+        torch.cuda.synchronize()
+        assert M.moe_get_device_error() == 0
+        rows = int(layer.offsets[-1].item())
+        evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(stages) + 1)]
+        graph = torch.cuda.CUDAGraph()
+        cap_stream = torch.cuda.Stream()
+        cap_stream.wait_stream(stream)
+        with torch.cuda.stream(cap_stream):
+            with torch.cuda.graph(graph, stream=cap_stream):
+                step(cap_stream, evs)
+        stream.wait_stream(cap_stream)
+        for _ in range(3):
+            flush.zero_()
+            graph.replay()
+        torch.cuda.synchronize()
+        assert M.moe_get_device_error() == 0
+        if clocks is not None:
+            clocks.start()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        per_step = np.zeros(steps)
+        acc = np.zeros(len(stages))
+        for i in range(steps):
+            flush.zero_()                      # L2 flush outside the step
+            graph.replay()
+            torch.cuda.synchronize()           # read this step's in-graph events
+            per_step[i] = evs[0].elapsed_time(evs[-1])
+            acc += [evs[j].elapsed_time(evs[j + 1]) for j in range(len(stages))]
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        clk = clocks.stop() if clocks is not None else None
+        assert M.moe_get_device_error() == 0
+        del graph
+        return per_step, {n: float(acc[j] / steps) for j, n in enumerate(names)}, rows, clk
 
-    clocks = ClockSampler(local_rank)
-    clocks.start()
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    per_step = np.zeros(args.steps)
-    stage_acc = np.zeros(len(stage_names))
-    for i in range(args.steps):
-        flush.zero_()                      # L2 flush outside the step
-        graph.replay()
-        torch.cuda.synchronize()           # read this step's in-graph events
-        per_step[i] = evs[0].elapsed_time(evs[8])
-        stage_acc += [evs[j].elapsed_time(evs[j + 1]) for j in range(len(stage_names))]
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    clk = clocks.stop()
-    stage_ms = {n: float(stage_acc[j] / args.steps) for j, n in enumerate(stage_names)}
-    total_ms = float(per_step.sum())
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    def max_over_ranks(v):
+        if world > 1:
+            t = torch.tensor([v], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            v = float(t.item())
+        return v
+
+    layer = make_layer(args.combine)
+    per_step, stage_ms, A, clk = time_layer(layer, args.steps, ClockSampler(local_rank))
+    total_ms = max_over_ranks(float(per_step.sum()))
     ms_per_step = total_ms / args.steps
     value = cfg.T * world * args.steps / (total_ms / 1e3)
+
+    other = None
+    if args.combine == "fused" and args.rows_steps > 0:
+        # the bitwise-reproducible form (gated rows + ordered combine), same inputs
+        rl = make_layer("rows")
+        ps, sm, _, _ = time_layer(rl, args.rows_steps)
+        t = max_over_ranks(float(ps.sum()))
+        other = {"combine": "rows (gated rows + ordered combine, bitwise reproducible)",
+                 "ms_per_step": round(t / args.rows_steps, 4),
+                 "value": round(cfg.T * world * args.rows_steps / (t / 1e3), 1), "steps": args.rows_steps,
+                 "stages_ms": {k_: round(v, 4) for k_, v in sm.items()}}
+        del rl
+        torch.cuda.empty_cache()
 
     # end to end through the public API with host buffers (pinned), copies inside the timing
     x_host = torch.from_numpy(x_np).to(dt).pin_memory()
@@ -248,11 +265,7 @@ def run_ours(args):
         y_host.copy_(layer.y, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
     e2e_value = cfg.T * world * e2e_steps / (e2e_ms / 1e3)
     h2d_bytes = x_host.numel() * x_host.element_size()
     d2h_bytes = y_host.numel() * y_host.element_size()
@@ -262,9 +275,18 @@ def run_ours(args):
     flops = 4.0 * A * cfg.d * cfg.F
     achieved = flops / (gate_up_ms * 1e-3) / 1e12
     peak = pk["bf16_tflops"]
-    rb, ob = layer.y_perm.element_size(), layer.y.element_size()
-    roof_ms, roof_steps = layer_roofline_ms(cfg, A, pk, rb, ob)
+    fused = args.combine == "fused"
+    rb = 4 if fused else layer.y_perm.element_size()
+    ob = layer.y.element_size()
+    roof_ms, roof_steps = layer_roofline_ms(cfg, A, pk, rb, ob, fused)
     traffic = GATE_UP_TRAFFIC.get(args.workload)
+    down_ms = stage_ms["down_combine" if fused else "down"]
+    thr = {"down_tflops": round(2.0 * A * cfg.F * cfg.d / (down_ms * 1e-3) / 1e12, 1),
+           "permute_gbs": round((cfg.T * cfg.d * 2 + A * cfg.d * 2) / (stage_ms["permute"] * 1e-3) / 1e9, 1),
+           "route_gbs": round((cfg.T * cfg.d * 2 + cfg.T * cfg.E * 8 + cfg.T * cfg.k * 8) /
+                              (stage_ms["route"] * 1e-3) / 1e9, 1)}
+    if not fused:
+        thr["combine_gbs"] = round((A * cfg.d * rb + cfg.T * cfg.d * ob) / (stage_ms["combine"] * 1e-3) / 1e9, 1)
 
     out = None
     if rank == 0:
@@ -276,6 +298,8 @@ def run_ours(args):
             "data": "synthetic (seeded; integer-grid router inputs, N(0,0.02) bf16 expert weights)",
             "config": {"workload": args.workload, "T": cfg.T, "d": cfg.d, "E": cfg.E, "k": cfg.k, "F": cfg.F,
                        "F_shared": cfg.F_s, "score": cfg.score, "capacity": cap, "rows": A,
+                       "combine": ("fused into the down GEMM (fp32 atomics into y)" if fused
+                                   else "gated rows + ordered combine"),
                        "parallelism": f"replicas x{world} (independent token batches, no collective)",
                        "l2": "flushed before every step (256 MB write)"},
             "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d_bytes,
@@ -289,13 +313,8 @@ def run_ours(args):
                                "tokens_per_s": round(cfg.T / (roof_ms / 1e3), 1)},
             "stages_ms": {k_: round(v, 4) for k_, v in stage_ms.items()},
             "stage_roofline_ms": {k_: round(v, 4) for k_, v in roof_steps.items()},
-            "stage_throughput": {
-                "down_tflops": round(2.0 * A * cfg.F * cfg.d / (stage_ms["down"] * 1e-3) / 1e12, 1),
-                "permute_gbs": round((cfg.T * cfg.d * 2 + A * cfg.d * 2) / (stage_ms["permute"] * 1e-3) / 1e9, 1),
-                "combine_gbs": round((A * cfg.d * rb + cfg.T * cfg.d * ob) / (stage_ms["combine"] * 1e-3) / 1e9, 1),
-                "route_gbs": round((cfg.T * cfg.d * 2 + cfg.T * cfg.E * 8 + cfg.T * cfg.k * 8) /
-                                   (stage_ms["route"] * 1e-3) / 1e9, 1),
-            },
+            "stage_throughput": thr,
+            "rows_variant": other,
             "clocks": clk,
             "cpu_baseline": cpu,
         }
@@ -410,6 +429,10 @@ def main():
     ap.add_argument("--tokens", type=int, default=None,
                     help="override T (smaller cases of the same kernels, e.g. for profiler captures)")
     ap.add_argument("--e2e-steps", type=int, default=50, help="steps timed through host buffers")
+    ap.add_argument("--combine", choices=["fused", "rows"], default="fused",
+                    help="fused: combine inside the down GEMM; rows: gated rows + ordered combine")
+    ap.add_argument("--rows-steps", type=int, default=100,
+                    help="with --combine fused, also time the rows form for this many steps (0 = skip)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -13,6 +13,7 @@
  *   moe_expert_down      grouped GEMM  Y = gate_of_row * (H Wd^T)       (per expert)
  *   moe_grouped_ffn      the two GEMMs above back to back
  *   moe_combine          gate-weighted sum of each token's rows (+ shared expert)
+ *   moe_expert_down_combine  the down GEMM with the combine fused into its epilogue
  *   moe_router_stats     per-expert load, aux loss, z-loss, drops, imbalance
  *
  * Sources (web pages on Mixture-of-Experts, cited by title and section):
@@ -51,7 +52,9 @@
  *     gated expert rows and the layer output are written in the dtype the caller picks
  *     (fp32 keeps H as the only rounding inside the layer; bf16 rounds each row and the
  *     output once more).  The combine sums in fp32 in slot order j = 0..k-1, then adds
- *     the shared expert, then converts to the output dtype.
+ *     the shared expert, then converts to the output dtype.  moe_expert_down_combine
+ *     adds the same fp32 terms in the order its tiles finish instead (not bitwise
+ *     reproducible; each result is within fp32 rounding of the ordered sum).
  */
 #ifndef MOE_B200_H
 #define MOE_B200_H
@@ -236,6 +239,29 @@ MOE_API moe_status moe_grouped_ffn(const void* x_rows, int32_t dtype, const int3
                            int32_t E, int32_t d, int32_t F, int64_t rows_max,
                            const void* W_gu, const void* W_dn, const float* gate_of_row,
                            void* h, int32_t y_dtype, void* y_rows, void* stream);
+
+/* ------------------------------------------------------------------------------------
+ * moe_expert_down_combine -- the down projection with the combine fused into it:
+ *     y[token_of_row[r]] += gate_of_row[r] * (H[r] W_dn[e]^T)   for every kept row r.
+ * The same sum as moe_expert_down followed by moe_combine ([Handbook-News] "MoE 到底
+ * 省了什么": gather the experts' results back per token), without writing the gated
+ * rows to memory.
+ *   h, offsets, W_dn, gate_of_row: as moe_expert_down (gate_of_row NULL = weight 1)
+ *   token_of_row (device) [rows_max] int32 from moe_histogram_scan
+ *   T        rows of y;   y (device) [T, d] fp32, 16-byte aligned
+ *   accumulate 0: y is zeroed first (cudaMemsetAsync on stream);
+ *              1: rows are added onto y's contents (e.g. a shared expert's output
+ *                 written there by moe_expert_down with E = 1 and y_dtype MOE_F32).
+ * Each token's terms are added with fp32 atomics in the order the tiles finish, so y
+ * is not bitwise reproducible from run to run (each result is within fp32 rounding of
+ * the ordered sum); moe_combine is the reproducible form.  A token index outside
+ * [0, T) is skipped and recorded as MOE_DEVERR_ROW.
+ * ---------------------------------------------------------------------------------- */
+MOE_API moe_status moe_expert_down_combine(const void* h, int32_t dtype, const int32_t* offsets,
+                           int32_t E, int32_t d, int32_t F, int64_t rows_max,
+                           const void* W_dn, const float* gate_of_row,
+                           const int32_t* token_of_row, int32_t T, int32_t accumulate,
+                           float* y, void* stream);
 
 /* ------------------------------------------------------------------------------------
  * moe_combine -- y[t] = sum_j g_j * y_rows[row_of[t, j]]  (+ shared_y[t]).

@@ -207,6 +207,29 @@ moe_status moe_grouped_ffn(const void* x_rows, int32_t dtype, const int32_t* off
   return moe_expert_down(h, dtype, offsets, E, d, F, rows_max, W_dn, gate_of_row, y_dtype, y_rows, stream);
 }
 
+moe_status moe_expert_down_combine(const void* h, int32_t dtype, const int32_t* offsets, int32_t E, int32_t d,
+                                   int32_t F, int64_t rows_max, const void* W_dn, const float* gate_of_row,
+                                   const int32_t* token_of_row, int32_t T, int32_t accumulate, float* y,
+                                   void* stream) {
+  if (T < 0 || (accumulate != 0 && accumulate != 1)) return MOE_ERR_INVALID_ARG;
+  if ((long long)T >= kMaxT) return MOE_ERR_UNSUPPORTED;
+  moe_status st = check_ffn(h, dtype, offsets, E, d, F, rows_max, W_dn, y);
+  if (st != MOE_OK) return st;
+  if (T == 0) return MOE_OK;
+  if (!y || (rows_max > 0 && !token_of_row)) return MOE_ERR_INVALID_ARG;
+  if (!accumulate) {
+    st = cuda_status(cudaMemsetAsync(y, 0, (size_t)T * (size_t)d * sizeof(float), S(stream)));
+    if (st != MOE_OK) return st;
+  }
+  if (rows_max == 0) return MOE_OK;
+  if (dtype == MOE_BF16) {
+    st = launch_down_combine_tc(h, offsets, E, d, F, rows_max, W_dn, gate_of_row, token_of_row, T, y, S(stream));
+    if (st != MOE_ERR_UNSUPPORTED) return st;
+  }
+  return launch_down_combine_simt(h, dtype, offsets, E, d, F, rows_max, W_dn, gate_of_row, token_of_row, T, y,
+                                  S(stream));
+}
+
 moe_status moe_combine(const void* y_rows, int32_t rows_dtype, const int32_t* row_of, const float* topk_gate,
                        const void* shared_y, int32_t T, int32_t d, int32_t k, int64_t rows_max, int32_t y_dtype,
                        void* y, void* stream) {

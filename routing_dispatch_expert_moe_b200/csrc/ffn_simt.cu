@@ -6,6 +6,7 @@
 // 0..F-1 and W_up in rows F..2F-1; W_dn[e] is [d, F].
 //   gate_up: H[r, f] = silu(sum_c X[r,c] Wg[f,c]) * (sum_c X[r,c] Wu[f,c])
 //   down:    Y[r, n] = gate_of_row[r] * sum_f H[r,f] Wd[n,f]
+//   down + combine: y[token_of_row[r], n] += gate_of_row[r] * sum_f H[r,f] Wd[n,f]  (fp32 atomics)
 // Expert FFN: "Mixture of Experts Explained" (zh), section "什么是混合专家模型" (each
 // expert is an FFN); SwiGLU form silu(x Wg^T) * (x Wu^T) Wd^T without biases.
 //
@@ -39,13 +40,14 @@ __device__ __forceinline__ void st_elem<__nv_bfloat16>(__nv_bfloat16* p, float v
 
 // MODE 0: gate_up (A = x_rows [*, d], B = W_gu [E][2F][d], out = H [*, F])
 // MODE 1: down    (A = H [*, F], B = W_dn [E][d][F], out = Y [*, d], scaled by gate_of_row)
+// MODE 2: down + combine (as MODE 1, out = y [T, d] fp32, rows added into their token's row)
 // OT: output element type (MODE 0 writes H in the activation dtype; MODE 1 writes the
 // gated rows in the caller's choice of bf16 or fp32).
 template <typename DT, int MODE, typename OT>
 __global__ void __launch_bounds__(kThreads)
 grouped_simt_kernel(const DT* __restrict__ A, const DT* __restrict__ B, const int32_t* __restrict__ offsets,
                     int E, int K, int N, int F, long long rows_max, const float* __restrict__ gate_of_row,
-                    OT* __restrict__ out, int* err) {
+                    OT* __restrict__ out, const int32_t* __restrict__ token_of_row, int n_tokens, int* err) {
   __shared__ int tile_start[kMaxE + 1];
   __shared__ int sh32[32];
   __shared__ __align__(16) float As[kBK][kBM + 4];
@@ -112,7 +114,15 @@ grouped_simt_kernel(const DT* __restrict__ A, const DT* __restrict__ B, const in
       const int r = ty * 4 + i;
       if (r >= tc.rows) continue;
       const long long row = tc.row0 + r;
-      const float gsc = (MODE == 1 && gate_of_row) ? __ldg(gate_of_row + row) : 1.f;
+      const float gsc = (MODE != 0 && gate_of_row) ? __ldg(gate_of_row + row) : 1.f;
+      int tok = 0;
+      if (MODE == 2) {
+        tok = __ldg(token_of_row + row);
+        if ((unsigned)tok >= (unsigned)n_tokens) {
+          record_error(err, MOE_DEVERR_ROW);
+          continue;
+        }
+      }
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int n = n0 + tx * 4 + j;
@@ -124,7 +134,8 @@ grouped_simt_kernel(const DT* __restrict__ A, const DT* __restrict__ B, const in
         } else {
           v = acc[i][j] * gsc;
         }
-        st_elem<OT>(out + row * N + n, v);
+        if (MODE == 2) atomicAdd(reinterpret_cast<float*>(out) + (long long)tok * N + n, v);
+        else st_elem<OT>(out + row * N + n, v);
       }
     }
   }
@@ -132,11 +143,12 @@ grouped_simt_kernel(const DT* __restrict__ A, const DT* __restrict__ B, const in
 
 template <typename DT, int MODE, typename OT>
 moe_status run_simt(const void* A, const void* B, const int32_t* offsets, int E, int K, int N, int F,
-                    long long rows_max, const float* gate_of_row, void* out, cudaStream_t s) {
+                    long long rows_max, const float* gate_of_row, void* out, cudaStream_t s,
+                    const int32_t* token_of_row = nullptr, int n_tokens = 0) {
   const int grid = 2 * num_sms();
   grouped_simt_kernel<DT, MODE, OT><<<grid, kThreads, 0, s>>>(
       static_cast<const DT*>(A), static_cast<const DT*>(B), offsets, E, K, N, F, rows_max, gate_of_row,
-      static_cast<OT*>(out), err_ptr());
+      static_cast<OT*>(out), token_of_row, n_tokens, err_ptr());
   return check_launch();
 }
 
@@ -161,6 +173,16 @@ moe_status launch_down_simt(const void* h, int dtype, const int32_t* offsets, in
   return f32out ? run_simt<__nv_bfloat16, 1, float>(h, W_dn, offsets, E, F, d, F, rows_max, gate_of_row, y_rows, s)
                 : run_simt<__nv_bfloat16, 1, __nv_bfloat16>(h, W_dn, offsets, E, F, d, F, rows_max, gate_of_row,
                                                             y_rows, s);
+}
+
+moe_status launch_down_combine_simt(const void* h, int dtype, const int32_t* offsets, int E, int d, int F,
+                                    long long rows_max, const void* W_dn, const float* gate_of_row,
+                                    const int32_t* token_of_row, int T, float* y, cudaStream_t s) {
+  if (rows_max == 0 || T == 0) return MOE_OK;
+  if (dtype == MOE_F32)
+    return run_simt<float, 2, float>(h, W_dn, offsets, E, F, d, F, rows_max, gate_of_row, y, s, token_of_row, T);
+  return run_simt<__nv_bfloat16, 2, float>(h, W_dn, offsets, E, F, d, F, rows_max, gate_of_row, y, s, token_of_row,
+                                          T);
 }
 
 }  // namespace moe

@@ -11,7 +11,12 @@
 //       128x256 accumulator carries g (columns 0..127) and u (128..255) for the same
 //       128 features; the epilogue writes H = silu(g) * u as bf16.
 //   MODE 1 (down): A = H [rows, F], B = W_dn[e] ([d, F]); the epilogue scales each row
-//       by gate_of_row and writes bf16.
+//       by gate_of_row and writes bf16 or fp32 rows.
+//   MODE 3 (down + combine): as MODE 1, but the gated row is added into the fp32 output
+//       row of its token (y[token_of_row[r]] += ...) with 16-byte vector atomics, so the
+//       gated rows never reach memory and no separate combine pass runs.  The fp32 sum
+//       order over a token's experts is whatever order the tiles finish in.
+//   MODE 2 (router logits on the tensor cores, see below).
 //
 // Per CTA (1 per SM, 192 threads):
 //   warp 0   TMA producer: 128x64 A tile + 256x64 B tile per stage (128-byte swizzle),
@@ -266,8 +271,29 @@ __device__ __forceinline__ void stage_store32(uint8_t* stage, const float (&v)[3
   __syncwarp();
 }
 
+// MODE 3: the same turn-around, then each 16-byte piece is added into the output row of
+// its token (tok: this lane's row's token, -1 = skip).  Every atomic instruction of the
+// warp covers 4 rows x 128 contiguous bytes.
+__device__ __forceinline__ void stage_red32(uint8_t* stage, const float (&v)[32], int lane, float* y, int tok,
+                                            long long ld, int col, int ncols) {
+  float4* dst = reinterpret_cast<float4*>(stage + lane * kStagePitchF32);
+#pragma unroll
+  for (int q = 0; q < 8; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+  __syncwarp();
+  const int rs = lane >> 3, cv = lane & 7;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int r = i * 4 + rs;
+    const int t = __shfl_sync(0xffffffffu, tok, r);
+    const float4 x = *reinterpret_cast<const float4*>(stage + r * kStagePitchF32 + cv * 16);
+    if (t >= 0 && col + cv * 4 + 4 <= ncols)
+      atomicAdd(reinterpret_cast<float4*>(y + (long long)t * ld + col + cv * 4), x);
+  }
+  __syncwarp();
+}
+
 // OutT: element type of the output rows (MODE 0 always writes bf16 H; MODE 1 writes
-// bf16 or fp32 gated rows).
+// bf16 or fp32 gated rows; MODE 3 adds into fp32 token rows).
 // One tile's epilogue for one warp: its 32 accumulator rows (TMEM lanes at taddr) become
 // output rows wrow0 .. wrow0 + wrows - 1.  The whole warp must call it (tcgen05.ld is
 // .sync.aligned); rows past wrows are read but not stored.
@@ -278,8 +304,31 @@ __device__ __forceinline__ void stage_store32(uint8_t* stage, const float (&v)[3
 template <int MODE, typename OutT>
 __device__ __forceinline__ void epilogue_tile(uint32_t taddr, uint8_t* stage, int lane, long long wrow0, int wrows,
                                               int n_tile, int F, int N_out, const float* __restrict__ gate_of_row,
-                                              OutT* __restrict__ out) {
-  if constexpr (MODE == 0) {
+                                              OutT* __restrict__ out, const int32_t* __restrict__ token_of_row,
+                                              int n_tokens, int* err) {
+  if constexpr (MODE == 3) {
+    const int n0 = n_tile * BN;
+    const float gs = (lane < wrows && gate_of_row) ? __ldg(gate_of_row + wrow0 + lane) : 1.f;
+    int tok = -1;
+    if (lane < wrows) {
+      tok = __ldg(token_of_row + wrow0 + lane);
+      if ((unsigned)tok >= (unsigned)n_tokens) {
+        record_error(err, MOE_DEVERR_ROW);
+        tok = -1;
+      }
+    }
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+      uint32_t v32[32];
+      tmem_ld32(taddr + c * 32, v32);
+      tmem_wait_ld();
+      tmem_regs_ready(v32);
+      float y[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) y[i] = __uint_as_float(v32[i]) * gs;
+      stage_red32(stage, y, lane, reinterpret_cast<float*>(out), tok, N_out, n0 + c * 32, N_out);
+    }
+  } else if constexpr (MODE == 0) {
     const int f0 = n_tile * 128;
 #pragma unroll 1
     for (int c = 0; c < 4; ++c) {
@@ -340,7 +389,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
 grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                        const int32_t* __restrict__ offsets, int E, int K, int N_out, int F,
                        long long rows_max, const float* __restrict__ gate_of_row,
-                       OutT* __restrict__ out, int* err) {
+                       OutT* __restrict__ out, const int32_t* __restrict__ token_of_row, int n_tokens,
+                       int* err) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
@@ -351,7 +401,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::misc + 4);
 
   // MODE 0: 128 H columns per tile (128 gate + 128 up accumulator columns)
-  const int n_tiles = MODE == 0 ? (F + 127) / 128 : (MODE == 1 ? (N_out + BN - 1) / BN : (N_out + 63) / 64);
+  const int n_tiles = MODE == 0 ? (F + 127) / 128 : ((MODE == 1 || MODE == 3) ? (N_out + BN - 1) / BN : (N_out + 63) / 64);
   build_tile_starts(offsets, E, BM, n_tiles, rows_max, tile_start, sh32, err);
   const int total = tile_start[E];
   if ((int)blockIdx.x >= total) return;   // uniform: nothing allocated yet
@@ -409,7 +459,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
             const int g_row = tc.e * 2 * F + tc.n_tile * 128;
             tma_load_2d(b_dst, &tmB, full, kb * BK, g_row);
             tma_load_2d(b_dst + B_STAGE / 2, &tmB, full, kb * BK, g_row + F);
-          } else if (MODE == 1) {
+          } else if (MODE == 1 || MODE == 3) {
             tma_load_2d(b_dst, &tmB, full, kb * BK, tc.e * N_out + tc.n_tile * BN);
           } else {
             tma_load_2d(b_dst, &tmB, full, kb * BK, tc.n_tile * BN);   // router: 256 rows per n-tile
@@ -474,7 +524,8 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
       const long long wrow0 = (long long)tc.row0 + q * 32;          // first row of this warp
       const int wrows = min(32, max(0, tc.rows - q * 32));          // valid rows of this warp
       (void)r_in;
-      epilogue_tile<MODE, OutT>(taddr, stage, lane, wrow0, wrows, tc.n_tile, F, N_out, gate_of_row, out);
+      epilogue_tile<MODE, OutT>(taddr, stage, lane, wrow0, wrows, tc.n_tile, F, N_out, gate_of_row, out,
+                                token_of_row, n_tokens, err);
       tc_fence_before();
       mbar_arrive(bar_tempty + 8 * acc);
     }
@@ -519,7 +570,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
 grouped_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         const int32_t* __restrict__ offsets, int E, int K, int N_out, int F,
                         long long rows_max, const float* __restrict__ gate_of_row,
-                        OutT* __restrict__ out, int* err) {
+                        OutT* __restrict__ out, const int32_t* __restrict__ token_of_row, int n_tokens,
+                       int* err) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
@@ -532,7 +584,7 @@ grouped_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
   const int cid = (int)(blockIdx.x >> 1), ncl = (int)(gridDim.x >> 1);
   constexpr int PM = 2 * BM;                                 // rows per pair tile
 
-  const int n_tiles = MODE == 0 ? (F + 127) / 128 : (MODE == 1 ? (N_out + BN - 1) / BN : (N_out + 63) / 64);
+  const int n_tiles = MODE == 0 ? (F + 127) / 128 : ((MODE == 1 || MODE == 3) ? (N_out + BN - 1) / BN : (N_out + 63) / 64);
   build_tile_starts(offsets, E, PM, n_tiles, rows_max, tile_start, sh32, err);
   const int total = tile_start[E];
   if (cid >= total) return;   // both CTAs of the pair see the same cid: uniform, nothing allocated
@@ -583,7 +635,7 @@ grouped_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
         const int a_row = tc.row0 + (int)rank * BM;
         int b_row;
         if (MODE == 0) b_row = tc.e * 2 * F + (rank ? F : 0) + tc.n_tile * 128;   // even: gate, odd: up
-        else if (MODE == 1) b_row = tc.e * N_out + tc.n_tile * BN + (int)rank * BM;
+        else if (MODE == 1 || MODE == 3) b_row = tc.e * N_out + tc.n_tile * BN + (int)rank * BM;
         else b_row = tc.n_tile * BN + (int)rank * BM;
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1u, abort_flag, err)) { ok = false; break; }
@@ -647,7 +699,8 @@ grouped_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
       const int cta_rows = min(BM, max(0, tc.rows - (int)rank * BM));
       const long long wrow0 = (long long)tc.row0 + (int)rank * BM + q * 32;
       const int wrows = min(32, max(0, cta_rows - q * 32));
-      epilogue_tile<MODE, OutT>(taddr, stage, lane, wrow0, wrows, tc.n_tile, F, N_out, gate_of_row, out);
+      epilogue_tile<MODE, OutT>(taddr, stage, lane, wrow0, wrows, tc.n_tile, F, N_out, gate_of_row, out,
+                                token_of_row, n_tokens, err);
       tc_fence_before();
       mbar_arrive_cluster(map_to_rank(bar_tempty + 8 * acc, 0));
     }
@@ -695,7 +748,8 @@ bool make_map(CUtensorMap* m, const void* ptr, unsigned long long rows, unsigned
 
 template <int MODE, typename OutT>
 moe_status launch_tc(const CUtensorMap& ma, const CUtensorMap& mb, const int32_t* offsets, int E, int K, int N_out,
-                     int F, long long rows_max, const float* gate_of_row, void* out, cudaStream_t s) {
+                     int F, long long rows_max, const float* gate_of_row, void* out, cudaStream_t s,
+                     const int32_t* token_of_row = nullptr, int n_tokens = 0) {
   static int configured[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -706,13 +760,14 @@ moe_status launch_tc(const CUtensorMap& ma, const CUtensorMap& mb, const int32_t
     if (e != cudaSuccess) return cuda_status(e);
     configured[dev] = 1;
   }
-  const int n_tiles = MODE == 0 ? (F + 127) / 128 : (MODE == 1 ? (N_out + BN - 1) / BN : (N_out + 63) / 64);
+  const int n_tiles = MODE == 0 ? (F + 127) / 128 : ((MODE == 1 || MODE == 3) ? (N_out + BN - 1) / BN : (N_out + 63) / 64);
   const long long max_tiles = ((rows_max + BM - 1) / BM + E) * (long long)n_tiles;
   int grid = num_sms();
   if (max_tiles < grid) grid = (int)max_tiles;
   if (grid < 1) grid = 1;
   grouped_gemm_tc_kernel<MODE, OutT><<<grid, kThreadsTC, kSmemBytes, s>>>(
-      ma, mb, offsets, E, K, N_out, F, rows_max, gate_of_row, static_cast<OutT*>(out), err_ptr());
+      ma, mb, offsets, E, K, N_out, F, rows_max, gate_of_row, static_cast<OutT*>(out), token_of_row, n_tokens,
+      err_ptr());
   return check_launch();
 }
 
@@ -727,7 +782,8 @@ static bool use_pairs(long long rows_max, int groups) { return groups > 0 && row
 
 template <int MODE, typename OutT>
 moe_status launch_tc2(const CUtensorMap& ma, const CUtensorMap& mb, const int32_t* offsets, int E, int K, int N_out,
-                      int F, long long rows_max, const float* gate_of_row, void* out, cudaStream_t s) {
+                      int F, long long rows_max, const float* gate_of_row, void* out, cudaStream_t s,
+                      const int32_t* token_of_row = nullptr, int n_tokens = 0) {
   static int configured[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -738,7 +794,7 @@ moe_status launch_tc2(const CUtensorMap& ma, const CUtensorMap& mb, const int32_
     if (e != cudaSuccess) return cuda_status(e);
     configured[dev] = 1;
   }
-  const int n_tiles = MODE == 0 ? (F + 127) / 128 : (MODE == 1 ? (N_out + BN - 1) / BN : (N_out + 63) / 64);
+  const int n_tiles = MODE == 0 ? (F + 127) / 128 : ((MODE == 1 || MODE == 3) ? (N_out + BN - 1) / BN : (N_out + 63) / 64);
   const long long max_tiles = ((rows_max + 2 * BM - 1) / (2 * BM) + E) * (long long)n_tiles;
   int pairs = num_sms() / 2;
   if (max_tiles < pairs) pairs = (int)max_tiles;
@@ -756,7 +812,8 @@ moe_status launch_tc2(const CUtensorMap& ma, const CUtensorMap& mb, const int32_
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cuda_status(cudaLaunchKernelEx(&cfg, grouped_gemm_tc2_kernel<MODE, OutT>, ma, mb, offsets, E, K, N_out, F,
-                                        rows_max, gate_of_row, static_cast<OutT*>(out), err_ptr()));
+                                        rows_max, gate_of_row, static_cast<OutT*>(out), token_of_row, n_tokens,
+                                        err_ptr()));
 }
 
 moe_status launch_router_logits_tc(const void* x, const int32_t* offs2, int T, int d, int E, const void* W3,
@@ -799,6 +856,21 @@ moe_status launch_down_tc(const void* h, const int32_t* offsets, int E, int d, i
   }
   if (y_dtype == MOE_F32) return launch_tc<1, float>(ma, mb, offsets, E, F, d, F, rows_max, gate_of_row, y_rows, s);
   return launch_tc<1, __nv_bfloat16>(ma, mb, offsets, E, F, d, F, rows_max, gate_of_row, y_rows, s);
+}
+
+// Down GEMM with the combine fused into its epilogue: y[token_of_row[r]] += gate_of_row[r] *
+// (H[r] W_dn[e]^T), y fp32 [T, d] already initialised by the caller.
+moe_status launch_down_combine_tc(const void* h, const int32_t* offsets, int E, int d, int F, long long rows_max,
+                                  const void* W_dn, const float* gate_of_row, const int32_t* token_of_row, int T,
+                                  float* y, cudaStream_t s) {
+  if (rows_max == 0 || T == 0) return MOE_OK;
+  if (F < BK || d < 8) return MOE_ERR_UNSUPPORTED;
+  const bool pair = use_pairs(rows_max, E);
+  CUtensorMap ma, mb;
+  if (!make_map(&ma, h, (unsigned long long)rows_max, F, BM)) return MOE_ERR_UNSUPPORTED;
+  if (!make_map(&mb, W_dn, (unsigned long long)E * d, F, pair ? BM : BN)) return MOE_ERR_UNSUPPORTED;
+  if (pair) return launch_tc2<3, float>(ma, mb, offsets, E, F, d, F, rows_max, gate_of_row, y, s, token_of_row, T);
+  return launch_tc<3, float>(ma, mb, offsets, E, F, d, F, rows_max, gate_of_row, y, s, token_of_row, T);
 }
 
 }  // namespace moe

@@ -100,30 +100,33 @@ stats_partial_kernel(const float* __restrict__ logits, int T, int E, int score, 
   }
 }
 
-// Stage 2: one CTA of 1024 threads.  P_e: one warp per expert, lanes take the partials
-// in a fixed strided order (8 loads in flight), then a fixed butterfly.  The four
-// per-expert sums (aux, kept, variance, max) are reduced together in one pass.
+// Stage 2: one CTA of 1024 threads.  P_e: the threads form G = 1024 / E groups of E;
+// thread (g, e) sums partial rows g, g + G, g + 2G, ... of expert e (consecutive threads
+// read consecutive experts of one row: whole lines per warp load, 8 loads in flight),
+// then the G group sums are added in group order.  The four per-expert sums (aux, kept,
+// variance, max) are reduced together in one pass.
 __global__ void __launch_bounds__(1024)
 stats_final_kernel(const double* __restrict__ partP, const double* __restrict__ partZ, int nparts,
                    const int32_t* __restrict__ counts, const int32_t* __restrict__ kept, int T, int E,
                    int k, float* __restrict__ load, float* __restrict__ stats5) {
   __shared__ double Ps[1024];
+  __shared__ double grp[1024];
   __shared__ double red[4][32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  for (int e = warp; e < E; e += nw) {
+  const int G = max(1, (int)blockDim.x / E);                 // E <= 1024
+  if ((int)threadIdx.x < G * E) {
+    const int e = (int)threadIdx.x % E, g = (int)threadIdx.x / E;
     double p = 0.0;
-    int b = lane;
-    for (; b + 32 * 7 < nparts; b += 32 * 8) {
+    int b = g;
+    for (; b + 7 * G < nparts; b += 8 * G) {
       double v[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = __ldg(partP + (long long)(b + 32 * u) * E + e);
+      for (int u = 0; u < 8; ++u) v[u] = __ldg(partP + (long long)(b + u * G) * E + e);
 #pragma unroll
       for (int u = 0; u < 8; ++u) p += v[u];
     }
-    for (; b < nparts; b += 32) p += __ldg(partP + (long long)b * E + e);
-#pragma unroll
-    for (int o = 16; o; o >>= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
-    if (lane == 0) Ps[e] = p;
+    for (; b < nparts; b += G) p += __ldg(partP + (long long)b * E + e);
+    grp[threadIdx.x] = p;
   }
   double z = 0.0;
   if (warp == nw - 1) {                       // the z partials, on the last warp
@@ -138,6 +141,12 @@ stats_final_kernel(const double* __restrict__ partP, const double* __restrict__ 
     for (; b < nparts; b += 32) z += __ldg(partZ + b);
 #pragma unroll
     for (int o = 16; o; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    double p = 0.0;
+    for (int g = 0; g < G; ++g) p += grp[g * E + e];
+    Ps[e] = p;
   }
   __syncthreads();
   const double TK = (double)T * k;

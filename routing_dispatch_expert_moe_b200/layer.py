@@ -4,8 +4,14 @@ MoELayer owns preallocated device buffers for a maximum token count and runs, on
 stream with no host synchronisation:
 
     moe_route -> moe_histogram_scan -> moe_permute -> moe_expert_gate_up
-      -> moe_expert_down (gate fused) [-> shared expert: gate_up/down with E = 1]
-      -> moe_combine [-> moe_router_stats]
+      combine="rows":  -> moe_expert_down (gate fused) [-> shared expert: gate_up/down
+                       with E = 1] -> moe_combine
+      combine="fused": [-> shared expert, written into y] -> moe_expert_down_combine
+    [-> moe_router_stats]
+
+"rows" sums each token's terms in slot order and is bitwise reproducible; "fused" adds
+them into y with fp32 atomics inside the down GEMM (no gated-row buffer, no combine
+pass), so its y differs from run to run by fp32 rounding only.
 
 Orchestration only: every step runs in the library's CUDA kernels.
 """
@@ -33,9 +39,17 @@ class MoEWeights:
 class MoELayer:
     def __init__(self, weights: MoEWeights, k: int, T_max: int, score: str = "softmax",
                  renormalize: bool = True, scale: float = 1.0, capacity: int = -1,
-                 rows_dtype: torch.dtype = torch.float32, out_dtype: torch.dtype = torch.float32):
+                 rows_dtype: torch.dtype = torch.float32, out_dtype: torch.dtype = torch.float32,
+                 combine: str = "rows"):
         """rows_dtype: gated expert rows (and the shared expert's output); out_dtype: y.
-        fp32 (the default) leaves H as the only bf16 rounding inside the layer."""
+        fp32 (the default) leaves H as the only bf16 rounding inside the layer.
+        combine: "rows" (gated rows + ordered combine) or "fused" (down GEMM adds into an
+        fp32 y; needs out_dtype fp32)."""
+        if combine not in ("rows", "fused"):
+            raise ValueError(f"combine must be 'rows' or 'fused', got {combine!r}")
+        if combine == "fused" and out_dtype != torch.float32:
+            raise ValueError("combine='fused' accumulates into an fp32 y: out_dtype must be torch.float32")
+        self.combine_mode = combine
         w = weights
         self.w = w
         self.d, self.E = w.Wg.shape
@@ -61,7 +75,7 @@ class MoELayer:
         self.gate_of_row = torch.empty(R, dtype=f32, device=dev)
         self.x_perm = torch.empty((R, d), dtype=self.dtype, device=dev)
         self.h = torch.empty((R, F), dtype=self.dtype, device=dev)
-        self.y_perm = torch.empty((R, d), dtype=rows_dtype, device=dev)
+        self.y_perm = torch.empty((R, d), dtype=rows_dtype, device=dev) if combine == "rows" else None
         self.y = torch.empty((T_max, d), dtype=out_dtype, device=dev)
         self.load = torch.empty(E, dtype=f32, device=dev)
         self.stats5 = torch.empty(5, dtype=f32, device=dev)
@@ -71,7 +85,7 @@ class MoELayer:
             self.F_s = w.W_dn_s.shape[2]
             self.shared_offsets = torch.tensor([0, T_max], dtype=i32, device=dev)
             self.h_s = torch.empty((T_max, self.F_s), dtype=self.dtype, device=dev)
-            self.y_s = torch.empty((T_max, d), dtype=rows_dtype, device=dev)
+            self.y_s = torch.empty((T_max, d), dtype=rows_dtype, device=dev) if combine == "rows" else None
 
     # individual steps (so that a caller can time them one by one)
     def route(self, x, stream=None):
@@ -94,11 +108,17 @@ class MoELayer:
                           stream=stream)
 
     def shared(self, x, stream=None):
+        """Shared expert (weight 1): into y_s ("rows"), or straight into y ("fused")."""
         T = x.shape[0]
         if T != self.T_max:
             self.shared_offsets[1].fill_(T)
+        out = self.y_s[:T] if self.combine_mode == "rows" else self.y[:T]
         M.moe_expert_gate_up(x, self.shared_offsets, self.w.W_gu_s, T, self.h_s[:T], stream)
-        M.moe_expert_down(self.h_s[:T], self.shared_offsets, self.w.W_dn_s, T, None, self.y_s[:T], stream=stream)
+        M.moe_expert_down(self.h_s[:T], self.shared_offsets, self.w.W_dn_s, T, None, out, stream=stream)
+
+    def down_combine(self, T, stream=None):
+        M.moe_expert_down_combine(self.h, self.offsets, self.w.W_dn, self.rows_max, self.token_of_row, self.y[:T],
+                                  self.gate_of_row, accumulate=self.has_shared, stream=stream)
 
     def combine(self, T, stream=None):
         M.moe_combine(self.y_perm, self.row_of[:T], T, self.rows_max, None,
@@ -108,22 +128,34 @@ class MoELayer:
         M.moe_router_stats(self.logits[:T], self.counts, self.kept, self.k, self.score, self.load, self.stats5,
                            self.ws, stream)
 
+    def stages(self, x: torch.Tensor, with_stats: bool = True):
+        """The forward as (name, fn(stream)) steps in launch order."""
+        T = x.shape[0]
+        st = [("route", lambda s: self.route(x, s)),
+              ("histogram_scan", lambda s: self.histogram_scan(T, s)),
+              ("permute", lambda s: self.permute(x, s)),
+              ("gate_up", lambda s: self.gate_up(s))]
+        if self.combine_mode == "rows":
+            st.append(("down", lambda s: self.down(s)))
+            if self.has_shared:
+                st.append(("shared", lambda s: self.shared(x, s)))
+            st.append(("combine", lambda s: self.combine(T, s)))
+        else:
+            if self.has_shared:
+                st.append(("shared", lambda s: self.shared(x, s)))
+            st.append(("down_combine", lambda s: self.down_combine(T, s)))
+        if with_stats:
+            st.append(("stats", lambda s: self.stats(T, s)))
+        return st
+
     def forward(self, x: torch.Tensor, stream=None, with_stats: bool = True) -> torch.Tensor:
         T = x.shape[0]
         if T > self.T_max:
             raise ValueError(f"T={T} exceeds T_max={self.T_max}")
         if x.dtype != self.dtype:
             raise ValueError(f"x must be {self.dtype}")
-        self.route(x, stream)
-        self.histogram_scan(T, stream)
-        self.permute(x, stream)
-        self.gate_up(stream)
-        self.down(stream)
-        if self.has_shared:
-            self.shared(x, stream)
-        self.combine(T, stream)
-        if with_stats:
-            self.stats(T, stream)
+        for _, fn in self.stages(x, with_stats):
+            fn(stream)
         return self.y[:T]
 
     # ---------------------------------------------------------------- CUDA graph
@@ -153,6 +185,8 @@ class MoELayer:
     # library kernels launched by one forward (the scan's workspace memset is not a kernel)
     def launches_per_forward(self, with_stats: bool = True) -> int:
         n = 2 + 2 + 1 + 1 + 1 + 1          # route(2) scan(2) permute gate_up down combine
+        if self.combine_mode == "fused":
+            n -= 1                         # down_combine (its zero fill is a memset, not a kernel)
         if self.has_shared:
             n += 2
         if with_stats:

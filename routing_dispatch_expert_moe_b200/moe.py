@@ -48,6 +48,8 @@ _SIGNATURES = {
                                _i32, _c_void_p, _c_void_p]),
     "moe_grouped_ffn": (_i32, [_c_void_p, _i32, _c_void_p, _i32, _i32, _i32, _i64, _c_void_p, _c_void_p,
                                _c_void_p, _c_void_p, _i32, _c_void_p, _c_void_p]),
+    "moe_expert_down_combine": (_i32, [_c_void_p, _i32, _c_void_p, _i32, _i32, _i32, _i64, _c_void_p, _c_void_p,
+                                       _c_void_p, _i32, _i32, _c_void_p, _c_void_p]),
     "moe_combine": (_i32, [_c_void_p, _i32, _c_void_p, _c_void_p, _c_void_p, _i32, _i32, _i32, _i64, _i32,
                            _c_void_p, _c_void_p]),
     "moe_router_stats_workspace_bytes": (_size, [_i32, _i32]),
@@ -252,6 +254,27 @@ def moe_expert_down(h, offsets, W_dn, rows_max: int, gate_of_row=None, y_rows=No
     _check("moe_expert_down", lib().moe_expert_down(_p(h), _dt(h), _p(offsets), E, d, F, rows_max, _p(W_dn),
                                                     _p(gate_of_row), _dt(y_rows), _p(y_rows), _stream(stream)))
     return y_rows
+
+
+def moe_expert_down_combine(h, offsets, W_dn, rows_max: int, token_of_row, y, gate_of_row=None,
+                            accumulate: bool = False, stream=None):
+    """y[token_of_row[r]] += gate_of_row[r] * (H[r] W_dn^T) into fp32 y [T, d] (zeroed first
+    unless accumulate); the combine fused into the down GEMM, summed with fp32 atomics."""
+    E, d, F = W_dn.shape
+    _need(h, "h")
+    _need(offsets, "offsets", torch.int32, (E + 1,))
+    _need(W_dn, "W_dn", h.dtype)
+    _need(token_of_row, "token_of_row", torch.int32)
+    if gate_of_row is not None:
+        _need(gate_of_row, "gate_of_row", torch.float32)
+    _need(y, "y", torch.float32)
+    if y.dim() != 2 or y.shape[1] != d:
+        raise ValueError(f"y must be [T, {d}]")
+    _check("moe_expert_down_combine",
+           lib().moe_expert_down_combine(_p(h), _dt(h), _p(offsets), E, d, F, rows_max, _p(W_dn), _p(gate_of_row),
+                                         _p(token_of_row), y.shape[0], 1 if accumulate else 0, _p(y),
+                                         _stream(stream)))
+    return y
 
 
 def moe_grouped_ffn(x_rows, offsets, W_gu, W_dn, rows_max: int, gate_of_row=None, h=None, y_rows=None,

@@ -132,6 +132,14 @@ def test_ffn_host_validation(L):
     g = L.moe_expert_down
     assert g(FAKE, 0, FAKE, 4, 128, 64, -1, FAKE, NUL, 1, FAKE, NUL) == 1
     assert g(FAKE, 0, FAKE, 4, 128, 64, 128, FAKE, NUL, 7, FAKE, NUL) == 1        # y dtype
+    h = L.moe_expert_down_combine      # (h, dt, offs, E, d, F, rows_max, W_dn, gate, tok, T, accumulate, y, s)
+    assert h(FAKE, 0, FAKE, 4, 128, 64, 128, FAKE, NUL, FAKE, 64, 2, FAKE, NUL) == 1      # accumulate flag
+    assert h(FAKE, 0, FAKE, 4, 128, 64, 128, FAKE, NUL, FAKE, -1, 0, FAKE, NUL) == 1      # T < 0
+    assert h(FAKE, 0, FAKE, 4, 128, 64, 128, FAKE, NUL, NUL, 64, 0, FAKE, NUL) == 1       # token_of_row
+    assert h(FAKE, 0, FAKE, 4, 128, 64, 128, FAKE, NUL, FAKE, 64, 0, NUL, NUL) == 1       # y
+    assert h(FAKE, 0, FAKE, 4, 128, 64, 128, FAKE, NUL, FAKE, 64, 0, ctypes.c_void_p(4104), NUL) == 2
+    assert h(FAKE, 0, FAKE, 4, 100, 64, 128, FAKE, NUL, FAKE, 64, 0, FAKE, NUL) == 2      # d % 8
+    assert h(FAKE, 0, FAKE, 4, 128, 64, 128, FAKE, NUL, FAKE, 0, 0, FAKE, NUL) == 0       # no tokens
 
 
 def test_permute_combine_host_validation(L):

@@ -250,3 +250,109 @@ def test_c5_stress_full_size_per_assignment_capacity():
 @pytest.mark.slow
 def test_c5_stress_full_size_literal_capacity():
     full_size_check("c5_stress", per_assignment=False)
+
+
+# ---------------------------------------------------------------- combine fused into the down GEMM
+FUSED = [c for c in SMALL if c.name in ("softmax_bf16", "sigmoid_bias_shared", "sqrt_softplus_capacity_zipf",
+                                         "ragged_multitile", "fp32_small", "bf16_d_below_tile")]
+
+
+def _ordered_terms_bound(rows_layer, T, k):
+    """Elementwise bound on |fused y - ordered y|: both are fp32 sums of the same n <= k + 1
+    terms (the gated rows and the shared expert's row) in different orders, so they differ
+    by at most (n - 1) * 2^-23 * sum |terms|."""
+    yp = rows_layer.y_perm.float()
+    row_of = rows_layer.row_of[:T].long()
+    acc = torch.zeros((T, yp.shape[1]), dtype=torch.float64, device=yp.device)
+    for j in range(k):
+        r = row_of[:, j]
+        m = r >= 0
+        acc[m] += yp[r[m]].double().abs()
+    if rows_layer.has_shared:
+        acc += rows_layer.y_s[:T].double().abs()
+    return (k * 2.0 ** -23 * acc).cpu().numpy()
+
+
+@pytest.mark.parametrize("cfg", FUSED, ids=lambda c: c.name)
+def test_fused_down_combine_parity(cfg):
+    host, dev = U.make_inputs(cfg)
+    cap = O.capacity(cfg.T, cfg.E, cfg.k, cfg.capacity_factor, True)
+    rl, gr = U.gpu_forward(cfg, dev, cap)
+    fl, gf = U.gpu_forward(cfg, dev, cap, combine="fused")
+    for key in ("topk_idx", "topk_gate", "row_of", "offsets", "token_of_row", "gate_of_row"):
+        assert np.array_equal(gf[key], gr[key]), key
+    # against the oracle, with the same bar as the ordered combine
+    gu, dn = U.expert_getters(host)
+    bf16 = cfg.act == "bf16"
+    o = O.layer_routing(U.cfg_dict(cfg), host["x"], host["Wg"], host["off"], host["bias"], True)
+    n = gf["n_rows"]
+    yp_o = O.grouped_ffn(O.permute(host["x"], o["row_of"], n), o["offsets"], gu, dn, o["gate_of_row"], bf16)
+    sh = host["shared"]
+    ys = O.shared_expert(host["x"], sh[0], sh[1], bf16) if sh is not None else None
+    y_o = O.combine(yp_o, o["row_of"], ys)
+    if np.any(y_o):
+        U.assert_y_close(gf["y"], y_o, "y (fused)")
+    # against the ordered sum of the very same fp32 terms
+    bound = _ordered_terms_bound(rl, cfg.T, cfg.k)
+    diff = np.abs(gf["y"] - gr["y"])
+    assert (diff <= bound + 1e-30).all(), f"fused vs ordered: max excess {(diff - bound).max():.3g}"
+    # a dropped-everywhere token gets exactly the shared expert's row (or zero)
+    dropped = (gr["row_of"] < 0).all(axis=1)
+    if dropped.any():
+        ref = rl.y_s[:cfg.T].float().cpu().numpy() if rl.has_shared else np.zeros_like(gf["y"])
+        assert np.array_equal(gf["y"][dropped], ref[dropped].astype(np.float64))
+
+
+def test_fused_down_combine_graph_replay():
+    cfg = SMALL[1]
+    host, dev = U.make_inputs(cfg)
+    cap = O.capacity(cfg.T, cfg.E, cfg.k, cfg.capacity_factor, True)
+    rl, gr = U.gpu_forward(cfg, dev, cap)
+    layer = U.build_layer(cfg, dev, cap, combine="fused")
+    x_static = dev["x"].clone()
+    layer.capture(x_static)
+    for _ in range(3):
+        y = layer.replay()
+    torch.cuda.synchronize()
+    from routing_dispatch_expert_moe_b200 import moe as M
+    assert M.moe_get_device_error() == 0
+    bound = _ordered_terms_bound(rl, cfg.T, cfg.k)
+    assert (np.abs(y.double().cpu().numpy() - gr["y"]) <= bound + 1e-30).all()
+
+
+def test_fused_bad_token_is_reported_not_trapped():
+    from routing_dispatch_expert_moe_b200 import moe as M
+    for cfg in (SMALL[0], SMALL[6]):                          # tensor-core and fp32 SIMT forms
+        host, dev = U.make_inputs(cfg)
+        layer, g = U.gpu_forward(cfg, dev, -1, combine="fused")
+        tok = layer.token_of_row.clone()
+        tok[5] = cfg.T + 7                                     # outside [0, T): skipped, recorded
+        M.moe_expert_down_combine(layer.h, layer.offsets, layer.w.W_dn, layer.rows_max, tok, layer.y[:cfg.T],
+                                  layer.gate_of_row)
+        torch.cuda.synchronize()
+        assert M.moe_get_device_error() == 3
+
+
+def fused_full_size_check(name):
+    cfg = I.CONFIGS[name]
+    host, dev = U.make_inputs(cfg)
+    cap = O.capacity(cfg.T, cfg.E, cfg.k, cfg.capacity_factor, True)
+    layer, g = U.gpu_forward(cfg, dev, cap, combine="fused")
+    o = O.layer_routing(U.cfg_dict(cfg), host["x"], host["Wg"], host["off"], host["bias"], True)
+    U.assert_routing_equal(g, o)
+    toks = U.stratified_tokens(o, cap)
+    gu, dn = U.expert_getters(host)
+    sub = O.layer_outputs_for_tokens(toks, host["x"], o, gu, dn, True, shared=host["shared"])
+    U.assert_y_close(g["y"][toks], sub["y"], "y fused (sampled)")
+    del layer, dev
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.slow
+def test_c2_handbook_full_size_fused_combine():
+    fused_full_size_check("c2_handbook")
+
+
+@pytest.mark.slow
+def test_c3_fine_grained_full_size_fused_combine():
+    fused_full_size_check("c3_fine_grained")
