@@ -31,9 +31,10 @@ METRIC = "MoE-layer fwd tokens/s on 1 B200; grouped-GEMM TFLOP/s; route/permute 
 UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-# DRAM traffic of the dominant kernel (moe_expert_gate_up) per launch, from an ncu capture of
-# the same kernel build (see profiles/); None when the kernel changed since the capture.
-GATE_UP_TRAFFIC = {}
+# DRAM traffic (read + write bytes) of the dominant kernel, the gate/up GEMM, per launch, keyed
+# by (workload, dispatch), from an ncu capture of the same kernel build (summaries under
+# profiles/); absent when the kernel changed since the capture.
+GATE_UP_TRAFFIC = {("c2_handbook", "permute"): 805563136 + 121037824}
 
 
 def peaks():
@@ -98,10 +99,11 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
-def layer_roofline_ms(cfg, A, pk, rb=4, ob=4, fused=False):
+def layer_roofline_ms(cfg, A, pk, rb=4, ob=4, fused=False, gather=False):
     """Sum over steps of max(compute, memory) time at the measured peaks (algorithmic bytes / flops).
     rb / ob: bytes per element of the gated rows / of the layer output.  fused: the combine runs
-    inside the down GEMM, whose algorithmic bytes are then H, W_dn and y (zero fill + result)."""
+    inside the down GEMM, whose algorithmic bytes are then H, W_dn and y (zero fill + result).
+    gather: the permute runs inside the gate/up GEMM, whose algorithmic bytes are then x, W_gu, H."""
     T, d, E, k, F = cfg.T, cfg.d, cfg.E, cfg.k, cfg.F
     hbm = pk["hbm_gbs"] * 1e9
     tc = pk["bf16_tflops"] * 1e12
@@ -110,10 +112,13 @@ def layer_roofline_ms(cfg, A, pk, rb=4, ob=4, fused=False):
     steps = {
         "route": max(2 * T * d * E / fp32, (T * d * b + d * E * 4 + T * E * 4 + T * k * 8) / hbm),
         "histogram_scan": (T * k * 4 * 3 + A * 8) / hbm,
-        "permute": (T * d * b + A * d * b) / hbm,
-        "gate_up": max(4 * A * d * F / tc, (A * d * b + E * 2 * F * d * b + A * F * b) / hbm),
         "stats": (T * E * 4) / hbm,
     }
+    if gather:
+        steps["gate_up_gather"] = max(4 * A * d * F / tc, (T * d * b + E * 2 * F * d * b + A * F * b) / hbm)
+    else:
+        steps["permute"] = (T * d * b + A * d * b) / hbm
+        steps["gate_up"] = max(4 * A * d * F / tc, (A * d * b + E * 2 * F * d * b + A * F * b) / hbm)
     if fused:
         steps["down_combine"] = max(2 * A * F * d / tc, (A * F * b + E * d * F * b + 2 * T * d * 4) / hbm)
     else:
@@ -159,8 +164,9 @@ def run_ours(args):
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
 
-    def make_layer(mode):
-        return MoELayer(w, cfg.k, cfg.T, cfg.score, cfg.renormalize, cfg.scale, cap, combine=mode)
+    def make_layer(combine, dispatch):
+        return MoELayer(w, cfg.k, cfg.T, cfg.score, cfg.renormalize, cfg.scale, cap, combine=combine,
+                        dispatch=dispatch)
 
     def time_layer(layer, steps, clocks=None):
         """Warm-up, then `steps` replays of one forward captured as a CUDA graph whose timing
@@ -225,21 +231,21 @@ def run_ours(args):
             v = float(t.item())
         return v
 
-    layer = make_layer(args.combine)
+    layer = make_layer(args.combine, args.dispatch)
     per_step, stage_ms, A, clk = time_layer(layer, args.steps, ClockSampler(local_rank))
     total_ms = max_over_ranks(float(per_step.sum()))
     ms_per_step = total_ms / args.steps
     value = cfg.T * world * args.steps / (total_ms / 1e3)
 
     other = None
-    if args.combine == "fused" and args.rows_steps > 0:
-        # the bitwise-reproducible form (gated rows + ordered combine), same inputs
-        rl = make_layer("rows")
-        ps, sm, _, _ = time_layer(rl, args.rows_steps)
+    if (args.combine, args.dispatch) != ("rows", "permute") and args.unfused_steps > 0:
+        # the unfused form (permute copy, gated rows, ordered combine: bitwise reproducible), same inputs
+        rl = make_layer("rows", "permute")
+        ps, sm, _, _ = time_layer(rl, args.unfused_steps)
         t = max_over_ranks(float(ps.sum()))
-        other = {"combine": "rows (gated rows + ordered combine, bitwise reproducible)",
-                 "ms_per_step": round(t / args.rows_steps, 4),
-                 "value": round(cfg.T * world * args.rows_steps / (t / 1e3), 1), "steps": args.rows_steps,
+        other = {"dispatch": "permute", "combine": "rows (gated rows + ordered combine, bitwise reproducible)",
+                 "ms_per_step": round(t / args.unfused_steps, 4),
+                 "value": round(cfg.T * world * args.unfused_steps / (t / 1e3), 1), "steps": args.unfused_steps,
                  "stages_ms": {k_: round(v, 4) for k_, v in sm.items()}}
         del rl
         torch.cuda.empty_cache()
@@ -271,20 +277,22 @@ def run_ours(args):
     d2h_bytes = y_host.numel() * y_host.element_size()
 
     pk, pk_src = peaks()
-    gate_up_ms = stage_ms["gate_up"]
+    gather = args.dispatch == "gather"
+    gate_up_ms = stage_ms["gate_up_gather" if gather else "gate_up"]
     flops = 4.0 * A * cfg.d * cfg.F
     achieved = flops / (gate_up_ms * 1e-3) / 1e12
     peak = pk["bf16_tflops"]
     fused = args.combine == "fused"
     rb = 4 if fused else layer.y_perm.element_size()
     ob = layer.y.element_size()
-    roof_ms, roof_steps = layer_roofline_ms(cfg, A, pk, rb, ob, fused)
-    traffic = GATE_UP_TRAFFIC.get(args.workload)
+    roof_ms, roof_steps = layer_roofline_ms(cfg, A, pk, rb, ob, fused, gather)
+    traffic = GATE_UP_TRAFFIC.get((args.workload, args.dispatch))
     down_ms = stage_ms["down_combine" if fused else "down"]
     thr = {"down_tflops": round(2.0 * A * cfg.F * cfg.d / (down_ms * 1e-3) / 1e12, 1),
-           "permute_gbs": round((cfg.T * cfg.d * 2 + A * cfg.d * 2) / (stage_ms["permute"] * 1e-3) / 1e9, 1),
            "route_gbs": round((cfg.T * cfg.d * 2 + cfg.T * cfg.E * 8 + cfg.T * cfg.k * 8) /
                               (stage_ms["route"] * 1e-3) / 1e9, 1)}
+    if not gather:
+        thr["permute_gbs"] = round((cfg.T * cfg.d * 2 + A * cfg.d * 2) / (stage_ms["permute"] * 1e-3) / 1e9, 1)
     if not fused:
         thr["combine_gbs"] = round((A * cfg.d * rb + cfg.T * cfg.d * ob) / (stage_ms["combine"] * 1e-3) / 1e9, 1)
 
@@ -298,6 +306,7 @@ def run_ours(args):
             "data": "synthetic (seeded; integer-grid router inputs, N(0,0.02) bf16 expert weights)",
             "config": {"workload": args.workload, "T": cfg.T, "d": cfg.d, "E": cfg.E, "k": cfg.k, "F": cfg.F,
                        "F_shared": cfg.F_s, "score": cfg.score, "capacity": cap, "rows": A,
+                       "dispatch": ("gathered inside the gate/up GEMM" if gather else "permute copy"),
                        "combine": ("fused into the down GEMM (fp32 atomics into y)" if fused
                                    else "gated rows + ordered combine"),
                        "parallelism": f"replicas x{world} (independent token batches, no collective)",
@@ -305,7 +314,9 @@ def run_ours(args):
             "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d_bytes,
                     "d2h_bytes_per_step": d2h_bytes, "steps": e2e_steps},
             "gpu_launches": args.steps * layer.launches_per_forward(True),
-            "roofline": {"bound": "tensor", "kernel": "moe_expert_gate_up (tcgen05 grouped GEMM + SwiGLU)",
+            "roofline": {"bound": "tensor",
+                         "kernel": ("moe_expert_gate_up_gather (tcgen05 grouped GEMM, gathered rows, SwiGLU)"
+                                    if gather else "moe_expert_gate_up (tcgen05 grouped GEMM + SwiGLU)"),
                          "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
                          "frac": round(achieved / peak, 4), "traffic": traffic,
                          "peak_source": f"{pk_src} bf16_tflops (burst)"},
@@ -314,7 +325,7 @@ def run_ours(args):
             "stages_ms": {k_: round(v, 4) for k_, v in stage_ms.items()},
             "stage_roofline_ms": {k_: round(v, 4) for k_, v in roof_steps.items()},
             "stage_throughput": thr,
-            "rows_variant": other,
+            "unfused_variant": other,
             "clocks": clk,
             "cpu_baseline": cpu,
         }
@@ -431,8 +442,10 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=50, help="steps timed through host buffers")
     ap.add_argument("--combine", choices=["fused", "rows"], default="fused",
                     help="fused: combine inside the down GEMM; rows: gated rows + ordered combine")
-    ap.add_argument("--rows-steps", type=int, default=100,
-                    help="with --combine fused, also time the rows form for this many steps (0 = skip)")
+    ap.add_argument("--dispatch", choices=["gather", "permute"], default="permute",
+                    help="gather: the gate/up GEMM reads token rows through the row map; permute: x_perm copy")
+    ap.add_argument("--unfused-steps", type=int, default=100,
+                    help="also time the unfused form (permute + rows) for this many steps (0 = skip)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -10,6 +10,7 @@
  *                        expert-contiguous row offsets and the row maps
  *   moe_permute          gather tokens into expert-contiguous rows
  *   moe_expert_gate_up   grouped GEMM  H = silu(X Wg^T) * (X Wu^T)       (per expert)
+ *   moe_expert_gate_up_gather  the same with the permute fused into it (X read via the row map)
  *   moe_expert_down      grouped GEMM  Y = gate_of_row * (H Wd^T)       (per expert)
  *   moe_grouped_ffn      the two GEMMs above back to back
  *   moe_combine          gate-weighted sum of each token's rows (+ shared expert)
@@ -229,6 +230,18 @@ MOE_API moe_status moe_permute(const void* x, int32_t dtype, int32_t T, int32_t 
  * A shared expert is the call with E = 1, offsets = {0, T} and x_rows = x.
  * ---------------------------------------------------------------------------------- */
 MOE_API moe_status moe_expert_gate_up(const void* x_rows, int32_t dtype, const int32_t* offsets,
+                              int32_t E, int32_t d, int32_t F, int64_t rows_max,
+                              const void* W_gu, void* h, void* stream);
+/* moe_expert_gate_up_gather -- moe_expert_gate_up with the dispatch fused into it: row r
+ * of the GEMM's A operand is read from x[token_of_row[r]] directly ([Handbook-News]
+ * "MoE 到底省了什么": sending each token to its experts), so the permuted copy x_perm is
+ * neither written nor read and moe_permute is not needed before it.
+ *   x (device) [T, d] dtype;  token_of_row (device) [rows_max] int32 from
+ *   moe_histogram_scan;  the other arguments as moe_expert_gate_up.
+ * H is bitwise identical to moe_permute followed by moe_expert_gate_up.  A token index
+ * outside [0, T) reads as a zero row and is recorded as MOE_DEVERR_ROW. */
+MOE_API moe_status moe_expert_gate_up_gather(const void* x, int32_t dtype, int32_t T,
+                              const int32_t* token_of_row, const int32_t* offsets,
                               int32_t E, int32_t d, int32_t F, int64_t rows_max,
                               const void* W_gu, void* h, void* stream);
 MOE_API moe_status moe_expert_down(const void* h, int32_t dtype, const int32_t* offsets,

@@ -184,6 +184,21 @@ moe_status moe_expert_gate_up(const void* x_rows, int32_t dtype, const int32_t* 
   return launch_gate_up_simt(x_rows, dtype, offsets, E, d, F, rows_max, W_gu, h, S(stream));
 }
 
+moe_status moe_expert_gate_up_gather(const void* x, int32_t dtype, int32_t T, const int32_t* token_of_row,
+                                     const int32_t* offsets, int32_t E, int32_t d, int32_t F, int64_t rows_max,
+                                     const void* W_gu, void* h, void* stream) {
+  if (T < 0) return MOE_ERR_INVALID_ARG;
+  if ((long long)T >= kMaxT) return MOE_ERR_UNSUPPORTED;
+  moe_status st = check_ffn(x, dtype, offsets, E, d, F, rows_max, W_gu, h);
+  if (st != MOE_OK || rows_max == 0 || T == 0) return st;
+  if (!token_of_row) return MOE_ERR_INVALID_ARG;
+  if (dtype == MOE_BF16) {
+    st = launch_gate_up_gather_tc(x, token_of_row, T, offsets, E, d, F, rows_max, W_gu, h, S(stream));
+    if (st != MOE_ERR_UNSUPPORTED) return st;
+  }
+  return launch_gate_up_gather_simt(x, dtype, token_of_row, T, offsets, E, d, F, rows_max, W_gu, h, S(stream));
+}
+
 moe_status moe_expert_down(const void* h, int32_t dtype, const int32_t* offsets, int32_t E, int32_t d, int32_t F,
                            int64_t rows_max, const void* W_dn, const float* gate_of_row, int32_t y_dtype,
                            void* y_rows, void* stream) {

@@ -7,6 +7,7 @@
 //   gate_up: H[r, f] = silu(sum_c X[r,c] Wg[f,c]) * (sum_c X[r,c] Wu[f,c])
 //   down:    Y[r, n] = gate_of_row[r] * sum_f H[r,f] Wd[n,f]
 //   down + combine: y[token_of_row[r], n] += gate_of_row[r] * sum_f H[r,f] Wd[n,f]  (fp32 atomics)
+//   gate_up, gathered: as gate_up with X[r] = x[token_of_row[r]] (no permuted copy of x)
 // Expert FFN: "Mixture of Experts Explained" (zh), section "什么是混合专家模型" (each
 // expert is an FFN); SwiGLU form silu(x Wg^T) * (x Wu^T) Wd^T without biases.
 //
@@ -41,6 +42,7 @@ __device__ __forceinline__ void st_elem<__nv_bfloat16>(__nv_bfloat16* p, float v
 // MODE 0: gate_up (A = x_rows [*, d], B = W_gu [E][2F][d], out = H [*, F])
 // MODE 1: down    (A = H [*, F], B = W_dn [E][d][F], out = Y [*, d], scaled by gate_of_row)
 // MODE 2: down + combine (as MODE 1, out = y [T, d] fp32, rows added into their token's row)
+// MODE 3: gate_up with A = x [T, d] read through token_of_row
 // OT: output element type (MODE 0 writes H in the activation dtype; MODE 1 writes the
 // gated rows in the caller's choice of bf16 or fp32).
 template <typename DT, int MODE, typename OT>
@@ -52,18 +54,35 @@ grouped_simt_kernel(const DT* __restrict__ A, const DT* __restrict__ B, const in
   __shared__ int sh32[32];
   __shared__ __align__(16) float As[kBK][kBM + 4];
   __shared__ __align__(16) float Bs[kBK][kBN + 4];
-  __shared__ __align__(16) float Us[MODE == 0 ? kBK : 1][kBN + 4];
+  constexpr bool GU = MODE == 0 || MODE == 3;               // gate/up (else down)
+  __shared__ __align__(16) float Us[GU ? kBK : 1][kBN + 4];
+  __shared__ int toks[MODE == 3 ? kBM : 1];
 
   const int n_tiles = (N + kBN - 1) / kBN;
   build_tile_starts(offsets, E, kBM, n_tiles, rows_max, tile_start, sh32, err);
   const int total = tile_start[E];
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-  const long long b_rows = MODE == 0 ? 2LL * F : (long long)N;   // B rows per expert
+  const long long b_rows = GU ? 2LL * F : (long long)N;   // B rows per expert
 
   for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
     const TileCoord tc = tile_coord(tile_start, offsets, E, kBM, tile);
     const int n0 = tc.n_tile * kBN;
     const DT* Be = B + (long long)tc.e * b_rows * K;
+    if (MODE == 3) {
+      __syncthreads();                                     // the previous tile is done with toks
+      for (int i = threadIdx.x; i < kBM; i += kThreads) {
+        int t = -1;
+        if (i < tc.rows) {
+          t = __ldg(token_of_row + tc.row0 + i);
+          if ((unsigned)t >= (unsigned)n_tokens) {
+            record_error(err, MOE_DEVERR_ROW);
+            t = -1;
+          }
+        }
+        toks[i] = t;
+      }
+      __syncthreads();
+    }
     float acc[4][4], accu[4][4];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
@@ -76,7 +95,8 @@ grouped_simt_kernel(const DT* __restrict__ A, const DT* __restrict__ B, const in
       for (int i = threadIdx.x; i < kBM * kBK; i += kThreads) {
         const int r = i / kBK, kk = i % kBK;
         float v = 0.f;
-        if (r < tc.rows && k0 + kk < K) v = ld_elem(A + (long long)(tc.row0 + r) * K + k0 + kk);
+        const long long arow = MODE == 3 ? (long long)toks[r] : (long long)(tc.row0 + r);
+        if (r < tc.rows && arow >= 0 && k0 + kk < K) v = ld_elem(A + arow * K + k0 + kk);
         As[kk][r] = v;
       }
       for (int i = threadIdx.x; i < kBN * kBK; i += kThreads) {
@@ -84,10 +104,10 @@ grouped_simt_kernel(const DT* __restrict__ A, const DT* __restrict__ B, const in
         float g = 0.f, u = 0.f;
         if (n0 + n < N && k0 + kk < K) {
           g = ld_elem(Be + (long long)(n0 + n) * K + k0 + kk);
-          if (MODE == 0) u = ld_elem(Be + (long long)(F + n0 + n) * K + k0 + kk);
+          if (GU) u = ld_elem(Be + (long long)(F + n0 + n) * K + k0 + kk);
         }
         Bs[kk][n] = g;
-        if (MODE == 0) Us[kk][n] = u;
+        if (GU) Us[kk][n] = u;
       }
       __syncthreads();
 #pragma unroll
@@ -99,7 +119,7 @@ grouped_simt_kernel(const DT* __restrict__ A, const DT* __restrict__ B, const in
         for (int i = 0; i < 4; ++i)
 #pragma unroll
           for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
-        if (MODE == 0) {
+        if (GU) {
           const float4 u = *reinterpret_cast<const float4*>(&Us[kk][tx * 4]);
           const float uv[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
@@ -114,7 +134,7 @@ grouped_simt_kernel(const DT* __restrict__ A, const DT* __restrict__ B, const in
       const int r = ty * 4 + i;
       if (r >= tc.rows) continue;
       const long long row = tc.row0 + r;
-      const float gsc = (MODE != 0 && gate_of_row) ? __ldg(gate_of_row + row) : 1.f;
+      const float gsc = (!GU && gate_of_row) ? __ldg(gate_of_row + row) : 1.f;
       int tok = 0;
       if (MODE == 2) {
         tok = __ldg(token_of_row + row);
@@ -128,7 +148,7 @@ grouped_simt_kernel(const DT* __restrict__ A, const DT* __restrict__ B, const in
         const int n = n0 + tx * 4 + j;
         if (n >= N) continue;
         float v;
-        if (MODE == 0) {
+        if (GU) {
           const float g = acc[i][j];
           v = g / (1.f + expf(-g)) * accu[i][j];
         } else {
@@ -183,6 +203,16 @@ moe_status launch_down_combine_simt(const void* h, int dtype, const int32_t* off
     return run_simt<float, 2, float>(h, W_dn, offsets, E, F, d, F, rows_max, gate_of_row, y, s, token_of_row, T);
   return run_simt<__nv_bfloat16, 2, float>(h, W_dn, offsets, E, F, d, F, rows_max, gate_of_row, y, s, token_of_row,
                                           T);
+}
+
+moe_status launch_gate_up_gather_simt(const void* x, int dtype, const int32_t* token_of_row, int T,
+                                      const int32_t* offsets, int E, int d, int F, long long rows_max,
+                                      const void* W_gu, void* h, cudaStream_t s) {
+  if (rows_max == 0 || T == 0) return MOE_OK;
+  if (dtype == MOE_F32)
+    return run_simt<float, 3, float>(x, W_gu, offsets, E, d, F, F, rows_max, nullptr, h, s, token_of_row, T);
+  return run_simt<__nv_bfloat16, 3, __nv_bfloat16>(x, W_gu, offsets, E, d, F, F, rows_max, nullptr, h, s,
+                                                  token_of_row, T);
 }
 
 }  // namespace moe

@@ -16,6 +16,10 @@
 //       row of its token (y[token_of_row[r]] += ...) with 16-byte vector atomics, so the
 //       gated rows never reach memory and no separate combine pass runs.  The fp32 sum
 //       order over a token's experts is whatever order the tiles finish in.
+//   MODE 4 (gate_up, gathered): as MODE 0, but the A rows are gathered straight from the
+//       token matrix, A row r = x[token_of_row[r]], so no permuted copy of x is written
+//       or read.  The producer warp copies them with 16-byte cp.async into the same
+//       128-byte-swizzled layout TMA writes; B still arrives by TMA.
 //   MODE 2 (router logits on the tensor cores, see below).
 //
 // Per CTA (1 per SM, 192 threads):
@@ -125,6 +129,30 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
       : "memory");
+}
+
+// 16-byte cp.async global -> shared; src_bytes = 0 writes zeros without reading.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+// Arrive on the mbarrier once all of this thread's earlier cp.async copies have landed
+// (the barrier's expected count includes this arrival: .noinc).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+// Orders generic-proxy shared-memory writes this thread has observed (here: other
+// threads' cp.async copies, acquired through an mbarrier) before its later async-proxy
+// accesses (the tensor cores read operands through the async proxy).
+__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// Output column tiles per row tile: 128 H features per gate/up tile (128 gate + 128 up
+// accumulator columns), 256 outputs per down tile, 64 experts per router tile.
+template <int MODE>
+__host__ __device__ __forceinline__ int n_tiles_of(int F, int N_out) {
+  if (MODE == 0 || MODE == 4) return (F + 127) / 128;
+  if (MODE == 1 || MODE == 3) return (N_out + BN - 1) / BN;
+  return (N_out + 63) / 64;
 }
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -271,11 +299,25 @@ __device__ __forceinline__ void stage_store32(uint8_t* stage, const float (&v)[3
   __syncwarp();
 }
 
+// L2 policy that keeps lines resident ahead of streaming data (the fp32 output rows the
+// fused combine adds into are touched by every expert of their token).
+__device__ __forceinline__ uint64_t l2_evict_last_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+// 16-byte vector atomic add (no return value) with an L2 cache policy.
+__device__ __forceinline__ void red_add_v4(float* p, const float4& v, uint64_t pol) {
+  asm volatile("red.global.add.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p), "f"(v.x), "f"(v.y),
+               "f"(v.z), "f"(v.w), "l"(pol)
+               : "memory");
+}
+
 // MODE 3: the same turn-around, then each 16-byte piece is added into the output row of
 // its token (tok: this lane's row's token, -1 = skip).  Every atomic instruction of the
 // warp covers 4 rows x 128 contiguous bytes.
 __device__ __forceinline__ void stage_red32(uint8_t* stage, const float (&v)[32], int lane, float* y, int tok,
-                                            long long ld, int col, int ncols) {
+                                            long long ld, int col, int ncols, uint64_t pol) {
   float4* dst = reinterpret_cast<float4*>(stage + lane * kStagePitchF32);
 #pragma unroll
   for (int q = 0; q < 8; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
@@ -286,8 +328,7 @@ __device__ __forceinline__ void stage_red32(uint8_t* stage, const float (&v)[32]
     const int r = i * 4 + rs;
     const int t = __shfl_sync(0xffffffffu, tok, r);
     const float4 x = *reinterpret_cast<const float4*>(stage + r * kStagePitchF32 + cv * 16);
-    if (t >= 0 && col + cv * 4 + 4 <= ncols)
-      atomicAdd(reinterpret_cast<float4*>(y + (long long)t * ld + col + cv * 4), x);
+    if (t >= 0 && col + cv * 4 + 4 <= ncols) red_add_v4(y + (long long)t * ld + col + cv * 4, x, pol);
   }
   __syncwarp();
 }
@@ -309,6 +350,7 @@ __device__ __forceinline__ void epilogue_tile(uint32_t taddr, uint8_t* stage, in
   if constexpr (MODE == 3) {
     const int n0 = n_tile * BN;
     const float gs = (lane < wrows && gate_of_row) ? __ldg(gate_of_row + wrow0 + lane) : 1.f;
+    const uint64_t pol = l2_evict_last_policy();
     int tok = -1;
     if (lane < wrows) {
       tok = __ldg(token_of_row + wrow0 + lane);
@@ -326,9 +368,9 @@ __device__ __forceinline__ void epilogue_tile(uint32_t taddr, uint8_t* stage, in
       float y[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) y[i] = __uint_as_float(v32[i]) * gs;
-      stage_red32(stage, y, lane, reinterpret_cast<float*>(out), tok, N_out, n0 + c * 32, N_out);
+      stage_red32(stage, y, lane, reinterpret_cast<float*>(out), tok, N_out, n0 + c * 32, N_out, pol);
     }
-  } else if constexpr (MODE == 0) {
+  } else if constexpr (MODE == 0 || MODE == 4) {
     const int f0 = n_tile * 128;
 #pragma unroll 1
     for (int c = 0; c < 4; ++c) {
@@ -384,13 +426,89 @@ __device__ __forceinline__ void epilogue_tile(uint32_t taddr, uint8_t* stage, in
   }
 }
 
+// Producer warp of the gathered gate/up GEMM (MODE 4).  Per stage, lane 0 arms the full
+// barrier with the B bytes and issues B's TMA loads; every lane copies its share of the
+// 128 A rows (lane = 16-byte chunk lane & 7 of rows lane >> 3, +4, +8, ...), each row
+// x[token_of_row[r]][k-block], with cp.async into the 128-byte-swizzled layout: chunk c
+// of row r lands at r * 128 + ((c ^ (r & 7)) * 16).  Rows past the tile and columns past
+// K are zero-filled.  Each lane then queues a hardware arrival on the stage's full
+// barrier that fires when its copies have landed (count 1 + 32), so the warp moves on
+// to the next stage at once; the MMA thread fences the stage for the async proxy after
+// its wait.
+// (Measured: slower than the permute copy plus the box-loaded GEMM, because every A tile
+// is re-read once per n-tile as 128-byte rows; it saves the permuted buffer.)
+__device__ __forceinline__ void gather_producer(const CUtensorMap* tmB, uint32_t sb, uint32_t bar_full,
+                                                uint32_t bar_empty, const int* tile_start,
+                                                const int32_t* __restrict__ offsets, int E, int K, int F,
+                                                const int32_t* __restrict__ token_of_row, int n_tokens,
+                                                const __nv_bfloat16* __restrict__ x, volatile int* abort_flag,
+                                                int* err) {
+  const int lane = threadIdx.x & 31;
+  const int cv = lane & 7, rsub = lane >> 3;
+  const int KB = (K + BK - 1) / BK;
+  const int total = tile_start[E];
+  int stage = 0;
+  uint32_t phase = 0;
+  int last_phase[STAGES];
+#pragma unroll
+  for (int s = 0; s < STAGES; ++s) last_phase[s] = -1;
+  bool ok = true;
+  for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+    const TileCoord tc = tile_coord(tile_start, offsets, E, BM, tile);
+    int tok[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int r = i * 4 + rsub;
+      int t = -1;
+      if (r < tc.rows) {
+        t = __ldg(token_of_row + tc.row0 + r);
+        if ((unsigned)t >= (unsigned)n_tokens) {
+          record_error(err, MOE_DEVERR_ROW);
+          t = -1;
+        }
+      }
+      tok[i] = t;
+    }
+    const int g_row = tc.e * 2 * F + tc.n_tile * 128;
+    for (int kb = 0; kb < KB; ++kb) {
+      const bool got = mbar_wait(bar_empty + 8 * stage, phase ^ 1u, abort_flag, err);
+      if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+      const uint32_t full = bar_full + 8 * stage;
+      const uint32_t a_dst = sb + L::a + stage * A_STAGE;
+      if (lane == 0) {
+        const uint32_t b_dst = sb + L::b + stage * B_STAGE;
+        mbar_expect_tx(full, B_STAGE);
+        tma_load_2d(b_dst, tmB, full, kb * BK, g_row);
+        tma_load_2d(b_dst + B_STAGE / 2, tmB, full, kb * BK, g_row + F);
+        last_phase[stage] = (int)phase;
+      }
+      const int kcol = kb * BK + cv * 8;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int r = i * 4 + rsub;
+        const bool v = tok[i] >= 0 && kcol < K;
+        const __nv_bfloat16* src = x + (v ? (long long)tok[i] * K + kcol : 0LL);
+        cp_async16(a_dst + r * 128 + ((cv ^ (r & 7)) << 4), src, v ? 16u : 0u);
+      }
+      cp_async_arrive_noinc(full);
+      if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+    }
+  }
+  cp_async_wait_all();                      // no copy may land after the CTA has exited
+  if (!ok && lane == 0) {
+    // let every issued B copy land before the CTA can exit
+    for (int s = 0; s < STAGES; ++s)
+      if (last_phase[s] >= 0) mbar_wait_drain(bar_full + 8 * s, (uint32_t)last_phase[s], err);
+  }
+}
+
 template <int MODE, typename OutT>
 __global__ void __launch_bounds__(kThreadsTC, 1)
 grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                        const int32_t* __restrict__ offsets, int E, int K, int N_out, int F,
                        long long rows_max, const float* __restrict__ gate_of_row,
                        OutT* __restrict__ out, const int32_t* __restrict__ token_of_row, int n_tokens,
-                       int* err) {
+                       const __nv_bfloat16* __restrict__ a_gather, int* err) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
@@ -400,8 +518,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::misc + 4);
 
-  // MODE 0: 128 H columns per tile (128 gate + 128 up accumulator columns)
-  const int n_tiles = MODE == 0 ? (F + 127) / 128 : ((MODE == 1 || MODE == 3) ? (N_out + BN - 1) / BN : (N_out + 63) / 64);
+  const int n_tiles = n_tiles_of<MODE>(F, N_out);
   build_tile_starts(offsets, E, BM, n_tiles, rows_max, tile_start, sh32, err);
   const int total = tile_start[E];
   if ((int)blockIdx.x >= total) return;   // uniform: nothing allocated yet
@@ -414,7 +531,8 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(bar_full + 8 * s, 1);
+      // gathered A: the B expect_tx arrival plus one cp.async arrival per producer lane
+      mbar_init(bar_full + 8 * s, MODE == 4 ? 1 + 32 : 1);
       mbar_init(bar_empty + 8 * s, 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -437,7 +555,10 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
   const uint32_t tmem_base = *tmem_slot;
   const int KB = (K + BK - 1) / BK;
 
-  if (warp == 0) {
+  if (MODE == 4 && warp == 0) {
+    gather_producer(&tmB, sb, bar_full, bar_empty, tile_start, offsets, E, K, F, token_of_row, n_tokens, a_gather,
+                    abort_flag, err);
+  } else if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       int stage = 0;
@@ -490,6 +611,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag, err)) { ok = false; break; }
           tc_fence_after();
+          if (MODE == 4) fence_proxy_async_smem();   // A rows were written by cp.async (generic proxy)
           const uint64_t adesc = sw128_desc(sb + L::a + stage * A_STAGE);
           const uint64_t bdesc = sw128_desc(sb + L::b + stage * B_STAGE);
 #pragma unroll
@@ -584,7 +706,7 @@ grouped_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
   const int cid = (int)(blockIdx.x >> 1), ncl = (int)(gridDim.x >> 1);
   constexpr int PM = 2 * BM;                                 // rows per pair tile
 
-  const int n_tiles = MODE == 0 ? (F + 127) / 128 : ((MODE == 1 || MODE == 3) ? (N_out + BN - 1) / BN : (N_out + 63) / 64);
+  const int n_tiles = n_tiles_of<MODE>(F, N_out);
   build_tile_starts(offsets, E, PM, n_tiles, rows_max, tile_start, sh32, err);
   const int total = tile_start[E];
   if (cid >= total) return;   // both CTAs of the pair see the same cid: uniform, nothing allocated
@@ -749,7 +871,8 @@ bool make_map(CUtensorMap* m, const void* ptr, unsigned long long rows, unsigned
 template <int MODE, typename OutT>
 moe_status launch_tc(const CUtensorMap& ma, const CUtensorMap& mb, const int32_t* offsets, int E, int K, int N_out,
                      int F, long long rows_max, const float* gate_of_row, void* out, cudaStream_t s,
-                     const int32_t* token_of_row = nullptr, int n_tokens = 0) {
+                     const int32_t* token_of_row = nullptr, int n_tokens = 0,
+                     const __nv_bfloat16* a_gather = nullptr) {
   static int configured[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -760,14 +883,14 @@ moe_status launch_tc(const CUtensorMap& ma, const CUtensorMap& mb, const int32_t
     if (e != cudaSuccess) return cuda_status(e);
     configured[dev] = 1;
   }
-  const int n_tiles = MODE == 0 ? (F + 127) / 128 : ((MODE == 1 || MODE == 3) ? (N_out + BN - 1) / BN : (N_out + 63) / 64);
+  const int n_tiles = n_tiles_of<MODE>(F, N_out);
   const long long max_tiles = ((rows_max + BM - 1) / BM + E) * (long long)n_tiles;
   int grid = num_sms();
   if (max_tiles < grid) grid = (int)max_tiles;
   if (grid < 1) grid = 1;
   grouped_gemm_tc_kernel<MODE, OutT><<<grid, kThreadsTC, kSmemBytes, s>>>(
       ma, mb, offsets, E, K, N_out, F, rows_max, gate_of_row, static_cast<OutT*>(out), token_of_row, n_tokens,
-      err_ptr());
+      a_gather, err_ptr());
   return check_launch();
 }
 
@@ -794,7 +917,7 @@ moe_status launch_tc2(const CUtensorMap& ma, const CUtensorMap& mb, const int32_
     if (e != cudaSuccess) return cuda_status(e);
     configured[dev] = 1;
   }
-  const int n_tiles = MODE == 0 ? (F + 127) / 128 : ((MODE == 1 || MODE == 3) ? (N_out + BN - 1) / BN : (N_out + 63) / 64);
+  const int n_tiles = n_tiles_of<MODE>(F, N_out);
   const long long max_tiles = ((rows_max + 2 * BM - 1) / (2 * BM) + E) * (long long)n_tiles;
   int pairs = num_sms() / 2;
   if (max_tiles < pairs) pairs = (int)max_tiles;
@@ -871,6 +994,19 @@ moe_status launch_down_combine_tc(const void* h, const int32_t* offsets, int E, 
   if (!make_map(&mb, W_dn, (unsigned long long)E * d, F, pair ? BM : BN)) return MOE_ERR_UNSUPPORTED;
   if (pair) return launch_tc2<3, float>(ma, mb, offsets, E, F, d, F, rows_max, gate_of_row, y, s, token_of_row, T);
   return launch_tc<3, float>(ma, mb, offsets, E, F, d, F, rows_max, gate_of_row, y, s, token_of_row, T);
+}
+
+// Gate/up GEMM with the dispatch fused into its producer: A row r = x[token_of_row[r]]
+// (x [T, d] bf16), no permuted copy of x.  Single-CTA tiles (the gather producer fills
+// one CTA's stages).
+moe_status launch_gate_up_gather_tc(const void* x, const int32_t* token_of_row, int T, const int32_t* offsets, int E,
+                                    int d, int F, long long rows_max, const void* W_gu, void* h, cudaStream_t s) {
+  if (rows_max == 0 || T == 0) return MOE_OK;
+  if (d < BK || F < 8) return MOE_ERR_UNSUPPORTED;
+  CUtensorMap mb;
+  if (!make_map(&mb, W_gu, (unsigned long long)E * 2 * F, d, 128)) return MOE_ERR_UNSUPPORTED;
+  return launch_tc<4, __nv_bfloat16>(mb, mb, offsets, E, d, F, F, rows_max, nullptr, h, s, token_of_row, T,
+                                     static_cast<const __nv_bfloat16*>(x));
 }
 
 }  // namespace moe

@@ -3,7 +3,9 @@
 MoELayer owns preallocated device buffers for a maximum token count and runs, on one
 stream with no host synchronisation:
 
-    moe_route -> moe_histogram_scan -> moe_permute -> moe_expert_gate_up
+    moe_route -> moe_histogram_scan
+      dispatch="permute": -> moe_permute -> moe_expert_gate_up
+      dispatch="gather":  -> moe_expert_gate_up_gather (reads x through the row map)
       combine="rows":  -> moe_expert_down (gate fused) [-> shared expert: gate_up/down
                        with E = 1] -> moe_combine
       combine="fused": [-> shared expert, written into y] -> moe_expert_down_combine
@@ -40,11 +42,16 @@ class MoELayer:
     def __init__(self, weights: MoEWeights, k: int, T_max: int, score: str = "softmax",
                  renormalize: bool = True, scale: float = 1.0, capacity: int = -1,
                  rows_dtype: torch.dtype = torch.float32, out_dtype: torch.dtype = torch.float32,
-                 combine: str = "rows"):
+                 combine: str = "rows", dispatch: str = "permute"):
         """rows_dtype: gated expert rows (and the shared expert's output); out_dtype: y.
         fp32 (the default) leaves H as the only bf16 rounding inside the layer.
         combine: "rows" (gated rows + ordered combine) or "fused" (down GEMM adds into an
-        fp32 y; needs out_dtype fp32)."""
+        fp32 y; needs out_dtype fp32).
+        dispatch: "permute" (x_perm copy, then the GEMM) or "gather" (the GEMM reads the
+        token rows through token_of_row; same H bit for bit)."""
+        if dispatch not in ("permute", "gather"):
+            raise ValueError(f"dispatch must be 'permute' or 'gather', got {dispatch!r}")
+        self.dispatch_mode = dispatch
         if combine not in ("rows", "fused"):
             raise ValueError(f"combine must be 'rows' or 'fused', got {combine!r}")
         if combine == "fused" and out_dtype != torch.float32:
@@ -73,7 +80,7 @@ class MoELayer:
         self.row_of = torch.empty((T_max, k), dtype=i32, device=dev)
         self.token_of_row = torch.empty(R, dtype=i32, device=dev)
         self.gate_of_row = torch.empty(R, dtype=f32, device=dev)
-        self.x_perm = torch.empty((R, d), dtype=self.dtype, device=dev)
+        self.x_perm = torch.empty((R, d), dtype=self.dtype, device=dev) if dispatch == "permute" else None
         self.h = torch.empty((R, F), dtype=self.dtype, device=dev)
         self.y_perm = torch.empty((R, d), dtype=rows_dtype, device=dev) if combine == "rows" else None
         self.y = torch.empty((T_max, d), dtype=out_dtype, device=dev)
@@ -102,6 +109,9 @@ class MoELayer:
 
     def gate_up(self, stream=None):
         M.moe_expert_gate_up(self.x_perm, self.offsets, self.w.W_gu, self.rows_max, self.h, stream)
+
+    def gate_up_gather(self, x, stream=None):
+        M.moe_expert_gate_up_gather(x, self.token_of_row, self.offsets, self.w.W_gu, self.rows_max, self.h, stream)
 
     def down(self, stream=None):
         M.moe_expert_down(self.h, self.offsets, self.w.W_dn, self.rows_max, self.gate_of_row, self.y_perm,
@@ -132,9 +142,11 @@ class MoELayer:
         """The forward as (name, fn(stream)) steps in launch order."""
         T = x.shape[0]
         st = [("route", lambda s: self.route(x, s)),
-              ("histogram_scan", lambda s: self.histogram_scan(T, s)),
-              ("permute", lambda s: self.permute(x, s)),
-              ("gate_up", lambda s: self.gate_up(s))]
+              ("histogram_scan", lambda s: self.histogram_scan(T, s))]
+        if self.dispatch_mode == "permute":
+            st += [("permute", lambda s: self.permute(x, s)), ("gate_up", lambda s: self.gate_up(s))]
+        else:
+            st.append(("gate_up_gather", lambda s: self.gate_up_gather(x, s)))
         if self.combine_mode == "rows":
             st.append(("down", lambda s: self.down(s)))
             if self.has_shared:
@@ -187,6 +199,8 @@ class MoELayer:
         n = 2 + 2 + 1 + 1 + 1 + 1          # route(2) scan(2) permute gate_up down combine
         if self.combine_mode == "fused":
             n -= 1                         # down_combine (its zero fill is a memset, not a kernel)
+        if self.dispatch_mode == "gather":
+            n -= 1                         # no permute
         if self.has_shared:
             n += 2
         if with_stats:

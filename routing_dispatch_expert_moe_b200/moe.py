@@ -44,6 +44,8 @@ _SIGNATURES = {
     "moe_permute": (_i32, [_c_void_p, _i32, _i32, _i32, _i32, _c_void_p, _i64, _c_void_p, _c_void_p]),
     "moe_expert_gate_up": (_i32, [_c_void_p, _i32, _c_void_p, _i32, _i32, _i32, _i64, _c_void_p, _c_void_p,
                                   _c_void_p]),
+    "moe_expert_gate_up_gather": (_i32, [_c_void_p, _i32, _i32, _c_void_p, _c_void_p, _i32, _i32, _i32, _i64,
+                                         _c_void_p, _c_void_p, _c_void_p]),
     "moe_expert_down": (_i32, [_c_void_p, _i32, _c_void_p, _i32, _i32, _i32, _i64, _c_void_p, _c_void_p,
                                _i32, _c_void_p, _c_void_p]),
     "moe_grouped_ffn": (_i32, [_c_void_p, _i32, _c_void_p, _i32, _i32, _i32, _i64, _c_void_p, _c_void_p,
@@ -237,6 +239,23 @@ def moe_expert_gate_up(x_rows, offsets, W_gu, rows_max: int, h=None, stream=None
         _need(h, "h", x_rows.dtype)
     _check("moe_expert_gate_up", lib().moe_expert_gate_up(_p(x_rows), _dt(x_rows), _p(offsets), E, d, F, rows_max,
                                                           _p(W_gu), _p(h), _stream(stream)))
+    return h
+
+
+def moe_expert_gate_up_gather(x, token_of_row, offsets, W_gu, rows_max: int, h=None, stream=None):
+    """H = silu(X Wg^T) * (X Wu^T) with X[r] = x[token_of_row[r]]: the permute fused into the GEMM."""
+    E, F2, d = W_gu.shape
+    F = F2 // 2
+    _need(x, "x")
+    if x.dim() != 2 or x.shape[1] != d:
+        raise ValueError(f"x must be [T, {d}]")
+    _need(token_of_row, "token_of_row", torch.int32)
+    _need(offsets, "offsets", torch.int32, (E + 1,))
+    _need(W_gu, "W_gu", x.dtype)
+    h = torch.empty((max(rows_max, 1), F), dtype=x.dtype, device=x.device) if h is None else _need(h, "h", x.dtype)
+    _check("moe_expert_gate_up_gather",
+           lib().moe_expert_gate_up_gather(_p(x), _dt(x), x.shape[0], _p(token_of_row), _p(offsets), E, d, F,
+                                           rows_max, _p(W_gu), _p(h), _stream(stream)))
     return h
 
 

@@ -71,18 +71,20 @@ def expert_getters(host):
     return gu, dn
 
 
-def build_layer(cfg, dev, capacity, rows_dtype=torch.float32, out_dtype=torch.float32, combine="rows"):
+def build_layer(cfg, dev, capacity, rows_dtype=torch.float32, out_dtype=torch.float32, combine="rows",
+                dispatch="permute"):
     from routing_dispatch_expert_moe_b200.layer import MoELayer, MoEWeights
     w = MoEWeights(Wg=dev["Wg"], W_gu=dev["W_gu"], W_dn=dev["W_dn"], logit_offset=dev["off"],
                    select_bias=dev["bias"], W_gu_s=dev["W_gu_s"], W_dn_s=dev["W_dn_s"])
     return MoELayer(w, cfg.k, cfg.T, cfg.score, cfg.renormalize, cfg.scale, capacity, rows_dtype, out_dtype,
-                    combine)
+                    combine, dispatch)
 
 
-def gpu_forward(cfg, dev, capacity, rows_dtype=torch.float32, out_dtype=torch.float32, combine="rows"):
+def gpu_forward(cfg, dev, capacity, rows_dtype=torch.float32, out_dtype=torch.float32, combine="rows",
+                dispatch="permute"):
     """Runs the layer through the C ABI; returns the layer object and host copies of every output."""
     from routing_dispatch_expert_moe_b200 import moe as M
-    layer = build_layer(cfg, dev, capacity, rows_dtype, out_dtype, combine)
+    layer = build_layer(cfg, dev, capacity, rows_dtype, out_dtype, combine, dispatch)
     y = layer.forward(dev["x"])
     torch.cuda.synchronize()
     code = M.moe_get_device_error()

@@ -132,6 +132,12 @@ def test_ffn_host_validation(L):
     g = L.moe_expert_down
     assert g(FAKE, 0, FAKE, 4, 128, 64, -1, FAKE, NUL, 1, FAKE, NUL) == 1
     assert g(FAKE, 0, FAKE, 4, 128, 64, 128, FAKE, NUL, 7, FAKE, NUL) == 1        # y dtype
+    q = L.moe_expert_gate_up_gather    # (x, dt, T, tok, offs, E, d, F, rows_max, W_gu, h, s)
+    assert q(FAKE, 0, -1, FAKE, FAKE, 4, 128, 64, 128, FAKE, FAKE, NUL) == 1       # T < 0
+    assert q(FAKE, 0, 64, NUL, FAKE, 4, 128, 64, 128, FAKE, FAKE, NUL) == 1        # token_of_row
+    assert q(FAKE, 0, 64, FAKE, FAKE, 4, 100, 64, 128, FAKE, FAKE, NUL) == 2       # d % 8
+    assert q(ctypes.c_void_p(4098), 0, 64, FAKE, FAKE, 4, 128, 64, 128, FAKE, FAKE, NUL) == 2   # alignment
+    assert q(FAKE, 0, 0, FAKE, FAKE, 4, 128, 64, 128, FAKE, FAKE, NUL) == 0        # no tokens
     h = L.moe_expert_down_combine      # (h, dt, offs, E, d, F, rows_max, W_dn, gate, tok, T, accumulate, y, s)
     assert h(FAKE, 0, FAKE, 4, 128, 64, 128, FAKE, NUL, FAKE, 64, 2, FAKE, NUL) == 1      # accumulate flag
     assert h(FAKE, 0, FAKE, 4, 128, 64, 128, FAKE, NUL, FAKE, -1, 0, FAKE, NUL) == 1      # T < 0

@@ -333,12 +333,13 @@ def test_fused_bad_token_is_reported_not_trapped():
         assert M.moe_get_device_error() == 3
 
 
-def fused_full_size_check(name):
+def fused_full_size_check(name, per_assignment=True):
+    """Both fusions (gathered gate/up, combine inside the down GEMM): the form bench.py times."""
     cfg = I.CONFIGS[name]
     host, dev = U.make_inputs(cfg)
-    cap = O.capacity(cfg.T, cfg.E, cfg.k, cfg.capacity_factor, True)
-    layer, g = U.gpu_forward(cfg, dev, cap, combine="fused")
-    o = O.layer_routing(U.cfg_dict(cfg), host["x"], host["Wg"], host["off"], host["bias"], True)
+    cap = O.capacity(cfg.T, cfg.E, cfg.k, cfg.capacity_factor, per_assignment)
+    layer, g = U.gpu_forward(cfg, dev, cap, combine="fused", dispatch="gather")
+    o = O.layer_routing(U.cfg_dict(cfg), host["x"], host["Wg"], host["off"], host["bias"], per_assignment)
     U.assert_routing_equal(g, o)
     toks = U.stratified_tokens(o, cap)
     gu, dn = U.expert_getters(host)
@@ -356,3 +357,39 @@ def test_c2_handbook_full_size_fused_combine():
 @pytest.mark.slow
 def test_c3_fine_grained_full_size_fused_combine():
     fused_full_size_check("c3_fine_grained")
+
+
+@pytest.mark.slow
+def test_c5_stress_full_size_fused_literal_capacity():
+    fused_full_size_check("c5_stress", per_assignment=False)
+
+
+# ---------------------------------------------------------------- permute fused into the gate/up GEMM
+GATHER = [c for c in SMALL if c.name in ("softmax_bf16", "sigmoid_bias_shared", "sqrt_softplus_capacity_zipf",
+                                          "ragged_multitile", "fp32_small", "bf16_d_below_tile",
+                                          "sigmoid_nobias_E_odd")]
+
+
+@pytest.mark.parametrize("cfg", GATHER, ids=lambda c: c.name)
+def test_gathered_gate_up_is_bitwise_the_permuted_one(cfg):
+    """Same A rows, same tiles, same accumulation order: H and the reproducible y agree bit for bit."""
+    host, dev = U.make_inputs(cfg)
+    cap = O.capacity(cfg.T, cfg.E, cfg.k, cfg.capacity_factor, True)
+    lp, gp = U.gpu_forward(cfg, dev, cap)
+    lg, gg = U.gpu_forward(cfg, dev, cap, dispatch="gather")
+    n = gp["n_rows"]
+    assert gg["n_rows"] == n
+    assert torch.equal(lp.h[:n], lg.h[:n]), "H differs between the gathered and the permuted GEMM"
+    assert np.array_equal(gp["y"], gg["y"])
+
+
+def test_gathered_bad_token_is_reported_not_trapped():
+    from routing_dispatch_expert_moe_b200 import moe as M
+    for cfg in (SMALL[0], SMALL[6]):                          # tensor-core and fp32 SIMT forms
+        host, dev = U.make_inputs(cfg)
+        layer, g = U.gpu_forward(cfg, dev, -1, dispatch="gather")
+        tok = layer.token_of_row.clone()
+        tok[3] = -5                                            # outside [0, T): zero row, recorded
+        M.moe_expert_gate_up_gather(dev["x"], tok, layer.offsets, layer.w.W_gu, layer.rows_max, layer.h)
+        torch.cuda.synchronize()
+        assert M.moe_get_device_error() == 3
