@@ -168,36 +168,39 @@ def run_ours(args):
         return MoELayer(w, cfg.k, cfg.T, cfg.score, cfg.renormalize, cfg.scale, cap, combine=combine,
                         dispatch=dispatch)
 
-    def time_layer(layer, steps, clocks=None):
-        """Warm-up, then `steps` replays of one forward captured as a CUDA graph whose timing
-        events are nodes inside the graph, on the stream the kernels run on.  L2 is flushed
-        (256 MB write) before every step, outside the timed span.  Returns per-step ms,
+    def capture(fn):
+        """One CUDA graph of fn(stream), captured on a side stream."""
+        g = torch.cuda.CUDAGraph()
+        cs = torch.cuda.Stream()
+        cs.wait_stream(stream)
+        with torch.cuda.stream(cs):
+            with torch.cuda.graph(g, stream=cs):
+                fn(cs)
+        stream.wait_stream(cs)
+        return g
+
+    def time_layer(layer, steps, clocks=None, breakdown_steps=0):
+        """Warm-up, then `steps` replays of one forward (the layer's own schedule, including
+        its second branch) captured as a CUDA graph with timing events as graph nodes on
+        the launching stream.  L2 is flushed (256 MB write) before every step, outside the
+        timed span.  breakdown_steps > 0: the same kernels replayed one stage after the
+        other with an event between stages, for the per-stage split.  Returns per-step ms,
         mean ms per stage, the rows processed and the clock record."""
-        stages = layer.stages(x)
-        names = [n for n, _ in stages]
-
-        def step(s, evs=None):
-            for i, (_, fn) in enumerate(stages):
-                if evs is not None:
-                    evs[i].record(s)
-                fn(s)
-            if evs is not None:
-                evs[len(stages)].record(s)
-
         for _ in range(args.warmup):
             flush.zero_()
-            step(stream)
+            layer.forward(x, stream)
         torch.cuda.synchronize()
         assert M.moe_get_device_error() == 0
         rows = int(layer.offsets[-1].item())
-        evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(stages) + 1)]
-        graph = torch.cuda.CUDAGraph()
-        cap_stream = torch.cuda.Stream()
-        cap_stream.wait_stream(stream)
-        with torch.cuda.stream(cap_stream):
-            with torch.cuda.graph(graph, stream=cap_stream):
-                step(cap_stream, evs)
-        stream.wait_stream(cap_stream)
+        ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
+        gu_name = "gate_up_gather" if layer.dispatch_mode == "gather" else "gate_up"
+
+        def fwd(s):
+            ev[0].record(s)
+            layer.forward(x, s, marks={gu_name: (ev[2], ev[3])})
+            ev[1].record(s)
+
+        graph = capture(fwd)
         for _ in range(3):
             flush.zero_()
             graph.replay()
@@ -209,20 +212,42 @@ def run_ours(args):
             dist.barrier()
         torch.cuda.synchronize()
         per_step = np.zeros(steps)
-        acc = np.zeros(len(stages))
+        gu_ms = 0.0
         for i in range(steps):
             flush.zero_()                      # L2 flush outside the step
             graph.replay()
             torch.cuda.synchronize()           # read this step's in-graph events
-            per_step[i] = evs[0].elapsed_time(evs[-1])
-            acc += [evs[j].elapsed_time(evs[j + 1]) for j in range(len(stages))]
+            per_step[i] = ev[0].elapsed_time(ev[1])
+            gu_ms += ev[2].elapsed_time(ev[3])
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
         clk = clocks.stop() if clocks is not None else None
         assert M.moe_get_device_error() == 0
         del graph
-        return per_step, {n: float(acc[j] / steps) for j, n in enumerate(names)}, rows, clk
+
+        stage_ms = {"timed_" + gu_name: gu_ms / steps}
+        if breakdown_steps > 0:
+            stages = layer.stages(x)
+            evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(stages) + 1)]
+
+            def seq(s):
+                for i, (_, fn) in enumerate(stages):
+                    evs[i].record(s)
+                    fn(s)
+                evs[len(stages)].record(s)
+
+            g2 = capture(seq)
+            acc = np.zeros(len(stages))
+            for i in range(breakdown_steps + 2):
+                flush.zero_()
+                g2.replay()
+                torch.cuda.synchronize()
+                if i >= 2:
+                    acc += [evs[j].elapsed_time(evs[j + 1]) for j in range(len(stages))]
+            stage_ms.update({n: float(acc[j] / breakdown_steps) for j, (n, _) in enumerate(stages)})
+            del g2
+        return per_step, stage_ms, rows, clk
 
     def max_over_ranks(v):
         if world > 1:
@@ -232,7 +257,8 @@ def run_ours(args):
         return v
 
     layer = make_layer(args.combine, args.dispatch)
-    per_step, stage_ms, A, clk = time_layer(layer, args.steps, ClockSampler(local_rank))
+    per_step, stage_ms, A, clk = time_layer(layer, args.steps, ClockSampler(local_rank),
+                                            breakdown_steps=args.breakdown_steps)
     total_ms = max_over_ranks(float(per_step.sum()))
     ms_per_step = total_ms / args.steps
     value = cfg.T * world * args.steps / (total_ms / 1e3)
@@ -241,7 +267,7 @@ def run_ours(args):
     if (args.combine, args.dispatch) != ("rows", "permute") and args.unfused_steps > 0:
         # the unfused form (permute copy, gated rows, ordered combine: bitwise reproducible), same inputs
         rl = make_layer("rows", "permute")
-        ps, sm, _, _ = time_layer(rl, args.unfused_steps)
+        ps, sm, _, _ = time_layer(rl, args.unfused_steps, breakdown_steps=min(args.breakdown_steps, 50))
         t = max_over_ranks(float(ps.sum()))
         other = {"dispatch": "permute", "combine": "rows (gated rows + ordered combine, bitwise reproducible)",
                  "ms_per_step": round(t / args.unfused_steps, 4),
@@ -278,7 +304,7 @@ def run_ours(args):
 
     pk, pk_src = peaks()
     gather = args.dispatch == "gather"
-    gate_up_ms = stage_ms["gate_up_gather" if gather else "gate_up"]
+    gate_up_ms = stage_ms["timed_gate_up_gather" if gather else "timed_gate_up"]   # inside the timed region
     flops = 4.0 * A * cfg.d * cfg.F
     achieved = flops / (gate_up_ms * 1e-3) / 1e12
     peak = pk["bf16_tflops"]
@@ -287,14 +313,17 @@ def run_ours(args):
     ob = layer.y.element_size()
     roof_ms, roof_steps = layer_roofline_ms(cfg, A, pk, rb, ob, fused, gather)
     traffic = GATE_UP_TRAFFIC.get((args.workload, args.dispatch))
-    down_ms = stage_ms["down_combine" if fused else "down"]
-    thr = {"down_tflops": round(2.0 * A * cfg.F * cfg.d / (down_ms * 1e-3) / 1e12, 1),
-           "route_gbs": round((cfg.T * cfg.d * 2 + cfg.T * cfg.E * 8 + cfg.T * cfg.k * 8) /
-                              (stage_ms["route"] * 1e-3) / 1e9, 1)}
-    if not gather:
-        thr["permute_gbs"] = round((cfg.T * cfg.d * 2 + A * cfg.d * 2) / (stage_ms["permute"] * 1e-3) / 1e9, 1)
-    if not fused:
-        thr["combine_gbs"] = round((A * cfg.d * rb + cfg.T * cfg.d * ob) / (stage_ms["combine"] * 1e-3) / 1e9, 1)
+    thr = {}                                # from the per-stage split, when it ran
+    if stage_ms.get("route"):
+        down_ms = stage_ms["down_combine" if fused else "down"]
+        thr["down_tflops"] = round(2.0 * A * cfg.F * cfg.d / (down_ms * 1e-3) / 1e12, 1)
+        thr["route_gbs"] = round((cfg.T * cfg.d * 2 + cfg.T * cfg.E * 8 + cfg.T * cfg.k * 8) /
+                                 (stage_ms["route"] * 1e-3) / 1e9, 1)
+        if not gather:
+            thr["permute_gbs"] = round((cfg.T * cfg.d * 2 + A * cfg.d * 2) / (stage_ms["permute"] * 1e-3) / 1e9, 1)
+        if not fused:
+            thr["combine_gbs"] = round((A * cfg.d * rb + cfg.T * cfg.d * ob) / (stage_ms["combine"] * 1e-3) / 1e9,
+                                       1)
 
     out = None
     if rank == 0:
@@ -444,6 +473,8 @@ def main():
                     help="fused: combine inside the down GEMM; rows: gated rows + ordered combine")
     ap.add_argument("--dispatch", choices=["gather", "permute"], default="permute",
                     help="gather: the gate/up GEMM reads token rows through the row map; permute: x_perm copy")
+    ap.add_argument("--breakdown-steps", type=int, default=100,
+                    help="sequential replays for the per-stage split (0 = skip)")
     ap.add_argument("--unfused-steps", type=int, default=100,
                     help="also time the unfused form (permute + rows) for this many steps (0 = skip)")
     args = ap.parse_args()

@@ -309,6 +309,13 @@ MOE_API moe_status moe_router_stats(const float* logits, const int32_t* counts, 
                             float* load, float* stats5,
                             void* workspace, size_t workspace_bytes, void* stream);
 
+/* moe_zero -- clears `bytes` bytes at p (device) with cudaMemsetAsync on stream: the
+ * initial value for moe_expert_down_combine(..., accumulate = 1) when the caller wants
+ * to clear y off the critical path (e.g. on a second stream).  p must be 16-byte
+ * aligned; bytes = 0 does nothing.  This step has no counterpart on the pages (it only
+ * initialises an output buffer). */
+MOE_API moe_status moe_zero(void* p, size_t bytes, void* stream);
+
 /* Largest workspace any of the calls above needs for these sizes. */
 MOE_API size_t moe_workspace_bytes(int32_t T, int32_t d, int32_t E, int32_t k);
 

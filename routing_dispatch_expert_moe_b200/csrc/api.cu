@@ -284,6 +284,13 @@ size_t moe_workspace_bytes(int32_t T, int32_t d, int32_t E, int32_t k) {
   return m > c ? m : c;
 }
 
+moe_status moe_zero(void* p, size_t bytes, void* stream) {
+  if (bytes == 0) return MOE_OK;
+  if (!p) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(p)) return MOE_ERR_UNSUPPORTED;
+  return cuda_status(cudaMemsetAsync(p, 0, bytes, S(stream)));
+}
+
 moe_status moe_get_device_error(int32_t* code, void* stream) {
   if (!code) return MOE_ERR_INVALID_ARG;
   *code = 0;

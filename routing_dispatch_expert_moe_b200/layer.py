@@ -42,13 +42,16 @@ class MoELayer:
     def __init__(self, weights: MoEWeights, k: int, T_max: int, score: str = "softmax",
                  renormalize: bool = True, scale: float = 1.0, capacity: int = -1,
                  rows_dtype: torch.dtype = torch.float32, out_dtype: torch.dtype = torch.float32,
-                 combine: str = "rows", dispatch: str = "permute"):
+                 combine: str = "rows", dispatch: str = "permute", overlap: bool = True):
         """rows_dtype: gated expert rows (and the shared expert's output); out_dtype: y.
         fp32 (the default) leaves H as the only bf16 rounding inside the layer.
         combine: "rows" (gated rows + ordered combine) or "fused" (down GEMM adds into an
         fp32 y; needs out_dtype fp32).
         dispatch: "permute" (x_perm copy, then the GEMM) or "gather" (the GEMM reads the
-        token rows through token_of_row; same H bit for bit)."""
+        token rows through token_of_row; same H bit for bit).
+        overlap: run the work nothing on the main path waits for (router statistics, and
+        clearing y for the fused combine) on a second stream forked from and joined back
+        to the caller's stream (one CUDA graph with two branches when captured)."""
         if dispatch not in ("permute", "gather"):
             raise ValueError(f"dispatch must be 'permute' or 'gather', got {dispatch!r}")
         self.dispatch_mode = dispatch
@@ -87,6 +90,10 @@ class MoELayer:
         self.load = torch.empty(E, dtype=f32, device=dev)
         self.stats5 = torch.empty(5, dtype=f32, device=dev)
         self.ws = torch.empty(max(M.moe_workspace_bytes(T_max, d, E, k), 16), dtype=torch.uint8, device=dev)
+        self.overlap = overlap
+        if overlap:
+            self._side = torch.cuda.Stream(device=dev)
+            self._ev_fork, self._ev_routed, self._ev_join = (torch.cuda.Event() for _ in range(3))
         self.has_shared = w.W_gu_s is not None
         if self.has_shared:
             self.F_s = w.W_dn_s.shape[2]
@@ -126,9 +133,11 @@ class MoELayer:
         M.moe_expert_gate_up(x, self.shared_offsets, self.w.W_gu_s, T, self.h_s[:T], stream)
         M.moe_expert_down(self.h_s[:T], self.shared_offsets, self.w.W_dn_s, T, None, out, stream=stream)
 
-    def down_combine(self, T, stream=None):
+    def down_combine(self, T, stream=None, accumulate=None):
+        """accumulate: add onto y as it stands (default: only when the shared expert wrote it)."""
+        acc = self.has_shared if accumulate is None else accumulate
         M.moe_expert_down_combine(self.h, self.offsets, self.w.W_dn, self.rows_max, self.token_of_row, self.y[:T],
-                                  self.gate_of_row, accumulate=self.has_shared, stream=stream)
+                                  self.gate_of_row, accumulate=acc, stream=stream)
 
     def combine(self, T, stream=None):
         M.moe_combine(self.y_perm, self.row_of[:T], T, self.rows_max, None,
@@ -160,14 +169,58 @@ class MoELayer:
             st.append(("stats", lambda s: self.stats(T, s)))
         return st
 
-    def forward(self, x: torch.Tensor, stream=None, with_stats: bool = True) -> torch.Tensor:
+    def forward(self, x: torch.Tensor, stream=None, with_stats: bool = True, marks=None) -> torch.Tensor:
+        """marks: optional {stage name: (event, event)} recorded on the main stream right
+        before and after that stage (for timing one kernel inside the real schedule)."""
         T = x.shape[0]
         if T > self.T_max:
             raise ValueError(f"T={T} exceeds T_max={self.T_max}")
         if x.dtype != self.dtype:
             raise ValueError(f"x must be {self.dtype}")
-        for _, fn in self.stages(x, with_stats):
-            fn(stream)
+        s = torch.cuda.current_stream() if stream is None else stream
+
+        def run(name, fn):
+            m = marks.get(name) if marks else None
+            if m is not None:
+                m[0].record(s)
+            fn(s)
+            if m is not None:
+                m[1].record(s)
+
+        if not self.overlap:
+            for name, fn in self.stages(x, with_stats):
+                run(name, fn)
+            return self.y[:T]
+        side = self._side
+        fused = self.combine_mode == "fused"
+        self._ev_fork.record(s)                  # everything the caller queued before (e.g. a read of y)
+        side.wait_event(self._ev_fork)
+        if fused and not self.has_shared:
+            M.moe_zero(self.y[:T], side)         # the fused combine's starting value, off the main path
+        run("route", lambda s_: self.route(x, s_))
+        run("histogram_scan", lambda s_: self.histogram_scan(T, s_))
+        if with_stats:
+            self._ev_routed.record(s)
+            side.wait_event(self._ev_routed)
+            self.stats(T, side)
+        if self.dispatch_mode == "permute":
+            run("permute", lambda s_: self.permute(x, s_))
+            run("gate_up", lambda s_: self.gate_up(s_))
+        else:
+            run("gate_up_gather", lambda s_: self.gate_up_gather(x, s_))
+        if fused:
+            if self.has_shared:
+                run("shared", lambda s_: self.shared(x, s_))
+            self._ev_join.record(side)
+            s.wait_event(self._ev_join)
+            run("down_combine", lambda s_: self.down_combine(T, s_, accumulate=True))
+        else:
+            run("down", lambda s_: self.down(s_))
+            if self.has_shared:
+                run("shared", lambda s_: self.shared(x, s_))
+            run("combine", lambda s_: self.combine(T, s_))
+            self._ev_join.record(side)
+            s.wait_event(self._ev_join)
         return self.y[:T]
 
     # ---------------------------------------------------------------- CUDA graph

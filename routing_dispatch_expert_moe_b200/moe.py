@@ -59,6 +59,7 @@ _SIGNATURES = {
                                 _c_void_p, _size, _c_void_p]),
     "moe_workspace_bytes": (_size, [_i32, _i32, _i32, _i32]),
     "moe_get_device_error": (_i32, [ctypes.POINTER(_i32), _c_void_p]),
+    "moe_zero": (_i32, [_c_void_p, _size, _c_void_p]),
 }
 
 _lib = None
@@ -273,6 +274,13 @@ def moe_expert_down(h, offsets, W_dn, rows_max: int, gate_of_row=None, y_rows=No
     _check("moe_expert_down", lib().moe_expert_down(_p(h), _dt(h), _p(offsets), E, d, F, rows_max, _p(W_dn),
                                                     _p(gate_of_row), _dt(y_rows), _p(y_rows), _stream(stream)))
     return y_rows
+
+
+def moe_zero(t, stream=None):
+    """Clears a contiguous device tensor with the library's memset (stream-ordered)."""
+    _need(t, "t")
+    _check("moe_zero", lib().moe_zero(_p(t), t.numel() * t.element_size(), _stream(stream)))
+    return t
 
 
 def moe_expert_down_combine(h, offsets, W_dn, rows_max: int, token_of_row, y, gate_of_row=None,

@@ -158,6 +158,12 @@ def test_permute_combine_host_validation(L):
     assert L.moe_combine(FAKE, 0, FAKE, NUL, NUL, 64, 128, 4, 256, 5, FAKE, NUL) == 1     # y dtype
 
 
+def test_zero_host_validation(L):
+    assert L.moe_zero(NUL, 64, NUL) == 1
+    assert L.moe_zero(ctypes.c_void_p(4100), 64, NUL) == 2
+    assert L.moe_zero(NUL, 0, NUL) == 0
+
+
 def test_router_stats_host_validation(L):
     f = L.moe_router_stats
     assert f(FAKE, FAKE, FAKE, 64, 16, 4, 5, FAKE, FAKE, FAKE, 1 << 30, NUL) == 1

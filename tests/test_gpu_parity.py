@@ -393,3 +393,32 @@ def test_gathered_bad_token_is_reported_not_trapped():
         M.moe_expert_gate_up_gather(dev["x"], tok, layer.offsets, layer.w.W_gu, layer.rows_max, layer.h)
         torch.cuda.synchronize()
         assert M.moe_get_device_error() == 3
+
+
+def test_second_stream_schedule_matches_the_sequential_one():
+    """Statistics and the fused combine's zero fill on a second stream give the same results
+    as the one-stream order (bit for bit in the reproducible form)."""
+    cfg = SMALL[1]                                            # shared expert, bias, sigmoid
+    host, dev = U.make_inputs(cfg)
+    cap = O.capacity(cfg.T, cfg.E, cfg.k, cfg.capacity_factor, True)
+    from routing_dispatch_expert_moe_b200.layer import MoELayer, MoEWeights
+    w = MoEWeights(Wg=dev["Wg"], W_gu=dev["W_gu"], W_dn=dev["W_dn"], logit_offset=dev["off"],
+                   select_bias=dev["bias"], W_gu_s=dev["W_gu_s"], W_dn_s=dev["W_dn_s"])
+    outs = {}
+    for overlap in (False, True):
+        lay = MoELayer(w, cfg.k, cfg.T, cfg.score, cfg.renormalize, cfg.scale, cap, overlap=overlap)
+        y = lay.forward(dev["x"]).clone()
+        torch.cuda.synchronize()
+        outs[overlap] = (y, lay.stats5.clone(), lay.load.clone())
+    assert torch.equal(outs[False][0], outs[True][0])
+    assert torch.equal(outs[False][1], outs[True][1]) and torch.equal(outs[False][2], outs[True][2])
+    # fused combine without a shared expert: y cleared on the second stream
+    cfg2 = SMALL[0]
+    host2, dev2 = U.make_inputs(cfg2)
+    rl, gr = U.gpu_forward(cfg2, dev2, -1)
+    lay = U.build_layer(cfg2, dev2, -1, combine="fused")
+    lay.y.fill_(123.0)                                        # stale contents must not survive
+    y = lay.forward(dev2["x"])
+    torch.cuda.synchronize()
+    bound = _ordered_terms_bound(rl, cfg2.T, cfg2.k)
+    assert (np.abs(y.double().cpu().numpy() - gr["y"]) <= bound + 1e-30).all()
