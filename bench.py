@@ -46,6 +46,29 @@ def peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def max_over_ranks(v: float, device=None) -> float:
+    """Max of v over every rank of the process group (v itself without one).  All ranks
+    must call it at the same point: it is a collective."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(v)
+    t = torch.tensor([float(v)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank: int, world: int, steps: int, total_ms: float) -> float:
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's time (weak scaling:
+    each replica processes its own batch of tokens_per_rank per step)."""
+    return tokens_per_rank * world * steps / (total_ms / 1e3)
+
+
+def replica_seed(rank: int) -> int:
+    """Seed of a replica's token batch: every rank gets its own batch, same weights."""
+    return rank
+
+
 def env_rank():
     return int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)), int(os.environ.get("WORLD_SIZE", 1))
 
@@ -149,7 +172,7 @@ def run_ours(args):
     if args.tokens:
         cfg = cfg.with_(T=args.tokens)
     dt = torch.float32 if cfg.act == "f32" else torch.bfloat16
-    x_np = I.gen_x(cfg, seed=rank)                      # each replica has its own token batch
+    x_np = I.gen_x(cfg, seed=replica_seed(rank))        # each replica has its own token batch
     Wg, off, bias = I.gen_router(cfg, 0)
     W_gu, W_dn = I.gen_experts_torch(cfg, 0)
     sh = I.gen_shared(cfg, 0)
@@ -249,29 +272,22 @@ def run_ours(args):
             del g2
         return per_step, stage_ms, rows, clk
 
-    def max_over_ranks(v):
-        if world > 1:
-            t = torch.tensor([v], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            v = float(t.item())
-        return v
-
     layer = make_layer(args.combine, args.dispatch)
     per_step, stage_ms, A, clk = time_layer(layer, args.steps, ClockSampler(local_rank),
                                             breakdown_steps=args.breakdown_steps)
-    total_ms = max_over_ranks(float(per_step.sum()))
+    total_ms = max_over_ranks(float(per_step.sum()), dev)
     ms_per_step = total_ms / args.steps
-    value = cfg.T * world * args.steps / (total_ms / 1e3)
+    value = job_throughput(cfg.T, world, args.steps, total_ms)
 
     other = None
     if (args.combine, args.dispatch) != ("rows", "permute") and args.unfused_steps > 0:
         # the unfused form (permute copy, gated rows, ordered combine: bitwise reproducible), same inputs
         rl = make_layer("rows", "permute")
         ps, sm, _, _ = time_layer(rl, args.unfused_steps, breakdown_steps=min(args.breakdown_steps, 50))
-        t = max_over_ranks(float(ps.sum()))
+        t = max_over_ranks(float(ps.sum()), dev)
         other = {"dispatch": "permute", "combine": "rows (gated rows + ordered combine, bitwise reproducible)",
                  "ms_per_step": round(t / args.unfused_steps, 4),
-                 "value": round(cfg.T * world * args.unfused_steps / (t / 1e3), 1), "steps": args.unfused_steps,
+                 "value": round(job_throughput(cfg.T, world, args.unfused_steps, t), 1), "steps": args.unfused_steps,
                  "stages_ms": {k_: round(v, 4) for k_, v in sm.items()}}
         del rl
         torch.cuda.empty_cache()
@@ -297,8 +313,8 @@ def run_ours(args):
         y_host.copy_(layer.y, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
-    e2e_value = cfg.T * world * e2e_steps / (e2e_ms / 1e3)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
+    e2e_value = job_throughput(cfg.T, world, e2e_steps, e2e_ms)
     h2d_bytes = x_host.numel() * x_host.element_size()
     d2h_bytes = y_host.numel() * y_host.element_size()
 
