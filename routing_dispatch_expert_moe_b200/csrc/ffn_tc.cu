@@ -384,7 +384,9 @@ __device__ __forceinline__ void epilogue_tile(uint32_t taddr, uint8_t* stage, in
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
         const float gi = __uint_as_float(g[i]);
-        h[i] = gi / (1.f + expf(-gi)) * __uint_as_float(u[i]);
+        // fast exp / divide: H is rounded to bf16 next, far coarser than their error; the
+        // exact forms made this epilogue the bound of the gate/up GEMM
+        h[i] = __fdividef(gi, 1.f + __expf(-gi)) * __uint_as_float(u[i]);
       }
       stage_store32<OutT>(stage, h, lane, out, wrow0, wrows, F, f0 + c * 32, F);
     }
