@@ -342,11 +342,12 @@ __device__ __forceinline__ void stage_red32(uint8_t* stage, const float (&v)[32]
 //   MODE 1: 256 columns -> gate_of_row[row] * acc for outputs n_tile*256 + ...
 //   MODE 2: [0,64) x.hi, [64,128) x.mid, [128,192) x.lo of experts n_tile*64 + ... ->
 //           logit = (hi + mid) + lo + offset (gate_of_row carries the logit offset)
+// MODE 1 / 3 process the 32-column chunks [c_begin, c_end) of the 256 (a warp may own half).
 template <int MODE, typename OutT>
 __device__ __forceinline__ void epilogue_tile(uint32_t taddr, uint8_t* stage, int lane, long long wrow0, int wrows,
                                               int n_tile, int F, int N_out, const float* __restrict__ gate_of_row,
                                               OutT* __restrict__ out, const int32_t* __restrict__ token_of_row,
-                                              int n_tokens, int* err) {
+                                              int n_tokens, int* err, int c_begin = 0, int c_end = BN / 32) {
   if constexpr (MODE == 3) {
     const int n0 = n_tile * BN;
     const float gs = (lane < wrows && gate_of_row) ? __ldg(gate_of_row + wrow0 + lane) : 1.f;
@@ -360,7 +361,7 @@ __device__ __forceinline__ void epilogue_tile(uint32_t taddr, uint8_t* stage, in
       }
     }
 #pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
+    for (int c = c_begin; c < c_end; ++c) {
       uint32_t v32[32];
       tmem_ld32(taddr + c * 32, v32);
       tmem_wait_ld();
@@ -394,7 +395,7 @@ __device__ __forceinline__ void epilogue_tile(uint32_t taddr, uint8_t* stage, in
     const int n0 = n_tile * BN;
     const float gs = (lane < wrows && gate_of_row) ? __ldg(gate_of_row + wrow0 + lane) : 1.f;
 #pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
+    for (int c = c_begin; c < c_end; ++c) {
       uint32_t v32[32];
       tmem_ld32(taddr + c * 32, v32);
       tmem_wait_ld();
@@ -673,37 +674,47 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
 //   tempty[a] (even CTA only) : 256 epilogue threads of both CTAs
 // Cluster barriers after set-up and before teardown; every wait bounded.
 // =====================================================================================
-constexpr int STAGES2 = 6;
 constexpr int B2_STAGE = BM * BK * 2;                        // 128 B-rows per CTA: 16 KB
 
-struct L2 {
+// Configuration of the CTA-pair kernel.  WIDE (down GEMMs with a short K, chosen at
+// launch): eight epilogue warps, two per TMEM lane quarter, each taking half of the 256
+// output columns, and five stages to make room for their staging.  With K <= 512 a tile
+// has at most 8 k-blocks and its 256-column fp32 epilogue, not the operand stream, sets
+// the pace; at longer K the sixth stage is worth more (measured).
+template <bool WIDE>
+struct PairCfg {
+  static constexpr int stages = WIDE ? 5 : 6;
+  static constexpr int epi_warps = WIDE ? 8 : 4;
+  static constexpr int threads = 64 + 32 * epi_warps;
   static constexpr int a = 0;
-  static constexpr int b = STAGES2 * A_STAGE;
-  static constexpr int bars = b + STAGES2 * B2_STAGE;
-  static constexpr int nbars = 2 * STAGES2 + 4 + 1;
+  static constexpr int b = stages * A_STAGE;
+  static constexpr int bars = b + stages * B2_STAGE;
+  static constexpr int nbars = 2 * stages + 4 + 1;
   static constexpr int misc = bars + nbars * 8;
   static constexpr int tiles = misc + 16;
   static constexpr int sh32 = tiles + (kMaxE + 1) * 4;
   static constexpr int stage = (sh32 + 32 * 4 + 15) / 16 * 16;
-  static constexpr int end = stage + 4 * 32 * (32 * 4 + 16);
+  static constexpr int end = stage + epi_warps * kStageWarpBytes;
+  static constexpr size_t smem = end + 1024;
+  static_assert(smem <= 232448, "shared memory per CTA");
 };
-constexpr size_t kSmemBytes2 = L2::end + 1024;
 
-template <int MODE, typename OutT>
-__global__ void __launch_bounds__(kThreadsTC, 1)
+template <int MODE, typename OutT, bool WIDE>
+__global__ void __launch_bounds__(PairCfg<WIDE>::threads, 1)
 grouped_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         const int32_t* __restrict__ offsets, int E, int K, int N_out, int F,
                         long long rows_max, const float* __restrict__ gate_of_row,
                         OutT* __restrict__ out, const int32_t* __restrict__ token_of_row, int n_tokens,
                        int* err) {
+  using C = PairCfg<WIDE>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  int* tile_start = reinterpret_cast<int*>(smem + L2::tiles);
-  int* sh32 = reinterpret_cast<int*>(smem + L2::sh32);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L2::misc);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L2::misc + 4);
+  int* tile_start = reinterpret_cast<int*>(smem + C::tiles);
+  int* sh32 = reinterpret_cast<int*>(smem + C::sh32);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::misc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::misc + 4);
   const uint32_t rank = cluster_ctarank();                   // 0 = even CTA (MMA issuer)
   const int cid = (int)(blockIdx.x >> 1), ncl = (int)(gridDim.x >> 1);
   constexpr int PM = 2 * BM;                                 // rows per pair tile
@@ -713,20 +724,20 @@ grouped_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
   const int total = tile_start[E];
   if (cid >= total) return;   // both CTAs of the pair see the same cid: uniform, nothing allocated
 
-  const uint32_t bar_full = sb + L2::bars;
-  const uint32_t bar_empty = bar_full + 8 * STAGES2;
-  const uint32_t bar_tfull = bar_empty + 8 * STAGES2;
+  const uint32_t bar_full = sb + C::bars;
+  const uint32_t bar_empty = bar_full + 8 * C::stages;
+  const uint32_t bar_tfull = bar_empty + 8 * C::stages;
   const uint32_t bar_tempty = bar_tfull + 16;
   const uint32_t bar_fin = bar_tempty + 16;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES2; ++s) {
+    for (int s = 0; s < C::stages; ++s) {
       mbar_init(bar_full + 8 * s, 1);
       mbar_init(bar_empty + 8 * s, 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(bar_tfull + 8 * a, 1);
-      mbar_init(bar_tempty + 8 * a, 2 * 128);
+      mbar_init(bar_tempty + 8 * a, 2 * 32 * C::epi_warps);
     }
     mbar_init(bar_fin, 1);
     *abort_flag = 0;
@@ -750,9 +761,9 @@ grouped_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      int last_phase[STAGES2];
+      int last_phase[C::stages];
 #pragma unroll
-      for (int s = 0; s < STAGES2; ++s) last_phase[s] = -1;
+      for (int s = 0; s < C::stages; ++s) last_phase[s] = -1;
       bool ok = true;
       for (int tile = cid; ok && tile < total; tile += ncl) {
         const TileCoord tc = tile_coord(tile_start, offsets, E, PM, tile);
@@ -765,14 +776,14 @@ grouped_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
           if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1u, abort_flag, err)) { ok = false; break; }
           if (rank == 0) mbar_expect_tx(bar_full + 8 * stage, 2 * (A_STAGE + B2_STAGE));
           const uint32_t full_c = map_to_rank(bar_full + 8 * stage, 0);
-          tma_load_2d_pair(sb + L2::a + stage * A_STAGE, &tmA, full_c, kb * BK, a_row);
-          tma_load_2d_pair(sb + L2::b + stage * B2_STAGE, &tmB, full_c, kb * BK, b_row);
+          tma_load_2d_pair(sb + C::a + stage * A_STAGE, &tmA, full_c, kb * BK, a_row);
+          tma_load_2d_pair(sb + C::b + stage * B2_STAGE, &tmB, full_c, kb * BK, b_row);
           last_phase[stage] = (int)phase;
-          if (++stage == STAGES2) { stage = 0; phase ^= 1u; }
+          if (++stage == C::stages) { stage = 0; phase ^= 1u; }
         }
       }
       if (!ok && rank == 0) {
-        for (int s = 0; s < STAGES2; ++s)
+        for (int s = 0; s < C::stages; ++s)
           if (last_phase[s] >= 0) mbar_wait_drain(bar_full + 8 * s, (uint32_t)last_phase[s], err);
       }
     }
@@ -792,13 +803,13 @@ grouped_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag, err)) { ok = false; break; }
           tc_fence_after();
-          const uint64_t adesc = sw128_desc(sb + L2::a + stage * A_STAGE);
-          const uint64_t bdesc = sw128_desc(sb + L2::b + stage * B2_STAGE);
+          const uint64_t adesc = sw128_desc(sb + C::a + stage * A_STAGE);
+          const uint64_t bdesc = sw128_desc(sb + C::b + stage * B2_STAGE);
 #pragma unroll
           for (int kk = 0; kk < BK / UMMA_K; ++kk)
             umma_bf16_pair(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, (kb | kk) != 0 ? 1u : 0u);
           umma_commit_pair_both(bar_empty + 8 * stage);
-          if (++stage == STAGES2) { stage = 0; phase ^= 1u; }
+          if (++stage == C::stages) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
         umma_commit_pair_both(bar_tfull + 8 * acc);
@@ -808,8 +819,11 @@ grouped_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
     }
   } else {
     // ------------------------------------------------------------ epilogue (both CTAs)
-    const int q = warp & 3;
-    uint8_t* stage = smem + L2::stage + (warp - 2) * kStageWarpBytes;
+    const int q = warp & 3;                                  // TMEM lane quarter this warp may access
+    const int ew = warp - 2;
+    const int c_begin = WIDE ? (ew >> 2) * 4 : 0;            // its column chunks
+    const int c_end = WIDE ? c_begin + 4 : BN / 32;
+    uint8_t* stage = smem + C::stage + ew * kStageWarpBytes;
     int it = 0;
     for (int tile = cid; tile < total; tile += ncl, ++it) {
       const TileCoord tc = tile_coord(tile_start, offsets, E, PM, tile);
@@ -824,7 +838,7 @@ grouped_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
       const long long wrow0 = (long long)tc.row0 + (int)rank * BM + q * 32;
       const int wrows = min(32, max(0, cta_rows - q * 32));
       epilogue_tile<MODE, OutT>(taddr, stage, lane, wrow0, wrows, tc.n_tile, F, N_out, gate_of_row, out,
-                                token_of_row, n_tokens, err);
+                                token_of_row, n_tokens, err, c_begin, c_end);
       tc_fence_before();
       mbar_arrive_cluster(map_to_rank(bar_tempty + 8 * acc, 0));
     }
@@ -903,9 +917,11 @@ moe_status launch_tc(const CUtensorMap& ma, const CUtensorMap& mb, const int32_t
 // B = the split weight W3 [ceil(E/64) * 256, d]; writes logits [T, E] fp32 (+ offset).
 // CTA pairs pay off when groups average at least one full 256-row pair tile; smaller
 // groups keep the single-CTA kernel (less padding in ragged groups).
+// Down GEMMs with K = F up to this use the eight-epilogue-warp pair configuration.
+constexpr int kWideMaxK = 512;
 static bool use_pairs(long long rows_max, int groups) { return groups > 0 && rows_max / groups >= 2 * BM; }
 
-template <int MODE, typename OutT>
+template <int MODE, typename OutT, bool WIDE = false>
 moe_status launch_tc2(const CUtensorMap& ma, const CUtensorMap& mb, const int32_t* offsets, int E, int K, int N_out,
                       int F, long long rows_max, const float* gate_of_row, void* out, cudaStream_t s,
                       const int32_t* token_of_row = nullptr, int n_tokens = 0) {
@@ -914,8 +930,8 @@ moe_status launch_tc2(const CUtensorMap& ma, const CUtensorMap& mb, const int32_
   cudaGetDevice(&dev);
   dev &= 63;
   if (!configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_tc2_kernel<MODE, OutT>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes2);
+    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_tc2_kernel<MODE, OutT, WIDE>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PairCfg<WIDE>::smem);
     if (e != cudaSuccess) return cuda_status(e);
     configured[dev] = 1;
   }
@@ -926,8 +942,8 @@ moe_status launch_tc2(const CUtensorMap& ma, const CUtensorMap& mb, const int32_
   if (pairs < 1) pairs = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs, 1, 1);
-  cfg.blockDim = dim3(kThreadsTC, 1, 1);
-  cfg.dynamicSmemBytes = kSmemBytes2;
+  cfg.blockDim = dim3(PairCfg<WIDE>::threads, 1, 1);
+  cfg.dynamicSmemBytes = PairCfg<WIDE>::smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -936,7 +952,7 @@ moe_status launch_tc2(const CUtensorMap& ma, const CUtensorMap& mb, const int32_
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cuda_status(cudaLaunchKernelEx(&cfg, grouped_gemm_tc2_kernel<MODE, OutT>, ma, mb, offsets, E, K, N_out, F,
+  return cuda_status(cudaLaunchKernelEx(&cfg, grouped_gemm_tc2_kernel<MODE, OutT, WIDE>, ma, mb, offsets, E, K, N_out, F,
                                         rows_max, gate_of_row, static_cast<OutT*>(out), token_of_row, n_tokens,
                                         err_ptr()));
 }
@@ -975,6 +991,11 @@ moe_status launch_down_tc(const void* h, const int32_t* offsets, int E, int d, i
   if (!make_map(&ma, h, (unsigned long long)rows_max, F, BM)) return MOE_ERR_UNSUPPORTED;
   if (!make_map(&mb, W_dn, (unsigned long long)E * d, F, pair ? BM : BN)) return MOE_ERR_UNSUPPORTED;
   if (pair) {
+    if (F <= kWideMaxK) {
+      if (y_dtype == MOE_F32)
+        return launch_tc2<1, float, true>(ma, mb, offsets, E, F, d, F, rows_max, gate_of_row, y_rows, s);
+      return launch_tc2<1, __nv_bfloat16, true>(ma, mb, offsets, E, F, d, F, rows_max, gate_of_row, y_rows, s);
+    }
     if (y_dtype == MOE_F32)
       return launch_tc2<1, float>(ma, mb, offsets, E, F, d, F, rows_max, gate_of_row, y_rows, s);
     return launch_tc2<1, __nv_bfloat16>(ma, mb, offsets, E, F, d, F, rows_max, gate_of_row, y_rows, s);
@@ -994,6 +1015,8 @@ moe_status launch_down_combine_tc(const void* h, const int32_t* offsets, int E, 
   CUtensorMap ma, mb;
   if (!make_map(&ma, h, (unsigned long long)rows_max, F, BM)) return MOE_ERR_UNSUPPORTED;
   if (!make_map(&mb, W_dn, (unsigned long long)E * d, F, pair ? BM : BN)) return MOE_ERR_UNSUPPORTED;
+  if (pair && F <= kWideMaxK)
+    return launch_tc2<3, float, true>(ma, mb, offsets, E, F, d, F, rows_max, gate_of_row, y, s, token_of_row, T);
   if (pair) return launch_tc2<3, float>(ma, mb, offsets, E, F, d, F, rows_max, gate_of_row, y, s, token_of_row, T);
   return launch_tc<3, float>(ma, mb, offsets, E, F, d, F, rows_max, gate_of_row, y, s, token_of_row, T);
 }

@@ -22,77 +22,82 @@ namespace {
 
 constexpr int kStatsThreads = 256;
 
-__device__ __forceinline__ float warp_max_f(float v) {
-#pragma unroll
-  for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
-}
-__device__ __forceinline__ double warp_sum_dd(double v) {
-#pragma unroll
-  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
+// Score of one logit (fp32 transcendentals; every sum that uses them is fp64).
+__device__ __forceinline__ float score_f(float l, float m, int score) {
+  if (score == MOE_SCORE_SOFTMAX) return expf(l - m);
+  if (score == MOE_SCORE_SIGMOID) return 1.f / (1.f + expf(-l));
+  return sqrtf(fmaxf(l, 0.f) + log1pf(expf(-fabsf(l))));
 }
 
-template <int EPL>
+constexpr int kSub = 64;   // tokens per sub-chunk (normalisers held in shared memory)
+
+// Stage 1: each CTA owns tokens [t_begin, t_end), taken kSub at a time.
+//   (a) a warp per token: m = max_e l, se = sum_e exp(l - m), ss = sum_e s_e (fp64 sums,
+//       fixed lane-strided order and butterfly); z2 += (m + log se)^2;
+//   (b) a thread per expert: P_e += s_e(t) / ss(t) over the sub-chunk's tokens, in order.
+// Writes the CTA's P partials [E] and z2 partial.  Few registers per thread, so many warps
+// per SM hide the latency of the transcendentals at any E.
 __global__ void __launch_bounds__(kStatsThreads)
 stats_partial_kernel(const float* __restrict__ logits, int T, int E, int score, int tokens_per_cta,
                      double* __restrict__ partP, double* __restrict__ partZ) {
-  __shared__ double red[32 * EPL];            // running sum over warps, warp order
+  __shared__ float s_m[kSub];
+  __shared__ double s_inv[kSub];
   __shared__ double redz[kStatsThreads / 32];
   const unsigned lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int nwarps = kStatsThreads / 32;
   const long long t_begin = (long long)blockIdx.x * tokens_per_cta;
   const long long t_end = min((long long)T, t_begin + tokens_per_cta);
-
-  double P[EPL];
-#pragma unroll
-  for (int i = 0; i < EPL; ++i) P[i] = 0.0;
   double z2 = 0.0;
-  for (long long t = t_begin + warp; t < t_end; t += nwarps) {
-    float l[EPL];
-    float mf = -INFINITY;
+  // this thread's experts: e = threadIdx.x + i * kStatsThreads (E <= 1024: at most 4)
+  double P[4] = {0.0, 0.0, 0.0, 0.0};
+  for (long long c0 = t_begin; c0 < t_end; c0 += kSub) {
+    const int n = (int)min((long long)kSub, t_end - c0);
+    for (int i = warp; i < n; i += nwarps) {
+      const float* row = logits + (c0 + i) * E;
+      float mf = -INFINITY;
+      for (int e = lane; e < E; e += 32) mf = fmaxf(mf, __ldg(row + e));
 #pragma unroll
-    for (int i = 0; i < EPL; ++i) {
-      const int e = lane + 32 * i;
-      l[i] = e < E ? __ldg(logits + t * E + e) : -INFINITY;
-      mf = fmaxf(mf, l[i]);
-    }
-    const double m = (double)warp_max_f(mf);
-    double se = 0.0, ss = 0.0;
-    double sc[EPL];
-#pragma unroll
-    for (int i = 0; i < EPL; ++i) {
-      const bool ok = lane + 32 * i < (unsigned)E;
-      const double ex = ok ? exp((double)l[i] - m) : 0.0;
-      se += ex;
-      double s = 0.0;
-      if (ok) {
-        if (score == MOE_SCORE_SOFTMAX) s = ex;
-        else if (score == MOE_SCORE_SIGMOID) s = 1.0 / (1.0 + exp(-(double)l[i]));
-        else s = sqrt(fmax((double)l[i], 0.0) + log1p(exp(-fabs((double)l[i]))));
+      for (int o = 16; o; o >>= 1) mf = fmaxf(mf, __shfl_xor_sync(0xffffffffu, mf, o));
+      double se = 0.0, ss = 0.0;
+      for (int e = lane; e < E; e += 32) {
+        const float l = __ldg(row + e);
+        const float ex = expf(l - mf);
+        se += (double)ex;
+        ss += (double)(score == MOE_SCORE_SOFTMAX ? ex : score_f(l, mf, score));
       }
-      sc[i] = s;
-      ss += s;
+#pragma unroll
+      for (int o = 16; o; o >>= 1) {
+        se += __shfl_xor_sync(0xffffffffu, se, o);
+        ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      }
+      if (lane == 0) {
+        s_m[i] = mf;
+        s_inv[i] = 1.0 / ss;
+        const double lse = (double)mf + log(se);
+        z2 += lse * lse;
+      }
     }
-    se = warp_sum_dd(se);
-    ss = warp_sum_dd(ss);
-    const double inv = 1.0 / ss;
+    __syncthreads();
 #pragma unroll
-    for (int i = 0; i < EPL; ++i) P[i] += sc[i] * inv;
-    const double lse = m + log(se);
-    z2 += lse * lse;
-  }
-  for (int w = 0; w < nwarps; ++w) {
-    if (warp == w) {
-#pragma unroll
-      for (int i = 0; i < EPL; ++i) red[lane + 32 * i] = (w == 0 ? 0.0 : red[lane + 32 * i]) + P[i];
+    for (int q = 0; q < 4; ++q) {
+      const int e = (int)threadIdx.x + q * kStatsThreads;
+      if (e < E) {
+        double acc = P[q];
+        for (int i = 0; i < n; ++i)
+          acc += (double)score_f(__ldg(logits + (c0 + i) * E + e), s_m[i], score) * s_inv[i];
+        P[q] = acc;
+      }
     }
     __syncthreads();
   }
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int e = (int)threadIdx.x + q * kStatsThreads;
+    if (e < E) partP[(long long)blockIdx.x * E + e] = P[q];
+  }
   if (lane == 0) redz[warp] = z2;
   __syncthreads();
-  for (int e = threadIdx.x; e < E; e += kStatsThreads) partP[(long long)blockIdx.x * E + e] = red[e];
   if (threadIdx.x == 0) {
     double acc = 0.0;
     for (int w = 0; w < nwarps; ++w) acc += redz[w];
@@ -199,14 +204,6 @@ int stats_parts(int T) {
   return parts < want ? (parts < 1 ? 1 : parts) : want;
 }
 
-template <int EPL>
-moe_status run_partial(const float* logits, int T, int E, int score, int parts, double* pP, double* pZ,
-                       cudaStream_t s) {
-  const int tpc = (T + parts - 1) / parts;
-  stats_partial_kernel<EPL><<<parts, kStatsThreads, 0, s>>>(logits, T, E, score, tpc, pP, pZ);
-  return check_launch();
-}
-
 }  // namespace
 
 size_t router_stats_workspace_bytes(int T, int E) {
@@ -225,14 +222,9 @@ moe_status launch_router_stats(const float* logits, const int32_t* counts, const
   const int parts = stats_parts(T);
   double* pP = static_cast<double*>(ws);
   double* pZ = pP + (size_t)parts * E;
-  const int epl = (E + 31) / 32;
-  moe_status st;
-  if (epl <= 1) st = run_partial<1>(logits, T, E, score, parts, pP, pZ, s);
-  else if (epl <= 2) st = run_partial<2>(logits, T, E, score, parts, pP, pZ, s);
-  else if (epl <= 4) st = run_partial<4>(logits, T, E, score, parts, pP, pZ, s);
-  else if (epl <= 8) st = run_partial<8>(logits, T, E, score, parts, pP, pZ, s);
-  else if (epl <= 16) st = run_partial<16>(logits, T, E, score, parts, pP, pZ, s);
-  else st = run_partial<32>(logits, T, E, score, parts, pP, pZ, s);
+  const int tpc = (T + parts - 1) / parts;
+  stats_partial_kernel<<<parts, kStatsThreads, 0, s>>>(logits, T, E, score, tpc, pP, pZ);
+  moe_status st = check_launch();
   if (st != MOE_OK) return st;
   stats_final_kernel<<<1, 1024, 0, s>>>(pP, pZ, parts, counts, kept, T, E, k, load, stats5);
   return check_launch();
