@@ -63,9 +63,15 @@ struct L {
 };
 constexpr size_t kSmemBytes = L::end + 1024;                 // + alignment slack
 
-// instruction descriptor: D fp32, A bf16, B bf16, both K-major, N = 256, M = 128
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
-                            ((uint32_t)(BM >> 4) << 24);
+// instruction descriptor: D fp32, A bf16, B bf16, both K-major, N = n, M = m
+constexpr uint32_t make_idesc(int m, int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
+}
+// MMA width per mode: the router tile (MODE 2) holds three 64-column terms (hi, mid, lo)
+// of the split weight, so it issues N = 192; every other mode N = 256 (= BN).
+constexpr int kRouterN = 192;
+template <int MODE>
+constexpr int mma_n() { return MODE == 2 ? kRouterN : BN; }
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -158,12 +164,13 @@ __host__ __device__ __forceinline__ int n_tiles_of(int F, int N_out) {
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate)
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 __device__ __forceinline__ void umma_commit(uint32_t bar) {
@@ -172,8 +179,6 @@ __device__ __forceinline__ void umma_commit(uint32_t bar) {
 
 // ---- CTA-pair (cta_group::2) forms: an M=256 MMA issued by the pair's even CTA over
 // both CTAs' shared memory, accumulating into both CTAs' TMEM ----
-constexpr uint32_t kIdesc2 = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
-                             ((uint32_t)((2 * BM) >> 4) << 24);
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;
@@ -202,12 +207,13 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar_cluster)
       : "memory");
 }
-__device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+__device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                               uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(kIdesc2), "r"(accumulate)
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 // Completion of the pair's MMAs arrives on the barrier at this offset in both CTAs.
@@ -571,11 +577,11 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
       for (int s = 0; s < STAGES; ++s) last_phase[s] = -1;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
-        const TileCoord tc = tile_coord(tile_start, offsets, E, BM, tile);
+        const TileCoord tc = tile_coord(tile_start, offsets, E, BM, tile, MODE == 2 ? n_tiles : 0);
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1u, abort_flag, err)) { ok = false; break; }
           const uint32_t full = bar_full + 8 * stage;
-          mbar_expect_tx(full, A_STAGE + B_STAGE);
+          mbar_expect_tx(full, A_STAGE + mma_n<MODE>() * BK * 2);
           const uint32_t a_dst = sb + L::a + stage * A_STAGE;
           const uint32_t b_dst = sb + L::b + stage * B_STAGE;
           tma_load_2d(a_dst, &tmA, full, kb * BK, tc.row0);
@@ -586,7 +592,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
           } else if (MODE == 1 || MODE == 3) {
             tma_load_2d(b_dst, &tmB, full, kb * BK, tc.e * N_out + tc.n_tile * BN);
           } else {
-            tma_load_2d(b_dst, &tmB, full, kb * BK, tc.n_tile * BN);   // router: 256 rows per n-tile
+            tma_load_2d(b_dst, &tmB, full, kb * BK, tc.n_tile * BN);   // router: rows hi, mid, lo of the tile
           }
           last_phase[stage] = (int)phase;
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -619,7 +625,8 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
           const uint64_t bdesc = sw128_desc(sb + L::b + stage * B_STAGE);
 #pragma unroll
           for (int kk = 0; kk < BK / UMMA_K; ++kk)   // +32 bytes along K per step (>> 4 = 2)
-            umma_bf16(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, (kb | kk) != 0 ? 1u : 0u);
+            umma_bf16(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, make_idesc(BM, mma_n<MODE>()),
+                      (kb | kk) != 0 ? 1u : 0u);
           umma_commit(bar_empty + 8 * stage);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
@@ -637,7 +644,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
     uint8_t* stage = smem + L::stage + (warp - 2) * kStageWarpBytes;
     int it = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
-      const TileCoord tc = tile_coord(tile_start, offsets, E, BM, tile);
+      const TileCoord tc = tile_coord(tile_start, offsets, E, BM, tile, MODE == 2 ? n_tiles : 0);
       const int acc = it & 1;
       const uint32_t acc_phase = (uint32_t)(it >> 1) & 1u;
       const bool got = mbar_wait(bar_tfull + 8 * acc, acc_phase, abort_flag, err);
@@ -766,15 +773,15 @@ grouped_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
       for (int s = 0; s < C::stages; ++s) last_phase[s] = -1;
       bool ok = true;
       for (int tile = cid; ok && tile < total; tile += ncl) {
-        const TileCoord tc = tile_coord(tile_start, offsets, E, PM, tile);
+        const TileCoord tc = tile_coord(tile_start, offsets, E, PM, tile, MODE == 2 ? n_tiles : 0);
         const int a_row = tc.row0 + (int)rank * BM;
         int b_row;
         if (MODE == 0) b_row = tc.e * 2 * F + (rank ? F : 0) + tc.n_tile * 128;   // even: gate, odd: up
         else if (MODE == 1 || MODE == 3) b_row = tc.e * N_out + tc.n_tile * BN + (int)rank * BM;
-        else b_row = tc.n_tile * BN + (int)rank * BM;
+        else b_row = tc.n_tile * BN + (int)rank * (kRouterN / 2);   // router: half of hi, mid, lo
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1u, abort_flag, err)) { ok = false; break; }
-          if (rank == 0) mbar_expect_tx(bar_full + 8 * stage, 2 * (A_STAGE + B2_STAGE));
+          if (rank == 0) mbar_expect_tx(bar_full + 8 * stage, 2 * (A_STAGE + (mma_n<MODE>() / 2) * BK * 2));
           const uint32_t full_c = map_to_rank(bar_full + 8 * stage, 0);
           tma_load_2d_pair(sb + C::a + stage * A_STAGE, &tmA, full_c, kb * BK, a_row);
           tma_load_2d_pair(sb + C::b + stage * B2_STAGE, &tmB, full_c, kb * BK, b_row);
@@ -807,7 +814,8 @@ grouped_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
           const uint64_t bdesc = sw128_desc(sb + C::b + stage * B2_STAGE);
 #pragma unroll
           for (int kk = 0; kk < BK / UMMA_K; ++kk)
-            umma_bf16_pair(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, (kb | kk) != 0 ? 1u : 0u);
+            umma_bf16_pair(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, make_idesc(2 * BM, mma_n<MODE>()),
+                           (kb | kk) != 0 ? 1u : 0u);
           umma_commit_pair_both(bar_empty + 8 * stage);
           if (++stage == C::stages) { stage = 0; phase ^= 1u; }
         }
@@ -826,7 +834,7 @@ grouped_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
     uint8_t* stage = smem + C::stage + ew * kStageWarpBytes;
     int it = 0;
     for (int tile = cid; tile < total; tile += ncl, ++it) {
-      const TileCoord tc = tile_coord(tile_start, offsets, E, PM, tile);
+      const TileCoord tc = tile_coord(tile_start, offsets, E, PM, tile, MODE == 2 ? n_tiles : 0);
       const int acc = it & 1;
       const uint32_t acc_phase = (uint32_t)(it >> 1) & 1u;
       const bool got = mbar_wait(bar_tfull + 8 * acc, acc_phase, abort_flag, err);
@@ -965,7 +973,8 @@ moe_status launch_router_logits_tc(const void* x, const int32_t* offs2, int T, i
   const bool pair = use_pairs(T, 1);
   CUtensorMap ma, mb;
   if (!make_map(&ma, x, (unsigned long long)T, d, BM)) return MOE_ERR_UNSUPPORTED;
-  if (!make_map(&mb, W3, (unsigned long long)nt * 256, d, pair ? BM : BN)) return MOE_ERR_UNSUPPORTED;
+  // boxes cover the hi, mid and lo rows of a 256-row tile (the pad rows are never loaded)
+  if (!make_map(&mb, W3, (unsigned long long)nt * 256, d, pair ? kRouterN / 2 : kRouterN)) return MOE_ERR_UNSUPPORTED;
   if (pair) return launch_tc2<2, float>(ma, mb, offs2, 1, d, E, 0, T, logit_offset, logits, s);
   return launch_tc<2, float>(ma, mb, offs2, 1, d, E, 0, T, logit_offset, logits, s);
 }
