@@ -292,31 +292,60 @@ def run_ours(args):
         del rl
         torch.cuda.empty_cache()
 
-    # end to end through the public API with host buffers (pinned), copies inside the timing
+    # End to end through the public API with host buffers (pinned), copies inside the timing.
+    # Two layer instances (shared weights, their own buffers and CUDA graphs) let the copy
+    # of batch i+1 in, the forward of batch i and the copy of batch i-1 out run at once on
+    # three streams, as a serving loop would; every step still copies its input in and its
+    # result out inside the timed region.
     x_host = torch.from_numpy(x_np).to(dt).pin_memory()
-    y_host = torch.empty((cfg.T, cfg.d), dtype=layer.out_dtype).pin_memory()
+    y_host = [torch.empty((cfg.T, cfg.d), dtype=layer.out_dtype).pin_memory() for _ in range(2)]
     e2e_steps = max(3, args.e2e_steps)
-    layer.capture(x)                       # the layer's public graph API: capture once, replay per batch
-    for _ in range(2):
-        x.copy_(x_host, non_blocking=True)
-        layer.replay()
-        y_host.copy_(layer.y, non_blocking=True)
+    lays = [layer, make_layer(args.combine, args.dispatch)]
+    xs = [x, torch.empty_like(x)]
+    for l_, x_ in zip(lays, xs):
+        x_.copy_(x_host)
+        l_.capture(x_)                     # the layer's public graph API: capture once, replay per batch
+    s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in, ev_comp, ev_out = ([torch.cuda.Event() for _ in range(2)] for _ in range(3))
+
+    def e2e_run(n):
+        for i in range(n):
+            b = i & 1
+            s_in.wait_event(ev_comp[b])    # the forward that last read xs[b] has finished
+            with torch.cuda.stream(s_in):
+                xs[b].copy_(x_host, non_blocking=True)
+            ev_in[b].record(s_in)
+            s_comp.wait_event(ev_in[b])
+            s_comp.wait_event(ev_out[b])   # the copy-out that last read lays[b].y has finished
+            with torch.cuda.stream(s_comp):
+                lays[b].replay()
+            ev_comp[b].record(s_comp)
+            s_out.wait_event(ev_comp[b])
+            with torch.cuda.stream(s_out):
+                y_host[b].copy_(lays[b].y[:cfg.T], non_blocking=True)
+            ev_out[b].record(s_out)
+
+    for b in range(2):                     # events start out recorded (nothing pending)
+        ev_comp[b].record(s_comp)
+        ev_out[b].record(s_out)
+    e2e_run(4)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        x.copy_(x_host, non_blocking=True)
-        layer.replay()
-        y_host.copy_(layer.y, non_blocking=True)
-    e1.record(stream)
+    e0.record(s_in)
+    s_comp.wait_event(e0)
+    s_out.wait_event(e0)
+    e2e_run(e2e_steps)
+    s_in.wait_stream(s_out)
+    e1.record(s_in)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
     e2e_value = job_throughput(cfg.T, world, e2e_steps, e2e_ms)
     h2d_bytes = x_host.numel() * x_host.element_size()
-    d2h_bytes = y_host.numel() * y_host.element_size()
+    d2h_bytes = y_host[0].numel() * y_host[0].element_size()
+    del lays
 
     pk, pk_src = peaks()
     gather = args.dispatch == "gather"
@@ -357,7 +386,8 @@ def run_ours(args):
                        "parallelism": f"replicas x{world} (independent token batches, no collective)",
                        "l2": "flushed before every step (256 MB write)"},
             "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d_bytes,
-                    "d2h_bytes_per_step": d2h_bytes, "steps": e2e_steps},
+                    "d2h_bytes_per_step": d2h_bytes, "steps": e2e_steps,
+                    "schedule": "two layer instances, copy in / forward / copy out on three streams"},
             "gpu_launches": args.steps * layer.launches_per_forward(True),
             "roofline": {"bound": "tensor",
                          "kernel": ("moe_expert_gate_up_gather (tcgen05 grouped GEMM, gathered rows, SwiGLU)"
