@@ -144,6 +144,8 @@ def layer_roofline_ms(cfg, A, pk, rb=4, ob=4, fused=False, gather=False):
         steps["gate_up"] = max(4 * A * d * F / tc, (A * d * b + E * 2 * F * d * b + A * F * b) / hbm)
     if fused:
         steps["down_combine"] = max(2 * A * F * d / tc, (A * F * b + E * d * F * b + 2 * T * d * 4) / hbm)
+        if ob == 2:
+            steps["round_output"] = (T * d * 4 + T * d * 2) / hbm
     else:
         steps["down"] = max(2 * A * F * d / tc, (A * F * b + E * d * F * b + A * d * rb) / hbm)
         steps["combine"] = (A * d * rb + T * d * ob) / hbm
@@ -187,9 +189,11 @@ def run_ours(args):
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
 
+    out_dt = torch.bfloat16 if args.out_dtype == "bf16" else torch.float32
+
     def make_layer(combine, dispatch):
         return MoELayer(w, cfg.k, cfg.T, cfg.score, cfg.renormalize, cfg.scale, cap, combine=combine,
-                        dispatch=dispatch)
+                        dispatch=dispatch, out_dtype=out_dt)
 
     def capture(fn):
         """One CUDA graph of fn(stream), captured on a side stream."""
@@ -383,6 +387,7 @@ def run_ours(args):
                        "dispatch": ("gathered inside the gate/up GEMM" if gather else "permute copy"),
                        "combine": ("fused into the down GEMM (fp32 atomics into y)" if fused
                                    else "gated rows + ordered combine"),
+                       "out_dtype": args.out_dtype,
                        "parallelism": f"replicas x{world} (independent token batches, no collective)",
                        "l2": "flushed before every step (256 MB write)"},
             "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d_bytes,
@@ -519,6 +524,8 @@ def main():
                     help="fused: combine inside the down GEMM; rows: gated rows + ordered combine")
     ap.add_argument("--dispatch", choices=["gather", "permute"], default="permute",
                     help="gather: the gate/up GEMM reads token rows through the row map; permute: x_perm copy")
+    ap.add_argument("--out-dtype", choices=["bf16", "f32"], default="bf16",
+                    help="dtype of the layer output y (bf16: fp32 sums rounded once at the end)")
     ap.add_argument("--breakdown-steps", type=int, default=100,
                     help="sequential replays for the per-stage split (0 = skip)")
     ap.add_argument("--unfused-steps", type=int, default=100,

@@ -15,6 +15,7 @@
  *   moe_grouped_ffn      the two GEMMs above back to back
  *   moe_combine          gate-weighted sum of each token's rows (+ shared expert)
  *   moe_expert_down_combine  the down GEMM with the combine fused into its epilogue
+ *   moe_round_output     the combine's final rounding of an fp32 sum to bf16
  *   moe_router_stats     per-expert load, aux loss, z-loss, drops, imbalance
  *
  * Sources (web pages on Mixture-of-Experts, cited by title and section):
@@ -275,6 +276,18 @@ MOE_API moe_status moe_expert_down_combine(const void* h, int32_t dtype, const i
                            const void* W_dn, const float* gate_of_row,
                            const int32_t* token_of_row, int32_t T, int32_t accumulate,
                            float* y, void* stream);
+
+/* ------------------------------------------------------------------------------------
+ * moe_round_output -- y[i] = bf16_rne(y32[i]) for 0 <= i < n: the final rounding of the
+ * combine ([MoE-Explained] section "什么是稀疏性？", y = sum_i G(x)_i E_i(x), returned in
+ * the activation dtype) when the sum was accumulated in fp32, e.g. by
+ * moe_expert_down_combine.
+ *   y32 (device) [n] fp32;  y (device) [n] bf16 out;  both 16-byte aligned.
+ *   clear 1: y32[i] is set to 0 once read, so that it can take the next sum with
+ *         moe_expert_down_combine(..., accumulate = 1) and no separate clearing pass;
+ *         0: y32 is left as it is.
+ * ---------------------------------------------------------------------------------- */
+MOE_API moe_status moe_round_output(float* y32, int64_t n, void* y, int32_t clear, void* stream);
 
 /* ------------------------------------------------------------------------------------
  * moe_combine -- y[t] = sum_j g_j * y_rows[row_of[t, j]]  (+ shared_y[t]).

@@ -284,6 +284,14 @@ size_t moe_workspace_bytes(int32_t T, int32_t d, int32_t E, int32_t k) {
   return m > c ? m : c;
 }
 
+moe_status moe_round_output(float* y32, int64_t n, void* y, int32_t clear, void* stream) {
+  if (n < 0 || (clear != 0 && clear != 1)) return MOE_ERR_INVALID_ARG;
+  if (n == 0) return MOE_OK;
+  if (!y32 || !y) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(y32) || !aligned16(y)) return MOE_ERR_UNSUPPORTED;
+  return launch_round_bf16(y32, n, y, clear, S(stream));
+}
+
 moe_status moe_zero(void* p, size_t bytes, void* stream) {
   if (bytes == 0) return MOE_OK;
   if (!p) return MOE_ERR_INVALID_ARG;

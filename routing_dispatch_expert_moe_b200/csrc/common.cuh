@@ -121,6 +121,8 @@ moe_status launch_combine(const void* y_rows, int rows_dtype, const int32_t* row
                           const void* shared_y, int T, int d, int k, long long rows_max, int y_dtype,
                           void* y, cudaStream_t s);
 
+moe_status launch_round_bf16(float* in, long long n, void* out, int clear, cudaStream_t s);
+
 moe_status launch_router_stats(const float* logits, const int32_t* counts, const int32_t* kept,
                                int T, int E, int k, int score, float* load, float* stats5,
                                void* ws, cudaStream_t s);

@@ -176,6 +176,28 @@ moe_status combine_k(const void* y_rows, const int32_t* row_of, const float* top
   return run_combine<InT, OutT, 32>(y_rows, row_of, topk_gate, shared_y, T, d, k, rows_max, y, s);
 }
 
+// Final rounding of the combine: out[i] = bf16_rne(in[i]); with clear, in[i] = 0 after
+// it is read (so an accumulation buffer is ready for the next sum without a separate
+// fill).  Eight values per thread and step (two 16-byte loads, one 16-byte store),
+// grid-stride; a scalar tail for n % 8.
+__global__ void __launch_bounds__(256)
+round_bf16_kernel(float* __restrict__ in, long long n, __nv_bfloat16* __restrict__ out, int clear) {
+  const long long n8 = n / 8;
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += stride) {
+    float4* p = reinterpret_cast<float4*>(in) + 2 * i;
+    const float4 a = p[0];
+    const float4 b = p[1];
+    const float f[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    reinterpret_cast<uint4*>(out)[i] = pack8(f);
+    if (clear) p[0] = p[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  for (long long i = 8 * n8 + (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
+    out[i] = __float2bfloat16_rn(in[i]);
+    if (clear) in[i] = 0.f;
+  }
+}
+
 }  // namespace
 
 moe_status launch_permute(const void* x, int dtype, int T, int d, int k, const int32_t* row_of,
@@ -197,6 +219,16 @@ moe_status launch_combine(const void* y_rows, int rows_dtype, const int32_t* row
   if (in32) return combine_k<float, __nv_bfloat16>(y_rows, row_of, topk_gate, shared_y, T, d, k, rows_max, y, s);
   if (out32) return combine_k<__nv_bfloat16, float>(y_rows, row_of, topk_gate, shared_y, T, d, k, rows_max, y, s);
   return combine_k<__nv_bfloat16, __nv_bfloat16>(y_rows, row_of, topk_gate, shared_y, T, d, k, rows_max, y, s);
+}
+
+moe_status launch_round_bf16(float* in, long long n, void* out, int clear, cudaStream_t s) {
+  if (n == 0) return MOE_OK;
+  long long blocks = (n / 8 + 255) / 256;
+  const long long cap = 8LL * num_sms();
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  round_bf16_kernel<<<(unsigned)blocks, 256, 0, s>>>(in, n, static_cast<__nv_bfloat16*>(out), clear);
+  return check_launch();
 }
 
 }  // namespace moe

@@ -46,7 +46,7 @@ class MoELayer:
         """rows_dtype: gated expert rows (and the shared expert's output); out_dtype: y.
         fp32 (the default) leaves H as the only bf16 rounding inside the layer.
         combine: "rows" (gated rows + ordered combine) or "fused" (down GEMM adds into an
-        fp32 y; needs out_dtype fp32).
+        fp32 buffer, rounded once to bf16 at the end when out_dtype is bf16).
         dispatch: "permute" (x_perm copy, then the GEMM) or "gather" (the GEMM reads the
         token rows through token_of_row; same H bit for bit).
         overlap: run the work nothing on the main path waits for (router statistics, and
@@ -57,8 +57,8 @@ class MoELayer:
         self.dispatch_mode = dispatch
         if combine not in ("rows", "fused"):
             raise ValueError(f"combine must be 'rows' or 'fused', got {combine!r}")
-        if combine == "fused" and out_dtype != torch.float32:
-            raise ValueError("combine='fused' accumulates into an fp32 y: out_dtype must be torch.float32")
+        if out_dtype not in (torch.float32, torch.bfloat16):
+            raise ValueError("out_dtype must be torch.float32 or torch.bfloat16")
         self.combine_mode = combine
         w = weights
         self.w = w
@@ -87,6 +87,12 @@ class MoELayer:
         self.h = torch.empty((R, F), dtype=self.dtype, device=dev)
         self.y_perm = torch.empty((R, d), dtype=rows_dtype, device=dev) if combine == "rows" else None
         self.y = torch.empty((T_max, d), dtype=out_dtype, device=dev)
+        # the fused combine's fp32 sums: y itself, or a scratch rounded into a bf16 y at the end
+        self.y32 = None
+        if combine == "fused":
+            # a bf16 y: a separate fp32 buffer, zero at rest (the final rounding clears it)
+            self.y32 = self.y if out_dtype == torch.float32 else torch.zeros((T_max, d), dtype=f32, device=dev)
+        self._y32_at_rest_zero = combine == "fused" and self.y32 is not self.y
         self.load = torch.empty(E, dtype=f32, device=dev)
         self.stats5 = torch.empty(5, dtype=f32, device=dev)
         self.ws = torch.empty(max(M.moe_workspace_bytes(T_max, d, E, k), 16), dtype=torch.uint8, device=dev)
@@ -129,15 +135,20 @@ class MoELayer:
         T = x.shape[0]
         if T != self.T_max:
             self.shared_offsets[1].fill_(T)
-        out = self.y_s[:T] if self.combine_mode == "rows" else self.y[:T]
+        out = self.y_s[:T] if self.combine_mode == "rows" else self.y32[:T]
         M.moe_expert_gate_up(x, self.shared_offsets, self.w.W_gu_s, T, self.h_s[:T], stream)
         M.moe_expert_down(self.h_s[:T], self.shared_offsets, self.w.W_dn_s, T, None, out, stream=stream)
 
     def down_combine(self, T, stream=None, accumulate=None):
-        """accumulate: add onto y as it stands (default: only when the shared expert wrote it)."""
-        acc = self.has_shared if accumulate is None else accumulate
-        M.moe_expert_down_combine(self.h, self.offsets, self.w.W_dn, self.rows_max, self.token_of_row, self.y[:T],
+        """accumulate: add onto y as it stands (default: when the shared expert wrote it, or
+        when y32 is the zero-at-rest scratch of a bf16 output)."""
+        acc = (self.has_shared or self._y32_at_rest_zero) if accumulate is None else accumulate
+        M.moe_expert_down_combine(self.h, self.offsets, self.w.W_dn, self.rows_max, self.token_of_row, self.y32[:T],
                                   self.gate_of_row, accumulate=acc, stream=stream)
+
+    def round_output(self, T, stream=None):
+        """bf16 y from the fused combine's fp32 sums (the combine's final rounding)."""
+        M.moe_round_output(self.y32[:T], self.y[:T], clear=True, stream=stream)
 
     def combine(self, T, stream=None):
         M.moe_combine(self.y_perm, self.row_of[:T], T, self.rows_max, None,
@@ -165,6 +176,8 @@ class MoELayer:
             if self.has_shared:
                 st.append(("shared", lambda s: self.shared(x, s)))
             st.append(("down_combine", lambda s: self.down_combine(T, s)))
+            if self.y32 is not self.y:
+                st.append(("round_output", lambda s: self.round_output(T, s)))
         if with_stats:
             st.append(("stats", lambda s: self.stats(T, s)))
         return st
@@ -195,8 +208,8 @@ class MoELayer:
         fused = self.combine_mode == "fused"
         self._ev_fork.record(s)                  # everything the caller queued before (e.g. a read of y)
         side.wait_event(self._ev_fork)
-        if fused and not self.has_shared:
-            M.moe_zero(self.y[:T], side)         # the fused combine's starting value, off the main path
+        if fused and not self.has_shared and not self._y32_at_rest_zero:
+            M.moe_zero(self.y32[:T], side)       # the fused combine's starting value, off the main path
         run("route", lambda s_: self.route(x, s_))
         run("histogram_scan", lambda s_: self.histogram_scan(T, s_))
         if with_stats:
@@ -214,6 +227,8 @@ class MoELayer:
             self._ev_join.record(side)
             s.wait_event(self._ev_join)
             run("down_combine", lambda s_: self.down_combine(T, s_, accumulate=True))
+            if self.y32 is not self.y:
+                run("round_output", lambda s_: self.round_output(T, s_))
         else:
             run("down", lambda s_: self.down(s_))
             if self.has_shared:
@@ -252,6 +267,8 @@ class MoELayer:
         n = 2 + 2 + 1 + 1 + 1 + 1          # route(2) scan(2) permute gate_up down combine
         if self.combine_mode == "fused":
             n -= 1                         # down_combine (its zero fill is a memset, not a kernel)
+            if self.y32 is not self.y:
+                n += 1                     # round_output
         if self.dispatch_mode == "gather":
             n -= 1                         # no permute
         if self.has_shared:

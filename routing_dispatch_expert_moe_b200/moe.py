@@ -60,6 +60,7 @@ _SIGNATURES = {
     "moe_workspace_bytes": (_size, [_i32, _i32, _i32, _i32]),
     "moe_get_device_error": (_i32, [ctypes.POINTER(_i32), _c_void_p]),
     "moe_zero": (_i32, [_c_void_p, _size, _c_void_p]),
+    "moe_round_output": (_i32, [_c_void_p, _i64, _c_void_p, _i32, _c_void_p]),
 }
 
 _lib = None
@@ -274,6 +275,16 @@ def moe_expert_down(h, offsets, W_dn, rows_max: int, gate_of_row=None, y_rows=No
     _check("moe_expert_down", lib().moe_expert_down(_p(h), _dt(h), _p(offsets), E, d, F, rows_max, _p(W_dn),
                                                     _p(gate_of_row), _dt(y_rows), _p(y_rows), _stream(stream)))
     return y_rows
+
+
+def moe_round_output(y32, y, clear: bool = False, stream=None):
+    """y = bf16_rne(y32): the combine's final rounding of an fp32 sum (clear: zero y32 as it
+    is read, ready for the next accumulation)."""
+    _need(y32, "y32", torch.float32)
+    _need(y, "y", torch.bfloat16, tuple(y32.shape))
+    _check("moe_round_output", lib().moe_round_output(_p(y32), y32.numel(), _p(y), 1 if clear else 0,
+                                                       _stream(stream)))
+    return y
 
 
 def moe_zero(t, stream=None):

@@ -158,6 +158,14 @@ def test_permute_combine_host_validation(L):
     assert L.moe_combine(FAKE, 0, FAKE, NUL, NUL, 64, 128, 4, 256, 5, FAKE, NUL) == 1     # y dtype
 
 
+def test_round_output_host_validation(L):
+    assert L.moe_round_output(NUL, 64, FAKE, 0, NUL) == 1
+    assert L.moe_round_output(FAKE, -1, FAKE, 0, NUL) == 1
+    assert L.moe_round_output(FAKE, 64, FAKE, 2, NUL) == 1
+    assert L.moe_round_output(FAKE, 64, ctypes.c_void_p(4098), 0, NUL) == 2
+    assert L.moe_round_output(NUL, 0, NUL, 1, NUL) == 0
+
+
 def test_zero_host_validation(L):
     assert L.moe_zero(NUL, 64, NUL) == 1
     assert L.moe_zero(ctypes.c_void_p(4100), 64, NUL) == 2

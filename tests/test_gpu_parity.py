@@ -422,3 +422,52 @@ def test_second_stream_schedule_matches_the_sequential_one():
     torch.cuda.synchronize()
     bound = _ordered_terms_bound(rl, cfg2.T, cfg2.k)
     assert (np.abs(y.double().cpu().numpy() - gr["y"]) <= bound + 1e-30).all()
+
+
+def test_round_output_is_round_to_nearest_even_and_clears():
+    from routing_dispatch_expert_moe_b200 import moe as M
+    g = torch.Generator(device="cuda").manual_seed(3)
+    for n in (8 * 1000, 8 * 1000 + 5, 3):                       # vector body and scalar tail
+        y32 = torch.randn(n, device="cuda", generator=g) * 37.0
+        y32[:3] = torch.tensor([1.0 + 2.0 ** -8, -(1.0 + 3 * 2.0 ** -9), 0.0], device="cuda")   # ties to even
+        ref = y32.to(torch.bfloat16)
+        keep = y32.clone()
+        y = torch.empty(n, dtype=torch.bfloat16, device="cuda")
+        M.moe_round_output(y32, y)
+        torch.cuda.synchronize()
+        assert torch.equal(y, ref) and torch.equal(y32, keep)
+        M.moe_round_output(y32, y, clear=True)
+        torch.cuda.synchronize()
+        assert torch.equal(y, ref) and not torch.any(y32)
+
+
+@pytest.mark.parametrize("cfg", [c for c in FUSED if c.name in ("softmax_bf16", "sigmoid_bias_shared", "ragged_multitile")],
+                         ids=lambda c: c.name)
+def test_fused_combine_bf16_output(cfg):
+    """bf16 y: the fp32 sums rounded once.  Against the oracle within the fp32 bars plus one
+    bf16 step of |y|; the fp32 scratch is zero again after every forward, so a second
+    forward (no clearing pass) gives the same result up to the atomics' fp32 order."""
+    host, dev = U.make_inputs(cfg)
+    cap = O.capacity(cfg.T, cfg.E, cfg.k, cfg.capacity_factor, True)
+    lay = U.build_layer(cfg, dev, cap, out_dtype=torch.bfloat16, combine="fused")
+    ys = []
+    for _ in range(2):
+        y = lay.forward(dev["x"])
+        torch.cuda.synchronize()
+        assert y.dtype == torch.bfloat16
+        assert not torch.any(lay.y32)
+        ys.append(y.double().cpu().numpy())
+    from routing_dispatch_expert_moe_b200 import moe as M
+    assert M.moe_get_device_error() == 0
+    gu, dn = U.expert_getters(host)
+    o = O.layer_routing(U.cfg_dict(cfg), host["x"], host["Wg"], host["off"], host["bias"], True)
+    n = int(lay.offsets[-1].item())
+    yp_o = O.grouped_ffn(O.permute(host["x"], o["row_of"], n), o["offsets"], gu, dn, o["gate_of_row"], True)
+    sh = host["shared"]
+    y_s = O.shared_expert(host["x"], sh[0], sh[1], True) if sh is not None else None
+    y_o = O.combine(yp_o, o["row_of"], y_s)
+    rms = float(np.sqrt(np.mean(y_o ** 2)))
+    for y in ys:
+        excess = np.maximum(np.abs(y - y_o) - 2.0 ** -8 * np.abs(y_o), 0.0)
+        assert excess.max() <= U.Y_MAX_REL * rms and excess.mean() <= U.Y_MEAN_REL * rms
+    assert (np.abs(ys[0] - ys[1]) <= 2.0 ** -7 * np.abs(ys[0]) + 1e-30).all()
