@@ -34,11 +34,13 @@ permute_kernel(const uint4* __restrict__ x, int T, int nvec, int k, const int32_
       if (my_row < -1) my_row = -1;
     }
     const uint4* src = x + t * nvec;
-    for (int v0 = lane; v0 < nvec; v0 += 32 * UNROLL) {
+    // warp-uniform trip count: every lane reaches each shuffle below, also when a row has
+    // fewer than 32 vectors (lanes past the row's end only skip their loads and stores)
+    for (int base = 0; base < nvec; base += 32 * UNROLL) {
       uint4 buf[UNROLL];
 #pragma unroll
       for (int u = 0; u < UNROLL; ++u) {
-        const int v = v0 + 32 * u;
+        const int v = base + (int)lane + 32 * u;
         if (v < nvec) buf[u] = ld_stream(src + v);
       }
       for (int j = 0; j < k; ++j) {
@@ -47,7 +49,7 @@ permute_kernel(const uint4* __restrict__ x, int T, int nvec, int k, const int32_
         uint4* dst = x_perm + (long long)r * nvec;
 #pragma unroll
         for (int u = 0; u < UNROLL; ++u) {
-          const int v = v0 + 32 * u;
+          const int v = base + (int)lane + 32 * u;
           if (v < nvec) dst[v] = buf[u];
         }
       }

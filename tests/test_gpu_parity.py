@@ -76,6 +76,11 @@ SMALL = [
     I.small_config("fp32_small", T=200, d=64, E=8, k=2, F=64, act="f32", capacity_factor=1.25),
     I.small_config("bf16_d_below_tile", T=100, d=32, E=4, k=2, F=32),
     I.small_config("sigmoid_nobias_E_odd", T=333, d=96, E=37, k=5, F=40, score="sigmoid"),
+    # the largest supported E and k (32 experts per lane, widest rank tables), biased keys
+    I.small_config("max_E1024_k32", T=300, d=64, E=1024, k=32, F=64, score="sigmoid", scale=2.0,
+                   select_bias="uniform0.1"),
+    # a single expert: the router picks it for every token with gate 1
+    I.small_config("single_expert", T=100, d=64, E=1, k=1, F=64),
 ]
 
 
