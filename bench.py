@@ -190,10 +190,11 @@ def run_ours(args):
     stream = torch.cuda.current_stream()
 
     out_dt = torch.bfloat16 if args.out_dtype == "bf16" else torch.float32
+    rows_dt = torch.bfloat16 if args.rows_dtype == "bf16" else torch.float32
 
     def make_layer(combine, dispatch):
         return MoELayer(w, cfg.k, cfg.T, cfg.score, cfg.renormalize, cfg.scale, cap, combine=combine,
-                        dispatch=dispatch, out_dtype=out_dt)
+                        dispatch=dispatch, out_dtype=out_dt, rows_dtype=rows_dt)
 
     def capture(fn):
         """One CUDA graph of fn(stream), captured on a side stream."""
@@ -284,14 +285,18 @@ def run_ours(args):
     value = job_throughput(cfg.T, world, args.steps, total_ms)
 
     other = None
-    if (args.combine, args.dispatch) != ("rows", "permute") and args.unfused_steps > 0:
-        # the unfused form (permute copy, gated rows, ordered combine: bitwise reproducible), same inputs
-        rl = make_layer("rows", "permute")
-        ps, sm, _, _ = time_layer(rl, args.unfused_steps, breakdown_steps=min(args.breakdown_steps, 50))
+    if args.alt_steps > 0:
+        # the other combine form on the same inputs: fused into the down GEMM (fp32 atomics),
+        # or gated rows + ordered combine (bitwise reproducible)
+        alt = "fused" if args.combine == "rows" else "rows"
+        rl = make_layer(alt, "permute")
+        ps, sm, _, _ = time_layer(rl, args.alt_steps, breakdown_steps=min(args.breakdown_steps, 50))
         t = max_over_ranks(float(ps.sum()), dev)
-        other = {"dispatch": "permute", "combine": "rows (gated rows + ordered combine, bitwise reproducible)",
-                 "ms_per_step": round(t / args.unfused_steps, 4),
-                 "value": round(job_throughput(cfg.T, world, args.unfused_steps, t), 1), "steps": args.unfused_steps,
+        other = {"dispatch": "permute",
+                 "combine": ("fused into the down GEMM (fp32 atomics)" if alt == "fused"
+                             else "gated rows + ordered combine (bitwise reproducible)"),
+                 "ms_per_step": round(t / args.alt_steps, 4),
+                 "value": round(job_throughput(cfg.T, world, args.alt_steps, t), 1), "steps": args.alt_steps,
                  "stages_ms": {k_: round(v, 4) for k_, v in sm.items()}}
         del rl
         torch.cuda.empty_cache()
@@ -386,8 +391,8 @@ def run_ours(args):
                        "F_shared": cfg.F_s, "score": cfg.score, "capacity": cap, "rows": A,
                        "dispatch": ("gathered inside the gate/up GEMM" if gather else "permute copy"),
                        "combine": ("fused into the down GEMM (fp32 atomics into y)" if fused
-                                   else "gated rows + ordered combine"),
-                       "out_dtype": args.out_dtype,
+                                   else "gated rows + ordered combine (bitwise reproducible)"),
+                       "out_dtype": args.out_dtype, "rows_dtype": args.rows_dtype,
                        "parallelism": f"replicas x{world} (independent token batches, no collective)",
                        "l2": "flushed before every step (256 MB write)"},
             "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d_bytes,
@@ -405,7 +410,7 @@ def run_ours(args):
             "stages_ms": {k_: round(v, 4) for k_, v in stage_ms.items()},
             "stage_roofline_ms": {k_: round(v, 4) for k_, v in roof_steps.items()},
             "stage_throughput": thr,
-            "unfused_variant": other,
+            "alt_form": other,
             "clocks": clk,
             "cpu_baseline": cpu,
         }
@@ -520,16 +525,18 @@ def main():
     ap.add_argument("--tokens", type=int, default=None,
                     help="override T (smaller cases of the same kernels, e.g. for profiler captures)")
     ap.add_argument("--e2e-steps", type=int, default=50, help="steps timed through host buffers")
-    ap.add_argument("--combine", choices=["fused", "rows"], default="fused",
-                    help="fused: combine inside the down GEMM; rows: gated rows + ordered combine")
+    ap.add_argument("--combine", choices=["fused", "rows"], default="rows",
+                    help="rows: gated rows + ordered combine (reproducible); fused: combine inside the down GEMM")
     ap.add_argument("--dispatch", choices=["gather", "permute"], default="permute",
                     help="gather: the gate/up GEMM reads token rows through the row map; permute: x_perm copy")
     ap.add_argument("--out-dtype", choices=["bf16", "f32"], default="bf16",
                     help="dtype of the layer output y (bf16: fp32 sums rounded once at the end)")
+    ap.add_argument("--rows-dtype", choices=["f32", "bf16"], default="bf16",
+                    help="dtype of the gated expert rows (the combine='rows' form's down GEMM output)")
     ap.add_argument("--breakdown-steps", type=int, default=100,
                     help="sequential replays for the per-stage split (0 = skip)")
-    ap.add_argument("--unfused-steps", type=int, default=100,
-                    help="also time the unfused form (permute + rows) for this many steps (0 = skip)")
+    ap.add_argument("--alt-steps", type=int, default=100,
+                    help="also time the other combine form for this many steps (0 = skip)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

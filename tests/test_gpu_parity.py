@@ -475,4 +475,54 @@ def test_fused_combine_bf16_output(cfg):
     for y in ys:
         excess = np.maximum(np.abs(y - y_o) - 2.0 ** -8 * np.abs(y_o), 0.0)
         assert excess.max() <= U.Y_MAX_REL * rms and excess.mean() <= U.Y_MEAN_REL * rms
-    assert (np.abs(ys[0] - ys[1]) <= 2.0 ** -7 * np.abs(ys[0]) + 1e-30).all()
+    # two fp32 sums of the same terms in different atomic orders differ by at most
+    # k 2^-23 sum|terms| (cancellation can make that large next to |y|), and each is then
+    # rounded to bf16 (one step of the larger one)
+    row_of = o["row_of"]
+    terms = np.where(row_of[..., None] >= 0, np.abs(yp_o[np.maximum(row_of, 0)]), 0.0).sum(axis=1)
+    if y_s is not None:
+        terms = terms + np.abs(y_s)
+    bound = 2.0 ** -7 * np.maximum(np.abs(ys[0]), np.abs(ys[1])) + 2.0 * cfg.k * 2.0 ** -23 * terms
+    assert (np.abs(ys[0] - ys[1]) <= bound + 1e-30).all()
+
+
+# ---------------------------------------------------------------- bf16 rows and bf16 y at full size
+def bf16_full_size_check(name):
+    """The rounding points of the definition: gated rows rounded to bf16, y rounded to bf16
+    (the form bench.py times).  Routing in full, rows and y on the stratified token sample,
+    against bounds derived from every rounding point."""
+    cfg = I.CONFIGS[name]
+    host, dev = U.make_inputs(cfg)
+    cap = O.capacity(cfg.T, cfg.E, cfg.k, cfg.capacity_factor, True)
+    layer, g = U.gpu_forward(cfg, dev, cap, torch.bfloat16, torch.bfloat16)
+    o = O.layer_routing(U.cfg_dict(cfg), host["x"], host["Wg"], host["off"], host["bias"], True)
+    U.assert_routing_equal(g, o)
+    toks = U.stratified_tokens(o, cap)
+    gu, dn = U.expert_getters(host)
+    sub = O.layer_outputs_for_tokens(toks, host["x"], o, gu, dn, True, shared=host["shared"], round_rows=True,
+                                     round_out=True)
+    rows = o["row_of"][toks]
+    kept = rows >= 0
+    ii, jj = np.nonzero(kept)
+    hb = U.row_bounds(host["x"], toks[ii], o["topk_idx"][toks][ii, jj], o["topk_gate"][toks][ii, jj], gu, dn)
+    yp_g = layer.y_perm[torch.from_numpy(rows[kept]).long().cuda()].float().cpu().numpy()
+    U.assert_rows_close(yp_g, sub["slot_rows"][kept], hb, "y_perm bf16 (sampled)", rows_bf16=True)
+    slot_hb = np.zeros_like(sub["slot_rows"])
+    slot_hb[ii, jj] = hb
+    ys = None
+    if host["shared"] is not None:
+        xs = np.asarray(host["x"])[toks]
+        ys = O.shared_expert(xs, host["shared"][0], host["shared"][1], True, round_out=True)
+    U.assert_y_close_bf16(g["y"][toks], sub["y"], sub["slot_rows"], slot_hb, ys)
+    del layer, dev
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.slow
+def test_c2_handbook_full_size_bf16_rows_and_output():
+    bf16_full_size_check("c2_handbook")
+
+
+@pytest.mark.slow
+def test_c3_fine_grained_full_size_bf16_rows_and_output():
+    bf16_full_size_check("c3_fine_grained")
