@@ -34,7 +34,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM traffic (read + write bytes) of the dominant kernel, the gate/up GEMM, per launch, keyed
 # by (workload, dispatch), from an ncu capture of the same kernel build (summaries under
 # profiles/); absent when the kernel changed since the capture.
-GATE_UP_TRAFFIC = {("c2_handbook", "permute"): 805551104 + 122634752}
+GATE_UP_TRAFFIC = {("c2_handbook", "permute"): 808491520 + 126081024}
 
 
 def peaks():
