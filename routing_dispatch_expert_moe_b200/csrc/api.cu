@@ -38,7 +38,6 @@ constexpr long long kMaxT = 1LL << 24;
 inline cudaStream_t S(void* s) { return static_cast<cudaStream_t>(s); }
 
 bool dtype_ok(int32_t dt) { return dt == MOE_BF16 || dt == MOE_F32; }
-int esize(int32_t dt) { return dt == MOE_F32 ? 4 : 2; }
 
 moe_status check_dims(int32_t T, int32_t E, int32_t k) {
   if (T < 0 || E < 1 || k < 1 || k > E) return MOE_ERR_INVALID_ARG;

@@ -5,7 +5,8 @@
 // (experts receive uneven numbers of tokens; handle them without padding or drops).
 // SwiGLU form: H = silu(X Wg^T) * (X Wu^T), Y = gate * (H Wd^T), no biases.
 //
-// One persistent kernel template, two epilogues:
+// Two persistent kernel templates (single CTA, and CTA pairs below), one per-mode
+// producer and epilogue:
 //   MODE 0 (gate_up): A = X [rows, d], B = W_gu[e] ([2F, d], gate rows then up rows).
 //       A 256-wide B tile holds 128 gate rows and the matching 128 up rows, so one
 //       128x256 accumulator carries g (columns 0..127) and u (128..255) for the same
@@ -20,7 +21,10 @@
 //       token matrix, A row r = x[token_of_row[r]], so no permuted copy of x is written
 //       or read.  The producer warp copies them with 16-byte cp.async into the same
 //       128-byte-swizzled layout TMA writes; B still arrives by TMA.
-//   MODE 2 (router logits on the tensor cores, see below).
+//   MODE 2 (router): A = x [T, d], B = the exact three-term bf16 split of W_g (hi, mid,
+//       lo rows per 64 experts); N = 192 MMAs; the epilogue sums the three terms and the
+//       logit offset in fp32.  Tiles walk n fastest (the split weight is small; each slice
+//       of x is read once).
 //
 // Per CTA (1 per SM, 192 threads):
 //   warp 0   TMA producer: 128x64 A tile + 256x64 B tile per stage (128-byte swizzle),
@@ -34,6 +38,9 @@
 // writes a row outside its expert's range or a column outside the output width.
 // Every barrier wait is bounded (MOE_DEVERR_PIPE_TIMEOUT, then an orderly exit: MMAs
 // drained, outstanding TMA loads awaited, TMEM freed).
+// The CTA-pair kernel (further below) runs 256x256 tiles over two SMs with cta_group::2
+// MMAs; it is used when groups average at least 256 rows.  No load uses cluster
+// multicast.
 #include <cuda.h>
 
 #include "common.cuh"
