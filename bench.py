@@ -64,6 +64,12 @@ def job_throughput(tokens_per_rank: int, world: int, steps: int, total_ms: float
     return tokens_per_rank * world * steps / (total_ms / 1e3)
 
 
+def workload_config(name: str, cfg, cap: int) -> dict:
+    """The workload identity both arms report (the same keys and values in each line)."""
+    return {"workload": name, "T": cfg.T, "d": cfg.d, "E": cfg.E, "k": cfg.k, "F": cfg.F, "F_shared": cfg.F_s,
+            "score": cfg.score, "capacity": cap}
+
+
 def replica_seed(rank: int) -> int:
     """Seed of a replica's token batch: every rank gets its own batch, same weights."""
     return rank
@@ -387,8 +393,7 @@ def run_ours(args):
             "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if dt == torch.bfloat16 else "f32",
             "data": "synthetic (seeded; integer-grid router inputs, N(0,0.02) bf16 expert weights)",
-            "config": {"workload": args.workload, "T": cfg.T, "d": cfg.d, "E": cfg.E, "k": cfg.k, "F": cfg.F,
-                       "F_shared": cfg.F_s, "score": cfg.score, "capacity": cap, "rows": A,
+            "config": {**workload_config(args.workload, cfg, cap), "rows": A,
                        "dispatch": ("gathered inside the gate/up GEMM" if gather else "permute copy"),
                        "combine": ("fused into the down GEMM (fp32 atomics into y)" if fused
                                    else "gated rows + ordered combine (bitwise reproducible)"),
@@ -486,6 +491,7 @@ def run_reference(args):
     rank, _, world = env_rank()
     if rank != 0:
         return None
+    from oracle import moe_oracle as O
     from routing_dispatch_expert_moe_b200 import inputs as I
     cfg = I.CONFIGS[args.workload]
     setup = _oracle_setup(cfg)
@@ -506,7 +512,7 @@ def run_reference(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total / args.steps * 1e3, 2),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded)",
-            "config": {"workload": args.workload, "T": cfg.T, "d": cfg.d, "E": cfg.E, "k": cfg.k, "F": cfg.F},
+            "config": workload_config(args.workload, cfg, O.capacity(cfg.T, cfg.E, cfg.k, cfg.capacity_factor, True)),
             "cpu_baseline": {"value": round(value, 2), "unit": UNIT, "cores": _threads(), "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": round(value, 2), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
