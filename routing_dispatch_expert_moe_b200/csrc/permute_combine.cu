@@ -102,13 +102,17 @@ __device__ __forceinline__ void store8<float>(void* base, long long e, const flo
   p[1] = make_float4(f[4], f[5], f[6], f[7]);
 }
 
-// KMAX: compile-time bound on k (multiple of 8); a token's rows are loaded 8 slots at a
-// time (8 independent loads in flight per lane) and added in slot order.
+// KMAX: compile-time bound on k (multiple of 8).  The token's kept slots are first
+// compacted, in slot order, into krow / kgate (warp-uniform, static register indices), so
+// dropped slots cost nothing and every batch of loads is full.  Each lane then loads up to
+// 8 kept rows for VPI consecutive 8-element vectors (8 * VPI independent loads in flight)
+// and adds them in slot order: the same fp32 sum as visiting every slot.
 template <typename InT, typename OutT, int KMAX>
 __global__ void __launch_bounds__(256)
 combine_kernel(const void* __restrict__ y_rows, const int32_t* __restrict__ row_of,
                const float* __restrict__ topk_gate, const void* __restrict__ shared_y, int T, int d, int k,
                long long rows_max, void* __restrict__ y, int* err) {
+  constexpr int VPI = sizeof(InT) == 2 ? 2 : 1;       // vectors per lane per step
   const unsigned lane = threadIdx.x & 31;
   const int warps = blockDim.x >> 5;
   const long long nw = (long long)gridDim.x * warps;
@@ -123,33 +127,56 @@ combine_kernel(const void* __restrict__ y_rows, const int32_t* __restrict__ row_
       if (my_row < -1) my_row = -1;
       if (scale) my_gate = __ldg(topk_gate + t * k + lane);
     }
-    int rows[KMAX];
-    float gates[KMAX];
+    // kept slots in slot order -> positions 0 .. nk-1 (all lanes hold the same values)
+    int krow[KMAX];
+    float kgate[KMAX];
+#pragma unroll
+    for (int p = 0; p < KMAX; ++p) { krow[p] = -1; kgate[p] = 0.f; }
+    int nk = 0;
 #pragma unroll
     for (int j = 0; j < KMAX; ++j) {
-      rows[j] = __shfl_sync(0xffffffffu, my_row, j & 31);
-      gates[j] = __shfl_sync(0xffffffffu, my_gate, j & 31);
-    }
-    for (int v = lane; v < n8; v += 32) {
-      float acc[8];
+      const int r = __shfl_sync(0xffffffffu, my_row, j & 31);
+      const float g = __shfl_sync(0xffffffffu, my_gate, j & 31);
+      if (j < k && r >= 0) {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+        for (int p = 0; p <= j; ++p)
+          if (p == nk) { krow[p] = r; kgate[p] = g; }
+        ++nk;
+      }
+    }
+    for (int v0 = lane; v0 < n8; v0 += 32 * VPI) {
+      float acc[VPI][8];
+#pragma unroll
+      for (int u = 0; u < VPI; ++u)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[u][i] = 0.f;
 #pragma unroll
       for (int j0 = 0; j0 < KMAX; j0 += 8) {
-        Row8<InT> buf[8];
+        if (j0 >= nk) break;
+        Row8<InT> buf[VPI][8];
 #pragma unroll
         for (int jj = 0; jj < 8; ++jj)
-          if (rows[j0 + jj] >= 0) buf[jj].load(y_rows, (long long)rows[j0 + jj] * d + v * 8);
+#pragma unroll
+          for (int u = 0; u < VPI; ++u)
+            if (j0 + jj < nk && v0 + 32 * u < n8)
+              buf[u][jj].load(y_rows, (long long)krow[j0 + jj] * d + (v0 + 32 * u) * 8);
 #pragma unroll
         for (int jj = 0; jj < 8; ++jj)
-          if (rows[j0 + jj] >= 0) buf[jj].add(acc, gates[j0 + jj], scale);
+#pragma unroll
+          for (int u = 0; u < VPI; ++u)
+            if (j0 + jj < nk && v0 + 32 * u < n8) buf[u][jj].add(acc[u], kgate[j0 + jj], scale);
       }
-      if (shared_y) {
-        Row8<InT> sv;
-        sv.load(shared_y, t * d + v * 8);
-        sv.add(acc, 1.f, false);
+#pragma unroll
+      for (int u = 0; u < VPI; ++u) {
+        const int v = v0 + 32 * u;
+        if (v >= n8) continue;
+        if (shared_y) {
+          Row8<InT> sv;
+          sv.load(shared_y, t * d + v * 8);
+          sv.add(acc[u], 1.f, false);
+        }
+        store8<OutT>(y, t * d + v * 8, acc[u]);
       }
-      store8<OutT>(y, t * d + v * 8, acc);
     }
   }
 }
