@@ -52,6 +52,12 @@ Readings taken where the pages are silent (each listed again in the design notes
   R15 aux loss = E * sum_e f_e P_e with f_e the pre-drop fraction of assignments
      and P_e the mean routing probability (softmax, or scores / their sum).
   R16 z-loss = mean_t (logsumexp_e l[t,e])^2.
+  R20 forced-uniform routing: slot j of token t takes expert (t k + j) mod E.
+  R21 hash routing: Floyd's sampling of k distinct experts driven by the MurmurHash3
+     finalizer of the token id (hash_experts).
+  R22 the fixed rules keep the learned path's gates over the chosen experts.
+  R23 noisy top-k: the standard normal draws are an input; KeepTopK on H with ties to
+     the lower index; gates = Softmax over the kept H.
 
 Parity status: every function here is pinned by the CPU tests (brute force,
 closed forms, invariants, hand-derived golden fixtures); none is "parity unpinned".
@@ -182,6 +188,103 @@ def decision_margin(keys: np.ndarray, k: int) -> np.ndarray:
         return np.full(keys.shape[0], np.inf)
     s = -np.sort(-np.asarray(keys, np.float64), axis=1)
     return s[:, k - 1] - s[:, k]
+
+
+# ---------------------------------------------------------------------------
+# Routing variants
+#   forced-uniform selection: [Handbook-News] "真正难在三个环节" item 2 (a control run
+#     that forced routing to be uniform was about 1.5x faster; it shows the speed
+#     headroom only, not a training recipe);
+#   hash selection by token id: [Handbook-Digest] "已确认", routing bullet (the first
+#     three MoE layers of DeepSeek-V4 choose experts by a fixed hash of the token id);
+#   noisy top-k: [MoE-Explained] "什么是稀疏性？", eq. H(x)_i = (x.W_g)_i +
+#     StandardNormal() * Softplus((x.W_noise)_i), then KeepTopK and Softmax.
+# The pages give neither the hash nor the gates of the fixed rules (R20-R23).
+# ---------------------------------------------------------------------------
+MASK32 = 0xFFFFFFFF
+
+
+def fmix32(h: int) -> int:
+    """The MurmurHash3 32-bit finalizer (Appleby): two xor-shift-multiply rounds and a
+    final xor-shift, all modulo 2^32.  A bijection on 32-bit words."""
+    h &= MASK32
+    h ^= h >> 16
+    h = (h * 0x85EBCA6B) & MASK32
+    h ^= h >> 13
+    h = (h * 0xC2B2AE35) & MASK32
+    h ^= h >> 16
+    return h
+
+
+def floyd_sample(words, E: int, k: int) -> list:
+    """k distinct values out of range(E) from k 32-bit words, by Floyd's sampling
+    (Bentley and Floyd, "A sample of brilliance"): for j = 0 .. k-1 with n = E - k + j,
+    r = words[j] mod (n + 1); take r unless it is already taken, else take n (never
+    taken yet: earlier picks are all below it).  With uniform words every k-subset is
+    equally likely (up to the modulo bias of a 32-bit word).  Keeps the draw order."""
+    if not 1 <= k <= E:
+        raise ValueError("need 1 <= k <= E")
+    chosen = []
+    for j in range(k):
+        n = E - k + j
+        r = int(words[j]) % (n + 1)
+        chosen.append(n if r in chosen else r)
+    return chosen
+
+
+def hash_experts(token_id: int, seed: int, E: int, k: int) -> list:
+    """The k experts of a token id (R21): floyd_sample of the words
+    h_j = fmix32(fmix32(id xor seed) + j), j = 0 .. k-1."""
+    base = fmix32((token_id & MASK32) ^ (seed & MASK32))
+    return floyd_sample([fmix32((base + j) & MASK32) for j in range(k)], E, k)
+
+
+def fixed_selection(T: int, E: int, k: int, rule: str, token_id=None, seed: int = 0) -> np.ndarray:
+    """topk_idx [T, k] of a fixed rule.
+
+    "uniform" (R20): slot j of token t takes expert (t k + j) mod E, so every expert
+      receives floor(T k / E) or ceil(T k / E) assignments;
+    "hash" (R21): hash_experts(token_id[t], seed, E, k).
+    """
+    if not 1 <= k <= E:
+        raise ValueError("need 1 <= k <= E")
+    idx = np.empty((T, k), np.int32)
+    for t in range(T):
+        if rule == "uniform":
+            idx[t] = [(t * k + j) % E for j in range(k)]
+        elif rule == "hash":
+            idx[t] = hash_experts(int(token_id[t]), seed, E, k)
+        else:
+            raise ValueError(rule)
+    return idx
+
+
+def route_fixed(logits, k: int, score: str, renormalize: bool, scale: float, rule: str,
+                token_id=None, seed: int = 0) -> dict:
+    """A fixed selection rule with the learned path's gates over the chosen experts (R22)."""
+    l = np.asarray(logits, np.float64)
+    idx = fixed_selection(l.shape[0], l.shape[1], k, rule, token_id, seed)
+    return {"topk_idx": idx, "topk_gate": gates(l, idx, score, renormalize, scale)}
+
+
+def softplus(z):
+    """log(1 + e^z), written max(z, 0) + log1p(e^-|z|) (same value, no overflow)."""
+    z = np.asarray(z, np.float64)
+    return np.maximum(z, 0.0) + np.log1p(np.exp(-np.abs(z)))
+
+
+def noisy_logits(logits, logits_noise, noise) -> np.ndarray:
+    """H = l + n * softplus(l_noise) ([MoE-Explained] eq. H(x)_i; the StandardNormal()
+    draws n are an input, R23)."""
+    return np.asarray(logits, np.float64) + np.asarray(noise, np.float64) * softplus(logits_noise)
+
+
+def route_noisy(logits, logits_noise, noise, k: int, scale: float = 1.0) -> dict:
+    """Noisy top-k gating: KeepTopK on H (ties to the lower index), then the softmax over
+    the kept H ([MoE-Explained] eq. G(x) = Softmax(KeepTopK(H(x), k))), times scale."""
+    H = noisy_logits(logits, logits_noise, noise)
+    idx = top_k(H, k)
+    return {"H": H, "topk_idx": idx, "topk_gate": gates(H, idx, "softmax", True, scale)}
 
 
 # ---------------------------------------------------------------------------
