@@ -184,12 +184,24 @@ def run_ours(args):
     Wg, off, bias = I.gen_router(cfg, 0)
     W_gu, W_dn = I.gen_experts_torch(cfg, 0)
     sh = I.gen_shared(cfg, 0)
+    routing = args.routing
+    if routing != "learned" and bias is not None:
+        bias = None                                     # a fixed rule has no selection to bias
     w = MoEWeights(Wg=torch.from_numpy(Wg).to(dev), W_gu=W_gu.to(dev), W_dn=W_dn.to(dev),
                    logit_offset=None if off is None else torch.from_numpy(off).to(dev),
                    select_bias=None if bias is None else torch.from_numpy(bias).to(dev),
                    W_gu_s=None if sh is None else torch.from_numpy(sh[0]).to(dt).unsqueeze(0).to(dev),
-                   W_dn_s=None if sh is None else torch.from_numpy(sh[1]).to(dt).unsqueeze(0).to(dev))
+                   W_dn_s=None if sh is None else torch.from_numpy(sh[1]).to(dt).unsqueeze(0).to(dev),
+                   W_noise=(torch.from_numpy(I.gen_noise_router(cfg, 0)).to(dev) if routing == "noisy" else None))
     del W_gu, W_dn
+    # the routing rule's own per-batch inputs (token ids for hash routing, normal draws for
+    # noisy top-k), resident like x
+    rin_np = {}
+    if routing == "hash":
+        rin_np["token_id"] = I.gen_token_ids(cfg, seed=replica_seed(rank))
+    elif routing == "noisy":
+        rin_np["noise"] = I.gen_noise(cfg, seed=replica_seed(rank))
+    rin = {k_: torch.from_numpy(v).to(dev) for k_, v in rin_np.items()}
     cap = M.moe_capacity(cfg.T, cfg.E, cfg.k, cfg.capacity_factor, True)
     x = torch.from_numpy(x_np).to(dt).to(dev)
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
@@ -200,7 +212,7 @@ def run_ours(args):
 
     def make_layer(combine, dispatch):
         return MoELayer(w, cfg.k, cfg.T, cfg.score, cfg.renormalize, cfg.scale, cap, combine=combine,
-                        dispatch=dispatch, out_dtype=out_dt, rows_dtype=rows_dt)
+                        dispatch=dispatch, out_dtype=out_dt, rows_dtype=rows_dt, routing=routing)
 
     def capture(fn):
         """One CUDA graph of fn(stream), captured on a side stream."""
@@ -222,7 +234,7 @@ def run_ours(args):
         mean ms per stage, the rows processed and the clock record."""
         for _ in range(args.warmup):
             flush.zero_()
-            layer.forward(x, stream)
+            layer.forward(x, stream, **rin)
         torch.cuda.synchronize()
         assert M.moe_get_device_error() == 0
         rows = int(layer.offsets[-1].item())
@@ -231,7 +243,7 @@ def run_ours(args):
 
         def fwd(s):
             ev[0].record(s)
-            layer.forward(x, s, marks={gu_name: (ev[2], ev[3])})
+            layer.forward(x, s, marks={gu_name: (ev[2], ev[3])}, **rin)
             ev[1].record(s)
 
         graph = capture(fwd)
@@ -262,7 +274,7 @@ def run_ours(args):
 
         stage_ms = {"timed_" + gu_name: gu_ms / steps}
         if breakdown_steps > 0:
-            stages = layer.stages(x)
+            stages = layer.stages(x, True, rin.get("token_id"), rin.get("noise"))
             evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(stages) + 1)]
 
             def seq(s):
@@ -317,9 +329,13 @@ def run_ours(args):
     e2e_steps = max(3, args.e2e_steps)
     lays = [layer, make_layer(args.combine, args.dispatch)]
     xs = [x, torch.empty_like(x)]
-    for l_, x_ in zip(lays, xs):
+    rin_host = {k_: torch.from_numpy(v).pin_memory() for k_, v in rin_np.items()}
+    rins = [rin, {k_: torch.empty_like(v) for k_, v in rin.items()}]
+    for l_, x_, r_ in zip(lays, xs, rins):
         x_.copy_(x_host)
-        l_.capture(x_)                     # the layer's public graph API: capture once, replay per batch
+        for k_, v in rin_host.items():
+            r_[k_].copy_(v)
+        l_.capture(x_, token_id=r_.get("token_id"), noise=r_.get("noise"))   # capture once, replay per batch
     s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
     ev_in, ev_comp, ev_out = ([torch.cuda.Event() for _ in range(2)] for _ in range(3))
 
@@ -329,6 +345,8 @@ def run_ours(args):
             s_in.wait_event(ev_comp[b])    # the forward that last read xs[b] has finished
             with torch.cuda.stream(s_in):
                 xs[b].copy_(x_host, non_blocking=True)
+                for k_, v in rin_host.items():
+                    rins[b][k_].copy_(v, non_blocking=True)
             ev_in[b].record(s_in)
             s_comp.wait_event(ev_in[b])
             s_comp.wait_event(ev_out[b])   # the copy-out that last read lays[b].y has finished
@@ -358,7 +376,8 @@ def run_ours(args):
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
     e2e_value = job_throughput(cfg.T, world, e2e_steps, e2e_ms)
-    h2d_bytes = x_host.numel() * x_host.element_size()
+    h2d_bytes = x_host.numel() * x_host.element_size() + sum(v.numel() * v.element_size()
+                                                             for v in rin_host.values())
     d2h_bytes = y_host[0].numel() * y_host[0].element_size()
     del lays
 
@@ -387,7 +406,8 @@ def run_ours(args):
 
     out = None
     if rank == 0:
-        cpu = cpu_baseline(cfg, budget_s=args.cpu_budget) if (world == 1 and not args.no_cpu_baseline) else None
+        cpu = (cpu_baseline(cfg, budget_s=args.cpu_budget)
+               if (world == 1 and not args.no_cpu_baseline and routing == "learned") else None)
         out = {
             "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
@@ -398,6 +418,7 @@ def run_ours(args):
                        "combine": ("fused into the down GEMM (fp32 atomics into y)" if fused
                                    else "gated rows + ordered combine (bitwise reproducible)"),
                        "out_dtype": args.out_dtype, "rows_dtype": args.rows_dtype,
+                       **({"routing": routing} if routing != "learned" else {}),
                        "parallelism": f"replicas x{world} (independent token batches, no collective)",
                        "l2": "flushed before every step (256 MB write)"},
             "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d_bytes,
@@ -539,6 +560,9 @@ def main():
                     help="dtype of the layer output y (bf16: fp32 sums rounded once at the end)")
     ap.add_argument("--rows-dtype", choices=["f32", "bf16"], default="bf16",
                     help="dtype of the gated expert rows (the combine='rows' form's down GEMM output)")
+    ap.add_argument("--routing", choices=["learned", "uniform", "hash", "noisy"], default="learned",
+                    help="expert selection: the learned top-k (the layer's definition), forced-uniform, a hash "
+                         "of synthetic Zipf token ids, or noisy top-k (softmax workloads); not the reference arm")
     ap.add_argument("--breakdown-steps", type=int, default=100,
                     help="sequential replays for the per-stage split (0 = skip)")
     ap.add_argument("--alt-steps", type=int, default=100,
@@ -546,6 +570,8 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.impl == "reference" and args.routing != "learned":
+        ap.error("--routing applies to our arm only (the oracle arm times the learned router)")
     out = run_reference(args) if args.impl == "reference" else run_ours(args)
     if out is not None:
         print(json.dumps(out), flush=True)

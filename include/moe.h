@@ -91,6 +91,11 @@ typedef enum {
 
 typedef enum { MOE_BF16 = 0, MOE_F32 = 1 } moe_dtype;
 
+typedef enum {
+  MOE_SELECT_UNIFORM = 0,       /* slot j of token t takes expert (t k + j) mod E        */
+  MOE_SELECT_HASH = 1           /* k distinct experts from a hash of the token id         */
+} moe_select_rule;
+
 /* Device error codes recorded by kernels (first one wins until read). */
 #define MOE_DEVERR_NONE 0
 #define MOE_DEVERR_EXPERT_ID 1      /* a topk_idx entry outside [0, E)                   */
@@ -143,6 +148,76 @@ MOE_API moe_status moe_route(const void* x, int32_t x_dtype, const float* Wg,
                      int32_t score, int32_t renormalize, float scale,
                      float* logits, int32_t* topk_idx, float* topk_gate,
                      void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------------------
+ * moe_router_logits -- the router alone: logits = x . Wg (+ logit_offset), fp32.
+ * [MoE-Explained] section "什么是稀疏性？" (x . W_g); section "Switch Transformer"
+ * (router in full precision); [Handbook-News] "真正难在三个环节" item 1 (FP32 routing).
+ * The same GEMM as moe_route (bf16 x with d >= 64 and E % 4 == 0: tensor cores with
+ * W_g split exactly into three bf16 terms; otherwise fp32 SIMT), without the top-k.  It
+ * also gives the noise logits x . W_noise of moe_route_noisy.
+ *   x            (device) [T, d], x_dtype;  16-byte aligned
+ *   Wg           (device) [d, E] fp32
+ *   logit_offset (device) [E] fp32 or NULL
+ *   logits       (device) [T, E] fp32 out
+ *   workspace    (device) >= moe_router_logits_workspace_bytes(T, d, E) bytes (may be
+ *                NULL if 0)
+ * Errors: INVALID_ARG for a null pointer, T < 0, E < 1 or an unknown dtype;
+ * UNSUPPORTED for E > 1024, d % 8 != 0 or an unaligned x; WORKSPACE if too small.
+ * ---------------------------------------------------------------------------------- */
+MOE_API size_t moe_router_logits_workspace_bytes(int32_t T, int32_t d, int32_t E);
+MOE_API moe_status moe_router_logits(const void* x, int32_t x_dtype, const float* Wg,
+                     const float* logit_offset, int32_t T, int32_t d, int32_t E,
+                     float* logits, void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------------------
+ * moe_route_fixed -- a fixed selection rule with the learned router's gates.
+ * MOE_SELECT_UNIFORM: [Handbook-News] "真正难在三个环节" item 2 (a control run with
+ *   routing forced uniform was about 1.5x faster: the speed headroom of balance).  Slot
+ *   j of token t takes expert (t k + j) mod E, so every expert receives floor(T k / E)
+ *   or ceil(T k / E) assignments.
+ * MOE_SELECT_HASH: [Handbook-Digest] "已确认" (DeepSeek-V4's first three MoE layers
+ *   choose experts by a fixed hash of the token id).  Floyd's sampling of k distinct
+ *   experts: with base = fmix32(token_id[t] ^ seed) (fmix32 = MurmurHash3's 32-bit
+ *   finalizer) and, for j = 0 .. k-1, n = E - k + j and r = fmix32(base + j) mod (n + 1),
+ *   slot j takes r unless an earlier slot holds it, else n.  Same id, same experts.
+ *   logits      (device) [T, E] fp32: the router logits (moe_router_logits)
+ *   score, renormalize, scale: as moe_route; the gates of the chosen experts follow
+ *               moe_route's rule (softmax over the chosen logits, the full softmax
+ *               probability, or the chosen scores over their sum / the scores) x scale
+ *   rule        moe_select_rule
+ *   token_id    (device) [T] int32 for MOE_SELECT_HASH (any value), else may be NULL
+ *   seed        mixed into the hash
+ *   topk_idx    (device) [T, k] int32 out, in slot order (not sorted)
+ *   topk_gate   (device) [T, k] fp32 out
+ * Errors: INVALID_ARG for a null pointer, T < 0, k < 1, k > E, an unknown score or rule,
+ * renormalize not 0/1 or a non-finite scale; UNSUPPORTED for E > 1024 or k > 32.
+ * ---------------------------------------------------------------------------------- */
+MOE_API moe_status moe_route_fixed(const float* logits, int32_t T, int32_t E, int32_t k,
+                     int32_t score, int32_t renormalize, float scale, int32_t rule,
+                     const int32_t* token_id, uint32_t seed, int32_t* topk_idx,
+                     float* topk_gate, void* stream);
+
+/* ------------------------------------------------------------------------------------
+ * moe_route_noisy -- noisy top-k gating.
+ * [MoE-Explained] section "什么是稀疏性？": H(x)_i = (x . W_g)_i + StandardNormal() *
+ * Softplus((x . W_noise)_i); G(x) = Softmax(KeepTopK(H(x), k)).
+ *   logits       (device) [T, E] fp32: x . W_g (+ offset)
+ *   logits_noise (device) [T, E] fp32: x . W_noise (moe_router_logits with W_noise)
+ *   noise        (device) [T, E] fp32: the standard normal draws, supplied by the caller
+ *   scale        multiplies the gates
+ *   H            (device) [T, E] fp32 out: l + n * softplus(l_noise) in fp32, softplus
+ *                as max(z, 0) + log1p(exp(-|z|)), one rounding for the product and sum;
+ *                must not overlap the inputs
+ *   topk_idx     (device) [T, k] int32 out: the k largest H, ties to the lower index,
+ *                order H descending then index ascending
+ *   topk_gate    (device) [T, k] fp32 out: softmax over the kept H, x scale
+ * Errors: INVALID_ARG for a null pointer, T < 0, k < 1, k > E or a non-finite scale;
+ * UNSUPPORTED for E > 1024 or k > 32.
+ * ---------------------------------------------------------------------------------- */
+MOE_API moe_status moe_route_noisy(const float* logits, const float* logits_noise,
+                     const float* noise, int32_t T, int32_t E, int32_t k, float scale,
+                     float* H, int32_t* topk_idx, float* topk_gate, void* stream);
 
 /* ------------------------------------------------------------------------------------
  * moe_histogram_scan -- counts, capacity, token-order ranks, offsets, row maps.

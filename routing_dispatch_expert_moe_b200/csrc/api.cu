@@ -112,6 +112,50 @@ moe_status moe_route(const void* x, int32_t x_dtype, const float* Wg, const floa
                       topk_idx, topk_gate, workspace, S(stream));
 }
 
+size_t moe_router_logits_workspace_bytes(int32_t T, int32_t d, int32_t E) {
+  if (T < 0 || d < 1 || E < 1) return 0;
+  return router_logits_workspace_bytes(T, d, E);
+}
+
+moe_status moe_router_logits(const void* x, int32_t x_dtype, const float* Wg, const float* logit_offset, int32_t T,
+                             int32_t d, int32_t E, float* logits, void* workspace, size_t workspace_bytes,
+                             void* stream) {
+  moe_status st = check_dims(T, E, 1);
+  if (st != MOE_OK) return st;
+  if ((st = check_d(d)) != MOE_OK) return st;
+  if (!dtype_ok(x_dtype)) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x || !Wg || !logits) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x)) return MOE_ERR_UNSUPPORTED;
+  const size_t need = router_logits_workspace_bytes(T, d, E);
+  if (need > 0 && (!workspace || workspace_bytes < need)) return MOE_ERR_WORKSPACE;
+  return launch_router_logits(x, x_dtype, Wg, logit_offset, T, d, E, logits, workspace, S(stream));
+}
+
+moe_status moe_route_fixed(const float* logits, int32_t T, int32_t E, int32_t k, int32_t score, int32_t renormalize,
+                           float scale, int32_t rule, const int32_t* token_id, uint32_t seed, int32_t* topk_idx,
+                           float* topk_gate, void* stream) {
+  moe_status st = check_dims(T, E, k);
+  if (st != MOE_OK) return st;
+  if (score < MOE_SCORE_SOFTMAX || score > MOE_SCORE_SQRT_SOFTPLUS || (renormalize != 0 && renormalize != 1) ||
+      !isfinite(scale) || (rule != MOE_SELECT_UNIFORM && rule != MOE_SELECT_HASH))
+    return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!logits || !topk_idx || !topk_gate || (rule == MOE_SELECT_HASH && !token_id)) return MOE_ERR_INVALID_ARG;
+  return launch_route_fixed(logits, T, E, k, score, renormalize, scale, rule, token_id, seed, topk_idx, topk_gate,
+                            S(stream));
+}
+
+moe_status moe_route_noisy(const float* logits, const float* logits_noise, const float* noise, int32_t T, int32_t E,
+                           int32_t k, float scale, float* H, int32_t* topk_idx, float* topk_gate, void* stream) {
+  moe_status st = check_dims(T, E, k);
+  if (st != MOE_OK) return st;
+  if (!isfinite(scale)) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!logits || !logits_noise || !noise || !H || !topk_idx || !topk_gate) return MOE_ERR_INVALID_ARG;
+  return launch_route_noisy(logits, logits_noise, noise, T, E, k, scale, H, topk_idx, topk_gate, S(stream));
+}
+
 size_t moe_histogram_scan_workspace_bytes(int32_t T, int32_t k, int32_t E) {
   if (T < 0 || k < 1 || E < 1) return 0;
   return histogram_scan_workspace_bytes(T, k, E);

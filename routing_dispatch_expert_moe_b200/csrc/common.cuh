@@ -104,6 +104,14 @@ moe_status launch_route(const void* x, int x_dtype, const float* Wg, const float
                         int renormalize, float scale, float* logits, int32_t* topk_idx,
                         float* topk_gate, void* ws, cudaStream_t s);
 size_t route_workspace_bytes(int T, int d, int E);
+moe_status launch_router_logits(const void* x, int x_dtype, const float* Wg, const float* logit_offset, int T,
+                                int d, int E, float* logits, void* ws, cudaStream_t s);
+size_t router_logits_workspace_bytes(int T, int d, int E);
+moe_status launch_route_fixed(const float* logits, int T, int E, int k, int score, int renormalize, float scale,
+                              int rule, const int32_t* token_id, uint32_t seed, int32_t* topk_idx,
+                              float* topk_gate, cudaStream_t s);
+moe_status launch_route_noisy(const float* logits, const float* logits_noise, const float* noise, int T, int E,
+                              int k, float scale, float* H, int32_t* topk_idx, float* topk_gate, cudaStream_t s);
 
 moe_status launch_histogram_scan(const int32_t* topk_idx, const float* topk_gate, int T, int k,
                                  int E, int capacity, int32_t* counts, int32_t* kept,

@@ -361,14 +361,17 @@ topk_kernel(const float* __restrict__ partial, int nsplit, long long split_strid
       }
     }
 
-    // gates (fp32)
+    // gates (fp32 results).  The softmax over the kept logits takes the difference to the
+    // maximum and its exponential in fp64: an fp32 difference of two logits far apart is
+    // itself rounded, by up to half an ulp of the difference, which moves a small gate by
+    // that much relatively; in fp64 the gate is within half an fp32 ulp.
     const bool act = lane < (unsigned)k;
     float g;
     if (score == MOE_SCORE_SOFTMAX) {
       if (renorm) {
         const float m = warp_max(act ? sel_logit : -INFINITY);
-        const float ex = act ? expf(sel_logit - m) : 0.f;
-        g = ex / warp_sum(ex);
+        const double ex = act ? exp((double)sel_logit - (double)m) : 0.0;
+        g = (float)(ex / warp_sum_d(ex));
       } else {
         float mf = -INFINITY;
 #pragma unroll
@@ -506,12 +509,116 @@ moe_status run_topk(bool bias, const float* partial, int nsplit, long long split
   return check_launch();
 }
 
+// ---------------------------------------------------------------------------------
+// Routing variants (the learned router's logits are still computed; only the
+// selection changes, and the gates follow the learned path's rule):
+//   forced-uniform selection: handbook news post, "真正难在三个环节" item 2 (a control
+//     run with routing forced uniform was about 1.5x faster: the speed headroom);
+//   hash selection: handbook digest, "已确认" (DeepSeek-V4 picks the experts of its
+//     first three MoE layers by a fixed hash of the token id);
+//   noisy top-k: "Mixture of Experts Explained", section "什么是稀疏性？", eq.
+//     H(x)_i = (x.W_g)_i + StandardNormal() * Softplus((x.W_noise)_i).
+// ---------------------------------------------------------------------------------
+
+// MurmurHash3's 32-bit finalizer (Appleby): a bijection on 32-bit words.
+__device__ __forceinline__ uint32_t fmix32(uint32_t h) {
+  h ^= h >> 16;
+  h *= 0x85ebca6bu;
+  h ^= h >> 13;
+  h *= 0xc2b2ae35u;
+  h ^= h >> 16;
+  return h;
+}
+
+// One warp per token; lane j < k owns slot j.
+//   uniform: slot j of token t takes expert (t k + j) mod E;
+//   hash:    Floyd's sampling of k distinct experts out of E, draw j from the word
+//            fmix32(fmix32(id ^ seed) + j): with n = E - k + j, r = word mod (n + 1);
+//            slot j takes r unless an earlier slot holds it (one ballot), else n.
+// Gates as in topk_kernel, over the chosen experts' logits.
+__global__ void __launch_bounds__(256)
+fixed_select_kernel(const float* __restrict__ logits, int T, int E, int k, int score, int renorm,
+                    float scale, int rule, const int32_t* __restrict__ token_id, uint32_t seed,
+                    int32_t* __restrict__ topk_idx, float* __restrict__ topk_gate) {
+  const unsigned lane = threadIdx.x & 31;
+  const int warps = blockDim.x >> 5;
+  const long long gw = (long long)blockIdx.x * warps + (threadIdx.x >> 5);
+  const long long nw = (long long)gridDim.x * warps;
+  const bool act = lane < (unsigned)k;
+  for (long long t = gw; t < T; t += nw) {
+    int mine = 0;
+    if (rule == MOE_SELECT_UNIFORM) {
+      mine = (int)((t * k + lane) % E);
+    } else {
+      const uint32_t base = fmix32((uint32_t)__ldg(token_id + t) ^ seed);
+      for (int j = 0; j < k; ++j) {                 // same trip count on every lane
+        const int n = E - k + j;
+        const int r = (int)(fmix32(base + (uint32_t)j) % (uint32_t)(n + 1));
+        const bool dup = __any_sync(0xffffffffu, lane < (unsigned)j && mine == r);
+        if (lane == (unsigned)j) mine = dup ? n : r;
+      }
+    }
+    const float* row = logits + t * E;
+    const float l = act ? __ldg(row + mine) : 0.f;
+    float g;
+    if (score == MOE_SCORE_SOFTMAX) {
+      if (renorm) {                                 // fp64 difference and exponential, as topk_kernel
+        const float m = warp_max(act ? l : -INFINITY);
+        const double ex = act ? exp((double)l - (double)m) : 0.0;
+        g = (float)(ex / warp_sum_d(ex));
+      } else {
+        float mf = -INFINITY;
+        for (int e = lane; e < E; e += 32) mf = fmaxf(mf, __ldg(row + e));
+        const float M = warp_max(mf);
+        float zs = 0.f;
+        for (int e = lane; e < E; e += 32) zs += expf(__ldg(row + e) - M);
+        g = expf(l - M) / warp_sum(zs);
+      }
+    } else {
+      const float sc = act ? score_f(l, score) : 0.f;
+      g = renorm ? sc / warp_sum(sc) : sc;
+    }
+    if (act) {
+      topk_idx[t * k + lane] = mine;
+      topk_gate[t * k + lane] = g * scale;
+    }
+  }
+}
+
+// H = l + n * softplus(l_noise) in fp32 (softplus written max(z, 0) + log1p(exp(-|z|))),
+// one rounding for the product and sum.  Grid-stride over the T x E elements.
+__global__ void __launch_bounds__(256)
+noisy_logits_kernel(const float* __restrict__ logits, const float* __restrict__ logits_noise,
+                    const float* __restrict__ noise, long long n, float* __restrict__ H) {
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (long long)gridDim.x * blockDim.x) {
+    const float z = __ldg(logits_noise + i);
+    const float sp = fmaxf(z, 0.f) + log1pf(expf(-fabsf(z)));
+    H[i] = fmaf(__ldg(noise + i), sp, __ldg(logits + i));
+  }
+}
+
 }  // namespace
 
 // The tensor-core router takes bf16 x with d >= 64 and E a multiple of 4 (16-byte logit
 // rows); anything else runs the fp32 SIMT router.
 static bool tc_router_ok(int x_dtype, int d, int E) { return x_dtype == MOE_BF16 && d >= 64 && E % 4 == 0; }
 static size_t tc_router_w3_bytes(int d, int E) { return (size_t)((E + 63) / 64) * 256 * d * 2; }
+
+// Split W_g into three bf16 terms, then one tcgen05 GEMM writes logits (+ offset).
+// Workspace: 256 bytes (the one-group offsets {0, T}) + the split weight.
+static moe_status tc_logits(const void* x, const float* Wg, const float* logit_offset, int T, int d, int E,
+                            float* logits, void* ws, cudaStream_t s) {
+  int32_t* offs2 = static_cast<int32_t*>(ws);
+  __nv_bfloat16* W3 = reinterpret_cast<__nv_bfloat16*>(static_cast<char*>(ws) + 256);
+  moe_status st = cuda_status(cudaMemsetAsync(W3, 0, tc_router_w3_bytes(d, E), s));
+  if (st != MOE_OK) return st;
+  dim3 g((d + 31) / 32, (E + 31) / 32);
+  split_router_weight_kernel<<<g, 256, 0, s>>>(Wg, d, E, W3, offs2, T);
+  st = check_launch();
+  if (st != MOE_OK) return st;
+  return launch_router_logits_tc(x, offs2, T, d, E, W3, logit_offset, logits, s);
+}
 
 size_t route_workspace_bytes(int T, int d, int E) {
   if (T <= 0 || E <= 0 || d <= 0) return 0;
@@ -531,16 +638,7 @@ moe_status launch_route(const void* x, int x_dtype, const float* Wg, const float
   const long long split_stride = (long long)T * E;
   moe_status st = MOE_ERR_UNSUPPORTED;
   if (tc_router_ok(x_dtype, d, E)) {
-    // split W_g into three bf16 terms, then one tcgen05 GEMM writes logits (+ offset)
-    int32_t* offs2 = static_cast<int32_t*>(ws);
-    __nv_bfloat16* W3 = reinterpret_cast<__nv_bfloat16*>(static_cast<char*>(ws) + 256);
-    st = cuda_status(cudaMemsetAsync(W3, 0, tc_router_w3_bytes(d, E), s));
-    if (st != MOE_OK) return st;
-    dim3 g((d + 31) / 32, (E + 31) / 32);
-    split_router_weight_kernel<<<g, 256, 0, s>>>(Wg, d, E, W3, offs2, T);
-    st = check_launch();
-    if (st != MOE_OK) return st;
-    st = launch_router_logits_tc(x, offs2, T, d, E, W3, logit_offset, logits, s);
+    st = tc_logits(x, Wg, logit_offset, T, d, E, logits, ws, s);
     if (st != MOE_OK && st != MOE_ERR_UNSUPPORTED) return st;
     if (st == MOE_OK) p.nsplit = 1;
   }
@@ -556,6 +654,64 @@ moe_status launch_route(const void* x, int x_dtype, const float* Wg, const float
   const bool bias = select_bias != nullptr;
 #define MOE_TOPK(N) return run_topk<N>(bias, partial, p.nsplit, split_stride, logit_offset, select_bias, T, E, k, \
                                        score, renormalize, scale, logits, write, topk_idx, topk_gate, s)
+  if (epl <= 1) MOE_TOPK(1);
+  if (epl <= 2) MOE_TOPK(2);
+  if (epl <= 4) MOE_TOPK(4);
+  if (epl <= 8) MOE_TOPK(8);
+  if (epl <= 16) MOE_TOPK(16);
+  MOE_TOPK(32);
+#undef MOE_TOPK
+}
+
+size_t router_logits_workspace_bytes(int T, int d, int E) {
+  if (T <= 0 || E <= 0 || d <= 0) return 0;
+  return (E % 4 == 0 && d >= 64) ? 256 + tc_router_w3_bytes(d, E) : 0;
+}
+
+// The router alone: the tensor-core GEMM where it applies, else the SIMT GEMM in one
+// pass over d (no split, so it writes the logits with their offset itself).
+moe_status launch_router_logits(const void* x, int x_dtype, const float* Wg, const float* logit_offset, int T,
+                                int d, int E, float* logits, void* ws, cudaStream_t s) {
+  if (T == 0) return MOE_OK;
+  if (tc_router_ok(x_dtype, d, E)) {
+    const moe_status st = tc_logits(x, Wg, logit_offset, T, d, E, logits, ws, s);
+    if (st != MOE_ERR_UNSUPPORTED) return st;
+  }
+  LogitsPlan p = plan_logits(T, d, E);
+  p.nsplit = 1;
+  p.chunks_per_split = (d + kKC - 1) / kKC;
+  const long long stride = (long long)T * E;
+  return x_dtype == MOE_F32 ? dispatch_logits<float>(x, Wg, logit_offset, T, d, E, p, logits, stride, s)
+                            : dispatch_logits<__nv_bfloat16>(x, Wg, logit_offset, T, d, E, p, logits, stride, s);
+}
+
+moe_status launch_route_fixed(const float* logits, int T, int E, int k, int score, int renormalize, float scale,
+                              int rule, const int32_t* token_id, uint32_t seed, int32_t* topk_idx,
+                              float* topk_gate, cudaStream_t s) {
+  if (T == 0) return MOE_OK;
+  long long blocks = ((long long)T + 7) / 8;                 // 8 warps (tokens) per block
+  const long long cap = (long long)num_sms() * 8;
+  if (blocks > cap) blocks = cap;
+  fixed_select_kernel<<<(unsigned)blocks, 256, 0, s>>>(logits, T, E, k, score, renormalize, scale, rule, token_id,
+                                                       seed, topk_idx, topk_gate);
+  return check_launch();
+}
+
+moe_status launch_route_noisy(const float* logits, const float* logits_noise, const float* noise, int T, int E,
+                              int k, float scale, float* H, int32_t* topk_idx, float* topk_gate, cudaStream_t s) {
+  if (T == 0) return MOE_OK;
+  const long long n = (long long)T * E;
+  long long blocks = (n + 255) / 256;
+  const long long cap = (long long)num_sms() * 16;
+  if (blocks > cap) blocks = cap;
+  noisy_logits_kernel<<<(unsigned)blocks, 256, 0, s>>>(logits, logits_noise, noise, n, H);
+  moe_status st = check_launch();
+  if (st != MOE_OK) return st;
+  // KeepTopK on H, then the softmax over the kept H (the learned softmax router's path
+  // with H in place of the logits; no offset, no selection bias)
+  const int epl = (E + 31) / 32;
+#define MOE_TOPK(N) return run_topk<N>(false, H, 1, n, nullptr, nullptr, T, E, k, MOE_SCORE_SOFTMAX, 1, scale, \
+                                       H, 0, topk_idx, topk_gate, s)
   if (epl <= 1) MOE_TOPK(1);
   if (epl <= 2) MOE_TOPK(2);
   if (epl <= 4) MOE_TOPK(4);

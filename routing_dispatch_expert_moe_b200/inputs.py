@@ -84,6 +84,7 @@ CONFIGS = {
 
 # stream ids
 _S_X, _S_WG, _S_OFF, _S_BIAS, _S_SHARED = 1, 2, 3, 4, 5
+_S_WNOISE, _S_NOISE, _S_TOKEN_ID = 6, 7, 8
 _S_EXPERT_BASE = 1000
 
 
@@ -128,6 +129,31 @@ def gen_router(cfg: MoEConfig, seed: int = 0):
     elif cfg.select_bias is not None:
         raise ValueError(cfg.select_bias)
     return Wg, off, bias
+
+
+def gen_noise_router(cfg: MoEConfig, seed: int = 0) -> np.ndarray:
+    """Noise-router weight W_noise [d, E] fp32 on the router's grid (exact fp32 logits)."""
+    z = _rng(seed, _S_WNOISE).standard_normal((cfg.d, cfg.E), dtype=np.float32) * 0.02
+    if cfg.act == "f32":
+        return np.clip(np.rint(z * 256.0), -32, 32).astype(np.float32) / 256.0
+    return np.clip(np.rint(z * 1024.0), -64, 64).astype(np.float32) / 1024.0
+
+
+def gen_noise(cfg: MoEConfig, seed: int = 0, T: Optional[int] = None) -> np.ndarray:
+    """Standard normal draws [T, E] fp32 for noisy top-k gating."""
+    T = cfg.T if T is None else T
+    return _rng(seed, _S_NOISE).standard_normal((T, cfg.E), dtype=np.float32)
+
+
+def gen_token_ids(cfg: MoEConfig, seed: int = 0, T: Optional[int] = None, vocab: int = 32768,
+                  s: float = 1.0) -> np.ndarray:
+    """Token ids [T] int32 with text-like (Zipf) frequencies: rank r of the vocabulary drawn with
+    probability proportional to r^-s, ranks mapped to ids by a seeded permutation."""
+    T = cfg.T if T is None else T
+    rng = _rng(seed, _S_TOKEN_ID)
+    p = np.arange(1, vocab + 1, dtype=np.float64) ** -s
+    ranks = rng.choice(vocab, size=T, p=p / p.sum())
+    return rng.permutation(vocab)[ranks].astype(np.int32)
 
 
 def _weights(cfg: MoEConfig, rng: np.random.Generator, shape) -> np.ndarray:
@@ -201,4 +227,4 @@ def fits_exact_fp32(cfg: MoEConfig) -> bool:
 
 
 __all__ = ["MoEConfig", "CONFIGS", "SCORES", "gen_x", "gen_router", "gen_expert", "gen_experts",
-           "gen_shared", "small_config", "fits_exact_fp32"]
+           "gen_shared", "gen_noise_router", "gen_noise", "gen_token_ids", "small_config", "fits_exact_fp32"]

@@ -4,6 +4,8 @@ MoELayer owns preallocated device buffers for a maximum token count and runs, on
 stream with no host synchronisation:
 
     moe_route -> moe_histogram_scan
+      (routing="uniform" / "hash": moe_router_logits -> moe_route_fixed;
+       routing="noisy": moe_router_logits for W_g and W_noise -> moe_route_noisy)
       dispatch="permute": -> moe_permute -> moe_expert_gate_up
       dispatch="gather":  -> moe_expert_gate_up_gather (reads x through the row map)
       combine="rows":  -> moe_expert_down (gate fused) [-> shared expert: gate_up/down
@@ -36,13 +38,15 @@ class MoEWeights:
     select_bias: Optional[torch.Tensor] = None    # [E] f32
     W_gu_s: Optional[torch.Tensor] = None     # [1, 2F_s, d] shared expert
     W_dn_s: Optional[torch.Tensor] = None     # [1, d, F_s]
+    W_noise: Optional[torch.Tensor] = None    # [d, E] f32: noise router (routing="noisy")
 
 
 class MoELayer:
     def __init__(self, weights: MoEWeights, k: int, T_max: int, score: str = "softmax",
                  renormalize: bool = True, scale: float = 1.0, capacity: int = -1,
                  rows_dtype: torch.dtype = torch.float32, out_dtype: torch.dtype = torch.float32,
-                 combine: str = "rows", dispatch: str = "permute", overlap: bool = True):
+                 combine: str = "rows", dispatch: str = "permute", overlap: bool = True,
+                 routing: str = "learned", hash_seed: int = 0):
         """rows_dtype: gated expert rows (and the shared expert's output); out_dtype: y.
         fp32 (the default) leaves H as the only bf16 rounding inside the layer.
         combine: "rows" (gated rows + ordered combine) or "fused" (down GEMM adds into an
@@ -51,7 +55,19 @@ class MoELayer:
         token rows through token_of_row; same H bit for bit).
         overlap: run the work nothing on the main path waits for (router statistics, and
         clearing y for the fused combine) on a second stream forked from and joined back
-        to the caller's stream (one CUDA graph with two branches when captured)."""
+        to the caller's stream (one CUDA graph with two branches when captured).
+        routing: "learned" (top-k of the router), "uniform" (forced-uniform selection),
+        "hash" (experts from a hash of the token ids given to forward, seeded by
+        hash_seed) or "noisy" (noisy top-k with weights.W_noise and the standard normal
+        draws given to forward; softmax gating).  The fixed rules keep the learned gates
+        over the chosen experts; the router statistics always use the router logits."""
+        if routing not in ("learned", "uniform", "hash", "noisy"):
+            raise ValueError(f"routing must be learned, uniform, hash or noisy, got {routing!r}")
+        if routing != "learned" and weights.select_bias is not None:
+            raise ValueError("a selection bias only applies to the learned top-k")
+        if routing == "noisy" and (weights.W_noise is None or score != "softmax"):
+            raise ValueError("noisy top-k needs weights.W_noise and softmax scoring")
+        self.routing, self.hash_seed = routing, hash_seed
         if dispatch not in ("permute", "gather"):
             raise ValueError(f"dispatch must be 'permute' or 'gather', got {dispatch!r}")
         self.dispatch_mode = dispatch
@@ -93,6 +109,9 @@ class MoELayer:
             # a bf16 y: a separate fp32 buffer, zero at rest (the final rounding clears it)
             self.y32 = self.y if out_dtype == torch.float32 else torch.zeros((T_max, d), dtype=f32, device=dev)
         self._y32_at_rest_zero = combine == "fused" and self.y32 is not self.y
+        if routing == "noisy":
+            self.logits_noise = torch.empty((T_max, E), dtype=f32, device=dev)
+            self.H = torch.empty((T_max, E), dtype=f32, device=dev)
         self.load = torch.empty(E, dtype=f32, device=dev)
         self.stats5 = torch.empty(5, dtype=f32, device=dev)
         self.ws = torch.empty(max(M.moe_workspace_bytes(T_max, d, E, k), 16), dtype=torch.uint8, device=dev)
@@ -108,10 +127,25 @@ class MoELayer:
             self.y_s = torch.empty((T_max, d), dtype=rows_dtype, device=dev) if combine == "rows" else None
 
     # individual steps (so that a caller can time them one by one)
-    def route(self, x, stream=None):
-        M.moe_route(x, self.w.Wg, self.k, self.score, self.renormalize, self.scale, self.w.logit_offset,
-                    self.w.select_bias, self.logits[:x.shape[0]], self.topk_idx[:x.shape[0]],
-                    self.topk_gate[:x.shape[0]], self.ws, stream)
+    def route(self, x, stream=None, token_id=None, noise=None):
+        T = x.shape[0]
+        if self.routing == "learned":
+            M.moe_route(x, self.w.Wg, self.k, self.score, self.renormalize, self.scale, self.w.logit_offset,
+                        self.w.select_bias, self.logits[:T], self.topk_idx[:T], self.topk_gate[:T], self.ws, stream)
+            return
+        M.moe_router_logits(x, self.w.Wg, self.w.logit_offset, self.logits[:T], self.ws, stream)
+        if self.routing == "noisy":
+            if noise is None:
+                raise ValueError("noisy routing needs the standard normal draws (noise=[T, E] f32)")
+            M.moe_router_logits(x, self.w.W_noise, None, self.logits_noise[:T], self.ws, stream)
+            M.moe_route_noisy(self.logits[:T], self.logits_noise[:T], noise, self.k, self.scale, self.H[:T],
+                              self.topk_idx[:T], self.topk_gate[:T], stream)
+            return
+        if self.routing == "hash" and token_id is None:
+            raise ValueError("hash routing needs token_id ([T] int32)")
+        M.moe_route_fixed(self.logits[:T], self.k, self.routing, self.score, self.renormalize, self.scale,
+                          token_id if self.routing == "hash" else None, self.hash_seed, self.topk_idx[:T],
+                          self.topk_gate[:T], stream)
 
     def histogram_scan(self, T, stream=None):
         M.moe_histogram_scan(self.topk_idx[:T], self.topk_gate[:T], self.E, self.capacity, self.counts, self.kept,
@@ -158,10 +192,10 @@ class MoELayer:
         M.moe_router_stats(self.logits[:T], self.counts, self.kept, self.k, self.score, self.load, self.stats5,
                            self.ws, stream)
 
-    def stages(self, x: torch.Tensor, with_stats: bool = True):
+    def stages(self, x: torch.Tensor, with_stats: bool = True, token_id=None, noise=None):
         """The forward as (name, fn(stream)) steps in launch order."""
         T = x.shape[0]
-        st = [("route", lambda s: self.route(x, s)),
+        st = [("route", lambda s: self.route(x, s, token_id, noise)),
               ("histogram_scan", lambda s: self.histogram_scan(T, s))]
         if self.dispatch_mode == "permute":
             st += [("permute", lambda s: self.permute(x, s)), ("gate_up", lambda s: self.gate_up(s))]
@@ -182,9 +216,12 @@ class MoELayer:
             st.append(("stats", lambda s: self.stats(T, s)))
         return st
 
-    def forward(self, x: torch.Tensor, stream=None, with_stats: bool = True, marks=None) -> torch.Tensor:
+    def forward(self, x: torch.Tensor, stream=None, with_stats: bool = True, marks=None, token_id=None,
+                noise=None) -> torch.Tensor:
         """marks: optional {stage name: (event, event)} recorded on the main stream right
-        before and after that stage (for timing one kernel inside the real schedule)."""
+        before and after that stage (for timing one kernel inside the real schedule).
+        token_id ([T] int32, routing="hash") and noise ([T, E] f32, routing="noisy") are
+        that batch's inputs of the routing rule."""
         T = x.shape[0]
         if T > self.T_max:
             raise ValueError(f"T={T} exceeds T_max={self.T_max}")
@@ -201,7 +238,7 @@ class MoELayer:
                 m[1].record(s)
 
         if not self.overlap:
-            for name, fn in self.stages(x, with_stats):
+            for name, fn in self.stages(x, with_stats, token_id, noise):
                 run(name, fn)
             return self.y[:T]
         side = self._side
@@ -210,7 +247,7 @@ class MoELayer:
         side.wait_event(self._ev_fork)
         if fused and not self.has_shared and not self._y32_at_rest_zero:
             M.moe_zero(self.y32[:T], side)       # the fused combine's starting value, off the main path
-        run("route", lambda s_: self.route(x, s_))
+        run("route", lambda s_: self.route(x, s_, token_id, noise))
         run("histogram_scan", lambda s_: self.histogram_scan(T, s_))
         if with_stats:
             self._ev_routed.record(s)
@@ -239,22 +276,23 @@ class MoELayer:
         return self.y[:T]
 
     # ---------------------------------------------------------------- CUDA graph
-    def capture(self, x_static: torch.Tensor, with_stats: bool = True) -> None:
+    def capture(self, x_static: torch.Tensor, with_stats: bool = True, token_id=None, noise=None) -> None:
         """Records one forward over the fixed input buffer x_static into a CUDA graph.
 
         Replaying it (replay()) runs the same library kernels with no host work per
-        step.  Write the next batch into x_static before each replay.  One eager forward
-        runs first so that every per-device lookup happens outside the capture.
+        step.  Write the next batch into x_static (and token_id / noise, when the routing
+        rule reads them) before each replay.  One eager forward runs first so that every
+        per-device lookup happens outside the capture.
         """
         self.x_static = x_static
-        self.forward(x_static, with_stats=with_stats)
+        self.forward(x_static, with_stats=with_stats, token_id=token_id, noise=noise)
         torch.cuda.synchronize()
         s = torch.cuda.Stream()
         s.wait_stream(torch.cuda.current_stream())
         self.graph = torch.cuda.CUDAGraph()
         with torch.cuda.stream(s):
             with torch.cuda.graph(self.graph, stream=s):
-                self.forward(x_static, stream=s, with_stats=with_stats)
+                self.forward(x_static, stream=s, with_stats=with_stats, token_id=token_id, noise=noise)
         torch.cuda.current_stream().wait_stream(s)
         torch.cuda.synchronize()
 
@@ -263,8 +301,15 @@ class MoELayer:
         return self.y[:self.x_static.shape[0]]
 
     # library kernels launched by one forward (the scan's workspace memset is not a kernel)
+    def _router_gemm_launches(self) -> int:
+        # tensor-core router: the weight split and the GEMM; else one SIMT GEMM
+        tc = self.dtype == torch.bfloat16 and self.d >= 64 and self.E % 4 == 0
+        return 2 if tc else 1
+
     def launches_per_forward(self, with_stats: bool = True) -> int:
-        n = 2 + 2 + 1 + 1 + 1 + 1          # route(2) scan(2) permute gate_up down combine
+        r = self._router_gemm_launches()
+        route = {"learned": r + 1, "uniform": r + 1, "hash": r + 1, "noisy": 2 * r + 2}[self.routing]
+        n = route + 2 + 1 + 1 + 1 + 1      # route, scan(2) permute gate_up down combine
         if self.combine_mode == "fused":
             n -= 1                         # down_combine (its zero fill is a memset, not a kernel)
             if self.y32 is not self.y:

@@ -19,6 +19,7 @@ LIB_PATH = os.environ.get("MOE_B200_LIB", os.path.join(_HERE, "libmoe_b200.so"))
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_DEVICE = range(6)
 SCORE = {"softmax": 0, "sigmoid": 1, "sqrt_softplus": 2}
+SELECT = {"uniform": 0, "hash": 1}
 DTYPE = {torch.bfloat16: 0, torch.float32: 1}
 DEVERR = {0: "none", 1: "expert id out of range", 2: "duplicate expert in a token", 3: "row index out of range",
           4: "scan look-back timeout", 5: "GEMM pipeline timeout"}
@@ -36,6 +37,13 @@ _SIGNATURES = {
     "moe_route_workspace_bytes": (_size, [_i32, _i32, _i32]),
     "moe_route": (_i32, [_c_void_p, _i32, _c_void_p, _c_void_p, _c_void_p, _i32, _i32, _i32, _i32, _i32, _i32,
                          _f32, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _size, _c_void_p]),
+    "moe_router_logits_workspace_bytes": (_size, [_i32, _i32, _i32]),
+    "moe_router_logits": (_i32, [_c_void_p, _i32, _c_void_p, _c_void_p, _i32, _i32, _i32, _c_void_p, _c_void_p,
+                                 _size, _c_void_p]),
+    "moe_route_fixed": (_i32, [_c_void_p, _i32, _i32, _i32, _i32, _i32, _f32, _i32, _c_void_p, ctypes.c_uint32,
+                               _c_void_p, _c_void_p, _c_void_p]),
+    "moe_route_noisy": (_i32, [_c_void_p, _c_void_p, _c_void_p, _i32, _i32, _i32, _f32, _c_void_p, _c_void_p,
+                               _c_void_p, _c_void_p]),
     "moe_histogram_scan_workspace_bytes": (_size, [_i32, _i32, _i32]),
     "moe_histogram_scan": (_i32, [_c_void_p, _c_void_p, _i32, _i32, _i32, _i32, _c_void_p, _c_void_p, _c_void_p,
                                   _c_void_p, _c_void_p, _c_void_p, _c_void_p, _size, _c_void_p]),
@@ -175,6 +183,65 @@ def moe_route(x, Wg, k: int, score: str = "softmax", renormalize: bool = True, s
                                         SCORE[score], 1 if renormalize else 0, float(scale), _p(logits),
                                         _p(topk_idx), _p(topk_gate), _p(ws), nb, _stream(stream)))
     return logits, topk_idx, topk_gate
+
+
+def moe_router_logits(x, Wg, logit_offset=None, logits=None, workspace=None, stream=None):
+    """The router alone: logits [T,E] f32 = x . Wg (+ logit_offset)."""
+    T, d = x.shape
+    E = Wg.shape[1]
+    _need(x, "x")
+    _need(Wg, "Wg", torch.float32, (d, E))
+    if logit_offset is not None:
+        _need(logit_offset, "logit_offset", torch.float32, (E,))
+    dev = x.device
+    logits = torch.empty((T, E), dtype=torch.float32, device=dev) if logits is None else \
+        _need(logits, "logits", torch.float32, (T, E))
+    nb = int(lib().moe_router_logits_workspace_bytes(T, d, E))
+    ws = _ws(nb, dev, workspace)
+    _check("moe_router_logits", lib().moe_router_logits(_p(x), _dt(x), _p(Wg), _p(logit_offset), T, d, E,
+                                                        _p(logits), _p(ws), nb, _stream(stream)))
+    return logits
+
+
+def moe_route_fixed(logits, k: int, rule: str = "uniform", score: str = "softmax", renormalize: bool = True,
+                    scale: float = 1.0, token_id=None, seed: int = 0, topk_idx=None, topk_gate=None, stream=None):
+    """Forced-uniform or hash selection with the learned gates.  Returns (topk_idx, topk_gate)."""
+    T, E = logits.shape
+    _need(logits, "logits", torch.float32)
+    if rule not in SELECT:
+        raise ValueError(f"rule must be one of {sorted(SELECT)}")
+    if token_id is not None:
+        _need(token_id, "token_id", torch.int32, (T,))
+    elif rule == "hash":
+        raise ValueError("hash selection needs token_id")
+    dev = logits.device
+    topk_idx = torch.empty((T, k), dtype=torch.int32, device=dev) if topk_idx is None else \
+        _need(topk_idx, "topk_idx", torch.int32, (T, k))
+    topk_gate = torch.empty((T, k), dtype=torch.float32, device=dev) if topk_gate is None else \
+        _need(topk_gate, "topk_gate", torch.float32, (T, k))
+    _check("moe_route_fixed", lib().moe_route_fixed(_p(logits), T, E, k, SCORE[score], 1 if renormalize else 0,
+                                                    float(scale), SELECT[rule], _p(token_id),
+                                                    int(seed) & 0xFFFFFFFF, _p(topk_idx), _p(topk_gate),
+                                                    _stream(stream)))
+    return topk_idx, topk_gate
+
+
+def moe_route_noisy(logits, logits_noise, noise, k: int, scale: float = 1.0, H=None, topk_idx=None,
+                    topk_gate=None, stream=None):
+    """Noisy top-k gating.  Returns (H [T,E] f32, topk_idx [T,k] i32, topk_gate [T,k] f32)."""
+    T, E = logits.shape
+    _need(logits, "logits", torch.float32)
+    _need(logits_noise, "logits_noise", torch.float32, (T, E))
+    _need(noise, "noise", torch.float32, (T, E))
+    dev = logits.device
+    H = torch.empty((T, E), dtype=torch.float32, device=dev) if H is None else _need(H, "H", torch.float32, (T, E))
+    topk_idx = torch.empty((T, k), dtype=torch.int32, device=dev) if topk_idx is None else \
+        _need(topk_idx, "topk_idx", torch.int32, (T, k))
+    topk_gate = torch.empty((T, k), dtype=torch.float32, device=dev) if topk_gate is None else \
+        _need(topk_gate, "topk_gate", torch.float32, (T, k))
+    _check("moe_route_noisy", lib().moe_route_noisy(_p(logits), _p(logits_noise), _p(noise), T, E, k, float(scale),
+                                                    _p(H), _p(topk_idx), _p(topk_gate), _stream(stream)))
+    return H, topk_idx, topk_gate
 
 
 def moe_histogram_scan(topk_idx, topk_gate, E: int, capacity: int = -1, counts=None, kept=None, offsets=None,

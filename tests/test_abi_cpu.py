@@ -100,6 +100,54 @@ def test_route_empty_batch_is_ok_without_launch(L):
     assert _route(L, T=0, x=NUL, logits=NUL, idx=NUL, gate=NUL) == 0
 
 
+def test_router_logits_host_validation(L):
+    f = L.moe_router_logits            # (x, dt, Wg, off, T, d, E, logits, ws, wsb, s)
+    assert f(NUL, 0, FAKE, NUL, 64, 128, 16, FAKE, FAKE, 1 << 30, NUL) == 1          # x
+    assert f(FAKE, 0, FAKE, NUL, 64, 128, 16, NUL, FAKE, 1 << 30, NUL) == 1          # logits
+    assert f(FAKE, 5, FAKE, NUL, 64, 128, 16, FAKE, FAKE, 1 << 30, NUL) == 1         # dtype
+    assert f(FAKE, 0, FAKE, NUL, -1, 128, 16, FAKE, FAKE, 1 << 30, NUL) == 1         # T < 0
+    assert f(FAKE, 0, FAKE, NUL, 64, 128, 2048, FAKE, FAKE, 1 << 30, NUL) == 2       # E > 1024
+    assert f(FAKE, 0, FAKE, NUL, 64, 100, 16, FAKE, FAKE, 1 << 30, NUL) == 2         # d % 8
+    assert f(ctypes.c_void_p(4104), 0, FAKE, NUL, 64, 128, 16, FAKE, FAKE, 1 << 30, NUL) == 2
+    need = L.moe_router_logits_workspace_bytes(64, 128, 16)
+    assert need > 0
+    assert f(FAKE, 0, FAKE, NUL, 64, 128, 16, FAKE, FAKE, need - 1, NUL) == 3
+    assert L.moe_router_logits_workspace_bytes(64, 128, 18) == 0                    # E % 4: SIMT, no workspace
+    assert f(NUL, 0, NUL, NUL, 0, 128, 16, NUL, NUL, 0, NUL) == 0                    # T = 0: nothing to do
+
+
+def test_route_fixed_host_validation(L):
+    f = L.moe_route_fixed              # (logits, T, E, k, score, renorm, scale, rule, token_id, seed, idx, gate, s)
+    ok = dict(l=FAKE, T=64, E=16, k=4, sc=0, rn=1, scale=1.0, rule=0, tid=NUL, seed=0, idx=FAKE, g=FAKE)
+
+    def call(**kw):
+        a = dict(ok)
+        a.update(kw)
+        return f(a["l"], a["T"], a["E"], a["k"], a["sc"], a["rn"], a["scale"], a["rule"], a["tid"], a["seed"],
+                 a["idx"], a["g"], NUL)
+
+    assert call(rule=2) == 1
+    assert call(rule=1) == 1                   # hash without token ids
+    assert call(k=17) == 1                     # k > E
+    assert call(sc=3) == 1
+    assert call(rn=2) == 1
+    assert call(scale=float("inf")) == 1
+    assert call(l=NUL) == 1
+    assert call(E=2000, k=4) == 2
+    assert call(k=33, E=64) == 2
+    assert call(T=0, l=NUL, idx=NUL, g=NUL) == 0
+
+
+def test_route_noisy_host_validation(L):
+    f = L.moe_route_noisy              # (logits, logits_noise, noise, T, E, k, scale, H, idx, gate, s)
+    assert f(FAKE, FAKE, NUL, 64, 16, 4, 1.0, FAKE, FAKE, FAKE, NUL) == 1             # noise
+    assert f(FAKE, FAKE, FAKE, 64, 16, 4, 1.0, NUL, FAKE, FAKE, NUL) == 1             # H
+    assert f(FAKE, FAKE, FAKE, 64, 16, 17, 1.0, FAKE, FAKE, FAKE, NUL) == 1           # k > E
+    assert f(FAKE, FAKE, FAKE, 64, 16, 4, float("nan"), FAKE, FAKE, FAKE, NUL) == 1
+    assert f(FAKE, FAKE, FAKE, 64, 2048, 4, 1.0, FAKE, FAKE, FAKE, NUL) == 2
+    assert f(NUL, NUL, NUL, 0, 16, 4, 1.0, NUL, NUL, NUL, NUL) == 0
+
+
 def test_histogram_scan_host_validation(L):
     f = L.moe_histogram_scan
     ok = dict(idx=FAKE, g=FAKE, T=64, k=4, E=16, cap=-1, c=FAKE, kp=FAKE, o=FAKE, r=FAKE, t=FAKE, gr=FAKE,
