@@ -139,7 +139,9 @@ MOE_API int64_t moe_rows_max(int32_t T, int32_t E, int32_t k, int32_t capacity);
  *   workspace    (device) >= moe_route_workspace_bytes(T, d, E) bytes (may be NULL if 0)
  * Gates: softmax + renormalize -> softmax over the k kept logits; softmax without
  * renormalize -> the full softmax probability; sigmoid / sqrt(softplus) -> kept scores
- * over their sum (renormalize) or the scores; all then times scale.
+ * over their sum (renormalize) or the scores; all then times scale.  The softmax over
+ * the kept logits takes each difference to their maximum and its exponential in fp64,
+ * then rounds the gate to fp32 (the same for moe_route_fixed and moe_route_noisy).
  * ---------------------------------------------------------------------------------- */
 MOE_API size_t moe_route_workspace_bytes(int32_t T, int32_t d, int32_t E);
 MOE_API moe_status moe_route(const void* x, int32_t x_dtype, const float* Wg,
