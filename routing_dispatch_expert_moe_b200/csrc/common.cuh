@@ -154,7 +154,8 @@ moe_status launch_gate_up_gather_simt(const void* x, int dtype, const int32_t* t
 moe_status launch_gate_up_gather_tc(const void* x, const int32_t* token_of_row, int T, const int32_t* offsets, int E,
                                     int d, int F, long long rows_max, const void* W_gu, void* h, cudaStream_t s);
 moe_status launch_router_logits_tc(const void* x, const int32_t* offs2, int T, int d, int E, const void* W3,
-                                   const float* logit_offset, float* logits, cudaStream_t s);
+                                   const float* logit_offset, float* logits, cudaStream_t s, int splits);
+int router_k_splits(int T, int d, int E);
 moe_status launch_gate_up_tc(const void* x_rows, const int32_t* offsets, int E, int d, int F,
                              long long rows_max, const void* W_gu, void* h, cudaStream_t s);
 moe_status launch_down_tc(const void* h, const int32_t* offsets, int E, int d, int F,

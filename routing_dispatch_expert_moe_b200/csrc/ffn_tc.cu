@@ -160,12 +160,33 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 __device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 // Output column tiles per row tile: 128 H features per gate/up tile (128 gate + 128 up
-// accumulator columns), 256 outputs per down tile, 64 experts per router tile.
+// accumulator columns), 256 outputs per down tile, 64 experts per router tile.  The
+// router (MODE 2, CTA-pair kernel) may also split K: F then carries the number of K
+// splits S, and its n-tile index is expert tile * S + split.
 template <int MODE>
 __host__ __device__ __forceinline__ int n_tiles_of(int F, int N_out) {
   if (MODE == 0 || MODE == 4) return (F + 127) / 128;
   if (MODE == 1 || MODE == 3) return (N_out + BN - 1) / BN;
-  return (N_out + 63) / 64;
+  return ((N_out + 63) / 64) * (F > 1 ? F : 1);
+}
+
+// The k-blocks [kb0, kb1) of one tile.  Router tiles (MODE 2) with S = F > 1 splits take
+// the split-th of S equal runs of ceil(KB / S) k-blocks; the host keeps KB >= 4 S, so no
+// run is empty.  Every other tile runs all KB k-blocks.
+struct KSplit {
+  int n_tile, split, kb0, kb1;
+};
+template <int MODE>
+__device__ __forceinline__ KSplit k_split(int n_tile, int F, int KB) {
+  KSplit k{n_tile, 0, 0, KB};
+  if (MODE == 2 && F > 1) {
+    const int per = (KB + F - 1) / F;
+    k.n_tile = n_tile / F;
+    k.split = n_tile - k.n_tile * F;
+    k.kb0 = k.split * per;
+    k.kb1 = min(KB, k.kb0 + per);
+  }
+  return k;
 }
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -781,12 +802,13 @@ grouped_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
       bool ok = true;
       for (int tile = cid; ok && tile < total; tile += ncl) {
         const TileCoord tc = tile_coord(tile_start, offsets, E, PM, tile, MODE == 2 ? n_tiles : 0);
+        const KSplit ks = k_split<MODE>(tc.n_tile, F, KB);
         const int a_row = tc.row0 + (int)rank * BM;
         int b_row;
         if (MODE == 0) b_row = tc.e * 2 * F + (rank ? F : 0) + tc.n_tile * 128;   // even: gate, odd: up
         else if (MODE == 1 || MODE == 3) b_row = tc.e * N_out + tc.n_tile * BN + (int)rank * BM;
-        else b_row = tc.n_tile * BN + (int)rank * (kRouterN / 2);   // router: half of hi, mid, lo
-        for (int kb = 0; kb < KB; ++kb) {
+        else b_row = ks.n_tile * BN + (int)rank * (kRouterN / 2);   // router: half of hi, mid, lo
+        for (int kb = ks.kb0; kb < ks.kb1; ++kb) {
           if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1u, abort_flag, err)) { ok = false; break; }
           if (rank == 0) mbar_expect_tx(bar_full + 8 * stage, 2 * (A_STAGE + (mma_n<MODE>() / 2) * BK * 2));
           const uint32_t full_c = map_to_rank(bar_full + 8 * stage, 0);
@@ -814,7 +836,10 @@ grouped_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
         if (!mbar_wait(bar_tempty + 8 * acc, acc_phase ^ 1u, abort_flag, err)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-        for (int kb = 0; kb < KB; ++kb) {
+        int n_tile_of_tile = 0;
+        if (MODE == 2) n_tile_of_tile = tile_coord(tile_start, offsets, E, PM, tile, n_tiles).n_tile;
+        const KSplit ks = k_split<MODE>(n_tile_of_tile, F, KB);
+        for (int kb = ks.kb0; kb < ks.kb1; ++kb) {
           if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag, err)) { ok = false; break; }
           tc_fence_after();
           const uint64_t adesc = sw128_desc(sb + C::a + stage * A_STAGE);
@@ -822,7 +847,7 @@ grouped_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
 #pragma unroll
           for (int kk = 0; kk < BK / UMMA_K; ++kk)
             umma_bf16_pair(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, make_idesc(2 * BM, mma_n<MODE>()),
-                           (kb | kk) != 0 ? 1u : 0u);
+                           (kb != ks.kb0 || kk != 0) ? 1u : 0u);
           umma_commit_pair_both(bar_empty + 8 * stage);
           if (++stage == C::stages) { stage = 0; phase ^= 1u; }
         }
@@ -852,8 +877,11 @@ grouped_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
       const int cta_rows = min(BM, max(0, tc.rows - (int)rank * BM));
       const long long wrow0 = (long long)tc.row0 + (int)rank * BM + q * 32;
       const int wrows = min(32, max(0, cta_rows - q * 32));
-      epilogue_tile<MODE, OutT>(taddr, stage, lane, wrow0, wrows, tc.n_tile, F, N_out, gate_of_row, out,
-                                token_of_row, n_tokens, err, c_begin, c_end);
+      const KSplit ks = k_split<MODE>(tc.n_tile, F, KB);
+      // a K split of the router writes its partial logits to plane `split` of [S, rows, E]
+      OutT* o = MODE == 2 ? out + (long long)ks.split * rows_max * N_out : out;
+      epilogue_tile<MODE, OutT>(taddr, stage, lane, wrow0, wrows, MODE == 2 ? ks.n_tile : tc.n_tile, F, N_out,
+                                gate_of_row, o, token_of_row, n_tokens, err, c_begin, c_end);
       tc_fence_before();
       mbar_arrive_cluster(map_to_rank(bar_tempty + 8 * acc, 0));
     }
@@ -972,17 +1000,32 @@ moe_status launch_tc2(const CUtensorMap& ma, const CUtensorMap& mb, const int32_
                                         err_ptr()));
 }
 
+// K splits for the router GEMM: when its pair tiles would leave CTA pairs idle, split K
+// into S equal runs (S a power of two, at most 8, each run at least 4 k-blocks) so that
+// up to one tile per pair is in flight.  The partial logits then go to S planes and the
+// top-k kernel adds them in plane order (and the offset).  1 for the single-CTA kernel.
+int router_k_splits(int T, int d, int E) {
+  if (T <= 0 || E <= 0 || d < BK || !use_pairs(T, 1)) return 1;
+  const long long tiles = (long long)((T + 2 * BM - 1) / (2 * BM)) * ((E + 63) / 64);
+  const int KB = (d + BK - 1) / BK;
+  const int pairs = num_sms() / 2;
+  int S = 1;
+  while (S < 8 && tiles * 2 * S <= pairs && KB >= 4 * 2 * S) S *= 2;
+  return S;
+}
+
 moe_status launch_router_logits_tc(const void* x, const int32_t* offs2, int T, int d, int E, const void* W3,
-                                   const float* logit_offset, float* logits, cudaStream_t s) {
+                                   const float* logit_offset, float* logits, cudaStream_t s, int splits) {
   if (T == 0) return MOE_OK;
   if (d < BK || d % 8 != 0 || E % 4 != 0) return MOE_ERR_UNSUPPORTED;
   const int nt = (E + 63) / 64;
   const bool pair = use_pairs(T, 1);
+  if (splits < 1 || (splits > 1 && (!pair || (d + BK - 1) / BK < 4 * splits))) return MOE_ERR_INVALID_ARG;
   CUtensorMap ma, mb;
   if (!make_map(&ma, x, (unsigned long long)T, d, BM)) return MOE_ERR_UNSUPPORTED;
   // boxes cover the hi, mid and lo rows of a 256-row tile (the pad rows are never loaded)
   if (!make_map(&mb, W3, (unsigned long long)nt * 256, d, pair ? kRouterN / 2 : kRouterN)) return MOE_ERR_UNSUPPORTED;
-  if (pair) return launch_tc2<2, float>(ma, mb, offs2, 1, d, E, 0, T, logit_offset, logits, s);
+  if (pair) return launch_tc2<2, float>(ma, mb, offs2, 1, d, E, splits, T, logit_offset, logits, s);
   return launch_tc<2, float>(ma, mb, offs2, 1, d, E, 0, T, logit_offset, logits, s);
 }
 

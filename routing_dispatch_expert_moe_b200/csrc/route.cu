@@ -605,26 +605,33 @@ noisy_logits_kernel(const float* __restrict__ logits, const float* __restrict__ 
 static bool tc_router_ok(int x_dtype, int d, int E) { return x_dtype == MOE_BF16 && d >= 64 && E % 4 == 0; }
 static size_t tc_router_w3_bytes(int d, int E) { return (size_t)((E + 63) / 64) * 256 * d * 2; }
 
-// Split W_g into three bf16 terms, then one tcgen05 GEMM writes logits (+ offset).
-// Workspace: 256 bytes (the one-group offsets {0, T}) + the split weight.
+// Split W_g into three bf16 terms, then one tcgen05 GEMM writes logits (+ offset), or,
+// with splits > 1, the partial logits of each K run to planes [splits, T, E] (no offset).
+// Workspace: 256 bytes (the one-group offsets {0, T}) + the split weight (+ the planes,
+// placed by the caller).  The split weight's rows for experts past E and its pad rows are
+// left unwritten: they only reach accumulator columns that are never stored.
 static moe_status tc_logits(const void* x, const float* Wg, const float* logit_offset, int T, int d, int E,
-                            float* logits, void* ws, cudaStream_t s) {
+                            float* out, void* ws, cudaStream_t s, int splits) {
   int32_t* offs2 = static_cast<int32_t*>(ws);
   __nv_bfloat16* W3 = reinterpret_cast<__nv_bfloat16*>(static_cast<char*>(ws) + 256);
-  moe_status st = cuda_status(cudaMemsetAsync(W3, 0, tc_router_w3_bytes(d, E), s));
-  if (st != MOE_OK) return st;
   dim3 g((d + 31) / 32, (E + 31) / 32);
   split_router_weight_kernel<<<g, 256, 0, s>>>(Wg, d, E, W3, offs2, T);
-  st = check_launch();
+  moe_status st = check_launch();
   if (st != MOE_OK) return st;
-  return launch_router_logits_tc(x, offs2, T, d, E, W3, logit_offset, logits, s);
+  return launch_router_logits_tc(x, offs2, T, d, E, W3, splits > 1 ? nullptr : logit_offset, out, s, splits);
+}
+
+// The K-split planes of the tensor-core router sit after the split weight.
+static size_t tc_router_planes_bytes(int T, int d, int E) {
+  const int S = router_k_splits(T, d, E);
+  return S > 1 ? (size_t)S * T * E * sizeof(float) : 0;
 }
 
 size_t route_workspace_bytes(int T, int d, int E) {
   if (T <= 0 || E <= 0 || d <= 0) return 0;
   LogitsPlan p = plan_logits(T, d, E);
   const size_t simt = p.nsplit > 1 ? (size_t)p.nsplit * T * E * sizeof(float) : 0;
-  const size_t tc = (E % 4 == 0 && d >= 64) ? 256 + tc_router_w3_bytes(d, E) : 0;
+  const size_t tc = (E % 4 == 0 && d >= 64) ? 256 + tc_router_w3_bytes(d, E) + tc_router_planes_bytes(T, d, E) : 0;
   return simt > tc ? simt : tc;
 }
 
@@ -638,9 +645,15 @@ moe_status launch_route(const void* x, int x_dtype, const float* Wg, const float
   const long long split_stride = (long long)T * E;
   moe_status st = MOE_ERR_UNSUPPORTED;
   if (tc_router_ok(x_dtype, d, E)) {
-    st = tc_logits(x, Wg, logit_offset, T, d, E, logits, ws, s);
+    // K splits when the GEMM has too few tiles; the top-k adds the planes in order
+    const int S = router_k_splits(T, d, E);
+    float* planes = reinterpret_cast<float*>(static_cast<char*>(ws) + 256 + tc_router_w3_bytes(d, E));
+    st = tc_logits(x, Wg, logit_offset, T, d, E, S > 1 ? planes : logits, ws, s, S);
     if (st != MOE_OK && st != MOE_ERR_UNSUPPORTED) return st;
-    if (st == MOE_OK) p.nsplit = 1;
+    if (st == MOE_OK) {
+      p.nsplit = S;
+      partial = S > 1 ? planes : logits;
+    }
   }
   if (st == MOE_ERR_UNSUPPORTED) {
     partial = p.nsplit > 1 ? static_cast<float*>(ws) : logits;
@@ -674,7 +687,7 @@ moe_status launch_router_logits(const void* x, int x_dtype, const float* Wg, con
                                 int d, int E, float* logits, void* ws, cudaStream_t s) {
   if (T == 0) return MOE_OK;
   if (tc_router_ok(x_dtype, d, E)) {
-    const moe_status st = tc_logits(x, Wg, logit_offset, T, d, E, logits, ws, s);
+    const moe_status st = tc_logits(x, Wg, logit_offset, T, d, E, logits, ws, s, 1);
     if (st != MOE_ERR_UNSUPPORTED) return st;
   }
   LogitsPlan p = plan_logits(T, d, E);
