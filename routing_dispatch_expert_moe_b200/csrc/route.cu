@@ -402,7 +402,9 @@ topk_kernel(const float* __restrict__ partial, int nsplit, long long split_strid
 // (each subtraction is exact in fp32; hi + mid + lo carries w to about 24 bits, and x is
 // bf16, so every product x * term is exact in fp32).  Layout W3 [n_tiles * 256, d] bf16,
 // K-major: n-tile j holds experts 64j..64j+63 as rows [0,64) hi, [64,128) mid,
-// [128,192) lo, [192,256) zero.  One 32 x 32 shared-memory transpose per block.
+// [128,192) lo, [192,256) padding (never written, never loaded; rows of experts past E
+// are not written either: they only feed accumulator columns that are never stored).
+// One 32 x 32 shared-memory transpose per block.
 // ---------------------------------------------------------------------------------
 __global__ void __launch_bounds__(256)
 split_router_weight_kernel(const float* __restrict__ Wg, int d, int E, __nv_bfloat16* __restrict__ W3,
