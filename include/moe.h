@@ -136,7 +136,9 @@ MOE_API int64_t moe_rows_max(int32_t T, int32_t E, int32_t k, int32_t capacity);
  *   logits       (device) [T, E] fp32 out: x . Wg + logit_offset
  *   topk_idx     (device) [T, k] int32 out
  *   topk_gate    (device) [T, k] fp32 out
- *   workspace    (device) >= moe_route_workspace_bytes(T, d, E) bytes (may be NULL if 0)
+ *   workspace    (device) >= moe_route_workspace_bytes(T, d, E) bytes (may be NULL if 0);
+ *                the query covers every call with at most T tokens (same d, E): a smaller
+ *                batch may split the router GEMM more ways
  * Gates: softmax + renormalize -> softmax over the k kept logits; softmax without
  * renormalize -> the full softmax probability; sigmoid / sqrt(softplus) -> kept scores
  * over their sum (renormalize) or the scores; all then times scale.  The softmax over
@@ -406,7 +408,8 @@ MOE_API moe_status moe_router_stats(const float* logits, const int32_t* counts, 
  * initialises an output buffer). */
 MOE_API moe_status moe_zero(void* p, size_t bytes, void* stream);
 
-/* Largest workspace any of the calls above needs for these sizes. */
+/* Largest workspace any of the calls above needs for these sizes, for every call with
+ * at most T tokens (each size query covers the batches below its T). */
 MOE_API size_t moe_workspace_bytes(int32_t T, int32_t d, int32_t E, int32_t k);
 
 /* Reads and clears the current device's error word (synchronises `stream`).

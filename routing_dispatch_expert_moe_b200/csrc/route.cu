@@ -629,12 +629,30 @@ static size_t tc_router_planes_bytes(int T, int d, int E) {
   return S > 1 ? (size_t)S * T * E * sizeof(float) : 0;
 }
 
-size_t route_workspace_bytes(int T, int d, int E) {
+// Workspace one call with exactly T tokens uses: the split weight and, when the router
+// splits K, its partial logits (tensor cores) or its split-K partials (SIMT).
+static size_t route_workspace_at(int T, int d, int E) {
   if (T <= 0 || E <= 0 || d <= 0) return 0;
   LogitsPlan p = plan_logits(T, d, E);
   const size_t simt = p.nsplit > 1 ? (size_t)p.nsplit * T * E * sizeof(float) : 0;
   const size_t tc = (E % 4 == 0 && d >= 64) ? 256 + tc_router_w3_bytes(d, E) + tc_router_planes_bytes(T, d, E) : 0;
   return simt > tc ? simt : tc;
+}
+
+// The query covers every batch of at most T tokens, so one workspace serves a layer whose
+// batches vary: a smaller batch may split K more ways and use more.  Both split choices
+// depend on the batch only through its number of row tiles (128, 256 or 512 rows for the
+// SIMT router, 256-row pairs for the tensor cores, which also start at 256 rows), which is
+// constant on each run (128 (q - 1), 128 q]; the bytes grow with the tokens inside a run,
+// so the top of each run (and T itself) bounds it.
+size_t route_workspace_bytes(int T, int d, int E) {
+  if (T <= 0 || E <= 0 || d <= 0) return 0;
+  size_t most = route_workspace_at(T, d, E);
+  for (int t = 128; t < T; t += 128) {
+    const size_t w = route_workspace_at(t, d, E);
+    if (w > most) most = w;
+  }
+  return most;
 }
 
 moe_status launch_route(const void* x, int x_dtype, const float* Wg, const float* logit_offset,

@@ -79,6 +79,20 @@ def _route(L, **kw):
                        a["renorm"], a["scale"], a["logits"], a["idx"], a["gate"], a["ws"], a["wsb"], a["s"])
 
 
+@pytest.mark.parametrize("d,E", [(2048, 64), (4096, 63), (7168, 896), (1024, 36), (64, 8), (512, 1024)])
+def test_workspace_queries_cover_every_smaller_batch(L, d, E):
+    """A smaller batch may split the router GEMM more ways (SIMT split-K, tensor-core K
+    runs), so a query for T must cover every T' <= T: one layer workspace serves them all."""
+    ts = sorted(set(list(range(1, 1200, 37)) + list(range(1024, 20000, 389)) + [256, 2368, 4608, 4864, 5000, 8192]))
+    prev_r = prev_w = 0
+    for T in ts:
+        r = L.moe_route_workspace_bytes(T, d, E)
+        w = L.moe_workspace_bytes(T, d, E, 8)
+        assert r >= prev_r and w >= prev_w, (T, r, prev_r)
+        assert w >= r
+        prev_r, prev_w = r, w
+
+
 @pytest.mark.parametrize("kw,status", [
     (dict(x=NUL), 1), (dict(Wg=NUL), 1), (dict(logits=NUL), 1), (dict(k=17), 1), (dict(k=0), 1),
     (dict(E=0), 1), (dict(T=-1), 1), (dict(score=3), 1), (dict(dt=7), 1), (dict(renorm=2), 1),
