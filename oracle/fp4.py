@@ -144,7 +144,7 @@ def nvfp4_quantize(W, block: int = NV_BLOCK) -> tuple:
     if K % block:
         raise ValueError("K must be a multiple of the block size")
     amax = float(np.abs(W).max()) if W.size else 0.0
-    s_t = amax / (E2M1_MAX * E4M3_MAX) if amax > 0 else 1.0
+    s_t = float(np.float32(amax / (E2M1_MAX * E4M3_MAX))) if amax > 0 else 1.0   # an fp32 scale (R25)
     s_b = np.empty((rows, K // block), np.float64)
     codes = np.empty((rows, K), np.uint8)
     for r in range(rows):
