@@ -92,6 +92,11 @@ typedef enum {
 typedef enum { MOE_BF16 = 0, MOE_F32 = 1 } moe_dtype;
 
 typedef enum {
+  MOE_FP4_MX = 0,               /* MXFP4: 32-element blocks, E8M0 power-of-two scales      */
+  MOE_FP4_NV = 1                /* NVFP4: 16-element blocks, E4M3 scales + an fp32 scale   */
+} moe_fp4_format;
+
+typedef enum {
   MOE_SELECT_UNIFORM = 0,       /* slot j of token t takes expert (t k + j) mod E        */
   MOE_SELECT_HASH = 1           /* k distinct experts from a hash of the token id         */
 } moe_select_rule;
@@ -407,6 +412,34 @@ MOE_API moe_status moe_router_stats(const float* logits, const int32_t* counts, 
  * aligned; bytes = 0 does nothing.  This step has no counterpart on the pages (it only
  * initialises an output buffer). */
 MOE_API moe_status moe_zero(void* p, size_t bytes, void* stream);
+
+/* ------------------------------------------------------------------------------------
+ * moe_quantize_fp4_host / moe_dequantize_fp4_host -- 4-bit expert weights, packed on the
+ * host once at load time.
+ * [Handbook-Digest] "已确认", bullet "量化与推理" (Kimi K3's routed experts in MXFP4;
+ * NVIDIA's NVFP4 training with key layers in BF16).  Formats:
+ *   element  FP4 E2M1 (magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6), w / scale rounded to
+ *            nearest, ties to the even mantissa bit, magnitudes above 6 saturating;
+ *   MXFP4    32-element blocks, scale 2^E stored as the byte E + 127 (E8M0),
+ *            E = floor(log2 amax_block) - 2 clamped to [-127, 127] (-127 if all zero);
+ *   NVFP4    16-element blocks, scale byte = FP8 E4M3 of amax_block / 6 / s_t (nearest
+ *            even, saturating at 448), and one fp32 tensor scale s_t = amax / (6 * 448)
+ *            (1 if all zero); a block whose scale rounds to 0 stores zeros.
+ *   W            (host) [rows, K] fp32, row-major (the K-major weight: W_gu or W_dn rows)
+ *   codes        (host) [rows, K/2] bytes: element 2j in the low nibble of byte j
+ *   scales       (host) [rows, K/block] bytes, block = moe_fp4_block_size(fmt)
+ *   tensor_scale (host) one fp32 (NVFP4 only; may be NULL for MXFP4)
+ *   threads      host threads (0 = all cores); the result does not depend on it
+ * Dequantization returns code value x block scale (x tensor scale), rounded to fp32.
+ * Errors: INVALID_ARG for a null pointer, negative sizes or threads, or an unknown format;
+ * UNSUPPORTED when K is not a multiple of the block.  No device memory is touched.
+ * ---------------------------------------------------------------------------------- */
+MOE_API int32_t moe_fp4_block_size(int32_t fmt);
+MOE_API moe_status moe_quantize_fp4_host(const float* W, int64_t rows, int64_t K, int32_t fmt,
+                     uint8_t* codes, uint8_t* scales, float* tensor_scale, int32_t threads);
+MOE_API moe_status moe_dequantize_fp4_host(const uint8_t* codes, const uint8_t* scales,
+                     const float* tensor_scale, int64_t rows, int64_t K, int32_t fmt,
+                     float* W, int32_t threads);
 
 /* Largest workspace any of the calls above needs for these sizes, for every call with
  * at most T tokens (each size query covers the batches below its T). */

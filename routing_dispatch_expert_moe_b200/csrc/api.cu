@@ -156,6 +156,32 @@ moe_status moe_route_noisy(const float* logits, const float* logits_noise, const
   return launch_route_noisy(logits, logits_noise, noise, T, E, k, scale, H, topk_idx, topk_gate, S(stream));
 }
 
+int32_t moe_fp4_block_size(int32_t fmt) { return fp4_block(fmt); }
+
+moe_status moe_quantize_fp4_host(const float* W, int64_t rows, int64_t K, int32_t fmt, uint8_t* codes,
+                                 uint8_t* scales, float* tensor_scale, int32_t threads) {
+  const int B = fp4_block(fmt);
+  if (B < 0 || rows < 0 || K < 0 || threads < 0) return MOE_ERR_INVALID_ARG;
+  if (K % B != 0) return MOE_ERR_UNSUPPORTED;
+  if (fmt == MOE_FP4_NV && !tensor_scale) return MOE_ERR_INVALID_ARG;
+  if (rows == 0 || K == 0) {
+    if (fmt == MOE_FP4_NV) *tensor_scale = 1.0f;
+    return MOE_OK;
+  }
+  if (!W || !codes || !scales) return MOE_ERR_INVALID_ARG;
+  return quantize_fp4_host(W, rows, K, fmt, codes, scales, tensor_scale, threads);
+}
+
+moe_status moe_dequantize_fp4_host(const uint8_t* codes, const uint8_t* scales, const float* tensor_scale,
+                                   int64_t rows, int64_t K, int32_t fmt, float* W, int32_t threads) {
+  const int B = fp4_block(fmt);
+  if (B < 0 || rows < 0 || K < 0 || threads < 0) return MOE_ERR_INVALID_ARG;
+  if (K % B != 0) return MOE_ERR_UNSUPPORTED;
+  if (rows == 0 || K == 0) return MOE_OK;
+  if (!codes || !scales || !W || (fmt == MOE_FP4_NV && !tensor_scale)) return MOE_ERR_INVALID_ARG;
+  return dequantize_fp4_host(codes, scales, tensor_scale, rows, K, fmt, W, threads);
+}
+
 size_t moe_histogram_scan_workspace_bytes(int32_t T, int32_t k, int32_t E) {
   if (T < 0 || k < 1 || E < 1) return 0;
   return histogram_scan_workspace_bytes(T, k, E);

@@ -129,6 +129,12 @@ moe_status launch_combine(const void* y_rows, int rows_dtype, const int32_t* row
                           const void* shared_y, int T, int d, int k, long long rows_max, int y_dtype,
                           void* y, cudaStream_t s);
 
+int fp4_block(int fmt);
+moe_status quantize_fp4_host(const float* W, long long rows, long long K, int fmt, uint8_t* codes, uint8_t* scales,
+                             float* tensor_scale, int threads);
+moe_status dequantize_fp4_host(const uint8_t* codes, const uint8_t* scales, const float* tensor_scale, long long rows,
+                               long long K, int fmt, float* W, int threads);
+
 moe_status launch_round_bf16(float* in, long long n, void* out, int clear, cudaStream_t s);
 
 moe_status launch_router_stats(const float* logits, const int32_t* counts, const int32_t* kept,

@@ -20,6 +20,7 @@ LIB_PATH = os.environ.get("MOE_B200_LIB", os.path.join(_HERE, "libmoe_b200.so"))
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_DEVICE = range(6)
 SCORE = {"softmax": 0, "sigmoid": 1, "sqrt_softplus": 2}
 SELECT = {"uniform": 0, "hash": 1}
+FP4 = {"mxfp4": 0, "nvfp4": 1}
 DTYPE = {torch.bfloat16: 0, torch.float32: 1}
 DEVERR = {0: "none", 1: "expert id out of range", 2: "duplicate expert in a token", 3: "row index out of range",
           4: "scan look-back timeout", 5: "GEMM pipeline timeout"}
@@ -44,6 +45,9 @@ _SIGNATURES = {
                                _c_void_p, _c_void_p, _c_void_p]),
     "moe_route_noisy": (_i32, [_c_void_p, _c_void_p, _c_void_p, _i32, _i32, _i32, _f32, _c_void_p, _c_void_p,
                                _c_void_p, _c_void_p]),
+    "moe_fp4_block_size": (_i32, [_i32]),
+    "moe_quantize_fp4_host": (_i32, [_c_void_p, _i64, _i64, _i32, _c_void_p, _c_void_p, _c_void_p, _i32]),
+    "moe_dequantize_fp4_host": (_i32, [_c_void_p, _c_void_p, _c_void_p, _i64, _i64, _i32, _c_void_p, _i32]),
     "moe_histogram_scan_workspace_bytes": (_size, [_i32, _i32, _i32]),
     "moe_histogram_scan": (_i32, [_c_void_p, _c_void_p, _i32, _i32, _i32, _i32, _c_void_p, _c_void_p, _c_void_p,
                                   _c_void_p, _c_void_p, _c_void_p, _c_void_p, _size, _c_void_p]),
@@ -242,6 +246,43 @@ def moe_route_noisy(logits, logits_noise, noise, k: int, scale: float = 1.0, H=N
     _check("moe_route_noisy", lib().moe_route_noisy(_p(logits), _p(logits_noise), _p(noise), T, E, k, float(scale),
                                                     _p(H), _p(topk_idx), _p(topk_gate), _stream(stream)))
     return H, topk_idx, topk_gate
+
+
+def _host_ptr(a):
+    return ctypes.c_void_p(a.ctypes.data)
+
+
+def moe_quantize_fp4_host(W, fmt: str = "mxfp4", threads: int = 0):
+    """4-bit expert weights packed on the host: W [rows, K] (numpy, fp32) ->
+    (codes uint8 [rows, K/2], scales uint8 [rows, K/block], tensor_scale float or None)."""
+    import numpy as np
+    if fmt not in FP4:
+        raise ValueError(f"fmt must be one of {sorted(FP4)}")
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    rows, K = W.shape
+    block = int(lib().moe_fp4_block_size(FP4[fmt]))
+    codes = np.zeros((rows, K // 2), np.uint8)
+    scales = np.zeros((rows, max(K // block, 0)), np.uint8)
+    ts = np.ones(1, np.float32)
+    _check("moe_quantize_fp4_host", lib().moe_quantize_fp4_host(_host_ptr(W), rows, K, FP4[fmt], _host_ptr(codes),
+                                                                _host_ptr(scales), _host_ptr(ts), int(threads)))
+    return codes, scales, (float(ts[0]) if fmt == "nvfp4" else None)
+
+
+def moe_dequantize_fp4_host(codes, scales, tensor_scale, K: int, fmt: str = "mxfp4", threads: int = 0):
+    """Inverse of moe_quantize_fp4_host: fp32 W [rows, K] (numpy)."""
+    import numpy as np
+    if fmt not in FP4:
+        raise ValueError(f"fmt must be one of {sorted(FP4)}")
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    rows = codes.shape[0]
+    W = np.empty((rows, K), np.float32)
+    ts = np.array([1.0 if tensor_scale is None else tensor_scale], np.float32)
+    _check("moe_dequantize_fp4_host", lib().moe_dequantize_fp4_host(_host_ptr(codes), _host_ptr(scales),
+                                                                    _host_ptr(ts), rows, K, FP4[fmt],
+                                                                    _host_ptr(W), int(threads)))
+    return W
 
 
 def moe_histogram_scan(topk_idx, topk_gate, E: int, capacity: int = -1, counts=None, kept=None, offsets=None,
