@@ -26,8 +26,10 @@
  *   [Handbook-Article] "Hugging Face开源MoE训练手册：基于80万GH200卡时沉淀Megatron-LM实战" (zicq.com)
  *
  * Conventions for every call
- *   - Pointers marked (device) must point to device memory owned by the caller;
- *     the library allocates nothing and keeps no state except one device error word.
+ *   - Pointers marked (device) must point to device memory owned by the caller, and
+ *     pointers marked (host) to host memory; the library allocates nothing and keeps no
+ *     state except one device error word (and the fixed scratch array of
+ *     moe_histogram_scan_noalloc).
  *   - All launches are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
  *     stream).  No call synchronises the host, except moe_get_device_error.
  *   - Layouts are dense row-major (C order) with the leading dimension equal to the
@@ -430,7 +432,8 @@ MOE_API moe_status moe_zero(void* p, size_t bytes, void* stream);
  *   scales       (host) [rows, K/block] bytes, block = moe_fp4_block_size(fmt)
  *   tensor_scale (host) one fp32 (NVFP4 only; may be NULL for MXFP4)
  *   threads      host threads (0 = all cores); the result does not depend on it
- * Dequantization returns code value x block scale (x tensor scale), rounded to fp32.
+ * Both run on the host and return when done (no stream, no launch).  Dequantization
+ * returns code value x block scale (x tensor scale), rounded to fp32.
  * Errors: INVALID_ARG for a null pointer, negative sizes or threads, or an unknown format;
  * UNSUPPORTED when K is not a multiple of the block.  No device memory is touched.
  * ---------------------------------------------------------------------------------- */
