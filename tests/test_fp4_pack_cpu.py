@@ -119,3 +119,28 @@ def test_fp4_host_validation(M):
     assert d(P, P, None, 2, 40, 0, F, 0) == 2
     assert d(None, P, None, 2, 64, 0, F, 0) == 1
     assert d(None, None, None, 0, 64, 0, None, 0) == 0
+
+
+def test_pack_matches_the_oracle_on_random_blocks(M):
+    """Randomised: rows of mixed magnitudes, signs, exact zeros and values on E2M1
+    midpoints, for both formats."""
+    from hypothesis import given, settings, strategies as st
+    from hypothesis.extra import numpy as hnp
+
+    vals = st.one_of(st.floats(-1e6, 1e6, width=32), st.sampled_from([0.0, -0.0, 0.25, 0.75, 2.5, 5.0, -3.5]))
+
+    @settings(max_examples=60, deadline=None, derandomize=True)
+    @given(hnp.arrays(np.float32, st.tuples(st.integers(1, 6), st.sampled_from([32, 64, 96])), elements=vals))
+    def check(W):
+        for fmt in ("mxfp4", "nvfp4"):
+            codes, scales, ts = M.moe_quantize_fp4_host(W, fmt, threads=2)
+            if fmt == "mxfp4":
+                E, oc = Q.mxfp4_quantize(W)
+                assert np.array_equal(scales.astype(np.int32) - 127, E)
+            else:
+                st_, sb, oc = Q.nvfp4_quantize(W)
+                assert ts == st_
+                assert np.array_equal(torch.from_numpy(scales.copy()).view(torch.float8_e4m3fn).double().numpy(), sb)
+            assert np.array_equal(_nibbles(codes), oc)
+
+    check()
