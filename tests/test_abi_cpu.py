@@ -249,3 +249,27 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     with pytest.raises(RuntimeError):
         m.lib()
     importlib.reload(m)
+
+
+def test_capacity_and_rows_max_agree_with_the_oracle_on_random_sizes(L):
+    """The library's host arithmetic against the oracle: the capacity formula in both
+    readings, and the rows bound holding every plan the oracle builds."""
+    import numpy as np
+    from oracle import moe_oracle as O
+    rng = np.random.default_rng(11)
+    for _ in range(400):
+        T = int(rng.integers(0, 40000))
+        E = int(rng.integers(1, 1025))
+        k = int(rng.integers(1, min(E, 32) + 1))
+        cf = float(rng.choice([0.0, -1.0, rng.uniform(0.01, 4.0), 1.0, 1.25]))
+        for per in (True, False):
+            want = O.capacity(T, E, k, cf if cf > 0 else None, per)
+            assert L.moe_capacity(T, E, k, cf, 1 if per else 0) == want, (T, E, k, cf, per)
+    for _ in range(60):
+        T, E = int(rng.integers(1, 300)), int(rng.integers(1, 40))
+        k = int(rng.integers(1, min(E, 8) + 1))
+        cap = int(rng.choice([-1, 0, 1, int(rng.integers(1, 60))]))
+        idx = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
+        plan = O.dispatch_plan(idx, np.ones((T, k)), E, cap)
+        assert int(plan["offsets"][-1]) <= L.moe_rows_max(T, E, k, cap)
+        assert L.moe_rows_max(T, E, k, cap) == (T * k if cap < 0 else min(T * k, E * cap))
