@@ -4,8 +4,10 @@
 
 A step is one pass of the whole layer (router, top-k, histogram/scan, permute, grouped
 gate/up GEMM + SwiGLU, grouped down GEMM x gate, combine, router statistics) over one
-batch of synthetic tokens of the handbook-scale workload (T=8192, d=2048, E=64, k=8,
-F=1024, bf16, fp32 router).  Inputs are resident in HBM; L2 is flushed (256 MB write)
+batch of synthetic tokens.  The default workload is the largest one, the very-many-
+experts stress layer (T=32768, d=7168, E=896, k=16, F=256, sqrt(softplus) scores, Zipf
+skew, capacity factor 1.0 with token-order dropping; bf16 with an fp32 router);
+--workload picks another.  Inputs are resident in HBM; L2 is flushed (256 MB write)
 before every step and each step is timed with CUDA events on the launching stream.
 With N > 1 (torchrun) every rank runs an independent replica on its own token batch
 (the layer has no data-path collective); the timing is the max over ranks.
@@ -33,9 +35,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM traffic (read + write bytes) of the dominant kernel, the gate/up GEMM, per launch, keyed
 # by (workload, dispatch), from an ncu capture of the same kernel build (summaries under
-# profiles/); absent when the kernel changed since the capture.  The last capture (934.6 MB
-# on the handbook workload, the algorithmic 939.5 MB) predates an edit of the CTA-pair
-# kernel template (the router's K split), so no entry is current.
+# profiles/); absent when the kernel changed since the capture.
 GATE_UP_TRAFFIC = {}
 
 
@@ -130,37 +130,51 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
-def layer_roofline_ms(cfg, A, pk, rb=4, ob=4, fused=False, gather=False):
+def layer_roofline_ms(cfg, A, pk, rb=4, ob=4, fused=False, gather=False, E_act=None):
     """Sum over steps of max(compute, memory) time at the measured peaks (algorithmic bytes / flops).
-    rb / ob: bytes per element of the gated rows / of the layer output.  fused: the combine runs
-    inside the down GEMM, whose algorithmic bytes are then H, W_dn and y (zero fill + result).
-    gather: the permute runs inside the gate/up GEMM, whose algorithmic bytes are then x, W_gu, H."""
+    A: kept assignment rows; E_act: experts with at least one kept row (only their weights are
+    read).  rb / ob: bytes per element of the gated rows / of the layer output.  fused: the
+    combine runs inside the down GEMM, whose algorithmic bytes are then H, W_dn and y (zero
+    fill + result).  gather: the permute runs inside the gate/up GEMM, whose algorithmic bytes
+    are then x, W_gu, H.  The router is priced at its algorithmic 2 T d E flops on the bf16
+    tensor cores (however many terms an implementation issues) or its bytes, whichever is
+    slower, so the sum is a lower bound for any implementation."""
     T, d, E, k, F = cfg.T, cfg.d, cfg.E, cfg.k, cfg.F
+    Ea = E if E_act is None else E_act
     hbm = pk["hbm_gbs"] * 1e9
     tc = pk["bf16_tflops"] * 1e12
-    fp32 = 148 * 128 * 2 * pk.get("sm_max_mhz", 1965.0) * 1e6      # FMA lanes x 2 x clock
     b = 2
     steps = {
-        "route": max(2 * T * d * E / fp32, (T * d * b + d * E * 4 + T * E * 4 + T * k * 8) / hbm),
+        "route": max(2 * T * d * E / tc, (T * d * b + d * E * 4 + T * E * 4 + T * k * 8) / hbm),
         "histogram_scan": (T * k * 4 * 3 + A * 8) / hbm,
         "stats": (T * E * 4) / hbm,
     }
     if gather:
-        steps["gate_up_gather"] = max(4 * A * d * F / tc, (T * d * b + E * 2 * F * d * b + A * F * b) / hbm)
+        steps["gate_up_gather"] = max(4 * A * d * F / tc, (T * d * b + Ea * 2 * F * d * b + A * F * b) / hbm)
     else:
         steps["permute"] = (T * d * b + A * d * b) / hbm
-        steps["gate_up"] = max(4 * A * d * F / tc, (A * d * b + E * 2 * F * d * b + A * F * b) / hbm)
+        steps["gate_up"] = max(4 * A * d * F / tc, (A * d * b + Ea * 2 * F * d * b + A * F * b) / hbm)
     if fused:
-        steps["down_combine"] = max(2 * A * F * d / tc, (A * F * b + E * d * F * b + 2 * T * d * 4) / hbm)
+        steps["down_combine"] = max(2 * A * F * d / tc, (A * F * b + Ea * d * F * b + 2 * T * d * 4) / hbm)
         if ob == 2:
             steps["round_output"] = (T * d * 4 + T * d * 2) / hbm
     else:
-        steps["down"] = max(2 * A * F * d / tc, (A * F * b + E * d * F * b + A * d * rb) / hbm)
+        steps["down"] = max(2 * A * F * d / tc, (A * F * b + Ea * d * F * b + A * d * rb) / hbm)
         steps["combine"] = (A * d * rb + T * d * ob) / hbm
     if cfg.F_s:
         Fs = cfg.F_s
         steps["shared"] = max(6 * T * d * Fs / tc, (T * d * b + 3 * d * Fs * b + T * Fs * b + T * d * rb) / hbm)
     return sum(steps.values()) * 1e3, {k_: v * 1e3 for k_, v in steps.items()}
+
+
+def gate_up_work(cfg, A, E_act, gather=False):
+    """Algorithmic work of one gate/up GEMM launch: 4 d F flops per kept assignment row, and the
+    bytes it must move: its A rows (the permuted copy, or x itself when gathered), the weights of
+    every expert that has a row (2 F x d each), and H (F per row); all bf16."""
+    flops = 4.0 * A * cfg.d * cfg.F
+    rows_in = (cfg.T if gather else A) * cfg.d * 2
+    nbytes = rows_in + E_act * 2 * cfg.F * cfg.d * 2 + A * cfg.F * 2
+    return flops, nbytes
 
 
 def run_ours(args):
@@ -240,6 +254,7 @@ def run_ours(args):
         torch.cuda.synchronize()
         assert M.moe_get_device_error() == 0
         rows = int(layer.offsets[-1].item())
+        e_act = int((layer.kept > 0).sum().item())
         ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
         gu_name = "gate_up_gather" if layer.dispatch_mode == "gather" else "gate_up"
 
@@ -295,11 +310,11 @@ def run_ours(args):
                     acc += [evs[j].elapsed_time(evs[j + 1]) for j in range(len(stages))]
             stage_ms.update({n: float(acc[j] / breakdown_steps) for j, (n, _) in enumerate(stages)})
             del g2
-        return per_step, stage_ms, rows, clk
+        return per_step, stage_ms, (rows, e_act), clk
 
     layer = make_layer(args.combine, args.dispatch)
-    per_step, stage_ms, A, clk = time_layer(layer, args.steps, ClockSampler(local_rank),
-                                            breakdown_steps=args.breakdown_steps)
+    per_step, stage_ms, (A, E_act), clk = time_layer(layer, args.steps, ClockSampler(local_rank),
+                                                     breakdown_steps=args.breakdown_steps)
     total_ms = max_over_ranks(float(per_step.sum()), dev)
     ms_per_step = total_ms / args.steps
     value = job_throughput(cfg.T, world, args.steps, total_ms)
@@ -386,18 +401,31 @@ def run_ours(args):
     pk, pk_src = peaks()
     gather = args.dispatch == "gather"
     gate_up_ms = stage_ms["timed_gate_up_gather" if gather else "timed_gate_up"]   # inside the timed region
-    flops = 4.0 * A * cfg.d * cfg.F
-    achieved = flops / (gate_up_ms * 1e-3) / 1e12
-    peak = pk["bf16_tflops"]
+    flops, gu_bytes = gate_up_work(cfg, A, E_act, gather)
+    t_tensor, t_hbm = flops / (pk["bf16_tflops"] * 1e12), gu_bytes / (pk["hbm_gbs"] * 1e9)
+    if t_tensor >= t_hbm:
+        roof = {"bound": "tensor", "achieved": round(flops / (gate_up_ms * 1e-3) / 1e12, 1),
+                "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "peak_source": f"{pk_src} bf16_tflops (burst)"}
+    else:
+        roof = {"bound": "hbm", "achieved": round(gu_bytes / (gate_up_ms * 1e-3) / 1e9, 1),
+                "peak": pk["hbm_gbs"], "unit": "GB/s", "peak_source": f"{pk_src} hbm_gbs"}
+    roof["frac"] = round(roof["achieved"] / roof["peak"], 4)
+    roof["algorithmic"] = {"flops": flops, "bytes": gu_bytes, "rows": A, "experts_with_rows": E_act,
+                           "tensor_ms": round(t_tensor * 1e3, 4), "hbm_ms": round(t_hbm * 1e3, 4),
+                           "kernel_ms": round(gate_up_ms, 4)}
+    roof["traffic"] = GATE_UP_TRAFFIC.get((args.workload, args.dispatch, A))
     fused = args.combine == "fused"
     rb = 4 if fused else layer.y_perm.element_size()
     ob = layer.y.element_size()
-    roof_ms, roof_steps = layer_roofline_ms(cfg, A, pk, rb, ob, fused, gather)
-    traffic = GATE_UP_TRAFFIC.get((args.workload, args.dispatch))
+    roof_ms, roof_steps = layer_roofline_ms(cfg, A, pk, rb, ob, fused, gather, E_act)
     thr = {}                                # from the per-stage split, when it ran
     if stage_ms.get("route"):
         down_ms = stage_ms["down_combine" if fused else "down"]
         thr["down_tflops"] = round(2.0 * A * cfg.F * cfg.d / (down_ms * 1e-3) / 1e12, 1)
+        thr["down_gbs"] = round((A * cfg.F * 2 + E_act * cfg.d * cfg.F * 2 + (0 if fused else A * cfg.d * rb)) /
+                                (down_ms * 1e-3) / 1e9, 1)
+        thr["gate_up_gbs"] = round(gu_bytes / (stage_ms["gate_up_gather" if gather else "gate_up"] * 1e-3) / 1e9, 1)
+        thr["route_tflops"] = round(2.0 * cfg.T * cfg.d * cfg.E / (stage_ms["route"] * 1e-3) / 1e12, 1)
         thr["route_gbs"] = round((cfg.T * cfg.d * 2 + cfg.T * cfg.E * 8 + cfg.T * cfg.k * 8) /
                                  (stage_ms["route"] * 1e-3) / 1e9, 1)
         if not gather:
@@ -408,7 +436,7 @@ def run_ours(args):
 
     out = None
     if rank == 0:
-        cpu = (cpu_baseline(cfg, budget_s=args.cpu_budget)
+        cpu = (cpu_baseline(cfg, args.ref_tokens, budget_s=args.cpu_budget)
                if (world == 1 and not args.no_cpu_baseline and routing == "learned") else None)
         out = {
             "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -426,13 +454,9 @@ def run_ours(args):
             "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d_bytes,
                     "d2h_bytes_per_step": d2h_bytes, "steps": e2e_steps,
                     "schedule": "two layer instances, copy in / forward / copy out on three streams"},
-            "gpu_launches": args.steps * layer.launches_per_forward(True),
-            "roofline": {"bound": "tensor",
-                         "kernel": ("moe_expert_gate_up_gather (tcgen05 grouped GEMM, gathered rows, SwiGLU)"
-                                    if gather else "moe_expert_gate_up (tcgen05 grouped GEMM + SwiGLU)"),
-                         "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
-                         "frac": round(achieved / peak, 4), "traffic": traffic,
-                         "peak_source": f"{pk_src} bf16_tflops (burst)"},
+            "gpu_launches": args.steps * layer.launches_per_forward(True, cfg.T),
+            "roofline": {"kernel": ("moe_expert_gate_up_gather (tcgen05 grouped GEMM, gathered rows, SwiGLU)"
+                                    if gather else "moe_expert_gate_up (tcgen05 grouped GEMM + SwiGLU)"), **roof},
             "layer_roofline": {"ms": round(roof_ms, 4), "frac": round(roof_ms / ms_per_step, 4),
                                "tokens_per_s": round(cfg.T / (roof_ms / 1e3), 1)},
             "stages_ms": {k_: round(v, 4) for k_, v in stage_ms.items()},
@@ -460,14 +484,14 @@ def _oracle_step(cfg, x_np, Wg, off, bias, gu, dn, sh, tokens):
 
 
 def _oracle_setup(cfg):
+    """Inputs for the oracle; each expert's weights are widened to float64 when the oracle asks
+    for them (the stress workload's experts would take about 40 GB of float64 at once)."""
     from routing_dispatch_expert_moe_b200 import inputs as I
     x_np = I.gen_x(cfg, 0)
     Wg, off, bias = I.gen_router(cfg, 0)
     W_gu, W_dn = I.gen_experts_torch(cfg, 0)
-    gu = {e: W_gu[e].double().numpy() for e in range(cfg.E)}      # model weights as the oracle reads them
-    dn = {e: W_dn[e].double().numpy() for e in range(cfg.E)}
     sh = I.gen_shared(cfg, 0)
-    return x_np, Wg, off, bias, (lambda e: gu[e]), (lambda e: dn[e]), sh
+    return x_np, Wg, off, bias, (lambda e: W_gu[e].double().numpy()), (lambda e: W_dn[e].double().numpy()), sh
 
 
 def _threads():
@@ -479,24 +503,39 @@ def _threads():
         return os.cpu_count() or 1
 
 
-def cpu_baseline(cfg, budget_s=15.0):
-    """The oracle on a bounded token sample of the same workload, timed on the host cores."""
+def oracle_sample_run(cfg, setup, n_tokens, steps, warmup, seed):
+    """The oracle as it stands, timed on the host: each step is one pass of the whole layer
+    over a fresh random sample of n_tokens tokens of the workload (routing, capacity and the
+    dispatch plan of that sample, the SwiGLU experts in float64, the combine).  Returns
+    (tokens/s, total seconds, per-step seconds)."""
+    rng = np.random.default_rng(seed)
+    for _ in range(warmup):
+        _oracle_step(cfg, *setup, rng.choice(cfg.T, size=n_tokens, replace=False))
+    times = []
+    for _ in range(steps):
+        tok = rng.choice(cfg.T, size=n_tokens, replace=False)
+        t0 = time.perf_counter()
+        _oracle_step(cfg, *setup, tok)
+        times.append(time.perf_counter() - t0)
+    total = float(np.sum(times))
+    return n_tokens * steps / total, total, times
+
+
+def oracle_sample_text(cfg, n_tokens, steps, total_s):
+    return (f"{steps} steps of {n_tokens} of {cfg.T} tokens each (fresh random sample per step): routing, "
+            f"capacity and dispatch plan of the sample, SwiGLU experts in float64 numpy, combine; {total_s:.1f} s")
+
+
+def cpu_baseline(cfg, n_tokens=48, budget_s=15.0):
+    """The oracle on the host cores, on the same per-step token sample as the reference arm
+    (bench.py --impl reference): as many steps as fit in about budget_s seconds."""
     setup = _oracle_setup(cfg)
-    rng = np.random.default_rng(1)
-    n = 64
-    tokens = rng.choice(cfg.T, size=n, replace=False)
-    t0 = time.perf_counter()
-    _oracle_step(cfg, *setup, tokens)
-    dt1 = time.perf_counter() - t0
-    n = int(min(cfg.T, max(64, n * budget_s / max(dt1, 1e-3))))
-    tokens = rng.choice(cfg.T, size=n, replace=False)
-    t0 = time.perf_counter()
-    _oracle_step(cfg, *setup, tokens)
-    dt2 = time.perf_counter() - t0
-    return {"value": round(n / dt2, 2), "unit": UNIT, "cores": _threads(), "kind": "oracle",
-            "sample": f"{n} of {cfg.T} tokens (random), full layer per token: routing, dispatch plan, "
-                      f"SwiGLU experts (float64 numpy), combine; {dt2:.1f} s",
-            "host_cpu": _cpu_model(), "nproc": os.cpu_count()}
+    _, t1, _ = oracle_sample_run(cfg, setup, n_tokens, 1, 1, seed=1)
+    steps = int(max(1, min(200, budget_s / max(t1, 1e-3))))
+    value, total, _ = oracle_sample_run(cfg, setup, n_tokens, steps, 0, seed=2)
+    return {"value": round(value, 2), "unit": UNIT, "cores": _threads(), "kind": "oracle",
+            "sample": oracle_sample_text(cfg, n_tokens, steps, total), "host_cpu": _cpu_model(),
+            "nproc": os.cpu_count()}
 
 
 def _cpu_model():
@@ -518,26 +557,15 @@ def run_reference(args):
     from routing_dispatch_expert_moe_b200 import inputs as I
     cfg = I.CONFIGS[args.workload]
     setup = _oracle_setup(cfg)
-    rng = np.random.default_rng(2)
     n = args.ref_tokens
-    for _ in range(args.warmup):
-        _oracle_step(cfg, *setup, rng.choice(cfg.T, size=n, replace=False))
-    times = []
-    for _ in range(args.steps):
-        tok = rng.choice(cfg.T, size=n, replace=False)
-        t0 = time.perf_counter()
-        _oracle_step(cfg, *setup, tok)
-        times.append(time.perf_counter() - t0)
-    total = float(np.sum(times))
-    value = n * args.steps / total
-    sample = f"{n} of {cfg.T} tokens per step (random), full layer per token, float64 numpy oracle"
+    value, total, _ = oracle_sample_run(cfg, setup, n, args.steps, args.warmup, seed=2)
     return {"impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total / args.steps * 1e3, 2),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded)",
             "config": workload_config(args.workload, cfg, O.capacity(cfg.T, cfg.E, cfg.k, cfg.capacity_factor, True)),
             "cpu_baseline": {"value": round(value, 2), "unit": UNIT, "cores": _threads(), "kind": "oracle",
-                             "sample": sample},
+                             "sample": oracle_sample_text(cfg, n, args.steps, total)},
             "e2e": {"value": round(value, 2), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
@@ -547,10 +575,11 @@ def main():
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="c2_handbook")
+    ap.add_argument("--workload", default="c5_stress")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--ref-tokens", type=int, default=48, help="tokens per reference-arm step")
+    ap.add_argument("--ref-tokens", type=int, default=48,
+                    help="tokens per oracle step (the reference arm and cpu_baseline time the same sample)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="override T (smaller cases of the same kernels, e.g. for profiler captures)")
     ap.add_argument("--e2e-steps", type=int, default=50, help="steps timed through host buffers")

@@ -4,6 +4,7 @@
  * The library computes the forward pass of a token-choice top-k Mixture-of-Experts
  * layer on one GPU, one stream-ordered step per call:
  *
+ *   moe_prepare_router_weight  the router's exact bf16 split of W_g, once at load time
  *   moe_route            router logits (fp32), scoring, optional selection-only bias,
  *                        top-k, renormalised and scaled gates
  *   moe_histogram_scan   per-expert counts, capacity clamp, token-order ranks,
@@ -128,6 +129,33 @@ MOE_API int32_t moe_capacity(int32_t T, int32_t E, int32_t k, double capacity_fa
 MOE_API int64_t moe_rows_max(int32_t T, int32_t E, int32_t k, int32_t capacity);
 
 /* ------------------------------------------------------------------------------------
+ * moe_prepare_router_weight -- the tensor-core router's operand, made once at load time.
+ * [MoE-Explained] section "Switch Transformer" (the router stays in full precision);
+ * [Handbook-News] "真正难在三个环节" item 1 (FP32 routing).
+ * The router multiplies a bf16 x by an fp32 W_g on bf16 tensor cores by splitting W_g
+ * exactly into three bf16 terms, hi = bf16(w), mid = bf16(w - hi), lo = bf16(w - hi -
+ * mid): the three carry all 24 significant bits of w, every product x * term is exact
+ * in fp32, and the MMAs accumulate in fp32, so the logits are fp32 sums of the exact
+ * products x . W_g.  This call writes that split for a given W_g; W_g does not change
+ * between forwards, so do it once (and again whenever W_g changes) and pass the result
+ * to moe_route / moe_router_logits.
+ *   Wg          (device) [d, E] fp32
+ *   Wg_split    (device) out, moe_router_weight_bytes(d, E) bytes, 16-byte aligned,
+ *               owned by the caller.  Layout: experts in n = ceil(E / 256) tiles of
+ *               NE = 32 * ceil(ceil(E / n) / 32) experts; tile j holds, as rows of a
+ *               K-major bf16 matrix [3 n NE, d], the hi terms of experts j NE .. j NE +
+ *               NE - 1, then their mid terms, then their lo terms (zero past E).
+ * moe_router_weight_bytes returns 0 when the tensor-core router does not apply to (d, E)
+ * (d < 64, d % 8 != 0, E % 4 != 0 or E > 1024); moe_prepare_router_weight then returns
+ * MOE_ERR_UNSUPPORTED and the router reads W_g directly.
+ * Errors: INVALID_ARG for a null pointer, d < 1 or E < 1; UNSUPPORTED as above or for an
+ * unaligned Wg_split; WORKSPACE when bytes is below the query.
+ * ---------------------------------------------------------------------------------- */
+MOE_API size_t moe_router_weight_bytes(int32_t d, int32_t E);
+MOE_API moe_status moe_prepare_router_weight(const float* Wg, int32_t d, int32_t E, void* Wg_split,
+                     size_t bytes, void* stream);
+
+/* ------------------------------------------------------------------------------------
  * moe_route -- router, scoring, top-k and gates.
  * [MoE-Explained] section "什么是稀疏性？": G_sigma(x) = Softmax(x . W_g),
  * KeepTopK(v, k), G(x) = Softmax(KeepTopK(H(x), k)); section "Switch Transformer"
@@ -137,6 +165,8 @@ MOE_API int64_t moe_rows_max(int32_t T, int32_t E, int32_t k, int32_t capacity);
  *
  *   x            (device) [T, d], x_dtype (MOE_BF16 or MOE_F32)
  *   Wg           (device) [d, E] fp32
+ *   Wg_split     (device) the result of moe_prepare_router_weight for this Wg, or NULL:
+ *                the call then splits W_g itself, into the workspace (one more launch)
  *   logit_offset (device) [E] fp32 or NULL: added to every logit (enters selection and gates)
  *   select_bias  (device) [E] fp32 or NULL: added to the score for selection only
  *   score        moe_score;  renormalize 0/1;  scale multiplies the final gates
@@ -144,8 +174,13 @@ MOE_API int64_t moe_rows_max(int32_t T, int32_t E, int32_t k, int32_t capacity);
  *   topk_idx     (device) [T, k] int32 out
  *   topk_gate    (device) [T, k] fp32 out
  *   workspace    (device) >= moe_route_workspace_bytes(T, d, E) bytes (may be NULL if 0);
- *                the query covers every call with at most T tokens (same d, E): a smaller
- *                batch may split the router GEMM more ways
+ *                the query covers every call with at most T tokens (same d, E), with or
+ *                without a prepared weight
+ * Paths: bf16 x with T >= 256, d >= 64 and E % 4 == 0 runs one tensor-core kernel (CTA
+ * pairs, 256 tokens per tile) that also selects the top-k and computes the gates in its
+ * epilogue (softmax scores with a selection bias add a separate top-k pass: their keys
+ * need the whole row's normaliser first).  Otherwise an fp32 SIMT GEMM and a top-k
+ * kernel run.
  * Gates: softmax + renormalize -> softmax over the k kept logits; softmax without
  * renormalize -> the full softmax probability; sigmoid / sqrt(softplus) -> kept scores
  * over their sum (renormalize) or the scores; all then times scale.  The softmax over
@@ -153,7 +188,7 @@ MOE_API int64_t moe_rows_max(int32_t T, int32_t E, int32_t k, int32_t capacity);
  * then rounds the gate to fp32 (the same for moe_route_fixed and moe_route_noisy).
  * ---------------------------------------------------------------------------------- */
 MOE_API size_t moe_route_workspace_bytes(int32_t T, int32_t d, int32_t E);
-MOE_API moe_status moe_route(const void* x, int32_t x_dtype, const float* Wg,
+MOE_API moe_status moe_route(const void* x, int32_t x_dtype, const float* Wg, const void* Wg_split,
                      const float* logit_offset, const float* select_bias,
                      int32_t T, int32_t d, int32_t E, int32_t k,
                      int32_t score, int32_t renormalize, float scale,
@@ -164,20 +199,23 @@ MOE_API moe_status moe_route(const void* x, int32_t x_dtype, const float* Wg,
  * moe_router_logits -- the router alone: logits = x . Wg (+ logit_offset), fp32.
  * [MoE-Explained] section "什么是稀疏性？" (x . W_g); section "Switch Transformer"
  * (router in full precision); [Handbook-News] "真正难在三个环节" item 1 (FP32 routing).
- * The same GEMM as moe_route (bf16 x with d >= 64 and E % 4 == 0: tensor cores with
- * W_g split exactly into three bf16 terms; otherwise fp32 SIMT), without the top-k.  It
+ * The same GEMM as moe_route (bf16 x with T >= 256, d >= 64 and E % 4 == 0: tensor
+ * cores over the three-term split of W_g; otherwise fp32 SIMT), without the top-k.  It
  * also gives the noise logits x . W_noise of moe_route_noisy.
  *   x            (device) [T, d], x_dtype;  16-byte aligned
  *   Wg           (device) [d, E] fp32
+ *   Wg_split     (device) moe_prepare_router_weight's result for this Wg, or NULL (split
+ *                into the workspace by the call)
  *   logit_offset (device) [E] fp32 or NULL
  *   logits       (device) [T, E] fp32 out
  *   workspace    (device) >= moe_router_logits_workspace_bytes(T, d, E) bytes (may be
  *                NULL if 0)
  * Errors: INVALID_ARG for a null pointer, T < 0, E < 1 or an unknown dtype;
- * UNSUPPORTED for E > 1024, d % 8 != 0 or an unaligned x; WORKSPACE if too small.
+ * UNSUPPORTED for E > 1024, d % 8 != 0 or an unaligned x or Wg_split; WORKSPACE if too
+ * small.
  * ---------------------------------------------------------------------------------- */
 MOE_API size_t moe_router_logits_workspace_bytes(int32_t T, int32_t d, int32_t E);
-MOE_API moe_status moe_router_logits(const void* x, int32_t x_dtype, const float* Wg,
+MOE_API moe_status moe_router_logits(const void* x, int32_t x_dtype, const float* Wg, const void* Wg_split,
                      const float* logit_offset, int32_t T, int32_t d, int32_t E,
                      float* logits, void* workspace, size_t workspace_bytes, void* stream);
 
@@ -272,10 +310,16 @@ MOE_API moe_status moe_histogram_scan(const int32_t* topk_idx, const float* topk
  * __device__ array that every GPU using the library keeps until the process exits.
  *
  *   - Limit: moe_histogram_scan_workspace_bytes(T, k, E) must be <= 4 MiB (4194304);
- *     larger sizes return MOE_ERR_WORKSPACE without launching anything.  The handbook
- *     workload (T=8192, k=8, E=64) needs about 0.3 MiB, T=32768 k=16 E=896 about 2.5 MiB.
+ *     larger sizes return MOE_ERR_WORKSPACE without launching anything (this check comes
+ *     before the pointer checks).  The handbook workload (T=8192, k=8, E=64) needs about
+ *     0.3 MiB, T=32768 k=16 E=896 about 2.5 MiB.
+ *   - The kernels run on the CURRENT device and use that device's copy of the array: the
+ *     buffers must live on the current device.  Device ordinals 64 and above return
+ *     MOE_ERR_UNSUPPORTED.
  *   - The first call on a device looks up the array's device address (once per device,
- *     with that device current); make that first call before any stream capture.
+ *     with that device current); make that first call before any stream capture.  The
+ *     address is kept for the life of the process: after cudaDeviceReset the library
+ *     must be unloaded and loaded again.
  *   - The call allocates nothing: it clears the part of the array that must start at
  *     zero with one memset node on `stream`, then launches the same kernels.
  *   - Every call shares the one array, which keeps the previous call's contents.  Calls

@@ -15,14 +15,18 @@ static thread_local cudaError_t g_last_cuda = cudaSuccess;
 cudaError_t& last_cuda_error_ref() { return g_last_cuda; }
 
 int* err_ptr() {
-  static int* cached[64] = {nullptr};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  if (!cached[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_moe_device_error) == cudaSuccess) cached[dev] = static_cast<int*>(p);
+  static std::atomic<int*> cached[kMaxDevices];
+  const int dev = device_slot();
+  if (dev < 0) return nullptr;
+  int* p = cached[dev].load(std::memory_order_acquire);
+  if (!p) {
+    void* a = nullptr;
+    if (cudaGetSymbolAddress(&a, g_moe_device_error) == cudaSuccess) {
+      p = static_cast<int*>(a);
+      cached[dev].store(p, std::memory_order_release);
+    }
   }
-  return cached[dev];
+  return p;
 }
 
 }  // namespace moe
@@ -90,10 +94,27 @@ int64_t moe_rows_max(int32_t T, int32_t E, int32_t k, int32_t capacity) {
 
 size_t moe_route_workspace_bytes(int32_t T, int32_t d, int32_t E) {
   if (T < 0 || d < 1 || E < 1) return 0;
-  return route_workspace_bytes(T, d, E);
+  return route_workspace_bytes(T, d, E, false);
 }
 
-moe_status moe_route(const void* x, int32_t x_dtype, const float* Wg, const float* logit_offset,
+size_t moe_router_weight_bytes(int32_t d, int32_t E) {
+  if (d < 1 || E < 1 || E > kMaxE || d % 8 != 0) return 0;
+  return router_weight_bytes(d, E);
+}
+
+moe_status moe_prepare_router_weight(const float* Wg, int32_t d, int32_t E, void* Wg_split, size_t bytes,
+                                     void* stream) {
+  if (d < 1 || E < 1) return MOE_ERR_INVALID_ARG;
+  if (E > kMaxE || d % 8 != 0) return MOE_ERR_UNSUPPORTED;
+  const size_t need = router_weight_bytes(d, E);
+  if (need == 0) return MOE_ERR_UNSUPPORTED;
+  if (!Wg || !Wg_split) return MOE_ERR_INVALID_ARG;
+  if (bytes < need) return MOE_ERR_WORKSPACE;
+  if (!aligned16(Wg_split)) return MOE_ERR_UNSUPPORTED;
+  return launch_prepare_router_weight(Wg, d, E, Wg_split, S(stream));
+}
+
+moe_status moe_route(const void* x, int32_t x_dtype, const float* Wg, const void* Wg_split, const float* logit_offset,
                      const float* select_bias, int32_t T, int32_t d, int32_t E, int32_t k, int32_t score,
                      int32_t renormalize, float scale, float* logits, int32_t* topk_idx, float* topk_gate,
                      void* workspace, size_t workspace_bytes, void* stream) {
@@ -105,31 +126,31 @@ moe_status moe_route(const void* x, int32_t x_dtype, const float* Wg, const floa
     return MOE_ERR_INVALID_ARG;
   if (T == 0) return MOE_OK;
   if (!x || !Wg || !logits || !topk_idx || !topk_gate) return MOE_ERR_INVALID_ARG;
-  if (!aligned16(x)) return MOE_ERR_UNSUPPORTED;
-  const size_t need = route_workspace_bytes(T, d, E);
+  if (!aligned16(x) || !aligned16(Wg_split)) return MOE_ERR_UNSUPPORTED;
+  const size_t need = route_workspace_bytes(T, d, E, Wg_split != nullptr);
   if (need > 0 && (!workspace || workspace_bytes < need)) return MOE_ERR_WORKSPACE;
-  return launch_route(x, x_dtype, Wg, logit_offset, select_bias, T, d, E, k, score, renormalize, scale, logits,
-                      topk_idx, topk_gate, workspace, S(stream));
+  return launch_route(x, x_dtype, Wg, Wg_split, logit_offset, select_bias, T, d, E, k, score, renormalize, scale,
+                      logits, topk_idx, topk_gate, workspace, S(stream));
 }
 
 size_t moe_router_logits_workspace_bytes(int32_t T, int32_t d, int32_t E) {
   if (T < 0 || d < 1 || E < 1) return 0;
-  return router_logits_workspace_bytes(T, d, E);
+  return router_logits_workspace_bytes(T, d, E, false);
 }
 
-moe_status moe_router_logits(const void* x, int32_t x_dtype, const float* Wg, const float* logit_offset, int32_t T,
-                             int32_t d, int32_t E, float* logits, void* workspace, size_t workspace_bytes,
-                             void* stream) {
+moe_status moe_router_logits(const void* x, int32_t x_dtype, const float* Wg, const void* Wg_split,
+                             const float* logit_offset, int32_t T, int32_t d, int32_t E, float* logits,
+                             void* workspace, size_t workspace_bytes, void* stream) {
   moe_status st = check_dims(T, E, 1);
   if (st != MOE_OK) return st;
   if ((st = check_d(d)) != MOE_OK) return st;
   if (!dtype_ok(x_dtype)) return MOE_ERR_INVALID_ARG;
   if (T == 0) return MOE_OK;
   if (!x || !Wg || !logits) return MOE_ERR_INVALID_ARG;
-  if (!aligned16(x)) return MOE_ERR_UNSUPPORTED;
-  const size_t need = router_logits_workspace_bytes(T, d, E);
+  if (!aligned16(x) || !aligned16(Wg_split)) return MOE_ERR_UNSUPPORTED;
+  const size_t need = router_logits_workspace_bytes(T, d, E, Wg_split != nullptr);
   if (need > 0 && (!workspace || workspace_bytes < need)) return MOE_ERR_WORKSPACE;
-  return launch_router_logits(x, x_dtype, Wg, logit_offset, T, d, E, logits, workspace, S(stream));
+  return launch_router_logits(x, x_dtype, Wg, Wg_split, logit_offset, T, d, E, logits, workspace, S(stream));
 }
 
 moe_status moe_route_fixed(const float* logits, int32_t T, int32_t E, int32_t k, int32_t score, int32_t renormalize,
@@ -209,6 +230,8 @@ moe_status moe_histogram_scan_noalloc(const int32_t* topk_idx, const float* topk
   moe_status st = check_dims(T, E, k);
   if (st != MOE_OK) return st;
   if (capacity < -1) return MOE_ERR_INVALID_ARG;
+  // sizes beyond the fixed scratch are refused before the pointers are even looked at
+  if (histogram_scan_workspace_bytes(T, k, E) > histogram_scan_noalloc_limit()) return MOE_ERR_WORKSPACE;
   if (!counts || !kept || !offsets) return MOE_ERR_INVALID_ARG;
   if (T > 0 && (!topk_idx || !topk_gate || !row_of || !token_of_row || !gate_of_row)) return MOE_ERR_INVALID_ARG;
   const long long rows_max = moe_rows_max(T, E, k, capacity);

@@ -5,6 +5,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "moe.h"
 
 namespace moe {
@@ -66,17 +68,51 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   return t;
 }
 
-inline int num_sms() {
-  static int cached[64] = {0};
+// Host-side per-device tables (kernel attributes raised once, symbol addresses looked up
+// once) are indexed by the CUDA device ordinal; ordinals from kMaxDevices up are not
+// supported.  Entries are atomics: several host threads may race to fill one, and since
+// every writer stores the same value the race is benign.
+constexpr int kMaxDevices = 64;
+
+// The current device's ordinal, or -1 when it cannot be read or has no table slot.
+inline int device_slot() {
   int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64) dev = 0;
-  if (!cached[dev]) {
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
+  return dev;
+}
+
+// Raises a kernel's dynamic shared-memory limit once per device (never inside a launch
+// sequence that may be captured into a CUDA graph after the first call on that device).
+template <typename Kernel>
+inline moe_status ensure_smem_limit(std::atomic<int> (&done)[kMaxDevices], Kernel kern, size_t bytes) {
+  const int dev = device_slot();
+  if (dev < 0) return MOE_ERR_UNSUPPORTED;
+  if (done[dev].load(std::memory_order_acquire)) return MOE_OK;
+  const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e != cudaSuccess) {
+    last_cuda_error_ref() = e;
+    return MOE_ERR_CUDA;
+  }
+  done[dev].store(1, std::memory_order_release);
+  return MOE_OK;
+}
+
+inline int num_sms() {
+  static std::atomic<int> cached[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+  if (dev < 0 || dev >= kMaxDevices) {
     int n = 0;
     cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    cached[dev] = n > 0 ? n : 148;
+    return n > 0 ? n : 148;
   }
-  return cached[dev];
+  int n = cached[dev].load(std::memory_order_relaxed);
+  if (!n) {
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+    cached[dev].store(n, std::memory_order_relaxed);
+  }
+  return n;
 }
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -99,14 +135,28 @@ inline moe_status cuda_status(cudaError_t e) {
 }
 
 // ---- launchers implemented in the kernel files (arguments already validated) ----
-moe_status launch_route(const void* x, int x_dtype, const float* Wg, const float* logit_offset,
-                        const float* select_bias, int T, int d, int E, int k, int score,
-                        int renormalize, float scale, float* logits, int32_t* topk_idx,
-                        float* topk_gate, void* ws, cudaStream_t s);
-size_t route_workspace_bytes(int T, int d, int E);
-moe_status launch_router_logits(const void* x, int x_dtype, const float* Wg, const float* logit_offset, int T,
-                                int d, int E, float* logits, void* ws, cudaStream_t s);
-size_t router_logits_workspace_bytes(int T, int d, int E);
+moe_status launch_route(const void* x, int x_dtype, const float* Wg, const void* Wg_split, const float* logit_offset,
+                        const float* select_bias, int T, int d, int E, int k, int score, int renormalize,
+                        float scale, float* logits, int32_t* topk_idx, float* topk_gate, void* ws, cudaStream_t s);
+size_t route_workspace_bytes(int T, int d, int E, bool prepared);
+moe_status launch_router_logits(const void* x, int x_dtype, const float* Wg, const void* Wg_split,
+                                const float* logit_offset, int T, int d, int E, float* logits, void* ws,
+                                cudaStream_t s);
+size_t router_logits_workspace_bytes(int T, int d, int E, bool prepared);
+
+// Tensor-core router (router_tc.cu): experts in n_tiles tiles of NE (a multiple of 32,
+// at most kRouterMaxNE) per GEMM tile.
+constexpr int kRouterMaxNE = 256;
+struct RouterGeom {
+  int NE, n_tiles;
+};
+RouterGeom router_geom(int E);
+size_t router_weight_bytes(int d, int E);          // prepared (split) weight; 0 = no tensor-core router
+bool tc_router_applies(int x_dtype, int T, int d, int E);
+moe_status launch_prepare_router_weight(const float* Wg, int d, int E, void* W3, cudaStream_t s);
+moe_status launch_router_tc(const void* x, int T, int d, int E, const void* W3, const float* logit_offset,
+                            float* logits, int fuse_k, const float* sel_bias, int score, int renorm, float scale,
+                            int32_t* topk_idx, float* topk_gate, cudaStream_t s);
 moe_status launch_route_fixed(const float* logits, int T, int E, int k, int score, int renormalize, float scale,
                               int rule, const int32_t* token_id, uint32_t seed, int32_t* topk_idx,
                               float* topk_gate, cudaStream_t s);
@@ -118,6 +168,7 @@ moe_status launch_histogram_scan(const int32_t* topk_idx, const float* topk_gate
                                  int32_t* offsets, int32_t* row_of, int32_t* token_of_row,
                                  float* gate_of_row, long long rows_max, void* ws, cudaStream_t s);
 size_t histogram_scan_workspace_bytes(int T, int k, int E);
+size_t histogram_scan_noalloc_limit();
 moe_status launch_histogram_scan_noalloc(const int32_t* topk_idx, const float* topk_gate, int T, int k, int E,
                                          int capacity, int32_t* counts, int32_t* kept, int32_t* offsets,
                                          int32_t* row_of, int32_t* token_of_row, float* gate_of_row,
@@ -159,9 +210,14 @@ moe_status launch_gate_up_gather_simt(const void* x, int dtype, const int32_t* t
                                       const void* W_gu, void* h, cudaStream_t s);
 moe_status launch_gate_up_gather_tc(const void* x, const int32_t* token_of_row, int T, const int32_t* offsets, int E,
                                     int d, int F, long long rows_max, const void* W_gu, void* h, cudaStream_t s);
-moe_status launch_router_logits_tc(const void* x, const int32_t* offs2, int T, int d, int E, const void* W3,
-                                   const float* logit_offset, float* logits, cudaStream_t s, int splits);
-int router_k_splits(int T, int d, int E);
+// Weight-major grouped GEMMs (ffn_wm.cu): tiles of 256 weight rows x the expert's tokens.
+moe_status launch_gate_up_wm(const void* x_rows, const int32_t* offsets, int E, int d, int F, long long rows_max,
+                             const void* W_gu, void* h, cudaStream_t s);
+moe_status launch_down_wm(const void* h, const int32_t* offsets, int E, int d, int F, long long rows_max,
+                          const void* W_dn, const float* gate_of_row, int y_dtype, void* y_rows, cudaStream_t s);
+// Whether a grouped GEMM over E experts and rows_max rows takes the weight-major tiles.
+bool prefer_weight_major(long long rows_max, int E);
+
 moe_status launch_gate_up_tc(const void* x_rows, const int32_t* offsets, int E, int d, int F,
                              long long rows_max, const void* W_gu, void* h, cudaStream_t s);
 moe_status launch_down_tc(const void* h, const int32_t* offsets, int E, int d, int F,

@@ -21,10 +21,6 @@
 //       token matrix, A row r = x[token_of_row[r]], so no permuted copy of x is written
 //       or read.  The producer warp copies them with 16-byte cp.async into the same
 //       128-byte-swizzled layout TMA writes; B still arrives by TMA.
-//   MODE 2 (router): A = x [T, d], B = the exact three-term bf16 split of W_g (hi, mid,
-//       lo rows per 64 experts); N = 192 MMAs; the epilogue sums the three terms and the
-//       logit offset in fp32.  Tiles walk n fastest (the split weight is small; each slice
-//       of x is read once).
 //
 // Per CTA (1 per SM, 192 threads):
 //   warp 0   TMA producer: 128x64 A tile + 256x64 B tile per stage (128-byte swizzle),
@@ -42,20 +38,22 @@
 // MMAs; it is used when groups average at least 256 rows.  No load uses cluster
 // multicast.
 #include <cuda.h>
+#include <stdlib.h>
+#include <string.h>
 
 #include "common.cuh"
+#include "tc_prims.cuh"
 #include "tile_sched.cuh"
 
 namespace moe {
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4, UMMA_K = 16;
+constexpr int BM = 128, BN = 256, STAGES = 4;
 constexpr int kThreadsTC = 192;
 constexpr int A_STAGE = BM * BK * 2;   // 16 KB
 constexpr int B_STAGE = BN * BK * 2;   // 32 KB
 constexpr int kMaxE = 1024;
 constexpr uint32_t kTmemCols = 512;
-constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s per barrier wait
 
 struct L {
   static constexpr int a = 0;
@@ -69,80 +67,6 @@ struct L {
   static constexpr int end = stage + 4 * 32 * (32 * 4 + 16);
 };
 constexpr size_t kSmemBytes = L::end + 1024;                 // + alignment slack
-
-// instruction descriptor: D fp32, A bf16, B bf16, both K-major, N = n, M = m
-constexpr uint32_t make_idesc(int m, int n) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
-}
-// MMA width per mode: the router tile (MODE 2) holds three 64-column terms (hi, mid, lo)
-// of the split weight, so it issues N = 192; every other mode N = 256 (= BN).
-constexpr int kRouterN = 192;
-template <int MODE>
-constexpr int mma_n() { return MODE == 2 ? kRouterN : BN; }
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void fence_mbar_init() {
-  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}\n"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Bounded wait.  Returns false when the limit passes (records the error, raises the
-// CTA's abort flag) or when another role has already aborted.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* err) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 63u) == 0u) {
-      if (*abort_flag) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
-        record_error(err, MOE_DEVERR_PIPE_TIMEOUT);
-        *abort_flag = 1;
-        return false;
-      }
-    }
-  }
-}
-// Bounded wait that ignores the abort flag (used to drain in-flight work on exit).
-__device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity, int* err) {
-  const uint64_t t0 = global_timer_ns();
-  for (uint32_t i = 0;; ++i) {
-    if (mbar_try_wait(bar, parity)) return;
-    if ((i & 63u) == 63u && global_timer_ns() - t0 > kWaitLimitNs) {
-      record_error(err, MOE_DEVERR_PIPE_TIMEOUT);
-      return;
-    }
-  }
-}
-
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
-      : "memory");
-}
 
 // 16-byte cp.async global -> shared; src_bytes = 0 writes zeros without reading.
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
@@ -160,177 +84,11 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 __device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 // Output column tiles per row tile: 128 H features per gate/up tile (128 gate + 128 up
-// accumulator columns), 256 outputs per down tile, 64 experts per router tile.  The
-// router (MODE 2, CTA-pair kernel) may also split K: F then carries the number of K
-// splits S, and its n-tile index is expert tile * S + split.
+// accumulator columns), 256 outputs per down tile.
 template <int MODE>
 __host__ __device__ __forceinline__ int n_tiles_of(int F, int N_out) {
   if (MODE == 0 || MODE == 4) return (F + 127) / 128;
-  if (MODE == 1 || MODE == 3) return (N_out + BN - 1) / BN;
-  return ((N_out + 63) / 64) * (F > 1 ? F : 1);
-}
-
-// The k-blocks [kb0, kb1) of one tile.  Router tiles (MODE 2) with S = F > 1 splits take
-// the split-th of S equal runs of ceil(KB / S) k-blocks; the host keeps KB >= 4 S, so no
-// run is empty.  Every other tile runs all KB k-blocks.
-struct KSplit {
-  int n_tile, split, kb0, kb1;
-};
-template <int MODE>
-__device__ __forceinline__ KSplit k_split(int n_tile, int F, int KB) {
-  KSplit k{n_tile, 0, 0, KB};
-  if (MODE == 2 && F > 1) {
-    const int per = (KB + F - 1) / F;
-    k.n_tile = n_tile / F;
-    k.split = n_tile - k.n_tile * F;
-    k.kb0 = k.split * per;
-    k.kb1 = min(KB, k.kb0 + per);
-  }
-  return k;
-}
-
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                          uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-__device__ __forceinline__ void umma_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
-}
-
-// ---- CTA-pair (cta_group::2) forms: an M=256 MMA issued by the pair's even CTA over
-// both CTAs' shared memory, accumulating into both CTAs' TMEM ----
-
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-// The same shared-memory object in CTA `rank` of the cluster (shared::cluster address).
-__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
-  return r;
-}
-__device__ __forceinline__ void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
-}
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
-}
-// TMA load into this CTA's shared memory whose completion is counted on an mbarrier that
-// may live in the peer CTA (the pair's even CTA); no multicast.
-__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar_cluster, int x,
-                                                 int y) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
-      "[%4];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar_cluster)
-      : "memory");
-}
-__device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                               uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-// Completion of the pair's MMAs arrives on the barrier at this offset in both CTAs.
-__device__ __forceinline__ void umma_commit_pair_both(uint32_t bar) {
-  const uint16_t both = 0x3;
-  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
-               ::"r"(bar), "h"(both)
-               : "memory");
-}
-__device__ __forceinline__ void umma_commit_pair(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
-}
-
-// K-major operand in the canonical 128-byte-swizzle layout written by TMA:
-// rows of 128 bytes (64 bf16), 8-row atoms of 1024 bytes stacked densely.
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
-  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);   // start address >> 4
-  d |= (uint64_t)1 << 16;                            // leading byte offset (unused when swizzled)
-  d |= (uint64_t)(1024 >> 4) << 32;                  // stride byte offset: one 8-row atom
-  d |= (uint64_t)1 << 46;                            // descriptor version for sm_100
-  d |= (uint64_t)2 << 61;                            // 128-byte swizzle
-  return d;
-}
-
-#define MOE_R32(r) \
-  "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), \
-  "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), \
-  "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), \
-  "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-#define MOE_RW32(r) \
-  "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]), \
-  "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), \
-  "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), \
-  "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
-
-// 32 consecutive fp32 accumulator columns of this thread's TMEM lane.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-      : MOE_R32(r)
-      : "r"(taddr));
-}
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-// Ties the loaded registers to the preceding wait so no use is scheduled above it.
-__device__ __forceinline__ void tmem_regs_ready(uint32_t (&r)[32]) { asm volatile("" : MOE_RW32(r)); }
-
-// Epilogue staging: each epilogue warp turns its 32 rows x 32 columns (one value per
-// lane-row from tcgen05.ld) around in shared memory, so that every global store
-// instruction writes whole 128-byte lines of 4 (fp32) or 8 (bf16) rows instead of 32
-// half-filled sectors.  Row pitch padded by 16 bytes: conflict-free 16-byte accesses.
-constexpr int kStagePitchF32 = 32 * 4 + 16;
-constexpr int kStagePitchB16 = 32 * 2 + 16;
-constexpr int kStageWarpBytes = 32 * kStagePitchF32;
-
-template <typename OutT>
-__device__ __forceinline__ void stage_store32(uint8_t* stage, const float (&v)[32], int lane, OutT* out,
-                                              long long row0, int rows_valid, long long ld, int col, int ncols) {
-  if constexpr (sizeof(OutT) == 4) {
-    float4* dst = reinterpret_cast<float4*>(stage + lane * kStagePitchF32);
-#pragma unroll
-    for (int q = 0; q < 8; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-    __syncwarp();
-    const int rs = lane >> 3, cv = lane & 7;       // 4 rows per pass, 8 x 16 B per row
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int r = i * 4 + rs;
-      const float4 x = *reinterpret_cast<const float4*>(stage + r * kStagePitchF32 + cv * 16);
-      if (r < rows_valid && col + cv * 4 + 4 <= ncols)
-        *reinterpret_cast<float4*>(out + (row0 + r) * ld + col + cv * 4) = x;
-    }
-  } else {
-    uint4* dst = reinterpret_cast<uint4*>(stage + lane * kStagePitchB16);
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-      dst[q] = make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
-                          pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
-    __syncwarp();
-    const int rs = lane >> 2, cv = lane & 3;       // 8 rows per pass, 4 x 16 B per row
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int r = i * 8 + rs;
-      const uint4 x = *reinterpret_cast<const uint4*>(stage + r * kStagePitchB16 + cv * 16);
-      if (r < rows_valid && col + cv * 8 + 8 <= ncols)
-        *reinterpret_cast<uint4*>(out + (row0 + r) * ld + col + cv * 8) = x;
-    }
-  }
-  __syncwarp();
+  return (N_out + BN - 1) / BN;
 }
 
 // L2 policy that keeps lines resident ahead of streaming data (the fp32 output rows the
@@ -374,8 +132,6 @@ __device__ __forceinline__ void stage_red32(uint8_t* stage, const float (&v)[32]
 // .sync.aligned); rows past wrows are read but not stored.
 //   MODE 0: columns [0,128) gate, [128,256) up -> H = silu(g) * u for features n_tile*128 + ...
 //   MODE 1: 256 columns -> gate_of_row[row] * acc for outputs n_tile*256 + ...
-//   MODE 2: [0,64) x.hi, [64,128) x.mid, [128,192) x.lo of experts n_tile*64 + ... ->
-//           logit = (hi + mid) + lo + offset (gate_of_row carries the logit offset)
 // MODE 1 / 3 process the 32-column chunks [c_begin, c_end) of the 256 (a warp may own half).
 template <int MODE, typename OutT>
 __device__ __forceinline__ void epilogue_tile(uint32_t taddr, uint8_t* stage, int lane, long long wrow0, int wrows,
@@ -425,7 +181,8 @@ __device__ __forceinline__ void epilogue_tile(uint32_t taddr, uint8_t* stage, in
       }
       stage_store32<OutT>(stage, h, lane, out, wrow0, wrows, F, f0 + c * 32, F);
     }
-  } else if constexpr (MODE == 1) {
+  } else {
+    static_assert(MODE == 1, "grouped GEMM modes: 0 gate/up, 1 down, 3 down + combine, 4 gathered gate/up");
     const int n0 = n_tile * BN;
     const float gs = (lane < wrows && gate_of_row) ? __ldg(gate_of_row + wrow0 + lane) : 1.f;
 #pragma unroll 1
@@ -438,27 +195,6 @@ __device__ __forceinline__ void epilogue_tile(uint32_t taddr, uint8_t* stage, in
 #pragma unroll
       for (int i = 0; i < 32; ++i) y[i] = __uint_as_float(v32[i]) * gs;
       stage_store32<OutT>(stage, y, lane, out, wrow0, wrows, N_out, n0 + c * 32, N_out);
-    }
-  } else {
-    const int e0 = n_tile * 64;
-#pragma unroll 1
-    for (int c = 0; c < 2; ++c) {
-      uint32_t a[32], b[32], l3[32];
-      tmem_ld32(taddr + c * 32, a);
-      tmem_ld32(taddr + 64 + c * 32, b);
-      tmem_ld32(taddr + 128 + c * 32, l3);
-      tmem_wait_ld();
-      tmem_regs_ready(a);
-      tmem_regs_ready(b);
-      tmem_regs_ready(l3);
-      float lv[32];
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const int e = e0 + c * 32 + i;
-        const float off = (gate_of_row && e < N_out) ? __ldg(gate_of_row + e) : 0.f;
-        lv[i] = ((__uint_as_float(a[i]) + __uint_as_float(b[i])) + __uint_as_float(l3[i])) + off;
-      }
-      stage_store32<OutT>(stage, lv, lane, out, wrow0, wrows, N_out, e0 + c * 32, N_out);
     }
   }
 }
@@ -605,11 +341,11 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
       for (int s = 0; s < STAGES; ++s) last_phase[s] = -1;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
-        const TileCoord tc = tile_coord(tile_start, offsets, E, BM, tile, MODE == 2 ? n_tiles : 0);
+        const TileCoord tc = tile_coord(tile_start, offsets, E, BM, tile);
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1u, abort_flag, err)) { ok = false; break; }
           const uint32_t full = bar_full + 8 * stage;
-          mbar_expect_tx(full, A_STAGE + mma_n<MODE>() * BK * 2);
+          mbar_expect_tx(full, A_STAGE + B_STAGE);
           const uint32_t a_dst = sb + L::a + stage * A_STAGE;
           const uint32_t b_dst = sb + L::b + stage * B_STAGE;
           tma_load_2d(a_dst, &tmA, full, kb * BK, tc.row0);
@@ -617,10 +353,8 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
             const int g_row = tc.e * 2 * F + tc.n_tile * 128;
             tma_load_2d(b_dst, &tmB, full, kb * BK, g_row);
             tma_load_2d(b_dst + B_STAGE / 2, &tmB, full, kb * BK, g_row + F);
-          } else if (MODE == 1 || MODE == 3) {
-            tma_load_2d(b_dst, &tmB, full, kb * BK, tc.e * N_out + tc.n_tile * BN);
           } else {
-            tma_load_2d(b_dst, &tmB, full, kb * BK, tc.n_tile * BN);   // router: rows hi, mid, lo of the tile
+            tma_load_2d(b_dst, &tmB, full, kb * BK, tc.e * N_out + tc.n_tile * BN);
           }
           last_phase[stage] = (int)phase;
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -653,7 +387,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
           const uint64_t bdesc = sw128_desc(sb + L::b + stage * B_STAGE);
 #pragma unroll
           for (int kk = 0; kk < BK / UMMA_K; ++kk)   // +32 bytes along K per step (>> 4 = 2)
-            umma_bf16(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, make_idesc(BM, mma_n<MODE>()),
+            umma_bf16(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, make_idesc(BM, BN),
                       (kb | kk) != 0 ? 1u : 0u);
           umma_commit(bar_empty + 8 * stage);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -672,7 +406,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
     uint8_t* stage = smem + L::stage + (warp - 2) * kStageWarpBytes;
     int it = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
-      const TileCoord tc = tile_coord(tile_start, offsets, E, BM, tile, MODE == 2 ? n_tiles : 0);
+      const TileCoord tc = tile_coord(tile_start, offsets, E, BM, tile);
       const int acc = it & 1;
       const uint32_t acc_phase = (uint32_t)(it >> 1) & 1u;
       const bool got = mbar_wait(bar_tfull + 8 * acc, acc_phase, abort_flag, err);
@@ -801,16 +535,14 @@ grouped_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
       for (int s = 0; s < C::stages; ++s) last_phase[s] = -1;
       bool ok = true;
       for (int tile = cid; ok && tile < total; tile += ncl) {
-        const TileCoord tc = tile_coord(tile_start, offsets, E, PM, tile, MODE == 2 ? n_tiles : 0);
-        const KSplit ks = k_split<MODE>(tc.n_tile, F, KB);
+        const TileCoord tc = tile_coord(tile_start, offsets, E, PM, tile);
         const int a_row = tc.row0 + (int)rank * BM;
         int b_row;
         if (MODE == 0) b_row = tc.e * 2 * F + (rank ? F : 0) + tc.n_tile * 128;   // even: gate, odd: up
-        else if (MODE == 1 || MODE == 3) b_row = tc.e * N_out + tc.n_tile * BN + (int)rank * BM;
-        else b_row = ks.n_tile * BN + (int)rank * (kRouterN / 2);   // router: half of hi, mid, lo
-        for (int kb = ks.kb0; kb < ks.kb1; ++kb) {
+        else b_row = tc.e * N_out + tc.n_tile * BN + (int)rank * BM;
+        for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1u, abort_flag, err)) { ok = false; break; }
-          if (rank == 0) mbar_expect_tx(bar_full + 8 * stage, 2 * (A_STAGE + (mma_n<MODE>() / 2) * BK * 2));
+          if (rank == 0) mbar_expect_tx(bar_full + 8 * stage, 2 * (A_STAGE + B2_STAGE));
           const uint32_t full_c = map_to_rank(bar_full + 8 * stage, 0);
           tma_load_2d_pair(sb + C::a + stage * A_STAGE, &tmA, full_c, kb * BK, a_row);
           tma_load_2d_pair(sb + C::b + stage * B2_STAGE, &tmB, full_c, kb * BK, b_row);
@@ -836,18 +568,14 @@ grouped_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
         if (!mbar_wait(bar_tempty + 8 * acc, acc_phase ^ 1u, abort_flag, err)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-        int n_tile_of_tile = 0;
-        if (MODE == 2) n_tile_of_tile = tile_coord(tile_start, offsets, E, PM, tile, n_tiles).n_tile;
-        const KSplit ks = k_split<MODE>(n_tile_of_tile, F, KB);
-        for (int kb = ks.kb0; kb < ks.kb1; ++kb) {
+        for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag, err)) { ok = false; break; }
           tc_fence_after();
           const uint64_t adesc = sw128_desc(sb + C::a + stage * A_STAGE);
           const uint64_t bdesc = sw128_desc(sb + C::b + stage * B2_STAGE);
 #pragma unroll
           for (int kk = 0; kk < BK / UMMA_K; ++kk)
-            umma_bf16_pair(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, make_idesc(2 * BM, mma_n<MODE>()),
-                           (kb != ks.kb0 || kk != 0) ? 1u : 0u);
+            umma_bf16_pair(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, make_idesc(2 * BM, BN), (kb | kk) != 0 ? 1u : 0u);
           umma_commit_pair_both(bar_empty + 8 * stage);
           if (++stage == C::stages) { stage = 0; phase ^= 1u; }
         }
@@ -866,7 +594,7 @@ grouped_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
     uint8_t* stage = smem + C::stage + ew * kStageWarpBytes;
     int it = 0;
     for (int tile = cid; tile < total; tile += ncl, ++it) {
-      const TileCoord tc = tile_coord(tile_start, offsets, E, PM, tile, MODE == 2 ? n_tiles : 0);
+      const TileCoord tc = tile_coord(tile_start, offsets, E, PM, tile);
       const int acc = it & 1;
       const uint32_t acc_phase = (uint32_t)(it >> 1) & 1u;
       const bool got = mbar_wait(bar_tfull + 8 * acc, acc_phase, abort_flag, err);
@@ -877,11 +605,8 @@ grouped_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
       const int cta_rows = min(BM, max(0, tc.rows - (int)rank * BM));
       const long long wrow0 = (long long)tc.row0 + (int)rank * BM + q * 32;
       const int wrows = min(32, max(0, cta_rows - q * 32));
-      const KSplit ks = k_split<MODE>(tc.n_tile, F, KB);
-      // a K split of the router writes its partial logits to plane `split` of [S, rows, E]
-      OutT* o = MODE == 2 ? out + (long long)ks.split * rows_max * N_out : out;
-      epilogue_tile<MODE, OutT>(taddr, stage, lane, wrow0, wrows, MODE == 2 ? ks.n_tile : tc.n_tile, F, N_out,
-                                gate_of_row, o, token_of_row, n_tokens, err, c_begin, c_end);
+      epilogue_tile<MODE, OutT>(taddr, stage, lane, wrow0, wrows, tc.n_tile, F, N_out, gate_of_row, out,
+                                token_of_row, n_tokens, err, c_begin, c_end);
       tc_fence_before();
       mbar_arrive_cluster(map_to_rank(bar_tempty + 8 * acc, 0));
     }
@@ -895,53 +620,14 @@ grouped_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
   }
 }
 
-// ---------------------------------------------------------------- host side
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
-  return fn;
-}
-
-// 2D bf16 tensor [rows, cols] row-major; box = box_rows x 64 columns, 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* ptr, unsigned long long rows, unsigned long long cols, unsigned box_rows) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-  cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int MODE, typename OutT>
 moe_status launch_tc(const CUtensorMap& ma, const CUtensorMap& mb, const int32_t* offsets, int E, int K, int N_out,
                      int F, long long rows_max, const float* gate_of_row, void* out, cudaStream_t s,
                      const int32_t* token_of_row = nullptr, int n_tokens = 0,
                      const __nv_bfloat16* a_gather = nullptr) {
-  static int configured[64] = {0};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64) dev = 0;
-  if (!configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_tc_kernel<MODE, OutT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kSmemBytes);
-    if (e != cudaSuccess) return cuda_status(e);
-    configured[dev] = 1;
-  }
+  static std::atomic<int> configured[kMaxDevices];
+  const moe_status st = ensure_smem_limit(configured, grouped_gemm_tc_kernel<MODE, OutT>, kSmemBytes);
+  if (st != MOE_OK) return st;
   const int n_tiles = n_tiles_of<MODE>(F, N_out);
   const long long max_tiles = ((rows_max + BM - 1) / BM + E) * (long long)n_tiles;
   int grid = num_sms();
@@ -956,8 +642,6 @@ moe_status launch_tc(const CUtensorMap& ma, const CUtensorMap& mb, const int32_t
 }  // namespace
 
 // Returns MOE_ERR_UNSUPPORTED when a tensor map cannot be encoded (caller falls back).
-// Router logits on the tensor cores: A = x [T, d] bf16 (one group, offs2 = {0, T}),
-// B = the split weight W3 [ceil(E/64) * 256, d]; writes logits [T, E] fp32 (+ offset).
 // CTA pairs pay off when groups average at least one full 256-row pair tile; smaller
 // groups keep the single-CTA kernel (less padding in ragged groups).
 // Down GEMMs with K = F up to this use the eight-epilogue-warp pair configuration.
@@ -968,16 +652,10 @@ template <int MODE, typename OutT, bool WIDE = false>
 moe_status launch_tc2(const CUtensorMap& ma, const CUtensorMap& mb, const int32_t* offsets, int E, int K, int N_out,
                       int F, long long rows_max, const float* gate_of_row, void* out, cudaStream_t s,
                       const int32_t* token_of_row = nullptr, int n_tokens = 0) {
-  static int configured[64] = {0};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  dev &= 63;
-  if (!configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_tc2_kernel<MODE, OutT, WIDE>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PairCfg<WIDE>::smem);
-    if (e != cudaSuccess) return cuda_status(e);
-    configured[dev] = 1;
-  }
+  static std::atomic<int> configured[kMaxDevices];
+  const moe_status st =
+      ensure_smem_limit(configured, grouped_gemm_tc2_kernel<MODE, OutT, WIDE>, PairCfg<WIDE>::smem);
+  if (st != MOE_OK) return st;
   const int n_tiles = n_tiles_of<MODE>(F, N_out);
   const long long max_tiles = ((rows_max + 2 * BM - 1) / (2 * BM) + E) * (long long)n_tiles;
   int pairs = num_sms() / 2;
@@ -1000,39 +678,29 @@ moe_status launch_tc2(const CUtensorMap& ma, const CUtensorMap& mb, const int32_
                                         err_ptr()));
 }
 
-// K splits for the router GEMM: when its pair tiles would leave CTA pairs idle, split K
-// into S equal runs (S a power of two, at most 8, each run at least 4 k-blocks) so that
-// up to one tile per pair is in flight.  The partial logits then go to S planes and the
-// top-k kernel adds them in plane order (and the offset).  1 for the single-CTA kernel.
-int router_k_splits(int T, int d, int E) {
-  if (T <= 0 || E <= 0 || d < BK || !use_pairs(T, 1)) return 1;
-  const long long tiles = (long long)((T + 2 * BM - 1) / (2 * BM)) * ((E + 63) / 64);
-  const int KB = (d + BK - 1) / BK;
-  const int pairs = num_sms() / 2;
-  int S = 1;
-  while (S < 8 && tiles * 2 * S <= pairs && KB >= 4 * 2 * S) S *= 2;
-  return S;
-}
+// Token-major tiles (this file) pay off when the groups are large: a 256-row tile is then
+// full.  When the groups average under kWeightMajorBelow rows -- many experts, or a cap
+// that keeps few rows each -- skew leaves most experts with a few dozen rows, and the
+// weight-major tiles (ffn_wm.cu), whose token side is the group rounded up to 32, waste
+// far less tensor work.  MOE_B200_EXPERT_TILES=tokens|weights overrides the choice (for
+// measuring one against the other).
+constexpr long long kWeightMajorBelow = 1024;
 
-moe_status launch_router_logits_tc(const void* x, const int32_t* offs2, int T, int d, int E, const void* W3,
-                                   const float* logit_offset, float* logits, cudaStream_t s, int splits) {
-  if (T == 0) return MOE_OK;
-  if (d < BK || d % 8 != 0 || E % 4 != 0) return MOE_ERR_UNSUPPORTED;
-  const int nt = (E + 63) / 64;
-  const bool pair = use_pairs(T, 1);
-  if (splits < 1 || (splits > 1 && (!pair || (d + BK - 1) / BK < 4 * splits))) return MOE_ERR_INVALID_ARG;
-  CUtensorMap ma, mb;
-  if (!make_map(&ma, x, (unsigned long long)T, d, BM)) return MOE_ERR_UNSUPPORTED;
-  // boxes cover the hi, mid and lo rows of a 256-row tile (the pad rows are never loaded)
-  if (!make_map(&mb, W3, (unsigned long long)nt * 256, d, pair ? kRouterN / 2 : kRouterN)) return MOE_ERR_UNSUPPORTED;
-  if (pair) return launch_tc2<2, float>(ma, mb, offs2, 1, d, E, splits, T, logit_offset, logits, s);
-  return launch_tc<2, float>(ma, mb, offs2, 1, d, E, 0, T, logit_offset, logits, s);
+bool prefer_weight_major(long long rows_max, int E) {
+  const char* v = getenv("MOE_B200_EXPERT_TILES");      // read per call: a host-side string lookup
+  if (v && strcmp(v, "tokens") == 0) return false;
+  if (v && strcmp(v, "weights") == 0) return true;
+  return E > 0 && rows_max / E < kWeightMajorBelow;
 }
 
 moe_status launch_gate_up_tc(const void* x_rows, const int32_t* offsets, int E, int d, int F, long long rows_max,
                              const void* W_gu, void* h, cudaStream_t s) {
   if (rows_max == 0) return MOE_OK;
   if (d < BK || F < 8) return MOE_ERR_UNSUPPORTED;
+  if (prefer_weight_major(rows_max, E)) {
+    const moe_status st = launch_gate_up_wm(x_rows, offsets, E, d, F, rows_max, W_gu, h, s);
+    if (st != MOE_ERR_UNSUPPORTED) return st;
+  }
   CUtensorMap ma, mb;
   if (!make_map(&ma, x_rows, (unsigned long long)rows_max, d, BM)) return MOE_ERR_UNSUPPORTED;
   if (!make_map(&mb, W_gu, (unsigned long long)E * 2 * F, d, 128)) return MOE_ERR_UNSUPPORTED;
@@ -1045,6 +713,10 @@ moe_status launch_down_tc(const void* h, const int32_t* offsets, int E, int d, i
                           const void* W_dn, const float* gate_of_row, int y_dtype, void* y_rows, cudaStream_t s) {
   if (rows_max == 0) return MOE_OK;
   if (F < BK || d < 8) return MOE_ERR_UNSUPPORTED;
+  if (prefer_weight_major(rows_max, E)) {
+    const moe_status st = launch_down_wm(h, offsets, E, d, F, rows_max, W_dn, gate_of_row, y_dtype, y_rows, s);
+    if (st != MOE_ERR_UNSUPPORTED) return st;
+  }
   const bool pair = use_pairs(rows_max, E);
   CUtensorMap ma, mb;
   if (!make_map(&ma, h, (unsigned long long)rows_max, F, BM)) return MOE_ERR_UNSUPPORTED;

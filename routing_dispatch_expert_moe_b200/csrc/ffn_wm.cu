@@ -1,0 +1,347 @@
+// Weight-major grouped expert GEMMs on the 5th-generation tensor cores (sm_100a): the
+// expert's weight rows are the MMA's M side and the expert's tokens its N side.
+//
+// Expert FFN: "Hugging Face 图解 Mixture of Experts（MoE）原理、训练与推理权衡", section
+// "什么是混合专家模型" (each expert is an FFN) and section "更多关于高效训练的内容"
+// (experts receive uneven numbers of tokens; handle them without padding or drops).
+//
+// Why a second orientation.  The token-major kernels (ffn_tc.cu) give a CTA pair 256
+// token rows of one expert; an expert with 41 rows still costs a 256-row tile of tensor
+// work.  With many experts and skewed loads (most experts hold a few dozen rows, a few
+// hold hundreds) that padding, not the weights, sets the time.  Here a tile is 256 output
+// features (weight rows, 128 per CTA) x N tokens, N = the expert's rows rounded up to 32
+// (at most NT): a 41-row expert pads to 64 columns.  Each tile streams its weight slab
+// once; the token blocks of one weight slab are consecutive tiles, so CTAs running at the
+// same time share the slab through L2.
+//
+//   MODE 0 (gate/up): A = W_gate[e] and W_up[e] rows f0 .. f0+255 (two M=256 MMAs per k
+//       step into two accumulators, g in columns [0, 128), u in [128, 256)), B = N <= 128
+//       rows of x_perm; the epilogue writes H[token][f] = silu(g) * u as bf16.
+//   MODE 1 (down):    A = W_dn[e] rows n0 .. n0+255, B = N <= 256 rows of H; the epilogue
+//       writes gate_of_row[token] * acc to the gated rows (bf16 or fp32).
+//
+// CTA pairs (cta_group::2): each CTA stages 128 weight rows and N/2 token rows per
+// 64-wide k-block (TMA, 128-byte swizzle); the even CTA issues the MMAs; the accumulator
+// rows (features) of each CTA land in its own TMEM.  Epilogue: a thread owns one feature
+// (its TMEM lane) for 32 tokens per tcgen05.ld; a shared-memory turn-around writes whole
+// 128-byte lines of token rows.  Two accumulators of 256 columns let the epilogue of one
+// tile overlap the next tile's mainloop.  Every wait is bounded (MOE_DEVERR_PIPE_TIMEOUT,
+// then an orderly exit).  No load uses cluster multicast.
+#include "common.cuh"
+#include "tc_prims.cuh"
+#include "tile_sched.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kWMaxE = 1024;
+constexpr uint32_t kWTmemCols = 512;
+constexpr int kWRows = 128;                     // weight rows per CTA (256 per pair)
+constexpr int kWBlock = kWRows * BK * 2;       // 16 KB: one 128-row operand block
+
+template <int MODE>
+struct WmCfg {
+  static constexpr int NT = MODE == 0 ? 128 : 256;            // tokens per tile (MMA N at most)
+  static constexpr int a_blocks = MODE == 0 ? 2 : 1;           // gate + up, or down
+  static constexpr int b_bytes = (NT / 2) * BK * 2;            // this CTA's token rows per stage
+  static constexpr int stage_bytes = a_blocks * kWBlock + b_bytes;
+  static constexpr int stages = MODE == 0 ? 5 : 6;
+  static constexpr int epi_warps = 4;
+  static constexpr int threads = 64 + 32 * epi_warps;
+  static constexpr int bars = stages * stage_bytes;
+  static constexpr int nbars = 2 * stages + 4 + 1;
+  static constexpr int misc = bars + nbars * 8;
+  static constexpr int tiles = misc + 16;
+  static constexpr int sh32 = tiles + (kWMaxE + 1) * 4;
+  static constexpr int stage = (sh32 + 32 * 4 + 127) / 128 * 128;
+  static constexpr int end = stage + epi_warps * kStageWarpBytes;
+  static constexpr size_t smem = end + 1024;
+  static_assert(smem <= 232448, "shared memory per CTA");
+  static_assert(stage_bytes % 1024 == 0, "stages must keep the 1024-byte swizzle alignment");
+};
+
+// Output feature tiles (256 per pair) per token block.
+template <int MODE>
+__host__ __device__ __forceinline__ int wm_m_tiles(int F, int d) {
+  return MODE == 0 ? (F + 255) / 256 : (d + 255) / 256;
+}
+
+// MMA width for a tile of `rows` tokens: rows rounded up to 32, at most NT.
+template <int MODE>
+__device__ __forceinline__ int wm_n(int rows) {
+  const int n = (rows + 31) / 32 * 32;
+  return n < WmCfg<MODE>::NT ? n : WmCfg<MODE>::NT;
+}
+
+// The turn-around of the weight-major epilogue: thread `lane` holds output column col +
+// lane for the 32 tokens row0 .. row0+31 (v[i] = token i).  It writes them as column lane
+// of a 32 x 32 tile in shared memory, then the warp stores whole token rows (16 bytes per
+// lane: 8 bf16 or 4 fp32 columns) -- rows past rows_valid and columns past ncols skipped.
+template <typename OutT>
+__device__ __forceinline__ void stage_store32_t(uint8_t* stage, const float (&v)[32], int lane, OutT* out,
+                                                long long row0, int rows_valid, long long ld, int col, int ncols) {
+  if constexpr (sizeof(OutT) == 4) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) *reinterpret_cast<float*>(stage + i * kStagePitchF32 + lane * 4) = v[i];
+    __syncwarp();
+    const int rs = lane >> 3, cv = lane & 7;       // 4 rows per pass, 8 x 16 B per row
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int r = i * 4 + rs;
+      const float4 x = *reinterpret_cast<const float4*>(stage + r * kStagePitchF32 + cv * 16);
+      if (r < rows_valid && col + cv * 4 + 4 <= ncols)
+        *reinterpret_cast<float4*>(out + (row0 + r) * ld + col + cv * 4) = x;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      *reinterpret_cast<__nv_bfloat16*>(stage + i * kStagePitchB16 + lane * 2) = __float2bfloat16_rn(v[i]);
+    __syncwarp();
+    const int rs = lane >> 2, cv = lane & 3;       // 8 rows per pass, 4 x 16 B per row
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = i * 8 + rs;
+      const uint4 x = *reinterpret_cast<const uint4*>(stage + r * kStagePitchB16 + cv * 16);
+      if (r < rows_valid && col + cv * 8 + 8 <= ncols)
+        *reinterpret_cast<uint4*>(out + (row0 + r) * ld + col + cv * 8) = x;
+    }
+  }
+  __syncwarp();
+}
+
+template <int MODE, typename OutT>
+__global__ void __launch_bounds__(WmCfg<MODE>::threads, 1)
+grouped_gemm_wm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                       const int32_t* __restrict__ offsets, int E, int K, int d, int F, long long rows_max,
+                       const float* __restrict__ gate_of_row, OutT* __restrict__ out, int* err) {
+  using C = WmCfg<MODE>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int* tile_start = reinterpret_cast<int*>(smem + C::tiles);
+  int* sh32 = reinterpret_cast<int*>(smem + C::sh32);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::misc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::misc + 4);
+  const uint32_t rank = cluster_ctarank();
+  const int cid = (int)(blockIdx.x >> 1), ncl = (int)(gridDim.x >> 1);
+
+  const int m_tiles = wm_m_tiles<MODE>(F, d);
+  build_tile_starts(offsets, E, C::NT, m_tiles, rows_max, tile_start, sh32, err);
+  const int total = tile_start[E];
+  if (cid >= total) return;   // both CTAs of the pair see the same cid: uniform, nothing allocated
+
+  const uint32_t bar_full = sb + C::bars;
+  const uint32_t bar_empty = bar_full + 8 * C::stages;
+  const uint32_t bar_tfull = bar_empty + 8 * C::stages;
+  const uint32_t bar_tempty = bar_tfull + 16;
+  const uint32_t bar_fin = bar_tempty + 16;
+  auto a_blk = [&](int s, int a) { return sb + (uint32_t)(s * C::stage_bytes + a * kWBlock); };
+  auto b_blk = [&](int s) { return sb + (uint32_t)(s * C::stage_bytes + C::a_blocks * kWBlock); };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::stages; ++s) {
+      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_empty + 8 * s, 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(bar_tfull + 8 * a, 1);
+      mbar_init(bar_tempty + 8 * a, 2 * 32 * C::epi_warps);
+    }
+    mbar_init(bar_fin, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(kWTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int KB = (K + BK - 1) / BK;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer (both CTAs)
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int last_phase[C::stages];
+#pragma unroll
+      for (int s = 0; s < C::stages; ++s) last_phase[s] = -1;
+      bool ok = true;
+      for (int tile = cid; ok && tile < total; tile += ncl) {
+        const TileCoord tc = tile_coord(tile_start, offsets, E, C::NT, tile);
+        const int n = wm_n<MODE>(tc.rows);
+        // this CTA's weight rows, and its half of the tile's tokens (columns [rank n/2, ...))
+        const int w_row = MODE == 0 ? tc.e * 2 * F + tc.n_tile * 256 + (int)rank * kWRows
+                                    : tc.e * d + tc.n_tile * 256 + (int)rank * kWRows;
+        const int x_row = tc.row0 + (int)rank * (n / 2);
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1u, abort_flag, err)) { ok = false; break; }
+          if (rank == 0) mbar_expect_tx(bar_full + 8 * stage, 2u * (uint32_t)C::stage_bytes);
+          const uint32_t full_c = map_to_rank(bar_full + 8 * stage, 0);
+          tma_load_2d_pair(a_blk(stage, 0), &tmW, full_c, kb * BK, w_row);
+          if (MODE == 0) tma_load_2d_pair(a_blk(stage, 1), &tmW, full_c, kb * BK, w_row + F);
+          tma_load_2d_pair(b_blk(stage), &tmX, full_c, kb * BK, x_row);
+          last_phase[stage] = (int)phase;
+          if (++stage == C::stages) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok && rank == 0) {
+        for (int s = 0; s < C::stages; ++s)
+          if (last_phase[s] >= 0) mbar_wait_drain(bar_full + 8 * s, (uint32_t)last_phase[s], err);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (even CTA)
+    if (lane == 0 && rank == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      for (int tile = cid; ok && tile < total; tile += ncl, ++it) {
+        const int acc = it & 1;
+        const uint32_t acc_phase = (uint32_t)(it >> 1) & 1u;
+        const TileCoord tc = tile_coord(tile_start, offsets, E, C::NT, tile);
+        const uint32_t idesc = make_idesc(2 * kWRows, wm_n<MODE>(tc.rows));
+        if (!mbar_wait(bar_tempty + 8 * acc, acc_phase ^ 1u, abort_flag, err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * 256);
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag, err)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t bdesc = sw128_desc(b_blk(stage));
+          const uint64_t adesc0 = sw128_desc(a_blk(stage, 0));
+          const uint64_t adesc1 = sw128_desc(a_blk(stage, MODE == 0 ? 1 : 0));
+#pragma unroll
+          for (int kk = 0; kk < BK / UMMA_K; ++kk) {   // +32 bytes along K per step (>> 4 = 2)
+            const uint32_t accumulate = (kb | kk) != 0 ? 1u : 0u;
+            umma_bf16_pair(d_tmem, adesc0 + 2 * kk, bdesc + 2 * kk, idesc, accumulate);
+            if (MODE == 0) umma_bf16_pair(d_tmem + 128, adesc1 + 2 * kk, bdesc + 2 * kk, idesc, accumulate);
+          }
+          umma_commit_pair_both(bar_empty + 8 * stage);
+          if (++stage == C::stages) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma_commit_pair_both(bar_tfull + 8 * acc);
+      }
+      umma_commit_pair(bar_fin);
+      mbar_wait_drain(bar_fin, 0, err);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int q = warp & 3;                                  // TMEM lane quarter of this warp
+    uint8_t* stage = smem + C::stage + (warp - 2) * kStageWarpBytes;
+    int it = 0;
+    for (int tile = cid; tile < total; tile += ncl, ++it) {
+      const TileCoord tc = tile_coord(tile_start, offsets, E, C::NT, tile);
+      const int acc = it & 1;
+      const uint32_t acc_phase = (uint32_t)(it >> 1) & 1u;
+      const bool got = mbar_wait(bar_tfull + 8 * acc, acc_phase, abort_flag, err);
+      if (!__all_sync(0xffffffffu, got)) break;
+      __syncwarp();
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * 256);
+      const int col0 = tc.n_tile * 256 + (int)rank * kWRows + q * 32;   // this warp's first feature
+      const int chunks = (tc.rows + 31) / 32;
+#pragma unroll 1
+      for (int c = 0; c < chunks; ++c) {
+        const long long r0 = (long long)tc.row0 + c * 32;
+        const int rv = min(32, tc.rows - c * 32);
+        float h[32];
+        if constexpr (MODE == 0) {
+          uint32_t g[32], u[32];
+          tmem_ld32(taddr + c * 32, g);
+          tmem_ld32(taddr + 128 + c * 32, u);
+          tmem_wait_ld();
+          tmem_regs_ready(g);
+          tmem_regs_ready(u);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float gi = __uint_as_float(g[i]);
+            // fast exp / divide: H is rounded to bf16 next, far coarser than their error
+            h[i] = __fdividef(gi, 1.f + __expf(-gi)) * __uint_as_float(u[i]);
+          }
+          stage_store32_t<OutT>(stage, h, lane, out, r0, rv, F, col0, F);
+        } else {
+          uint32_t v[32];
+          tmem_ld32(taddr + c * 32, v);
+          tmem_wait_ld();
+          tmem_regs_ready(v);
+          const float gs = (gate_of_row && lane < rv) ? __ldg(gate_of_row + r0 + lane) : 1.f;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) h[i] = __uint_as_float(v[i]) * __shfl_sync(0xffffffffu, gs, i);
+          stage_store32_t<OutT>(stage, h, lane, out, r0, rv, d, col0, d);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive_cluster(map_to_rank(bar_tempty + 8 * acc, 0));
+    }
+  }
+
+  __syncthreads();
+  cluster_sync();                                           // no remote arrive after a CTA exits
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kWTmemCols) : "memory");
+  }
+}
+
+template <int MODE, typename OutT>
+moe_status launch_wm(const CUtensorMap& mw, const CUtensorMap& mx, const int32_t* offsets, int E, int K, int d,
+                     int F, long long rows_max, const float* gate_of_row, void* out, cudaStream_t s) {
+  using C = WmCfg<MODE>;
+  static std::atomic<int> configured[kMaxDevices];
+  const moe_status st = ensure_smem_limit(configured, grouped_gemm_wm_kernel<MODE, OutT>, C::smem);
+  if (st != MOE_OK) return st;
+  const long long max_tiles = ((rows_max + C::NT - 1) / C::NT + E) * (long long)wm_m_tiles<MODE>(F, d);
+  int pairs = num_sms() / 2;
+  if (max_tiles < pairs) pairs = (int)max_tiles;
+  if (pairs < 1) pairs = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cfg.blockDim = dim3(C::threads, 1, 1);
+  cfg.dynamicSmemBytes = C::smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cuda_status(cudaLaunchKernelEx(&cfg, grouped_gemm_wm_kernel<MODE, OutT>, mw, mx, offsets, E, K, d, F,
+                                        rows_max, gate_of_row, static_cast<OutT*>(out), err_ptr()));
+}
+
+}  // namespace
+
+// Gate/up, weight-major: H [rows_max, F] bf16 from x_perm [rows_max, d] and W_gu [E][2F][d].
+moe_status launch_gate_up_wm(const void* x_rows, const int32_t* offsets, int E, int d, int F, long long rows_max,
+                             const void* W_gu, void* h, cudaStream_t s) {
+  if (rows_max == 0) return MOE_OK;
+  if (d < BK || F < 8) return MOE_ERR_UNSUPPORTED;
+  CUtensorMap mw, mx;
+  if (!make_map(&mw, W_gu, (unsigned long long)E * 2 * F, d, kWRows)) return MOE_ERR_UNSUPPORTED;
+  if (!make_map(&mx, x_rows, (unsigned long long)rows_max, d, WmCfg<0>::NT / 2)) return MOE_ERR_UNSUPPORTED;
+  return launch_wm<0, __nv_bfloat16>(mw, mx, offsets, E, d, d, F, rows_max, nullptr, h, s);
+}
+
+// Down, weight-major: gated rows [rows_max, d] (bf16 or fp32) from H [rows_max, F] and W_dn [E][d][F].
+moe_status launch_down_wm(const void* h, const int32_t* offsets, int E, int d, int F, long long rows_max,
+                          const void* W_dn, const float* gate_of_row, int y_dtype, void* y_rows, cudaStream_t s) {
+  if (rows_max == 0) return MOE_OK;
+  if (F < BK || d < 8) return MOE_ERR_UNSUPPORTED;
+  CUtensorMap mw, mx;
+  if (!make_map(&mw, W_dn, (unsigned long long)E * d, F, kWRows)) return MOE_ERR_UNSUPPORTED;
+  if (!make_map(&mx, h, (unsigned long long)rows_max, F, WmCfg<1>::NT / 2)) return MOE_ERR_UNSUPPORTED;
+  if (y_dtype == MOE_F32) return launch_wm<1, float>(mw, mx, offsets, E, F, d, F, rows_max, gate_of_row, y_rows, s);
+  return launch_wm<1, __nv_bfloat16>(mw, mx, offsets, E, F, d, F, rows_max, gate_of_row, y_rows, s);
+}
+
+}  // namespace moe

@@ -1,5 +1,5 @@
 // Host-side packing of expert weights into 4-bit block-scaled formats, once at load time
-// (the weights are constant across steps, like the router's split weight per call).
+// (the weights are constant across steps, like the router's prepared split weight).
 //
 // Source: handbook digest (agihunt.info), "已确认", bullet "量化与推理": Kimi K3's routed
 // experts in MXFP4; NVIDIA's NVFP4 training with key layers kept in BF16.  The pages name

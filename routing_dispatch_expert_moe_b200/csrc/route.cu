@@ -9,12 +9,16 @@
 // softmax, sigmoid and sqrt(softplus) routers.  Handbook digest (agihunt.info):
 // routing scale factor near sqrt(k).
 //
-// Two kernels:
+// The tensor-core router with the top-k in its epilogue (router_tc.cu) serves bf16 x
+// with at least 256 tokens; this file holds the rest:
 //   logits_kernel  tiled SIMT GEMM  l = x . Wg (+ offset), fp32 FMA; W_g and x staged
 //                  through shared memory, 8 experts x TM tokens per thread, optional
-//                  split over d (partials summed in a fixed order by the next kernel).
+//                  split over d (partials summed in a fixed order by the next kernel);
+//                  for fp32 x, small batches, d < 64 or E not a multiple of 4.
 //   topk_kernel    one warp per token: lanes own experts lane, lane+32, ...; k rounds of
-//                  a shuffle arg-max on (key desc, index asc); gates in fp32.
+//                  a shuffle arg-max on (key desc, index asc); gates in fp32.  After the
+//                  SIMT router, after the tensor-core router for softmax scores with a
+//                  selection bias, and for noisy top-k.
 #include "common.cuh"
 
 #include <float.h>
@@ -396,48 +400,6 @@ topk_kernel(const float* __restrict__ partial, int nsplit, long long split_strid
   }
 }
 
-// ---------------------------------------------------------------------------------
-// Tensor-core router operand: W_g [d, E] fp32 split into three bf16 terms
-//   hi = bf16(w), mid = bf16(w - hi), lo = bf16(w - hi - mid)
-// (each subtraction is exact in fp32; hi + mid + lo carries w to about 24 bits, and x is
-// bf16, so every product x * term is exact in fp32).  Layout W3 [n_tiles * 256, d] bf16,
-// K-major: n-tile j holds experts 64j..64j+63 as rows [0,64) hi, [64,128) mid,
-// [128,192) lo, [192,256) padding (never written, never loaded; rows of experts past E
-// are not written either: they only feed accumulator columns that are never stored).
-// One 32 x 32 shared-memory transpose per block.
-// ---------------------------------------------------------------------------------
-__global__ void __launch_bounds__(256)
-split_router_weight_kernel(const float* __restrict__ Wg, int d, int E, __nv_bfloat16* __restrict__ W3,
-                           int32_t* __restrict__ offs2, int T) {
-  __shared__ float tile[32][33];
-  const int c0 = blockIdx.x * 32, e0 = blockIdx.y * 32;
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;   // 32 x 8
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int c = c0 + ty + 8 * i, e = e0 + tx;
-    tile[ty + 8 * i][tx] = (c < d && e < E) ? __ldg(Wg + (long long)c * E + e) : 0.f;
-  }
-  __syncthreads();
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int e = e0 + ty + 8 * i, c = c0 + tx;
-    if (e >= E || c >= d) continue;
-    const float w = tile[tx][ty + 8 * i];
-    const __nv_bfloat16 hi = __float2bfloat16_rn(w);
-    const float r1 = w - __bfloat162float(hi);
-    const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
-    const __nv_bfloat16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
-    const long long base = (long long)(e >> 6) * 256 + (e & 63);
-    W3[(base + 0) * d + c] = hi;
-    W3[(base + 64) * d + c] = mid;
-    W3[(base + 128) * d + c] = lo;
-  }
-  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
-    offs2[0] = 0;
-    offs2[1] = T;
-  }
-}
-
 struct LogitsPlan {
   int BE, TM, BT, nsplit, chunks_per_split;
   size_t smem;
@@ -466,14 +428,10 @@ moe_status run_logits(const void* x, const float* Wg, const float* off, int T, i
   auto kern = logits_kernel<XT, BE, TM>;
   // the shared-memory size is fixed per instantiation: raise the limit once per device,
   // never inside a launch sequence that may be captured into a CUDA graph
-  static int configured[64] = {0};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  dev &= 63;
-  if (p.smem > 48 * 1024 && !configured[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
-    if (e != cudaSuccess) return cuda_status(e);
-    configured[dev] = 1;
+  static std::atomic<int> configured[kMaxDevices];
+  if (p.smem > 48 * 1024) {
+    const moe_status st = ensure_smem_limit(configured, kern, p.smem);
+    if (st != MOE_OK) return st;
   }
   dim3 grid((T + p.BT - 1) / p.BT, (E + BE - 1) / BE, p.nsplit);
   kern<<<grid, kLogitThreads, p.smem, s>>>(x, Wg, off, T, d, E, p.chunks_per_split, out, split_stride);
@@ -602,91 +560,48 @@ noisy_logits_kernel(const float* __restrict__ logits, const float* __restrict__ 
 
 }  // namespace
 
-// The tensor-core router takes bf16 x with d >= 64 and E a multiple of 4 (16-byte logit
-// rows); anything else runs the fp32 SIMT router.
-static bool tc_router_ok(int x_dtype, int d, int E) { return x_dtype == MOE_BF16 && d >= 64 && E % 4 == 0; }
-static size_t tc_router_w3_bytes(int d, int E) { return (size_t)((E + 63) / 64) * 256 * d * 2; }
-
-// Split W_g into three bf16 terms, then one tcgen05 GEMM writes logits (+ offset), or,
-// with splits > 1, the partial logits of each K run to planes [splits, T, E] (no offset).
-// Workspace: 256 bytes (the one-group offsets {0, T}) + the split weight (+ the planes,
-// placed by the caller).  The split weight's rows for experts past E and its pad rows are
-// left unwritten: they only reach accumulator columns that are never stored.
-static moe_status tc_logits(const void* x, const float* Wg, const float* logit_offset, int T, int d, int E,
-                            float* out, void* ws, cudaStream_t s, int splits) {
-  int32_t* offs2 = static_cast<int32_t*>(ws);
-  __nv_bfloat16* W3 = reinterpret_cast<__nv_bfloat16*>(static_cast<char*>(ws) + 256);
-  dim3 g((d + 31) / 32, (E + 31) / 32);
-  split_router_weight_kernel<<<g, 256, 0, s>>>(Wg, d, E, W3, offs2, T);
-  moe_status st = check_launch();
-  if (st != MOE_OK) return st;
-  return launch_router_logits_tc(x, offs2, T, d, E, W3, splits > 1 ? nullptr : logit_offset, out, s, splits);
-}
-
-// The K-split planes of the tensor-core router sit after the split weight.
-static size_t tc_router_planes_bytes(int T, int d, int E) {
-  const int S = router_k_splits(T, d, E);
-  return S > 1 ? (size_t)S * T * E * sizeof(float) : 0;
-}
-
-// Workspace one call with exactly T tokens uses: the split weight and, when the router
-// splits K, its partial logits (tensor cores) or its split-K partials (SIMT).
-static size_t route_workspace_at(int T, int d, int E) {
+// SIMT router workspace of a call with exactly T tokens: its split-K partials.
+static size_t simt_workspace_at(int T, int d, int E) {
   if (T <= 0 || E <= 0 || d <= 0) return 0;
   LogitsPlan p = plan_logits(T, d, E);
-  const size_t simt = p.nsplit > 1 ? (size_t)p.nsplit * T * E * sizeof(float) : 0;
-  const size_t tc = (E % 4 == 0 && d >= 64) ? 256 + tc_router_w3_bytes(d, E) + tc_router_planes_bytes(T, d, E) : 0;
-  return simt > tc ? simt : tc;
+  return p.nsplit > 1 ? (size_t)p.nsplit * T * E * sizeof(float) : 0;
 }
 
-// The query covers every batch of at most T tokens, so one workspace serves a layer whose
-// batches vary: a smaller batch may split K more ways and use more.  Both split choices
-// depend on the batch only through its number of row tiles (128, 256 or 512 rows for the
-// SIMT router, 256-row pairs for the tensor cores, which also start at 256 rows), which is
-// constant on each run (128 (q - 1), 128 q]; the bytes grow with the tokens inside a run,
-// so the top of each run (and T itself) bounds it.
-size_t route_workspace_bytes(int T, int d, int E) {
+// The query covers every batch of at most T tokens and either x dtype, so one workspace
+// serves a layer whose batches vary.  The SIMT router (fp32 x, batches under 256 tokens,
+// shapes the tensor cores do not take) may split K more ways for a smaller batch: the
+// split choice depends on the batch only through its number of row tiles (128, 256 or
+// 512 rows), constant on each run (128 (q - 1), 128 q], and the bytes grow with the
+// tokens inside a run, so the top of each run (and T itself) bounds it.  The tensor-core
+// router needs room for the split weight when it is not given a prepared one.
+size_t route_workspace_bytes(int T, int d, int E, bool prepared) {
   if (T <= 0 || E <= 0 || d <= 0) return 0;
-  size_t most = route_workspace_at(T, d, E);
+  size_t most = simt_workspace_at(T, d, E);
   for (int t = 128; t < T; t += 128) {
-    const size_t w = route_workspace_at(t, d, E);
+    const size_t w = simt_workspace_at(t, d, E);
+    if (w > most) most = w;
+  }
+  if (!prepared && tc_router_applies(MOE_BF16, T, d, E)) {
+    const size_t w = router_weight_bytes(d, E);
     if (w > most) most = w;
   }
   return most;
 }
 
-moe_status launch_route(const void* x, int x_dtype, const float* Wg, const float* logit_offset,
-                        const float* select_bias, int T, int d, int E, int k, int score,
-                        int renormalize, float scale, float* logits, int32_t* topk_idx,
-                        float* topk_gate, void* ws, cudaStream_t s) {
-  if (T == 0) return MOE_OK;
-  LogitsPlan p = plan_logits(T, d, E);
-  float* partial = logits;
-  const long long split_stride = (long long)T * E;
-  moe_status st = MOE_ERR_UNSUPPORTED;
-  if (tc_router_ok(x_dtype, d, E)) {
-    // K splits when the GEMM has too few tiles; the top-k adds the planes in order
-    const int S = router_k_splits(T, d, E);
-    float* planes = reinterpret_cast<float*>(static_cast<char*>(ws) + 256 + tc_router_w3_bytes(d, E));
-    st = tc_logits(x, Wg, logit_offset, T, d, E, S > 1 ? planes : logits, ws, s, S);
-    if (st != MOE_OK && st != MOE_ERR_UNSUPPORTED) return st;
-    if (st == MOE_OK) {
-      p.nsplit = S;
-      partial = S > 1 ? planes : logits;
-    }
-  }
-  if (st == MOE_ERR_UNSUPPORTED) {
-    partial = p.nsplit > 1 ? static_cast<float*>(ws) : logits;
-    st = x_dtype == MOE_F32
-             ? dispatch_logits<float>(x, Wg, logit_offset, T, d, E, p, partial, split_stride, s)
-             : dispatch_logits<__nv_bfloat16>(x, Wg, logit_offset, T, d, E, p, partial, split_stride, s);
-  }
-  if (st != MOE_OK) return st;
-  const int write = p.nsplit > 1 ? 1 : 0;
+template <int EPL>
+static moe_status topk_dispatch(bool bias, const float* partial, int nsplit, long long split_stride, const float* off,
+                                const float* sel_bias, int T, int E, int k, int score, int renorm, float scale,
+                                float* logits, int write_logits, int32_t* idx, float* gate, cudaStream_t s) {
+  return run_topk<EPL>(bias, partial, nsplit, split_stride, off, sel_bias, T, E, k, score, renorm, scale, logits,
+                       write_logits, idx, gate, s);
+}
+
+static moe_status run_topk_any(bool bias, const float* partial, int nsplit, long long split_stride, const float* off,
+                               const float* sel_bias, int T, int E, int k, int score, int renorm, float scale,
+                               float* logits, int write_logits, int32_t* idx, float* gate, cudaStream_t s) {
   const int epl = (E + 31) / 32;
-  const bool bias = select_bias != nullptr;
-#define MOE_TOPK(N) return run_topk<N>(bias, partial, p.nsplit, split_stride, logit_offset, select_bias, T, E, k, \
-                                       score, renormalize, scale, logits, write, topk_idx, topk_gate, s)
+#define MOE_TOPK(N) return topk_dispatch<N>(bias, partial, nsplit, split_stride, off, sel_bias, T, E, k, score, renorm, \
+                                            scale, logits, write_logits, idx, gate, s)
   if (epl <= 1) MOE_TOPK(1);
   if (epl <= 2) MOE_TOPK(2);
   if (epl <= 4) MOE_TOPK(4);
@@ -696,18 +611,65 @@ moe_status launch_route(const void* x, int x_dtype, const float* Wg, const float
 #undef MOE_TOPK
 }
 
-size_t router_logits_workspace_bytes(int T, int d, int E) {
-  if (T <= 0 || E <= 0 || d <= 0) return 0;
-  return (E % 4 == 0 && d >= 64) ? 256 + tc_router_w3_bytes(d, E) : 0;
+// The prepared weight to use: the caller's, or one split into the workspace now.
+static moe_status router_weight(const float* Wg, const void* Wg_split, int d, int E, void* ws, const void** W3,
+                                cudaStream_t s) {
+  if (Wg_split) {
+    *W3 = Wg_split;
+    return MOE_OK;
+  }
+  *W3 = ws;
+  return launch_prepare_router_weight(Wg, d, E, ws, s);
+}
+
+moe_status launch_route(const void* x, int x_dtype, const float* Wg, const void* Wg_split, const float* logit_offset,
+                        const float* select_bias, int T, int d, int E, int k, int score, int renormalize,
+                        float scale, float* logits, int32_t* topk_idx, float* topk_gate, void* ws, cudaStream_t s) {
+  if (T == 0) return MOE_OK;
+  const bool bias = select_bias != nullptr;
+  if (tc_router_applies(x_dtype, T, d, E)) {
+    const void* W3 = nullptr;
+    moe_status st = router_weight(Wg, Wg_split, d, E, ws, &W3, s);
+    if (st != MOE_OK) return st;
+    // top-k and gates in the GEMM's epilogue, except for softmax scores with a selection
+    // bias, whose keys need the whole row's normaliser before any comparison
+    const bool fuse = !(score == MOE_SCORE_SOFTMAX && bias);
+    st = launch_router_tc(x, T, d, E, W3, logit_offset, logits, fuse ? k : 0, select_bias, score, renormalize, scale,
+                          topk_idx, topk_gate, s);
+    if (st != MOE_ERR_UNSUPPORTED) {
+      if (st != MOE_OK || fuse) return st;
+      return run_topk_any(bias, logits, 1, (long long)T * E, logit_offset, select_bias, T, E, k, score, renormalize,
+                          scale, logits, 0, topk_idx, topk_gate, s);
+    }
+  }
+  LogitsPlan p = plan_logits(T, d, E);
+  float* partial = p.nsplit > 1 ? static_cast<float*>(ws) : logits;
+  const long long split_stride = (long long)T * E;
+  moe_status st = x_dtype == MOE_F32
+                      ? dispatch_logits<float>(x, Wg, logit_offset, T, d, E, p, partial, split_stride, s)
+                      : dispatch_logits<__nv_bfloat16>(x, Wg, logit_offset, T, d, E, p, partial, split_stride, s);
+  if (st != MOE_OK) return st;
+  return run_topk_any(bias, partial, p.nsplit, split_stride, logit_offset, select_bias, T, E, k, score, renormalize,
+                      scale, logits, p.nsplit > 1 ? 1 : 0, topk_idx, topk_gate, s);
+}
+
+size_t router_logits_workspace_bytes(int T, int d, int E, bool prepared) {
+  if (T <= 0 || E <= 0 || d <= 0 || prepared) return 0;
+  // any batch of at least 256 tokens takes the tensor-core path
+  return (T >= 256 && tc_router_applies(MOE_BF16, T, d, E)) ? router_weight_bytes(d, E) : 0;
 }
 
 // The router alone: the tensor-core GEMM where it applies, else the SIMT GEMM in one
 // pass over d (no split, so it writes the logits with their offset itself).
-moe_status launch_router_logits(const void* x, int x_dtype, const float* Wg, const float* logit_offset, int T,
-                                int d, int E, float* logits, void* ws, cudaStream_t s) {
+moe_status launch_router_logits(const void* x, int x_dtype, const float* Wg, const void* Wg_split,
+                                const float* logit_offset, int T, int d, int E, float* logits, void* ws,
+                                cudaStream_t s) {
   if (T == 0) return MOE_OK;
-  if (tc_router_ok(x_dtype, d, E)) {
-    const moe_status st = tc_logits(x, Wg, logit_offset, T, d, E, logits, ws, s, 1);
+  if (tc_router_applies(x_dtype, T, d, E)) {
+    const void* W3 = nullptr;
+    moe_status st = router_weight(Wg, Wg_split, d, E, ws, &W3, s);
+    if (st != MOE_OK) return st;
+    st = launch_router_tc(x, T, d, E, W3, logit_offset, logits, 0, nullptr, 0, 0, 1.f, nullptr, nullptr, s);
     if (st != MOE_ERR_UNSUPPORTED) return st;
   }
   LogitsPlan p = plan_logits(T, d, E);
@@ -742,16 +704,8 @@ moe_status launch_route_noisy(const float* logits, const float* logits_noise, co
   if (st != MOE_OK) return st;
   // KeepTopK on H, then the softmax over the kept H (the learned softmax router's path
   // with H in place of the logits; no offset, no selection bias)
-  const int epl = (E + 31) / 32;
-#define MOE_TOPK(N) return run_topk<N>(false, H, 1, n, nullptr, nullptr, T, E, k, MOE_SCORE_SOFTMAX, 1, scale, \
-                                       H, 0, topk_idx, topk_gate, s)
-  if (epl <= 1) MOE_TOPK(1);
-  if (epl <= 2) MOE_TOPK(2);
-  if (epl <= 4) MOE_TOPK(4);
-  if (epl <= 8) MOE_TOPK(8);
-  if (epl <= 16) MOE_TOPK(16);
-  MOE_TOPK(32);
-#undef MOE_TOPK
+  return run_topk_any(false, H, 1, n, nullptr, nullptr, T, E, k, MOE_SCORE_SOFTMAX, 1, scale, H, 0, topk_idx,
+                      topk_gate, s);
 }
 
 }  // namespace moe

@@ -238,22 +238,24 @@ size_t rank_smem_bytes(int k, int E) {
 constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
 static __device__ __align__(256) unsigned char g_scan_scratch[kNoAllocScratchBytes];
 
-// Device address of g_scan_scratch on the current device, looked up once per device.
+// Device address of g_scan_scratch on the current device, looked up once per device
+// (the first call on a device makes the lookup, so it must come before any stream
+// capture on that device).
 static moe_status noalloc_scratch(void** out) {
-  static void* cached[64] = {nullptr};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_status(e);
-  if (dev < 0 || dev >= 64) return MOE_ERR_UNSUPPORTED;
-  if (!cached[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_scan_scratch);
+  static std::atomic<void*> cached[kMaxDevices];
+  const int dev = device_slot();
+  if (dev < 0) return MOE_ERR_UNSUPPORTED;
+  void* p = cached[dev].load(std::memory_order_acquire);
+  if (!p) {
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_scan_scratch);
     if (e != cudaSuccess) return cuda_status(e);
-    cached[dev] = p;
+    cached[dev].store(p, std::memory_order_release);
   }
-  *out = cached[dev];
+  *out = p;
   return MOE_OK;
 }
+
+size_t histogram_scan_noalloc_limit() { return kNoAllocScratchBytes; }
 
 moe_status launch_histogram_scan_noalloc(const int32_t* topk_idx, const float* topk_gate, int T, int k, int E,
                                          int capacity, int32_t* counts, int32_t* kept, int32_t* offsets,
@@ -293,16 +295,9 @@ moe_status launch_histogram_scan(const int32_t* topk_idx, const float* topk_gate
   const size_t smem = rank_smem_bytes(k, E);
   // raise the limit once per device to the largest size any supported (k, E) needs, so
   // that no attribute call happens inside a launch sequence captured into a CUDA graph
-  static int configured[64] = {0};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  dev &= 63;
-  if (!configured[dev]) {
-    st = cuda_status(cudaFuncSetAttribute(rank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          (int)rank_smem_bytes(32, 1024)));
-    if (st != MOE_OK) return st;
-    configured[dev] = 1;
-  }
+  static std::atomic<int> configured[kMaxDevices];
+  st = ensure_smem_limit(configured, rank_kernel, rank_smem_bytes(32, 1024));
+  if (st != MOE_OK) return st;
   int* err = err_ptr();
   rank_kernel<<<nchunks, kRankThreads, smem, s>>>(topk_idx, T, k, E, capacity, nchunks, w.ticket, w.status,
                                                  w.rank, counts, kept, offsets, err);

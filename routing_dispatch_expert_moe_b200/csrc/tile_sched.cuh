@@ -77,14 +77,10 @@ __device__ __forceinline__ void build_tile_starts(const int32_t* __restrict__ of
   __syncthreads();
 }
 
-// Tile index -> coordinates.  Default: m fastest inside an expert, then n, so that the
-// CTAs working at one time share each weight tile (the large operand of the expert
-// GEMMs).  n_fastest_tiles > 0 (the number of n-tiles): n fastest, so that they share each
-// row tile instead
-// -- for a single group with a small weight matrix (the router), where re-reading the
-// rows once per n-tile would cost a pass over the activations each time.
+// Tile index -> coordinates: m fastest inside an expert, then n, so that the CTAs working
+// at one time share each weight tile (the large operand of the expert GEMMs).
 __device__ __forceinline__ TileCoord tile_coord(const int* tile_start, const int32_t* __restrict__ offsets,
-                                                int E, int BM, int tile, int n_fastest_tiles = 0) {
+                                                int E, int BM, int tile) {
   int lo = 0, hi = E;  // find last e with tile_start[e] <= tile
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
@@ -96,14 +92,8 @@ __device__ __forceinline__ TileCoord tile_coord(const int* tile_start, const int
   const int a = __ldg(offsets + lo), b = __ldg(offsets + lo + 1);
   const int mt = (b - a + BM - 1) / BM;
   const int local = tile - tile_start[lo];
-  int m;
-  if (n_fastest_tiles > 0) {
-    m = local / n_fastest_tiles;
-    c.n_tile = local - m * n_fastest_tiles;
-  } else {
-    c.n_tile = local / mt;
-    m = local - c.n_tile * mt;
-  }
+  c.n_tile = local / mt;
+  const int m = local - c.n_tile * mt;
   c.row0 = a + m * BM;
   c.rows = min(BM, b - c.row0);
   return c;

@@ -115,6 +115,9 @@ class MoELayer:
         self.load = torch.empty(E, dtype=f32, device=dev)
         self.stats5 = torch.empty(5, dtype=f32, device=dev)
         self.ws = torch.empty(max(M.moe_workspace_bytes(T_max, d, E, k), 16), dtype=torch.uint8, device=dev)
+        # the router's exact bf16 split of W_g (and of W_noise), made once here
+        self.Wg_split = M.moe_prepare_router_weight(w.Wg)
+        self.W_noise_split = M.moe_prepare_router_weight(w.W_noise) if routing == "noisy" else None
         self.overlap = overlap
         if overlap:
             self._side = torch.cuda.Stream(device=dev)
@@ -131,13 +134,16 @@ class MoELayer:
         T = x.shape[0]
         if self.routing == "learned":
             M.moe_route(x, self.w.Wg, self.k, self.score, self.renormalize, self.scale, self.w.logit_offset,
-                        self.w.select_bias, self.logits[:T], self.topk_idx[:T], self.topk_gate[:T], self.ws, stream)
+                        self.w.select_bias, self.logits[:T], self.topk_idx[:T], self.topk_gate[:T], self.ws, stream,
+                        Wg_split=self.Wg_split)
             return
-        M.moe_router_logits(x, self.w.Wg, self.w.logit_offset, self.logits[:T], self.ws, stream)
+        M.moe_router_logits(x, self.w.Wg, self.w.logit_offset, self.logits[:T], self.ws, stream,
+                            Wg_split=self.Wg_split)
         if self.routing == "noisy":
             if noise is None:
                 raise ValueError("noisy routing needs the standard normal draws (noise=[T, E] f32)")
-            M.moe_router_logits(x, self.w.W_noise, None, self.logits_noise[:T], self.ws, stream)
+            M.moe_router_logits(x, self.w.W_noise, None, self.logits_noise[:T], self.ws, stream,
+                                Wg_split=self.W_noise_split)
             M.moe_route_noisy(self.logits[:T], self.logits_noise[:T], noise, self.k, self.scale, self.H[:T],
                               self.topk_idx[:T], self.topk_gate[:T], stream)
             return
@@ -301,15 +307,22 @@ class MoELayer:
         return self.y[:self.x_static.shape[0]]
 
     # library kernels launched by one forward (the scan's workspace memset is not a kernel)
-    def _router_gemm_launches(self) -> int:
-        # tensor-core router: the weight split and the GEMM; else one SIMT GEMM
-        tc = self.dtype == torch.bfloat16 and self.d >= 64 and self.E % 4 == 0
-        return 2 if tc else 1
+    def _route_launches(self, T: int) -> int:
+        """Router kernels: one tensor-core kernel (top-k and gates in its epilogue, plus a
+        top-k pass for softmax scores with a selection bias), or the SIMT GEMM and top-k."""
+        tc = self.dtype == torch.bfloat16 and T >= 256 and self.d >= 64 and self.E % 4 == 0
+        if self.routing == "learned":
+            if tc:
+                return 2 if (self.score == "softmax" and self.w.select_bias is not None) else 1
+            return 2
+        gemm = 1                              # the tensor-core or the SIMT logits kernel
+        if self.routing == "noisy":
+            return 2 * gemm + 2               # two router GEMMs, the noise pass, the top-k
+        return gemm + 1                       # the GEMM and the fixed selection
 
-    def launches_per_forward(self, with_stats: bool = True) -> int:
-        r = self._router_gemm_launches()
-        route = {"learned": r + 1, "uniform": r + 1, "hash": r + 1, "noisy": 2 * r + 2}[self.routing]
-        n = route + 2 + 1 + 1 + 1 + 1      # route, scan(2) permute gate_up down combine
+    def launches_per_forward(self, with_stats: bool = True, T: int = None) -> int:
+        T = self.T_max if T is None else T
+        n = self._route_launches(T) + 2 + 1 + 1 + 1 + 1   # route, scan(2) permute gate_up down combine
         if self.combine_mode == "fused":
             n -= 1                         # down_combine (its zero fill is a memset, not a kernel)
             if self.y32 is not self.y:

@@ -36,11 +36,13 @@ _SIGNATURES = {
     "moe_capacity": (_i32, [_i32, _i32, _i32, _f64, _i32]),
     "moe_rows_max": (_i64, [_i32, _i32, _i32, _i32]),
     "moe_route_workspace_bytes": (_size, [_i32, _i32, _i32]),
-    "moe_route": (_i32, [_c_void_p, _i32, _c_void_p, _c_void_p, _c_void_p, _i32, _i32, _i32, _i32, _i32, _i32,
-                         _f32, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _size, _c_void_p]),
+    "moe_router_weight_bytes": (_size, [_i32, _i32]),
+    "moe_prepare_router_weight": (_i32, [_c_void_p, _i32, _i32, _c_void_p, _size, _c_void_p]),
+    "moe_route": (_i32, [_c_void_p, _i32, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _i32, _i32, _i32, _i32, _i32,
+                         _i32, _f32, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _size, _c_void_p]),
     "moe_router_logits_workspace_bytes": (_size, [_i32, _i32, _i32]),
-    "moe_router_logits": (_i32, [_c_void_p, _i32, _c_void_p, _c_void_p, _i32, _i32, _i32, _c_void_p, _c_void_p,
-                                 _size, _c_void_p]),
+    "moe_router_logits": (_i32, [_c_void_p, _i32, _c_void_p, _c_void_p, _c_void_p, _i32, _i32, _i32, _c_void_p,
+                                 _c_void_p, _size, _c_void_p]),
     "moe_route_fixed": (_i32, [_c_void_p, _i32, _i32, _i32, _i32, _i32, _f32, _i32, _c_void_p, ctypes.c_uint32,
                                _c_void_p, _c_void_p, _c_void_p]),
     "moe_route_noisy": (_i32, [_c_void_p, _c_void_p, _c_void_p, _i32, _i32, _i32, _f32, _c_void_p, _c_void_p,
@@ -163,14 +165,39 @@ def moe_workspace_bytes(T: int, d: int, E: int, k: int) -> int:
 
 
 # ---------------------------------------------------------------- the calls
+def moe_router_weight_bytes(d: int, E: int) -> int:
+    return int(lib().moe_router_weight_bytes(d, E))
+
+
+def moe_prepare_router_weight(Wg, Wg_split=None, stream=None):
+    """The tensor-core router's exact three-term bf16 split of Wg [d, E] f32, made once when
+    the weights are loaded.  Returns the uint8 device buffer, or None when the tensor-core
+    router does not apply to (d, E) (the router then reads Wg directly)."""
+    d, E = Wg.shape
+    _need(Wg, "Wg", torch.float32, (d, E))
+    nb = moe_router_weight_bytes(d, E)
+    if nb == 0:
+        return None
+    Wg_split = torch.empty(nb, dtype=torch.uint8, device=Wg.device) if Wg_split is None else \
+        _need(Wg_split, "Wg_split", torch.uint8)
+    if Wg_split.numel() < nb:
+        raise ValueError(f"Wg_split must hold {nb} bytes, got {Wg_split.numel()}")
+    _check("moe_prepare_router_weight", lib().moe_prepare_router_weight(_p(Wg), d, E, _p(Wg_split), nb,
+                                                                        _stream(stream)))
+    return Wg_split
+
+
 def moe_route(x, Wg, k: int, score: str = "softmax", renormalize: bool = True, scale: float = 1.0,
               logit_offset=None, select_bias=None, logits=None, topk_idx=None, topk_gate=None,
-              workspace=None, stream=None):
-    """Router logits, top-k and gates.  Returns (logits [T,E] f32, topk_idx [T,k] i32, topk_gate [T,k] f32)."""
+              workspace=None, stream=None, Wg_split=None):
+    """Router logits, top-k and gates.  Returns (logits [T,E] f32, topk_idx [T,k] i32, topk_gate [T,k] f32).
+    Wg_split: moe_prepare_router_weight(Wg)'s buffer (None: the call splits Wg itself)."""
     T, d = x.shape
     E = Wg.shape[1]
     _need(x, "x")
     _need(Wg, "Wg", torch.float32, (d, E))
+    if Wg_split is not None:
+        _need(Wg_split, "Wg_split", torch.uint8)
     for t, n in ((logit_offset, "logit_offset"), (select_bias, "select_bias")):
         if t is not None:
             _need(t, n, torch.float32, (E,))
@@ -183,18 +210,20 @@ def moe_route(x, Wg, k: int, score: str = "softmax", renormalize: bool = True, s
         _need(topk_gate, "topk_gate", torch.float32, (T, k))
     nb = int(lib().moe_route_workspace_bytes(T, d, E))
     ws = _ws(nb, dev, workspace)
-    _check("moe_route", lib().moe_route(_p(x), _dt(x), _p(Wg), _p(logit_offset), _p(select_bias), T, d, E, k,
-                                        SCORE[score], 1 if renormalize else 0, float(scale), _p(logits),
+    _check("moe_route", lib().moe_route(_p(x), _dt(x), _p(Wg), _p(Wg_split), _p(logit_offset), _p(select_bias), T, d,
+                                        E, k, SCORE[score], 1 if renormalize else 0, float(scale), _p(logits),
                                         _p(topk_idx), _p(topk_gate), _p(ws), nb, _stream(stream)))
     return logits, topk_idx, topk_gate
 
 
-def moe_router_logits(x, Wg, logit_offset=None, logits=None, workspace=None, stream=None):
+def moe_router_logits(x, Wg, logit_offset=None, logits=None, workspace=None, stream=None, Wg_split=None):
     """The router alone: logits [T,E] f32 = x . Wg (+ logit_offset)."""
     T, d = x.shape
     E = Wg.shape[1]
     _need(x, "x")
     _need(Wg, "Wg", torch.float32, (d, E))
+    if Wg_split is not None:
+        _need(Wg_split, "Wg_split", torch.uint8)
     if logit_offset is not None:
         _need(logit_offset, "logit_offset", torch.float32, (E,))
     dev = x.device
@@ -202,8 +231,8 @@ def moe_router_logits(x, Wg, logit_offset=None, logits=None, workspace=None, str
         _need(logits, "logits", torch.float32, (T, E))
     nb = int(lib().moe_router_logits_workspace_bytes(T, d, E))
     ws = _ws(nb, dev, workspace)
-    _check("moe_router_logits", lib().moe_router_logits(_p(x), _dt(x), _p(Wg), _p(logit_offset), T, d, E,
-                                                        _p(logits), _p(ws), nb, _stream(stream)))
+    _check("moe_router_logits", lib().moe_router_logits(_p(x), _dt(x), _p(Wg), _p(Wg_split), _p(logit_offset), T, d,
+                                                        E, _p(logits), _p(ws), nb, _stream(stream)))
     return logits
 
 
@@ -313,18 +342,31 @@ def moe_histogram_scan_noalloc(topk_idx, topk_gate, E: int, capacity: int, count
                                token_of_row, gate_of_row, stream=None):
     """moe_histogram_scan without a workspace, for callers that cannot allocate device memory:
     the library's own 4 MiB scratch array is used instead.  Every output buffer must be
-    passed in (this wrapper allocates nothing either).  Calls that overlap on the GPU race
-    on the shared scratch; the first call on a device must come before any stream capture."""
+    passed in (this wrapper allocates nothing either), all on topk_idx's device, which is
+    made current for the call.  Calls that overlap on the GPU race on the shared scratch;
+    the first call on a device must come before any stream capture."""
     T, k = topk_idx.shape
     _need(topk_idx, "topk_idx", torch.int32)
     _need(topk_gate, "topk_gate", torch.float32, (T, k))
-    for t, n, dt in ((counts, "counts", torch.int32), (kept, "kept", torch.int32), (offsets, "offsets", torch.int32),
-                     (row_of, "row_of", torch.int32), (token_of_row, "token_of_row", torch.int32),
-                     (gate_of_row, "gate_of_row", torch.float32)):
-        _need(t, n, dt)
-    _check("moe_histogram_scan_noalloc", lib().moe_histogram_scan_noalloc(
-        _p(topk_idx), _p(topk_gate), T, k, E, capacity, _p(counts), _p(kept), _p(offsets), _p(row_of),
-        _p(token_of_row), _p(gate_of_row), _stream(stream)))
+    rows = max(moe_rows_max(T, E, k, capacity), 1)
+    for t, n, dt, shape in ((counts, "counts", torch.int32, (E,)), (kept, "kept", torch.int32, (E,)),
+                            (offsets, "offsets", torch.int32, (E + 1,)), (row_of, "row_of", torch.int32, (T, k)),
+                            (token_of_row, "token_of_row", torch.int32, None),
+                            (gate_of_row, "gate_of_row", torch.float32, None)):
+        _need(t, n, dt, shape)
+    for t, n in ((token_of_row, "token_of_row"), (gate_of_row, "gate_of_row")):
+        if t.numel() < rows:
+            raise ValueError(f"{n} must hold at least moe_rows_max(T, E, k, capacity) = {rows} entries, "
+                             f"got {t.numel()}")
+    dev = topk_idx.device
+    for t, n in ((topk_gate, "topk_gate"), (counts, "counts"), (kept, "kept"), (offsets, "offsets"),
+                 (row_of, "row_of"), (token_of_row, "token_of_row"), (gate_of_row, "gate_of_row")):
+        if t.device != dev:
+            raise ValueError(f"{n} is on {t.device}, topk_idx on {dev}: every buffer must be on one device")
+    with torch.cuda.device(dev):
+        _check("moe_histogram_scan_noalloc", lib().moe_histogram_scan_noalloc(
+            _p(topk_idx), _p(topk_gate), T, k, E, capacity, _p(counts), _p(kept), _p(offsets), _p(row_of),
+            _p(token_of_row), _p(gate_of_row), _stream(stream)))
 
 
 def moe_permute(x, row_of, rows_max: int, x_perm=None, stream=None):

@@ -26,8 +26,11 @@ int main(void) {
   CHECK(moe_route_workspace_bytes(8192, 2048, 64) > 0);
   CHECK(moe_workspace_bytes(8192, 2048, 64, 8) >= moe_histogram_scan_workspace_bytes(8192, 8, 64));
   /* a device call rejected on the host: null x, nothing launched */
-  CHECK(moe_route(NULL, MOE_BF16, NULL, NULL, NULL, 64, 128, 16, 4, MOE_SCORE_SOFTMAX, 1, 1.0f, NULL, NULL,
+  CHECK(moe_route(NULL, MOE_BF16, NULL, NULL, NULL, NULL, 64, 128, 16, 4, MOE_SCORE_SOFTMAX, 1, 1.0f, NULL, NULL,
                   NULL, NULL, 0, NULL) == MOE_ERR_INVALID_ARG);
+  /* the router's prepared split: three bf16 terms of 64 experts x 2048 */
+  CHECK(moe_router_weight_bytes(2048, 64) == (size_t)3 * 64 * 2048 * 2);
+  CHECK(moe_prepare_router_weight(NULL, 2048, 64, NULL, 0, NULL) == MOE_ERR_INVALID_ARG);
   /* FP4: one MXFP4 block of 32 values that E2M1 represents exactly after the 2^-3 scale */
   {
     static const float mags[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};

@@ -207,6 +207,22 @@ def assert_y_close_bf16(gy, oy, slot_rows, slot_hbound, shared_y=None):
     return float(err.max()) / rms, float(err.mean()) / rms
 
 
+def bar_report(gy, oy):
+    """The layer's stated bar (max|err| <= 2e-2 rms, mean|err| <= 2e-3 rms) on a bf16 output:
+    observed max and mean error over rms, and the elements past the max bar with their
+    error counted in bf16 steps of the reference value (a correct sum in a different order
+    may land one step away, and one step at |y| > 4 rms is more than 2e-2 rms)."""
+    gy = np.asarray(gy, np.float64)
+    oy = np.asarray(oy, np.float64)
+    rms = float(np.sqrt(np.mean(oy ** 2)))
+    err = np.abs(gy - oy)
+    over = err > Y_MAX_REL * rms
+    steps = err[over] / bf16_step(oy[over]) if over.any() else np.zeros(0)
+    return {"max_rel": float(err.max()) / rms, "mean_rel": float(err.mean()) / rms, "n": int(err.size),
+            "n_over_max_bar": int(over.sum()), "max_steps_over": float(steps.max()) if steps.size else 0.0,
+            "min_abs_over_rms": float(np.abs(oy[over]).min() / rms) if over.any() else None}
+
+
 def assert_stats_close(g, o_stats, dropped_exact=True):
     np.testing.assert_allclose(g["load"], o_stats["load"], rtol=1e-6, atol=0)
     s = g["stats5"].astype(np.float64)

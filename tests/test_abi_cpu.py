@@ -72,17 +72,18 @@ NUL = None
 
 
 def _route(L, **kw):
-    a = dict(x=FAKE, dt=0, Wg=FAKE, off=NUL, bias=NUL, T=64, d=128, E=16, k=4, score=0, renorm=1, scale=1.0,
+    a = dict(x=FAKE, dt=0, Wg=FAKE, W3=NUL, off=NUL, bias=NUL, T=64, d=128, E=16, k=4, score=0, renorm=1, scale=1.0,
              logits=FAKE, idx=FAKE, gate=FAKE, ws=FAKE, wsb=1 << 30, s=NUL)
     a.update(kw)
-    return L.moe_route(a["x"], a["dt"], a["Wg"], a["off"], a["bias"], a["T"], a["d"], a["E"], a["k"], a["score"],
-                       a["renorm"], a["scale"], a["logits"], a["idx"], a["gate"], a["ws"], a["wsb"], a["s"])
+    return L.moe_route(a["x"], a["dt"], a["Wg"], a["W3"], a["off"], a["bias"], a["T"], a["d"], a["E"], a["k"],
+                       a["score"], a["renorm"], a["scale"], a["logits"], a["idx"], a["gate"], a["ws"], a["wsb"],
+                       a["s"])
 
 
 @pytest.mark.parametrize("d,E", [(2048, 64), (4096, 63), (7168, 896), (1024, 36), (64, 8), (512, 1024)])
 def test_workspace_queries_cover_every_smaller_batch(L, d, E):
-    """A smaller batch may split the router GEMM more ways (SIMT split-K, tensor-core K
-    runs), so a query for T must cover every T' <= T: one layer workspace serves them all."""
+    """A smaller batch may split the SIMT router's GEMM more ways, so a query for T must
+    cover every T' <= T: one layer workspace serves them all."""
     ts = sorted(set(list(range(1, 1200, 37)) + list(range(1024, 20000, 389)) + [256, 2368, 4608, 4864, 5000, 8192]))
     prev_r = prev_w = 0
     for T in ts:
@@ -97,7 +98,7 @@ def test_workspace_queries_cover_every_smaller_batch(L, d, E):
     (dict(x=NUL), 1), (dict(Wg=NUL), 1), (dict(logits=NUL), 1), (dict(k=17), 1), (dict(k=0), 1),
     (dict(E=0), 1), (dict(T=-1), 1), (dict(score=3), 1), (dict(dt=7), 1), (dict(renorm=2), 1),
     (dict(scale=float("nan")), 1), (dict(E=1025, k=4), 2), (dict(k=33, E=64), 2), (dict(d=100), 2),
-    (dict(x=ctypes.c_void_p(4104)), 2),
+    (dict(x=ctypes.c_void_p(4104)), 2), (dict(W3=ctypes.c_void_p(4104)), 2),
 ])
 def test_route_host_validation(L, kw, status):
     assert _route(L, **kw) == status
@@ -108,6 +109,28 @@ def test_route_workspace_check(L):
     if need:
         assert _route(L, d=4096, wsb=need - 1) == 3
         assert _route(L, d=4096, ws=NUL) == 3
+    # the tensor-core path (T >= 256) splits W_g into the workspace unless given the split
+    need = L.moe_route_workspace_bytes(512, 2048, 64)
+    assert need >= L.moe_router_weight_bytes(2048, 64) > 0
+    assert _route(L, T=512, d=2048, E=64, wsb=need - 1) == 3
+
+
+def test_router_weight_size_and_prepare_validation(L):
+    # experts in ceil(E / 256) tiles of NE = 32 * ceil(ceil(E / tiles) / 32), three bf16 terms each
+    for d, E, NE, tiles in ((2048, 64, 64, 1), (4096, 256, 256, 1), (7168, 896, 224, 4), (512, 1024, 256, 4),
+                            (64, 8, 32, 1), (128, 260, 160, 2), (4096, 520, 192, 3)):
+        assert L.moe_router_weight_bytes(d, E) == tiles * 3 * NE * d * 2, (d, E)
+    assert L.moe_router_weight_bytes(56, 64) == 0          # d < 64: SIMT router, no split
+    assert L.moe_router_weight_bytes(2048, 66) == 0        # E % 4
+    assert L.moe_router_weight_bytes(2048, 2048) == 0      # E > 1024
+    f = L.moe_prepare_router_weight                        # (Wg, d, E, out, bytes, stream)
+    nb = L.moe_router_weight_bytes(2048, 64)
+    assert f(NUL, 2048, 64, FAKE, nb, NUL) == 1
+    assert f(FAKE, 2048, 64, NUL, nb, NUL) == 1
+    assert f(FAKE, 0, 64, FAKE, nb, NUL) == 1
+    assert f(FAKE, 2048, 64, FAKE, nb - 1, NUL) == 3
+    assert f(FAKE, 2048, 66, FAKE, nb, NUL) == 2
+    assert f(FAKE, 2048, 64, ctypes.c_void_p(4104), nb, NUL) == 2
 
 
 def test_route_empty_batch_is_ok_without_launch(L):
@@ -115,7 +138,8 @@ def test_route_empty_batch_is_ok_without_launch(L):
 
 
 def test_router_logits_host_validation(L):
-    f = L.moe_router_logits            # (x, dt, Wg, off, T, d, E, logits, ws, wsb, s)
+    def f(*a):                         # (x, dt, Wg, off, T, d, E, logits, ws, wsb, s), Wg_split NULL
+        return L.moe_router_logits(a[0], a[1], a[2], NUL, *a[3:])
     assert f(NUL, 0, FAKE, NUL, 64, 128, 16, FAKE, FAKE, 1 << 30, NUL) == 1          # x
     assert f(FAKE, 0, FAKE, NUL, 64, 128, 16, NUL, FAKE, 1 << 30, NUL) == 1          # logits
     assert f(FAKE, 5, FAKE, NUL, 64, 128, 16, FAKE, FAKE, 1 << 30, NUL) == 1         # dtype
@@ -123,10 +147,11 @@ def test_router_logits_host_validation(L):
     assert f(FAKE, 0, FAKE, NUL, 64, 128, 2048, FAKE, FAKE, 1 << 30, NUL) == 2       # E > 1024
     assert f(FAKE, 0, FAKE, NUL, 64, 100, 16, FAKE, FAKE, 1 << 30, NUL) == 2         # d % 8
     assert f(ctypes.c_void_p(4104), 0, FAKE, NUL, 64, 128, 16, FAKE, FAKE, 1 << 30, NUL) == 2
-    need = L.moe_router_logits_workspace_bytes(64, 128, 16)
-    assert need > 0
-    assert f(FAKE, 0, FAKE, NUL, 64, 128, 16, FAKE, FAKE, need - 1, NUL) == 3
-    assert L.moe_router_logits_workspace_bytes(64, 128, 18) == 0                    # E % 4: SIMT, no workspace
+    assert L.moe_router_logits_workspace_bytes(64, 128, 16) == 0                    # under 256 tokens: SIMT
+    need = L.moe_router_logits_workspace_bytes(512, 128, 16)
+    assert need == L.moe_router_weight_bytes(128, 16) > 0                           # the split, made by the call
+    assert f(FAKE, 0, FAKE, NUL, 512, 128, 16, FAKE, FAKE, need - 1, NUL) == 3
+    assert L.moe_router_logits_workspace_bytes(512, 128, 18) == 0                   # E % 4: SIMT, no workspace
     assert f(NUL, 0, NUL, NUL, 0, 128, 16, NUL, NUL, 0, NUL) == 0                    # T = 0: nothing to do
 
 

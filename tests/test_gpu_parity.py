@@ -3,6 +3,8 @@ inputs, element by element.  Small shapes compare every output of every step; th
 full-size workloads compare routing in full and expert outputs on a stratified token
 sample (each token's output depends only on its own row, routing and the weights).
 """
+import json
+
 import numpy as np
 import pytest
 import torch
@@ -84,14 +86,24 @@ SMALL = [
 ]
 
 
+# Both tile orientations of the grouped GEMMs: token-major (256 rows of one expert per CTA
+# pair) and weight-major (256 weight rows x the expert's tokens); the library picks one from
+# the average group size, MOE_B200_EXPERT_TILES forces it.
+TILES = ["tokens", "weights"]
+
+
+@pytest.mark.parametrize("tiles", TILES)
 @pytest.mark.parametrize("cfg", SMALL, ids=lambda c: c.name)
-def test_small_full_parity(cfg):
+def test_small_full_parity(cfg, tiles, monkeypatch):
+    monkeypatch.setenv("MOE_B200_EXPERT_TILES", tiles)
     full_check(cfg)
 
 
+@pytest.mark.parametrize("tiles", TILES)
 @pytest.mark.parametrize("cfg", [SMALL[0], SMALL[1], SMALL[4]], ids=lambda c: c.name)
-def test_bf16_rows_and_bf16_output(cfg):
+def test_bf16_rows_and_bf16_output(cfg, tiles, monkeypatch):
     """The bandwidth-saving variant: gated rows and y stored in bf16 (two more roundings)."""
+    monkeypatch.setenv("MOE_B200_EXPERT_TILES", tiles)
     host, dev = U.make_inputs(cfg)
     cap = O.capacity(cfg.T, cfg.E, cfg.k, cfg.capacity_factor)
     layer, g = U.gpu_forward(cfg, dev, cap, torch.bfloat16, torch.bfloat16)
@@ -514,8 +526,18 @@ def bf16_full_size_check(name):
         xs = np.asarray(host["x"])[toks]
         ys = O.shared_expert(xs, host["shared"][0], host["shared"][1], True, round_out=True)
     U.assert_y_close_bf16(g["y"][toks], sub["y"], sub["slot_rows"], slot_hb, ys)
+    # the stated bar itself: the mean always; the max wherever it holds -- an element past
+    # it must be a large output (above 2 rms; one bf16 step there is 2^-7 of the value) at
+    # most two bf16 steps of its value away (one from the output's own rounding, one from
+    # the rounded rows summed into it)
+    rep = U.bar_report(g["y"][toks], sub["y"])
+    print(f"\nbf16 form {name}: " + json.dumps(rep))
+    assert rep["mean_rel"] <= U.Y_MEAN_REL
+    if rep["n_over_max_bar"]:
+        assert rep["max_steps_over"] <= 2.0 and rep["min_abs_over_rms"] > 2.0, rep
     del layer, dev
     torch.cuda.empty_cache()
+    return rep
 
 
 @pytest.mark.slow
@@ -526,3 +548,22 @@ def test_c2_handbook_full_size_bf16_rows_and_output():
 @pytest.mark.slow
 def test_c3_fine_grained_full_size_bf16_rows_and_output():
     bf16_full_size_check("c3_fine_grained")
+
+
+@pytest.mark.slow
+def test_c4_coarse_full_size_bf16_rows_and_output():
+    bf16_full_size_check("c4_coarse")
+
+
+@pytest.mark.slow
+def test_c5_stress_full_size_bf16_rows_and_output():
+    """The form and workload bench.py times by default."""
+    bf16_full_size_check("c5_stress")
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name,tiles", [("c2_handbook", "weights"), ("c5_stress", "tokens")])
+def test_full_size_bf16_form_other_tile_orientation(name, tiles, monkeypatch):
+    """The orientation the library does not pick for this workload, at full size."""
+    monkeypatch.setenv("MOE_B200_EXPERT_TILES", tiles)
+    bf16_full_size_check(name)

@@ -56,10 +56,12 @@ ROUTER = [
     I.small_config("tc_ragged_offset", T=1000, d=128, E=36, k=4, F=64, logit_offset="zipf1.2"),
     I.small_config("simt_E_odd", T=333, d=128, E=37, k=3, F=64),
     I.small_config("simt_fp32", T=256, d=64, E=8, k=2, F=64, act="f32"),
-    I.small_config("tc_E1024", T=130, d=64, E=1024, k=32, F=64, logit_offset="normal0.5"),
-    # few row tiles: moe_route splits K (8 and 4 runs), moe_router_logits does not
-    I.small_config("tc_ksplit8", T=512, d=2048, E=64, k=8, F=64),
-    I.small_config("tc_ksplit4_ragged_offset", T=700, d=1024, E=36, k=4, F=64, logit_offset="zipf1.2"),
+    I.small_config("simt_small_batch_E1024", T=130, d=64, E=1024, k=32, F=64, logit_offset="normal0.5"),
+    I.small_config("tc_E1024", T=300, d=64, E=1024, k=32, F=64, logit_offset="normal0.5"),
+    # few row tiles: most CTA pairs idle; a ragged last tile of 700 - 512 tokens
+    I.small_config("tc_long_d", T=512, d=2048, E=64, k=8, F=64),
+    I.small_config("tc_ragged_tiles_offset", T=700, d=1024, E=36, k=4, F=64, logit_offset="zipf1.2"),
+    I.small_config("tc_three_expert_tiles", T=520, d=256, E=520, k=6, F=64, score="sigmoid"),
 ]
 
 

@@ -3,6 +3,8 @@
 The argument checks run before the constructor touches any device memory, so CPU
 tensors stand in for the weights.
 """
+import types
+
 import pytest
 import torch
 
@@ -38,26 +40,31 @@ def test_layer_rejects_bad_arguments_before_allocating(kw, msg):
 class _Stub:
     """The attributes launches_per_forward reads, without building a layer."""
     launches_per_forward = MoELayer.launches_per_forward
-    _router_gemm_launches = MoELayer._router_gemm_launches
+    _route_launches = MoELayer._route_launches
 
     def __init__(self, routing="learned", dtype=torch.bfloat16, d=2048, E=64, combine="rows", dispatch="permute",
-                 shared=False, fused_bf16=False):
+                 shared=False, fused_bf16=False, T_max=8192, score="softmax", bias=False):
         self.routing, self.dtype, self.d, self.E = routing, dtype, d, E
         self.combine_mode, self.dispatch_mode, self.has_shared = combine, dispatch, shared
+        self.T_max, self.score = T_max, score
+        self.w = types.SimpleNamespace(select_bias=torch.zeros(E) if bias else None)
         self.y = object()
         self.y32 = object() if fused_bf16 else self.y
 
 
 def test_launch_count_matches_the_kernels_each_form_runs():
-    # handbook default: split + router GEMM + top-k, rank + scatter, permute, gate/up, down,
-    # combine; statistics partial + final (the launch list shows these 11 kernels)
-    assert _Stub().launches_per_forward(True) == 11
-    assert _Stub().launches_per_forward(False) == 9
-    assert _Stub(dtype=torch.float32).launches_per_forward(True) == 10       # one SIMT router GEMM
+    # handbook default: the tensor-core router with the top-k in its epilogue, rank +
+    # scatter, permute, gate/up, down, combine; statistics partial + final (9 kernels)
+    assert _Stub().launches_per_forward(True) == 9
+    assert _Stub().launches_per_forward(False) == 7
+    assert _Stub(dtype=torch.float32).launches_per_forward(True) == 10       # SIMT router GEMM + top-k
     assert _Stub(E=37).launches_per_forward(True) == 10                      # E % 4: SIMT router
-    assert _Stub(routing="uniform").launches_per_forward(True) == 11         # top-k -> fixed selection
-    assert _Stub(routing="noisy").launches_per_forward(True) == 14           # two router GEMMs + H + top-k
-    assert _Stub(combine="fused").launches_per_forward(True) == 10
-    assert _Stub(combine="fused", fused_bf16=True).launches_per_forward(True) == 11
-    assert _Stub(dispatch="gather").launches_per_forward(True) == 10
-    assert _Stub(shared=True).launches_per_forward(True) == 13
+    assert _Stub(T_max=200).launches_per_forward(True) == 10                 # under 256 tokens: SIMT router
+    assert _Stub(score="softmax", bias=True).launches_per_forward(True) == 10   # + a separate top-k pass
+    assert _Stub(score="sigmoid", bias=True).launches_per_forward(True) == 9    # biased keys fused
+    assert _Stub(routing="uniform").launches_per_forward(True) == 10         # router logits -> fixed selection
+    assert _Stub(routing="noisy").launches_per_forward(True) == 12           # two router GEMMs + H + top-k
+    assert _Stub(combine="fused").launches_per_forward(True) == 8
+    assert _Stub(combine="fused", fused_bf16=True).launches_per_forward(True) == 9
+    assert _Stub(dispatch="gather").launches_per_forward(True) == 8
+    assert _Stub(shared=True).launches_per_forward(True) == 11
