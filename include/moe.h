@@ -298,6 +298,27 @@ MOE_API moe_status moe_histogram_scan(const int32_t* topk_idx, const float* topk
                               void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------------------
+ * moe_scan_wait_check -- diagnostic: makes the histogram/scan's bounded wait run out.
+ * (No counterpart on the pages: it tests the library's own recovery path.)
+ * The look-back of moe_histogram_scan's rank kernel waits for the running totals of the
+ * chunks of 256 tokens before it; every such wait is bounded.  This call runs the same
+ * kernels with the first chunk withheld, so every later chunk waits for a word that is
+ * never published.  Each wait gives up after wait_ns nanoseconds, records
+ * MOE_DEVERR_SCAN_TIMEOUT in the device error word and lets the kernel finish; the
+ * call returns MOE_OK once launched, and the context stays usable.  Nothing traps or
+ * faults: every index stays bounded whatever the totals.  The outputs are not meaningful.
+ *   arguments as moe_histogram_scan, plus
+ *   wait_ns      1e3 .. 1e9: the per-wait limit (the ordinary calls use one second)
+ * Errors: INVALID_ARG for T <= 256 (there must be a chunk after the first), a null
+ * pointer or wait_ns outside its range; WORKSPACE as moe_histogram_scan.
+ * ---------------------------------------------------------------------------------- */
+MOE_API moe_status moe_scan_wait_check(const int32_t* topk_idx, const float* topk_gate,
+                              int32_t T, int32_t k, int32_t E, int32_t capacity,
+                              int32_t* counts, int32_t* kept, int32_t* offsets,
+                              int32_t* row_of, int32_t* token_of_row, float* gate_of_row,
+                              uint64_t wait_ns, void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------------------
  * moe_histogram_scan_noalloc -- moe_histogram_scan for callers that cannot allocate.
  * (No counterpart on the pages: this is a deployment convenience, not part of the method.)
  *

@@ -239,6 +239,23 @@ moe_status moe_histogram_scan_noalloc(const int32_t* topk_idx, const float* topk
                                        token_of_row, gate_of_row, rows_max, S(stream));
 }
 
+moe_status moe_scan_wait_check(const int32_t* topk_idx, const float* topk_gate, int32_t T, int32_t k, int32_t E,
+                               int32_t capacity, int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* row_of,
+                               int32_t* token_of_row, float* gate_of_row, uint64_t wait_ns, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+  moe_status st = check_dims(T, E, k);
+  if (st != MOE_OK) return st;
+  if (capacity < -1 || wait_ns < 1000ull || wait_ns > 1000000000ull) return MOE_ERR_INVALID_ARG;
+  if (T <= 256) return MOE_ERR_INVALID_ARG;              // needs a chunk after the withheld first one
+  if (!counts || !kept || !offsets || !topk_idx || !topk_gate || !row_of || !token_of_row || !gate_of_row)
+    return MOE_ERR_INVALID_ARG;
+  const size_t need = histogram_scan_workspace_bytes(T, k, E);
+  if (!workspace || workspace_bytes < need) return MOE_ERR_WORKSPACE;
+  const long long rows_max = moe_rows_max(T, E, k, capacity);
+  return launch_scan_wait_check(topk_idx, topk_gate, T, k, E, capacity, counts, kept, offsets, row_of, token_of_row,
+                                gate_of_row, rows_max, workspace, (unsigned long long)wait_ns, S(stream));
+}
+
 moe_status moe_permute(const void* x, int32_t dtype, int32_t T, int32_t d, int32_t k, const int32_t* row_of,
                        int64_t rows_max, void* x_perm, void* stream) {
   if (T < 0 || k < 1 || rows_max < 0) return MOE_ERR_INVALID_ARG;

@@ -169,6 +169,10 @@ moe_status launch_histogram_scan(const int32_t* topk_idx, const float* topk_gate
                                  float* gate_of_row, long long rows_max, void* ws, cudaStream_t s);
 size_t histogram_scan_workspace_bytes(int T, int k, int E);
 size_t histogram_scan_noalloc_limit();
+moe_status launch_scan_wait_check(const int32_t* topk_idx, const float* topk_gate, int T, int k, int E,
+                                  int capacity, int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* row_of,
+                                  int32_t* token_of_row, float* gate_of_row, long long rows_max, void* ws,
+                                  unsigned long long wait_ns, cudaStream_t s);
 moe_status launch_histogram_scan_noalloc(const int32_t* topk_idx, const float* topk_gate, int T, int k, int E,
                                          int capacity, int32_t* counts, int32_t* kept, int32_t* offsets,
                                          int32_t* row_of, int32_t* token_of_row, float* gate_of_row,

@@ -70,7 +70,7 @@ __global__ void __launch_bounds__(kRankThreads)
 rank_kernel(const int32_t* __restrict__ topk_idx, int T, int k, int E, int capacity, int nchunks,
             uint32_t* __restrict__ ticket, uint32_t* __restrict__ status, int32_t* __restrict__ rank,
             int32_t* __restrict__ counts, int32_t* __restrict__ kept, int32_t* __restrict__ offsets,
-            int* err) {
+            unsigned long long spin_limit_ns, int* err) {
   extern __shared__ __align__(16) uint32_t sm[];
   uint32_t* masks = sm;                                            // [8][E]
   uint32_t* wpre = masks + 8 * E;                                  // [8][E] warp-exclusive prefix
@@ -127,7 +127,7 @@ rank_kernel(const int32_t* __restrict__ topk_idx, int T, int k, int E, int capac
         const uint32_t f = v & ~kValMask;
         if (f == 0u) {
           if (spins == 0) t_start = global_timer_ns();
-          if ((++spins & 63u) == 0u && global_timer_ns() - t_start > kSpinLimitNs) {
+          if ((++spins & 63u) == 0u && global_timer_ns() - t_start > spin_limit_ns) {
             record_error(err, MOE_DEVERR_SCAN_TIMEOUT);
             break;
           }
@@ -278,10 +278,36 @@ size_t histogram_scan_workspace_bytes(int T, int k, int E) {
   return align256(256 + (size_t)C * E * 4) + align256((size_t)T * k * 4);
 }
 
+// The kernels of moe_histogram_scan.  first_ticket > 0 and spin_limit_ns: the diagnostic
+// form of moe_scan_wait_check (chunks 0 .. first_ticket - 1 never run, so the look-back of
+// every later chunk waits for words nobody publishes, until spin_limit_ns).
+static moe_status run_histogram_scan(const int32_t* topk_idx, const float* topk_gate, int T, int k, int E,
+                                     int capacity, int32_t* counts, int32_t* kept, int32_t* offsets,
+                                     int32_t* row_of, int32_t* token_of_row, float* gate_of_row, long long rows_max,
+                                     void* ws, cudaStream_t s, unsigned first_ticket,
+                                     unsigned long long spin_limit_ns);
+
 moe_status launch_histogram_scan(const int32_t* topk_idx, const float* topk_gate, int T, int k,
                                  int E, int capacity, int32_t* counts, int32_t* kept,
                                  int32_t* offsets, int32_t* row_of, int32_t* token_of_row,
                                  float* gate_of_row, long long rows_max, void* ws, cudaStream_t s) {
+  return run_histogram_scan(topk_idx, topk_gate, T, k, E, capacity, counts, kept, offsets, row_of, token_of_row,
+                            gate_of_row, rows_max, ws, s, 0u, kSpinLimitNs);
+}
+
+moe_status launch_scan_wait_check(const int32_t* topk_idx, const float* topk_gate, int T, int k, int E,
+                                  int capacity, int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* row_of,
+                                  int32_t* token_of_row, float* gate_of_row, long long rows_max, void* ws,
+                                  unsigned long long wait_ns, cudaStream_t s) {
+  return run_histogram_scan(topk_idx, topk_gate, T, k, E, capacity, counts, kept, offsets, row_of, token_of_row,
+                            gate_of_row, rows_max, ws, s, 1u, wait_ns);
+}
+
+static moe_status run_histogram_scan(const int32_t* topk_idx, const float* topk_gate, int T, int k, int E,
+                                     int capacity, int32_t* counts, int32_t* kept, int32_t* offsets,
+                                     int32_t* row_of, int32_t* token_of_row, float* gate_of_row, long long rows_max,
+                                     void* ws, cudaStream_t s, unsigned first_ticket,
+                                     unsigned long long spin_limit_ns) {
   if (T == 0) {
     moe_status st = cuda_status(cudaMemsetAsync(counts, 0, (size_t)E * 4, s));
     if (st == MOE_OK) st = cuda_status(cudaMemsetAsync(kept, 0, (size_t)E * 4, s));
@@ -291,6 +317,10 @@ moe_status launch_histogram_scan(const int32_t* topk_idx, const float* topk_gate
   ScanWs w = carve(ws, T, k, E);
   moe_status st = cuda_status(cudaMemsetAsync(ws, 0, w.clear_bytes, s));
   if (st != MOE_OK) return st;
+  if (first_ticket) {   // the ticket counter starts past the withheld chunks (a small value: one byte)
+    st = cuda_status(cudaMemsetAsync(w.ticket, (int)first_ticket, 1, s));
+    if (st != MOE_OK) return st;
+  }
   const int nchunks = (T + kChunk - 1) / kChunk;
   const size_t smem = rank_smem_bytes(k, E);
   // raise the limit once per device to the largest size any supported (k, E) needs, so
@@ -300,7 +330,7 @@ moe_status launch_histogram_scan(const int32_t* topk_idx, const float* topk_gate
   if (st != MOE_OK) return st;
   int* err = err_ptr();
   rank_kernel<<<nchunks, kRankThreads, smem, s>>>(topk_idx, T, k, E, capacity, nchunks, w.ticket, w.status,
-                                                 w.rank, counts, kept, offsets, err);
+                                                 w.rank, counts, kept, offsets, spin_limit_ns, err);
   st = check_launch();
   if (st != MOE_OK) return st;
   const long long A = (long long)T * k;

@@ -55,6 +55,8 @@ _SIGNATURES = {
                                   _c_void_p, _c_void_p, _c_void_p, _c_void_p, _size, _c_void_p]),
     "moe_histogram_scan_noalloc": (_i32, [_c_void_p, _c_void_p, _i32, _i32, _i32, _i32, _c_void_p, _c_void_p,
                                           _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p]),
+    "moe_scan_wait_check": (_i32, [_c_void_p, _c_void_p, _i32, _i32, _i32, _i32, _c_void_p, _c_void_p, _c_void_p,
+                                   _c_void_p, _c_void_p, _c_void_p, ctypes.c_uint64, _c_void_p, _size, _c_void_p]),
     "moe_permute": (_i32, [_c_void_p, _i32, _i32, _i32, _i32, _c_void_p, _i64, _c_void_p, _c_void_p]),
     "moe_expert_gate_up": (_i32, [_c_void_p, _i32, _c_void_p, _i32, _i32, _i32, _i64, _c_void_p, _c_void_p,
                                   _c_void_p]),
@@ -367,6 +369,27 @@ def moe_histogram_scan_noalloc(topk_idx, topk_gate, E: int, capacity: int, count
         _check("moe_histogram_scan_noalloc", lib().moe_histogram_scan_noalloc(
             _p(topk_idx), _p(topk_gate), T, k, E, capacity, _p(counts), _p(kept), _p(offsets), _p(row_of),
             _p(token_of_row), _p(gate_of_row), _stream(stream)))
+
+
+def moe_scan_wait_check(topk_idx, topk_gate, E: int, wait_ns: int, capacity: int = -1, stream=None):
+    """Diagnostic: the histogram/scan with its first chunk withheld, so that every look-back
+    wait runs out after wait_ns and records MOE_DEVERR_SCAN_TIMEOUT (read it with
+    moe_get_device_error).  The outputs are not meaningful."""
+    T, k = topk_idx.shape
+    _need(topk_idx, "topk_idx", torch.int32)
+    _need(topk_gate, "topk_gate", torch.float32, (T, k))
+    dev = topk_idx.device
+    rows = max(moe_rows_max(T, E, k, capacity), 1)
+    i32 = torch.int32
+    counts, kept = torch.empty(E, dtype=i32, device=dev), torch.empty(E, dtype=i32, device=dev)
+    offsets, row_of = torch.empty(E + 1, dtype=i32, device=dev), torch.empty((T, k), dtype=i32, device=dev)
+    token_of_row = torch.empty(rows, dtype=i32, device=dev)
+    gate_of_row = torch.empty(rows, dtype=torch.float32, device=dev)
+    nb = int(lib().moe_histogram_scan_workspace_bytes(T, k, E))
+    ws = torch.empty(max(nb, 16), dtype=torch.uint8, device=dev)
+    _check("moe_scan_wait_check", lib().moe_scan_wait_check(
+        _p(topk_idx), _p(topk_gate), T, k, E, capacity, _p(counts), _p(kept), _p(offsets), _p(row_of),
+        _p(token_of_row), _p(gate_of_row), int(wait_ns), _p(ws), nb, _stream(stream)))
 
 
 def moe_permute(x, row_of, rows_max: int, x_perm=None, stream=None):

@@ -298,3 +298,14 @@ def test_capacity_and_rows_max_agree_with_the_oracle_on_random_sizes(L):
         plan = O.dispatch_plan(idx, np.ones((T, k)), E, cap)
         assert int(plan["offsets"][-1]) <= L.moe_rows_max(T, E, k, cap)
         assert L.moe_rows_max(T, E, k, cap) == (T * k if cap < 0 else min(T * k, E * cap))
+
+
+def test_scan_wait_check_host_validation(L):
+    f = L.moe_scan_wait_check          # (idx, gate, T, k, E, cap, counts, kept, offs, row_of, tor, gor, ns, ws, wsb, s)
+
+    def call(T=1000, ns=10 ** 6, ws=FAKE, wsb=1 << 30, ptr=FAKE):
+        return f(ptr, FAKE, T, 4, 64, -1, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ns, ws, wsb, NUL)
+    assert call(T=256) == 1                      # no chunk after the withheld first one
+    assert call(ns=999) == 1 and call(ns=2 * 10 ** 9) == 1
+    assert call(ptr=NUL) == 1
+    assert call(ws=NUL) == 3 and call(wsb=16) == 3
