@@ -16,6 +16,7 @@
  *   moe_grouped_ffn      the two GEMMs above back to back
  *   moe_combine          gate-weighted sum of each token's rows (+ shared expert)
  *   moe_expert_down_combine  the down GEMM with the combine fused into its epilogue
+ *   moe_expert_gate_up_fp4 / moe_expert_down_fp4  the expert GEMMs with 4-bit weights
  *   moe_round_output     the combine's final rounding of an fp32 sum to bf16
  *   moe_router_stats     per-expert load, aux loss, z-loss, drops, imbalance
  *
@@ -508,6 +509,36 @@ MOE_API moe_status moe_quantize_fp4_host(const float* W, int64_t rows, int64_t K
 MOE_API moe_status moe_dequantize_fp4_host(const uint8_t* codes, const uint8_t* scales,
                      const float* tensor_scale, int64_t rows, int64_t K, int32_t fmt,
                      float* W, int32_t threads);
+
+/* ------------------------------------------------------------------------------------
+ * moe_expert_gate_up_fp4 / moe_expert_down_fp4 -- the grouped expert GEMMs with 4-bit
+ * expert weights (weight-only: activations, H and the gated rows stay as in the bf16
+ * calls).  [Handbook-Digest] "已确认", bullet "量化与推理" (routed experts in MXFP4;
+ * NVFP4 with key layers kept in BF16).
+ * The weights are the packed form of moe_quantize_fp4_host, in device memory:
+ *   codes         (device) [rows, K/2] bytes (element 2j in the low nibble of byte j)
+ *   scales        (device) [rows, K / moe_fp4_block_size(fmt)] bytes
+ *   tensor_scale  (device) [E] fp32, expert e's NVFP4 tensor scale (quantize each expert
+ *                 separately); NULL for MXFP4
+ *   gate/up: rows = E * 2F (expert e's F gate rows, then its F up rows), K = d;
+ *   down:    rows = E * d, K = F.
+ * Every weight is code value x block scale (x tensor scale).  The kernel expands each
+ * stage of codes to bf16 in shared memory (exact: at most 6 significant bits) and runs
+ * the bf16 tensor-core MMAs with fp32 accumulation; the NVFP4 tensor scale multiplies the
+ * accumulators.  Weight-major tiles (256 weight rows x the expert's tokens), whatever the
+ * group sizes.  Other arguments as moe_expert_gate_up / moe_expert_down (bf16 rows only).
+ * Errors: INVALID_ARG for a null pointer, a bad format, a missing NVFP4 tensor scale or a
+ * negative size; UNSUPPORTED for E > 1024, d or F not a multiple of 64, fp32 activations
+ * or an unaligned pointer.
+ * ---------------------------------------------------------------------------------- */
+MOE_API moe_status moe_expert_gate_up_fp4(const void* x_rows, const int32_t* offsets, int32_t E,
+                     int32_t d, int32_t F, int64_t rows_max, const uint8_t* codes,
+                     const uint8_t* scales, int32_t fmt, const float* tensor_scale, void* h,
+                     void* stream);
+MOE_API moe_status moe_expert_down_fp4(const void* h, const int32_t* offsets, int32_t E, int32_t d,
+                     int32_t F, int64_t rows_max, const uint8_t* codes, const uint8_t* scales,
+                     int32_t fmt, const float* tensor_scale, const float* gate_of_row,
+                     int32_t y_dtype, void* y_rows, void* stream);
 
 /* Largest workspace any of the calls above needs for these sizes, for every call with
  * at most T tokens (each size query covers the batches below its T). */

@@ -167,6 +167,52 @@ def nvfp4_dequantize(s_t: float, s_b, codes, block: int = NV_BLOCK) -> np.ndarra
     return out
 
 
+# ---------------------------------------------------------------------------
+# The packed layout (what a 4-bit expert GEMM reads): codes [rows, K/2] bytes with element
+# 2j in the low nibble of byte j; scale bytes [rows, K/block]: E8M0 (MXFP4, the byte E + 127)
+# or FP8 E4M3 (NVFP4); and, for NVFP4, one fp32 tensor scale.
+# ---------------------------------------------------------------------------
+def e4m3_decode(byte: int) -> float:
+    """Value of an FP8 E4M3 byte s|eeee|mmm: normal (e > 0) 2^(e-7) (1 + m/8), subnormal
+    (e = 0) m 2^-9; exponent 15 with mantissa 7 is NaN (never written by the quantizer)."""
+    s, e, m = (byte >> 7) & 1, (byte >> 3) & 15, byte & 7
+    if e == 15 and m == 7:
+        return math.nan
+    mag = m * 2.0 ** -9 if e == 0 else 2.0 ** (e - 7) * (1.0 + m / 8.0)
+    return -mag if s else mag
+
+
+def pack_codes(codes) -> np.ndarray:
+    """Element codes [rows, K] -> bytes [rows, K/2], element 2j in the low nibble of byte j."""
+    c = np.asarray(codes, np.uint8)
+    return (c[:, 0::2] | (c[:, 1::2] << 4)).astype(np.uint8)
+
+
+def decode_packed(codes, scales, fmt: str, tensor_scale: float = 1.0) -> np.ndarray:
+    """Dequantized weights [rows, K] (float64) of the packed layout: code value x block
+    scale (x tensor scale for NVFP4).  Table-driven: the 16 code values from e2m1_decode and
+    the 256 scale values from their byte layouts."""
+    codes = np.asarray(codes, np.uint8)
+    scales = np.asarray(scales, np.uint8)
+    rows, half = codes.shape
+    K = 2 * half
+    block = MX_BLOCK if fmt == "mxfp4" else NV_BLOCK
+    if scales.shape != (rows, K // block):
+        raise ValueError("scales must be [rows, K / block]")
+    vals = np.array([e2m1_decode(c) for c in range(16)], np.float64)
+    if fmt == "mxfp4":
+        svals = np.array([2.0 ** (b - 127) for b in range(256)], np.float64)
+    elif fmt == "nvfp4":
+        svals = np.array([e4m3_decode(b) for b in range(256)], np.float64)
+    else:
+        raise ValueError(fmt)
+    el = np.empty((rows, K), np.uint8)
+    el[:, 0::2] = codes & 15
+    el[:, 1::2] = codes >> 4
+    W = vals[el] * np.repeat(svals[scales], block, axis=1)
+    return W * (float(tensor_scale) if fmt == "nvfp4" else 1.0)
+
+
 def fake_quantize(W, fmt: str) -> np.ndarray:
     """W -> its dequantized 4-bit form ("mxfp4" or "nvfp4"), the weights the experts run on (R26)."""
     if fmt == "mxfp4":

@@ -331,6 +331,37 @@ moe_status moe_grouped_ffn(const void* x_rows, int32_t dtype, const int32_t* off
   return moe_expert_down(h, dtype, offsets, E, d, F, rows_max, W_dn, gate_of_row, y_dtype, y_rows, stream);
 }
 
+static moe_status check_fp4(const void* a, const int32_t* offsets, int32_t E, int32_t d, int32_t F, int64_t rows_max,
+                            const uint8_t* codes, const uint8_t* scales, int32_t fmt, const float* tensor_scale,
+                            const void* out) {
+  if (E < 1 || d < 1 || F < 1 || rows_max < 0 || fp4_block(fmt) < 0) return MOE_ERR_INVALID_ARG;
+  if (E > kMaxE || d % 64 != 0 || F % 64 != 0 || rows_max >= (1LL << 31)) return MOE_ERR_UNSUPPORTED;
+  if (!offsets || !codes || !scales || (fmt == MOE_FP4_NV && !tensor_scale)) return MOE_ERR_INVALID_ARG;
+  if (rows_max > 0 && (!a || !out)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(a) || !aligned16(codes) || !aligned16(scales) || !aligned16(out)) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+moe_status moe_expert_gate_up_fp4(const void* x_rows, const int32_t* offsets, int32_t E, int32_t d, int32_t F,
+                                  int64_t rows_max, const uint8_t* codes, const uint8_t* scales, int32_t fmt,
+                                  const float* tensor_scale, void* h, void* stream) {
+  moe_status st = check_fp4(x_rows, offsets, E, d, F, rows_max, codes, scales, fmt, tensor_scale, h);
+  if (st != MOE_OK || rows_max == 0) return st;
+  return launch_gate_up_fp4(x_rows, offsets, E, d, F, rows_max, codes, scales, fmt, tensor_scale, h, S(stream));
+}
+
+moe_status moe_expert_down_fp4(const void* h, const int32_t* offsets, int32_t E, int32_t d, int32_t F,
+                               int64_t rows_max, const uint8_t* codes, const uint8_t* scales, int32_t fmt,
+                               const float* tensor_scale, const float* gate_of_row, int32_t y_dtype, void* y_rows,
+                               void* stream) {
+  moe_status st = check_fp4(h, offsets, E, d, F, rows_max, codes, scales, fmt, tensor_scale, y_rows);
+  if (st != MOE_OK) return st;
+  if (!dtype_ok(y_dtype)) return MOE_ERR_INVALID_ARG;
+  if (rows_max == 0) return MOE_OK;
+  return launch_down_fp4(h, offsets, E, d, F, rows_max, codes, scales, fmt, tensor_scale, gate_of_row, y_dtype,
+                         y_rows, S(stream));
+}
+
 moe_status moe_expert_down_combine(const void* h, int32_t dtype, const int32_t* offsets, int32_t E, int32_t d,
                                    int32_t F, int64_t rows_max, const void* W_dn, const float* gate_of_row,
                                    const int32_t* token_of_row, int32_t T, int32_t accumulate, float* y,

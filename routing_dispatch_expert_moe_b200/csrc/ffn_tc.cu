@@ -78,10 +78,6 @@ __device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
   asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
-// Orders generic-proxy shared-memory writes this thread has observed (here: other
-// threads' cp.async copies, acquired through an mbarrier) before its later async-proxy
-// accesses (the tensor cores read operands through the async proxy).
-__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 // Output column tiles per row tile: 128 H features per gate/up tile (128 gate + 128 up
 // accumulator columns), 256 outputs per down tile.

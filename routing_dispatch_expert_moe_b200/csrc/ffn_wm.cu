@@ -109,6 +109,49 @@ __device__ __forceinline__ void stage_store32_t(uint8_t* stage, const float (&v)
   __syncwarp();
 }
 
+// One tile's epilogue for one warp: features col0 .. col0+31 (its TMEM lanes) of the tile's
+// tokens, 32 tokens per tcgen05.ld.  wscale multiplies every accumulator (the 4-bit
+// weights' per-tensor scale; 1 for bf16 weights).
+//   MODE 0: H[token][f] = silu(wscale g) * (wscale u), bf16;
+//   MODE 1: y[token][n] = gate_of_row[token] * wscale * acc.
+template <int MODE, typename OutT>
+__device__ __forceinline__ void wm_epilogue_tile(uint32_t taddr, uint8_t* stage, int lane, const TileCoord& tc,
+                                                 int rank, int q, int d, int F, float wscale,
+                                                 const float* __restrict__ gate_of_row, OutT* __restrict__ out) {
+  const int col0 = tc.n_tile * 256 + rank * kWRows + q * 32;   // this warp's first feature
+  const int chunks = (tc.rows + 31) / 32;
+#pragma unroll 1
+  for (int c = 0; c < chunks; ++c) {
+    const long long r0 = (long long)tc.row0 + c * 32;
+    const int rv = min(32, tc.rows - c * 32);
+    float h[32];
+    if constexpr (MODE == 0) {
+      uint32_t g[32], u[32];
+      tmem_ld32(taddr + c * 32, g);
+      tmem_ld32(taddr + 128 + c * 32, u);
+      tmem_wait_ld();
+      tmem_regs_ready(g);
+      tmem_regs_ready(u);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float gi = __uint_as_float(g[i]) * wscale;
+        // fast exp / divide: H is rounded to bf16 next, far coarser than their error
+        h[i] = __fdividef(gi, 1.f + __expf(-gi)) * (__uint_as_float(u[i]) * wscale);
+      }
+      stage_store32_t<OutT>(stage, h, lane, out, r0, rv, F, col0, F);
+    } else {
+      uint32_t v[32];
+      tmem_ld32(taddr + c * 32, v);
+      tmem_wait_ld();
+      tmem_regs_ready(v);
+      const float gs = ((gate_of_row && lane < rv) ? __ldg(gate_of_row + r0 + lane) : 1.f) * wscale;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) h[i] = __uint_as_float(v[i]) * __shfl_sync(0xffffffffu, gs, i);
+      stage_store32_t<OutT>(stage, h, lane, out, r0, rv, d, col0, d);
+    }
+  }
+}
+
 template <int MODE, typename OutT>
 __global__ void __launch_bounds__(WmCfg<MODE>::threads, 1)
 grouped_gemm_wm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
@@ -247,38 +290,7 @@ grouped_gemm_wm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
       __syncwarp();
       tc_fence_after();
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * 256);
-      const int col0 = tc.n_tile * 256 + (int)rank * kWRows + q * 32;   // this warp's first feature
-      const int chunks = (tc.rows + 31) / 32;
-#pragma unroll 1
-      for (int c = 0; c < chunks; ++c) {
-        const long long r0 = (long long)tc.row0 + c * 32;
-        const int rv = min(32, tc.rows - c * 32);
-        float h[32];
-        if constexpr (MODE == 0) {
-          uint32_t g[32], u[32];
-          tmem_ld32(taddr + c * 32, g);
-          tmem_ld32(taddr + 128 + c * 32, u);
-          tmem_wait_ld();
-          tmem_regs_ready(g);
-          tmem_regs_ready(u);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float gi = __uint_as_float(g[i]);
-            // fast exp / divide: H is rounded to bf16 next, far coarser than their error
-            h[i] = __fdividef(gi, 1.f + __expf(-gi)) * __uint_as_float(u[i]);
-          }
-          stage_store32_t<OutT>(stage, h, lane, out, r0, rv, F, col0, F);
-        } else {
-          uint32_t v[32];
-          tmem_ld32(taddr + c * 32, v);
-          tmem_wait_ld();
-          tmem_regs_ready(v);
-          const float gs = (gate_of_row && lane < rv) ? __ldg(gate_of_row + r0 + lane) : 1.f;
-#pragma unroll
-          for (int i = 0; i < 32; ++i) h[i] = __uint_as_float(v[i]) * __shfl_sync(0xffffffffu, gs, i);
-          stage_store32_t<OutT>(stage, h, lane, out, r0, rv, d, col0, d);
-        }
-      }
+      wm_epilogue_tile<MODE, OutT>(taddr, stage, lane, tc, (int)rank, q, d, F, 1.f, gate_of_row, out);
       tc_fence_before();
       mbar_arrive_cluster(map_to_rank(bar_tempty + 8 * acc, 0));
     }
@@ -290,6 +302,321 @@ grouped_gemm_wm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kWTmemCols) : "memory");
   }
+}
+
+// =====================================================================================
+// 4-bit expert weights (weight-only): the same weight-major tiles, with each stage's
+// weight blocks arriving as packed E2M1 codes (a quarter of the bytes) and expanded to
+// bf16 in shared memory by four converter warps before the MMAs read them.
+//
+// Handbook digest (agihunt.info), "已确认", bullet "量化与推理": routed experts in MXFP4
+// (Kimi K3), NVFP4 training with key layers kept in BF16 (Nemotron 3).  The activations
+// stay bf16, and a kind::f16 MMA multiplies bf16 by bf16, so the weights are expanded:
+//   value = e2m1(code) * block scale, exact in bf16 (at most 2 significant bits times a
+//   power of two (MXFP4, E8M0 scale) or times an E4M3 scale of at most 4 bits (NVFP4));
+//   the NVFP4 per-tensor fp32 scale multiplies the fp32 accumulator in the epilogue.
+// Weight layout (as moe_quantize_fp4_host writes it): codes [rows, K/2] bytes, element 2j
+// in the low nibble of byte j; scales [rows, K/block] bytes (E8M0 for MXFP4, block 32;
+// E4M3 for NVFP4, block 16); K a multiple of 64.
+//
+// Per stage and CTA: TMA brings the codes of its weight rows (128 rows x 32 bytes per
+// block) and its token rows; a converter thread owns one weight row of each block: it
+// reads its row's 2 (MX) or 4 (NV) scale bytes for the k-block from global memory, looks
+// each code byte up in a 256-entry table of bf16 pairs, scales the pair and writes 16-byte
+// chunks into the 128-byte-swizzled operand layout the MMA reads (chunk c of row r at
+// r * 128 + ((c ^ (r & 7)) * 16)).  Barriers per stage: packed[s] (this CTA's TMA bytes),
+// full[s] on the even CTA (the 2 x 128 converter threads, after a proxy fence), empty[s]
+// (the MMAs' completion, both CTAs).
+// =====================================================================================
+template <int MODE>
+struct Wm4Cfg {
+  static constexpr int NT = WmCfg<MODE>::NT;
+  static constexpr int a_blocks = WmCfg<MODE>::a_blocks;
+  static constexpr int b_bytes = WmCfg<MODE>::b_bytes;
+  static constexpr int packed_block = kWRows * BK / 2;          // 4 KB of codes per weight block
+  static constexpr int stage_bytes = a_blocks * kWBlock + b_bytes + a_blocks * packed_block;
+  static constexpr int stages = MODE == 0 ? 4 : 5;
+  static constexpr int epi_warps = 4, cvt_warps = 4;
+  static constexpr int threads = 64 + 32 * (epi_warps + cvt_warps);
+  static constexpr int bars = stages * stage_bytes;
+  static constexpr int nbars = 3 * stages + 4 + 1;
+  static constexpr int misc = bars + nbars * 8;
+  static constexpr int lut = (misc + 16 + 15) / 16 * 16;       // uint32 [256]: code byte -> bf16 pair
+  static constexpr int tiles = lut + 256 * 4;
+  static constexpr int sh32 = tiles + (kWMaxE + 1) * 4;
+  static constexpr int stage = (sh32 + 32 * 4 + 127) / 128 * 128;
+  static constexpr int end = stage + epi_warps * kStageWarpBytes;
+  static constexpr size_t smem = end + 1024;
+  static_assert(smem <= 232448, "shared memory per CTA");
+  static_assert((a_blocks * kWBlock + b_bytes) % 1024 == 0 && stage_bytes % 1024 == 0, "swizzle alignment");
+};
+
+// bf16 bits of an E2M1 code: sign, then 0 / 0.5 (exponent field 0) or 2^(e-1) (1 + m/2).
+__device__ __forceinline__ uint32_t e2m1_bf16_bits(uint32_t c) {
+  const uint32_t e = (c >> 1) & 3u, m = c & 1u;
+  const uint32_t mag = e ? (((e + 126u) << 7) | (m << 6)) : (m ? 0x3F00u : 0u);
+  return ((c & 8u) << 12) | mag;
+}
+
+// bf16 of a block scale byte: E8M0 (2^(b - 127); b = 0 is 2^-127, a bf16 subnormal) or
+// E4M3 (normal 2^(e-7) (1 + m/8), subnormal m 2^-9).  Both exact in bf16.
+template <int FMT>
+__device__ __forceinline__ uint32_t scale_bf16_bits(uint32_t b) {
+  if (FMT == MOE_FP4_MX) return b ? (b << 7) : 0x0040u;
+  const uint32_t e = (b >> 3) & 15u, m = b & 7u;
+  if (e) return ((e + 120u) << 7) | (m << 4);
+  const __nv_bfloat16 v = __float2bfloat16_rn((float)m * 0.001953125f);
+  return (uint32_t)(*reinterpret_cast<const uint16_t*>(&v));
+}
+
+// Expands one 128 x 64 block row of codes into bf16: 32 code bytes at src, scale bytes
+// packed little-endian in sc (2 for MX: chunks 0-3 and 4-7; 4 for NV: chunk pairs).
+template <int FMT>
+__device__ __forceinline__ void convert_row(const uint8_t* src, uint32_t sc, const uint32_t* lut, uint8_t* dst_block,
+                                            int r) {
+  const uint4 c0 = *reinterpret_cast<const uint4*>(src);
+  const uint4 c1 = *reinterpret_cast<const uint4*>(src + 16);
+  const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {                 // chunk c: elements 8c .. 8c+7 (code bytes 4c .. 4c+3)
+    const uint32_t sb = FMT == MOE_FP4_MX ? scale_bf16_bits<FMT>((sc >> (8 * (c >> 2))) & 0xffu)
+                                          : scale_bf16_bits<FMT>((sc >> (8 * (c >> 1))) & 0xffu);
+    const __nv_bfloat162 s2 = __halves2bfloat162(*reinterpret_cast<const __nv_bfloat16*>(&sb),
+                                                 *reinterpret_cast<const __nv_bfloat16*>(&sb));
+    uint32_t o[4];
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const uint32_t pair = lut[(w[c] >> (8 * b)) & 0xffu];
+      __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&pair);
+      v = __hmul2(v, s2);                       // exact: at most 6 significant bits
+      o[b] = *reinterpret_cast<uint32_t*>(&v);
+    }
+    *reinterpret_cast<uint4*>(dst_block + r * 128 + ((c ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+template <int MODE, int FMT, typename OutT>
+__global__ void __launch_bounds__(Wm4Cfg<MODE>::threads, 1)
+grouped_gemm_wm4_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmX,
+                        const uint8_t* __restrict__ scales, const float* __restrict__ tensor_scale,
+                        const int32_t* __restrict__ offsets, int E, int K, int d, int F, long long rows_max,
+                        const float* __restrict__ gate_of_row, OutT* __restrict__ out, int* err) {
+  using C = Wm4Cfg<MODE>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int* tile_start = reinterpret_cast<int*>(smem + C::tiles);
+  int* sh32 = reinterpret_cast<int*>(smem + C::sh32);
+  uint32_t* lut = reinterpret_cast<uint32_t*>(smem + C::lut);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::misc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::misc + 4);
+  const uint32_t rank = cluster_ctarank();
+  const int cid = (int)(blockIdx.x >> 1), ncl = (int)(gridDim.x >> 1);
+
+  const int m_tiles = wm_m_tiles<MODE>(F, d);
+  build_tile_starts(offsets, E, C::NT, m_tiles, rows_max, tile_start, sh32, err);
+  const int total = tile_start[E];
+  if (cid >= total) return;   // both CTAs of the pair see the same cid: uniform, nothing allocated
+
+  const uint32_t bar_packed = sb + C::bars;
+  const uint32_t bar_full = bar_packed + 8 * C::stages;
+  const uint32_t bar_empty = bar_full + 8 * C::stages;
+  const uint32_t bar_tfull = bar_empty + 8 * C::stages;
+  const uint32_t bar_tempty = bar_tfull + 16;
+  const uint32_t bar_fin = bar_tempty + 16;
+  auto a_off = [&](int s, int a) { return s * C::stage_bytes + a * kWBlock; };
+  auto b_off = [&](int s) { return s * C::stage_bytes + C::a_blocks * kWBlock; };
+  auto p_off = [&](int s, int a) { return s * C::stage_bytes + C::a_blocks * kWBlock + C::b_bytes + a * C::packed_block; };
+
+  for (int i = threadIdx.x; i < 256; i += blockDim.x)
+    lut[i] = e2m1_bf16_bits(i & 15u) | (e2m1_bf16_bits(i >> 4) << 16);   // low nibble = lower element
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::stages; ++s) {
+      mbar_init(bar_packed + 8 * s, 1);
+      mbar_init(bar_full + 8 * s, 2 * 32 * C::cvt_warps);
+      mbar_init(bar_empty + 8 * s, 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(bar_tfull + 8 * a, 1);
+      mbar_init(bar_tempty + 8 * a, 2 * 32 * C::epi_warps);
+    }
+    mbar_init(bar_fin, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(kWTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int KB = K / BK;                                     // K is a multiple of 64
+  constexpr int kBlockElems = FMT == MOE_FP4_MX ? 32 : 16;
+  const long long scale_ld = K / kBlockElems;                // scale bytes per weight row
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer (both CTAs)
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int last_phase[C::stages];
+#pragma unroll
+      for (int s = 0; s < C::stages; ++s) last_phase[s] = -1;
+      bool ok = true;
+      for (int tile = cid; ok && tile < total; tile += ncl) {
+        const TileCoord tc = tile_coord(tile_start, offsets, E, C::NT, tile);
+        const int n = wm_n<MODE>(tc.rows);
+        const int w_row = MODE == 0 ? tc.e * 2 * F + tc.n_tile * 256 + (int)rank * kWRows
+                                    : tc.e * d + tc.n_tile * 256 + (int)rank * kWRows;
+        const int x_row = tc.row0 + (int)rank * (n / 2);
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1u, abort_flag, err)) { ok = false; break; }
+          const uint32_t pk = bar_packed + 8 * stage;
+          mbar_expect_tx(pk, (uint32_t)(C::a_blocks * C::packed_block + C::b_bytes));
+          tma_load_2d(sb + (uint32_t)p_off(stage, 0), &tmC, pk, kb * (BK / 2), w_row);
+          if (MODE == 0) tma_load_2d(sb + (uint32_t)p_off(stage, 1), &tmC, pk, kb * (BK / 2), w_row + F);
+          tma_load_2d(sb + (uint32_t)b_off(stage), &tmX, pk, kb * BK, x_row);
+          last_phase[stage] = (int)phase;
+          if (++stage == C::stages) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) {
+        for (int s = 0; s < C::stages; ++s)
+          if (last_phase[s] >= 0) mbar_wait_drain(bar_packed + 8 * s, (uint32_t)last_phase[s], err);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (even CTA)
+    if (lane == 0 && rank == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      for (int tile = cid; ok && tile < total; tile += ncl, ++it) {
+        const int acc = it & 1;
+        const uint32_t acc_phase = (uint32_t)(it >> 1) & 1u;
+        const TileCoord tc = tile_coord(tile_start, offsets, E, C::NT, tile);
+        const uint32_t idesc = make_idesc(2 * kWRows, wm_n<MODE>(tc.rows));
+        if (!mbar_wait(bar_tempty + 8 * acc, acc_phase ^ 1u, abort_flag, err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * 256);
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag, err)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t bdesc = sw128_desc(sb + (uint32_t)b_off(stage));
+          const uint64_t adesc0 = sw128_desc(sb + (uint32_t)a_off(stage, 0));
+          const uint64_t adesc1 = sw128_desc(sb + (uint32_t)a_off(stage, MODE == 0 ? 1 : 0));
+#pragma unroll
+          for (int kk = 0; kk < BK / UMMA_K; ++kk) {
+            const uint32_t accumulate = (kb | kk) != 0 ? 1u : 0u;
+            umma_bf16_pair(d_tmem, adesc0 + 2 * kk, bdesc + 2 * kk, idesc, accumulate);
+            if (MODE == 0) umma_bf16_pair(d_tmem + 128, adesc1 + 2 * kk, bdesc + 2 * kk, idesc, accumulate);
+          }
+          umma_commit_pair_both(bar_empty + 8 * stage);
+          if (++stage == C::stages) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma_commit_pair_both(bar_tfull + 8 * acc);
+      }
+      umma_commit_pair(bar_fin);
+      mbar_wait_drain(bar_fin, 0, err);
+    }
+  } else if (warp < 2 + C::epi_warps) {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int q = warp & 3;
+    uint8_t* stage = smem + C::stage + (warp - 2) * kStageWarpBytes;
+    int it = 0;
+    for (int tile = cid; tile < total; tile += ncl, ++it) {
+      const TileCoord tc = tile_coord(tile_start, offsets, E, C::NT, tile);
+      const int acc = it & 1;
+      const uint32_t acc_phase = (uint32_t)(it >> 1) & 1u;
+      const bool got = mbar_wait(bar_tfull + 8 * acc, acc_phase, abort_flag, err);
+      if (!__all_sync(0xffffffffu, got)) break;
+      __syncwarp();
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * 256);
+      const float ws = tensor_scale ? __ldg(tensor_scale + tc.e) : 1.f;
+      wm_epilogue_tile<MODE, OutT>(taddr, stage, lane, tc, (int)rank, q, d, F, ws, gate_of_row, out);
+      tc_fence_before();
+      mbar_arrive_cluster(map_to_rank(bar_tempty + 8 * acc, 0));
+    }
+  } else {
+    // ------------------------------------------------------------ converters (both CTAs)
+    const int r = threadIdx.x - 64 - 32 * C::epi_warps;     // the weight row of each block it expands
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int tile = cid; tile < total; tile += ncl) {
+      const TileCoord tc = tile_coord(tile_start, offsets, E, C::NT, tile);
+      const long long w_row = MODE == 0 ? (long long)tc.e * 2 * F + tc.n_tile * 256 + (int)rank * kWRows + r
+                                        : (long long)tc.e * d + tc.n_tile * 256 + (int)rank * kWRows + r;
+      // rows past the weight matrix (the last tile's padding) read no scales
+      const long long rows_total = MODE == 0 ? (long long)E * 2 * F : (long long)E * d;
+      bool ok = true;
+      for (int kb = 0; kb < KB; ++kb) {
+        uint32_t sc[2] = {0u, 0u};
+#pragma unroll
+        for (int a = 0; a < C::a_blocks; ++a) {
+          const long long row = w_row + (a ? F : 0);
+          if (row < rows_total) {
+            const uint8_t* p = scales + row * scale_ld + (long long)kb * (BK / kBlockElems);
+            sc[a] = FMT == MOE_FP4_MX ? (uint32_t)__ldg(reinterpret_cast<const uint16_t*>(p))
+                                      : __ldg(reinterpret_cast<const uint32_t*>(p));
+          }
+        }
+        const bool got = mbar_wait(bar_packed + 8 * stage, phase, abort_flag, err);
+        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+#pragma unroll
+        for (int a = 0; a < C::a_blocks; ++a)
+          convert_row<FMT>(smem + p_off(stage, a) + r * (BK / 2), sc[a], lut, smem + a_off(stage, a), r);
+        fence_proxy_async_smem();                           // the MMAs read these through the async proxy
+        mbar_arrive_cluster(map_to_rank(bar_full + 8 * stage, 0));
+        if (++stage == C::stages) { stage = 0; phase ^= 1u; }
+      }
+      if (!ok) break;
+    }
+  }
+
+  __syncthreads();
+  cluster_sync();                                           // no remote arrive after a CTA exits
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kWTmemCols) : "memory");
+  }
+}
+
+template <int MODE, int FMT, typename OutT>
+moe_status launch_wm4(const CUtensorMap& mc, const CUtensorMap& mx, const uint8_t* scales, const float* tscale,
+                      const int32_t* offsets, int E, int K, int d, int F, long long rows_max, const float* gate_of_row,
+                      void* out, cudaStream_t s) {
+  using C = Wm4Cfg<MODE>;
+  static std::atomic<int> configured[kMaxDevices];
+  const moe_status st = ensure_smem_limit(configured, grouped_gemm_wm4_kernel<MODE, FMT, OutT>, C::smem);
+  if (st != MOE_OK) return st;
+  const long long max_tiles = ((rows_max + C::NT - 1) / C::NT + E) * (long long)wm_m_tiles<MODE>(F, d);
+  int pairs = num_sms() / 2;
+  if (max_tiles < pairs) pairs = (int)max_tiles;
+  if (pairs < 1) pairs = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cfg.blockDim = dim3(C::threads, 1, 1);
+  cfg.dynamicSmemBytes = C::smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cuda_status(cudaLaunchKernelEx(&cfg, grouped_gemm_wm4_kernel<MODE, FMT, OutT>, mc, mx, scales, tscale,
+                                        offsets, E, K, d, F, rows_max, gate_of_row, static_cast<OutT*>(out),
+                                        err_ptr()));
 }
 
 template <int MODE, typename OutT>
@@ -342,6 +669,43 @@ moe_status launch_down_wm(const void* h, const int32_t* offsets, int E, int d, i
   if (!make_map(&mx, h, (unsigned long long)rows_max, F, WmCfg<1>::NT / 2)) return MOE_ERR_UNSUPPORTED;
   if (y_dtype == MOE_F32) return launch_wm<1, float>(mw, mx, offsets, E, F, d, F, rows_max, gate_of_row, y_rows, s);
   return launch_wm<1, __nv_bfloat16>(mw, mx, offsets, E, F, d, F, rows_max, gate_of_row, y_rows, s);
+}
+
+// Gate/up and down with 4-bit weights, weight-major.  Codes [rows, K/2] and scales
+// [rows, K / block] as moe_quantize_fp4_host writes them (rows = E 2F or E d); tensor_scale
+// [E] fp32 per expert (NVFP4) or NULL (MXFP4).  K (d for gate/up, F for down) must be a
+// multiple of 64.
+moe_status launch_gate_up_fp4(const void* x_rows, const int32_t* offsets, int E, int d, int F, long long rows_max,
+                              const uint8_t* codes, const uint8_t* scales, int fmt, const float* tensor_scale,
+                              void* h, cudaStream_t s) {
+  if (rows_max == 0) return MOE_OK;
+  CUtensorMap mc, mx;
+  if (!make_map_u8(&mc, codes, (unsigned long long)E * 2 * F, d / 2, BK / 2, kWRows)) return MOE_ERR_UNSUPPORTED;
+  if (!make_map(&mx, x_rows, (unsigned long long)rows_max, d, WmCfg<0>::NT / 2)) return MOE_ERR_UNSUPPORTED;
+  if (fmt == MOE_FP4_MX)
+    return launch_wm4<0, MOE_FP4_MX, __nv_bfloat16>(mc, mx, scales, nullptr, offsets, E, d, d, F, rows_max, nullptr,
+                                                     h, s);
+  return launch_wm4<0, MOE_FP4_NV, __nv_bfloat16>(mc, mx, scales, tensor_scale, offsets, E, d, d, F, rows_max,
+                                                   nullptr, h, s);
+}
+
+moe_status launch_down_fp4(const void* h, const int32_t* offsets, int E, int d, int F, long long rows_max,
+                           const uint8_t* codes, const uint8_t* scales, int fmt, const float* tensor_scale,
+                           const float* gate_of_row, int y_dtype, void* y_rows, cudaStream_t s) {
+  if (rows_max == 0) return MOE_OK;
+  CUtensorMap mc, mx;
+  if (!make_map_u8(&mc, codes, (unsigned long long)E * d, F / 2, BK / 2, kWRows)) return MOE_ERR_UNSUPPORTED;
+  if (!make_map(&mx, h, (unsigned long long)rows_max, F, WmCfg<1>::NT / 2)) return MOE_ERR_UNSUPPORTED;
+  const float* ts = fmt == MOE_FP4_NV ? tensor_scale : nullptr;
+#define MOE_WM4(FMT, T) \
+  return launch_wm4<1, FMT, T>(mc, mx, scales, ts, offsets, E, F, d, F, rows_max, gate_of_row, y_rows, s)
+  if (fmt == MOE_FP4_MX) {
+    if (y_dtype == MOE_F32) MOE_WM4(MOE_FP4_MX, float);
+    MOE_WM4(MOE_FP4_MX, __nv_bfloat16);
+  }
+  if (y_dtype == MOE_F32) MOE_WM4(MOE_FP4_NV, float);
+  MOE_WM4(MOE_FP4_NV, __nv_bfloat16);
+#undef MOE_WM4
 }
 
 }  // namespace moe

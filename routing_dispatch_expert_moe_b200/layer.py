@@ -39,6 +39,10 @@ class MoEWeights:
     W_gu_s: Optional[torch.Tensor] = None     # [1, 2F_s, d] shared expert
     W_dn_s: Optional[torch.Tensor] = None     # [1, d, F_s]
     W_noise: Optional[torch.Tensor] = None    # [d, E] f32: noise router (routing="noisy")
+    # 4-bit routed experts (moe.Fp4Weights of W_gu and W_dn, e.g. from moe.quantize_experts_fp4):
+    # used in place of W_gu / W_dn by the expert GEMMs (the shared expert stays bf16)
+    W_gu_fp4: Optional[object] = None
+    W_dn_fp4: Optional[object] = None
 
 
 class MoELayer:
@@ -61,6 +65,11 @@ class MoELayer:
         hash_seed) or "noisy" (noisy top-k with weights.W_noise and the standard normal
         draws given to forward; softmax gating).  The fixed rules keep the learned gates
         over the chosen experts; the router statistics always use the router logits."""
+        self.fp4 = weights.W_gu_fp4 is not None
+        if self.fp4 and (weights.W_dn_fp4 is None or combine != "rows" or dispatch != "permute"
+                         or weights.W_gu.dtype != torch.bfloat16):
+            raise ValueError("4-bit experts need both W_gu_fp4 and W_dn_fp4, bf16 activations, "
+                             "combine='rows' and dispatch='permute'")
         if routing not in ("learned", "uniform", "hash", "noisy"):
             raise ValueError(f"routing must be learned, uniform, hash or noisy, got {routing!r}")
         if routing != "learned" and weights.select_bias is not None:
@@ -161,12 +170,20 @@ class MoELayer:
         M.moe_permute(x, self.row_of[:x.shape[0]], self.rows_max, self.x_perm, stream)
 
     def gate_up(self, stream=None):
+        if self.fp4:
+            M.moe_expert_gate_up_fp4(self.x_perm, self.offsets, self.w.W_gu_fp4, self.E, self.F, self.rows_max,
+                                     self.h, stream)
+            return
         M.moe_expert_gate_up(self.x_perm, self.offsets, self.w.W_gu, self.rows_max, self.h, stream)
 
     def gate_up_gather(self, x, stream=None):
         M.moe_expert_gate_up_gather(x, self.token_of_row, self.offsets, self.w.W_gu, self.rows_max, self.h, stream)
 
     def down(self, stream=None):
+        if self.fp4:
+            M.moe_expert_down_fp4(self.h, self.offsets, self.w.W_dn_fp4, self.E, self.d, self.rows_max,
+                                  self.gate_of_row, self.y_perm, stream=stream)
+            return
         M.moe_expert_down(self.h, self.offsets, self.w.W_dn, self.rows_max, self.gate_of_row, self.y_perm,
                           stream=stream)
 

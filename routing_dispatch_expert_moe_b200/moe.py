@@ -77,6 +77,10 @@ _SIGNATURES = {
     "moe_get_device_error": (_i32, [ctypes.POINTER(_i32), _c_void_p]),
     "moe_zero": (_i32, [_c_void_p, _size, _c_void_p]),
     "moe_round_output": (_i32, [_c_void_p, _i64, _c_void_p, _i32, _c_void_p]),
+    "moe_expert_gate_up_fp4": (_i32, [_c_void_p, _c_void_p, _i32, _i32, _i32, _i64, _c_void_p, _c_void_p, _i32,
+                                      _c_void_p, _c_void_p, _c_void_p]),
+    "moe_expert_down_fp4": (_i32, [_c_void_p, _c_void_p, _i32, _i32, _i32, _i64, _c_void_p, _c_void_p, _i32,
+                                   _c_void_p, _c_void_p, _i32, _c_void_p, _c_void_p]),
 }
 
 _lib = None
@@ -314,6 +318,79 @@ def moe_dequantize_fp4_host(codes, scales, tensor_scale, K: int, fmt: str = "mxf
                                                                     _host_ptr(ts), rows, K, FP4[fmt],
                                                                     _host_ptr(W), int(threads)))
     return W
+
+
+class Fp4Weights:
+    """One expert weight tensor in a 4-bit format, on the device: codes [rows, K/2] uint8,
+    scales [rows, K/block] uint8 and, for NVFP4, tensor_scale [E] f32 (one per expert).
+    rows = E * 2F for W_gu (gate rows then up rows per expert), E * d for W_dn."""
+
+    def __init__(self, fmt: str, codes, scales, tensor_scale=None):
+        if fmt not in FP4:
+            raise ValueError(f"fmt must be one of {sorted(FP4)}")
+        self.fmt, self.codes, self.scales, self.tensor_scale = fmt, codes, scales, tensor_scale
+
+
+def quantize_experts_fp4(W, fmt: str = "mxfp4", device="cuda", threads: int = 0) -> Fp4Weights:
+    """Packs stacked expert weights W [E, rows_e, K] (torch, any float dtype, on the host)
+    with the library's host packer, one expert at a time (NVFP4: one tensor scale per
+    expert), and copies the result to the device."""
+    import numpy as np
+    E, R, K = W.shape
+    block = int(lib().moe_fp4_block_size(FP4[fmt]))
+    codes = torch.empty((E * R, K // 2), dtype=torch.uint8)
+    scales = torch.empty((E * R, K // block), dtype=torch.uint8)
+    ts = np.ones(E, np.float32)
+    for e in range(E):
+        c, sc, t = moe_quantize_fp4_host(W[e].float().numpy(), fmt, threads)
+        codes[e * R:(e + 1) * R] = torch.from_numpy(c)
+        scales[e * R:(e + 1) * R] = torch.from_numpy(sc)
+        if t is not None:
+            ts[e] = t
+    return Fp4Weights(fmt, codes.to(device), scales.to(device),
+                      torch.from_numpy(ts).to(device) if fmt == "nvfp4" else None)
+
+
+def _need_fp4(w: Fp4Weights, rows: int, K: int, E: int):
+    if not isinstance(w, Fp4Weights):
+        raise ValueError("expected Fp4Weights")
+    block = int(lib().moe_fp4_block_size(FP4[w.fmt]))
+    _need(w.codes, "codes", torch.uint8, (rows, K // 2))
+    _need(w.scales, "scales", torch.uint8, (rows, K // block))
+    if w.fmt == "nvfp4":
+        _need(w.tensor_scale, "tensor_scale", torch.float32, (E,))
+
+
+def moe_expert_gate_up_fp4(x_rows, offsets, W_gu: Fp4Weights, E: int, F: int, rows_max: int, h=None, stream=None):
+    """H = silu(X Wg^T) * (X Wu^T) with 4-bit weights W_gu (rows E * 2F, K = d)."""
+    d = x_rows.shape[1]
+    _need(x_rows, "x_rows", torch.bfloat16)
+    _need(offsets, "offsets", torch.int32, (E + 1,))
+    _need_fp4(W_gu, E * 2 * F, d, E)
+    h = torch.empty((max(rows_max, 1), F), dtype=torch.bfloat16, device=x_rows.device) if h is None else \
+        _need(h, "h", torch.bfloat16)
+    _check("moe_expert_gate_up_fp4", lib().moe_expert_gate_up_fp4(
+        _p(x_rows), _p(offsets), E, d, F, rows_max, _p(W_gu.codes), _p(W_gu.scales), FP4[W_gu.fmt],
+        _p(W_gu.tensor_scale), _p(h), _stream(stream)))
+    return h
+
+
+def moe_expert_down_fp4(h, offsets, W_dn: Fp4Weights, E: int, d: int, rows_max: int, gate_of_row=None, y_rows=None,
+                        y_dtype=None, stream=None):
+    """Gated rows = gate_of_row * (H W_dn^T) with 4-bit weights W_dn (rows E * d, K = F)."""
+    F = h.shape[1]
+    _need(h, "h", torch.bfloat16)
+    _need(offsets, "offsets", torch.int32, (E + 1,))
+    _need_fp4(W_dn, E * d, F, E)
+    if gate_of_row is not None:
+        _need(gate_of_row, "gate_of_row", torch.float32)
+    y_dtype = y_rows.dtype if y_rows is not None else (y_dtype or torch.float32)
+    y_rows = torch.empty((max(rows_max, 1), d), dtype=y_dtype, device=h.device) if y_rows is None else \
+        _need(y_rows, "y_rows")
+    _check("moe_expert_down_fp4", lib().moe_expert_down_fp4(
+        _p(h), _p(offsets), E, d, F, rows_max, _p(W_dn.codes), _p(W_dn.scales), FP4[W_dn.fmt],
+        _p(W_dn.tensor_scale), _p(gate_of_row), _dt(y_rows), _p(y_rows), _stream(stream)))
+    return y_rows
 
 
 def moe_histogram_scan(topk_idx, topk_gate, E: int, capacity: int = -1, counts=None, kept=None, offsets=None,

@@ -309,3 +309,21 @@ def test_scan_wait_check_host_validation(L):
     assert call(ns=999) == 1 and call(ns=2 * 10 ** 9) == 1
     assert call(ptr=NUL) == 1
     assert call(ws=NUL) == 3 and call(wsb=16) == 3
+
+
+def test_fp4_gemm_host_validation(L):
+    gu = L.moe_expert_gate_up_fp4      # (x, offs, E, d, F, rows, codes, scales, fmt, ts, h, s)
+    dn = L.moe_expert_down_fp4         # (h, offs, E, d, F, rows, codes, scales, fmt, ts, gate, ydt, y, s)
+
+    def g(**kw):
+        a = dict(x=FAKE, offs=FAKE, E=8, d=128, F=64, rows=100, codes=FAKE, scales=FAKE, fmt=0, ts=NUL, out=FAKE)
+        a.update(kw)
+        return gu(a["x"], a["offs"], a["E"], a["d"], a["F"], a["rows"], a["codes"], a["scales"], a["fmt"], a["ts"],
+                  a["out"], NUL)
+    assert g(fmt=2) == 1 and g(codes=NUL) == 1 and g(offs=NUL) == 1 and g(x=NUL) == 1
+    assert g(fmt=1) == 1                                   # NVFP4 needs the tensor scales
+    assert g(d=96) == 2 and g(F=32) == 2 and g(E=2000) == 2
+    assert g(codes=ctypes.c_void_p(4104)) == 2 and g(scales=ctypes.c_void_p(4100)) == 2
+    assert g(rows=0, x=NUL, out=NUL) == 0                  # nothing to do
+    assert dn(FAKE, FAKE, 8, 128, 64, 100, FAKE, FAKE, 0, NUL, NUL, 7, FAKE, NUL) == 1   # output dtype
+    assert dn(FAKE, FAKE, 8, 128, 64, 100, FAKE, FAKE, 1, NUL, NUL, 0, FAKE, NUL) == 1   # NVFP4 without scales

@@ -151,3 +151,49 @@ def test_fake_quantize_formats():
         assert np.array_equal(Q.fake_quantize(D, fmt), D) if fmt == "mxfp4" else True   # MX: idempotent
     with pytest.raises(ValueError):
         Q.fake_quantize(W, "fp8")
+
+
+def test_e4m3_decode_matches_the_library_float8_on_every_byte():
+    import torch
+    b = np.arange(256, dtype=np.uint8)
+    lib = torch.from_numpy(b.copy()).view(torch.float8_e4m3fn).float().numpy().astype(np.float64)
+    ours = np.array([Q.e4m3_decode(int(v)) for v in b])
+    nan = np.isnan(lib)
+    assert np.array_equal(np.isnan(ours), nan) and int(nan.sum()) == 2          # 0x7f and 0xff
+    assert np.array_equal(ours[~nan], lib[~nan])
+
+
+def test_e4m3_decode_hand_values():
+    assert Q.e4m3_decode(0x7E) == 448.0                      # e = 15, m = 6: the largest finite
+    assert Q.e4m3_decode(0x38) == 1.0                        # e = 7, m = 0
+    assert Q.e4m3_decode(0x01) == 2.0 ** -9                  # the smallest subnormal
+    assert Q.e4m3_decode(0x08) == 2.0 ** -6                  # the smallest normal
+    assert Q.e4m3_decode(0xB8) == -1.0
+
+
+@pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4"])
+def test_decode_packed_equals_the_scalar_dequantizers(fmt):
+    rng = np.random.default_rng(11)
+    W = rng.normal(0, 0.02, (7, 64)) * np.logspace(-3, 3, 7)[:, None]
+    if fmt == "mxfp4":
+        E, codes = Q.mxfp4_quantize(W)
+        want = Q.mxfp4_dequantize(E, codes)
+        got = Q.decode_packed(Q.pack_codes(codes), (E + 127).astype(np.uint8), fmt)
+    else:
+        s_t, s_b, codes = Q.nvfp4_quantize(W)
+        want = Q.nvfp4_dequantize(s_t, s_b, codes)
+        import torch
+        sb_bytes = torch.from_numpy(s_b.astype(np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+        got = Q.decode_packed(Q.pack_codes(codes), sb_bytes, fmt, s_t)
+    assert np.array_equal(got, want)
+
+
+def test_decode_packed_hand_example():
+    # one MXFP4 row of 64: byte 0x72 = elements (code 2 = 1.0, code 7 = 6.0); scales 2^0, 2^-3
+    codes = np.full((1, 32), 0x72, np.uint8)
+    scales = np.array([[127, 124]], np.uint8)
+    W = Q.decode_packed(codes, scales, "mxfp4")
+    assert list(W[0, :4]) == [1.0, 6.0, 1.0, 6.0] and list(W[0, 32:34]) == [0.125, 0.75]
+    # sign nibble: 0xA9 = elements (code 9 = -0.5, code 10 = -1.0), NVFP4 scale 0x38 = 1, tensor scale 2
+    W = Q.decode_packed(np.full((1, 8), 0xA9, np.uint8), np.full((1, 1), 0x38, np.uint8), "nvfp4", 2.0)
+    assert list(W[0, :2]) == [-1.0, -2.0]
