@@ -299,6 +299,58 @@ MOE_API moe_status moe_histogram_scan(const int32_t* topk_idx, const float* topk
                               void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------------------
+ * Expert-parallel forward (one process per GPU, G ranks): the per-rank building blocks.
+ * [MoE-Explained] section "让 MoE 起飞" / expert parallelism (experts on different
+ * workers; tokens are sent to the workers holding their experts and the results sent
+ * back) and section "Switch Transformer" (expert capacity); [Handbook-News] "真正难在三个
+ * 环节" item 3 (the dispatch / combine all-to-all of every MoE layer).
+ * Rank h owns experts [h E/G, (h+1) E/G) (E % G == 0).  The global token order is rank
+ * 0's tokens, then rank 1's, ...; capacity drops follow it.  A rank's forward:
+ *   moe_route (all E experts) -> moe_histogram_scan (capacity -1: the local counts) ->
+ *   all-gather the counts [G][E] -> moe_ep_plan_host -> moe_histogram_scan_caps (the
+ *   rank's kept limit per expert) -> moe_permute (rows grouped by expert, so by
+ *   destination) -> all-to-all (send_rows / recv_rows) -> moe_ep_regroup (source-major to
+ *   expert-major) -> the grouped GEMMs over the local experts (no gate) ->
+ *   moe_ep_regroup inverse -> all-to-all back -> moe_combine with topk_gate.
+ *
+ * moe_histogram_scan_caps -- moe_histogram_scan with a per-expert capacity: expert e keeps
+ *   its first caps[e] assignments in token order (caps: device [E] int32).  The row
+ *   buffers hold T*k rows.  Other arguments, workspace and errors as moe_histogram_scan.
+ *
+ * moe_ep_plan_host -- the dispatch plan of rank g, on the host.
+ *   counts        (host) [G][E] int32: every rank's per-expert assignment counts
+ *   capacity      slots per expert for the whole batch, or -1 (no dropping)
+ *   caps          (host) [E] out: kept[g][e] = clamp(capacity - sum_{s<g} counts[s][e], 0,
+ *                 counts[g][e]) (counts[g][e] without a capacity)
+ *   send_rows     (host) [G] out: rows rank g sends to each rank (its kept rows of that
+ *                 rank's experts)
+ *   recv_rows     (host) [G] out: rows each rank sends to rank g
+ *   local_offsets (host) [E/G + 1] out: rank g's experts' rows, expert by expert (sources
+ *                 in rank order inside an expert), as a grouped GEMM's offsets
+ *   regroup       (host) [G * E/G][3] int64 out: for source s and local expert j, entry
+ *                 s E/G + j = (row in the receive buffer, row in the expert-major buffer,
+ *                 rows)
+ *   Errors: INVALID_ARG for G < 1, g outside [0, G), negative counts, a null pointer or
+ *   capacity < -1; UNSUPPORTED for E % G != 0 or E > 1024.
+ *
+ * moe_ep_regroup -- row copies by a regroup table (device [n][3] int64, as written by
+ *   moe_ep_plan_host): inverse 0 copies src row (entry[0] + r) to dst row (entry[1] + r),
+ *   inverse 1 the other way; rows of row_bytes bytes (a multiple of 16).  An entry that
+ *   would leave either buffer records MOE_DEVERR_ROW and is skipped.
+ * ---------------------------------------------------------------------------------- */
+MOE_API moe_status moe_histogram_scan_caps(const int32_t* topk_idx, const float* topk_gate,
+                              int32_t T, int32_t k, int32_t E, const int32_t* caps,
+                              int32_t* counts, int32_t* kept, int32_t* offsets,
+                              int32_t* row_of, int32_t* token_of_row, float* gate_of_row,
+                              void* workspace, size_t workspace_bytes, void* stream);
+MOE_API moe_status moe_ep_plan_host(const int32_t* counts, int32_t G, int32_t g, int32_t E,
+                              int32_t capacity, int32_t* caps, int64_t* send_rows,
+                              int64_t* recv_rows, int32_t* local_offsets, int64_t* regroup);
+MOE_API moe_status moe_ep_regroup(const void* src, int64_t src_rows, int32_t row_bytes,
+                              const int64_t* table, int32_t n, int32_t inverse, void* dst,
+                              int64_t dst_rows, void* stream);
+
+/* ------------------------------------------------------------------------------------
  * moe_scan_wait_check -- diagnostic: makes the histogram/scan's bounded wait run out.
  * (No counterpart on the pages: it tests the library's own recovery path.)
  * The look-back of moe_histogram_scan's rank kernel waits for the running totals of the

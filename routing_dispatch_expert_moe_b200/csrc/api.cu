@@ -239,6 +239,42 @@ moe_status moe_histogram_scan_noalloc(const int32_t* topk_idx, const float* topk
                                        token_of_row, gate_of_row, rows_max, S(stream));
 }
 
+moe_status moe_histogram_scan_caps(const int32_t* topk_idx, const float* topk_gate, int32_t T, int32_t k, int32_t E,
+                                   const int32_t* caps, int32_t* counts, int32_t* kept, int32_t* offsets,
+                                   int32_t* row_of, int32_t* token_of_row, float* gate_of_row, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+  moe_status st = check_dims(T, E, k);
+  if (st != MOE_OK) return st;
+  if (!caps || !counts || !kept || !offsets) return MOE_ERR_INVALID_ARG;
+  if (T > 0 && (!topk_idx || !topk_gate || !row_of || !token_of_row || !gate_of_row)) return MOE_ERR_INVALID_ARG;
+  const size_t need = histogram_scan_workspace_bytes(T, k, E);
+  if (need > 0 && (!workspace || workspace_bytes < need)) return MOE_ERR_WORKSPACE;
+  return launch_histogram_scan_caps(topk_idx, topk_gate, T, k, E, caps, counts, kept, offsets, row_of, token_of_row,
+                                    gate_of_row, (long long)T * k, workspace, S(stream));
+}
+
+moe_status moe_ep_plan_host(const int32_t* counts, int32_t G, int32_t g, int32_t E, int32_t capacity, int32_t* caps,
+                            int64_t* send_rows, int64_t* recv_rows, int32_t* local_offsets, int64_t* regroup) {
+  if (G < 1 || g < 0 || g >= G || E < 1 || capacity < -1) return MOE_ERR_INVALID_ARG;
+  if (E % G != 0 || E > kMaxE) return MOE_ERR_UNSUPPORTED;
+  if (!counts || !caps || !send_rows || !recv_rows || !local_offsets || !regroup) return MOE_ERR_INVALID_ARG;
+  for (long long i = 0; i < (long long)G * E; ++i)
+    if (counts[i] < 0) return MOE_ERR_INVALID_ARG;
+  return ep_plan_host(counts, G, g, E, capacity, caps, send_rows, recv_rows, local_offsets, regroup);
+}
+
+moe_status moe_ep_regroup(const void* src, int64_t src_rows, int32_t row_bytes, const int64_t* table, int32_t n,
+                          int32_t inverse, void* dst, int64_t dst_rows, void* stream) {
+  if (src_rows < 0 || dst_rows < 0 || n < 0 || row_bytes < 1 || (inverse != 0 && inverse != 1))
+    return MOE_ERR_INVALID_ARG;
+  if (row_bytes % 16 != 0) return MOE_ERR_UNSUPPORTED;
+  if (n == 0) return MOE_OK;
+  if (!table || (src_rows > 0 && !src) || (dst_rows > 0 && !dst)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(src) || !aligned16(dst)) return MOE_ERR_UNSUPPORTED;
+  return launch_ep_regroup(src, src_rows, row_bytes, reinterpret_cast<const long long*>(table), n, inverse, dst,
+                           dst_rows, S(stream));
+}
+
 moe_status moe_scan_wait_check(const int32_t* topk_idx, const float* topk_gate, int32_t T, int32_t k, int32_t E,
                                int32_t capacity, int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* row_of,
                                int32_t* token_of_row, float* gate_of_row, uint64_t wait_ns, void* workspace,

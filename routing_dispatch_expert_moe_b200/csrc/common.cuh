@@ -169,6 +169,14 @@ moe_status launch_histogram_scan(const int32_t* topk_idx, const float* topk_gate
                                  float* gate_of_row, long long rows_max, void* ws, cudaStream_t s);
 size_t histogram_scan_workspace_bytes(int T, int k, int E);
 size_t histogram_scan_noalloc_limit();
+moe_status launch_histogram_scan_caps(const int32_t* topk_idx, const float* topk_gate, int T, int k, int E,
+                                      const int32_t* caps, int32_t* counts, int32_t* kept, int32_t* offsets,
+                                      int32_t* row_of, int32_t* token_of_row, float* gate_of_row, long long rows_max,
+                                      void* ws, cudaStream_t s);
+moe_status ep_plan_host(const int32_t* counts, int G, int g, int E, int capacity, int32_t* caps, int64_t* send_rows,
+                        int64_t* recv_rows, int32_t* local_offsets, int64_t* regroup);
+moe_status launch_ep_regroup(const void* src, long long src_rows, int row_bytes, const long long* table, int n,
+                             int inverse, void* dst, long long dst_rows, cudaStream_t s);
 moe_status launch_scan_wait_check(const int32_t* topk_idx, const float* topk_gate, int T, int k, int E,
                                   int capacity, int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* row_of,
                                   int32_t* token_of_row, float* gate_of_row, long long rows_max, void* ws,

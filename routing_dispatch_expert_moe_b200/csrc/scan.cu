@@ -67,7 +67,8 @@ __device__ __forceinline__ void st_volatile(uint32_t* p, uint32_t v) {
 }
 
 __global__ void __launch_bounds__(kRankThreads)
-rank_kernel(const int32_t* __restrict__ topk_idx, int T, int k, int E, int capacity, int nchunks,
+rank_kernel(const int32_t* __restrict__ topk_idx, int T, int k, int E, int capacity,
+            const int32_t* __restrict__ caps, int nchunks,
             uint32_t* __restrict__ ticket, uint32_t* __restrict__ status, int32_t* __restrict__ rank,
             int32_t* __restrict__ counts, int32_t* __restrict__ kept, int32_t* __restrict__ offsets,
             unsigned long long spin_limit_ns, int* err) {
@@ -166,7 +167,8 @@ rank_kernel(const int32_t* __restrict__ topk_idx, int T, int k, int E, int capac
       int kv = 0;
       if (e < E) {
         const int c = (int)tots[e];
-        kv = capacity < 0 ? c : min(c, capacity);
+        const int cap_e = caps ? max(0, __ldg(caps + e)) : capacity;
+        kv = cap_e < 0 ? c : min(c, cap_e);
         counts[e] = c;
         kept[e] = kv;
       }
@@ -201,7 +203,8 @@ rank_kernel(const int32_t* __restrict__ topk_idx, int T, int k, int E, int capac
 __global__ void __launch_bounds__(256)
 scatter_kernel(const int32_t* __restrict__ topk_idx, const float* __restrict__ topk_gate,
                const int32_t* __restrict__ rank, const int32_t* __restrict__ offsets, int T, int k,
-               int E, int capacity, long long rows_max, int32_t* __restrict__ row_of,
+               int E, int capacity, const int32_t* __restrict__ caps, long long rows_max,
+               int32_t* __restrict__ row_of,
                int32_t* __restrict__ token_of_row, float* __restrict__ gate_of_row, int* err) {
   const long long A = (long long)T * k;
   for (long long a = (long long)blockIdx.x * blockDim.x + threadIdx.x; a < A;
@@ -210,7 +213,8 @@ scatter_kernel(const int32_t* __restrict__ topk_idx, const float* __restrict__ t
     int row = -1;
     if ((unsigned)e < (unsigned)E) {
       const int r = __ldg(rank + a);
-      if (r >= 0 && (capacity < 0 || r < capacity)) {
+      const int cap_e = caps ? max(0, __ldg(caps + e)) : capacity;
+      if (r >= 0 && (cap_e < 0 || r < cap_e)) {
         const long long rr = (long long)__ldg(offsets + e) + r;
         if (rr < rows_max) row = (int)rr;
         else record_error(err, MOE_DEVERR_ROW);
@@ -282,16 +286,26 @@ size_t histogram_scan_workspace_bytes(int T, int k, int E) {
 // form of moe_scan_wait_check (chunks 0 .. first_ticket - 1 never run, so the look-back of
 // every later chunk waits for words nobody publishes, until spin_limit_ns).
 static moe_status run_histogram_scan(const int32_t* topk_idx, const float* topk_gate, int T, int k, int E,
-                                     int capacity, int32_t* counts, int32_t* kept, int32_t* offsets,
-                                     int32_t* row_of, int32_t* token_of_row, float* gate_of_row, long long rows_max,
-                                     void* ws, cudaStream_t s, unsigned first_ticket,
+                                     int capacity, const int32_t* caps, int32_t* counts, int32_t* kept,
+                                     int32_t* offsets, int32_t* row_of, int32_t* token_of_row, float* gate_of_row,
+                                     long long rows_max, void* ws, cudaStream_t s, unsigned first_ticket,
                                      unsigned long long spin_limit_ns);
 
 moe_status launch_histogram_scan(const int32_t* topk_idx, const float* topk_gate, int T, int k,
                                  int E, int capacity, int32_t* counts, int32_t* kept,
                                  int32_t* offsets, int32_t* row_of, int32_t* token_of_row,
                                  float* gate_of_row, long long rows_max, void* ws, cudaStream_t s) {
-  return run_histogram_scan(topk_idx, topk_gate, T, k, E, capacity, counts, kept, offsets, row_of, token_of_row,
+  return run_histogram_scan(topk_idx, topk_gate, T, k, E, capacity, nullptr, counts, kept, offsets, row_of,
+                            token_of_row, gate_of_row, rows_max, ws, s, 0u, kSpinLimitNs);
+}
+
+// The same with a per-expert capacity (device [E]): expert e keeps its first caps[e]
+// assignments in token order.
+moe_status launch_histogram_scan_caps(const int32_t* topk_idx, const float* topk_gate, int T, int k, int E,
+                                      const int32_t* caps, int32_t* counts, int32_t* kept, int32_t* offsets,
+                                      int32_t* row_of, int32_t* token_of_row, float* gate_of_row, long long rows_max,
+                                      void* ws, cudaStream_t s) {
+  return run_histogram_scan(topk_idx, topk_gate, T, k, E, -1, caps, counts, kept, offsets, row_of, token_of_row,
                             gate_of_row, rows_max, ws, s, 0u, kSpinLimitNs);
 }
 
@@ -299,14 +313,14 @@ moe_status launch_scan_wait_check(const int32_t* topk_idx, const float* topk_gat
                                   int capacity, int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* row_of,
                                   int32_t* token_of_row, float* gate_of_row, long long rows_max, void* ws,
                                   unsigned long long wait_ns, cudaStream_t s) {
-  return run_histogram_scan(topk_idx, topk_gate, T, k, E, capacity, counts, kept, offsets, row_of, token_of_row,
-                            gate_of_row, rows_max, ws, s, 1u, wait_ns);
+  return run_histogram_scan(topk_idx, topk_gate, T, k, E, capacity, nullptr, counts, kept, offsets, row_of,
+                            token_of_row, gate_of_row, rows_max, ws, s, 1u, wait_ns);
 }
 
 static moe_status run_histogram_scan(const int32_t* topk_idx, const float* topk_gate, int T, int k, int E,
-                                     int capacity, int32_t* counts, int32_t* kept, int32_t* offsets,
-                                     int32_t* row_of, int32_t* token_of_row, float* gate_of_row, long long rows_max,
-                                     void* ws, cudaStream_t s, unsigned first_ticket,
+                                     int capacity, const int32_t* caps, int32_t* counts, int32_t* kept,
+                                     int32_t* offsets, int32_t* row_of, int32_t* token_of_row, float* gate_of_row,
+                                     long long rows_max, void* ws, cudaStream_t s, unsigned first_ticket,
                                      unsigned long long spin_limit_ns) {
   if (T == 0) {
     moe_status st = cuda_status(cudaMemsetAsync(counts, 0, (size_t)E * 4, s));
@@ -329,7 +343,7 @@ static moe_status run_histogram_scan(const int32_t* topk_idx, const float* topk_
   st = ensure_smem_limit(configured, rank_kernel, rank_smem_bytes(32, 1024));
   if (st != MOE_OK) return st;
   int* err = err_ptr();
-  rank_kernel<<<nchunks, kRankThreads, smem, s>>>(topk_idx, T, k, E, capacity, nchunks, w.ticket, w.status,
+  rank_kernel<<<nchunks, kRankThreads, smem, s>>>(topk_idx, T, k, E, capacity, caps, nchunks, w.ticket, w.status,
                                                  w.rank, counts, kept, offsets, spin_limit_ns, err);
   st = check_launch();
   if (st != MOE_OK) return st;
@@ -337,7 +351,7 @@ static moe_status run_histogram_scan(const int32_t* topk_idx, const float* topk_
   long long blocks = (A + 255) / 256;
   const long long cap = (long long)num_sms() * 8;
   if (blocks > cap) blocks = cap;
-  scatter_kernel<<<(unsigned)blocks, 256, 0, s>>>(topk_idx, topk_gate, w.rank, offsets, T, k, E, capacity,
+  scatter_kernel<<<(unsigned)blocks, 256, 0, s>>>(topk_idx, topk_gate, w.rank, offsets, T, k, E, capacity, caps,
                                                   rows_max, row_of, token_of_row, gate_of_row, err);
   return check_launch();
 }

@@ -1,0 +1,179 @@
+"""Expert-parallel MoE-layer forward: one process per GPU, experts split over the ranks.
+
+"Mixture of Experts Explained" (zh), section "让 MoE 起飞" / expert parallelism: the experts
+live on different workers; every token is sent to the workers that hold its experts and
+the results come back.  Handbook news post, "真正难在三个环节" item 3: this dispatch and
+combine all-to-all is where a distributed MoE layer spends its time.
+
+Rank g of G holds its own batch of tokens, the whole router, and experts
+[g E/G, (g+1) E/G).  The global token order is rank 0's tokens, then rank 1's, ..., and
+the capacity (slots per expert for the whole batch) drops assignments in that order, so
+the result equals the single-GPU layer run on the concatenated batch.  One forward:
+
+    route (all E experts)  ->  local counts  ->  all-gather counts [G, E]
+    ->  moe_ep_plan_host (kept rows per expert in global token order, all-to-all sizes,
+        the regroup table)  ->  scan with per-expert capacity  ->  permute (rows grouped
+        by expert, hence by destination)  ->  all-to-all  ->  regroup (source-major ->
+        expert-major)  ->  grouped gate/up + down GEMMs of the local experts (no gate)
+    ->  regroup back  ->  all-to-all back  ->  combine with the gates.
+
+The exchange is torch.distributed's all_to_all_single (NCCL between GPUs); the split
+sizes need the plan on the host, so one small device-to-host copy of the counts happens
+per forward.  Every compute step is a library kernel (LibraryKernels); the steps are
+grouped behind one small interface so that the orchestration and the exchange can also
+be driven by other implementations of the same steps.
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Optional
+
+import numpy as np
+import torch
+import torch.distributed as dist
+
+from . import moe as M
+
+
+def ep_plan(counts: np.ndarray, g: int, capacity: int) -> dict:
+    """moe_ep_plan_host for rank g: counts [G, E] int32 (every rank's per-expert counts)."""
+    counts = np.ascontiguousarray(counts, np.int32)
+    G, E = counts.shape
+    El = E // G
+    caps = np.empty(E, np.int32)
+    send = np.empty(G, np.int64)
+    recv = np.empty(G, np.int64)
+    offs = np.empty(El + 1, np.int32)
+    table = np.empty((G * El, 3), np.int64)
+    ptr = lambda a: ctypes.c_void_p(a.ctypes.data)                       # noqa: E731
+    M._check("moe_ep_plan_host", M.lib().moe_ep_plan_host(ptr(counts), G, g, E, int(capacity), ptr(caps), ptr(send),
+                                                          ptr(recv), ptr(offs), ptr(table)))
+    return {"caps": caps, "send_rows": send, "recv_rows": recv, "local_offsets": offs, "regroup": table}
+
+
+class LibraryKernels:
+    """The forward's compute steps on the GPU, each one library call (moe.py)."""
+
+    def __init__(self, layer: "ExpertParallelMoE"):
+        self.L = layer
+
+    def route(self, x):
+        L = self.L
+        return M.moe_route(x, L.Wg, L.k, L.score, L.renormalize, L.scale, L.logit_offset, L.select_bias,
+                           Wg_split=L.Wg_split)
+
+    def counts(self, topk_idx):
+        return M.moe_histogram_scan(topk_idx, torch.zeros(topk_idx.shape, dtype=torch.float32,
+                                                          device=topk_idx.device), self.L.E, -1)["counts"]
+
+    def scan(self, topk_idx, topk_gate, caps):
+        T, k = topk_idx.shape
+        dev = topk_idx.device
+        i32 = torch.int32
+        out = dict(counts=torch.empty(self.L.E, dtype=i32, device=dev), kept=torch.empty(self.L.E, dtype=i32, device=dev),
+                   offsets=torch.empty(self.L.E + 1, dtype=i32, device=dev),
+                   row_of=torch.empty((T, k), dtype=i32, device=dev),
+                   token_of_row=torch.empty(max(T * k, 1), dtype=i32, device=dev),
+                   gate_of_row=torch.empty(max(T * k, 1), dtype=torch.float32, device=dev))
+        nb = int(M.lib().moe_histogram_scan_workspace_bytes(T, k, self.L.E))
+        ws = torch.empty(max(nb, 16), dtype=torch.uint8, device=dev)
+        caps_d = torch.from_numpy(caps).to(dev)
+        M._check("moe_histogram_scan_caps", M.lib().moe_histogram_scan_caps(
+            M._p(topk_idx), M._p(topk_gate), T, k, self.L.E, M._p(caps_d), M._p(out["counts"]), M._p(out["kept"]),
+            M._p(out["offsets"]), M._p(out["row_of"]), M._p(out["token_of_row"]), M._p(out["gate_of_row"]),
+            M._p(ws), nb, M._stream(None)))
+        return out
+
+    def permute(self, x, row_of, rows):
+        return M.moe_permute(x, row_of, rows)
+
+    def regroup(self, src, table, inverse, rows_out):
+        d = src.shape[1]
+        dst = torch.empty((max(rows_out, 1), d), dtype=src.dtype, device=src.device)
+        n = table.shape[0]
+        if n:
+            t = torch.from_numpy(np.ascontiguousarray(table)).to(src.device)
+            M._check("moe_ep_regroup", M.lib().moe_ep_regroup(
+                M._p(src), src.shape[0], d * src.element_size(), M._p(t), n, 1 if inverse else 0, M._p(dst),
+                dst.shape[0], M._stream(None)))
+        return dst
+
+    def ffn(self, x_local, offsets_local, rows):
+        L = self.L
+        offs = torch.from_numpy(offsets_local).to(x_local.device)
+        h = M.moe_expert_gate_up(x_local, offs, L.W_gu, rows)
+        return M.moe_expert_down(h, offs, L.W_dn, rows, None, y_dtype=L.rows_dtype)
+
+    def combine(self, y_rows, row_of, topk_gate, T):
+        return M.moe_combine(y_rows, row_of, T, y_rows.shape[0], topk_gate=topk_gate, y_dtype=self.L.out_dtype)
+
+
+class ExpertParallelMoE:
+    """One rank's share of an expert-parallel MoE layer.
+
+    Wg [d, E] f32 (the whole router), W_gu [E/G, 2F, d] and W_dn [E/G, d, F]: this rank's
+    experts, g E/G .. (g+1) E/G - 1.  capacity: slots per expert for the whole batch
+    across the ranks (moe_capacity of the global token count), or -1.  group: the process
+    group of the G ranks (None: the default group, or a single rank without one)."""
+
+    def __init__(self, Wg, W_gu, W_dn, k: int, score: str = "softmax", renormalize: bool = True,
+                 scale: float = 1.0, capacity: int = -1, logit_offset=None, select_bias=None, group=None,
+                 rows_dtype=torch.float32, out_dtype=torch.float32, kernels=None):
+        self.group = group
+        ready = dist.is_available() and dist.is_initialized()
+        self.G = dist.get_world_size(group) if ready else 1
+        self.g = dist.get_rank(group) if ready else 0
+        self.d, self.E = Wg.shape
+        if self.E % self.G:
+            raise ValueError(f"E={self.E} experts do not split over {self.G} ranks")
+        self.El = self.E // self.G
+        if W_gu.shape[0] != self.El or W_dn.shape[0] != self.El:
+            raise ValueError(f"this rank holds {self.El} experts: W_gu and W_dn must have {self.El} rows of experts")
+        self.Wg, self.W_gu, self.W_dn = Wg, W_gu, W_dn
+        self.k, self.score, self.renormalize, self.scale, self.capacity = k, score, renormalize, scale, capacity
+        self.logit_offset, self.select_bias = logit_offset, select_bias
+        self.rows_dtype, self.out_dtype = rows_dtype, out_dtype
+        self.kernels = kernels if kernels is not None else LibraryKernels(self)
+        self.Wg_split = M.moe_prepare_router_weight(Wg) if (kernels is None and Wg.is_cuda) else None
+        self.last_plan: Optional[dict] = None
+
+    # the exchange ------------------------------------------------------------------
+    def _all_gather_counts(self, counts):
+        if self.G == 1:
+            return counts.reshape(1, -1)
+        parts = [torch.empty_like(counts) for _ in range(self.G)]
+        dist.all_gather(parts, counts, group=self.group)
+        return torch.stack(parts)
+
+    def _all_to_all(self, rows, send_rows, recv_rows):
+        d = rows.shape[1]
+        out = torch.empty((int(recv_rows.sum()), d), dtype=rows.dtype, device=rows.device)
+        if self.G == 1:
+            out.copy_(rows[:out.shape[0]])
+            return out
+        dist.all_to_all_single(out, rows[:int(send_rows.sum())].contiguous(),
+                               output_split_sizes=[int(v) for v in recv_rows],
+                               input_split_sizes=[int(v) for v in send_rows], group=self.group)
+        return out
+
+    # the forward ---------------------------------------------------------------------
+    def forward(self, x):
+        kn = self.kernels
+        T = x.shape[0]
+        logits, topk_idx, topk_gate = kn.route(x)
+        counts = kn.counts(topk_idx)
+        allc = self._all_gather_counts(counts).cpu().numpy()        # the one device-to-host copy
+        plan = ep_plan(allc, self.g, self.capacity)
+        self.last_plan = plan
+        sc = kn.scan(topk_idx, topk_gate, plan["caps"])
+        n_send = int(plan["send_rows"].sum())
+        x_perm = kn.permute(x, sc["row_of"], max(T * self.k, 1))
+        recv = self._all_to_all(x_perm, plan["send_rows"], plan["recv_rows"])
+        n_local = int(plan["local_offsets"][-1])
+        x_local = kn.regroup(recv, plan["regroup"], False, n_local)
+        y_local = kn.ffn(x_local, plan["local_offsets"], n_local)
+        y_send = kn.regroup(y_local, plan["regroup"], True, int(plan["recv_rows"].sum()))
+        y_rows = self._all_to_all(y_send, plan["recv_rows"], plan["send_rows"])
+        assert y_rows.shape[0] == n_send
+        self.routing = {"logits": logits, "topk_idx": topk_idx, "topk_gate": topk_gate, **sc}
+        return kn.combine(y_rows, sc["row_of"], topk_gate, T)

@@ -57,6 +57,11 @@ _SIGNATURES = {
                                           _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p]),
     "moe_scan_wait_check": (_i32, [_c_void_p, _c_void_p, _i32, _i32, _i32, _i32, _c_void_p, _c_void_p, _c_void_p,
                                    _c_void_p, _c_void_p, _c_void_p, ctypes.c_uint64, _c_void_p, _size, _c_void_p]),
+    "moe_histogram_scan_caps": (_i32, [_c_void_p, _c_void_p, _i32, _i32, _i32, _c_void_p, _c_void_p, _c_void_p,
+                                       _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _size, _c_void_p]),
+    "moe_ep_plan_host": (_i32, [_c_void_p, _i32, _i32, _i32, _i32, _c_void_p, _c_void_p, _c_void_p, _c_void_p,
+                                _c_void_p]),
+    "moe_ep_regroup": (_i32, [_c_void_p, _i64, _i32, _c_void_p, _i32, _i32, _c_void_p, _i64, _c_void_p]),
     "moe_permute": (_i32, [_c_void_p, _i32, _i32, _i32, _i32, _c_void_p, _i64, _c_void_p, _c_void_p]),
     "moe_expert_gate_up": (_i32, [_c_void_p, _i32, _c_void_p, _i32, _i32, _i32, _i64, _c_void_p, _c_void_p,
                                   _c_void_p]),
