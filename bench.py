@@ -195,6 +195,8 @@ def run_ours(args):
     cfg = I.CONFIGS[args.workload]
     if args.tokens:
         cfg = cfg.with_(T=args.tokens)
+    if args.experts:
+        cfg = cfg.with_(E=args.experts)
     dt = torch.float32 if cfg.act == "f32" else torch.bfloat16
     x_np = I.gen_x(cfg, seed=replica_seed(rank))        # each replica has its own token batch
     Wg, off, bias = I.gen_router(cfg, 0)
@@ -226,8 +228,8 @@ def run_ours(args):
     out_dt = torch.bfloat16 if args.out_dtype == "bf16" else torch.float32
     rows_dt = torch.bfloat16 if args.rows_dtype == "bf16" else torch.float32
 
-    def make_layer(combine, dispatch):
-        return MoELayer(w, cfg.k, cfg.T, cfg.score, cfg.renormalize, cfg.scale, cap, combine=combine,
+    def make_layer(combine, dispatch, weights=None):
+        return MoELayer(weights or w, cfg.k, cfg.T, cfg.score, cfg.renormalize, cfg.scale, cap, combine=combine,
                         dispatch=dispatch, out_dtype=out_dt, rows_dtype=rows_dt, routing=routing)
 
     def capture(fn):
@@ -334,6 +336,39 @@ def run_ours(args):
                  "value": round(job_throughput(cfg.T, world, args.alt_steps, t), 1), "steps": args.alt_steps,
                  "stages_ms": {k_: round(v, 4) for k_, v in sm.items()}}
         del rl
+        torch.cuda.empty_cache()
+
+    # The routed experts in 4-bit formats (weight-only): the same layer and inputs, the expert
+    # GEMMs reading packed codes.  The codes are drawn at random on the device: the kernels do
+    # the same work whatever the code values (parity of these GEMMs is tested separately).
+    fp4_forms = {}
+    for fmt in ([] if args.fp4_steps <= 0 or dt != torch.bfloat16 else ["mxfp4", "nvfp4"]):
+        gen = torch.Generator(device=dev).manual_seed(7)
+        blk = 32 if fmt == "mxfp4" else 16
+
+        def packed(rows, K):
+            codes = torch.randint(0, 256, (rows, K // 2), dtype=torch.uint8, device=dev, generator=gen)
+            sc = torch.randint(119, 123, (rows, K // blk), dtype=torch.uint8, device=dev, generator=gen) \
+                if fmt == "mxfp4" else torch.randint(0x30, 0x50, (rows, K // blk), dtype=torch.uint8, device=dev,
+                                                     generator=gen)
+            ts = torch.full((cfg.E,), 2.0 ** -7, dtype=torch.float32, device=dev) if fmt == "nvfp4" else None
+            return M.Fp4Weights(fmt, codes, sc, ts)
+
+        w4 = MoEWeights(Wg=w.Wg, W_gu=w.W_gu, W_dn=w.W_dn, logit_offset=w.logit_offset, select_bias=w.select_bias,
+                        W_gu_s=w.W_gu_s, W_dn_s=w.W_dn_s,
+                        W_gu_fp4=packed(cfg.E * 2 * cfg.F, cfg.d), W_dn_fp4=packed(cfg.E * cfg.d, cfg.F))
+        l4 = make_layer("rows", "permute", w4)
+        ps, sm, (A4, E4), _ = time_layer(l4, args.fp4_steps, breakdown_steps=min(args.breakdown_steps, 50))
+        t = max_over_ranks(float(ps.sum()), dev)
+        gu_bytes4 = A4 * cfg.d * 2 + E4 * 2 * cfg.F * cfg.d // 2 + E4 * 2 * cfg.F * (cfg.d // blk) + A4 * cfg.F * 2
+        dn_bytes4 = A4 * cfg.F * 2 + E4 * cfg.d * cfg.F // 2 + E4 * cfg.d * (cfg.F // blk) + A4 * cfg.d * rows_dt.itemsize
+        fp4_forms[fmt] = {"ms_per_step": round(t / args.fp4_steps, 4),
+                          "value": round(job_throughput(cfg.T, world, args.fp4_steps, t), 1), "steps": args.fp4_steps,
+                          "stages_ms": {k_: round(v, 4) for k_, v in sm.items()},
+                          "gate_up_gbs": round(gu_bytes4 / (sm["gate_up"] * 1e-3) / 1e9, 1) if sm.get("gate_up") else None,
+                          "down_gbs": round(dn_bytes4 / (sm["down"] * 1e-3) / 1e9, 1) if sm.get("down") else None,
+                          "weights": "synthetic 4-bit codes and scales (random, on the device)"}
+        del l4, w4
         torch.cuda.empty_cache()
 
     # End to end through the public API with host buffers (pinned), copies inside the timing.
@@ -463,6 +498,7 @@ def run_ours(args):
             "stage_roofline_ms": {k_: round(v, 4) for k_, v in roof_steps.items()},
             "stage_throughput": thr,
             "alt_form": other,
+            "fp4_forms": fp4_forms or None,
             "clocks": clk,
             "cpu_baseline": cpu,
         }
@@ -582,6 +618,8 @@ def main():
                     help="tokens per oracle step (the reference arm and cpu_baseline time the same sample)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="override T (smaller cases of the same kernels, e.g. for profiler captures)")
+    ap.add_argument("--experts", type=int, default=None,
+                    help="override E (smaller cases of the same kernels, e.g. for profiler captures)")
     ap.add_argument("--e2e-steps", type=int, default=50, help="steps timed through host buffers")
     ap.add_argument("--combine", choices=["fused", "rows"], default="rows",
                     help="rows: gated rows + ordered combine (reproducible); fused: combine inside the down GEMM")
@@ -596,6 +634,8 @@ def main():
                          "of synthetic Zipf token ids, or noisy top-k (softmax workloads); not the reference arm")
     ap.add_argument("--breakdown-steps", type=int, default=100,
                     help="sequential replays for the per-stage split (0 = skip)")
+    ap.add_argument("--fp4-steps", type=int, default=30,
+                    help="also time the layer with 4-bit (MXFP4, NVFP4) routed experts for this many steps (0 = skip)")
     ap.add_argument("--alt-steps", type=int, default=100,
                     help="also time the other combine form for this many steps (0 = skip)")
     args = ap.parse_args()

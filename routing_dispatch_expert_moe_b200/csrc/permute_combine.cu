@@ -103,22 +103,28 @@ __device__ __forceinline__ void store8<float>(void* base, long long e, const flo
 }
 
 // KMAX: compile-time bound on k (multiple of 8).  The token's kept slots are first
-// compacted, in slot order, into krow / kgate (warp-uniform, static register indices), so
-// dropped slots cost nothing and every batch of loads is full.  Each lane then loads up to
-// 8 kept rows for VPI consecutive 8-element vectors (8 * VPI independent loads in flight)
-// and adds them in slot order: the same fp32 sum as visiting every slot.
+// compacted, in slot order, into a per-warp list in shared memory (a ballot gives each
+// kept slot its position), so dropped slots cost nothing, every batch of loads is full,
+// and the list costs no registers (two blocks fit on an SM).  Each lane then loads up to
+// 8 kept rows for VPI consecutive 8-element vectors (8 * VPI independent loads in
+// flight) and adds them in slot order: the same fp32 sum as visiting every slot.
 template <typename InT, typename OutT, int KMAX>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 2)
 combine_kernel(const void* __restrict__ y_rows, const int32_t* __restrict__ row_of,
                const float* __restrict__ topk_gate, const void* __restrict__ shared_y, int T, int d, int k,
                long long rows_max, void* __restrict__ y, int* err) {
   constexpr int VPI = sizeof(InT) == 2 ? 2 : 1;       // vectors per lane per step
+  __shared__ int s_row[8][32];
+  __shared__ float s_gate[8][32];
   const unsigned lane = threadIdx.x & 31;
+  const int wib = threadIdx.x >> 5;
   const int warps = blockDim.x >> 5;
   const long long nw = (long long)gridDim.x * warps;
   const bool scale = topk_gate != nullptr;
   const int n8 = d >> 3;
-  for (long long t = (long long)blockIdx.x * warps + (threadIdx.x >> 5); t < T; t += nw) {
+  int* krow = s_row[wib];
+  float* kgate = s_gate[wib];
+  for (long long t = (long long)blockIdx.x * warps + wib; t < T; t += nw) {
     int my_row = -1;
     float my_gate = 1.f;
     if (lane < (unsigned)k) {
@@ -127,23 +133,16 @@ combine_kernel(const void* __restrict__ y_rows, const int32_t* __restrict__ row_
       if (my_row < -1) my_row = -1;
       if (scale) my_gate = __ldg(topk_gate + t * k + lane);
     }
-    // kept slots in slot order -> positions 0 .. nk-1 (all lanes hold the same values)
-    int krow[KMAX];
-    float kgate[KMAX];
-#pragma unroll
-    for (int p = 0; p < KMAX; ++p) { krow[p] = -1; kgate[p] = 0.f; }
-    int nk = 0;
-#pragma unroll
-    for (int j = 0; j < KMAX; ++j) {
-      const int r = __shfl_sync(0xffffffffu, my_row, j & 31);
-      const float g = __shfl_sync(0xffffffffu, my_gate, j & 31);
-      if (j < k && r >= 0) {
-#pragma unroll
-        for (int p = 0; p <= j; ++p)
-          if (p == nk) { krow[p] = r; kgate[p] = g; }
-        ++nk;
-      }
+    // kept slots in slot order -> positions 0 .. nk-1
+    const unsigned kept = __ballot_sync(0xffffffffu, my_row >= 0);
+    const int nk = __popc(kept);
+    __syncwarp();                                       // the previous token's list is read
+    if (my_row >= 0) {
+      const int pos = __popc(kept & ((1u << lane) - 1u));
+      krow[pos] = my_row;
+      kgate[pos] = my_gate;
     }
+    __syncwarp();
     for (int v0 = lane; v0 < n8; v0 += 32 * VPI) {
       float acc[VPI][8];
 #pragma unroll
