@@ -604,7 +604,7 @@ grouped_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
       epilogue_tile<MODE, OutT>(taddr, stage, lane, wrow0, wrows, tc.n_tile, F, N_out, gate_of_row, out,
                                 token_of_row, n_tokens, err, c_begin, c_end);
       tc_fence_before();
-      mbar_arrive_cluster(map_to_rank(bar_tempty + 8 * acc, 0));
+      mbar_arrive_remote(map_to_rank(bar_tempty + 8 * acc, 0));
     }
   }
 

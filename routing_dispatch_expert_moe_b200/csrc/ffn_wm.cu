@@ -292,7 +292,7 @@ grouped_gemm_wm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * 256);
       wm_epilogue_tile<MODE, OutT>(taddr, stage, lane, tc, (int)rank, q, d, F, 1.f, gate_of_row, out);
       tc_fence_before();
-      mbar_arrive_cluster(map_to_rank(bar_tempty + 8 * acc, 0));
+      mbar_arrive_remote(map_to_rank(bar_tempty + 8 * acc, 0));
     }
   }
 
@@ -544,7 +544,7 @@ grouped_gemm_wm4_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_co
       const float ws = tensor_scale ? __ldg(tensor_scale + tc.e) : 1.f;
       wm_epilogue_tile<MODE, OutT>(taddr, stage, lane, tc, (int)rank, q, d, F, ws, gate_of_row, out);
       tc_fence_before();
-      mbar_arrive_cluster(map_to_rank(bar_tempty + 8 * acc, 0));
+      mbar_arrive_remote(map_to_rank(bar_tempty + 8 * acc, 0));
     }
   } else {
     // ------------------------------------------------------------ converters (both CTAs)

@@ -386,7 +386,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
         }
       }
       tc_fence_before();
-      mbar_arrive_cluster(map_to_rank(bar_tempty + 8 * acc, 0));
+      mbar_arrive_remote(map_to_rank(bar_tempty + 8 * acc, 0));
       if constexpr (kFused) {
         if (j == n_tiles - 1) {
           if (lane < wrows) topk_write<KMAX, BIAS>(st, row0 + lane, k, score, renorm, scale, topk_idx, topk_gate);

@@ -125,6 +125,14 @@ __device__ __forceinline__ void cluster_sync() {
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
+// Arrive on a barrier that may live in the peer CTA, releasing at CTA scope only.  The
+// accumulator-free signal of an epilogue needs no ordering of the thread's global stores
+// (only its TMEM reads, which tcgen05.wait::ld and tcgen05.fence::before_thread_sync
+// order); a cluster-scope release would make every epilogue thread wait until all of its
+// earlier global stores are visible cluster-wide, once per tile.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
 // TMA load into this CTA's shared memory whose completion is counted on an mbarrier that
 // may live in the peer CTA (the pair's even CTA); no multicast.
 __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar_cluster, int x,
