@@ -234,7 +234,7 @@ moe_status launch_down_fp4(const void* h, const int32_t* offsets, int E, int d, 
                            const uint8_t* codes, const uint8_t* scales, int fmt, const float* tensor_scale,
                            const float* gate_of_row, int y_dtype, void* y_rows, cudaStream_t s);
 // Whether a grouped GEMM over E experts and rows_max rows takes the weight-major tiles.
-bool prefer_weight_major(long long rows_max, int E);
+bool prefer_weight_major(long long rows_max, int E, bool down);
 
 moe_status launch_gate_up_tc(const void* x_rows, const int32_t* offsets, int E, int d, int F,
                              long long rows_max, const void* W_gu, void* h, cudaStream_t s);

@@ -678,22 +678,25 @@ moe_status launch_tc2(const CUtensorMap& ma, const CUtensorMap& mb, const int32_
 // full.  When the groups average under kWeightMajorBelow rows -- many experts, or a cap
 // that keeps few rows each -- skew leaves most experts with a few dozen rows, and the
 // weight-major tiles (ffn_wm.cu), whose token side is the group rounded up to 32, waste
-// far less tensor work.  MOE_B200_EXPERT_TILES=tokens|weights overrides the choice (for
-// measuring one against the other).
+// far less tensor work.  That holds for gate/up (K = d: long mainloops).  The down GEMM
+// (K = F, a few k-blocks per tile) measured faster token-major at every group size tried
+// (stress workload: 1.4 against 2.0 ms), so it takes weight-major tiles only when forced.
+// MOE_B200_EXPERT_TILES=tokens|weights overrides the choice for both (for measuring one
+// against the other).
 constexpr long long kWeightMajorBelow = 1024;
 
-bool prefer_weight_major(long long rows_max, int E) {
+bool prefer_weight_major(long long rows_max, int E, bool down) {
   const char* v = getenv("MOE_B200_EXPERT_TILES");      // read per call: a host-side string lookup
   if (v && strcmp(v, "tokens") == 0) return false;
   if (v && strcmp(v, "weights") == 0) return true;
-  return E > 0 && rows_max / E < kWeightMajorBelow;
+  return !down && E > 0 && rows_max / E < kWeightMajorBelow;
 }
 
 moe_status launch_gate_up_tc(const void* x_rows, const int32_t* offsets, int E, int d, int F, long long rows_max,
                              const void* W_gu, void* h, cudaStream_t s) {
   if (rows_max == 0) return MOE_OK;
   if (d < BK || F < 8) return MOE_ERR_UNSUPPORTED;
-  if (prefer_weight_major(rows_max, E)) {
+  if (prefer_weight_major(rows_max, E, false)) {
     const moe_status st = launch_gate_up_wm(x_rows, offsets, E, d, F, rows_max, W_gu, h, s);
     if (st != MOE_ERR_UNSUPPORTED) return st;
   }
@@ -709,7 +712,7 @@ moe_status launch_down_tc(const void* h, const int32_t* offsets, int E, int d, i
                           const void* W_dn, const float* gate_of_row, int y_dtype, void* y_rows, cudaStream_t s) {
   if (rows_max == 0) return MOE_OK;
   if (F < BK || d < 8) return MOE_ERR_UNSUPPORTED;
-  if (prefer_weight_major(rows_max, E)) {
+  if (prefer_weight_major(rows_max, E, true)) {
     const moe_status st = launch_down_wm(h, offsets, E, d, F, rows_max, W_dn, gate_of_row, y_dtype, y_rows, s);
     if (st != MOE_ERR_UNSUPPORTED) return st;
   }
