@@ -34,9 +34,15 @@ UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM traffic (read + write bytes) of the dominant kernel, the gate/up GEMM, per launch, keyed
-# by (workload, dispatch), from an ncu capture of the same kernel build (summaries under
-# profiles/); absent when the kernel changed since the capture.
-GATE_UP_TRAFFIC = {}
+# by (workload, dispatch, kept rows), from ncu captures of the same kernel build
+# (profiles/gate_up_traffic.md); absent when the kernel changed since the capture.  The
+# stress workload's entry is the reduced shape's measured traffic / algorithmic ratio
+# (1.019) times the full launch's algorithmic bytes (the capture holds a quarter of the
+# tokens and experts; both the weight and the row bytes grow with the units).
+GATE_UP_TRAFFIC = {
+    ("c2_handbook", "permute", 65536): 931982080,
+    ("c5_stress", "permute", 131356): 8687124497,
+}
 
 
 def peaks():
