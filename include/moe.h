@@ -567,9 +567,10 @@ MOE_API moe_status moe_dequantize_fp4_host(const uint8_t* codes, const uint8_t* 
  * expert weights (weight-only: activations, H and the gated rows stay as in the bf16
  * calls).  [Handbook-Digest] "已确认", bullet "量化与推理" (routed experts in MXFP4;
  * NVFP4 with key layers kept in BF16).
- * The weights are the packed form of moe_quantize_fp4_host, in device memory:
+ * The weights are the packed form of moe_quantize_fp4_host, in device memory, with the
+ * scales rearranged once by moe_prepare_fp4_scales:
  *   codes         (device) [rows, K/2] bytes (element 2j in the low nibble of byte j)
- *   scales        (device) [rows, K / moe_fp4_block_size(fmt)] bytes
+ *   scales        (device) the prepared scales: moe_fp4_scales_bytes(rows, K, fmt) bytes
  *   tensor_scale  (device) [E] fp32, expert e's NVFP4 tensor scale (quantize each expert
  *                 separately); NULL for MXFP4
  *   gate/up: rows = E * 2F (expert e's F gate rows, then its F up rows), K = d;
@@ -583,6 +584,18 @@ MOE_API moe_status moe_dequantize_fp4_host(const uint8_t* codes, const uint8_t* 
  * negative size; UNSUPPORTED for E > 1024, d or F not a multiple of 64, fp32 activations
  * or an unaligned pointer.
  * ---------------------------------------------------------------------------------- */
+/* moe_prepare_fp4_scales -- the 4-bit GEMMs' scale layout, made once at load time.
+ *   scales  (device) [rows, K / block] bytes as moe_quantize_fp4_host writes them
+ *   out     (device) moe_fp4_scales_bytes(rows, K, fmt) bytes, 16-byte aligned: k-block
+ *           major, out[kb][row][j] = scales[row][kb * (64 / block) + j] for the K/64
+ *           k-blocks of 64 elements, followed in each k-block by 256 zero rows, so that one
+ *           k-block's scales of 128 consecutive rows are one contiguous copy.
+ * moe_fp4_scales_bytes returns 0 for a bad format, negative sizes or K % 64 != 0.
+ * Errors: INVALID_ARG for a null pointer, negative sizes or a bad format; UNSUPPORTED for
+ * K % 64 != 0 or an unaligned out; WORKSPACE when bytes is below the query. */
+MOE_API size_t moe_fp4_scales_bytes(int64_t rows, int32_t K, int32_t fmt);
+MOE_API moe_status moe_prepare_fp4_scales(const uint8_t* scales, int64_t rows, int32_t K, int32_t fmt,
+                     uint8_t* out, size_t bytes, void* stream);
 MOE_API moe_status moe_expert_gate_up_fp4(const void* x_rows, const int32_t* offsets, int32_t E,
                      int32_t d, int32_t F, int64_t rows_max, const uint8_t* codes,
                      const uint8_t* scales, int32_t fmt, const float* tensor_scale, void* h,

@@ -367,6 +367,22 @@ moe_status moe_grouped_ffn(const void* x_rows, int32_t dtype, const int32_t* off
   return moe_expert_down(h, dtype, offsets, E, d, F, rows_max, W_dn, gate_of_row, y_dtype, y_rows, stream);
 }
 
+size_t moe_fp4_scales_bytes(int64_t rows, int32_t K, int32_t fmt) {
+  if (rows < 0 || K < 0 || K % 64 != 0 || fp4_block(fmt) < 0) return 0;
+  return fp4_scales_bytes(rows, K, fmt);
+}
+
+moe_status moe_prepare_fp4_scales(const uint8_t* scales, int64_t rows, int32_t K, int32_t fmt, uint8_t* out,
+                                  size_t bytes, void* stream) {
+  if (rows < 0 || K < 0 || fp4_block(fmt) < 0) return MOE_ERR_INVALID_ARG;
+  if (K % 64 != 0) return MOE_ERR_UNSUPPORTED;
+  if (!out || (rows > 0 && K > 0 && !scales)) return MOE_ERR_INVALID_ARG;
+  if (bytes < fp4_scales_bytes(rows, K, fmt)) return MOE_ERR_WORKSPACE;
+  if (!aligned16(out)) return MOE_ERR_UNSUPPORTED;
+  if (K == 0) return MOE_OK;
+  return launch_prepare_fp4_scales(scales, rows, K, fmt, out, S(stream));
+}
+
 static moe_status check_fp4(const void* a, const int32_t* offsets, int32_t E, int32_t d, int32_t F, int64_t rows_max,
                             const uint8_t* codes, const uint8_t* scales, int32_t fmt, const float* tensor_scale,
                             const void* out) {

@@ -233,6 +233,9 @@ moe_status launch_gate_up_fp4(const void* x_rows, const int32_t* offsets, int E,
 moe_status launch_down_fp4(const void* h, const int32_t* offsets, int E, int d, int F, long long rows_max,
                            const uint8_t* codes, const uint8_t* scales, int fmt, const float* tensor_scale,
                            const float* gate_of_row, int y_dtype, void* y_rows, cudaStream_t s);
+size_t fp4_scales_bytes(long long rows, int K, int fmt);
+moe_status launch_prepare_fp4_scales(const uint8_t* scales, long long rows, int K, int fmt, uint8_t* out,
+                                     cudaStream_t s);
 // Whether a grouped GEMM over E experts and rows_max rows takes the weight-major tiles.
 bool prefer_weight_major(long long rows_max, int E, bool down);
 

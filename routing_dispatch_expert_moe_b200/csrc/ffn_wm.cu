@@ -38,6 +38,7 @@ constexpr int kWMaxE = 1024;
 constexpr uint32_t kWTmemCols = 512;
 constexpr int kWRows = 128;                     // weight rows per CTA (256 per pair)
 constexpr int kWBlock = kWRows * BK * 2;       // 16 KB: one 128-row operand block
+constexpr int kFp4PadRows = 2 * kWRows;        // zero rows after the prepared 4-bit scales
 
 template <int MODE>
 struct WmCfg {
@@ -307,26 +308,32 @@ grouped_gemm_wm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
 // =====================================================================================
 // 4-bit expert weights (weight-only): the same weight-major tiles, with each stage's
 // weight blocks arriving as packed E2M1 codes (a quarter of the bytes) and expanded to
-// bf16 in shared memory by four converter warps before the MMAs read them.
+// bf16 in shared memory by eight converter warps before the MMAs read them.
 //
 // Handbook digest (agihunt.info), "已确认", bullet "量化与推理": routed experts in MXFP4
 // (Kimi K3), NVFP4 training with key layers kept in BF16 (Nemotron 3).  The activations
 // stay bf16, and a kind::f16 MMA multiplies bf16 by bf16, so the weights are expanded:
 //   value = e2m1(code) * block scale, exact in bf16 (at most 2 significant bits times a
 //   power of two (MXFP4, E8M0 scale) or times an E4M3 scale of at most 4 bits (NVFP4));
-//   the NVFP4 per-tensor fp32 scale multiplies the fp32 accumulator in the epilogue.
-// Weight layout (as moe_quantize_fp4_host writes it): codes [rows, K/2] bytes, element 2j
-// in the low nibble of byte j; scales [rows, K/block] bytes (E8M0 for MXFP4, block 32;
-// E4M3 for NVFP4, block 16); K a multiple of 64.
+//   the NVFP4 per-expert fp32 tensor scale multiplies the fp32 accumulators.
+// Weights: codes [rows, K/2] bytes as moe_quantize_fp4_host writes them (element 2j in the
+// low nibble of byte j), loaded by TMA; scales in the k-block-major layout of
+// moe_prepare_fp4_scales, [K/64][rows + 256][64/block] bytes, so the scales of one
+// k-block of 128 rows are one contiguous 256- or 512-byte bulk copy (the 256 zero rows
+// cover the blocks of the last tiles that start past the matrix, at most 127 rows past
+// it).  K a multiple of 64.
 //
-// Per stage and CTA: TMA brings the codes of its weight rows (128 rows x 32 bytes per
-// block) and its token rows; a converter thread owns one weight row of each block: it
-// reads its row's 2 (MX) or 4 (NV) scale bytes for the k-block from global memory, looks
-// each code byte up in a 256-entry table of bf16 pairs, scales the pair and writes 16-byte
-// chunks into the 128-byte-swizzled operand layout the MMA reads (chunk c of row r at
-// r * 128 + ((c ^ (r & 7)) * 16)).  Barriers per stage: packed[s] (this CTA's TMA bytes),
-// full[s] on the even CTA (the 2 x 128 converter threads, after a proxy fence), empty[s]
-// (the MMAs' completion, both CTAs).
+// Per stage and CTA: the codes and scales of its weight rows and its token rows land by
+// TMA and bulk copy on the CTA's own `packed` barrier.  A converter thread owns one weight
+// row of a block (gate/up: 256 threads for the two blocks of 128 rows; down: two threads
+// per row, four 16-byte chunks each).  It decodes each 32-bit word of codes (eight
+// elements) in registers: the three magnitude bits of four codes at once select the high
+// and low bytes of their bf16 values from two 8-byte tables (byte permutes), the sign
+// bits are moved into place, and the bf16 pairs are multiplied by the block scale.  Each
+// 16-byte chunk goes to the 128-byte-swizzled operand layout (chunk c of row r at
+// r * 128 + ((c ^ (r & 7)) * 16)); then a proxy fence and an arrive on the even CTA's
+// `full` barrier (2 x 256 converter threads).  `empty` (the MMAs' completion) frees the
+// stage in both CTAs.
 // =====================================================================================
 template <int MODE>
 struct Wm4Cfg {
@@ -334,29 +341,24 @@ struct Wm4Cfg {
   static constexpr int a_blocks = WmCfg<MODE>::a_blocks;
   static constexpr int b_bytes = WmCfg<MODE>::b_bytes;
   static constexpr int packed_block = kWRows * BK / 2;          // 4 KB of codes per weight block
-  static constexpr int stage_bytes = a_blocks * kWBlock + b_bytes + a_blocks * packed_block;
+  static constexpr int scale_block = kWRows * 4;                // up to 4 scale bytes per row and k-block
+  static constexpr int stage_bytes = a_blocks * kWBlock + b_bytes + a_blocks * (packed_block + scale_block);
+  static constexpr int stage_pitch = (stage_bytes + 1023) / 1024 * 1024;
   static constexpr int stages = MODE == 0 ? 4 : 5;
-  static constexpr int epi_warps = 4, cvt_warps = 4;
+  static constexpr int epi_warps = 4, cvt_warps = 8;
+  static constexpr int cvt_threads = 32 * cvt_warps;
   static constexpr int threads = 64 + 32 * (epi_warps + cvt_warps);
-  static constexpr int bars = stages * stage_bytes;
+  static constexpr int bars = stages * stage_pitch;
   static constexpr int nbars = 3 * stages + 4 + 1;
   static constexpr int misc = bars + nbars * 8;
-  static constexpr int lut = (misc + 16 + 15) / 16 * 16;       // uint32 [256]: code byte -> bf16 pair
-  static constexpr int tiles = lut + 256 * 4;
+  static constexpr int tiles = (misc + 16 + 15) / 16 * 16;
   static constexpr int sh32 = tiles + (kWMaxE + 1) * 4;
   static constexpr int stage = (sh32 + 32 * 4 + 127) / 128 * 128;
   static constexpr int end = stage + epi_warps * kStageWarpBytes;
   static constexpr size_t smem = end + 1024;
   static_assert(smem <= 232448, "shared memory per CTA");
-  static_assert((a_blocks * kWBlock + b_bytes) % 1024 == 0 && stage_bytes % 1024 == 0, "swizzle alignment");
+  static_assert((a_blocks * kWBlock + b_bytes) % 1024 == 0, "swizzle alignment");
 };
-
-// bf16 bits of an E2M1 code: sign, then 0 / 0.5 (exponent field 0) or 2^(e-1) (1 + m/2).
-__device__ __forceinline__ uint32_t e2m1_bf16_bits(uint32_t c) {
-  const uint32_t e = (c >> 1) & 3u, m = c & 1u;
-  const uint32_t mag = e ? (((e + 126u) << 7) | (m << 6)) : (m ? 0x3F00u : 0u);
-  return ((c & 8u) << 12) | mag;
-}
 
 // bf16 of a block scale byte: E8M0 (2^(b - 127); b = 0 is 2^-127, a bf16 subnormal) or
 // E4M3 (normal 2^(e-7) (1 + m/8), subnormal m 2^-9).  Both exact in bf16.
@@ -369,25 +371,41 @@ __device__ __forceinline__ uint32_t scale_bf16_bits(uint32_t b) {
   return (uint32_t)(*reinterpret_cast<const uint16_t*>(&v));
 }
 
-// Expands one 128 x 64 block row of codes into bf16: 32 code bytes at src, scale bytes
-// packed little-endian in sc (2 for MX: chunks 0-3 and 4-7; 4 for NV: chunk pairs).
+// Eight E2M1 codes (w: element i in bits 4i .. 4i+3) -> eight bf16 values (o[0] holds
+// elements 0 and 1, ...).  The magnitude codes 0..7 are 0, 0.5, 1, 1.5, 2, 3, 4, 6, whose
+// bf16 high bytes are 00 3F 3F 3F 40 40 40 40 and low bytes 00 00 80 C0 00 40 80 C0.
+__device__ __forceinline__ void e2m1x8_to_bf16(uint32_t w, uint32_t (&o)[4]) {
+  constexpr uint32_t HI0 = 0x3F3F3F00u, HI1 = 0x40404040u, LO0 = 0xC0800000u, LO1 = 0xC0804000u;
+  const uint32_t m = w & 0x77777777u;
+  const uint32_t lo_a = __byte_perm(LO0, LO1, m), hi_a = __byte_perm(HI0, HI1, m);
+  const uint32_t lo_b = __byte_perm(LO0, LO1, m >> 16), hi_b = __byte_perm(HI0, HI1, m >> 16);
+  const uint32_t sg = w & 0x88888888u;
+  o[0] = __byte_perm(lo_a, hi_a, 0x5140) | ((sg & 0x8u) << 12) | ((sg & 0x80u) << 24);
+  o[1] = __byte_perm(lo_a, hi_a, 0x7362) | ((sg & 0x800u) << 4) | ((sg & 0x8000u) << 16);
+  o[2] = __byte_perm(lo_b, hi_b, 0x5140) | ((sg & 0x80000u) >> 4) | ((sg & 0x800000u) << 8);
+  o[3] = __byte_perm(lo_b, hi_b, 0x7362) | ((sg & 0x8000000u) >> 12) | (sg & 0x80000000u);
+}
+
+// Expands chunks [c0, c1) of one row of a block: codes at src (32 bytes), the row's scale
+// bytes packed little-endian in sc (MX: 2, chunks 0-3 and 4-7; NV: 4, chunk pairs).
 template <int FMT>
-__device__ __forceinline__ void convert_row(const uint8_t* src, uint32_t sc, const uint32_t* lut, uint8_t* dst_block,
-                                            int r) {
-  const uint4 c0 = *reinterpret_cast<const uint4*>(src);
-  const uint4 c1 = *reinterpret_cast<const uint4*>(src + 16);
-  const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+__device__ __forceinline__ void convert_chunks(const uint8_t* src, uint32_t sc, uint8_t* dst_block, int r, int c0,
+                                               int c1) {
+  const uint4 q0 = *reinterpret_cast<const uint4*>(src);
+  const uint4 q1 = *reinterpret_cast<const uint4*>(src + 16);
+  const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
 #pragma unroll
-  for (int c = 0; c < 8; ++c) {                 // chunk c: elements 8c .. 8c+7 (code bytes 4c .. 4c+3)
+  for (int c = 0; c < 8; ++c) {
+    if (c < c0 || c >= c1) continue;
     const uint32_t sb = FMT == MOE_FP4_MX ? scale_bf16_bits<FMT>((sc >> (8 * (c >> 2))) & 0xffu)
                                           : scale_bf16_bits<FMT>((sc >> (8 * (c >> 1))) & 0xffu);
-    const __nv_bfloat162 s2 = __halves2bfloat162(*reinterpret_cast<const __nv_bfloat16*>(&sb),
-                                                 *reinterpret_cast<const __nv_bfloat16*>(&sb));
+    const uint32_t s2u = sb | (sb << 16);
+    const __nv_bfloat162 s2 = *reinterpret_cast<const __nv_bfloat162*>(&s2u);
     uint32_t o[4];
+    e2m1x8_to_bf16(w[c], o);
 #pragma unroll
     for (int b = 0; b < 4; ++b) {
-      const uint32_t pair = lut[(w[c] >> (8 * b)) & 0xffu];
-      __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&pair);
+      __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&o[b]);
       v = __hmul2(v, s2);                       // exact: at most 6 significant bits
       o[b] = *reinterpret_cast<uint32_t*>(&v);
     }
@@ -395,20 +413,28 @@ __device__ __forceinline__ void convert_row(const uint8_t* src, uint32_t sc, con
   }
 }
 
+// One-dimensional bulk copy global -> this CTA's shared memory, completing on an mbarrier.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
 template <int MODE, int FMT, typename OutT>
 __global__ void __launch_bounds__(Wm4Cfg<MODE>::threads, 1)
 grouped_gemm_wm4_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmX,
-                        const uint8_t* __restrict__ scales, const float* __restrict__ tensor_scale,
+                        const uint8_t* __restrict__ scales_t, const float* __restrict__ tensor_scale,
                         const int32_t* __restrict__ offsets, int E, int K, int d, int F, long long rows_max,
                         const float* __restrict__ gate_of_row, OutT* __restrict__ out, int* err) {
   using C = Wm4Cfg<MODE>;
+  constexpr int kBlockElems = FMT == MOE_FP4_MX ? 32 : 16;
+  constexpr int kSpr = BK / kBlockElems;                    // scale bytes per row and k-block
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int* tile_start = reinterpret_cast<int*>(smem + C::tiles);
   int* sh32 = reinterpret_cast<int*>(smem + C::sh32);
-  uint32_t* lut = reinterpret_cast<uint32_t*>(smem + C::lut);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::misc + 4);
   const uint32_t rank = cluster_ctarank();
@@ -425,16 +451,19 @@ grouped_gemm_wm4_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_co
   const uint32_t bar_tfull = bar_empty + 8 * C::stages;
   const uint32_t bar_tempty = bar_tfull + 16;
   const uint32_t bar_fin = bar_tempty + 16;
-  auto a_off = [&](int s, int a) { return s * C::stage_bytes + a * kWBlock; };
-  auto b_off = [&](int s) { return s * C::stage_bytes + C::a_blocks * kWBlock; };
-  auto p_off = [&](int s, int a) { return s * C::stage_bytes + C::a_blocks * kWBlock + C::b_bytes + a * C::packed_block; };
+  auto a_off = [&](int s, int a) { return s * C::stage_pitch + a * kWBlock; };
+  auto b_off = [&](int s) { return s * C::stage_pitch + C::a_blocks * kWBlock; };
+  auto p_off = [&](int s, int a) { return s * C::stage_pitch + C::a_blocks * kWBlock + C::b_bytes + a * C::packed_block; };
+  auto s_off = [&](int s, int a) {
+    return s * C::stage_pitch + C::a_blocks * (kWBlock + C::packed_block) + C::b_bytes + a * C::scale_block;
+  };
+  const long long rows_total = MODE == 0 ? (long long)E * 2 * F : (long long)E * d;
+  const long long rows_pad = rows_total + kFp4PadRows;     // the prepared scales' row count
 
-  for (int i = threadIdx.x; i < 256; i += blockDim.x)
-    lut[i] = e2m1_bf16_bits(i & 15u) | (e2m1_bf16_bits(i >> 4) << 16);   // low nibble = lower element
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::stages; ++s) {
       mbar_init(bar_packed + 8 * s, 1);
-      mbar_init(bar_full + 8 * s, 2 * 32 * C::cvt_warps);
+      mbar_init(bar_full + 8 * s, 2 * C::cvt_threads);
       mbar_init(bar_empty + 8 * s, 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -457,8 +486,6 @@ grouped_gemm_wm4_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_co
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int KB = K / BK;                                     // K is a multiple of 64
-  constexpr int kBlockElems = FMT == MOE_FP4_MX ? 32 : 16;
-  const long long scale_ld = K / kBlockElems;                // scale bytes per weight row
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer (both CTAs)
@@ -478,9 +505,14 @@ grouped_gemm_wm4_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_co
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1u, abort_flag, err)) { ok = false; break; }
           const uint32_t pk = bar_packed + 8 * stage;
-          mbar_expect_tx(pk, (uint32_t)(C::a_blocks * C::packed_block + C::b_bytes));
-          tma_load_2d(sb + (uint32_t)p_off(stage, 0), &tmC, pk, kb * (BK / 2), w_row);
-          if (MODE == 0) tma_load_2d(sb + (uint32_t)p_off(stage, 1), &tmC, pk, kb * (BK / 2), w_row + F);
+          mbar_expect_tx(pk, (uint32_t)(C::a_blocks * (C::packed_block + kWRows * kSpr) + C::b_bytes));
+#pragma unroll
+          for (int a = 0; a < C::a_blocks; ++a) {
+            const int row = w_row + (a ? F : 0);
+            tma_load_2d(sb + (uint32_t)p_off(stage, a), &tmC, pk, kb * (BK / 2), row);
+            bulk_load(sb + (uint32_t)s_off(stage, a), scales_t + ((long long)kb * rows_pad + row) * kSpr,
+                      (uint32_t)(kWRows * kSpr), pk);
+          }
           tma_load_2d(sb + (uint32_t)b_off(stage), &tmX, pk, kb * BK, x_row);
           last_phase[stage] = (int)phase;
           if (++stage == C::stages) { stage = 0; phase ^= 1u; }
@@ -548,37 +580,26 @@ grouped_gemm_wm4_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_co
     }
   } else {
     // ------------------------------------------------------------ converters (both CTAs)
-    const int r = threadIdx.x - 64 - 32 * C::epi_warps;     // the weight row of each block it expands
+    const int ct = threadIdx.x - 64 - 32 * C::epi_warps;     // 0 .. cvt_threads - 1
+    const int r = ct & (kWRows - 1);                         // its weight row of the block
+    const int a = MODE == 0 ? ct / kWRows : 0;               // gate/up: block (gate or up)
+    const int c0 = MODE == 0 ? 0 : (ct / kWRows) * 4;        // down: half of the row's chunks
+    const int c1 = MODE == 0 ? 8 : c0 + 4;
     int stage = 0;
     uint32_t phase = 0;
-    for (int tile = cid; tile < total; tile += ncl) {
-      const TileCoord tc = tile_coord(tile_start, offsets, E, C::NT, tile);
-      const long long w_row = MODE == 0 ? (long long)tc.e * 2 * F + tc.n_tile * 256 + (int)rank * kWRows + r
-                                        : (long long)tc.e * d + tc.n_tile * 256 + (int)rank * kWRows + r;
-      // rows past the weight matrix (the last tile's padding) read no scales
-      const long long rows_total = MODE == 0 ? (long long)E * 2 * F : (long long)E * d;
-      bool ok = true;
+    bool ok = true;
+    for (int tile = cid; ok && tile < total; tile += ncl) {
       for (int kb = 0; kb < KB; ++kb) {
-        uint32_t sc[2] = {0u, 0u};
-#pragma unroll
-        for (int a = 0; a < C::a_blocks; ++a) {
-          const long long row = w_row + (a ? F : 0);
-          if (row < rows_total) {
-            const uint8_t* p = scales + row * scale_ld + (long long)kb * (BK / kBlockElems);
-            sc[a] = FMT == MOE_FP4_MX ? (uint32_t)__ldg(reinterpret_cast<const uint16_t*>(p))
-                                      : __ldg(reinterpret_cast<const uint32_t*>(p));
-          }
-        }
         const bool got = mbar_wait(bar_packed + 8 * stage, phase, abort_flag, err);
         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-#pragma unroll
-        for (int a = 0; a < C::a_blocks; ++a)
-          convert_row<FMT>(smem + p_off(stage, a) + r * (BK / 2), sc[a], lut, smem + a_off(stage, a), r);
+        const uint8_t* sc_p = smem + s_off(stage, a) + r * kSpr;
+        const uint32_t sc = FMT == MOE_FP4_MX ? (uint32_t)*reinterpret_cast<const uint16_t*>(sc_p)
+                                              : *reinterpret_cast<const uint32_t*>(sc_p);
+        convert_chunks<FMT>(smem + p_off(stage, a) + r * (BK / 2), sc, smem + a_off(stage, a), r, c0, c1);
         fence_proxy_async_smem();                           // the MMAs read these through the async proxy
         mbar_arrive_cluster(map_to_rank(bar_full + 8 * stage, 0));
         if (++stage == C::stages) { stage = 0; phase ^= 1u; }
       }
-      if (!ok) break;
     }
   }
 
@@ -591,7 +612,7 @@ grouped_gemm_wm4_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_co
 }
 
 template <int MODE, int FMT, typename OutT>
-moe_status launch_wm4(const CUtensorMap& mc, const CUtensorMap& mx, const uint8_t* scales, const float* tscale,
+moe_status launch_wm4(const CUtensorMap& mc, const CUtensorMap& mx, const uint8_t* scales_t, const float* tscale,
                       const int32_t* offsets, int E, int K, int d, int F, long long rows_max, const float* gate_of_row,
                       void* out, cudaStream_t s) {
   using C = Wm4Cfg<MODE>;
@@ -614,9 +635,25 @@ moe_status launch_wm4(const CUtensorMap& mc, const CUtensorMap& mx, const uint8_
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cuda_status(cudaLaunchKernelEx(&cfg, grouped_gemm_wm4_kernel<MODE, FMT, OutT>, mc, mx, scales, tscale,
+  return cuda_status(cudaLaunchKernelEx(&cfg, grouped_gemm_wm4_kernel<MODE, FMT, OutT>, mc, mx, scales_t, tscale,
                                         offsets, E, K, d, F, rows_max, gate_of_row, static_cast<OutT*>(out),
                                         err_ptr()));
+}
+
+// The k-block-major scale layout: out[kb][row][j] = in[row][kb * (64/block) + j] for
+// rows < rows_total, zero for the padding rows.  One byte per thread, grid-stride.
+__global__ void __launch_bounds__(256)
+fp4_scales_kernel(const uint8_t* __restrict__ in, long long rows, int K, int spr, uint8_t* __restrict__ out) {
+  const long long rows_pad = rows + kFp4PadRows;
+  const long long per_kb = rows_pad * spr;
+  const long long n = (long long)(K / BK) * per_kb;
+  const long long ld = K / (BK / spr);                       // scale bytes per row of the input
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const long long kb = i / per_kb, rem = i - kb * per_kb;
+    const long long row = rem / spr;
+    const int j = (int)(rem - row * spr);
+    out[i] = row < rows ? __ldg(in + row * ld + kb * spr + j) : (uint8_t)0;
+  }
 }
 
 template <int MODE, typename OutT>
@@ -648,6 +685,24 @@ moe_status launch_wm(const CUtensorMap& mw, const CUtensorMap& mx, const int32_t
 
 }  // namespace
 
+size_t fp4_scales_bytes(long long rows, int K, int fmt) {
+  const int spr = BK / (fmt == MOE_FP4_MX ? 32 : 16);
+  return (size_t)(K / BK) * (size_t)(rows + kFp4PadRows) * spr;
+}
+
+moe_status launch_prepare_fp4_scales(const uint8_t* scales, long long rows, int K, int fmt, uint8_t* out,
+                                     cudaStream_t s) {
+  const int spr = BK / (fmt == MOE_FP4_MX ? 32 : 16);
+  const long long n = (long long)(K / BK) * (rows + kFp4PadRows) * spr;
+  long long blocks = (n + 255) / 256;
+  const long long cap = (long long)num_sms() * 16;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  fp4_scales_kernel<<<(unsigned)blocks, 256, 0, s>>>(scales, rows, K, spr, out);
+  return check_launch();
+}
+
+
 // Gate/up, weight-major: H [rows_max, F] bf16 from x_perm [rows_max, d] and W_gu [E][2F][d].
 moe_status launch_gate_up_wm(const void* x_rows, const int32_t* offsets, int E, int d, int F, long long rows_max,
                              const void* W_gu, void* h, cudaStream_t s) {
@@ -671,26 +726,26 @@ moe_status launch_down_wm(const void* h, const int32_t* offsets, int E, int d, i
   return launch_wm<1, __nv_bfloat16>(mw, mx, offsets, E, F, d, F, rows_max, gate_of_row, y_rows, s);
 }
 
-// Gate/up and down with 4-bit weights, weight-major.  Codes [rows, K/2] and scales
-// [rows, K / block] as moe_quantize_fp4_host writes them (rows = E 2F or E d); tensor_scale
-// [E] fp32 per expert (NVFP4) or NULL (MXFP4).  K (d for gate/up, F for down) must be a
-// multiple of 64.
+// Gate/up and down with 4-bit weights, weight-major.  Codes [rows, K/2] as
+// moe_quantize_fp4_host writes them (rows = E 2F or E d), scales in the layout of
+// launch_prepare_fp4_scales; tensor_scale [E] fp32 per expert (NVFP4) or NULL (MXFP4).  K
+// (d for gate/up, F for down) must be a multiple of 64.
 moe_status launch_gate_up_fp4(const void* x_rows, const int32_t* offsets, int E, int d, int F, long long rows_max,
-                              const uint8_t* codes, const uint8_t* scales, int fmt, const float* tensor_scale,
+                              const uint8_t* codes, const uint8_t* scales_t, int fmt, const float* tensor_scale,
                               void* h, cudaStream_t s) {
   if (rows_max == 0) return MOE_OK;
   CUtensorMap mc, mx;
   if (!make_map_u8(&mc, codes, (unsigned long long)E * 2 * F, d / 2, BK / 2, kWRows)) return MOE_ERR_UNSUPPORTED;
   if (!make_map(&mx, x_rows, (unsigned long long)rows_max, d, WmCfg<0>::NT / 2)) return MOE_ERR_UNSUPPORTED;
   if (fmt == MOE_FP4_MX)
-    return launch_wm4<0, MOE_FP4_MX, __nv_bfloat16>(mc, mx, scales, nullptr, offsets, E, d, d, F, rows_max, nullptr,
-                                                     h, s);
-  return launch_wm4<0, MOE_FP4_NV, __nv_bfloat16>(mc, mx, scales, tensor_scale, offsets, E, d, d, F, rows_max,
+    return launch_wm4<0, MOE_FP4_MX, __nv_bfloat16>(mc, mx, scales_t, nullptr, offsets, E, d, d, F, rows_max,
+                                                     nullptr, h, s);
+  return launch_wm4<0, MOE_FP4_NV, __nv_bfloat16>(mc, mx, scales_t, tensor_scale, offsets, E, d, d, F, rows_max,
                                                    nullptr, h, s);
 }
 
 moe_status launch_down_fp4(const void* h, const int32_t* offsets, int E, int d, int F, long long rows_max,
-                           const uint8_t* codes, const uint8_t* scales, int fmt, const float* tensor_scale,
+                           const uint8_t* codes, const uint8_t* scales_t, int fmt, const float* tensor_scale,
                            const float* gate_of_row, int y_dtype, void* y_rows, cudaStream_t s) {
   if (rows_max == 0) return MOE_OK;
   CUtensorMap mc, mx;
@@ -698,7 +753,7 @@ moe_status launch_down_fp4(const void* h, const int32_t* offsets, int E, int d, 
   if (!make_map(&mx, h, (unsigned long long)rows_max, F, WmCfg<1>::NT / 2)) return MOE_ERR_UNSUPPORTED;
   const float* ts = fmt == MOE_FP4_NV ? tensor_scale : nullptr;
 #define MOE_WM4(FMT, T) \
-  return launch_wm4<1, FMT, T>(mc, mx, scales, ts, offsets, E, F, d, F, rows_max, gate_of_row, y_rows, s)
+  return launch_wm4<1, FMT, T>(mc, mx, scales_t, ts, offsets, E, F, d, F, rows_max, gate_of_row, y_rows, s)
   if (fmt == MOE_FP4_MX) {
     if (y_dtype == MOE_F32) MOE_WM4(MOE_FP4_MX, float);
     MOE_WM4(MOE_FP4_MX, __nv_bfloat16);

@@ -82,6 +82,8 @@ _SIGNATURES = {
     "moe_get_device_error": (_i32, [ctypes.POINTER(_i32), _c_void_p]),
     "moe_zero": (_i32, [_c_void_p, _size, _c_void_p]),
     "moe_round_output": (_i32, [_c_void_p, _i64, _c_void_p, _i32, _c_void_p]),
+    "moe_fp4_scales_bytes": (_size, [_i64, _i32, _i32]),
+    "moe_prepare_fp4_scales": (_i32, [_c_void_p, _i64, _i32, _i32, _c_void_p, _size, _c_void_p]),
     "moe_expert_gate_up_fp4": (_i32, [_c_void_p, _c_void_p, _i32, _i32, _i32, _i64, _c_void_p, _c_void_p, _i32,
                                       _c_void_p, _c_void_p, _c_void_p]),
     "moe_expert_down_fp4": (_i32, [_c_void_p, _c_void_p, _i32, _i32, _i32, _i64, _c_void_p, _c_void_p, _i32,
@@ -326,14 +328,26 @@ def moe_dequantize_fp4_host(codes, scales, tensor_scale, K: int, fmt: str = "mxf
 
 
 class Fp4Weights:
-    """One expert weight tensor in a 4-bit format, on the device: codes [rows, K/2] uint8,
-    scales [rows, K/block] uint8 and, for NVFP4, tensor_scale [E] f32 (one per expert).
-    rows = E * 2F for W_gu (gate rows then up rows per expert), E * d for W_dn."""
+    """One expert weight tensor in a 4-bit format, on the device: codes [rows, K/2] uint8 and
+    scales [rows, K/block] uint8 as moe_quantize_fp4_host writes them and, for NVFP4,
+    tensor_scale [E] f32 (one per expert).  rows = E * 2F for W_gu (gate rows then up rows
+    per expert), E * d for W_dn.  The scales are rearranged once here for the GEMMs
+    (moe_prepare_fp4_scales); .scales keeps the packer's layout."""
 
-    def __init__(self, fmt: str, codes, scales, tensor_scale=None):
+    def __init__(self, fmt: str, codes, scales, tensor_scale=None, stream=None):
         if fmt not in FP4:
             raise ValueError(f"fmt must be one of {sorted(FP4)}")
         self.fmt, self.codes, self.scales, self.tensor_scale = fmt, codes, scales, tensor_scale
+        rows, half = codes.shape
+        K = 2 * half
+        _need(codes, "codes", torch.uint8)
+        _need(scales, "scales", torch.uint8)
+        nb = int(lib().moe_fp4_scales_bytes(rows, K, FP4[fmt]))
+        if nb == 0:
+            raise ValueError("K must be a multiple of 64")
+        self.scales_prepared = torch.empty(nb, dtype=torch.uint8, device=codes.device)
+        _check("moe_prepare_fp4_scales", lib().moe_prepare_fp4_scales(
+            _p(scales), rows, K, FP4[fmt], _p(self.scales_prepared), nb, _stream(stream)))
 
 
 def quantize_experts_fp4(W, fmt: str = "mxfp4", device="cuda", threads: int = 0) -> Fp4Weights:
@@ -375,7 +389,7 @@ def moe_expert_gate_up_fp4(x_rows, offsets, W_gu: Fp4Weights, E: int, F: int, ro
     h = torch.empty((max(rows_max, 1), F), dtype=torch.bfloat16, device=x_rows.device) if h is None else \
         _need(h, "h", torch.bfloat16)
     _check("moe_expert_gate_up_fp4", lib().moe_expert_gate_up_fp4(
-        _p(x_rows), _p(offsets), E, d, F, rows_max, _p(W_gu.codes), _p(W_gu.scales), FP4[W_gu.fmt],
+        _p(x_rows), _p(offsets), E, d, F, rows_max, _p(W_gu.codes), _p(W_gu.scales_prepared), FP4[W_gu.fmt],
         _p(W_gu.tensor_scale), _p(h), _stream(stream)))
     return h
 
@@ -393,7 +407,7 @@ def moe_expert_down_fp4(h, offsets, W_dn: Fp4Weights, E: int, d: int, rows_max: 
     y_rows = torch.empty((max(rows_max, 1), d), dtype=y_dtype, device=h.device) if y_rows is None else \
         _need(y_rows, "y_rows")
     _check("moe_expert_down_fp4", lib().moe_expert_down_fp4(
-        _p(h), _p(offsets), E, d, F, rows_max, _p(W_dn.codes), _p(W_dn.scales), FP4[W_dn.fmt],
+        _p(h), _p(offsets), E, d, F, rows_max, _p(W_dn.codes), _p(W_dn.scales_prepared), FP4[W_dn.fmt],
         _p(W_dn.tensor_scale), _p(gate_of_row), _dt(y_rows), _p(y_rows), _stream(stream)))
     return y_rows
 

@@ -327,3 +327,18 @@ def test_fp4_gemm_host_validation(L):
     assert g(rows=0, x=NUL, out=NUL) == 0                  # nothing to do
     assert dn(FAKE, FAKE, 8, 128, 64, 100, FAKE, FAKE, 0, NUL, NUL, 7, FAKE, NUL) == 1   # output dtype
     assert dn(FAKE, FAKE, 8, 128, 64, 100, FAKE, FAKE, 1, NUL, NUL, 0, FAKE, NUL) == 1   # NVFP4 without scales
+
+
+def test_fp4_scale_preparation_size_and_validation(L):
+    # k-block-major with 256 zero rows per k-block: (K/64) * (rows + 256) * (64 / block) bytes
+    assert L.moe_fp4_scales_bytes(512, 7168, 0) == (7168 // 64) * (512 + 256) * 2
+    assert L.moe_fp4_scales_bytes(512, 256, 1) == (256 // 64) * (512 + 256) * 4
+    assert L.moe_fp4_scales_bytes(512, 96, 0) == 0 and L.moe_fp4_scales_bytes(512, 128, 5) == 0
+    f = L.moe_prepare_fp4_scales       # (scales, rows, K, fmt, out, bytes, stream)
+    nb = L.moe_fp4_scales_bytes(512, 128, 0)
+    assert f(FAKE, 512, 128, 0, NUL, nb, NUL) == 1
+    assert f(NUL, 512, 128, 0, FAKE, nb, NUL) == 1
+    assert f(FAKE, 512, 128, 7, FAKE, nb, NUL) == 1
+    assert f(FAKE, 512, 96, 0, FAKE, nb, NUL) == 2
+    assert f(FAKE, 512, 128, 0, FAKE, nb - 1, NUL) == 3
+    assert f(FAKE, 512, 128, 0, ctypes.c_void_p(4100), nb, NUL) == 2

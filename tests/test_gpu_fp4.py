@@ -73,6 +73,21 @@ def _groups(E, rows_each, seed):
     return counts, offsets
 
 
+# ------------------------------------------------------------------ the prepared scale layout
+@pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4"])
+def test_prepared_scales_are_the_documented_rearrangement(fmt):
+    rows, K = 384, 320
+    _, scales, _ = synthetic_fp4(rows, K, fmt, seed=9)
+    w = to_device(fmt, np.zeros((rows, K // 2), np.uint8), scales, np.ones(1, np.float32) if fmt == "nvfp4" else None)
+    torch.cuda.synchronize()
+    spr = 64 // (32 if fmt == "mxfp4" else 16)
+    want = np.zeros((K // 64, rows + 256, spr), np.uint8)
+    for kb in range(K // 64):
+        want[kb, :rows] = scales[:, kb * spr:(kb + 1) * spr]
+    got = w.scales_prepared.cpu().numpy()
+    assert got.size == want.size and np.array_equal(got.reshape(want.shape), want)
+
+
 # ------------------------------------------------------------------ exact against the bf16 GEMMs
 @pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4"])
 @pytest.mark.parametrize("E,d,F,rows_each", [(5, 128, 192, [0, 1, 45, 300, 129]), (3, 256, 64, [256, 97, 33]),
