@@ -151,6 +151,7 @@ struct RouterGeom {
   int NE, n_tiles;
 };
 RouterGeom router_geom(int E);
+bool router_side_by_side(int NE);
 size_t router_weight_bytes(int d, int E);          // prepared (split) weight; 0 = no tensor-core router
 bool tc_router_applies(int x_dtype, int T, int d, int E);
 moe_status launch_prepare_router_weight(const float* Wg, int d, int E, void* W3, cudaStream_t s);

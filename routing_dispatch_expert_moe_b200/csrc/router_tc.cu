@@ -45,6 +45,8 @@
 #include "tc_prims.cuh"
 
 #include <float.h>
+#include <stdlib.h>
+#include <string.h>
 
 namespace moe {
 namespace {
@@ -226,7 +228,11 @@ __device__ __forceinline__ void topk_write(const TopK<KMAX, BIAS>& st, long long
   }
 }
 
-template <int KMAX, bool BIAS>
+// SIDE: the three terms side by side in one MMA of N = 3 NE (NE <= 64), summed in the
+// epilogue, instead of three MMAs of N = NE into one accumulator: at small NE, four wide
+// MMAs per k-block instead of twelve narrow ones.  The prepared weight is the same (a
+// tile's hi, mid, lo rows are contiguous); each CTA loads its 3 NE / 2 rows in one box.
+template <int KMAX, bool BIAS, bool SIDE>
 __global__ void __launch_bounds__(kRThreads, 1)
 router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW, int T, int d,
                  int E, int NE, int n_tiles, int stages, const float* __restrict__ logit_offset,
@@ -298,8 +304,12 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
           if (rank == 0) mbar_expect_tx(bar_full + 8 * stage, 2u * (uint32_t)(kRAStage + 3 * term_bytes));
           const uint32_t full_c = map_to_rank(bar_full + 8 * stage, 0);
           tma_load_2d_pair(a_stage(stage), &tmX, full_c, kb * BK, a_row);
+          if (SIDE) {
+            tma_load_2d_pair(b_stage(stage, 0), &tmW, full_c, kb * BK, j * 3 * NE + (int)rank * (3 * half));
+          } else {
 #pragma unroll
-          for (int t = 0; t < 3; ++t) tma_load_2d_pair(b_stage(stage, t), &tmW, full_c, kb * BK, b_row + t * NE);
+            for (int t = 0; t < 3; ++t) tma_load_2d_pair(b_stage(stage, t), &tmW, full_c, kb * BK, b_row + t * NE);
+          }
           last_phase[stage] = (int)phase;
           if (++stage == stages) { stage = 0; phase ^= 1u; }
         }
@@ -312,7 +322,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (even CTA)
     if (lane == 0 && rank == 0) {
-      const uint32_t idesc = make_idesc(2 * RBM, NE);
+      const uint32_t idesc = make_idesc(2 * RBM, SIDE ? 3 * NE : NE);
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
@@ -331,10 +341,15 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
 #pragma unroll
           for (int t = 0; t < 3; ++t) bdesc[t] = sw128_desc(b_stage(stage, t));
 #pragma unroll
-          for (int kk = 0; kk < BK / UMMA_K; ++kk)
+          for (int kk = 0; kk < BK / UMMA_K; ++kk) {
+            if (SIDE) {                   // columns [0, NE) hi, [NE, 2 NE) mid, [2 NE, 3 NE) lo
+              umma_bf16_pair(d_tmem, adesc + 2 * kk, bdesc[0] + 2 * kk, idesc, (kb | kk) != 0 ? 1u : 0u);
+            } else {
 #pragma unroll
-            for (int t = 0; t < 3; ++t)   // +32 bytes along K per step (>> 4 = 2)
-              umma_bf16_pair(d_tmem, adesc + 2 * kk, bdesc[t] + 2 * kk, idesc, (kb | kk | t) != 0 ? 1u : 0u);
+              for (int t = 0; t < 3; ++t)   // +32 bytes along K per step (>> 4 = 2)
+                umma_bf16_pair(d_tmem, adesc + 2 * kk, bdesc[t] + 2 * kk, idesc, (kb | kk | t) != 0 ? 1u : 0u);
+            }
+          }
           umma_commit_pair_both(bar_empty + 8 * stage);
           if (++stage == stages) { stage = 0; phase ^= 1u; }
         }
@@ -366,15 +381,30 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
 #pragma unroll 1
       for (int c = 0; c < NE / 32; ++c) {
         uint32_t v[32];
-        tmem_ld32(taddr + c * 32, v);
-        tmem_wait_ld();
-        tmem_regs_ready(v);
         float lv[32];
+        tmem_ld32(taddr + c * 32, v);
+        if (SIDE) {
+          uint32_t v1[32], v2[32];
+          tmem_ld32(taddr + NE + c * 32, v1);
+          tmem_ld32(taddr + 2 * NE + c * 32, v2);
+          tmem_wait_ld();
+          tmem_regs_ready(v);
+          tmem_regs_ready(v1);
+          tmem_regs_ready(v2);
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            lv[i] = (__uint_as_float(v[i]) + __uint_as_float(v1[i])) + __uint_as_float(v2[i]);
+        } else {
+          tmem_wait_ld();
+          tmem_regs_ready(v);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) lv[i] = __uint_as_float(v[i]);
+        }
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const int e = e0 + c * 32 + i;
           const float off = (logit_offset && e < E) ? __ldg(logit_offset + e) : 0.f;
-          lv[i] = __uint_as_float(v[i]) + off;
+          lv[i] += off;
         }
         stage_store32<float>(stage, lv, lane, logits, row0, wrows, E, e0 + c * 32, E);
         if constexpr (kFused) {
@@ -435,12 +465,12 @@ prepare_router_weight_kernel(const float* __restrict__ Wg, int d, int E, int NE,
   }
 }
 
-template <int KMAX, bool BIAS>
+template <int KMAX, bool BIAS, bool SIDE>
 moe_status launch_router_kernel(const CUtensorMap& mx, const CUtensorMap& mw, int T, int d, int E, int NE,
                                 int n_tiles, const float* off, float* logits, const float* sel_bias, int k,
                                 int score, int renorm, float scale, int32_t* idx, float* gate, cudaStream_t s) {
   static std::atomic<int> configured[kMaxDevices];
-  moe_status st = ensure_smem_limit(configured, router_tc_kernel<KMAX, BIAS>, (size_t)kRSmemLimit);
+  moe_status st = ensure_smem_limit(configured, router_tc_kernel<KMAX, BIAS, SIDE>, (size_t)kRSmemLimit);
   if (st != MOE_OK) return st;
   // as many stages as fit next to the epilogue staging
   int stages = kRMaxStages;
@@ -463,11 +493,21 @@ moe_status launch_router_kernel(const CUtensorMap& mx, const CUtensorMap& mw, in
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cuda_status(cudaLaunchKernelEx(&cfg, router_tc_kernel<KMAX, BIAS>, mx, mw, T, d, E, NE, n_tiles, stages, off,
+  return cuda_status(cudaLaunchKernelEx(&cfg, router_tc_kernel<KMAX, BIAS, SIDE>, mx, mw, T, d, E, NE, n_tiles, stages, off,
                                         logits, sel_bias, k, score, renorm, scale, idx, gate, err_ptr()));
 }
 
 }  // namespace
+
+// The side-by-side layout applies while the three terms fit one MMA (3 NE <= 256 columns,
+// 3 NE / 2 rows per CTA in one TMA box); MOE_B200_ROUTER_TERMS=stacked|side forces one
+// (for measuring one against the other).
+bool router_side_by_side(int NE) {
+  const char* v = getenv("MOE_B200_ROUTER_TERMS");
+  if (v && strcmp(v, "stacked") == 0) return false;
+  if (v && strcmp(v, "side") == 0) return NE <= 64;
+  return NE <= 64;
+}
 
 RouterGeom router_geom(int E) {
   RouterGeom g;
@@ -506,11 +546,16 @@ moe_status launch_router_tc(const void* x, int T, int d, int E, const void* W3, 
   const RouterGeom g = router_geom(E);
   CUtensorMap mx, mw;
   if (!make_map(&mx, x, (unsigned long long)T, d, RBM)) return MOE_ERR_UNSUPPORTED;
-  if (!make_map(&mw, W3, (unsigned long long)g.n_tiles * 3 * g.NE, d, g.NE / 2)) return MOE_ERR_UNSUPPORTED;
+  const unsigned box = router_side_by_side(g.NE) ? 3 * g.NE / 2 : g.NE / 2;
+  if (!make_map(&mw, W3, (unsigned long long)g.n_tiles * 3 * g.NE, d, box)) return MOE_ERR_UNSUPPORTED;
   const bool bias = sel_bias != nullptr;
-#define MOE_RT(KM, B)                                                                                         \
-  return launch_router_kernel<KM, B>(mx, mw, T, d, E, g.NE, g.n_tiles, logit_offset, logits, sel_bias, fuse_k, \
-                                     score, renorm, scale, topk_idx, topk_gate, s)
+  // NE <= 64: the three terms side by side (one MMA of N = 3 NE per k step)
+  const bool side = router_side_by_side(g.NE);
+#define MOE_RT(KM, B)                                                                                               \
+  return side ? launch_router_kernel<KM, B, true>(mx, mw, T, d, E, g.NE, g.n_tiles, logit_offset, logits, sel_bias, \
+                                                  fuse_k, score, renorm, scale, topk_idx, topk_gate, s)             \
+              : launch_router_kernel<KM, B, false>(mx, mw, T, d, E, g.NE, g.n_tiles, logit_offset, logits,         \
+                                                   sel_bias, fuse_k, score, renorm, scale, topk_idx, topk_gate, s)
   if (fuse_k <= 0) MOE_RT(0, false);
   if (fuse_k <= 8) {
     if (bias) MOE_RT(8, true);

@@ -231,3 +231,20 @@ def test_router_general_fp32_weights(T, d, E, k, score, renorm, with_bias):
         tb = tb * 0.25 + 1e-12                                 # score slope <= 1/4 (sigmoid)
     sure = O.decision_margin(o["keys"], k) > 2 * tb
     assert np.array_equal(gi[sure], o["topk_idx"][sure])
+
+
+@pytest.mark.parametrize("terms", ["side", "stacked"])
+@pytest.mark.parametrize("T,d,E,k,score", [(512, 256, 64, 8, "softmax"), (300, 128, 8, 2, "sigmoid"),
+                                          (700, 512, 36, 4, "sqrt_softplus")])
+def test_router_both_term_layouts_bit_exact(T, d, E, k, score, terms, monkeypatch):
+    """Up to 64 experts per tile the three split terms can sit side by side in one MMA;
+    both layouts must give the exact logits and routing."""
+    monkeypatch.setenv("MOE_B200_ROUTER_TERMS", terms)
+    M = _M()
+    x, W, off = exact_construction(T, d, E, seed=T + d, with_offset=True)
+    xd, Wd, offd = _bf16(x).cuda(), torch.from_numpy(W).cuda(), torch.from_numpy(off).cuda()
+    l, idx, gate = M.moe_route(xd, Wd, k, score, True, 1.0, offd, Wg_split=M.moe_prepare_router_weight(Wd))
+    _no_device_error()
+    o = O.route(x, W, k, score, True, 1.0, off, None)
+    assert np.array_equal(l.cpu().numpy().astype(np.float64), o["logits"])
+    assert np.array_equal(idx.cpu().numpy(), o["topk_idx"])
