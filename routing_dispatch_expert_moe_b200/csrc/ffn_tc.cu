@@ -414,8 +414,10 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
       const long long wrow0 = (long long)tc.row0 + q * 32;          // first row of this warp
       const int wrows = min(32, max(0, tc.rows - q * 32));          // valid rows of this warp
       (void)r_in;
-      epilogue_tile<MODE, OutT>(taddr, stage, lane, wrow0, wrows, tc.n_tile, F, N_out, gate_of_row, out,
-                                token_of_row, n_tokens, err);
+      // a warp past the group's last row has nothing to read or store (warp-uniform)
+      if (wrows > 0)
+        epilogue_tile<MODE, OutT>(taddr, stage, lane, wrow0, wrows, tc.n_tile, F, N_out, gate_of_row, out,
+                                  token_of_row, n_tokens, err);
       tc_fence_before();
       mbar_arrive(bar_tempty + 8 * acc);
     }
@@ -601,8 +603,11 @@ grouped_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
       const int cta_rows = min(BM, max(0, tc.rows - (int)rank * BM));
       const long long wrow0 = (long long)tc.row0 + (int)rank * BM + q * 32;
       const int wrows = min(32, max(0, cta_rows - q * 32));
-      epilogue_tile<MODE, OutT>(taddr, stage, lane, wrow0, wrows, tc.n_tile, F, N_out, gate_of_row, out,
-                                token_of_row, n_tokens, err, c_begin, c_end);
+      // a warp past the group's last row has nothing to read or store (warp-uniform): with
+      // many small groups most of a 256-row tile is padding
+      if (wrows > 0)
+        epilogue_tile<MODE, OutT>(taddr, stage, lane, wrow0, wrows, tc.n_tile, F, N_out, gate_of_row, out,
+                                  token_of_row, n_tokens, err, c_begin, c_end);
       tc_fence_before();
       mbar_arrive_remote(map_to_rank(bar_tempty + 8 * acc, 0));
     }

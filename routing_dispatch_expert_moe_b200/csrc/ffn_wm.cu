@@ -39,6 +39,7 @@ constexpr uint32_t kWTmemCols = 512;
 constexpr int kWRows = 128;                     // weight rows per CTA (256 per pair)
 constexpr int kWBlock = kWRows * BK * 2;       // 16 KB: one 128-row operand block
 constexpr int kFp4PadRows = 2 * kWRows;        // zero rows after the prepared 4-bit scales
+constexpr int kWXBox = 16;                      // token rows per TMA box: a tile loads only its n / 2 rows
 
 template <int MODE>
 struct WmCfg {
@@ -227,11 +228,13 @@ grouped_gemm_wm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
         const int x_row = tc.row0 + (int)rank * (n / 2);
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1u, abort_flag, err)) { ok = false; break; }
-          if (rank == 0) mbar_expect_tx(bar_full + 8 * stage, 2u * (uint32_t)C::stage_bytes);
+          if (rank == 0)
+            mbar_expect_tx(bar_full + 8 * stage, 2u * (uint32_t)(C::a_blocks * kWBlock + (n / 2) * BK * 2));
           const uint32_t full_c = map_to_rank(bar_full + 8 * stage, 0);
           tma_load_2d_pair(a_blk(stage, 0), &tmW, full_c, kb * BK, w_row);
           if (MODE == 0) tma_load_2d_pair(a_blk(stage, 1), &tmW, full_c, kb * BK, w_row + F);
-          tma_load_2d_pair(b_blk(stage), &tmX, full_c, kb * BK, x_row);
+          for (int xb = 0; xb < n / 2; xb += kWXBox)      // n / 2 is a multiple of 16
+            tma_load_2d_pair(b_blk(stage) + (uint32_t)(xb * BK * 2), &tmX, full_c, kb * BK, x_row + xb);
           last_phase[stage] = (int)phase;
           if (++stage == C::stages) { stage = 0; phase ^= 1u; }
         }
@@ -505,7 +508,7 @@ grouped_gemm_wm4_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_co
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1u, abort_flag, err)) { ok = false; break; }
           const uint32_t pk = bar_packed + 8 * stage;
-          mbar_expect_tx(pk, (uint32_t)(C::a_blocks * (C::packed_block + kWRows * kSpr) + C::b_bytes));
+          mbar_expect_tx(pk, (uint32_t)(C::a_blocks * (C::packed_block + kWRows * kSpr) + (n / 2) * BK * 2));
 #pragma unroll
           for (int a = 0; a < C::a_blocks; ++a) {
             const int row = w_row + (a ? F : 0);
@@ -513,7 +516,8 @@ grouped_gemm_wm4_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_co
             bulk_load(sb + (uint32_t)s_off(stage, a), scales_t + ((long long)kb * rows_pad + row) * kSpr,
                       (uint32_t)(kWRows * kSpr), pk);
           }
-          tma_load_2d(sb + (uint32_t)b_off(stage), &tmX, pk, kb * BK, x_row);
+          for (int xb = 0; xb < n / 2; xb += kWXBox)      // n / 2 is a multiple of 16
+            tma_load_2d(sb + (uint32_t)(b_off(stage) + xb * BK * 2), &tmX, pk, kb * BK, x_row + xb);
           last_phase[stage] = (int)phase;
           if (++stage == C::stages) { stage = 0; phase ^= 1u; }
         }
@@ -710,7 +714,7 @@ moe_status launch_gate_up_wm(const void* x_rows, const int32_t* offsets, int E, 
   if (d < BK || F < 8) return MOE_ERR_UNSUPPORTED;
   CUtensorMap mw, mx;
   if (!make_map(&mw, W_gu, (unsigned long long)E * 2 * F, d, kWRows)) return MOE_ERR_UNSUPPORTED;
-  if (!make_map(&mx, x_rows, (unsigned long long)rows_max, d, WmCfg<0>::NT / 2)) return MOE_ERR_UNSUPPORTED;
+  if (!make_map(&mx, x_rows, (unsigned long long)rows_max, d, kWXBox)) return MOE_ERR_UNSUPPORTED;
   return launch_wm<0, __nv_bfloat16>(mw, mx, offsets, E, d, d, F, rows_max, nullptr, h, s);
 }
 
@@ -721,7 +725,7 @@ moe_status launch_down_wm(const void* h, const int32_t* offsets, int E, int d, i
   if (F < BK || d < 8) return MOE_ERR_UNSUPPORTED;
   CUtensorMap mw, mx;
   if (!make_map(&mw, W_dn, (unsigned long long)E * d, F, kWRows)) return MOE_ERR_UNSUPPORTED;
-  if (!make_map(&mx, h, (unsigned long long)rows_max, F, WmCfg<1>::NT / 2)) return MOE_ERR_UNSUPPORTED;
+  if (!make_map(&mx, h, (unsigned long long)rows_max, F, kWXBox)) return MOE_ERR_UNSUPPORTED;
   if (y_dtype == MOE_F32) return launch_wm<1, float>(mw, mx, offsets, E, F, d, F, rows_max, gate_of_row, y_rows, s);
   return launch_wm<1, __nv_bfloat16>(mw, mx, offsets, E, F, d, F, rows_max, gate_of_row, y_rows, s);
 }
@@ -736,7 +740,7 @@ moe_status launch_gate_up_fp4(const void* x_rows, const int32_t* offsets, int E,
   if (rows_max == 0) return MOE_OK;
   CUtensorMap mc, mx;
   if (!make_map_u8(&mc, codes, (unsigned long long)E * 2 * F, d / 2, BK / 2, kWRows)) return MOE_ERR_UNSUPPORTED;
-  if (!make_map(&mx, x_rows, (unsigned long long)rows_max, d, WmCfg<0>::NT / 2)) return MOE_ERR_UNSUPPORTED;
+  if (!make_map(&mx, x_rows, (unsigned long long)rows_max, d, kWXBox)) return MOE_ERR_UNSUPPORTED;
   if (fmt == MOE_FP4_MX)
     return launch_wm4<0, MOE_FP4_MX, __nv_bfloat16>(mc, mx, scales_t, nullptr, offsets, E, d, d, F, rows_max,
                                                      nullptr, h, s);
@@ -750,7 +754,7 @@ moe_status launch_down_fp4(const void* h, const int32_t* offsets, int E, int d, 
   if (rows_max == 0) return MOE_OK;
   CUtensorMap mc, mx;
   if (!make_map_u8(&mc, codes, (unsigned long long)E * d, F / 2, BK / 2, kWRows)) return MOE_ERR_UNSUPPORTED;
-  if (!make_map(&mx, h, (unsigned long long)rows_max, F, WmCfg<1>::NT / 2)) return MOE_ERR_UNSUPPORTED;
+  if (!make_map(&mx, h, (unsigned long long)rows_max, F, kWXBox)) return MOE_ERR_UNSUPPORTED;
   const float* ts = fmt == MOE_FP4_NV ? tensor_scale : nullptr;
 #define MOE_WM4(FMT, T) \
   return launch_wm4<1, FMT, T>(mc, mx, scales_t, ts, offsets, E, F, d, F, rows_max, gate_of_row, y_rows, s)
