@@ -29,18 +29,20 @@ __device__ __forceinline__ float score_f(float l, float m, int score) {
   return sqrtf(fmaxf(l, 0.f) + log1pf(expf(-fabsf(l))));
 }
 
-constexpr int kSub = 64;   // tokens per sub-chunk (normalisers held in shared memory)
+constexpr int kSub = kStatsThreads / 32;   // tokens per sub-chunk: one per warp
 
 // Stage 1: each CTA owns tokens [t_begin, t_end), taken kSub at a time.
-//   (a) a warp per token: m = max_e l, se = sum_e exp(l - m), ss = sum_e s_e (fp64 sums,
-//       fixed lane-strided order and butterfly); z2 += (m + log se)^2;
-//   (b) a thread per expert: P_e += s_e(t) / ss(t) over the sub-chunk's tokens, in order.
-// Writes the CTA's P partials [E] and z2 partial.  Few registers per thread, so many warps
-// per SM hide the latency of the transcendentals at any E.
+//   (a) warp w takes token c0 + w: copies its logits into shared memory (independent
+//       coalesced loads) while taking m = max_e l, then se = sum_e exp(l - m) and
+//       ss = sum_e s_e (fp64 sums, fixed lane-strided order and butterfly), overwriting
+//       each logit by its score s_e; z2 += (m + log se)^2;
+//   (b) a thread per expert: P_e += s_e(t) / ss(t) over the sub-chunk's tokens, in order,
+//       from shared memory.
+// Every score is computed once.  Writes the CTA's P partials [E] and z2 partial.
 __global__ void __launch_bounds__(kStatsThreads)
 stats_partial_kernel(const float* __restrict__ logits, int T, int E, int score, int tokens_per_cta,
                      double* __restrict__ partP, double* __restrict__ partZ) {
-  __shared__ float s_m[kSub];
+  extern __shared__ float s_sc[];            // [kSub][E]
   __shared__ double s_inv[kSub];
   __shared__ double redz[kStatsThreads / 32];
   const unsigned lane = threadIdx.x & 31;
@@ -53,18 +55,26 @@ stats_partial_kernel(const float* __restrict__ logits, int T, int E, int score, 
   double P[4] = {0.0, 0.0, 0.0, 0.0};
   for (long long c0 = t_begin; c0 < t_end; c0 += kSub) {
     const int n = (int)min((long long)kSub, t_end - c0);
-    for (int i = warp; i < n; i += nwarps) {
-      const float* row = logits + (c0 + i) * E;
+    if (warp < n) {
+      const float* row = logits + (c0 + warp) * E;
+      float* srow = s_sc + warp * E;
       float mf = -INFINITY;
-      for (int e = lane; e < E; e += 32) mf = fmaxf(mf, __ldg(row + e));
+#pragma unroll 4
+      for (int e = lane; e < E; e += 32) {
+        const float l = __ldg(row + e);
+        srow[e] = l;
+        mf = fmaxf(mf, l);
+      }
 #pragma unroll
       for (int o = 16; o; o >>= 1) mf = fmaxf(mf, __shfl_xor_sync(0xffffffffu, mf, o));
       double se = 0.0, ss = 0.0;
       for (int e = lane; e < E; e += 32) {
-        const float l = __ldg(row + e);
+        const float l = srow[e];
         const float ex = expf(l - mf);
+        const float sv = score == MOE_SCORE_SOFTMAX ? ex : score_f(l, mf, score);
         se += (double)ex;
-        ss += (double)(score == MOE_SCORE_SOFTMAX ? ex : score_f(l, mf, score));
+        ss += (double)sv;
+        srow[e] = sv;
       }
 #pragma unroll
       for (int o = 16; o; o >>= 1) {
@@ -72,8 +82,7 @@ stats_partial_kernel(const float* __restrict__ logits, int T, int E, int score, 
         ss += __shfl_xor_sync(0xffffffffu, ss, o);
       }
       if (lane == 0) {
-        s_m[i] = mf;
-        s_inv[i] = 1.0 / ss;
+        s_inv[warp] = 1.0 / ss;
         const double lse = (double)mf + log(se);
         z2 += lse * lse;
       }
@@ -84,8 +93,7 @@ stats_partial_kernel(const float* __restrict__ logits, int T, int E, int score, 
       const int e = (int)threadIdx.x + q * kStatsThreads;
       if (e < E) {
         double acc = P[q];
-        for (int i = 0; i < n; ++i)
-          acc += (double)score_f(__ldg(logits + (c0 + i) * E + e), s_m[i], score) * s_inv[i];
+        for (int i = 0; i < n; ++i) acc += (double)s_sc[i * E + e] * s_inv[i];
         P[q] = acc;
       }
     }
@@ -223,7 +231,8 @@ moe_status launch_router_stats(const float* logits, const int32_t* counts, const
   double* pP = static_cast<double*>(ws);
   double* pZ = pP + (size_t)parts * E;
   const int tpc = (T + parts - 1) / parts;
-  stats_partial_kernel<<<parts, kStatsThreads, 0, s>>>(logits, T, E, score, tpc, pP, pZ);
+  stats_partial_kernel<<<parts, kStatsThreads, (size_t)kSub * E * sizeof(float), s>>>(logits, T, E, score, tpc, pP,
+                                                                                        pZ);
   moe_status st = check_launch();
   if (st != MOE_OK) return st;
   stats_final_kernel<<<1, 1024, 0, s>>>(pP, pZ, parts, counts, kept, T, E, k, load, stats5);
