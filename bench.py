@@ -41,7 +41,6 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # tokens and experts; both the weight and the row bytes grow with the units).
 GATE_UP_TRAFFIC = {
     ("c2_handbook", "permute", 65536): 931982080,
-    ("c5_stress", "permute", 131356): 8687124497,
 }
 
 
@@ -236,7 +235,8 @@ def run_ours(args):
 
     def make_layer(combine, dispatch, weights=None):
         return MoELayer(weights or w, cfg.k, cfg.T, cfg.score, cfg.renormalize, cfg.scale, cap, combine=combine,
-                        dispatch=dispatch, out_dtype=out_dt, rows_dtype=rows_dt, routing=routing)
+                        dispatch=dispatch, out_dtype=out_dt, rows_dtype=rows_dt, routing=routing,
+                        overlap=not args.no_overlap)
 
     def capture(fn):
         """One CUDA graph of fn(stream), captured on a side stream."""
@@ -642,6 +642,9 @@ def main():
                     help="sequential replays for the per-stage split (0 = skip)")
     ap.add_argument("--fp4-steps", type=int, default=30,
                     help="also time the layer with 4-bit (MXFP4, NVFP4) routed experts for this many steps (0 = skip)")
+    ap.add_argument("--no-overlap", action="store_true",
+                    help="run the router statistics on the main stream after the combine instead of on a "
+                         "second graph branch beside the expert GEMMs")
     ap.add_argument("--alt-steps", type=int, default=100,
                     help="also time the other combine form for this many steps (0 = skip)")
     args = ap.parse_args()

@@ -384,16 +384,19 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
         float lv[32];
         tmem_ld32(taddr + c * 32, v);
         if (SIDE) {
-          uint32_t v1[32], v2[32];
-          tmem_ld32(taddr + NE + c * 32, v1);
-          tmem_ld32(taddr + 2 * NE + c * 32, v2);
+          // (hi + mid) + lo, one 32-column block at a time (fewer live registers)
           tmem_wait_ld();
           tmem_regs_ready(v);
-          tmem_regs_ready(v1);
-          tmem_regs_ready(v2);
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            lv[i] = (__uint_as_float(v[i]) + __uint_as_float(v1[i])) + __uint_as_float(v2[i]);
+          for (int i = 0; i < 32; ++i) lv[i] = __uint_as_float(v[i]);
+#pragma unroll
+          for (int t = 1; t < 3; ++t) {
+            tmem_ld32(taddr + t * NE + c * 32, v);
+            tmem_wait_ld();
+            tmem_regs_ready(v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) lv[i] += __uint_as_float(v[i]);
+          }
         } else {
           tmem_wait_ld();
           tmem_regs_ready(v);
@@ -408,10 +411,18 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
         }
         stage_store32<float>(stage, lv, lane, logits, row0, wrows, E, e0 + c * 32, E);
         if constexpr (kFused) {
+          // the token's 32 logits are still in its staging row: a rolled loop over them
+          // keeps the selection code small (a pair may run this epilogue only once, from
+          // a cold instruction cache)
+          const float4* mine = reinterpret_cast<const float4*>(stage + lane * kStagePitchF32);
+#pragma unroll 1
+          for (int qd = 0; qd < 8; ++qd) {
+            const float4 f = mine[qd];
+            const float fv[4] = {f.x, f.y, f.z, f.w};
+            const int eb = e0 + c * 32 + 4 * qd;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int e = e0 + c * 32 + i;
-            if (e < E) topk_consider<KMAX, BIAS>(st, lv[i], e, score, full_softmax, sel_bias);
+            for (int i = 0; i < 4; ++i)
+              if (eb + i < E) topk_consider<KMAX, BIAS>(st, fv[i], eb + i, score, full_softmax, sel_bias);
           }
         }
       }
