@@ -226,6 +226,8 @@ moe_status launch_gate_up_gather_tc(const void* x, const int32_t* token_of_row, 
 // Weight-major grouped GEMMs (ffn_wm.cu): tiles of 256 weight rows x the expert's tokens.
 moe_status launch_gate_up_wm(const void* x_rows, const int32_t* offsets, int E, int d, int F, long long rows_max,
                              const void* W_gu, void* h, cudaStream_t s);
+moe_status launch_gate_up_wm_gather(const void* x, const int32_t* token_of_row, int T, const int32_t* offsets, int E,
+                                    int d, int F, long long rows_max, const void* W_gu, void* h, cudaStream_t s);
 moe_status launch_down_wm(const void* h, const int32_t* offsets, int E, int d, int F, long long rows_max,
                           const void* W_dn, const float* gate_of_row, int y_dtype, void* y_rows, cudaStream_t s);
 moe_status launch_gate_up_fp4(const void* x_rows, const int32_t* offsets, int E, int d, int F, long long rows_max,

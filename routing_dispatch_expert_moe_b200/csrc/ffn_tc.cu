@@ -68,17 +68,6 @@ struct L {
 };
 constexpr size_t kSmemBytes = L::end + 1024;                 // + alignment slack
 
-// 16-byte cp.async global -> shared; src_bytes = 0 writes zeros without reading.
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
-}
-// Arrive on the mbarrier once all of this thread's earlier cp.async copies have landed
-// (the barrier's expected count includes this arrival: .noinc).
-__device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
-
 // Output column tiles per row tile: 128 H features per gate/up tile (128 gate + 128 up
 // accumulator columns), 256 outputs per down tile.
 template <int MODE>
@@ -763,6 +752,10 @@ moe_status launch_gate_up_gather_tc(const void* x, const int32_t* token_of_row, 
                                     int d, int F, long long rows_max, const void* W_gu, void* h, cudaStream_t s) {
   if (rows_max == 0 || T == 0) return MOE_OK;
   if (d < BK || F < 8) return MOE_ERR_UNSUPPORTED;
+  if (prefer_weight_major(rows_max, E, false)) {
+    const moe_status st = launch_gate_up_wm_gather(x, token_of_row, T, offsets, E, d, F, rows_max, W_gu, h, s);
+    if (st != MOE_ERR_UNSUPPORTED) return st;
+  }
   CUtensorMap mb;
   if (!make_map(&mb, W_gu, (unsigned long long)E * 2 * F, d, 128)) return MOE_ERR_UNSUPPORTED;
   return launch_tc<4, __nv_bfloat16>(mb, mb, offsets, E, d, F, F, rows_max, nullptr, h, s, token_of_row, T,

@@ -51,7 +51,7 @@ struct WmCfg {
   static constexpr int epi_warps = 4;
   static constexpr int threads = 64 + 32 * epi_warps;
   static constexpr int bars = stages * stage_bytes;
-  static constexpr int nbars = 2 * stages + 4 + 1;
+  static constexpr int nbars = 3 * stages + 4 + 1;   // full, empty, tfull[2], tempty[2], fin, gathered
   static constexpr int misc = bars + nbars * 8;
   static constexpr int tiles = misc + 16;
   static constexpr int sh32 = tiles + (kWMaxE + 1) * 4;
@@ -154,11 +154,19 @@ __device__ __forceinline__ void wm_epilogue_tile(uint32_t taddr, uint8_t* stage,
   }
 }
 
-template <int MODE, typename OutT>
-__global__ void __launch_bounds__(WmCfg<MODE>::threads, 1)
+// GATHER (gate/up only): the token rows come straight from x [n_tokens, d] through
+// token_of_row (no permuted copy of x).  The producer warp's lanes copy them with 16-byte
+// cp.async into the swizzled layout and arrive on a local `gathered` barrier; a forwarder
+// warp waits on it, fences the rows for the async proxy and arrives on the even CTA's
+// `full` barrier, which also counts the weights' TMA bytes.
+template <int MODE, typename OutT, bool GATHER = false>
+__global__ void __launch_bounds__(WmCfg<MODE>::threads + (GATHER ? 32 : 0), 1)
 grouped_gemm_wm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                        const int32_t* __restrict__ offsets, int E, int K, int d, int F, long long rows_max,
-                       const float* __restrict__ gate_of_row, OutT* __restrict__ out, int* err) {
+                       const float* __restrict__ gate_of_row, OutT* __restrict__ out, int* err,
+                       const __nv_bfloat16* __restrict__ x_gather = nullptr,
+                       const int32_t* __restrict__ token_of_row = nullptr, int n_tokens = 0) {
+  static_assert(!GATHER || MODE == 0, "the gathered form is the gate/up GEMM's");
   using C = WmCfg<MODE>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -181,13 +189,15 @@ grouped_gemm_wm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
   const uint32_t bar_tfull = bar_empty + 8 * C::stages;
   const uint32_t bar_tempty = bar_tfull + 16;
   const uint32_t bar_fin = bar_tempty + 16;
+  const uint32_t bar_gath = bar_fin + 8;                   // [stages], GATHER only
   auto a_blk = [&](int s, int a) { return sb + (uint32_t)(s * C::stage_bytes + a * kWBlock); };
   auto b_blk = [&](int s) { return sb + (uint32_t)(s * C::stage_bytes + C::a_blocks * kWBlock); };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::stages; ++s) {
-      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_full + 8 * s, GATHER ? 1 + 2 : 1);     // + one forwarded arrival per CTA
       mbar_init(bar_empty + 8 * s, 1);
+      mbar_init(bar_gath + 8 * s, 32);                       // one cp.async arrival per producer lane
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(bar_tfull + 8 * a, 1);
@@ -210,7 +220,81 @@ grouped_gemm_wm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
   const uint32_t tmem_base = *tmem_slot;
   const int KB = (K + BK - 1) / BK;
 
-  if (warp == 0) {
+  if (GATHER && warp == 0) {
+    // ------------------------------------------------------------ gathering producer (both CTAs)
+    // lane: 16-byte chunk cv of rows rsub, rsub + 4, ... of this CTA's n / 2 token rows
+    const int cv = lane & 7, rsub = lane >> 3;
+    int stage = 0;
+    uint32_t phase = 0;
+    int last_phase[C::stages];
+#pragma unroll
+    for (int s = 0; s < C::stages; ++s) last_phase[s] = -1;
+    bool ok = true;
+    for (int tile = cid; ok && tile < total; tile += ncl) {
+      const TileCoord tc = tile_coord(tile_start, offsets, E, C::NT, tile);
+      const int half = wm_n<MODE>(tc.rows) / 2;
+      const int w_row = tc.e * 2 * F + tc.n_tile * 256 + (int)rank * kWRows;
+      const int r_base = (int)rank * half;                 // this CTA's first row of the tile
+      int tok[C::NT / 8];                                   // rows rsub + 4 i, i < NT / 8
+#pragma unroll
+      for (int i = 0; i < C::NT / 8; ++i) {
+        const int r = i * 4 + rsub;
+        int t = -1;
+        if (r < half && r_base + r < tc.rows) {
+          t = __ldg(token_of_row + tc.row0 + r_base + r);
+          if ((unsigned)t >= (unsigned)n_tokens) {
+            record_error(err, MOE_DEVERR_ROW);
+            t = -1;
+          }
+        }
+        tok[i] = t;
+      }
+      for (int kb = 0; kb < KB; ++kb) {
+        const bool got = mbar_wait(bar_empty + 8 * stage, phase ^ 1u, abort_flag, err);
+        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+        if (lane == 0) {
+          if (rank == 0) mbar_expect_tx(bar_full + 8 * stage, 2u * (uint32_t)(C::a_blocks * kWBlock));
+          const uint32_t full_c = map_to_rank(bar_full + 8 * stage, 0);
+          tma_load_2d_pair(a_blk(stage, 0), &tmW, full_c, kb * BK, w_row);
+          tma_load_2d_pair(a_blk(stage, 1), &tmW, full_c, kb * BK, w_row + F);
+          last_phase[stage] = (int)phase;
+        }
+        const uint32_t b_dst = b_blk(stage);
+        const int kcol = kb * BK + cv * 8;
+#pragma unroll
+        for (int i = 0; i < C::NT / 8; ++i) {
+          const int r = i * 4 + rsub;
+          if (r < half) {                                   // rows past the group are zeros
+            const bool v = tok[i] >= 0 && kcol < K;
+            const __nv_bfloat16* src = x_gather + (v ? (long long)tok[i] * K + kcol : 0LL);
+            cp_async16(b_dst + r * 128 + ((cv ^ (r & 7)) << 4), src, v ? 16u : 0u);
+          }
+        }
+        cp_async_arrive_noinc(bar_gath + 8 * stage);
+        if (++stage == C::stages) { stage = 0; phase ^= 1u; }
+      }
+    }
+    cp_async_wait_all();                                    // no copy may land after the CTA has exited
+    if (!ok && lane == 0 && rank == 0) {
+      for (int s = 0; s < C::stages; ++s)
+        if (last_phase[s] >= 0) mbar_wait_drain(bar_full + 8 * s, (uint32_t)last_phase[s], err);
+    }
+  } else if (GATHER && warp == 2 + C::epi_warps) {
+    // ------------------------------------------------------------ forwarder (both CTAs)
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = cid; ok && tile < total; tile += ncl) {
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(bar_gath + 8 * stage, phase, abort_flag, err)) { ok = false; break; }
+          fence_proxy_async_smem();                         // the MMAs read the rows through the async proxy
+          mbar_arrive_cluster(map_to_rank(bar_full + 8 * stage, 0));
+          if (++stage == C::stages) { stage = 0; phase ^= 1u; }
+        }
+      }
+    }
+  } else if (warp == 0) {
     // ------------------------------------------------------------ TMA producer (both CTAs)
     if (lane == 0) {
       int stage = 0;
@@ -262,6 +346,7 @@ grouped_gemm_wm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag, err)) { ok = false; break; }
           tc_fence_after();
+          if (GATHER) fence_proxy_async_smem();
           const uint64_t bdesc = sw128_desc(b_blk(stage));
           const uint64_t adesc0 = sw128_desc(a_blk(stage, 0));
           const uint64_t adesc1 = sw128_desc(a_blk(stage, MODE == 0 ? 1 : 0));
@@ -334,9 +419,9 @@ grouped_gemm_wm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
 // and low bytes of their bf16 values from two 8-byte tables (byte permutes), the sign
 // bits are moved into place, and the bf16 pairs are multiplied by the block scale.  Each
 // 16-byte chunk goes to the 128-byte-swizzled operand layout (chunk c of row r at
-// r * 128 + ((c ^ (r & 7)) * 16)); then a proxy fence and an arrive on the even CTA's
-// `full` barrier (2 x 256 converter threads).  `empty` (the MMAs' completion) frees the
-// stage in both CTAs.
+// r * 128 + ((c ^ (r & 7)) * 16)); then each thread's proxy fence, and one arrive per
+// converter warp on the even CTA's `full` barrier (2 x 8 warps).  `empty` (the MMAs'
+// completion) frees the stage in both CTAs.
 // =====================================================================================
 template <int MODE>
 struct Wm4Cfg {
@@ -466,7 +551,7 @@ grouped_gemm_wm4_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_co
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::stages; ++s) {
       mbar_init(bar_packed + 8 * s, 1);
-      mbar_init(bar_full + 8 * s, 2 * C::cvt_threads);
+      mbar_init(bar_full + 8 * s, 2 * C::cvt_warps);   // one arrive per converter warp of each CTA
       mbar_init(bar_empty + 8 * s, 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -601,7 +686,8 @@ grouped_gemm_wm4_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_co
                                               : *reinterpret_cast<const uint32_t*>(sc_p);
         convert_chunks<FMT>(smem + p_off(stage, a) + r * (BK / 2), sc, smem + a_off(stage, a), r, c0, c1);
         fence_proxy_async_smem();                           // the MMAs read these through the async proxy
-        mbar_arrive_cluster(map_to_rank(bar_full + 8 * stage, 0));
+        __syncwarp();                                       // the warp's chunks are written and fenced
+        if (lane == 0) mbar_arrive_cluster(map_to_rank(bar_full + 8 * stage, 0));
         if (++stage == C::stages) { stage = 0; phase ^= 1u; }
       }
     }
@@ -660,12 +746,14 @@ fp4_scales_kernel(const uint8_t* __restrict__ in, long long rows, int K, int spr
   }
 }
 
-template <int MODE, typename OutT>
+template <int MODE, typename OutT, bool GATHER = false>
 moe_status launch_wm(const CUtensorMap& mw, const CUtensorMap& mx, const int32_t* offsets, int E, int K, int d,
-                     int F, long long rows_max, const float* gate_of_row, void* out, cudaStream_t s) {
+                     int F, long long rows_max, const float* gate_of_row, void* out, cudaStream_t s,
+                     const __nv_bfloat16* x_gather = nullptr, const int32_t* token_of_row = nullptr,
+                     int n_tokens = 0) {
   using C = WmCfg<MODE>;
   static std::atomic<int> configured[kMaxDevices];
-  const moe_status st = ensure_smem_limit(configured, grouped_gemm_wm_kernel<MODE, OutT>, C::smem);
+  const moe_status st = ensure_smem_limit(configured, grouped_gemm_wm_kernel<MODE, OutT, GATHER>, C::smem);
   if (st != MOE_OK) return st;
   const long long max_tiles = ((rows_max + C::NT - 1) / C::NT + E) * (long long)wm_m_tiles<MODE>(F, d);
   int pairs = num_sms() / 2;
@@ -673,7 +761,7 @@ moe_status launch_wm(const CUtensorMap& mw, const CUtensorMap& mx, const int32_t
   if (pairs < 1) pairs = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs, 1, 1);
-  cfg.blockDim = dim3(C::threads, 1, 1);
+  cfg.blockDim = dim3(C::threads + (GATHER ? 32 : 0), 1, 1);
   cfg.dynamicSmemBytes = C::smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -683,8 +771,9 @@ moe_status launch_wm(const CUtensorMap& mw, const CUtensorMap& mx, const int32_t
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cuda_status(cudaLaunchKernelEx(&cfg, grouped_gemm_wm_kernel<MODE, OutT>, mw, mx, offsets, E, K, d, F,
-                                        rows_max, gate_of_row, static_cast<OutT*>(out), err_ptr()));
+  return cuda_status(cudaLaunchKernelEx(&cfg, grouped_gemm_wm_kernel<MODE, OutT, GATHER>, mw, mx, offsets, E, K, d,
+                                        F, rows_max, gate_of_row, static_cast<OutT*>(out), err_ptr(), x_gather,
+                                        token_of_row, n_tokens));
 }
 
 }  // namespace
@@ -716,6 +805,18 @@ moe_status launch_gate_up_wm(const void* x_rows, const int32_t* offsets, int E, 
   if (!make_map(&mw, W_gu, (unsigned long long)E * 2 * F, d, kWRows)) return MOE_ERR_UNSUPPORTED;
   if (!make_map(&mx, x_rows, (unsigned long long)rows_max, d, kWXBox)) return MOE_ERR_UNSUPPORTED;
   return launch_wm<0, __nv_bfloat16>(mw, mx, offsets, E, d, d, F, rows_max, nullptr, h, s);
+}
+
+// Gate/up, weight-major, gathered: H [rows_max, F] bf16 from the token rows x[token_of_row[r]]
+// (x [T, d] bf16) and W_gu [E][2F][d]; no permuted copy of x.
+moe_status launch_gate_up_wm_gather(const void* x, const int32_t* token_of_row, int T, const int32_t* offsets, int E,
+                                    int d, int F, long long rows_max, const void* W_gu, void* h, cudaStream_t s) {
+  if (rows_max == 0 || T == 0) return MOE_OK;
+  if (d < BK || F < 8) return MOE_ERR_UNSUPPORTED;
+  CUtensorMap mw;
+  if (!make_map(&mw, W_gu, (unsigned long long)E * 2 * F, d, kWRows)) return MOE_ERR_UNSUPPORTED;
+  return launch_wm<0, __nv_bfloat16, true>(mw, mw, offsets, E, d, d, F, rows_max, nullptr, h, s,
+                                           static_cast<const __nv_bfloat16*>(x), token_of_row, T);
 }
 
 // Down, weight-major: gated rows [rows_max, d] (bf16 or fp32) from H [rows_max, F] and W_dn [E][d][F].

@@ -387,9 +387,12 @@ GATHER = [c for c in SMALL if c.name in ("softmax_bf16", "sigmoid_bias_shared", 
                                           "sigmoid_nobias_E_odd")]
 
 
+@pytest.mark.parametrize("tiles", TILES)
 @pytest.mark.parametrize("cfg", GATHER, ids=lambda c: c.name)
-def test_gathered_gate_up_is_bitwise_the_permuted_one(cfg):
-    """Same A rows, same tiles, same accumulation order: H and the reproducible y agree bit for bit."""
+def test_gathered_gate_up_is_bitwise_the_permuted_one(cfg, tiles, monkeypatch):
+    """Same token rows, same tiles, same accumulation order: H and the reproducible y agree
+    bit for bit, in both tile orientations (weight-major: the rows gathered by cp.async)."""
+    monkeypatch.setenv("MOE_B200_EXPERT_TILES", tiles)
     host, dev = U.make_inputs(cfg)
     cap = O.capacity(cfg.T, cfg.E, cfg.k, cfg.capacity_factor, True)
     lp, gp = U.gpu_forward(cfg, dev, cap)
@@ -400,8 +403,10 @@ def test_gathered_gate_up_is_bitwise_the_permuted_one(cfg):
     assert np.array_equal(gp["y"], gg["y"])
 
 
-def test_gathered_bad_token_is_reported_not_trapped():
+@pytest.mark.parametrize("tiles", TILES)
+def test_gathered_bad_token_is_reported_not_trapped(tiles, monkeypatch):
     from routing_dispatch_expert_moe_b200 import moe as M
+    monkeypatch.setenv("MOE_B200_EXPERT_TILES", tiles)
     for cfg in (SMALL[0], SMALL[6]):                          # tensor-core and fp32 SIMT forms
         host, dev = U.make_inputs(cfg)
         layer, g = U.gpu_forward(cfg, dev, -1, dispatch="gather")
