@@ -332,10 +332,10 @@ def run_ours(args):
         # the other combine form on the same inputs: fused into the down GEMM (fp32 atomics),
         # or gated rows + ordered combine (bitwise reproducible)
         alt = "fused" if args.combine == "rows" else "rows"
-        rl = make_layer(alt, "permute")
+        rl = make_layer(alt, layer.dispatch_mode)
         ps, sm, _, _ = time_layer(rl, args.alt_steps, breakdown_steps=min(args.breakdown_steps, 50))
         t = max_over_ranks(float(ps.sum()), dev)
-        other = {"dispatch": "permute",
+        other = {"dispatch": rl.dispatch_mode,
                  "combine": ("fused into the down GEMM (fp32 atomics)" if alt == "fused"
                              else "gated rows + ordered combine (bitwise reproducible)"),
                  "ms_per_step": round(t / args.alt_steps, 4),
@@ -440,7 +440,7 @@ def run_ours(args):
     del lays
 
     pk, pk_src = peaks()
-    gather = args.dispatch == "gather"
+    gather = layer.dispatch_mode == "gather"
     gate_up_ms = stage_ms["timed_gate_up_gather" if gather else "timed_gate_up"]   # inside the timed region
     flops, gu_bytes = gate_up_work(cfg, A, E_act, gather)
     t_tensor, t_hbm = flops / (pk["bf16_tflops"] * 1e12), gu_bytes / (pk["hbm_gbs"] * 1e9)
@@ -454,7 +454,7 @@ def run_ours(args):
     roof["algorithmic"] = {"flops": flops, "bytes": gu_bytes, "rows": A, "experts_with_rows": E_act,
                            "tensor_ms": round(t_tensor * 1e3, 4), "hbm_ms": round(t_hbm * 1e3, 4),
                            "kernel_ms": round(gate_up_ms, 4)}
-    roof["traffic"] = GATE_UP_TRAFFIC.get((args.workload, args.dispatch, A))
+    roof["traffic"] = GATE_UP_TRAFFIC.get((args.workload, layer.dispatch_mode, A))
     fused = args.combine == "fused"
     rb = 4 if fused else layer.y_perm.element_size()
     ob = layer.y.element_size()
@@ -629,8 +629,9 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=50, help="steps timed through host buffers")
     ap.add_argument("--combine", choices=["fused", "rows"], default="rows",
                     help="rows: gated rows + ordered combine (reproducible); fused: combine inside the down GEMM")
-    ap.add_argument("--dispatch", choices=["gather", "permute"], default="permute",
-                    help="gather: the gate/up GEMM reads token rows through the row map; permute: x_perm copy")
+    ap.add_argument("--dispatch", choices=["auto", "gather", "permute"], default="auto",
+                    help="gather: the gate/up GEMM reads token rows through the row map; permute: x_perm copy; "
+                         "auto: gather where the gate/up GEMM takes weight-major tiles, else permute")
     ap.add_argument("--out-dtype", choices=["bf16", "f32"], default="bf16",
                     help="dtype of the layer output y (bf16: fp32 sums rounded once at the end)")
     ap.add_argument("--rows-dtype", choices=["f32", "bf16"], default="bf16",

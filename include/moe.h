@@ -129,6 +129,17 @@ MOE_API int32_t moe_capacity(int32_t T, int32_t E, int32_t k, double capacity_fa
 /* Rows the permuted buffers must hold: T*k when capacity < 0, else min(T*k, E*capacity). */
 MOE_API int64_t moe_rows_max(int32_t T, int32_t E, int32_t k, int32_t capacity);
 
+/* Which tile orientation the bf16 gate/up GEMMs (moe_expert_gate_up and
+ * moe_expert_gate_up_gather) take for these sizes: 1 = weight-major (256 weight rows x
+ * an expert's tokens; chosen when the groups average under 1024 rows, rows_max / E), 0 =
+ * token-major (256 token rows of one expert x 256 outputs).  The environment variable
+ * MOE_B200_EXPERT_TILES=tokens|weights overrides the choice, here as in the GEMMs.  A
+ * caller can use it to pick its dispatch form: the gathered gate/up reads x through
+ * token_of_row at no extra cost in the weight-major orientation (the token rows are the
+ * small operand), while the token-major one re-reads each row once per output tile.
+ * Returns -1 for rows_max < 0 or E < 1.  Host only. */
+MOE_API int32_t moe_gate_up_weight_major(int64_t rows_max, int32_t E);
+
 /* ------------------------------------------------------------------------------------
  * moe_prepare_router_weight -- the tensor-core router's operand, made once at load time.
  * [MoE-Explained] section "Switch Transformer" (the router stays in full precision);

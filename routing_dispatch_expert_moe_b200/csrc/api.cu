@@ -92,6 +92,11 @@ int64_t moe_rows_max(int32_t T, int32_t E, int32_t k, int32_t capacity) {
   return c < A ? c : A;
 }
 
+int32_t moe_gate_up_weight_major(int64_t rows_max, int32_t E) {
+  if (rows_max < 0 || E < 1) return -1;
+  return prefer_weight_major(rows_max, E, false) ? 1 : 0;
+}
+
 size_t moe_route_workspace_bytes(int32_t T, int32_t d, int32_t E) {
   if (T < 0 || d < 1 || E < 1) return 0;
   return route_workspace_bytes(T, d, E, false);

@@ -55,8 +55,9 @@ class MoELayer:
         fp32 (the default) leaves H as the only bf16 rounding inside the layer.
         combine: "rows" (gated rows + ordered combine) or "fused" (down GEMM adds into an
         fp32 buffer, rounded once to bf16 at the end when out_dtype is bf16).
-        dispatch: "permute" (x_perm copy, then the GEMM) or "gather" (the GEMM reads the
-        token rows through token_of_row; same H bit for bit).
+        dispatch: "permute" (x_perm copy, then the GEMM), "gather" (the GEMM reads the
+        token rows through token_of_row; same H bit for bit) or "auto" (gather where the
+        gate/up GEMM takes weight-major tiles, moe_gate_up_weight_major; permute otherwise).
         overlap: run the work nothing on the main path waits for (router statistics, and
         clearing y for the fused combine) on a second stream forked from and joined back
         to the caller's stream (one CUDA graph with two branches when captured).
@@ -66,10 +67,10 @@ class MoELayer:
         draws given to forward; softmax gating).  The fixed rules keep the learned gates
         over the chosen experts; the router statistics always use the router logits."""
         self.fp4 = weights.W_gu_fp4 is not None
-        if self.fp4 and (weights.W_dn_fp4 is None or combine != "rows" or dispatch != "permute"
+        if self.fp4 and (weights.W_dn_fp4 is None or combine != "rows" or dispatch == "gather"
                          or weights.W_gu.dtype != torch.bfloat16):
             raise ValueError("4-bit experts need both W_gu_fp4 and W_dn_fp4, bf16 activations, "
-                             "combine='rows' and dispatch='permute'")
+                             "combine='rows' and dispatch='permute' (or 'auto')")
         if routing not in ("learned", "uniform", "hash", "noisy"):
             raise ValueError(f"routing must be learned, uniform, hash or noisy, got {routing!r}")
         if routing != "learned" and weights.select_bias is not None:
@@ -77,9 +78,8 @@ class MoELayer:
         if routing == "noisy" and (weights.W_noise is None or score != "softmax"):
             raise ValueError("noisy top-k needs weights.W_noise and softmax scoring")
         self.routing, self.hash_seed = routing, hash_seed
-        if dispatch not in ("permute", "gather"):
-            raise ValueError(f"dispatch must be 'permute' or 'gather', got {dispatch!r}")
-        self.dispatch_mode = dispatch
+        if dispatch not in ("permute", "gather", "auto"):
+            raise ValueError(f"dispatch must be 'permute', 'gather' or 'auto', got {dispatch!r}")
         if combine not in ("rows", "fused"):
             raise ValueError(f"combine must be 'rows' or 'fused', got {combine!r}")
         if out_dtype not in (torch.float32, torch.bfloat16):
@@ -97,6 +97,12 @@ class MoELayer:
         self.device = dev
         E, d, F = self.E, self.d, self.F
         self.rows_max = M.moe_rows_max(T_max, E, k, capacity)
+        if dispatch == "auto":
+            # gathered where the gate/up GEMM takes weight-major tiles (the token rows are its
+            # small operand, read once either way); the permute copy otherwise
+            wm = self.dtype == torch.bfloat16 and not self.fp4 and M.moe_gate_up_weight_major(self.rows_max, E)
+            dispatch = "gather" if wm else "permute"
+        self.dispatch_mode = dispatch
         R = max(self.rows_max, 1)
         f32, i32 = torch.float32, torch.int32
         self.logits = torch.empty((T_max, E), dtype=f32, device=dev)

@@ -35,6 +35,7 @@ _SIGNATURES = {
     "moe_last_cuda_error": (ctypes.c_char_p, []),
     "moe_capacity": (_i32, [_i32, _i32, _i32, _f64, _i32]),
     "moe_rows_max": (_i64, [_i32, _i32, _i32, _i32]),
+    "moe_gate_up_weight_major": (_i32, [_i64, _i32]),
     "moe_route_workspace_bytes": (_size, [_i32, _i32, _i32]),
     "moe_router_weight_bytes": (_size, [_i32, _i32]),
     "moe_prepare_router_weight": (_i32, [_c_void_p, _i32, _i32, _c_void_p, _size, _c_void_p]),
@@ -171,6 +172,14 @@ def moe_capacity(T: int, E: int, k: int, capacity_factor: Optional[float], per_a
 
 def moe_rows_max(T: int, E: int, k: int, capacity: int) -> int:
     return int(lib().moe_rows_max(T, E, k, capacity))
+
+
+def moe_gate_up_weight_major(rows_max: int, E: int) -> bool:
+    """True when the bf16 gate/up GEMMs take weight-major tiles for these sizes."""
+    r = int(lib().moe_gate_up_weight_major(rows_max, E))
+    if r < 0:
+        raise MoEError(f"moe_gate_up_weight_major: invalid sizes rows_max={rows_max}, E={E}")
+    return bool(r)
 
 
 def moe_workspace_bytes(T: int, d: int, E: int, k: int) -> int:

@@ -59,6 +59,20 @@ def test_rows_max(L):
     assert L.moe_rows_max(0, 8, 2, -1) == 0
 
 
+def test_gate_up_orientation_query(L, monkeypatch):
+    """Weight-major tiles below 1024 rows per expert on average; the override variable wins."""
+    monkeypatch.delenv("MOE_B200_EXPERT_TILES", raising=False)
+    assert L.moe_gate_up_weight_major(32768 * 16, 896) == 1          # stress layer: 585 rows per expert
+    assert L.moe_gate_up_weight_major(8192 * 8, 64) == 0             # handbook layer: 1024 rows per expert
+    assert L.moe_gate_up_weight_major(1023, 1) == 1
+    assert L.moe_gate_up_weight_major(1024, 1) == 0
+    assert L.moe_gate_up_weight_major(-1, 8) == -1 and L.moe_gate_up_weight_major(10, 0) == -1
+    monkeypatch.setenv("MOE_B200_EXPERT_TILES", "tokens")
+    assert L.moe_gate_up_weight_major(32768 * 16, 896) == 0
+    monkeypatch.setenv("MOE_B200_EXPERT_TILES", "weights")
+    assert L.moe_gate_up_weight_major(8192 * 8, 64) == 1
+
+
 def test_workspace_queries(L):
     assert L.moe_histogram_scan_workspace_bytes(8192, 8, 64) >= 8192 * 8 * 4
     assert L.moe_router_stats_workspace_bytes(8192, 64) > 0
