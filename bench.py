@@ -629,7 +629,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=50, help="steps timed through host buffers")
     ap.add_argument("--combine", choices=["fused", "rows"], default="rows",
                     help="rows: gated rows + ordered combine (reproducible); fused: combine inside the down GEMM")
-    ap.add_argument("--dispatch", choices=["auto", "gather", "permute"], default="auto",
+    ap.add_argument("--dispatch", choices=["auto", "gather", "permute"], default="permute",
                     help="gather: the gate/up GEMM reads token rows through the row map; permute: x_perm copy; "
                          "auto: gather where the gate/up GEMM takes weight-major tiles, else permute")
     ap.add_argument("--out-dtype", choices=["bf16", "f32"], default="bf16",

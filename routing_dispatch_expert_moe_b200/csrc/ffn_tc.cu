@@ -170,16 +170,26 @@ __device__ __forceinline__ void epilogue_tile(uint32_t taddr, uint8_t* stage, in
     static_assert(MODE == 1, "grouped GEMM modes: 0 gate/up, 1 down, 3 down + combine, 4 gathered gate/up");
     const int n0 = n_tile * BN;
     const float gs = (lane < wrows && gate_of_row) ? __ldg(gate_of_row + wrow0 + lane) : 1.f;
+    // two 32-column chunks per TMEM wait: with K = F of a few k-blocks this epilogue is as
+    // long as the tile's mainloop, and each wait is a full TMEM round trip
 #pragma unroll 1
-    for (int c = c_begin; c < c_end; ++c) {
-      uint32_t v32[32];
-      tmem_ld32(taddr + c * 32, v32);
+    for (int c = c_begin; c < c_end; c += 2) {
+      const bool two = c + 1 < c_end;                      // warp-uniform
+      uint32_t va[32], vb[32];
+      tmem_ld32(taddr + c * 32, va);
+      if (two) tmem_ld32(taddr + (c + 1) * 32, vb);
       tmem_wait_ld();
-      tmem_regs_ready(v32);
+      tmem_regs_ready(va);
+      tmem_regs_ready(vb);
       float y[32];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) y[i] = __uint_as_float(v32[i]) * gs;
+      for (int i = 0; i < 32; ++i) y[i] = __uint_as_float(va[i]) * gs;
       stage_store32<OutT>(stage, y, lane, out, wrow0, wrows, N_out, n0 + c * 32, N_out);
+      if (two) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) y[i] = __uint_as_float(vb[i]) * gs;
+        stage_store32<OutT>(stage, y, lane, out, wrow0, wrows, N_out, n0 + (c + 1) * 32, N_out);
+      }
     }
   }
 }
@@ -636,7 +646,15 @@ moe_status launch_tc(const CUtensorMap& ma, const CUtensorMap& mb, const int32_t
 // groups keep the single-CTA kernel (less padding in ragged groups).
 // Down GEMMs with K = F up to this use the eight-epilogue-warp pair configuration.
 constexpr int kWideMaxK = 512;
-static bool use_pairs(long long rows_max, int groups) { return groups > 0 && rows_max / groups >= 2 * BM; }
+// Token-major tiles: CTA pairs (256 rows per tile) when the groups average at least 256
+// rows, single CTAs (128 rows) otherwise; MOE_B200_TOKEN_TILES=pairs|single forces one
+// (for measuring one against the other).
+static bool use_pairs(long long rows_max, int groups) {
+  const char* v = getenv("MOE_B200_TOKEN_TILES");
+  if (v && strcmp(v, "pairs") == 0) return groups > 0;
+  if (v && strcmp(v, "single") == 0) return false;
+  return groups > 0 && rows_max / groups >= 2 * BM;
+}
 
 template <int MODE, typename OutT, bool WIDE = false>
 moe_status launch_tc2(const CUtensorMap& ma, const CUtensorMap& mb, const int32_t* offsets, int E, int K, int N_out,

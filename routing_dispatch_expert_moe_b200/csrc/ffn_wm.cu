@@ -142,14 +142,27 @@ __device__ __forceinline__ void wm_epilogue_tile(uint32_t taddr, uint8_t* stage,
       }
       stage_store32_t<OutT>(stage, h, lane, out, r0, rv, F, col0, F);
     } else {
-      uint32_t v[32];
+      // two 32-token chunks per TMEM wait (the tile's mainloop is only K / 64 k-blocks)
+      const bool two = c + 1 < chunks;                     // warp-uniform
+      uint32_t v[32], vb[32];
       tmem_ld32(taddr + c * 32, v);
+      if (two) tmem_ld32(taddr + (c + 1) * 32, vb);
       tmem_wait_ld();
       tmem_regs_ready(v);
+      tmem_regs_ready(vb);
       const float gs = ((gate_of_row && lane < rv) ? __ldg(gate_of_row + r0 + lane) : 1.f) * wscale;
 #pragma unroll
       for (int i = 0; i < 32; ++i) h[i] = __uint_as_float(v[i]) * __shfl_sync(0xffffffffu, gs, i);
       stage_store32_t<OutT>(stage, h, lane, out, r0, rv, d, col0, d);
+      if (two) {
+        const long long r0b = r0 + 32;
+        const int rvb = min(32, tc.rows - (c + 1) * 32);
+        const float gsb = ((gate_of_row && lane < rvb) ? __ldg(gate_of_row + r0b + lane) : 1.f) * wscale;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) h[i] = __uint_as_float(vb[i]) * __shfl_sync(0xffffffffu, gsb, i);
+        stage_store32_t<OutT>(stage, h, lane, out, r0b, rvb, d, col0, d);
+        ++c;
+      }
     }
   }
 }
@@ -248,6 +261,10 @@ grouped_gemm_wm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
           }
         }
         tok[i] = t;
+        // the tile reads each of its token rows in 64-element pieces over K / 64 stages:
+        // ask L2 for the whole row up front (one contiguous request per row), so the
+        // 128-byte cp.async pieces below mostly hit L2
+        if (cv == 0 && t >= 0) prefetch_l2(x_gather + (long long)t * K, (uint32_t)K * 2u);
       }
       for (int kb = 0; kb < KB; ++kb) {
         const bool got = mbar_wait(bar_empty + 8 * stage, phase ^ 1u, abort_flag, err);

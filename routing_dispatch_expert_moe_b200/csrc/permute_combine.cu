@@ -106,14 +106,16 @@ __device__ __forceinline__ void store8<float>(void* base, long long e, const flo
 // compacted, in slot order, into a per-warp list in shared memory (a ballot gives each
 // kept slot its position), so dropped slots cost nothing, every batch of loads is full,
 // and the list costs no registers (two blocks fit on an SM).  Each lane then loads up to
-// 8 kept rows for VPI consecutive 8-element vectors (8 * VPI independent loads in
-// flight) and adds them in slot order: the same fp32 sum as visiting every slot.
+// 4 kept rows for VPI 8-element vectors (4 * VPI = 16 independent 16-byte loads in flight
+// once a token keeps 4 rows, the common case when capacity drops most slots) and adds them
+// in slot order: the same fp32 sum as visiting every slot.
 template <typename InT, typename OutT, int KMAX>
 __global__ void __launch_bounds__(256, 2)
 combine_kernel(const void* __restrict__ y_rows, const int32_t* __restrict__ row_of,
                const float* __restrict__ topk_gate, const void* __restrict__ shared_y, int T, int d, int k,
                long long rows_max, void* __restrict__ y, int* err) {
-  constexpr int VPI = sizeof(InT) == 2 ? 2 : 1;       // vectors per lane per step
+  constexpr int VPI = sizeof(InT) == 2 ? 4 : 2;       // vectors per lane per step
+  constexpr int R = 4;                                 // kept rows per batch of loads
   __shared__ int s_row[8][32];
   __shared__ float s_gate[8][32];
   const unsigned lane = threadIdx.x & 31;
@@ -149,18 +151,18 @@ combine_kernel(const void* __restrict__ y_rows, const int32_t* __restrict__ row_
       for (int u = 0; u < VPI; ++u)
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc[u][i] = 0.f;
-#pragma unroll
-      for (int j0 = 0; j0 < KMAX; j0 += 8) {
+#pragma unroll 1
+      for (int j0 = 0; j0 < KMAX; j0 += R) {
         if (j0 >= nk) break;
-        Row8<InT> buf[VPI][8];
+        Row8<InT> buf[VPI][R];
 #pragma unroll
-        for (int jj = 0; jj < 8; ++jj)
+        for (int jj = 0; jj < R; ++jj)
 #pragma unroll
           for (int u = 0; u < VPI; ++u)
             if (j0 + jj < nk && v0 + 32 * u < n8)
               buf[u][jj].load(y_rows, (long long)krow[j0 + jj] * d + (v0 + 32 * u) * 8);
 #pragma unroll
-        for (int jj = 0; jj < 8; ++jj)
+        for (int jj = 0; jj < R; ++jj)
 #pragma unroll
           for (int u = 0; u < VPI; ++u)
             if (j0 + jj < nk && v0 + 32 * u < n8) buf[u][jj].add(acc[u], kgate[j0 + jj], scale);
