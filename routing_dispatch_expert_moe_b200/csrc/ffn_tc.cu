@@ -646,14 +646,18 @@ moe_status launch_tc(const CUtensorMap& ma, const CUtensorMap& mb, const int32_t
 // groups keep the single-CTA kernel (less padding in ragged groups).
 // Down GEMMs with K = F up to this use the eight-epilogue-warp pair configuration.
 constexpr int kWideMaxK = 512;
-// Token-major tiles: CTA pairs (256 rows per tile) when the groups average at least 256
-// rows, single CTAs (128 rows) otherwise; MOE_B200_TOKEN_TILES=pairs|single forces one
-// (for measuring one against the other).
+constexpr long long kPairRowsMin = 1024;
+
+// Token-major tiles: CTA pairs (256 rows per tile) when the groups average at least 1024
+// rows, single CTAs (128 rows) otherwise: with smaller groups most tiles are part-empty,
+// and a 128-row tile wastes half the tensor work of a 256-row one (measured on the stress
+// layer's down GEMM, 585 rows per expert at most and 146 on average: 1.15 ms single
+// against 1.29 ms in pairs).  MOE_B200_TOKEN_TILES=pairs|single forces one.
 static bool use_pairs(long long rows_max, int groups) {
   const char* v = getenv("MOE_B200_TOKEN_TILES");
   if (v && strcmp(v, "pairs") == 0) return groups > 0;
   if (v && strcmp(v, "single") == 0) return false;
-  return groups > 0 && rows_max / groups >= 2 * BM;
+  return groups > 0 && rows_max / groups >= kPairRowsMin;
 }
 
 template <int MODE, typename OutT, bool WIDE = false>

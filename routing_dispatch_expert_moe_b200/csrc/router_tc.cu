@@ -188,43 +188,44 @@ __device__ __forceinline__ void topk_consider(TopK<KMAX, BIAS>& st, float l, int
   }
 }
 
-// Gates of the selected experts for one token, written by the thread that owns it.
+// Gates of the selected experts for one token, written by the thread that owns it.  The
+// kept logits go to the thread's scratch row (KMAX floats of shared memory) and the gates
+// are computed in rolled loops over it: each pair may run this once, from a cold
+// instruction cache, so one copy of the fp64 exp code instead of 2 KMAX inlined ones.
+// Same operations in the same order as a direct evaluation.
 template <int KMAX, bool BIAS>
 __device__ __forceinline__ void topk_write(const TopK<KMAX, BIAS>& st, long long t, int k, int score, int renorm,
-                                           float scale, int32_t* __restrict__ topk_idx, float* __restrict__ topk_gate) {
-  float g[KMAX];
-  if (score == MOE_SCORE_SOFTMAX) {
-    if (renorm) {
-      // softmax over the kept logits; the first entry holds the largest logit (no bias)
-      const double m = (double)st.logit_of(0);
-      double z = 0.0;
-#pragma unroll
-      for (int j = 0; j < KMAX; ++j)
-        if (j < k) z += exp((double)st.logit_of(j) - m);
-#pragma unroll
-      for (int j = 0; j < KMAX; ++j) g[j] = j < k ? (float)(exp((double)st.logit_of(j) - m) / z) : 0.f;
-    } else {
-#pragma unroll
-      for (int j = 0; j < KMAX; ++j)
-        g[j] = j < k ? (float)(exp((double)st.logit_of(j) - (double)st.M) / st.Z) : 0.f;
-    }
-  } else {
-    float s = 0.f;
-#pragma unroll
-    for (int j = 0; j < KMAX; ++j) {
-      g[j] = j < k ? score_f(st.logit_of(j), score) : 0.f;
-      s += g[j];
-    }
-    if (renorm) {
-#pragma unroll
-      for (int j = 0; j < KMAX; ++j) g[j] = g[j] / s;
-    }
-  }
+                                           float scale, float* scratch, int32_t* __restrict__ topk_idx,
+                                           float* __restrict__ topk_gate) {
 #pragma unroll
   for (int j = 0; j < KMAX; ++j) {
     if (j < k) {
       topk_idx[t * k + j] = st.index_of(j);
-      topk_gate[t * k + j] = g[j] * scale;
+      scratch[j] = st.logit_of(j);
+    }
+  }
+  float* g_out = topk_gate + t * k;
+  if (score == MOE_SCORE_SOFTMAX) {
+    if (renorm) {
+      // softmax over the kept logits; the first entry holds the largest logit (no bias)
+      const double m = (double)scratch[0];
+      double z = 0.0;
+#pragma unroll 1
+      for (int j = 0; j < k; ++j) z += exp((double)scratch[j] - m);
+#pragma unroll 1
+      for (int j = 0; j < k; ++j) g_out[j] = (float)(exp((double)scratch[j] - m) / z) * scale;
+    } else {
+#pragma unroll 1
+      for (int j = 0; j < k; ++j) g_out[j] = (float)(exp((double)scratch[j] - (double)st.M) / st.Z) * scale;
+    }
+  } else {
+    float s = 0.f;
+#pragma unroll 1
+    for (int j = 0; j < k; ++j) s += score_f(scratch[j], score);
+#pragma unroll 1
+    for (int j = 0; j < k; ++j) {
+      const float g = score_f(scratch[j], score);
+      g_out[j] = (renorm ? g / s : g) * scale;
     }
   }
 }
@@ -441,7 +442,9 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
       mbar_arrive_remote(map_to_rank(bar_tempty + 8 * acc, 0));
       if constexpr (kFused) {
         if (j == n_tiles - 1) {
-          if (lane < wrows) topk_write<KMAX, BIAS>(st, row0 + lane, k, score, renorm, scale, topk_idx, topk_gate);
+          if (lane < wrows)
+            topk_write<KMAX, BIAS>(st, row0 + lane, k, score, renorm, scale,
+                                   reinterpret_cast<float*>(stage + lane * kStagePitchF32), topk_idx, topk_gate);
           st.reset();
         }
       }

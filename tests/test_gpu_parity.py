@@ -86,16 +86,26 @@ SMALL = [
 ]
 
 
-# Both tile orientations of the grouped GEMMs: token-major (256 rows of one expert per CTA
-# pair) and weight-major (256 weight rows x the expert's tokens); the library picks one from
-# the average group size, MOE_B200_EXPERT_TILES forces it.
-TILES = ["tokens", "weights"]
+# Both tile orientations of the grouped GEMMs: token-major (128 rows of one expert per CTA,
+# or 256 per CTA pair) and weight-major (256 weight rows x the expert's tokens); the library
+# picks them from the average group size, MOE_B200_EXPERT_TILES and MOE_B200_TOKEN_TILES
+# force them.  "tokens" leaves the single / pair choice to the library (single CTAs on these
+# small shapes); "token_pairs" forces CTA pairs.
+TILES = ["tokens", "token_pairs", "weights"]
+
+
+def set_tiles(monkeypatch, tiles):
+    monkeypatch.setenv("MOE_B200_EXPERT_TILES", "weights" if tiles == "weights" else "tokens")
+    if tiles == "token_pairs":
+        monkeypatch.setenv("MOE_B200_TOKEN_TILES", "pairs")
+    else:
+        monkeypatch.delenv("MOE_B200_TOKEN_TILES", raising=False)
 
 
 @pytest.mark.parametrize("tiles", TILES)
 @pytest.mark.parametrize("cfg", SMALL, ids=lambda c: c.name)
 def test_small_full_parity(cfg, tiles, monkeypatch):
-    monkeypatch.setenv("MOE_B200_EXPERT_TILES", tiles)
+    set_tiles(monkeypatch, tiles)
     full_check(cfg)
 
 
@@ -103,7 +113,7 @@ def test_small_full_parity(cfg, tiles, monkeypatch):
 @pytest.mark.parametrize("cfg", [SMALL[0], SMALL[1], SMALL[4]], ids=lambda c: c.name)
 def test_bf16_rows_and_bf16_output(cfg, tiles, monkeypatch):
     """The bandwidth-saving variant: gated rows and y stored in bf16 (two more roundings)."""
-    monkeypatch.setenv("MOE_B200_EXPERT_TILES", tiles)
+    set_tiles(monkeypatch, tiles)
     host, dev = U.make_inputs(cfg)
     cap = O.capacity(cfg.T, cfg.E, cfg.k, cfg.capacity_factor)
     layer, g = U.gpu_forward(cfg, dev, cap, torch.bfloat16, torch.bfloat16)
@@ -392,7 +402,7 @@ GATHER = [c for c in SMALL if c.name in ("softmax_bf16", "sigmoid_bias_shared", 
 def test_gathered_gate_up_is_bitwise_the_permuted_one(cfg, tiles, monkeypatch):
     """Same token rows, same tiles, same accumulation order: H and the reproducible y agree
     bit for bit, in both tile orientations (weight-major: the rows gathered by cp.async)."""
-    monkeypatch.setenv("MOE_B200_EXPERT_TILES", tiles)
+    set_tiles(monkeypatch, tiles)
     host, dev = U.make_inputs(cfg)
     cap = O.capacity(cfg.T, cfg.E, cfg.k, cfg.capacity_factor, True)
     lp, gp = U.gpu_forward(cfg, dev, cap)
@@ -406,7 +416,7 @@ def test_gathered_gate_up_is_bitwise_the_permuted_one(cfg, tiles, monkeypatch):
 @pytest.mark.parametrize("tiles", TILES)
 def test_gathered_bad_token_is_reported_not_trapped(tiles, monkeypatch):
     from routing_dispatch_expert_moe_b200 import moe as M
-    monkeypatch.setenv("MOE_B200_EXPERT_TILES", tiles)
+    set_tiles(monkeypatch, tiles)
     for cfg in (SMALL[0], SMALL[6]):                          # tensor-core and fp32 SIMT forms
         host, dev = U.make_inputs(cfg)
         layer, g = U.gpu_forward(cfg, dev, -1, dispatch="gather")
@@ -573,5 +583,5 @@ def test_c5_stress_full_size_bf16_rows_and_output():
 @pytest.mark.parametrize("name,tiles", [("c2_handbook", "weights"), ("c5_stress", "tokens")])
 def test_full_size_bf16_form_other_tile_orientation(name, tiles, monkeypatch):
     """The orientation the library does not pick for this workload, at full size."""
-    monkeypatch.setenv("MOE_B200_EXPERT_TILES", tiles)
+    set_tiles(monkeypatch, tiles)
     bf16_full_size_check(name)
