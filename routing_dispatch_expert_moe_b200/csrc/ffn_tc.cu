@@ -122,10 +122,10 @@ template <int MODE, typename OutT>
 __device__ __forceinline__ void epilogue_tile(uint32_t taddr, uint8_t* stage, int lane, long long wrow0, int wrows,
                                               int n_tile, int F, int N_out, const float* __restrict__ gate_of_row,
                                               OutT* __restrict__ out, const int32_t* __restrict__ token_of_row,
-                                              int n_tokens, int* err, int c_begin = 0, int c_end = BN / 32) {
+                                              int n_tokens, int* err, float gs, int c_begin = 0,
+                                              int c_end = BN / 32) {
   if constexpr (MODE == 3) {
     const int n0 = n_tile * BN;
-    const float gs = (lane < wrows && gate_of_row) ? __ldg(gate_of_row + wrow0 + lane) : 1.f;
     const uint64_t pol = l2_evict_last_policy();
     int tok = -1;
     if (lane < wrows) {
@@ -169,7 +169,6 @@ __device__ __forceinline__ void epilogue_tile(uint32_t taddr, uint8_t* stage, in
   } else {
     static_assert(MODE == 1, "grouped GEMM modes: 0 gate/up, 1 down, 3 down + combine, 4 gathered gate/up");
     const int n0 = n_tile * BN;
-    const float gs = (lane < wrows && gate_of_row) ? __ldg(gate_of_row + wrow0 + lane) : 1.f;
     // two 32-column chunks per TMEM wait: with K = F of a few k-blocks this epilogue is as
     // long as the tile's mainloop, and each wait is a full TMEM round trip
 #pragma unroll 1
@@ -404,19 +403,22 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
       const TileCoord tc = tile_coord(tile_start, offsets, E, BM, tile);
       const int acc = it & 1;
       const uint32_t acc_phase = (uint32_t)(it >> 1) & 1u;
+      const long long wrow0 = (long long)tc.row0 + q * 32;          // first row of this warp
+      const int wrows = min(32, max(0, tc.rows - q * 32));          // valid rows of this warp
+      // the row's gate, fetched while the tile's MMAs still run
+      const float gs = ((MODE == 1 || MODE == 3) && lane < wrows && gate_of_row) ? __ldg(gate_of_row + wrow0 + lane)
+                                                                                  : 1.f;
       const bool got = mbar_wait(bar_tfull + 8 * acc, acc_phase, abort_flag, err);
       // tcgen05.ld is .sync.aligned: the whole warp goes on, or the whole warp stops
       if (!__all_sync(0xffffffffu, got)) break;
       __syncwarp();
       tc_fence_after();
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-      const long long wrow0 = (long long)tc.row0 + q * 32;          // first row of this warp
-      const int wrows = min(32, max(0, tc.rows - q * 32));          // valid rows of this warp
       (void)r_in;
       // a warp past the group's last row has nothing to read or store (warp-uniform)
       if (wrows > 0)
         epilogue_tile<MODE, OutT>(taddr, stage, lane, wrow0, wrows, tc.n_tile, F, N_out, gate_of_row, out,
-                                  token_of_row, n_tokens, err);
+                                  token_of_row, n_tokens, err, gs);
       tc_fence_before();
       mbar_arrive(bar_tempty + 8 * acc);
     }
@@ -594,19 +596,22 @@ grouped_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
       const TileCoord tc = tile_coord(tile_start, offsets, E, PM, tile);
       const int acc = it & 1;
       const uint32_t acc_phase = (uint32_t)(it >> 1) & 1u;
+      const int cta_rows = min(BM, max(0, tc.rows - (int)rank * BM));
+      const long long wrow0 = (long long)tc.row0 + (int)rank * BM + q * 32;
+      const int wrows = min(32, max(0, cta_rows - q * 32));
+      // the row's gate, fetched while the tile's MMAs still run
+      const float gs = ((MODE == 1 || MODE == 3) && lane < wrows && gate_of_row) ? __ldg(gate_of_row + wrow0 + lane)
+                                                                                  : 1.f;
       const bool got = mbar_wait(bar_tfull + 8 * acc, acc_phase, abort_flag, err);
       if (!__all_sync(0xffffffffu, got)) break;
       __syncwarp();
       tc_fence_after();
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-      const int cta_rows = min(BM, max(0, tc.rows - (int)rank * BM));
-      const long long wrow0 = (long long)tc.row0 + (int)rank * BM + q * 32;
-      const int wrows = min(32, max(0, cta_rows - q * 32));
       // a warp past the group's last row has nothing to read or store (warp-uniform): with
       // many small groups most of a 256-row tile is padding
       if (wrows > 0)
         epilogue_tile<MODE, OutT>(taddr, stage, lane, wrow0, wrows, tc.n_tile, F, N_out, gate_of_row, out,
-                                  token_of_row, n_tokens, err, c_begin, c_end);
+                                  token_of_row, n_tokens, err, gs, c_begin, c_end);
       tc_fence_before();
       mbar_arrive_remote(map_to_rank(bar_tempty + 8 * acc, 0));
     }

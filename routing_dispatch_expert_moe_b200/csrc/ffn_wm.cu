@@ -116,18 +116,29 @@ __device__ __forceinline__ void stage_store32_t(uint8_t* stage, const float (&v)
 // weights' per-tensor scale; 1 for bf16 weights).
 //   MODE 0: H[token][f] = silu(wscale g) * (wscale u), bf16;
 //   MODE 1: y[token][n] = gate_of_row[token] * wscale * acc.
+// Gate of the token in row c * 32 + lane of a weight-major tile (1 past the tile's rows, or
+// without gates).
+__device__ __forceinline__ float wm_gate(const float* __restrict__ gate_of_row, const TileCoord& tc, int c,
+                                         int lane) {
+  const int r = c * 32 + lane;
+  return (gate_of_row && r < tc.rows) ? __ldg(gate_of_row + tc.row0 + r) : 1.f;
+}
+
+// g0, g1 (MODE 1): this lane's gates of the tile's first two 32-token chunks, fetched by the
+// caller before the accumulator was ready; later gates are fetched one chunk pair ahead.
 template <int MODE, typename OutT>
 __device__ __forceinline__ void wm_epilogue_tile(uint32_t taddr, uint8_t* stage, int lane, const TileCoord& tc,
                                                  int rank, int q, int d, int F, float wscale,
-                                                 const float* __restrict__ gate_of_row, OutT* __restrict__ out) {
+                                                 const float* __restrict__ gate_of_row, OutT* __restrict__ out,
+                                                 float g0 = 1.f, float g1 = 1.f) {
   const int col0 = tc.n_tile * 256 + rank * kWRows + q * 32;   // this warp's first feature
   const int chunks = (tc.rows + 31) / 32;
+  if constexpr (MODE == 0) {
 #pragma unroll 1
-  for (int c = 0; c < chunks; ++c) {
-    const long long r0 = (long long)tc.row0 + c * 32;
-    const int rv = min(32, tc.rows - c * 32);
-    float h[32];
-    if constexpr (MODE == 0) {
+    for (int c = 0; c < chunks; ++c) {
+      const long long r0 = (long long)tc.row0 + c * 32;
+      const int rv = min(32, tc.rows - c * 32);
+      float h[32];
       uint32_t g[32], u[32];
       tmem_ld32(taddr + c * 32, g);
       tmem_ld32(taddr + 128 + c * 32, u);
@@ -141,8 +152,13 @@ __device__ __forceinline__ void wm_epilogue_tile(uint32_t taddr, uint8_t* stage,
         h[i] = __fdividef(gi, 1.f + __expf(-gi)) * (__uint_as_float(u[i]) * wscale);
       }
       stage_store32_t<OutT>(stage, h, lane, out, r0, rv, F, col0, F);
-    } else {
-      // two 32-token chunks per TMEM wait (the tile's mainloop is only K / 64 k-blocks)
+    }
+  } else {
+    // two 32-token chunks per TMEM wait (the tile's mainloop is only K / 64 k-blocks)
+    float ga = g0, gb = g1;
+#pragma unroll 1
+    for (int c = 0; c < chunks; c += 2) {
+      const float na = wm_gate(gate_of_row, tc, c + 2, lane), nb = wm_gate(gate_of_row, tc, c + 3, lane);
       const bool two = c + 1 < chunks;                     // warp-uniform
       uint32_t v[32], vb[32];
       tmem_ld32(taddr + c * 32, v);
@@ -150,19 +166,21 @@ __device__ __forceinline__ void wm_epilogue_tile(uint32_t taddr, uint8_t* stage,
       tmem_wait_ld();
       tmem_regs_ready(v);
       tmem_regs_ready(vb);
-      const float gs = ((gate_of_row && lane < rv) ? __ldg(gate_of_row + r0 + lane) : 1.f) * wscale;
+      float h[32];
+      const float gs = ga * wscale;
 #pragma unroll
       for (int i = 0; i < 32; ++i) h[i] = __uint_as_float(v[i]) * __shfl_sync(0xffffffffu, gs, i);
-      stage_store32_t<OutT>(stage, h, lane, out, r0, rv, d, col0, d);
+      stage_store32_t<OutT>(stage, h, lane, out, (long long)tc.row0 + c * 32, min(32, tc.rows - c * 32), d, col0,
+                            d);
       if (two) {
-        const long long r0b = r0 + 32;
-        const int rvb = min(32, tc.rows - (c + 1) * 32);
-        const float gsb = ((gate_of_row && lane < rvb) ? __ldg(gate_of_row + r0b + lane) : 1.f) * wscale;
+        const float gsb = gb * wscale;
 #pragma unroll
         for (int i = 0; i < 32; ++i) h[i] = __uint_as_float(vb[i]) * __shfl_sync(0xffffffffu, gsb, i);
-        stage_store32_t<OutT>(stage, h, lane, out, r0b, rvb, d, col0, d);
-        ++c;
+        stage_store32_t<OutT>(stage, h, lane, out, (long long)tc.row0 + (c + 1) * 32,
+                              min(32, tc.rows - (c + 1) * 32), d, col0, d);
       }
+      ga = na;
+      gb = nb;
     }
   }
 }
@@ -391,12 +409,15 @@ grouped_gemm_wm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
       const TileCoord tc = tile_coord(tile_start, offsets, E, C::NT, tile);
       const int acc = it & 1;
       const uint32_t acc_phase = (uint32_t)(it >> 1) & 1u;
+      // the first gates, fetched while the tile's MMAs still run
+      const float g0 = MODE == 1 ? wm_gate(gate_of_row, tc, 0, lane) : 1.f;
+      const float g1 = MODE == 1 ? wm_gate(gate_of_row, tc, 1, lane) : 1.f;
       const bool got = mbar_wait(bar_tfull + 8 * acc, acc_phase, abort_flag, err);
       if (!__all_sync(0xffffffffu, got)) break;
       __syncwarp();
       tc_fence_after();
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * 256);
-      wm_epilogue_tile<MODE, OutT>(taddr, stage, lane, tc, (int)rank, q, d, F, 1.f, gate_of_row, out);
+      wm_epilogue_tile<MODE, OutT>(taddr, stage, lane, tc, (int)rank, q, d, F, 1.f, gate_of_row, out, g0, g1);
       tc_fence_before();
       mbar_arrive_remote(map_to_rank(bar_tempty + 8 * acc, 0));
     }
@@ -674,13 +695,16 @@ grouped_gemm_wm4_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_co
       const TileCoord tc = tile_coord(tile_start, offsets, E, C::NT, tile);
       const int acc = it & 1;
       const uint32_t acc_phase = (uint32_t)(it >> 1) & 1u;
+      // the first gates, fetched while the tile's MMAs still run
+      const float g0 = MODE == 1 ? wm_gate(gate_of_row, tc, 0, lane) : 1.f;
+      const float g1 = MODE == 1 ? wm_gate(gate_of_row, tc, 1, lane) : 1.f;
       const bool got = mbar_wait(bar_tfull + 8 * acc, acc_phase, abort_flag, err);
       if (!__all_sync(0xffffffffu, got)) break;
       __syncwarp();
       tc_fence_after();
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * 256);
       const float ws = tensor_scale ? __ldg(tensor_scale + tc.e) : 1.f;
-      wm_epilogue_tile<MODE, OutT>(taddr, stage, lane, tc, (int)rank, q, d, F, ws, gate_of_row, out);
+      wm_epilogue_tile<MODE, OutT>(taddr, stage, lane, tc, (int)rank, q, d, F, ws, gate_of_row, out, g0, g1);
       tc_fence_before();
       mbar_arrive_remote(map_to_rank(bar_tempty + 8 * acc, 0));
     }

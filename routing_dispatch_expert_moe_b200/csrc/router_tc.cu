@@ -164,10 +164,16 @@ struct TopK {
   }
 };
 
+// The no-bias selection key: the logit's ordered image, then the complemented index (among
+// equal logits the lower index has the larger key).  NaN ranks as -inf.
+__device__ __forceinline__ uint64_t plain_key(float l, int e) {
+  const float kf = (l == l) ? l : -INFINITY;
+  return ((uint64_t)ord32(kf) << 32) | (uint32_t)(~(uint32_t)e);
+}
+
 template <int KMAX, bool BIAS>
-__device__ __forceinline__ void topk_consider(TopK<KMAX, BIAS>& st, float l, int e, int score, bool full_softmax,
-                                              const float* __restrict__ sel_bias) {
-  if (full_softmax && l == l && l != -INFINITY) {   // running normaliser of the full softmax
+__device__ __forceinline__ void topk_norm(TopK<KMAX, BIAS>& st, float l) {
+  if (l == l && l != -INFINITY) {                  // running normaliser of the full softmax
     if (l > st.M) {
       st.Z = st.Z * exp((double)st.M - (double)l) + 1.0;
       st.M = l;
@@ -175,6 +181,12 @@ __device__ __forceinline__ void topk_consider(TopK<KMAX, BIAS>& st, float l, int
       st.Z += exp((double)l - (double)st.M);
     }
   }
+}
+
+template <int KMAX, bool BIAS>
+__device__ __forceinline__ void topk_consider(TopK<KMAX, BIAS>& st, float l, int e, int score, bool full_softmax,
+                                              const float* __restrict__ sel_bias) {
+  if (full_softmax) topk_norm<KMAX, BIAS>(st, l);
   if (BIAS) {
     double kd = -INFINITY;
     if (l == l) {
@@ -183,8 +195,7 @@ __device__ __forceinline__ void topk_consider(TopK<KMAX, BIAS>& st, float l, int
     }
     st.insert(ord64(kd), e, l);
   } else {
-    const float kf = (l == l) ? l : -INFINITY;
-    st.insert(((uint64_t)ord32(kf) << 32) | (uint32_t)(~(uint32_t)e), e, l);
+    st.insert(plain_key(l, e), e, l);
   }
 }
 
@@ -427,14 +438,49 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
           // keeps the selection code small (a pair may run this epilogue only once, from
           // a cold instruction cache)
           const float4* mine = reinterpret_cast<const float4*>(stage + lane * kStagePitchF32);
+          const int ec = e0 + c * 32;
+          if constexpr (!BIAS) {
+            // Two passes.  First every candidate is tested against the thread's current
+            // k-th key (and feeds the full-softmax normaliser); then the warp inserts only
+            // the candidates that passed, lowest position first, as many rounds as the
+            // busiest lane needs.  The k-th key only grows, so a candidate that fails the
+            // test now would be rejected later too: the same selection as inserting every
+            // candidate in turn, without running the insertion wherever any one lane of
+            // the warp needs it.
+            uint32_t pass = 0;
 #pragma unroll 1
-          for (int qd = 0; qd < 8; ++qd) {
-            const float4 f = mine[qd];
-            const float fv[4] = {f.x, f.y, f.z, f.w};
-            const int eb = e0 + c * 32 + 4 * qd;
+            for (int qd = 0; qd < 8; ++qd) {
+              const float4 f = mine[qd];
+              const float fv[4] = {f.x, f.y, f.z, f.w};
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-              if (eb + i < E) topk_consider<KMAX, BIAS>(st, fv[i], eb + i, score, full_softmax, sel_bias);
+              for (int i = 0; i < 4; ++i) {
+                const int e = ec + 4 * qd + i;
+                if (e < E) {
+                  if (full_softmax) topk_norm<KMAX, BIAS>(st, fv[i]);
+                  if (plain_key(fv[i], e) > st.key[KMAX - 1]) pass |= 1u << (4 * qd + i);
+                }
+              }
+            }
+            const float* row = reinterpret_cast<const float*>(mine);
+#pragma unroll 1
+            while (__any_sync(0xffffffffu, pass != 0)) {
+              if (pass) {
+                const int p = __ffs(pass) - 1;
+                pass &= pass - 1;
+                const float l = row[p];
+                st.insert(plain_key(l, ec + p), ec + p, l);
+              }
+            }
+          } else {
+#pragma unroll 1
+            for (int qd = 0; qd < 8; ++qd) {
+              const float4 f = mine[qd];
+              const float fv[4] = {f.x, f.y, f.z, f.w};
+              const int eb = ec + 4 * qd;
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                if (eb + i < E) topk_consider<KMAX, BIAS>(st, fv[i], eb + i, score, full_softmax, sel_bias);
+            }
           }
         }
       }
