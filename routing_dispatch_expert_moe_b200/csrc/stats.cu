@@ -20,7 +20,8 @@
 namespace moe {
 namespace {
 
-constexpr int kStatsThreads = 256;
+constexpr int kStatsThreads = 512;
+constexpr int kStatsPer = (1024 + kStatsThreads - 1) / kStatsThreads;   // experts per thread (E <= 1024)
 
 // Score of one logit (fp32 transcendentals; every sum that uses them is fp64).
 __device__ __forceinline__ float score_f(float l, float m, int score) {
@@ -39,7 +40,7 @@ constexpr int kSub = kStatsThreads / 32;   // tokens per sub-chunk: one per warp
 //   (b) a thread per expert: P_e += s_e(t) / ss(t) over the sub-chunk's tokens, in order,
 //       from shared memory.
 // Every score is computed once.  Writes the CTA's P partials [E] and z2 partial.
-__global__ void __launch_bounds__(kStatsThreads)
+__global__ void __launch_bounds__(kStatsThreads, 2)
 stats_partial_kernel(const float* __restrict__ logits, int T, int E, int score, int tokens_per_cta,
                      double* __restrict__ partP, double* __restrict__ partZ) {
   extern __shared__ float s_sc[];            // [kSub][E]
@@ -51,8 +52,10 @@ stats_partial_kernel(const float* __restrict__ logits, int T, int E, int score, 
   const long long t_begin = (long long)blockIdx.x * tokens_per_cta;
   const long long t_end = min((long long)T, t_begin + tokens_per_cta);
   double z2 = 0.0;
-  // this thread's experts: e = threadIdx.x + i * kStatsThreads (E <= 1024: at most 4)
-  double P[4] = {0.0, 0.0, 0.0, 0.0};
+  // this thread's experts: e = threadIdx.x + i * kStatsThreads, i < kStatsPer
+  double P[kStatsPer];
+#pragma unroll
+  for (int q = 0; q < kStatsPer; ++q) P[q] = 0.0;
   for (long long c0 = t_begin; c0 < t_end; c0 += kSub) {
     const int n = (int)min((long long)kSub, t_end - c0);
     if (warp < n) {
@@ -68,6 +71,9 @@ stats_partial_kernel(const float* __restrict__ logits, int T, int E, int score, 
 #pragma unroll
       for (int o = 16; o; o >>= 1) mf = fmaxf(mf, __shfl_xor_sync(0xffffffffu, mf, o));
       double se = 0.0, ss = 0.0;
+      // unrolled so the transcendentals of several elements are in flight; the fp64 sums
+      // still add in element order
+#pragma unroll 4
       for (int e = lane; e < E; e += 32) {
         const float l = srow[e];
         const float ex = expf(l - mf);
@@ -89,7 +95,7 @@ stats_partial_kernel(const float* __restrict__ logits, int T, int E, int score, 
     }
     __syncthreads();
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
+    for (int q = 0; q < kStatsPer; ++q) {
       const int e = (int)threadIdx.x + q * kStatsThreads;
       if (e < E) {
         double acc = P[q];
@@ -100,7 +106,7 @@ stats_partial_kernel(const float* __restrict__ logits, int T, int E, int score, 
     __syncthreads();
   }
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
+  for (int q = 0; q < kStatsPer; ++q) {
     const int e = (int)threadIdx.x + q * kStatsThreads;
     if (e < E) partP[(long long)blockIdx.x * E + e] = P[q];
   }
@@ -113,34 +119,45 @@ stats_partial_kernel(const float* __restrict__ logits, int T, int E, int score, 
   }
 }
 
-// Stage 2: one CTA of 1024 threads.  P_e: the threads form G = 1024 / E groups of E;
-// thread (g, e) sums partial rows g, g + G, g + 2G, ... of expert e (consecutive threads
-// read consecutive experts of one row: whole lines per warp load, 8 loads in flight),
-// then the G group sums are added in group order.  The four per-expert sums (aux, kept,
-// variance, max) are reduced together in one pass.
-__global__ void __launch_bounds__(1024)
-stats_final_kernel(const double* __restrict__ partP, const double* __restrict__ partZ, int nparts,
-                   const int32_t* __restrict__ counts, const int32_t* __restrict__ kept, int T, int E,
-                   int k, float* __restrict__ load, float* __restrict__ stats5) {
-  __shared__ double Ps[1024];
-  __shared__ double grp[1024];
-  __shared__ double red[4][32];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  const int G = max(1, (int)blockDim.x / E);                 // E <= 1024
-  if ((int)threadIdx.x < G * E) {
-    const int e = (int)threadIdx.x % E, g = (int)threadIdx.x / E;
-    double p = 0.0;
-    int b = g;
-    for (; b + 7 * G < nparts; b += 8 * G) {
+// Stage 2a: P_e summed over the partial rows, 32 experts per CTA.  Lane = expert (whole
+// 256-byte lines per warp load), warp w takes rows w, w + 8, w + 16, ... (8 loads in
+// flight), then the 8 warp sums are added in warp order: a fixed order.
+__global__ void __launch_bounds__(256)
+stats_reduce_kernel(const double* __restrict__ partP, int nparts, int E, double* __restrict__ Pout) {
+  __shared__ double wsum[8][32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int e = blockIdx.x * 32 + lane;
+  double p = 0.0;
+  if (e < E) {
+    int b = warp;
+    for (; b + 8 * 7 < nparts; b += 8 * 8) {
       double v[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = __ldg(partP + (long long)(b + u * G) * E + e);
+      for (int u = 0; u < 8; ++u) v[u] = __ldg(partP + (long long)(b + 8 * u) * E + e);
 #pragma unroll
       for (int u = 0; u < 8; ++u) p += v[u];
     }
-    for (; b < nparts; b += G) p += __ldg(partP + (long long)b * E + e);
-    grp[threadIdx.x] = p;
+    for (; b < nparts; b += 8) p += __ldg(partP + (long long)b * E + e);
   }
+  wsum[warp][lane] = p;
+  __syncthreads();
+  if (warp == 0 && e < E) {
+    double t = 0.0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) t += wsum[w][lane];
+    Pout[e] = t;
+  }
+}
+
+// Stage 2b: one CTA of 1024 threads: the z partials, then the four per-expert sums (aux,
+// kept, variance, max) reduced together in one pass.
+__global__ void __launch_bounds__(1024)
+stats_final_kernel(const double* __restrict__ Psum, const double* __restrict__ partZ, int nparts,
+                   const int32_t* __restrict__ counts, const int32_t* __restrict__ kept, int T, int E,
+                   int k, float* __restrict__ load, float* __restrict__ stats5) {
+  __shared__ double Ps[1024];
+  __shared__ double red[4][32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   double z = 0.0;
   if (warp == nw - 1) {                       // the z partials, on the last warp
     int b = lane;
@@ -155,12 +172,7 @@ stats_final_kernel(const double* __restrict__ partP, const double* __restrict__ 
 #pragma unroll
     for (int o = 16; o; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
   }
-  __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    double p = 0.0;
-    for (int g = 0; g < G; ++g) p += grp[g * E + e];
-    Ps[e] = p;
-  }
+  for (int e = threadIdx.x; e < E; e += blockDim.x) Ps[e] = Psum[e];
   __syncthreads();
   const double TK = (double)T * k;
   const double mean = TK / E;
@@ -216,7 +228,7 @@ int stats_parts(int T) {
 
 size_t router_stats_workspace_bytes(int T, int E) {
   const int parts = stats_parts(T > 0 ? T : 1);
-  return ((size_t)parts * E + parts) * sizeof(double);
+  return ((size_t)parts * E + parts + E) * sizeof(double);   // partials [parts][E], z partials, P [E]
 }
 
 moe_status launch_router_stats(const float* logits, const int32_t* counts, const int32_t* kept,
@@ -230,12 +242,19 @@ moe_status launch_router_stats(const float* logits, const int32_t* counts, const
   const int parts = stats_parts(T);
   double* pP = static_cast<double*>(ws);
   double* pZ = pP + (size_t)parts * E;
+  double* pSum = pZ + parts;
   const int tpc = (T + parts - 1) / parts;
-  stats_partial_kernel<<<parts, kStatsThreads, (size_t)kSub * E * sizeof(float), s>>>(logits, T, E, score, tpc, pP,
-                                                                                        pZ);
+  static std::atomic<int> configured[kMaxDevices];
+  const size_t smem = (size_t)kSub * E * sizeof(float);    // up to 64 KB (E = 1024)
+  moe_status st0 = ensure_smem_limit(configured, stats_partial_kernel, (size_t)kSub * 1024 * sizeof(float));
+  if (st0 != MOE_OK) return st0;
+  stats_partial_kernel<<<parts, kStatsThreads, smem, s>>>(logits, T, E, score, tpc, pP, pZ);
   moe_status st = check_launch();
   if (st != MOE_OK) return st;
-  stats_final_kernel<<<1, 1024, 0, s>>>(pP, pZ, parts, counts, kept, T, E, k, load, stats5);
+  stats_reduce_kernel<<<(E + 31) / 32, 256, 0, s>>>(pP, parts, E, pSum);
+  st = check_launch();
+  if (st != MOE_OK) return st;
+  stats_final_kernel<<<1, 1024, 0, s>>>(pSum, pZ, parts, counts, kept, T, E, k, load, stats5);
   return check_launch();
 }
 

@@ -355,5 +355,5 @@ class MoELayer:
         if self.has_shared:
             n += 2
         if with_stats:
-            n += 2
+            n += 3                         # per-CTA partials, per-expert sums, scalars
         return n

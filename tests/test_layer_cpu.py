@@ -54,17 +54,18 @@ class _Stub:
 
 def test_launch_count_matches_the_kernels_each_form_runs():
     # handbook default: the tensor-core router with the top-k in its epilogue, rank +
-    # scatter, permute, gate/up, down, combine; statistics partial + final (9 kernels)
-    assert _Stub().launches_per_forward(True) == 9
+    # scatter, permute, gate/up, down, combine; statistics partials, per-expert sums and
+    # scalars (10 kernels)
+    assert _Stub().launches_per_forward(True) == 10
     assert _Stub().launches_per_forward(False) == 7
-    assert _Stub(dtype=torch.float32).launches_per_forward(True) == 10       # SIMT router GEMM + top-k
-    assert _Stub(E=37).launches_per_forward(True) == 10                      # E % 4: SIMT router
-    assert _Stub(T_max=200).launches_per_forward(True) == 10                 # under 256 tokens: SIMT router
-    assert _Stub(score="softmax", bias=True).launches_per_forward(True) == 10   # + a separate top-k pass
-    assert _Stub(score="sigmoid", bias=True).launches_per_forward(True) == 9    # biased keys fused
-    assert _Stub(routing="uniform").launches_per_forward(True) == 10         # router logits -> fixed selection
-    assert _Stub(routing="noisy").launches_per_forward(True) == 12           # two router GEMMs + H + top-k
-    assert _Stub(combine="fused").launches_per_forward(True) == 8
-    assert _Stub(combine="fused", fused_bf16=True).launches_per_forward(True) == 9
-    assert _Stub(dispatch="gather").launches_per_forward(True) == 8
-    assert _Stub(shared=True).launches_per_forward(True) == 11
+    assert _Stub(dtype=torch.float32).launches_per_forward(True) == 11       # SIMT router GEMM + top-k
+    assert _Stub(E=37).launches_per_forward(True) == 11                      # E % 4: SIMT router
+    assert _Stub(T_max=200).launches_per_forward(True) == 11                 # under 256 tokens: SIMT router
+    assert _Stub(score="softmax", bias=True).launches_per_forward(True) == 11   # + a separate top-k pass
+    assert _Stub(score="sigmoid", bias=True).launches_per_forward(True) == 10    # biased keys fused
+    assert _Stub(routing="uniform").launches_per_forward(True) == 11         # router logits -> fixed selection
+    assert _Stub(routing="noisy").launches_per_forward(True) == 13           # two router GEMMs + H + top-k
+    assert _Stub(combine="fused").launches_per_forward(True) == 9
+    assert _Stub(combine="fused", fused_bf16=True).launches_per_forward(True) == 10
+    assert _Stub(dispatch="gather").launches_per_forward(True) == 9
+    assert _Stub(shared=True).launches_per_forward(True) == 12
