@@ -111,11 +111,6 @@ __device__ __forceinline__ void stage_store32_t(uint8_t* stage, const float (&v)
   __syncwarp();
 }
 
-// One tile's epilogue for one warp: features col0 .. col0+31 (its TMEM lanes) of the tile's
-// tokens, 32 tokens per tcgen05.ld.  wscale multiplies every accumulator (the 4-bit
-// weights' per-tensor scale; 1 for bf16 weights).
-//   MODE 0: H[token][f] = silu(wscale g) * (wscale u), bf16;
-//   MODE 1: y[token][n] = gate_of_row[token] * wscale * acc.
 // Gate of the token in row c * 32 + lane of a weight-major tile (1 past the tile's rows, or
 // without gates).
 __device__ __forceinline__ float wm_gate(const float* __restrict__ gate_of_row, const TileCoord& tc, int c,
@@ -124,6 +119,11 @@ __device__ __forceinline__ float wm_gate(const float* __restrict__ gate_of_row, 
   return (gate_of_row && r < tc.rows) ? __ldg(gate_of_row + tc.row0 + r) : 1.f;
 }
 
+// One tile's epilogue for one warp: features col0 .. col0+31 (its TMEM lanes) of the tile's
+// tokens, 32 tokens per tcgen05.ld.  wscale multiplies every accumulator (the 4-bit
+// weights' per-tensor scale; 1 for bf16 weights).
+//   MODE 0: H[token][f] = silu(wscale g) * (wscale u), bf16;
+//   MODE 1: y[token][n] = gate_of_row[token] * wscale * acc.
 // g0, g1 (MODE 1): this lane's gates of the tile's first two 32-token chunks, fetched by the
 // caller before the accumulator was ready; later gates are fetched one chunk pair ahead.
 template <int MODE, typename OutT>
@@ -423,6 +423,10 @@ grouped_gemm_wm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
     }
   }
 
+  // converge each warp first: in the producer and MMA warps one lane ran the role's loop
+  // while the others went ahead, and the block barrier must see every warp whole, or it
+  // can let a thread through before the epilogue warps have finished reading TMEM
+  __syncwarp();
   __syncthreads();
   cluster_sync();                                           // no remote arrive after a CTA exits
   if (warp == 1) {
@@ -472,7 +476,6 @@ struct Wm4Cfg {
   static constexpr int stage_pitch = (stage_bytes + 1023) / 1024 * 1024;
   static constexpr int stages = MODE == 0 ? 4 : 5;
   static constexpr int epi_warps = 4, cvt_warps = 8;
-  static constexpr int cvt_threads = 32 * cvt_warps;
   static constexpr int threads = 64 + 32 * (epi_warps + cvt_warps);
   static constexpr int bars = stages * stage_pitch;
   static constexpr int nbars = 3 * stages + 4 + 1;
@@ -710,7 +713,7 @@ grouped_gemm_wm4_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_co
     }
   } else {
     // ------------------------------------------------------------ converters (both CTAs)
-    const int ct = threadIdx.x - 64 - 32 * C::epi_warps;     // 0 .. cvt_threads - 1
+    const int ct = threadIdx.x - 64 - 32 * C::epi_warps;     // 0 .. 32 cvt_warps - 1
     const int r = ct & (kWRows - 1);                         // its weight row of the block
     const int a = MODE == 0 ? ct / kWRows : 0;               // gate/up: block (gate or up)
     const int c0 = MODE == 0 ? 0 : (ct / kWRows) * 4;        // down: half of the row's chunks
@@ -734,6 +737,10 @@ grouped_gemm_wm4_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_co
     }
   }
 
+  // converge each warp first: in the producer and MMA warps one lane ran the role's loop
+  // while the others went ahead, and the block barrier must see every warp whole, or it
+  // can let a thread through before the epilogue warps have finished reading TMEM
+  __syncwarp();
   __syncthreads();
   cluster_sync();                                           // no remote arrive after a CTA exits
   if (warp == 1) {

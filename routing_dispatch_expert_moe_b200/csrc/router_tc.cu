@@ -497,6 +497,10 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     }
   }
 
+  // converge each warp first: in the producer and MMA warps one lane ran the role's loop
+  // while the others went ahead, and the block barrier must see every warp whole, or it
+  // can let a thread through before the epilogue warps have finished reading TMEM
+  __syncwarp();
   __syncthreads();
   cluster_sync();                                           // no remote arrive after a CTA exits
   if (warp == 1) {
