@@ -138,22 +138,28 @@ struct TopK {
     M = -INFINITY;
     Z = 0.0;
   }
+  // Insertion into the sorted list, all positions at once: compare the candidate with
+  // every entry (independent compares), then each entry at or after the insertion point
+  // takes its predecessor's value, the one at the insertion point the candidate.  Same
+  // result as bubbling the candidate down, without a chain of k dependent steps (the
+  // epilogue runs one warp per SM sub-partition, so dependent latency is not hidden).
   __device__ __forceinline__ void insert(uint64_t kc, int e, float l) {
     if (!(kc > key[KMAX - 1])) return;
+    bool up[KMAX];
 #pragma unroll
-    for (int i = 0; i < KMAX; ++i) {
-      const bool up = kc > key[i];
-      const uint64_t tk = key[i];
-      key[i] = up ? kc : tk;
-      kc = up ? tk : kc;
+    for (int i = 0; i < KMAX; ++i) up[i] = kc > key[i];
+#pragma unroll
+    for (int i = KMAX - 1; i >= 1; --i) {                  // descending: key[i - 1] is still old
+      key[i] = up[i] ? (up[i - 1] ? key[i - 1] : kc) : key[i];
       if (BIAS) {
-        const int ti = idx[i];
-        const float tl = lg[i];
-        idx[i] = up ? e : ti;
-        lg[i] = up ? l : tl;
-        e = up ? ti : e;
-        l = up ? tl : l;
+        idx[i] = up[i] ? (up[i - 1] ? idx[i - 1] : e) : idx[i];
+        lg[i] = up[i] ? (up[i - 1] ? lg[i - 1] : l) : lg[i];
       }
+    }
+    key[0] = up[0] ? kc : key[0];
+    if (BIAS) {
+      idx[0] = up[0] ? e : idx[0];
+      lg[0] = up[0] ? l : lg[0];
     }
   }
   __device__ __forceinline__ int index_of(int i) const {
@@ -447,8 +453,14 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             // test now would be rejected later too: the same selection as inserting every
             // candidate in turn, without running the insertion wherever any one lane of
             // the warp needs it.
+            // Every entry of the list has a lower index than this chunk's candidates, so a
+            // candidate's key exceeds the k-th key exactly when its logit (NaN as -inf)
+            // exceeds the k-th logit, or the list still has a free slot (key 0).
             uint32_t pass = 0;
-#pragma unroll 1
+            const uint64_t klast = st.key[KMAX - 1];
+            const bool open = klast == 0ull;
+            const float thr = unord32((uint32_t)(klast >> 32));
+#pragma unroll 2
             for (int qd = 0; qd < 8; ++qd) {
               const float4 f = mine[qd];
               const float fv[4] = {f.x, f.y, f.z, f.w};
@@ -457,7 +469,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 const int e = ec + 4 * qd + i;
                 if (e < E) {
                   if (full_softmax) topk_norm<KMAX, BIAS>(st, fv[i]);
-                  if (plain_key(fv[i], e) > st.key[KMAX - 1]) pass |= 1u << (4 * qd + i);
+                  if (open || (fv[i] == fv[i] && fv[i] > thr)) pass |= 1u << (4 * qd + i);
                 }
               }
             }
