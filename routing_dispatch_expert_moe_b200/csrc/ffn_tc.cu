@@ -438,10 +438,6 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
     }
   }
 
-  // converge each warp first: in the producer and MMA warps one lane ran the role's loop
-  // while the others went ahead, and the block barrier must see every warp whole, or it
-  // can let a thread through before the epilogue warps have finished reading TMEM
-  __syncwarp();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
@@ -635,10 +631,6 @@ grouped_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
     }
   }
 
-  // converge each warp first: in the producer and MMA warps one lane ran the role's loop
-  // while the others went ahead, and the block barrier must see every warp whole, or it
-  // can let a thread through before the epilogue warps have finished reading TMEM
-  __syncwarp();
   __syncthreads();
   cluster_sync();                                           // no remote arrive after a CTA exits
   if (warp == 1) {

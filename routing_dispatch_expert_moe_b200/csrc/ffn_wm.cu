@@ -423,10 +423,6 @@ grouped_gemm_wm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
     }
   }
 
-  // converge each warp first: in the producer and MMA warps one lane ran the role's loop
-  // while the others went ahead, and the block barrier must see every warp whole, or it
-  // can let a thread through before the epilogue warps have finished reading TMEM
-  __syncwarp();
   __syncthreads();
   cluster_sync();                                           // no remote arrive after a CTA exits
   if (warp == 1) {
@@ -737,10 +733,6 @@ grouped_gemm_wm4_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_co
     }
   }
 
-  // converge each warp first: in the producer and MMA warps one lane ran the role's loop
-  // while the others went ahead, and the block barrier must see every warp whole, or it
-  // can let a thread through before the epilogue warps have finished reading TMEM
-  __syncwarp();
   __syncthreads();
   cluster_sync();                                           // no remote arrive after a CTA exits
   if (warp == 1) {

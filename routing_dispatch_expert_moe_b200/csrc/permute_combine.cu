@@ -105,17 +105,19 @@ __device__ __forceinline__ void store8<float>(void* base, long long e, const flo
 // KMAX: compile-time bound on k (multiple of 8).  The token's kept slots are first
 // compacted, in slot order, into a per-warp list in shared memory (a ballot gives each
 // kept slot its position), so dropped slots cost nothing, every batch of loads is full,
-// and the list costs no registers (two blocks fit on an SM).  Each lane then loads up to
-// 4 kept rows for VPI 8-element vectors (4 * VPI = 16 independent 16-byte loads in flight
-// once a token keeps 4 rows, the common case when capacity drops most slots) and adds them
-// in slot order: the same fp32 sum as visiting every slot.
+// and the list costs no registers (two blocks fit on an SM).  Each lane then loads R kept
+// rows for VPI 8-element vectors (16 independent 16-byte loads in flight for bf16 rows)
+// and adds them in slot order: the same fp32 sum as visiting every slot.
 template <typename InT, typename OutT, int KMAX>
 __global__ void __launch_bounds__(256, 2)
 combine_kernel(const void* __restrict__ y_rows, const int32_t* __restrict__ row_of,
                const float* __restrict__ topk_gate, const void* __restrict__ shared_y, int T, int d, int k,
                long long rows_max, void* __restrict__ y, int* err) {
-  constexpr int VPI = sizeof(InT) == 2 ? 4 : 2;       // vectors per lane per step
-  constexpr int R = 4;                                 // kept rows per batch of loads
+  // kept rows per batch x vectors per lane: 16 loads in flight either way; k <= 8 keeps
+  // one batch for a token that keeps all its slots, larger k (where capacity drops most
+  // slots) four rows so that a token keeping four still fills the batch
+  constexpr int R = KMAX <= 8 ? 8 : 4;
+  constexpr int VPI = (sizeof(InT) == 2 ? 16 : 8) / R;
   __shared__ int s_row[8][32];
   __shared__ float s_gate[8][32];
   const unsigned lane = threadIdx.x & 31;

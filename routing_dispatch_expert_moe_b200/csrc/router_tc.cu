@@ -45,6 +45,7 @@
 #include "tc_prims.cuh"
 
 #include <float.h>
+#include <type_traits>
 #include <stdlib.h>
 #include <string.h>
 
@@ -114,14 +115,16 @@ __device__ __forceinline__ uint64_t ord64(double v) {
   return (u >> 63) ? ~u : (u | (1ull << 63));
 }
 
-// A thread's running top-KMAX.  No bias: key = ord32(logit) << 32 | ~e (index and logit
-// recoverable from the key).  Bias: key = ord64(score + bias), with index and logit kept
-// beside it.  Kept sorted descending; a candidate moves ahead of an entry only when its
-// key is strictly larger, so among equal keys the earlier (lower) expert stays ahead.
+// A thread's running top-KMAX, sorted by key descending.  No bias: key = ord32(logit)
+// (NaN as -inf), the logit recoverable from the key; candidates arrive in increasing
+// expert order and only a strictly larger key moves ahead of an entry, so among equal
+// logits the lower index stays ahead.  Bias: key = ord64(score + bias), the logit kept
+// beside it.  Key 0 is below every candidate's key and marks an empty slot.
 template <int KMAX, bool BIAS>
 struct TopK {
-  uint64_t key[KMAX];
-  int idx[BIAS ? KMAX : 1];
+  using Key = typename std::conditional<BIAS, uint64_t, uint32_t>::type;
+  Key key[KMAX];
+  int idx[KMAX];
   float lg[BIAS ? KMAX : 1];
   float M;      // running maximum logit (non-renormalised softmax gates)
   double Z;     // running sum of exp(l - M) in fp64
@@ -129,11 +132,9 @@ struct TopK {
   __device__ __forceinline__ void reset() {
 #pragma unroll
     for (int i = 0; i < KMAX; ++i) {
-      key[i] = 0ull;
-      if (BIAS) {
-        idx[i] = 0;
-        lg[i] = 0.f;
-      }
+      key[i] = 0;
+      idx[i] = 0;
+      if (BIAS) lg[i] = 0.f;
     }
     M = -INFINITY;
     Z = 0.0;
@@ -143,39 +144,30 @@ struct TopK {
   // takes its predecessor's value, the one at the insertion point the candidate.  Same
   // result as bubbling the candidate down, without a chain of k dependent steps (the
   // epilogue runs one warp per SM sub-partition, so dependent latency is not hidden).
-  __device__ __forceinline__ void insert(uint64_t kc, int e, float l) {
+  __device__ __forceinline__ void insert(Key kc, int e, float l) {
     if (!(kc > key[KMAX - 1])) return;
     bool up[KMAX];
 #pragma unroll
     for (int i = 0; i < KMAX; ++i) up[i] = kc > key[i];
 #pragma unroll
-    for (int i = KMAX - 1; i >= 1; --i) {                  // descending: key[i - 1] is still old
+    for (int i = KMAX - 1; i >= 1; --i) {                  // descending: entry i - 1 is still old
       key[i] = up[i] ? (up[i - 1] ? key[i - 1] : kc) : key[i];
-      if (BIAS) {
-        idx[i] = up[i] ? (up[i - 1] ? idx[i - 1] : e) : idx[i];
-        lg[i] = up[i] ? (up[i - 1] ? lg[i - 1] : l) : lg[i];
-      }
+      idx[i] = up[i] ? (up[i - 1] ? idx[i - 1] : e) : idx[i];
+      if (BIAS) lg[i] = up[i] ? (up[i - 1] ? lg[i - 1] : l) : lg[i];
     }
     key[0] = up[0] ? kc : key[0];
-    if (BIAS) {
-      idx[0] = up[0] ? e : idx[0];
-      lg[0] = up[0] ? l : lg[0];
-    }
+    idx[0] = up[0] ? e : idx[0];
+    if (BIAS) lg[0] = up[0] ? l : lg[0];
   }
-  __device__ __forceinline__ int index_of(int i) const {
-    return BIAS ? idx[i] : (int)(~(uint32_t)key[i]);
-  }
+  __device__ __forceinline__ int index_of(int i) const { return idx[i]; }
   __device__ __forceinline__ float logit_of(int i) const {
-    return BIAS ? lg[i] : unord32((uint32_t)(key[i] >> 32));
+    if constexpr (BIAS) return lg[i];
+    else return unord32(key[i]);
   }
 };
 
-// The no-bias selection key: the logit's ordered image, then the complemented index (among
-// equal logits the lower index has the larger key).  NaN ranks as -inf.
-__device__ __forceinline__ uint64_t plain_key(float l, int e) {
-  const float kf = (l == l) ? l : -INFINITY;
-  return ((uint64_t)ord32(kf) << 32) | (uint32_t)(~(uint32_t)e);
-}
+// The no-bias selection key: the logit's ordered image, NaN ranking as -inf.
+__device__ __forceinline__ uint32_t plain_key(float l) { return ord32((l == l) ? l : -INFINITY); }
 
 template <int KMAX, bool BIAS>
 __device__ __forceinline__ void topk_norm(TopK<KMAX, BIAS>& st, float l) {
@@ -201,7 +193,7 @@ __device__ __forceinline__ void topk_consider(TopK<KMAX, BIAS>& st, float l, int
     }
     st.insert(ord64(kd), e, l);
   } else {
-    st.insert(plain_key(l, e), e, l);
+    st.insert(plain_key(l), e, l);
   }
 }
 
@@ -457,9 +449,9 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             // candidate's key exceeds the k-th key exactly when its logit (NaN as -inf)
             // exceeds the k-th logit, or the list still has a free slot (key 0).
             uint32_t pass = 0;
-            const uint64_t klast = st.key[KMAX - 1];
-            const bool open = klast == 0ull;
-            const float thr = unord32((uint32_t)(klast >> 32));
+            const uint32_t klast = st.key[KMAX - 1];
+            const bool open = klast == 0u;
+            const float thr = unord32(klast);
 #pragma unroll 2
             for (int qd = 0; qd < 8; ++qd) {
               const float4 f = mine[qd];
@@ -480,7 +472,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 const int p = __ffs(pass) - 1;
                 pass &= pass - 1;
                 const float l = row[p];
-                st.insert(plain_key(l, ec + p), ec + p, l);
+                st.insert(plain_key(l), ec + p, l);
               }
             }
           } else {
@@ -509,10 +501,6 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     }
   }
 
-  // converge each warp first: in the producer and MMA warps one lane ran the role's loop
-  // while the others went ahead, and the block barrier must see every warp whole, or it
-  // can let a thread through before the epilogue warps have finished reading TMEM
-  __syncwarp();
   __syncthreads();
   cluster_sync();                                           // no remote arrive after a CTA exits
   if (warp == 1) {
