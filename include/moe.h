@@ -362,6 +362,76 @@ MOE_API moe_status moe_ep_regroup(const void* src, int64_t src_rows, int32_t row
                               int64_t dst_rows, void* stream);
 
 /* ------------------------------------------------------------------------------------
+ * The expert-parallel exchange fused into the dispatch and the combine, over peer memory.
+ * [MoE-Explained] section "让 MoE 起飞" (expert parallelism); [Handbook-News]
+ * "真正难在三个环节" item 3 (the dispatch and combine all-to-all is where the time goes).
+ * Each rank holds, for every owner h (itself included), a device pointer to h's
+ * expert-major row buffer (peer_rows, device [G] array of pointers: peers' memory mapped
+ * by moe_ipc_open_handle, or this GPU's own buffer) and its capacity in rows
+ * (peer_rows_cap, device [G] int64).  The owner's rows of its experts are laid out exactly
+ * as moe_ep_plan_host's local_offsets say (expert by expert, source ranks in order inside
+ * an expert), so a source can write each of its kept rows straight to its final place:
+ *   moe_route -> moe_histogram_scan (-1) -> all-gather counts -> moe_ep_plan_host (caps,
+ *   local_offsets) and moe_ep_dst_base_host (dst_base) -> moe_histogram_scan_caps ->
+ *   moe_ep_dispatch (x rows -> owners' buffers) -> a barrier of the G ranks -> the grouped
+ *   GEMMs over the local rows (no gate) -> a barrier -> moe_ep_combine (owners' result
+ *   rows -> y, with topk_gate).
+ * This replaces moe_permute, both all-to-alls, both regroupings and moe_combine.  The
+ * barriers are the caller's (a stream-ordered collective of the process group): no kernel
+ * here waits on another GPU.  No load uses cluster multicast.
+ *
+ * moe_ep_dst_base_host -- for rank g's kept rows of expert e, their first row in the
+ *   owner's buffer: local_offsets_owner[e mod E/G] + the rows of e kept by ranks before g.
+ *   counts (host) [G][E] int32, capacity as moe_ep_plan_host; dst_base (host) [E] out.
+ *   Errors as moe_ep_plan_host.
+ *
+ * moe_ep_dispatch -- x [T, d] (bf16 or fp32, dtype) of this rank; topk_idx, row_of [T, k]
+ *   and offsets [E+1] from moe_histogram_scan_caps (row_of indexes this rank's expert-major
+ *   rows, rows_max of them; offsets are this rank's); dst_base (device) [E] int32 from
+ *   moe_ep_dst_base_host.  Stores x[t] into peer_rows[e / (E/G)] at row dst_base[e] +
+ *   (row_of[t][j] - offsets[e]) for each kept slot j of expert e = topk_idx[t][j].  A slot
+ *   whose row is not expert e's, whose expert is out of range or whose position is past
+ *   the owner's capacity records MOE_DEVERR_ROW and is skipped; a null owner pointer is
+ *   skipped.  d * element size a multiple of 16; x 16-byte aligned.
+ *   Errors: INVALID_ARG for bad sizes or dtypes, E % G != 0 or a null pointer (T > 0);
+ *   UNSUPPORTED for a row size that is not a multiple of 16 bytes or a misaligned x.
+ *
+ * moe_ep_combine -- y [T, d] (y_dtype) = sum over the kept slots j, in slot order, of
+ *   topk_gate[t][j] * (the owner's row of that slot, rows_dtype), in fp32, rounded once;
+ *   tokens with no kept slot get zeros.  The rows are found as in moe_ep_dispatch, in
+ *   peer_rows (the owners' down-GEMM outputs, ungated).  The same sum as moe_combine with
+ *   topk_gate over those rows.  Errors as moe_ep_dispatch (d a multiple of 8, y 16-byte
+ *   aligned).
+ *
+ * moe_ipc_handle_bytes -- the size of a handle (64).
+ * moe_ipc_get_handle -- the CUDA IPC handle of the allocation holding the device pointer
+ *   ptr, and ptr's offset in it (handle: host, moe_ipc_handle_bytes bytes; offset: host).
+ * moe_ipc_open_handle -- maps another process's allocation into this one (peer access
+ *   enabled): *base is the mapping, *ptr = *base + offset.  Close with moe_ipc_close(base).
+ *   A handle from this same process cannot be opened (CUDA refuses it): a rank uses its
+ *   own pointer for itself.
+ * Errors: INVALID_ARG for null pointers or a pointer CUDA does not know; UNSUPPORTED when
+ * the driver entry point is missing; CUDA for a refused mapping.
+ * ---------------------------------------------------------------------------------- */
+MOE_API moe_status moe_ep_dst_base_host(const int32_t* counts, int32_t G, int32_t g, int32_t E,
+                              int32_t capacity, int32_t* dst_base);
+MOE_API moe_status moe_ep_dispatch(const void* x, int32_t dtype, int32_t T, int32_t d, int32_t k,
+                              const int32_t* topk_idx, const int32_t* row_of,
+                              const int32_t* offsets, const int32_t* dst_base, int32_t E,
+                              int32_t G, int64_t rows_max, const void* const* peer_rows,
+                              const int64_t* peer_rows_cap, void* stream);
+MOE_API moe_status moe_ep_combine(const void* const* peer_rows, int32_t rows_dtype,
+                              const int64_t* peer_rows_cap, int32_t G, const int32_t* topk_idx,
+                              const int32_t* row_of, const float* topk_gate,
+                              const int32_t* offsets, const int32_t* dst_base, int32_t E,
+                              int32_t T, int32_t d, int32_t k, int64_t rows_max,
+                              int32_t y_dtype, void* y, void* stream);
+MOE_API int32_t moe_ipc_handle_bytes(void);
+MOE_API moe_status moe_ipc_get_handle(const void* ptr, void* handle, int64_t* offset);
+MOE_API moe_status moe_ipc_open_handle(const void* handle, int64_t offset, void** ptr, void** base);
+MOE_API moe_status moe_ipc_close(void* base);
+
+/* ------------------------------------------------------------------------------------
  * moe_scan_wait_check -- diagnostic: makes the histogram/scan's bounded wait run out.
  * (No counterpart on the pages: it tests the library's own recovery path.)
  * The look-back of moe_histogram_scan's rank kernel waits for the running totals of the

@@ -41,6 +41,18 @@ constexpr long long kMaxT = 1LL << 24;
 
 inline cudaStream_t S(void* s) { return static_cast<cudaStream_t>(s); }
 
+// cuMemGetAddressRange through the runtime's driver entry point (the allocation that holds
+// a pointer: CUDA IPC hands out whole allocations).
+typedef int (*RangeFn)(void** base, size_t* bytes, void* ptr);
+static RangeFn range_fn() {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &p, cudaEnableDefault, &q) == cudaSuccess &&
+      q == cudaDriverEntryPointSuccess)
+    return reinterpret_cast<RangeFn>(p);
+  return nullptr;
+}
+
 bool dtype_ok(int32_t dt) { return dt == MOE_BF16 || dt == MOE_F32; }
 
 moe_status check_dims(int32_t T, int32_t E, int32_t k) {
@@ -278,6 +290,84 @@ moe_status moe_ep_regroup(const void* src, int64_t src_rows, int32_t row_bytes, 
   if (!aligned16(src) || !aligned16(dst)) return MOE_ERR_UNSUPPORTED;
   return launch_ep_regroup(src, src_rows, row_bytes, reinterpret_cast<const long long*>(table), n, inverse, dst,
                            dst_rows, S(stream));
+}
+
+moe_status moe_ep_dst_base_host(const int32_t* counts, int32_t G, int32_t g, int32_t E, int32_t capacity,
+                                int32_t* dst_base) {
+  if (G < 1 || g < 0 || g >= G || E < 1 || capacity < -1) return MOE_ERR_INVALID_ARG;
+  if (E % G != 0 || E > kMaxE) return MOE_ERR_UNSUPPORTED;
+  if (!counts || !dst_base) return MOE_ERR_INVALID_ARG;
+  for (long long i = 0; i < (long long)G * E; ++i)
+    if (counts[i] < 0) return MOE_ERR_INVALID_ARG;
+  return ep_dst_base_host(counts, G, g, E, capacity, dst_base);
+}
+
+moe_status moe_ep_dispatch(const void* x, int32_t dtype, int32_t T, int32_t d, int32_t k, const int32_t* topk_idx,
+                           const int32_t* row_of, const int32_t* offsets, const int32_t* dst_base, int32_t E,
+                           int32_t G, int64_t rows_max, const void* const* peer_rows, const int64_t* peer_rows_cap,
+                           void* stream) {
+  moe_status st = check_dims(T, E, k);
+  if (st != MOE_OK) return st;
+  if (dtype != MOE_BF16 && dtype != MOE_F32) return MOE_ERR_INVALID_ARG;
+  if (G < 1 || E % G != 0 || d < 1 || rows_max < 0) return MOE_ERR_INVALID_ARG;
+  if (((long long)d * (dtype == MOE_F32 ? 4 : 2)) % 16 != 0) return MOE_ERR_UNSUPPORTED;
+  if (T == 0) return MOE_OK;
+  if (!x || !topk_idx || !row_of || !offsets || !dst_base || !peer_rows || !peer_rows_cap) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x)) return MOE_ERR_UNSUPPORTED;
+  return launch_ep_dispatch(x, dtype, T, d, k, topk_idx, row_of, offsets, dst_base, E, G, peer_rows,
+                            reinterpret_cast<const long long*>(peer_rows_cap), rows_max, S(stream));
+}
+
+moe_status moe_ep_combine(const void* const* peer_rows, int32_t rows_dtype, const int64_t* peer_rows_cap, int32_t G,
+                          const int32_t* topk_idx, const int32_t* row_of, const float* topk_gate,
+                          const int32_t* offsets, const int32_t* dst_base, int32_t E, int32_t T, int32_t d, int32_t k,
+                          int64_t rows_max, int32_t y_dtype, void* y, void* stream) {
+  moe_status st = check_dims(T, E, k);
+  if (st != MOE_OK) return st;
+  if ((rows_dtype != MOE_BF16 && rows_dtype != MOE_F32) || (y_dtype != MOE_BF16 && y_dtype != MOE_F32))
+    return MOE_ERR_INVALID_ARG;
+  if (G < 1 || E % G != 0 || d < 1 || rows_max < 0) return MOE_ERR_INVALID_ARG;
+  if (d % 8 != 0) return MOE_ERR_UNSUPPORTED;
+  if (T == 0) return MOE_OK;
+  if (!peer_rows || !peer_rows_cap || !topk_idx || !row_of || !topk_gate || !offsets || !dst_base || !y)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(y)) return MOE_ERR_UNSUPPORTED;
+  return launch_ep_combine(peer_rows, rows_dtype, reinterpret_cast<const long long*>(peer_rows_cap), G, topk_idx,
+                           row_of, topk_gate, offsets, dst_base, E, T, d, k, rows_max, y_dtype, y, S(stream));
+}
+
+int32_t moe_ipc_handle_bytes(void) { return (int32_t)sizeof(cudaIpcMemHandle_t); }
+
+moe_status moe_ipc_get_handle(const void* ptr, void* handle, int64_t* offset) {
+  if (!ptr || !handle || !offset) return MOE_ERR_INVALID_ARG;
+  void* base = nullptr;
+  size_t bytes = 0;
+  static const RangeFn range = range_fn();
+  if (!range) return MOE_ERR_UNSUPPORTED;
+  if (range(&base, &bytes, const_cast<void*>(ptr)) != 0) return MOE_ERR_INVALID_ARG;
+  cudaIpcMemHandle_t h;
+  const moe_status st = cuda_status(cudaIpcGetMemHandle(&h, base));
+  if (st != MOE_OK) return st;
+  memcpy(handle, &h, sizeof(h));
+  *offset = (int64_t)(static_cast<const char*>(ptr) - static_cast<const char*>(base));
+  return MOE_OK;
+}
+
+moe_status moe_ipc_open_handle(const void* handle, int64_t offset, void** ptr, void** base) {
+  if (!handle || !ptr || !base || offset < 0) return MOE_ERR_INVALID_ARG;
+  cudaIpcMemHandle_t h;
+  memcpy(&h, handle, sizeof(h));
+  void* b = nullptr;
+  const moe_status st = cuda_status(cudaIpcOpenMemHandle(&b, h, cudaIpcMemLazyEnablePeerAccess));
+  if (st != MOE_OK) return st;
+  *base = b;
+  *ptr = static_cast<char*>(b) + offset;
+  return MOE_OK;
+}
+
+moe_status moe_ipc_close(void* base) {
+  if (!base) return MOE_ERR_INVALID_ARG;
+  return cuda_status(cudaIpcCloseMemHandle(base));
 }
 
 moe_status moe_scan_wait_check(const int32_t* topk_idx, const float* topk_gate, int32_t T, int32_t k, int32_t E,

@@ -176,6 +176,15 @@ moe_status launch_histogram_scan_caps(const int32_t* topk_idx, const float* topk
                                       void* ws, cudaStream_t s);
 moe_status ep_plan_host(const int32_t* counts, int G, int g, int E, int capacity, int32_t* caps, int64_t* send_rows,
                         int64_t* recv_rows, int32_t* local_offsets, int64_t* regroup);
+moe_status ep_dst_base_host(const int32_t* counts, int G, int g, int E, int capacity, int32_t* dst_base);
+moe_status launch_ep_dispatch(const void* x, int dtype, int T, int d, int k, const int32_t* topk_idx,
+                              const int32_t* row_of, const int32_t* offsets, const int32_t* dst_base, int E, int G,
+                              const void* const* peer_rows, const long long* peer_cap, long long rows_max,
+                              cudaStream_t s);
+moe_status launch_ep_combine(const void* const* peer_rows, int rows_dtype, const long long* peer_cap, int G,
+                             const int32_t* topk_idx, const int32_t* row_of, const float* topk_gate,
+                             const int32_t* offsets, const int32_t* dst_base, int E, int T, int d, int k,
+                             long long rows_max, int y_dtype, void* y, cudaStream_t s);
 moe_status launch_ep_regroup(const void* src, long long src_rows, int row_bytes, const long long* table, int n,
                              int inverse, void* dst, long long dst_rows, cudaStream_t s);
 moe_status launch_scan_wait_check(const int32_t* topk_idx, const float* topk_gate, int T, int k, int E,

@@ -23,6 +23,7 @@
 #include <vector>
 
 #include "common.cuh"
+#include "row8.cuh"
 
 namespace moe {
 namespace {
@@ -53,12 +54,168 @@ regroup_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, int vec_p
   }
 }
 
+// The owner's position of this rank's kept assignment (row r of its expert-major rows, of
+// expert e): dst_base[e] + (r - offsets[e]); -1 for a dropped slot, and -1 with the error
+// word set for a row that is not expert e's, an expert out of range or a position past
+// the owner's buffer.
+__device__ __forceinline__ long long ep_dst_of(int r, int e, const int32_t* __restrict__ offsets,
+                                               const int32_t* __restrict__ dst_base, int E, int El, int G,
+                                               const long long* __restrict__ peer_cap, long long rows_max, int* h_out,
+                                               int* err) {
+  *h_out = 0;
+  if (r < 0) return -1;
+  if ((unsigned)e >= (unsigned)E || (long long)r >= rows_max) {
+    record_error(err, MOE_DEVERR_ROW);
+    return -1;
+  }
+  const int o0 = __ldg(offsets + e), o1 = __ldg(offsets + e + 1);
+  const int h = e / El;
+  if (r < o0 || r >= o1 || h >= G) {
+    record_error(err, MOE_DEVERR_ROW);
+    return -1;
+  }
+  const long long dst = (long long)__ldg(dst_base + e) + (r - o0);
+  if (dst < 0 || dst >= __ldg(peer_cap + h)) {
+    record_error(err, MOE_DEVERR_ROW);
+    return -1;
+  }
+  *h_out = h;
+  return dst;
+}
+
+// Owner h's buffer (a peer's memory through NVLink, or this GPU's own).
+template <typename P>
+__device__ __forceinline__ P* peer_base(const void* const* __restrict__ peer_rows, int h) {
+  return reinterpret_cast<P*>(__ldg(reinterpret_cast<const unsigned long long*>(peer_rows) + h));
+}
+
+// Dispatch fused with the exchange: a warp per token reads x[t] once and stores it into
+// each kept slot's owner buffer at its final expert-major position.  The permute, the
+// all-to-all and the regrouping in one pass; 16-byte vectors, UNROLL per lane in flight.
+template <int UNROLL>
+__global__ void __launch_bounds__(256)
+ep_dispatch_kernel(const uint4* __restrict__ x, int T, int nvec, int k, const int32_t* __restrict__ topk_idx,
+                   const int32_t* __restrict__ row_of, const int32_t* __restrict__ offsets,
+                   const int32_t* __restrict__ dst_base, int E, int El, const void* const* __restrict__ peer_rows,
+                   const long long* __restrict__ peer_cap, int G, long long rows_max, int* err) {
+  const unsigned lane = threadIdx.x & 31;
+  const int warps = blockDim.x >> 5;
+  const long long nw = (long long)gridDim.x * warps;
+  for (long long t = (long long)blockIdx.x * warps + (threadIdx.x >> 5); t < T; t += nw) {
+    long long my_dst = -1;
+    int my_h = 0;
+    if (lane < (unsigned)k) {
+      const int r = __ldg(row_of + t * k + lane);
+      const int e = __ldg(topk_idx + t * k + lane);
+      my_dst = ep_dst_of(r, e, offsets, dst_base, E, El, G, peer_cap, rows_max, &my_h, err);
+    }
+    const uint4* src = x + t * nvec;
+    // warp-uniform trip count: every lane reaches each shuffle below
+    for (int base = 0; base < nvec; base += 32 * UNROLL) {
+      uint4 buf[UNROLL];
+#pragma unroll
+      for (int u = 0; u < UNROLL; ++u) {
+        const int v = base + (int)lane + 32 * u;
+        if (v < nvec) buf[u] = ld_stream(src + v);
+      }
+      for (int j = 0; j < k; ++j) {
+        const long long dst = __shfl_sync(0xffffffffu, my_dst, j);
+        const int h = __shfl_sync(0xffffffffu, my_h, j);
+        if (dst < 0) continue;
+        uint4* owner = peer_base<uint4>(peer_rows, h);
+        if (!owner) continue;
+        uint4* row = owner + dst * nvec;
+#pragma unroll
+        for (int u = 0; u < UNROLL; ++u) {
+          const int v = base + (int)lane + 32 * u;
+          if (v < nvec) row[v] = buf[u];
+        }
+      }
+    }
+  }
+}
+
+// Combine fused with the exchange back: a warp per token gathers its kept slots' rows from
+// their owners' buffers (peer loads), multiplies each by its gate and adds them in slot
+// order in fp32 (as moe_combine does with gates), then rounds to the output type.  The
+// kept slots' row pointers are compacted per warp in shared memory (a ballot gives
+// positions).
+template <typename InT, typename OutT, int KMAX>
+__global__ void __launch_bounds__(256, 2)
+ep_combine_kernel(const void* const* __restrict__ peer_rows, const long long* __restrict__ peer_cap, int G,
+                  const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ row_of,
+                  const float* __restrict__ topk_gate, const int32_t* __restrict__ offsets,
+                  const int32_t* __restrict__ dst_base, int E, int El, int T, int d, int k, long long rows_max,
+                  void* __restrict__ y, int* err) {
+  constexpr int R = KMAX <= 8 ? 8 : 4;                 // kept rows per batch of loads
+  constexpr int VPI = (sizeof(InT) == 2 ? 16 : 8) / R;  // 8-element vectors per lane per batch
+  __shared__ const InT* s_ptr[8][32];
+  __shared__ float s_gate[8][32];
+  const unsigned lane = threadIdx.x & 31;
+  const int wib = threadIdx.x >> 5;
+  const int warps = blockDim.x >> 5;
+  const long long nw = (long long)gridDim.x * warps;
+  const int n8 = d >> 3;
+  const InT** kptr = s_ptr[wib];
+  float* kgate = s_gate[wib];
+  for (long long t = (long long)blockIdx.x * warps + wib; t < T; t += nw) {
+    const InT* my_ptr = nullptr;
+    float my_gate = 0.f;
+    if (lane < (unsigned)k) {
+      const int r = __ldg(row_of + t * k + lane);
+      const int e = __ldg(topk_idx + t * k + lane);
+      int h = 0;
+      const long long dst = ep_dst_of(r, e, offsets, dst_base, E, El, G, peer_cap, rows_max, &h, err);
+      const InT* owner = dst >= 0 ? peer_base<const InT>(peer_rows, h) : nullptr;
+      if (owner) {
+        my_ptr = owner + dst * d;
+        my_gate = __ldg(topk_gate + t * k + lane);
+      }
+    }
+    const unsigned kept = __ballot_sync(0xffffffffu, my_ptr != nullptr);
+    const int nk = __popc(kept);
+    __syncwarp();                                       // the previous token's list is read
+    if (my_ptr) {
+      const int pos = __popc(kept & ((1u << lane) - 1u));
+      kptr[pos] = my_ptr;
+      kgate[pos] = my_gate;
+    }
+    __syncwarp();
+    for (int v0 = lane; v0 < n8; v0 += 32 * VPI) {
+      float acc[VPI][8];
+#pragma unroll
+      for (int u = 0; u < VPI; ++u)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[u][i] = 0.f;
+#pragma unroll 1
+      for (int j0 = 0; j0 < KMAX; j0 += R) {
+        if (j0 >= nk) break;
+        Row8<InT> buf[VPI][R];
+#pragma unroll
+        for (int jj = 0; jj < R; ++jj)
+#pragma unroll
+          for (int u = 0; u < VPI; ++u)
+            if (j0 + jj < nk && v0 + 32 * u < n8) buf[u][jj].load(kptr[j0 + jj], (long long)(v0 + 32 * u) * 8);
+#pragma unroll
+        for (int jj = 0; jj < R; ++jj)
+#pragma unroll
+          for (int u = 0; u < VPI; ++u)
+            if (j0 + jj < nk && v0 + 32 * u < n8) buf[u][jj].add(acc[u], kgate[j0 + jj], true);
+      }
+#pragma unroll
+      for (int u = 0; u < VPI; ++u) {
+        const int v = v0 + 32 * u;
+        if (v < n8) store8<OutT>(y, t * d + v * 8, acc[u]);
+      }
+    }
+  }
+}
+
 }  // namespace
 
-moe_status ep_plan_host(const int32_t* counts, int G, int g, int E, int capacity, int32_t* caps, int64_t* send_rows,
-                        int64_t* recv_rows, int32_t* local_offsets, int64_t* regroup) {
-  const int El = E / G;
-  // kept[s][e] in token order across the ranks
+// kept[s][e]: rank s's assignments to expert e that survive the capacity, the global token
+// order being rank 0's tokens, then rank 1's, ...
+static std::vector<int64_t> kept_matrix(const int32_t* counts, int G, int E, int capacity) {
   std::vector<int64_t> kept((size_t)G * E);
   for (int e = 0; e < E; ++e) {
     int64_t base = 0;
@@ -74,6 +231,13 @@ moe_status ep_plan_host(const int32_t* counts, int G, int g, int E, int capacity
       base += c;
     }
   }
+  return kept;
+}
+
+moe_status ep_plan_host(const int32_t* counts, int G, int g, int E, int capacity, int32_t* caps, int64_t* send_rows,
+                        int64_t* recv_rows, int32_t* local_offsets, int64_t* regroup) {
+  const int El = E / G;
+  const std::vector<int64_t> kept = kept_matrix(counts, G, E, capacity);
   for (int e = 0; e < E; ++e) caps[e] = (int32_t)kept[(size_t)g * E + e];
   for (int h = 0; h < G; ++h) {
     int64_t snd = 0, rcv = 0;
@@ -110,6 +274,25 @@ moe_status ep_plan_host(const int32_t* counts, int G, int g, int E, int capacity
   return MOE_OK;
 }
 
+// For rank g's rows of expert e (kept, in token order), their first position in the owner's
+// expert-major buffer: the owner's offset of e among its experts plus the rows of e that
+// earlier ranks keep.
+moe_status ep_dst_base_host(const int32_t* counts, int G, int g, int E, int capacity, int32_t* dst_base) {
+  const int El = E / G;
+  const std::vector<int64_t> kept = kept_matrix(counts, G, E, capacity);
+  for (int h = 0; h < G; ++h) {
+    int64_t loc = 0;                                   // owner h's rows before its expert j
+    for (int j = 0; j < El; ++j) {
+      const int e = h * El + j;
+      int64_t before = 0;
+      for (int s = 0; s < g; ++s) before += kept[(size_t)s * E + e];
+      dst_base[e] = (int32_t)(loc + before);
+      for (int s = 0; s < G; ++s) loc += kept[(size_t)s * E + e];
+    }
+  }
+  return MOE_OK;
+}
+
 moe_status launch_ep_regroup(const void* src, long long src_rows, int row_bytes, const long long* table, int n,
                              int inverse, void* dst, long long dst_rows, cudaStream_t s) {
   if (n == 0) return MOE_OK;
@@ -119,6 +302,61 @@ moe_status launch_ep_regroup(const void* src, long long src_rows, int row_bytes,
   regroup_kernel<<<blocks, 256, 0, s>>>(static_cast<const uint4*>(src), static_cast<uint4*>(dst), row_bytes / 16,
                                         table, n, inverse, src_rows, dst_rows, err_ptr());
   return check_launch();
+}
+
+
+moe_status launch_ep_dispatch(const void* x, int dtype, int T, int d, int k, const int32_t* topk_idx,
+                              const int32_t* row_of, const int32_t* offsets, const int32_t* dst_base, int E, int G,
+                              const void* const* peer_rows, const long long* peer_cap, long long rows_max,
+                              cudaStream_t s) {
+  if (T == 0) return MOE_OK;
+  const int esz = dtype == MOE_F32 ? 4 : 2;
+  const int nvec = d * esz / 16;
+  long long blocks = ((long long)T + 7) / 8;
+  const long long cap = (long long)num_sms() * 8;
+  if (blocks > cap) blocks = cap;
+  ep_dispatch_kernel<4><<<(unsigned)blocks, 256, 0, s>>>(static_cast<const uint4*>(x), T, nvec, k, topk_idx, row_of,
+                                                          offsets, dst_base, E, E / G, peer_rows, peer_cap, G,
+                                                          rows_max, err_ptr());
+  return check_launch();
+}
+
+template <typename InT, typename OutT>
+static moe_status ep_combine_k(const void* const* peer_rows, const long long* peer_cap, int G, const int32_t* topk_idx,
+                               const int32_t* row_of, const float* topk_gate, const int32_t* offsets,
+                               const int32_t* dst_base, int E, int T, int d, int k, long long rows_max, void* y,
+                               cudaStream_t s) {
+  long long blocks = ((long long)T + 7) / 8;
+  const long long cap = (long long)num_sms() * 8;
+  if (blocks > cap) blocks = cap;
+#define MOE_EPC(KM)                                                                                                 \
+  ep_combine_kernel<InT, OutT, KM><<<(unsigned)blocks, 256, 0, s>>>(peer_rows, peer_cap, G, topk_idx, row_of,    \
+                                                                     topk_gate, offsets, dst_base, E, E / G, T, d, \
+                                                                     k, rows_max, y, err_ptr())
+  if (k <= 8) MOE_EPC(8);
+  else if (k <= 16) MOE_EPC(16);
+  else MOE_EPC(32);
+#undef MOE_EPC
+  return check_launch();
+}
+
+moe_status launch_ep_combine(const void* const* peer_rows, int rows_dtype, const long long* peer_cap, int G,
+                             const int32_t* topk_idx, const int32_t* row_of, const float* topk_gate,
+                             const int32_t* offsets, const int32_t* dst_base, int E, int T, int d, int k,
+                             long long rows_max, int y_dtype, void* y, cudaStream_t s) {
+  if (T == 0) return MOE_OK;
+  const bool in32 = rows_dtype == MOE_F32, out32 = y_dtype == MOE_F32;
+  if (in32 && out32)
+    return ep_combine_k<float, float>(peer_rows, peer_cap, G, topk_idx, row_of, topk_gate, offsets, dst_base, E, T, d,
+                                      k, rows_max, y, s);
+  if (in32)
+    return ep_combine_k<float, __nv_bfloat16>(peer_rows, peer_cap, G, topk_idx, row_of, topk_gate, offsets, dst_base,
+                                              E, T, d, k, rows_max, y, s);
+  if (out32)
+    return ep_combine_k<__nv_bfloat16, float>(peer_rows, peer_cap, G, topk_idx, row_of, topk_gate, offsets, dst_base,
+                                              E, T, d, k, rows_max, y, s);
+  return ep_combine_k<__nv_bfloat16, __nv_bfloat16>(peer_rows, peer_cap, G, topk_idx, row_of, topk_gate, offsets,
+                                                    dst_base, E, T, d, k, rows_max, y, s);
 }
 
 }  // namespace moe

@@ -17,11 +17,18 @@ the result equals the single-GPU layer run on the concatenated batch.  One forwa
         expert-major)  ->  grouped gate/up + down GEMMs of the local experts (no gate)
     ->  regroup back  ->  all-to-all back  ->  combine with the gates.
 
-The exchange is torch.distributed's all_to_all_single (NCCL between GPUs); the split
-sizes need the plan on the host, so one small device-to-host copy of the counts happens
-per forward.  Every compute step is a library kernel (LibraryKernels); the steps are
-grouped behind one small interface so that the orchestration and the exchange can also
-be driven by other implementations of the same steps.
+Two exchanges:
+- exchange="nccl": torch.distributed's all_to_all_single between the steps above;
+- exchange="peer": every rank maps the other ranks' row buffers (CUDA IPC, one node) and
+  moe_ep_dispatch stores each kept token row straight into its owner's buffer at its final
+  expert-major place (the permute, the all-to-all and the regrouping in one kernel);
+  after the local GEMMs moe_ep_combine reads the result rows back from the owners and adds
+  them with the gates (the exchange back, the regrouping and the combine in one kernel).
+  Two stream-ordered collectives of one element separate the writers from the readers.
+Either way the split sizes need the plan on the host, so one small device-to-host copy of
+the counts happens per forward.  Every compute step is a library kernel (LibraryKernels);
+the steps are grouped behind one small interface so that the orchestration and the
+exchange can also be driven by other implementations of the same steps.
 """
 from __future__ import annotations
 
@@ -98,14 +105,24 @@ class LibraryKernels:
                 dst.shape[0], M._stream(None)))
         return dst
 
-    def ffn(self, x_local, offsets_local, rows):
+    def ffn(self, x_local, offsets_local, rows, out=None):
         L = self.L
         offs = torch.from_numpy(offsets_local).to(x_local.device)
         h = M.moe_expert_gate_up(x_local, offs, L.W_gu, rows)
-        return M.moe_expert_down(h, offs, L.W_dn, rows, None, y_dtype=L.rows_dtype)
+        return M.moe_expert_down(h, offs, L.W_dn, rows, None, y_rows=out, y_dtype=L.rows_dtype)
 
     def combine(self, y_rows, row_of, topk_gate, T):
         return M.moe_combine(y_rows, row_of, T, y_rows.shape[0], topk_gate=topk_gate, y_dtype=self.L.out_dtype)
+
+    def dispatch_peer(self, x, sc, dst_base, rows_max):
+        L = self.L
+        M.moe_ep_dispatch(x, sc["topk_idx"], sc["row_of"], sc["offsets"], dst_base, L.E, L.G, rows_max, L.peer_x,
+                          L.peer_cap)
+
+    def combine_peer(self, sc, topk_gate, dst_base, rows_max):
+        L = self.L
+        return M.moe_ep_combine(L.peer_y, L.rows_dtype, L.peer_cap, sc["topk_idx"], sc["row_of"], topk_gate,
+                                sc["offsets"], dst_base, L.E, L.G, L.d, rows_max, y_dtype=L.out_dtype)
 
 
 class ExpertParallelMoE:
@@ -118,7 +135,8 @@ class ExpertParallelMoE:
 
     def __init__(self, Wg, W_gu, W_dn, k: int, score: str = "softmax", renormalize: bool = True,
                  scale: float = 1.0, capacity: int = -1, logit_offset=None, select_bias=None, group=None,
-                 rows_dtype=torch.float32, out_dtype=torch.float32, kernels=None):
+                 rows_dtype=torch.float32, out_dtype=torch.float32, kernels=None, exchange: str = "nccl",
+                 max_tokens: int = 0):
         self.group = group
         ready = dist.is_available() and dist.is_initialized()
         self.G = dist.get_world_size(group) if ready else 1
@@ -136,6 +154,56 @@ class ExpertParallelMoE:
         self.kernels = kernels if kernels is not None else LibraryKernels(self)
         self.Wg_split = M.moe_prepare_router_weight(Wg) if (kernels is None and Wg.is_cuda) else None
         self.last_plan: Optional[dict] = None
+        if exchange not in ("nccl", "peer"):
+            raise ValueError(f"exchange must be 'nccl' or 'peer', got {exchange!r}")
+        self.exchange = exchange
+        self._mapped = []
+        if exchange == "peer":
+            self._map_peers(max_tokens)
+
+    # the peer buffers ----------------------------------------------------------------
+    def _map_peers(self, max_tokens: int):
+        """Allocates this rank's expert-major row buffers (room for every rank's kept rows of
+        its experts) and maps every other rank's (CUDA IPC; the ranks share one node)."""
+        if max_tokens < 1:
+            raise ValueError("exchange='peer' needs max_tokens (the largest per-rank batch)")
+        dev = self.Wg.device
+        cap = self.G * max_tokens * self.k
+        if self.capacity >= 0:
+            cap = min(cap, self.El * self.capacity)
+        cap = max(cap, 1)
+        self.x_local = torch.empty((cap, self.d), dtype=self.W_gu.dtype, device=dev)
+        self.y_local = torch.empty((cap, self.d), dtype=self.rows_dtype, device=dev)
+        addr_x, addr_y = [0] * self.G, [0] * self.G
+        if self.G == 1:
+            addr_x[0], addr_y[0] = self.x_local.data_ptr(), self.y_local.data_ptr()
+        else:
+            mine = (M.ipc_handle(self.x_local), M.ipc_handle(self.y_local))
+            every = [None] * self.G
+            dist.all_gather_object(every, mine, group=self.group)
+            for h in range(self.G):
+                if h == self.g:
+                    addr_x[h], addr_y[h] = self.x_local.data_ptr(), self.y_local.data_ptr()
+                    continue
+                (hx, ox), (hy, oy) = every[h]
+                addr_x[h], bx = M.ipc_open(hx, ox)
+                addr_y[h], by = M.ipc_open(hy, oy)
+                self._mapped += [bx, by]
+        self.peer_x = torch.tensor(addr_x, dtype=torch.int64, device=dev)
+        self.peer_y = torch.tensor(addr_y, dtype=torch.int64, device=dev)
+        self.peer_cap = torch.full((self.G,), cap, dtype=torch.int64, device=dev)
+        self._flag = torch.zeros(1, dtype=torch.float32, device=dev)
+
+    def close(self):
+        """Unmaps the other ranks' buffers (exchange='peer')."""
+        for b in self._mapped:
+            M.ipc_close(b)
+        self._mapped = []
+
+    def _barrier(self):
+        # stream-ordered: the next kernels on this rank start after every rank's earlier ones
+        if self.G > 1:
+            dist.all_reduce(self._flag, group=self.group)
 
     # the exchange ------------------------------------------------------------------
     def _all_gather_counts(self, counts):
@@ -158,6 +226,8 @@ class ExpertParallelMoE:
 
     # the forward ---------------------------------------------------------------------
     def forward(self, x):
+        if self.exchange == "peer":
+            return self._forward_peer(x)
         kn = self.kernels
         T = x.shape[0]
         logits, topk_idx, topk_gate = kn.route(x)
@@ -177,3 +247,28 @@ class ExpertParallelMoE:
         assert y_rows.shape[0] == n_send
         self.routing = {"logits": logits, "topk_idx": topk_idx, "topk_gate": topk_gate, **sc}
         return kn.combine(y_rows, sc["row_of"], topk_gate, T)
+
+    def _forward_peer(self, x):
+        kn = self.kernels
+        T = x.shape[0]
+        logits, topk_idx, topk_gate = kn.route(x)
+        counts = kn.counts(topk_idx)
+        allc = self._all_gather_counts(counts).cpu().numpy()        # the one device-to-host copy
+        plan = ep_plan(allc, self.g, self.capacity)
+        self.last_plan = plan
+        dst_base = torch.from_numpy(M.ep_dst_base(allc, self.g, self.capacity)).to(x.device)
+        sc = kn.scan(topk_idx, topk_gate, plan["caps"])
+        sc["topk_idx"] = topk_idx
+        n_local = int(plan["local_offsets"][-1])
+        if n_local > self.x_local.shape[0]:
+            raise RuntimeError("the exchange plan exceeds the peer buffers (max_tokens too small)")
+        rows_max = T * self.k
+        kn.dispatch_peer(x, sc, dst_base, rows_max)
+        self._barrier()                                               # every row has reached its owner
+        if n_local:
+            kn.ffn(self.x_local[:n_local], plan["local_offsets"], n_local, out=self.y_local[:n_local])
+        self._barrier()                                               # every owner's rows are ready
+        self.routing = {"logits": logits, "topk_idx": topk_idx, "topk_gate": topk_gate, **sc}
+        y = kn.combine_peer(sc, topk_gate, dst_base, rows_max)
+        self._barrier()                                               # no owner reuses its rows before all have read
+        return y

@@ -63,6 +63,15 @@ _SIGNATURES = {
     "moe_ep_plan_host": (_i32, [_c_void_p, _i32, _i32, _i32, _i32, _c_void_p, _c_void_p, _c_void_p, _c_void_p,
                                 _c_void_p]),
     "moe_ep_regroup": (_i32, [_c_void_p, _i64, _i32, _c_void_p, _i32, _i32, _c_void_p, _i64, _c_void_p]),
+    "moe_ep_dst_base_host": (_i32, [_c_void_p, _i32, _i32, _i32, _i32, _c_void_p]),
+    "moe_ep_dispatch": (_i32, [_c_void_p, _i32, _i32, _i32, _i32, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _i32,
+                               _i32, _i64, _c_void_p, _c_void_p, _c_void_p]),
+    "moe_ep_combine": (_i32, [_c_void_p, _i32, _c_void_p, _i32, _c_void_p, _c_void_p, _c_void_p, _c_void_p,
+                              _c_void_p, _i32, _i32, _i32, _i32, _i64, _i32, _c_void_p, _c_void_p]),
+    "moe_ipc_handle_bytes": (_i32, []),
+    "moe_ipc_get_handle": (_i32, [_c_void_p, _c_void_p, ctypes.POINTER(_i64)]),
+    "moe_ipc_open_handle": (_i32, [_c_void_p, _i64, ctypes.POINTER(_c_void_p), ctypes.POINTER(_c_void_p)]),
+    "moe_ipc_close": (_i32, [_c_void_p]),
     "moe_permute": (_i32, [_c_void_p, _i32, _i32, _i32, _i32, _c_void_p, _i64, _c_void_p, _c_void_p]),
     "moe_expert_gate_up": (_i32, [_c_void_p, _i32, _c_void_p, _i32, _i32, _i32, _i64, _c_void_p, _c_void_p,
                                   _c_void_p]),
@@ -655,3 +664,76 @@ def moe_get_device_error(stream=None) -> int:
     if st not in (MOE_OK, MOE_ERR_DEVICE):
         raise MoEError("moe_get_device_error", st)
     return int(code.value)
+
+
+# ---------------------------------------------------------------- expert-parallel exchange over peer memory
+def moe_ep_dispatch(x, topk_idx, row_of, offsets, dst_base, E: int, G: int, rows_max: int, peer_rows, peer_rows_cap,
+                    stream=None):
+    """Stores this rank's kept token rows into their owners' expert-major buffers.
+    peer_rows: device int64 [G] (buffer addresses), peer_rows_cap: device int64 [G] (rows)."""
+    T, d = x.shape
+    k = topk_idx.shape[1]
+    _need(x, "x")
+    _need(topk_idx, "topk_idx", torch.int32, (T, k))
+    _need(row_of, "row_of", torch.int32, (T, k))
+    _need(offsets, "offsets", torch.int32, (E + 1,))
+    _need(dst_base, "dst_base", torch.int32, (E,))
+    _need(peer_rows, "peer_rows", torch.int64, (G,))
+    _need(peer_rows_cap, "peer_rows_cap", torch.int64, (G,))
+    _check("moe_ep_dispatch", lib().moe_ep_dispatch(_p(x), _dt(x), T, d, k, _p(topk_idx), _p(row_of), _p(offsets),
+                                                    _p(dst_base), E, G, int(rows_max), _p(peer_rows),
+                                                    _p(peer_rows_cap), _stream(stream)))
+
+
+def moe_ep_combine(peer_rows, rows_dtype, peer_rows_cap, topk_idx, row_of, topk_gate, offsets, dst_base, E: int,
+                   G: int, d: int, rows_max: int, y=None, y_dtype=torch.float32, stream=None):
+    """y [T, d] = the gated sum of each token's kept rows, read from their owners' buffers."""
+    T, k = topk_idx.shape
+    dev = topk_idx.device
+    if y is None:
+        y = torch.empty((T, d), dtype=y_dtype, device=dev)
+    _need(y, "y", None, (T, d))
+    _need(topk_idx, "topk_idx", torch.int32, (T, k))
+    _need(row_of, "row_of", torch.int32, (T, k))
+    _need(topk_gate, "topk_gate", torch.float32, (T, k))
+    _need(offsets, "offsets", torch.int32, (E + 1,))
+    _need(dst_base, "dst_base", torch.int32, (E,))
+    _need(peer_rows, "peer_rows", torch.int64, (G,))
+    _need(peer_rows_cap, "peer_rows_cap", torch.int64, (G,))
+    _check("moe_ep_combine", lib().moe_ep_combine(_p(peer_rows), DTYPE[rows_dtype], _p(peer_rows_cap), G,
+                                                  _p(topk_idx), _p(row_of), _p(topk_gate), _p(offsets),
+                                                  _p(dst_base), E, T, d, k, int(rows_max), _dt(y), _p(y),
+                                                  _stream(stream)))
+    return y
+
+
+def ep_dst_base(counts, g: int, capacity: int):
+    """moe_ep_dst_base_host for rank g: counts [G, E] int32 (every rank's per-expert counts)."""
+    import numpy as np
+    counts = np.ascontiguousarray(counts, np.int32)
+    G, E = counts.shape
+    out = np.empty(E, np.int32)
+    _check("moe_ep_dst_base_host", lib().moe_ep_dst_base_host(ctypes.c_void_p(counts.ctypes.data), G, g, E,
+                                                              int(capacity), ctypes.c_void_p(out.ctypes.data)))
+    return out
+
+
+def ipc_handle(t: torch.Tensor):
+    """(handle bytes, offset) of the CUDA allocation holding tensor t, for another process."""
+    n = int(lib().moe_ipc_handle_bytes())
+    buf = ctypes.create_string_buffer(n)
+    off = _i64(0)
+    _check("moe_ipc_get_handle", lib().moe_ipc_get_handle(_p(t), buf, ctypes.byref(off)))
+    return buf.raw, int(off.value)
+
+
+def ipc_open(handle: bytes, offset: int):
+    """Maps another process's allocation: (address, base to pass to ipc_close)."""
+    ptr, base = _c_void_p(), _c_void_p()
+    _check("moe_ipc_open_handle", lib().moe_ipc_open_handle(handle, int(offset), ctypes.byref(ptr),
+                                                            ctypes.byref(base)))
+    return int(ptr.value), int(base.value)
+
+
+def ipc_close(base: int):
+    _check("moe_ipc_close", lib().moe_ipc_close(_c_void_p(base)))

@@ -356,3 +356,27 @@ def test_fp4_scale_preparation_size_and_validation(L):
     assert f(FAKE, 512, 96, 0, FAKE, nb, NUL) == 2
     assert f(FAKE, 512, 128, 0, FAKE, nb - 1, NUL) == 3
     assert f(FAKE, 512, 128, 0, ctypes.c_void_p(4100), nb, NUL) == 2
+
+
+def test_fused_exchange_host_validation(L):
+    """moe_ep_dispatch / moe_ep_combine / moe_ipc_*: every check before any launch or CUDA call."""
+    import ctypes
+    v = ctypes.c_void_p(16)                                           # never dereferenced: rejected first
+    d = L.moe_ep_dispatch
+    assert d(v, 0, 0, 64, 2, v, v, v, v, 8, 2, 0, v, v, None) == 0                 # T = 0: nothing to do
+    assert d(None, 0, 4, 64, 2, v, v, v, v, 8, 2, 8, v, v, None) == 1              # null x
+    assert d(v, 0, 4, 64, 2, v, v, v, v, 8, 3, 8, v, v, None) == 1                 # E % G != 0
+    assert d(v, 2, 4, 64, 2, v, v, v, v, 8, 2, 8, v, v, None) == 1                 # bad dtype
+    assert d(v, 0, 4, 12, 2, v, v, v, v, 8, 2, 8, v, v, None) == 2                 # 24-byte rows
+    assert d(v, 0, 4, 64, 2, v, v, v, v, 8, 2, 8, None, v, None) == 1              # no owner pointers
+    c = L.moe_ep_combine
+    assert c(v, 1, v, 2, v, v, v, v, v, 8, 0, 64, 2, 0, 1, v, None) == 0          # T = 0
+    assert c(None, 1, v, 2, v, v, v, v, v, 8, 4, 64, 2, 8, 1, v, None) == 1       # null owner pointers
+    assert c(v, 1, v, 2, v, v, None, v, v, 8, 4, 64, 2, 8, 1, v, None) == 1       # no gates
+    assert c(v, 1, v, 2, v, v, v, v, v, 8, 4, 60, 2, 8, 1, v, None) == 2          # d % 8
+    assert L.moe_ipc_handle_bytes() == 64
+    off = ctypes.c_int64(0)
+    assert L.moe_ipc_get_handle(None, ctypes.create_string_buffer(64), ctypes.byref(off)) == 1
+    p, b = ctypes.c_void_p(), ctypes.c_void_p()
+    assert L.moe_ipc_open_handle(None, 0, ctypes.byref(p), ctypes.byref(b)) == 1
+    assert L.moe_ipc_close(None) == 1

@@ -186,3 +186,36 @@ def test_plan_host_validation():
         ep_plan(-np.ones((2, 8), np.int32), 0, -1)                  # negative counts
     with pytest.raises(M.MoEError):
         ep_plan(np.zeros((2, 8), np.int32), 2, -1)                  # rank out of range
+
+
+def test_dst_base_puts_each_rank_where_the_owner_expects_it():
+    """moe_ep_dst_base_host: rank g's q-th kept row of expert e lands at dst_base[e] + q in
+    the owner's expert-major rows, the row the owner's regroup table gives it."""
+    sys.path.insert(0, ROOT)
+    from routing_dispatch_expert_moe_b200 import moe as M
+    from routing_dispatch_expert_moe_b200.ep import ep_plan
+    rng = np.random.default_rng(9)
+    for G, E, cap in ((2, 8, 5), (4, 16, 3), (3, 9, -1), (1, 4, 2), (4, 8, 0)):
+        counts = rng.integers(0, 9, size=(G, E)).astype(np.int32)
+        El = E // G
+        plans = [ep_plan(counts, h, cap) for h in range(G)]
+        for g in range(G):
+            base = M.ep_dst_base(counts, g, cap)
+            kept_g = plans[g]["caps"]
+            for e in range(E):
+                h, j = e // El, e % El
+                a, b, n = (int(v) for v in plans[h]["regroup"][g * El + j])
+                assert n == kept_g[e]
+                assert base[e] == b, (G, E, cap, g, e)
+                assert 0 <= base[e] and base[e] + n <= plans[h]["local_offsets"][-1]
+
+
+def test_dst_base_host_validation():
+    sys.path.insert(0, ROOT)
+    from routing_dispatch_expert_moe_b200 import moe as M
+    with pytest.raises(M.MoEError):
+        M.ep_dst_base(np.zeros((2, 7), np.int32), 0, -1)             # E % G != 0
+    with pytest.raises(M.MoEError):
+        M.ep_dst_base(-np.ones((2, 8), np.int32), 0, -1)             # negative counts
+    with pytest.raises(M.MoEError):
+        M.ep_dst_base(np.zeros((2, 8), np.int32), 2, -1)             # rank out of range

@@ -63,3 +63,23 @@ def test_expert_parallel_one_rank_matches_the_oracle(group, cfg):
     n = int(o["offsets"][-1])
     yp = O.grouped_ffn(O.permute(host["x"], o["row_of"], n), o["offsets"], gu, dn, o["gate_of_row"], True)
     U.assert_y_close(y.float().cpu().numpy().astype(np.float64), O.combine(yp, o["row_of"]), "y (expert-parallel)")
+
+
+@pytest.mark.parametrize("cfg", CASES, ids=lambda c: c.name)
+def test_peer_exchange_one_rank_equals_the_nccl_exchange(group, cfg):
+    """exchange='peer' (moe_ep_dispatch / moe_ep_combine into the owners' buffers) against
+    exchange='nccl' on the same inputs: the same rows through the same GEMMs and the same
+    fp32 sums, so y agrees bit for bit."""
+    from routing_dispatch_expert_moe_b200 import moe as M
+    from routing_dispatch_expert_moe_b200.ep import ExpertParallelMoE
+    host, dev = U.make_inputs(cfg)
+    cap = O.capacity(cfg.T, cfg.E, cfg.k, cfg.capacity_factor, True)
+    args = (dev["Wg"], dev["W_gu"], dev["W_dn"], cfg.k, cfg.score, cfg.renormalize, cfg.scale, cap, dev["off"])
+    y_n = ExpertParallelMoE(*args, group=group).forward(dev["x"])
+    lay = ExpertParallelMoE(*args, group=group, exchange="peer", max_tokens=cfg.T)
+    y_p = lay.forward(dev["x"])
+    y_p2 = lay.forward(dev["x"])                                   # the buffers are reused
+    torch.cuda.synchronize()
+    assert M.moe_get_device_error() == 0
+    assert torch.equal(y_n, y_p) and torch.equal(y_p, y_p2)
+    lay.close()
