@@ -68,7 +68,6 @@ struct L {
 };
 constexpr size_t kSmemBytes = L::end + 1024;                 // + alignment slack
 constexpr long long kPrefetchMax = 512 * 1024;               // largest weight slab the down GEMM prefetches
-constexpr int kRowBox = 16;                                  // rows per A box when loading only a group's rows
 
 // Output column tiles per row tile: 128 H features per gate/up tile (128 gate + 128 up
 // accumulator columns), 256 outputs per down tile.
@@ -278,7 +277,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
                        long long rows_max, const float* __restrict__ gate_of_row,
                        OutT* __restrict__ out, const int32_t* __restrict__ token_of_row, int n_tokens,
                        const __nv_bfloat16* __restrict__ a_gather, int* err,
-                       const __nv_bfloat16* __restrict__ b_raw = nullptr, int a_box = BM) {
+                       const __nv_bfloat16* __restrict__ b_raw = nullptr) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
@@ -354,14 +353,10 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1u, abort_flag, err)) { ok = false; break; }
           const uint32_t full = bar_full + 8 * stage;
-          // a_box < BM: only the group's rows, in boxes of a_box rows (the MMA still spans
-          // BM rows; the rows past the group are stale and never stored)
-          const int a_rows = a_box < BM ? min(BM, (tc.rows + a_box - 1) / a_box * a_box) : BM;
-          mbar_expect_tx(full, (uint32_t)(a_rows * BK * 2) + B_STAGE);
+          mbar_expect_tx(full, A_STAGE + B_STAGE);
           const uint32_t a_dst = sb + L::a + stage * A_STAGE;
           const uint32_t b_dst = sb + L::b + stage * B_STAGE;
-          for (int r = 0; r < a_rows; r += a_box) tma_load_2d(a_dst + (uint32_t)(r * BK * 2), &tmA, full, kb * BK,
-                                                              tc.row0 + r);
+          tma_load_2d(a_dst, &tmA, full, kb * BK, tc.row0);
           if (MODE == 0) {
             const int g_row = tc.e * 2 * F + tc.n_tile * 128;
             tma_load_2d(b_dst, &tmB, full, kb * BK, g_row);
@@ -648,7 +643,7 @@ template <int MODE, typename OutT>
 moe_status launch_tc(const CUtensorMap& ma, const CUtensorMap& mb, const int32_t* offsets, int E, int K, int N_out,
                      int F, long long rows_max, const float* gate_of_row, void* out, cudaStream_t s,
                      const int32_t* token_of_row = nullptr, int n_tokens = 0,
-                     const __nv_bfloat16* a_gather = nullptr, const void* b_raw = nullptr, int a_box = BM) {
+                     const __nv_bfloat16* a_gather = nullptr, const void* b_raw = nullptr) {
   static std::atomic<int> configured[kMaxDevices];
   const moe_status st = ensure_smem_limit(configured, grouped_gemm_tc_kernel<MODE, OutT>, kSmemBytes);
   if (st != MOE_OK) return st;
@@ -659,7 +654,7 @@ moe_status launch_tc(const CUtensorMap& ma, const CUtensorMap& mb, const int32_t
   if (grid < 1) grid = 1;
   grouped_gemm_tc_kernel<MODE, OutT><<<grid, kThreadsTC, kSmemBytes, s>>>(
       ma, mb, offsets, E, K, N_out, F, rows_max, gate_of_row, static_cast<OutT*>(out), token_of_row, n_tokens,
-      a_gather, err_ptr(), static_cast<const __nv_bfloat16*>(b_raw), a_box);
+      a_gather, err_ptr(), static_cast<const __nv_bfloat16*>(b_raw));
   return check_launch();
 }
 
@@ -758,8 +753,7 @@ moe_status launch_down_tc(const void* h, const int32_t* offsets, int E, int d, i
   }
   const bool pair = use_pairs(rows_max, E);
   CUtensorMap ma, mb;
-  // single-CTA tiles (small groups) load only each group's H rows, 16 at a time
-  if (!make_map(&ma, h, (unsigned long long)rows_max, F, pair ? BM : kRowBox)) return MOE_ERR_UNSUPPORTED;
+  if (!make_map(&ma, h, (unsigned long long)rows_max, F, BM)) return MOE_ERR_UNSUPPORTED;
   if (!make_map(&mb, W_dn, (unsigned long long)E * d, F, pair ? BM : BN)) return MOE_ERR_UNSUPPORTED;
   if (pair) {
     if (F <= kWideMaxK) {
@@ -773,9 +767,9 @@ moe_status launch_down_tc(const void* h, const int32_t* offsets, int E, int d, i
   }
   if (y_dtype == MOE_F32)
     return launch_tc<1, float>(ma, mb, offsets, E, F, d, F, rows_max, gate_of_row, y_rows, s, nullptr, 0, nullptr,
-                               W_dn, kRowBox);
+                               W_dn);
   return launch_tc<1, __nv_bfloat16>(ma, mb, offsets, E, F, d, F, rows_max, gate_of_row, y_rows, s, nullptr, 0,
-                                     nullptr, W_dn, kRowBox);
+                                     nullptr, W_dn);
 }
 
 // Down GEMM with the combine fused into its epilogue: y[token_of_row[r]] += gate_of_row[r] *
