@@ -67,7 +67,6 @@ struct L {
   static constexpr int end = stage + 4 * 32 * (32 * 4 + 16);
 };
 constexpr size_t kSmemBytes = L::end + 1024;                 // + alignment slack
-constexpr long long kPrefetchMax = 512 * 1024;               // largest weight slab the down GEMM prefetches
 
 // Output column tiles per row tile: 128 H features per gate/up tile (128 gate + 128 up
 // accumulator columns), 256 outputs per down tile.
@@ -276,8 +275,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
                        const int32_t* __restrict__ offsets, int E, int K, int N_out, int F,
                        long long rows_max, const float* __restrict__ gate_of_row,
                        OutT* __restrict__ out, const int32_t* __restrict__ token_of_row, int n_tokens,
-                       const __nv_bfloat16* __restrict__ a_gather, int* err,
-                       const __nv_bfloat16* __restrict__ b_raw = nullptr) {
+                       const __nv_bfloat16* __restrict__ a_gather, int* err) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
@@ -338,18 +336,6 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
         const TileCoord tc = tile_coord(tile_start, offsets, E, BM, tile);
-        if (MODE == 1 && b_raw) {
-          // down (a few k-blocks per tile): ask L2 for the next tile's weight slab, one
-          // contiguous stream, while this tile's box loads run
-          const int nt = tile + (int)gridDim.x;
-          if (nt < total) {
-            const TileCoord tn = tile_coord(tile_start, offsets, E, BM, nt);
-            const int r0 = tn.n_tile * BN, rows = min(BN, N_out - r0);
-            const long long bytes = (long long)rows * K * 2;
-            if (rows > 0 && bytes <= kPrefetchMax)
-              prefetch_l2(b_raw + ((long long)tn.e * N_out + r0) * K, (uint32_t)bytes);
-          }
-        }
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1u, abort_flag, err)) { ok = false; break; }
           const uint32_t full = bar_full + 8 * stage;
@@ -643,7 +629,7 @@ template <int MODE, typename OutT>
 moe_status launch_tc(const CUtensorMap& ma, const CUtensorMap& mb, const int32_t* offsets, int E, int K, int N_out,
                      int F, long long rows_max, const float* gate_of_row, void* out, cudaStream_t s,
                      const int32_t* token_of_row = nullptr, int n_tokens = 0,
-                     const __nv_bfloat16* a_gather = nullptr, const void* b_raw = nullptr) {
+                     const __nv_bfloat16* a_gather = nullptr) {
   static std::atomic<int> configured[kMaxDevices];
   const moe_status st = ensure_smem_limit(configured, grouped_gemm_tc_kernel<MODE, OutT>, kSmemBytes);
   if (st != MOE_OK) return st;
@@ -654,7 +640,7 @@ moe_status launch_tc(const CUtensorMap& ma, const CUtensorMap& mb, const int32_t
   if (grid < 1) grid = 1;
   grouped_gemm_tc_kernel<MODE, OutT><<<grid, kThreadsTC, kSmemBytes, s>>>(
       ma, mb, offsets, E, K, N_out, F, rows_max, gate_of_row, static_cast<OutT*>(out), token_of_row, n_tokens,
-      a_gather, err_ptr(), static_cast<const __nv_bfloat16*>(b_raw));
+      a_gather, err_ptr());
   return check_launch();
 }
 
@@ -766,10 +752,8 @@ moe_status launch_down_tc(const void* h, const int32_t* offsets, int E, int d, i
     return launch_tc2<1, __nv_bfloat16>(ma, mb, offsets, E, F, d, F, rows_max, gate_of_row, y_rows, s);
   }
   if (y_dtype == MOE_F32)
-    return launch_tc<1, float>(ma, mb, offsets, E, F, d, F, rows_max, gate_of_row, y_rows, s, nullptr, 0, nullptr,
-                               W_dn);
-  return launch_tc<1, __nv_bfloat16>(ma, mb, offsets, E, F, d, F, rows_max, gate_of_row, y_rows, s, nullptr, 0,
-                                     nullptr, W_dn);
+    return launch_tc<1, float>(ma, mb, offsets, E, F, d, F, rows_max, gate_of_row, y_rows, s);
+  return launch_tc<1, __nv_bfloat16>(ma, mb, offsets, E, F, d, F, rows_max, gate_of_row, y_rows, s);
 }
 
 // Down GEMM with the combine fused into its epilogue: y[token_of_row[r]] += gate_of_row[r] *
