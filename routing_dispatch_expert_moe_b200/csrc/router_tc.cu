@@ -58,7 +58,6 @@ constexpr int kRAStage = RBM * BK * 2;  // 16 KB of x per stage
 constexpr int kRMaxStages = 8;
 constexpr uint32_t kRTmemCols = 512;    // two accumulators of up to 256 columns
 constexpr int kRSmemLimit = 232448;     // 227 KB opt-in maximum per CTA
-constexpr int kRPrefetchChunk = 32768;  // bytes per L2 prefetch request
 
 struct RLayout {
   int stage_bytes, stages, bars, misc, staging, end;
@@ -245,8 +244,7 @@ __device__ __forceinline__ void topk_write(const TopK<KMAX, BIAS>& st, long long
 // tile's hi, mid, lo rows are contiguous); each CTA loads its 3 NE / 2 rows in one box.
 template <int KMAX, bool BIAS, bool SIDE>
 __global__ void __launch_bounds__(kRThreads, 1)
-router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
-                 const __nv_bfloat16* __restrict__ x, int T, int d,
+router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW, int T, int d,
                  int E, int NE, int n_tiles, int stages, const float* __restrict__ logit_offset,
                  float* __restrict__ logits, const float* __restrict__ sel_bias, int k, int score, int renorm,
                  float scale, int32_t* __restrict__ topk_idx, float* __restrict__ topk_gate, int* err) {
@@ -309,16 +307,6 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
       for (int i = 0; ok && unit_of(kFused, i, cid, ncl, n_rt, n_tiles, &rt, &j); ++i) {
         const int a_row = rt * 2 * RBM + (int)rank * RBM;
         const int b_row = j * 3 * NE + (int)rank * half;
-        if (n_tiles == 1 && a_row < T) {
-          // x is read once (one expert tile): ask L2 for this CTA's rows as one contiguous
-          // stream first, so the 128-byte box rows below hit L2 instead of each opening
-          // its own DRAM access
-          const long long r1 = min((long long)T, (long long)a_row + RBM);
-          const char* base = reinterpret_cast<const char*>(x + (long long)a_row * d);
-          const long long bytes = (r1 - a_row) * (long long)d * 2;
-          for (long long off = 0; off < bytes; off += kRPrefetchChunk)
-            prefetch_l2(base + off, (uint32_t)min((long long)kRPrefetchChunk, bytes - off));
-        }
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1u, abort_flag, err)) { ok = false; break; }
           if (rank == 0) mbar_expect_tx(bar_full + 8 * stage, 2u * (uint32_t)(kRAStage + 3 * term_bytes));
@@ -541,8 +529,7 @@ prepare_router_weight_kernel(const float* __restrict__ Wg, int d, int E, int NE,
 }
 
 template <int KMAX, bool BIAS, bool SIDE>
-moe_status launch_router_kernel(const CUtensorMap& mx, const CUtensorMap& mw, const void* x, int T, int d, int E,
-                                int NE,
+moe_status launch_router_kernel(const CUtensorMap& mx, const CUtensorMap& mw, int T, int d, int E, int NE,
                                 int n_tiles, const float* off, float* logits, const float* sel_bias, int k,
                                 int score, int renorm, float scale, int32_t* idx, float* gate, cudaStream_t s) {
   static std::atomic<int> configured[kMaxDevices];
@@ -569,8 +556,7 @@ moe_status launch_router_kernel(const CUtensorMap& mx, const CUtensorMap& mw, co
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cuda_status(cudaLaunchKernelEx(&cfg, router_tc_kernel<KMAX, BIAS, SIDE>, mx, mw,
-                                        static_cast<const __nv_bfloat16*>(x), T, d, E, NE, n_tiles, stages, off,
+  return cuda_status(cudaLaunchKernelEx(&cfg, router_tc_kernel<KMAX, BIAS, SIDE>, mx, mw, T, d, E, NE, n_tiles, stages, off,
                                         logits, sel_bias, k, score, renorm, scale, idx, gate, err_ptr()));
 }
 
@@ -629,9 +615,9 @@ moe_status launch_router_tc(const void* x, int T, int d, int E, const void* W3, 
   // NE <= 64: the three terms side by side (one MMA of N = 3 NE per k step)
   const bool side = router_side_by_side(g.NE);
 #define MOE_RT(KM, B)                                                                                            \
-  return side ? launch_router_kernel<KM, B, true>(mx, mw, x, T, d, E, g.NE, g.n_tiles, logit_offset, logits,       \
+  return side ? launch_router_kernel<KM, B, true>(mx, mw, T, d, E, g.NE, g.n_tiles, logit_offset, logits,       \
                                                   sel_bias, fuse_k, score, renorm, scale, topk_idx, topk_gate, s) \
-              : launch_router_kernel<KM, B, false>(mx, mw, x, T, d, E, g.NE, g.n_tiles, logit_offset, logits,      \
+              : launch_router_kernel<KM, B, false>(mx, mw, T, d, E, g.NE, g.n_tiles, logit_offset, logits,      \
                                                    sel_bias, fuse_k, score, renorm, scale, topk_idx, topk_gate, s)
   if (fuse_k <= 0) MOE_RT(0, false);
   if (fuse_k <= 8) {
