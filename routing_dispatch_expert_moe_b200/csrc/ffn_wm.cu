@@ -279,10 +279,6 @@ grouped_gemm_wm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
           }
         }
         tok[i] = t;
-        // the tile reads each of its token rows in 64-element pieces over K / 64 stages:
-        // ask L2 for the whole row up front (one contiguous request per row), so the
-        // 128-byte cp.async pieces below mostly hit L2
-        if (cv == 0 && t >= 0) prefetch_l2(x_gather + (long long)t * K, (uint32_t)K * 2u);
       }
       for (int kb = 0; kb < KB; ++kb) {
         const bool got = mbar_wait(bar_empty + 8 * stage, phase ^ 1u, abort_flag, err);
