@@ -51,7 +51,7 @@ struct WmCfg {
   static constexpr int epi_warps = 4;
   static constexpr int threads = 64 + 32 * epi_warps;
   static constexpr int bars = stages * stage_bytes;
-  static constexpr int nbars = 3 * stages + 4 + 1;   // full, empty, tfull[2], tempty[2], fin, gathered
+  static constexpr int nbars = 2 * stages + 4 + 1;   // full, empty, tfull[2], tempty[2], fin
   static constexpr int misc = bars + nbars * 8;
   static constexpr int tiles = misc + 16;
   static constexpr int sh32 = tiles + (kWMaxE + 1) * 4;
@@ -186,16 +186,14 @@ __device__ __forceinline__ void wm_epilogue_tile(uint32_t taddr, uint8_t* stage,
 }
 
 // GATHER (gate/up only): the token rows come straight from x [n_tokens, d] through
-// token_of_row (no permuted copy of x).  The producer warp's lanes copy them with 16-byte
-// cp.async into the swizzled layout and arrive on a local `gathered` barrier; a forwarder
-// warp waits on it, fences the rows for the async proxy and arrives on the even CTA's
-// `full` barrier, which also counts the weights' TMA bytes.
+// token_of_row (no permuted copy of x): TMA row gathers (four rows per instruction, one
+// lane per four rows) land them in the same swizzled layout as the tiled loads, counted
+// on the even CTA's `full` barrier with the weights' bytes; tmX maps x with a one-row box.
 template <int MODE, typename OutT, bool GATHER = false>
-__global__ void __launch_bounds__(WmCfg<MODE>::threads + (GATHER ? 32 : 0), 1)
+__global__ void __launch_bounds__(WmCfg<MODE>::threads, 1)
 grouped_gemm_wm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                        const int32_t* __restrict__ offsets, int E, int K, int d, int F, long long rows_max,
                        const float* __restrict__ gate_of_row, OutT* __restrict__ out, int* err,
-                       const __nv_bfloat16* __restrict__ x_gather = nullptr,
                        const int32_t* __restrict__ token_of_row = nullptr, int n_tokens = 0) {
   static_assert(!GATHER || MODE == 0, "the gathered form is the gate/up GEMM's");
   using C = WmCfg<MODE>;
@@ -220,15 +218,13 @@ grouped_gemm_wm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
   const uint32_t bar_tfull = bar_empty + 8 * C::stages;
   const uint32_t bar_tempty = bar_tfull + 16;
   const uint32_t bar_fin = bar_tempty + 16;
-  const uint32_t bar_gath = bar_fin + 8;                   // [stages], GATHER only
   auto a_blk = [&](int s, int a) { return sb + (uint32_t)(s * C::stage_bytes + a * kWBlock); };
   auto b_blk = [&](int s) { return sb + (uint32_t)(s * C::stage_bytes + C::a_blocks * kWBlock); };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::stages; ++s) {
-      mbar_init(bar_full + 8 * s, GATHER ? 1 + 2 : 1);     // + one forwarded arrival per CTA
+      mbar_init(bar_full + 8 * s, 1);
       mbar_init(bar_empty + 8 * s, 1);
-      mbar_init(bar_gath + 8 * s, 32);                       // one cp.async arrival per producer lane
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(bar_tfull + 8 * a, 1);
@@ -253,8 +249,9 @@ grouped_gemm_wm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
 
   if (GATHER && warp == 0) {
     // ------------------------------------------------------------ gathering producer (both CTAs)
-    // lane: 16-byte chunk cv of rows rsub, rsub + 4, ... of this CTA's n / 2 token rows
-    const int cv = lane & 7, rsub = lane >> 3;
+    // Lane j < n / 8 owns rows 4j .. 4j+3 of this CTA's n / 2 token rows and fetches them
+    // with one TMA row gather per k-block (rows past the group read token 0: their MMA
+    // columns are never stored); lane 0 also loads the weight slab.
     int stage = 0;
     uint32_t phase = 0;
     int last_phase[C::stages];
@@ -265,65 +262,39 @@ grouped_gemm_wm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
       const TileCoord tc = tile_coord(tile_start, offsets, E, C::NT, tile);
       const int half = wm_n<MODE>(tc.rows) / 2;
       const int w_row = tc.e * 2 * F + tc.n_tile * 256 + (int)rank * kWRows;
-      const int r_base = (int)rank * half;                 // this CTA's first row of the tile
-      int tok[C::NT / 8];                                   // rows rsub + 4 i, i < NT / 8
+      const bool mine = 4 * lane < half;
+      const int r0 = (int)rank * half + 4 * lane;           // this lane's first row of the tile
+      int t[4];
 #pragma unroll
-      for (int i = 0; i < C::NT / 8; ++i) {
-        const int r = i * 4 + rsub;
-        int t = -1;
-        if (r < half && r_base + r < tc.rows) {
-          t = __ldg(token_of_row + tc.row0 + r_base + r);
-          if ((unsigned)t >= (unsigned)n_tokens) {
+      for (int i = 0; i < 4; ++i) {
+        int v = 0;
+        if (mine && r0 + i < tc.rows) {
+          v = __ldg(token_of_row + tc.row0 + r0 + i);
+          if ((unsigned)v >= (unsigned)n_tokens) {
             record_error(err, MOE_DEVERR_ROW);
-            t = -1;
+            v = 0;
           }
         }
-        tok[i] = t;
+        t[i] = v;
       }
       for (int kb = 0; kb < KB; ++kb) {
         const bool got = mbar_wait(bar_empty + 8 * stage, phase ^ 1u, abort_flag, err);
         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+        const uint32_t full_c = map_to_rank(bar_full + 8 * stage, 0);
         if (lane == 0) {
-          if (rank == 0) mbar_expect_tx(bar_full + 8 * stage, 2u * (uint32_t)(C::a_blocks * kWBlock));
-          const uint32_t full_c = map_to_rank(bar_full + 8 * stage, 0);
+          if (rank == 0)
+            mbar_expect_tx(bar_full + 8 * stage, 2u * (uint32_t)(C::a_blocks * kWBlock + half * BK * 2));
           tma_load_2d_pair(a_blk(stage, 0), &tmW, full_c, kb * BK, w_row);
           tma_load_2d_pair(a_blk(stage, 1), &tmW, full_c, kb * BK, w_row + F);
           last_phase[stage] = (int)phase;
         }
-        const uint32_t b_dst = b_blk(stage);
-        const int kcol = kb * BK + cv * 8;
-#pragma unroll
-        for (int i = 0; i < C::NT / 8; ++i) {
-          const int r = i * 4 + rsub;
-          if (r < half) {                                   // rows past the group are zeros
-            const bool v = tok[i] >= 0 && kcol < K;
-            const __nv_bfloat16* src = x_gather + (v ? (long long)tok[i] * K + kcol : 0LL);
-            cp_async16(b_dst + r * 128 + ((cv ^ (r & 7)) << 4), src, v ? 16u : 0u);
-          }
-        }
-        cp_async_arrive_noinc(bar_gath + 8 * stage);
+        if (mine) tma_gather4_pair(b_blk(stage) + (uint32_t)(lane * 512), &tmX, full_c, kb * BK, t[0], t[1], t[2], t[3]);
         if (++stage == C::stages) { stage = 0; phase ^= 1u; }
       }
     }
-    cp_async_wait_all();                                    // no copy may land after the CTA has exited
     if (!ok && lane == 0 && rank == 0) {
       for (int s = 0; s < C::stages; ++s)
         if (last_phase[s] >= 0) mbar_wait_drain(bar_full + 8 * s, (uint32_t)last_phase[s], err);
-    }
-  } else if (GATHER && warp == 2 + C::epi_warps) {
-    // ------------------------------------------------------------ forwarder (both CTAs)
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      bool ok = true;
-      for (int tile = cid; ok && tile < total; tile += ncl) {
-        for (int kb = 0; kb < KB; ++kb) {
-          if (!mbar_wait(bar_gath + 8 * stage, phase, abort_flag, err)) { ok = false; break; }
-          fence_proxy_async_smem();                         // the MMAs read the rows through the async proxy
-          mbar_arrive_cluster(map_to_rank(bar_full + 8 * stage, 0));
-          if (++stage == C::stages) { stage = 0; phase ^= 1u; }
-        }
-      }
     }
   } else if (warp == 0) {
     // ------------------------------------------------------------ TMA producer (both CTAs)
@@ -377,7 +348,6 @@ grouped_gemm_wm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag, err)) { ok = false; break; }
           tc_fence_after();
-          if (GATHER) fence_proxy_async_smem();
           const uint64_t bdesc = sw128_desc(b_blk(stage));
           const uint64_t adesc0 = sw128_desc(a_blk(stage, 0));
           const uint64_t adesc1 = sw128_desc(a_blk(stage, MODE == 0 ? 1 : 0));
@@ -785,8 +755,7 @@ fp4_scales_kernel(const uint8_t* __restrict__ in, long long rows, int K, int spr
 template <int MODE, typename OutT, bool GATHER = false>
 moe_status launch_wm(const CUtensorMap& mw, const CUtensorMap& mx, const int32_t* offsets, int E, int K, int d,
                      int F, long long rows_max, const float* gate_of_row, void* out, cudaStream_t s,
-                     const __nv_bfloat16* x_gather = nullptr, const int32_t* token_of_row = nullptr,
-                     int n_tokens = 0) {
+                     const int32_t* token_of_row = nullptr, int n_tokens = 0) {
   using C = WmCfg<MODE>;
   static std::atomic<int> configured[kMaxDevices];
   const moe_status st = ensure_smem_limit(configured, grouped_gemm_wm_kernel<MODE, OutT, GATHER>, C::smem);
@@ -797,7 +766,7 @@ moe_status launch_wm(const CUtensorMap& mw, const CUtensorMap& mx, const int32_t
   if (pairs < 1) pairs = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs, 1, 1);
-  cfg.blockDim = dim3(C::threads + (GATHER ? 32 : 0), 1, 1);
+  cfg.blockDim = dim3(C::threads, 1, 1);
   cfg.dynamicSmemBytes = C::smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -808,8 +777,8 @@ moe_status launch_wm(const CUtensorMap& mw, const CUtensorMap& mx, const int32_t
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cuda_status(cudaLaunchKernelEx(&cfg, grouped_gemm_wm_kernel<MODE, OutT, GATHER>, mw, mx, offsets, E, K, d,
-                                        F, rows_max, gate_of_row, static_cast<OutT*>(out), err_ptr(), x_gather,
-                                        token_of_row, n_tokens));
+                                        F, rows_max, gate_of_row, static_cast<OutT*>(out), err_ptr(), token_of_row,
+                                        n_tokens));
 }
 
 }  // namespace
@@ -849,10 +818,10 @@ moe_status launch_gate_up_wm_gather(const void* x, const int32_t* token_of_row, 
                                     int d, int F, long long rows_max, const void* W_gu, void* h, cudaStream_t s) {
   if (rows_max == 0 || T == 0) return MOE_OK;
   if (d < BK || F < 8) return MOE_ERR_UNSUPPORTED;
-  CUtensorMap mw;
+  CUtensorMap mw, mx;
   if (!make_map(&mw, W_gu, (unsigned long long)E * 2 * F, d, kWRows)) return MOE_ERR_UNSUPPORTED;
-  return launch_wm<0, __nv_bfloat16, true>(mw, mw, offsets, E, d, d, F, rows_max, nullptr, h, s,
-                                           static_cast<const __nv_bfloat16*>(x), token_of_row, T);
+  if (!make_map(&mx, x, (unsigned long long)T, d, 1)) return MOE_ERR_UNSUPPORTED;   // one-row box: row gathers
+  return launch_wm<0, __nv_bfloat16, true>(mw, mx, offsets, E, d, d, F, rows_max, nullptr, h, s, token_of_row, T);
 }
 
 // Down, weight-major: gated rows [rows_max, d] (bf16 or fp32) from H [rows_max, F] and W_dn [E][d][F].
