@@ -416,16 +416,18 @@ grouped_gemm_wm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
 // it).  K a multiple of 64.
 //
 // Per stage and CTA: the codes and scales of its weight rows and its token rows land by
-// TMA and bulk copy on the CTA's own `packed` barrier.  A converter thread owns one weight
-// row of a block (gate/up: 256 threads for the two blocks of 128 rows; down: two threads
-// per row, four 16-byte chunks each).  It decodes each 32-bit word of codes (eight
+// TMA and bulk copy on the CTA's own `packed` barrier.  The eight converter warps form four
+// groups of two; group g decodes the stages g, g + 4, ..., so the four stages of the ring
+// are decoded side by side (one group for every stage took 1.5x as long).  A converter
+// thread owns two weight rows of its stages (all blocks and chunks of them).  It decodes
+// each 32-bit word of codes (eight
 // elements) in registers: the three magnitude bits of four codes at once select the high
 // and low bytes of their bf16 values from two 8-byte tables (byte permutes), the sign
 // bits are moved into place, and the bf16 pairs are multiplied by the block scale.  Each
 // 16-byte chunk goes to the 128-byte-swizzled operand layout (chunk c of row r at
 // r * 128 + ((c ^ (r & 7)) * 16)); then each thread's proxy fence, and one arrive per
-// converter warp on the even CTA's `full` barrier (2 x 8 warps).  `empty` (the MMAs'
-// completion) frees the stage in both CTAs.
+// converter warp of the stage's group on the even CTA's `full` barrier (2 x 2 warps).
+// `empty` (the MMAs' completion) frees the stage in both CTAs.
 // =====================================================================================
 template <int MODE>
 struct Wm4Cfg {
@@ -436,7 +438,11 @@ struct Wm4Cfg {
   static constexpr int scale_block = kWRows * 4;                // up to 4 scale bytes per row and k-block
   static constexpr int stage_bytes = a_blocks * kWBlock + b_bytes + a_blocks * (packed_block + scale_block);
   static constexpr int stage_pitch = (stage_bytes + 1023) / 1024 * 1024;
-  static constexpr int stages = MODE == 0 ? 4 : 5;
+  static constexpr int stages = 4;
+  // converter groups decoding stages side by side (one group per stage measured fastest:
+  // 4.08 -> 2.74 ms for the MXFP4 gate/up of the stress layer with one group); a group
+  // must see every phase of the stages it waits on, so the groups divide the stages
+  static constexpr int cvt_groups = 4;
   static constexpr int epi_warps = 4, cvt_warps = 8;
   static constexpr int threads = 64 + 32 * (epi_warps + cvt_warps);
   static constexpr int bars = stages * stage_pitch;
@@ -449,6 +455,9 @@ struct Wm4Cfg {
   static constexpr size_t smem = end + 1024;
   static_assert(smem <= 232448, "shared memory per CTA");
   static_assert((a_blocks * kWBlock + b_bytes) % 1024 == 0, "swizzle alignment");
+  static_assert(cvt_warps % cvt_groups == 0 && kWRows % (cvt_warps * 32 / cvt_groups) == 0,
+                "converter groups of whole warps, each thread the same number of weight rows");
+  static_assert(stages % cvt_groups == 0, "a converter group waits only on the stages it has seen");
 };
 
 // bf16 of a block scale byte: E8M0 (2^(b - 127); b = 0 is 2^-127, a bf16 subnormal) or
@@ -554,7 +563,7 @@ grouped_gemm_wm4_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_co
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::stages; ++s) {
       mbar_init(bar_packed + 8 * s, 1);
-      mbar_init(bar_full + 8 * s, 2 * C::cvt_warps);   // one arrive per converter warp of each CTA
+      mbar_init(bar_full + 8 * s, 2 * C::cvt_warps / C::cvt_groups);   // one arrive per warp of a group, both CTAs
       mbar_init(bar_empty + 8 * s, 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -675,25 +684,34 @@ grouped_gemm_wm4_kernel(const __grid_constant__ CUtensorMap tmC, const __grid_co
     }
   } else {
     // ------------------------------------------------------------ converters (both CTAs)
+    // kCvtGroups groups of warps take the stages in turn (group g the stages g, g + G, ...),
+    // so G stages are decoded at once; a thread owns kWRows / group-size weight rows of its
+    // stages (every block and chunk of them).
+    constexpr int G = C::cvt_groups, GT = C::cvt_warps * 32 / G;   // groups, threads per group
     const int ct = threadIdx.x - 64 - 32 * C::epi_warps;     // 0 .. 32 cvt_warps - 1
-    const int r = ct & (kWRows - 1);                         // its weight row of the block
-    const int a = MODE == 0 ? ct / kWRows : 0;               // gate/up: block (gate or up)
-    const int c0 = MODE == 0 ? 0 : (ct / kWRows) * 4;        // down: half of the row's chunks
-    const int c1 = MODE == 0 ? 8 : c0 + 4;
+    const int grp = ct / GT, r0 = ct % GT;                   // its group, its first row
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
+    int seq = 0;
     for (int tile = cid; ok && tile < total; tile += ncl) {
-      for (int kb = 0; kb < KB; ++kb) {
-        const bool got = mbar_wait(bar_packed + 8 * stage, phase, abort_flag, err);
-        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-        const uint8_t* sc_p = smem + s_off(stage, a) + r * kSpr;
-        const uint32_t sc = FMT == MOE_FP4_MX ? (uint32_t)*reinterpret_cast<const uint16_t*>(sc_p)
-                                              : *reinterpret_cast<const uint32_t*>(sc_p);
-        convert_chunks<FMT>(smem + p_off(stage, a) + r * (BK / 2), sc, smem + a_off(stage, a), r, c0, c1);
-        fence_proxy_async_smem();                           // the MMAs read these through the async proxy
-        __syncwarp();                                       // the warp's chunks are written and fenced
-        if (lane == 0) mbar_arrive_cluster(map_to_rank(bar_full + 8 * stage, 0));
+      for (int kb = 0; kb < KB; ++kb, ++seq) {
+        if (seq % G == grp) {
+          const bool got = mbar_wait(bar_packed + 8 * stage, phase, abort_flag, err);
+          if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+#pragma unroll
+          for (int r = r0; r < kWRows; r += GT)
+#pragma unroll
+            for (int a = 0; a < C::a_blocks; ++a) {
+              const uint8_t* sc_p = smem + s_off(stage, a) + r * kSpr;
+              const uint32_t sc = FMT == MOE_FP4_MX ? (uint32_t)*reinterpret_cast<const uint16_t*>(sc_p)
+                                                    : *reinterpret_cast<const uint32_t*>(sc_p);
+              convert_chunks<FMT>(smem + p_off(stage, a) + r * (BK / 2), sc, smem + a_off(stage, a), r, 0, 8);
+            }
+          fence_proxy_async_smem();                         // the MMAs read these through the async proxy
+          __syncwarp();                                     // the warp's rows are written and fenced
+          if (lane == 0) mbar_arrive_cluster(map_to_rank(bar_full + 8 * stage, 0));
+        }
         if (++stage == C::stages) { stage = 0; phase ^= 1u; }
       }
     }
