@@ -421,9 +421,9 @@ grouped_gemm_wm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_con
 // are decoded side by side (one group for every stage took 1.5x as long).  A converter
 // thread owns two weight rows of its stages (all blocks and chunks of them).  It decodes
 // each 32-bit word of codes (eight
-// elements) in registers: the three magnitude bits of four codes at once select the high
-// and low bytes of their bf16 values from two 8-byte tables (byte permutes), the sign
-// bits are moved into place, and the bf16 pairs are multiplied by the block scale.  Each
+// elements) in registers: shifts and masks place each code's bits in a bf16 (which reads
+// as 2^-126 times the code's value, subnormal codes included), byte permutes put the
+// pairs in order, and each bf16 pair is multiplied by 2^126, then by the block scale.  Each
 // 16-byte chunk goes to the 128-byte-swizzled operand layout (chunk c of row r at
 // r * 128 + ((c ^ (r & 7)) * 16)); then each thread's proxy fence, and one arrive per
 // converter warp of the stage's group on the even CTA's `full` barrier (2 x 2 warps).
@@ -471,19 +471,23 @@ __device__ __forceinline__ uint32_t scale_bf16_bits(uint32_t b) {
   return (uint32_t)(*reinterpret_cast<const uint16_t*>(&v));
 }
 
-// Eight E2M1 codes (w: element i in bits 4i .. 4i+3) -> eight bf16 values (o[0] holds
-// elements 0 and 1, ...).  The magnitude codes 0..7 are 0, 0.5, 1, 1.5, 2, 3, 4, 6, whose
-// bf16 high bytes are 00 3F 3F 3F 40 40 40 40 and low bytes 00 00 80 C0 00 40 80 C0.
-__device__ __forceinline__ void e2m1x8_to_bf16(uint32_t w, uint32_t (&o)[4]) {
-  constexpr uint32_t HI0 = 0x3F3F3F00u, HI1 = 0x40404040u, LO0 = 0xC0800000u, LO1 = 0xC0804000u;
-  const uint32_t m = w & 0x77777777u;
-  const uint32_t lo_a = __byte_perm(LO0, LO1, m), hi_a = __byte_perm(HI0, HI1, m);
-  const uint32_t lo_b = __byte_perm(LO0, LO1, m >> 16), hi_b = __byte_perm(HI0, HI1, m >> 16);
-  const uint32_t sg = w & 0x88888888u;
-  o[0] = __byte_perm(lo_a, hi_a, 0x5140) | ((sg & 0x8u) << 12) | ((sg & 0x80u) << 24);
-  o[1] = __byte_perm(lo_a, hi_a, 0x7362) | ((sg & 0x800u) << 4) | ((sg & 0x8000u) << 16);
-  o[2] = __byte_perm(lo_b, hi_b, 0x5140) | ((sg & 0x80000u) >> 4) | ((sg & 0x800000u) << 8);
-  o[3] = __byte_perm(lo_b, hi_b, 0x7362) | ((sg & 0x8000000u) >> 12) | (sg & 0x80000000u);
+// Eight E2M1 codes (w: element i in bits 4i .. 4i+3) -> the bits of eight bf16 values
+// 2^-126 times the codes' values (o[0] holds elements 0 and 1, ...).  A code's magnitude
+// bits e1 e0 m placed at bf16 bits 8..6, its sign at bit 15, read as a bf16 number:
+// exponent field e, so for e > 0 the value is 2^(e-127) (1 + m/2) and for e = 0 the
+// subnormal m 2^-127, while E2M1 is 2^(e-1) (1 + m/2) and m / 2: both 2^-126 times it.
+// One shift of the word places codes i and i + 4 in the two halves of a bf16 pair; byte
+// permutes then pair the elements in order.
+__device__ __forceinline__ void e2m1x8_to_bf16_bits(uint32_t w, uint32_t (&o)[4]) {
+  constexpr uint32_t MAG = 0x01C001C0u, SGN = 0x80008000u;
+  const uint32_t p0 = ((w << 6) & MAG) | ((w << 12) & SGN);   // elements 0, 4
+  const uint32_t p1 = ((w << 2) & MAG) | ((w << 8) & SGN);    // 1, 5
+  const uint32_t p2 = ((w >> 2) & MAG) | ((w << 4) & SGN);    // 2, 6
+  const uint32_t p3 = ((w >> 6) & MAG) | (w & SGN);           // 3, 7
+  o[0] = __byte_perm(p0, p1, 0x5410);
+  o[1] = __byte_perm(p2, p3, 0x5410);
+  o[2] = __byte_perm(p0, p1, 0x7632);
+  o[3] = __byte_perm(p2, p3, 0x7632);
 }
 
 // Expands chunks [c0, c1) of one row of a block: codes at src (32 bytes), the row's scale
@@ -501,12 +505,14 @@ __device__ __forceinline__ void convert_chunks(const uint8_t* src, uint32_t sc, 
                                           : scale_bf16_bits<FMT>((sc >> (8 * (c >> 1))) & 0xffu);
     const uint32_t s2u = sb | (sb << 16);
     const __nv_bfloat162 s2 = *reinterpret_cast<const __nv_bfloat162*>(&s2u);
+    constexpr uint32_t kTwo126 = 0x7E807E80u;   // bf16 pair 2^126, 2^126
+    const __nv_bfloat162 t2 = *reinterpret_cast<const __nv_bfloat162*>(&kTwo126);
     uint32_t o[4];
-    e2m1x8_to_bf16(w[c], o);
+    e2m1x8_to_bf16_bits(w[c], o);
 #pragma unroll
     for (int b = 0; b < 4; ++b) {
       __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&o[b]);
-      v = __hmul2(v, s2);                       // exact: at most 6 significant bits
+      v = __hmul2(__hmul2(v, t2), s2);          // exact: the code's value, then at most 6 significant bits
       o[b] = *reinterpret_cast<uint32_t*>(&v);
     }
     *reinterpret_cast<uint4*>(dst_block + r * 128 + ((c ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
