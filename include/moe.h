@@ -524,9 +524,10 @@ MOE_API moe_status moe_expert_gate_up(const void* x_rows, int32_t dtype, const i
  * neither written nor read and moe_permute is not needed before it.
  *   x (device) [T, d] dtype;  token_of_row (device) [rows_max] int32 from
  *   moe_histogram_scan;  the other arguments as moe_expert_gate_up.
- * The rows arrive by TMA row gathers (four rows per instruction).  H is bitwise identical
- * to moe_permute followed by moe_expert_gate_up.  A token index outside [0, T) is
- * recorded as MOE_DEVERR_ROW and row 0 of x is read in its place. */
+ * Weight-major tiles fetch the rows by TMA row gathers (four rows per instruction),
+ * token-major tiles by 16-byte cp.async.  H is bitwise identical to moe_permute followed
+ * by moe_expert_gate_up.  A token index outside [0, T) is recorded as MOE_DEVERR_ROW and
+ * a row of zeros (token-major) or row 0 of x (weight-major) is read in its place. */
 MOE_API moe_status moe_expert_gate_up_gather(const void* x, int32_t dtype, int32_t T,
                               const int32_t* token_of_row, const int32_t* offsets,
                               int32_t E, int32_t d, int32_t F, int64_t rows_max,

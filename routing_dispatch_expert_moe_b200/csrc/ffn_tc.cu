@@ -19,9 +19,8 @@
 //       order over a token's experts is whatever order the tiles finish in.
 //   MODE 4 (gate_up, gathered): as MODE 0, but the A rows are gathered straight from the
 //       token matrix, A row r = x[token_of_row[r]], so no permuted copy of x is written
-//       or read.  The producer warp's lanes fetch them with TMA row gathers
-//       (tile::gather4: four rows of 64 columns per instruction) into the same
-//       128-byte-swizzled layout the tiled loads write; B arrives by tiled TMA loads.
+//       or read.  The producer warp copies them with 16-byte cp.async into the same
+//       128-byte-swizzled layout TMA writes; B still arrives by TMA.
 //
 // Per CTA (1 per SM, 192 threads):
 //   warp 0   TMA producer: 128x64 A tile + 256x64 B tile per stage (128-byte swizzle),
@@ -194,18 +193,25 @@ __device__ __forceinline__ void epilogue_tile(uint32_t taddr, uint8_t* stage, in
   }
 }
 
-// Producer warp of the gathered gate/up GEMM (MODE 4).  Lane j owns A rows 4j .. 4j+3 of
-// the 128-row tile, x[token_of_row[r]] (rows past the group read token 0: their
-// accumulator rows are never stored), and fetches them with one TMA row gather per
-// k-block into the 128-byte-swizzled layout the tiled loads produce; lane 0 arms the full
-// barrier with the A and B bytes and issues B's TMA loads.  tmA maps x [n_tokens, K] with
-// a one-row box.
-__device__ __forceinline__ void gather_producer(const CUtensorMap* tmA, const CUtensorMap* tmB, uint32_t sb,
-                                                uint32_t bar_full, uint32_t bar_empty, const int* tile_start,
+// Producer warp of the gathered gate/up GEMM (MODE 4).  Per stage, lane 0 arms the full
+// barrier with the B bytes and issues B's TMA loads; every lane copies its share of the
+// 128 A rows (lane = 16-byte chunk lane & 7 of rows lane >> 3, +4, +8, ...), each row
+// x[token_of_row[r]][k-block], with cp.async into the 128-byte-swizzled layout: chunk c
+// of row r lands at r * 128 + ((c ^ (r & 7)) * 16).  Rows past the tile and columns past
+// K are zero-filled.  Each lane then queues a hardware arrival on the stage's full
+// barrier that fires when its copies have landed (count 1 + 32), so the warp moves on
+// to the next stage at once; the MMA thread fences the stage for the async proxy after
+// its wait.
+// (Measured: slower than the permute copy plus the box-loaded GEMM, because every A tile
+// is re-read once per n-tile as 128-byte rows; it saves the permuted buffer.)
+__device__ __forceinline__ void gather_producer(const CUtensorMap* tmB, uint32_t sb, uint32_t bar_full,
+                                                uint32_t bar_empty, const int* tile_start,
                                                 const int32_t* __restrict__ offsets, int E, int K, int F,
                                                 const int32_t* __restrict__ token_of_row, int n_tokens,
-                                                volatile int* abort_flag, int* err) {
+                                                const __nv_bfloat16* __restrict__ x, volatile int* abort_flag,
+                                                int* err) {
   const int lane = threadIdx.x & 31;
+  const int cv = lane & 7, rsub = lane >> 3;
   const int KB = (K + BK - 1) / BK;
   const int total = tile_start[E];
   int stage = 0;
@@ -216,38 +222,48 @@ __device__ __forceinline__ void gather_producer(const CUtensorMap* tmA, const CU
   bool ok = true;
   for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
     const TileCoord tc = tile_coord(tile_start, offsets, E, BM, tile);
-    int t[4];
+    int tok[32];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int r = 4 * lane + i;
-      int v = 0;
+    for (int i = 0; i < 32; ++i) {
+      const int r = i * 4 + rsub;
+      int t = -1;
       if (r < tc.rows) {
-        v = __ldg(token_of_row + tc.row0 + r);
-        if ((unsigned)v >= (unsigned)n_tokens) {
+        t = __ldg(token_of_row + tc.row0 + r);
+        if ((unsigned)t >= (unsigned)n_tokens) {
           record_error(err, MOE_DEVERR_ROW);
-          v = 0;
+          t = -1;
         }
       }
-      t[i] = v;
+      tok[i] = t;
     }
     const int g_row = tc.e * 2 * F + tc.n_tile * 128;
     for (int kb = 0; kb < KB; ++kb) {
       const bool got = mbar_wait(bar_empty + 8 * stage, phase ^ 1u, abort_flag, err);
       if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
       const uint32_t full = bar_full + 8 * stage;
+      const uint32_t a_dst = sb + L::a + stage * A_STAGE;
       if (lane == 0) {
         const uint32_t b_dst = sb + L::b + stage * B_STAGE;
-        mbar_expect_tx(full, A_STAGE + B_STAGE);
+        mbar_expect_tx(full, B_STAGE);
         tma_load_2d(b_dst, tmB, full, kb * BK, g_row);
         tma_load_2d(b_dst + B_STAGE / 2, tmB, full, kb * BK, g_row + F);
         last_phase[stage] = (int)phase;
       }
-      tma_gather4(sb + L::a + stage * A_STAGE + (uint32_t)(lane * 512), tmA, full, kb * BK, t[0], t[1], t[2], t[3]);
+      const int kcol = kb * BK + cv * 8;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int r = i * 4 + rsub;
+        const bool v = tok[i] >= 0 && kcol < K;
+        const __nv_bfloat16* src = x + (v ? (long long)tok[i] * K + kcol : 0LL);
+        cp_async16(a_dst + r * 128 + ((cv ^ (r & 7)) << 4), src, v ? 16u : 0u);
+      }
+      cp_async_arrive_noinc(full);
       if (++stage == STAGES) { stage = 0; phase ^= 1u; }
     }
   }
+  cp_async_wait_all();                      // no copy may land after the CTA has exited
   if (!ok && lane == 0) {
-    // let every issued copy land before the CTA can exit
+    // let every issued B copy land before the CTA can exit
     for (int s = 0; s < STAGES; ++s)
       if (last_phase[s] >= 0) mbar_wait_drain(bar_full + 8 * s, (uint32_t)last_phase[s], err);
   }
@@ -259,7 +275,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
                        const int32_t* __restrict__ offsets, int E, int K, int N_out, int F,
                        long long rows_max, const float* __restrict__ gate_of_row,
                        OutT* __restrict__ out, const int32_t* __restrict__ token_of_row, int n_tokens,
-                       int* err) {
+                       const __nv_bfloat16* __restrict__ a_gather, int* err) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
@@ -282,7 +298,8 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(bar_full + 8 * s, 1);
+      // gathered A: the B expect_tx arrival plus one cp.async arrival per producer lane
+      mbar_init(bar_full + 8 * s, MODE == 4 ? 1 + 32 : 1);
       mbar_init(bar_empty + 8 * s, 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -306,7 +323,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
   const int KB = (K + BK - 1) / BK;
 
   if (MODE == 4 && warp == 0) {
-    gather_producer(&tmA, &tmB, sb, bar_full, bar_empty, tile_start, offsets, E, K, F, token_of_row, n_tokens,
+    gather_producer(&tmB, sb, bar_full, bar_empty, tile_start, offsets, E, K, F, token_of_row, n_tokens, a_gather,
                     abort_flag, err);
   } else if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -359,6 +376,7 @@ grouped_gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_con
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag, err)) { ok = false; break; }
           tc_fence_after();
+          if (MODE == 4) fence_proxy_async_smem();   // A rows were written by cp.async (generic proxy)
           const uint64_t adesc = sw128_desc(sb + L::a + stage * A_STAGE);
           const uint64_t bdesc = sw128_desc(sb + L::b + stage * B_STAGE);
 #pragma unroll
@@ -506,53 +524,7 @@ grouped_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
   const uint32_t tmem_base = *tmem_slot;
   const int KB = (K + BK - 1) / BK;
 
-  if (MODE == 4 && warp == 0) {
-    // ------------------------------------------------------------ gathering producer (both CTAs)
-    // Lane j owns rows 4j .. 4j+3 of this CTA's 128 A rows, x[token_of_row[r]] (rows past
-    // the group read token 0: their accumulator rows are never stored), fetched with one
-    // TMA row gather per k-block; lane 0 arms the even CTA's barrier and loads B.
-    int stage = 0;
-    uint32_t phase = 0;
-    int last_phase[C::stages];
-#pragma unroll
-    for (int s = 0; s < C::stages; ++s) last_phase[s] = -1;
-    bool ok = true;
-    for (int tile = cid; ok && tile < total; tile += ncl) {
-      const TileCoord tc = tile_coord(tile_start, offsets, E, PM, tile);
-      const int b_row = tc.e * 2 * F + (rank ? F : 0) + tc.n_tile * 128;   // even: gate, odd: up
-      int t[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int r = (int)rank * BM + 4 * lane + i;
-        int v = 0;
-        if (r < tc.rows) {
-          v = __ldg(token_of_row + tc.row0 + r);
-          if ((unsigned)v >= (unsigned)n_tokens) {
-            record_error(err, MOE_DEVERR_ROW);
-            v = 0;
-          }
-        }
-        t[i] = v;
-      }
-      for (int kb = 0; kb < KB; ++kb) {
-        const bool got = mbar_wait(bar_empty + 8 * stage, phase ^ 1u, abort_flag, err);
-        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-        const uint32_t full_c = map_to_rank(bar_full + 8 * stage, 0);
-        if (lane == 0) {
-          if (rank == 0) mbar_expect_tx(bar_full + 8 * stage, 2 * (A_STAGE + B2_STAGE));
-          tma_load_2d_pair(sb + C::b + stage * B2_STAGE, &tmB, full_c, kb * BK, b_row);
-          last_phase[stage] = (int)phase;
-        }
-        tma_gather4_pair(sb + C::a + stage * A_STAGE + (uint32_t)(lane * 512), &tmA, full_c, kb * BK, t[0], t[1],
-                         t[2], t[3]);
-        if (++stage == C::stages) { stage = 0; phase ^= 1u; }
-      }
-    }
-    if (!ok && lane == 0 && rank == 0) {
-      for (int s = 0; s < C::stages; ++s)
-        if (last_phase[s] >= 0) mbar_wait_drain(bar_full + 8 * s, (uint32_t)last_phase[s], err);
-    }
-  } else if (warp == 0) {
+  if (warp == 0) {
     // ------------------------------------------------------------ TMA producer (both CTAs)
     if (lane == 0) {
       int stage = 0;
@@ -656,7 +628,8 @@ grouped_gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_co
 template <int MODE, typename OutT>
 moe_status launch_tc(const CUtensorMap& ma, const CUtensorMap& mb, const int32_t* offsets, int E, int K, int N_out,
                      int F, long long rows_max, const float* gate_of_row, void* out, cudaStream_t s,
-                     const int32_t* token_of_row = nullptr, int n_tokens = 0) {
+                     const int32_t* token_of_row = nullptr, int n_tokens = 0,
+                     const __nv_bfloat16* a_gather = nullptr) {
   static std::atomic<int> configured[kMaxDevices];
   const moe_status st = ensure_smem_limit(configured, grouped_gemm_tc_kernel<MODE, OutT>, kSmemBytes);
   if (st != MOE_OK) return st;
@@ -667,7 +640,7 @@ moe_status launch_tc(const CUtensorMap& ma, const CUtensorMap& mb, const int32_t
   if (grid < 1) grid = 1;
   grouped_gemm_tc_kernel<MODE, OutT><<<grid, kThreadsTC, kSmemBytes, s>>>(
       ma, mb, offsets, E, K, N_out, F, rows_max, gate_of_row, static_cast<OutT*>(out), token_of_row, n_tokens,
-      err_ptr());
+      a_gather, err_ptr());
   return check_launch();
 }
 
@@ -801,8 +774,8 @@ moe_status launch_down_combine_tc(const void* h, const int32_t* offsets, int E, 
 }
 
 // Gate/up GEMM with the dispatch fused into its producer: A row r = x[token_of_row[r]]
-// (x [T, d] bf16), no permuted copy of x, the rows fetched by TMA row gathers.  The tile
-// orientation and pairing follow the permuted form's choice for the same sizes.
+// (x [T, d] bf16), no permuted copy of x.  Single-CTA tiles (the gather producer fills
+// one CTA's stages).
 moe_status launch_gate_up_gather_tc(const void* x, const int32_t* token_of_row, int T, const int32_t* offsets, int E,
                                     int d, int F, long long rows_max, const void* W_gu, void* h, cudaStream_t s) {
   if (rows_max == 0 || T == 0) return MOE_OK;
@@ -811,12 +784,10 @@ moe_status launch_gate_up_gather_tc(const void* x, const int32_t* token_of_row, 
     const moe_status st = launch_gate_up_wm_gather(x, token_of_row, T, offsets, E, d, F, rows_max, W_gu, h, s);
     if (st != MOE_ERR_UNSUPPORTED) return st;
   }
-  CUtensorMap ma, mb;
-  if (!make_map(&ma, x, (unsigned long long)T, d, 1)) return MOE_ERR_UNSUPPORTED;   // one-row box: row gathers
+  CUtensorMap mb;
   if (!make_map(&mb, W_gu, (unsigned long long)E * 2 * F, d, 128)) return MOE_ERR_UNSUPPORTED;
-  if (use_pairs(rows_max, E))
-    return launch_tc2<4, __nv_bfloat16>(ma, mb, offsets, E, d, F, F, rows_max, nullptr, h, s, token_of_row, T);
-  return launch_tc<4, __nv_bfloat16>(ma, mb, offsets, E, d, F, F, rows_max, nullptr, h, s, token_of_row, T);
+  return launch_tc<4, __nv_bfloat16>(mb, mb, offsets, E, d, F, F, rows_max, nullptr, h, s, token_of_row, T,
+                                     static_cast<const __nv_bfloat16*>(x));
 }
 
 }  // namespace moe

@@ -84,19 +84,6 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
-// TMA row gather (tile::gather4): rows y0..y3 of a 2D tensor map whose box is 64
-// columns x 1 row, columns x .. x+63, land as four consecutive 128-byte rows at dst,
-// swizzled as a tiled load of the same map would place them (dst 512-byte aligned).
-// Coordinates must lie inside the tensor.  No multicast.
-__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y0, int y1,
-                                            int y2, int y3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes "
-      "[%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3), "r"(bar)
-      : "memory");
-}
-
 // Orders generic-proxy shared-memory writes this thread has made or observed (stores, or
 // other threads' cp.async copies acquired through an mbarrier) before later async-proxy
 // accesses (the tensor cores read operands through the async proxy).
@@ -156,8 +143,21 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar_cluster)
       : "memory");
 }
-// The row gather of a CTA pair: lands in this CTA's shared memory, completion counted on
-// the pair's even-CTA barrier.
+// 16-byte cp.async global -> shared; src_bytes = 0 writes zeros without reading.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+// Arrive on the mbarrier once all of this thread's earlier cp.async copies have landed
+// (the barrier's expected count includes this arrival: .noinc).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+// TMA row gather (tile::gather4) of a CTA pair: rows y0..y3 of a 2D tensor map whose box
+// is 64 columns x 1 row, columns x .. x+63, land as four consecutive 128-byte rows at dst
+// in this CTA's shared memory, swizzled as a tiled load of the same map would place them
+// (dst 512-byte aligned); completion is counted on the pair's even-CTA barrier.
+// Coordinates must lie inside the tensor.  No multicast.
 __device__ __forceinline__ void tma_gather4_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar_cluster, int x,
                                                  int y0, int y1, int y2, int y3) {
   asm volatile(

@@ -401,7 +401,8 @@ GATHER = [c for c in SMALL if c.name in ("softmax_bf16", "sigmoid_bias_shared", 
 @pytest.mark.parametrize("cfg", GATHER, ids=lambda c: c.name)
 def test_gathered_gate_up_is_bitwise_the_permuted_one(cfg, tiles, monkeypatch):
     """Same token rows, same tiles, same accumulation order: H and the reproducible y agree
-    bit for bit, in every tile form (the rows fetched by TMA row gathers)."""
+    bit for bit, in every tile form (weight-major: the rows fetched by TMA row gathers;
+    token-major: by cp.async)."""
     set_tiles(monkeypatch, tiles)
     host, dev = U.make_inputs(cfg)
     cap = O.capacity(cfg.T, cfg.E, cfg.k, cfg.capacity_factor, True)
@@ -421,7 +422,7 @@ def test_gathered_bad_token_is_reported_not_trapped(tiles, monkeypatch):
         host, dev = U.make_inputs(cfg)
         layer, g = U.gpu_forward(cfg, dev, -1, dispatch="gather")
         tok = layer.token_of_row.clone()
-        tok[3] = -5                                            # outside [0, T): recorded, row 0 read
+        tok[3] = -5                                            # outside [0, T): recorded, never read
         M.moe_expert_gate_up_gather(dev["x"], tok, layer.offsets, layer.w.W_gu, layer.rows_max, layer.h)
         torch.cuda.synchronize()
         assert M.moe_get_device_error() == 3
