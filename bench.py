@@ -40,8 +40,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # (1.019) times the full launch's algorithmic bytes (the capture holds a quarter of the
 # tokens and experts; both the weight and the row bytes grow with the units).
 GATE_UP_TRAFFIC = {
-    ("c2_handbook", "permute", 65536): 931483904,
-    ("c5_stress", "permute", 131356): 8687461198,
+    ("c2_handbook", "permute", 65536): 932886016,
+    ("c5_stress", "permute", 131356): 8784605026,
 }
 
 
