@@ -361,7 +361,8 @@ def test_fused_bad_token_is_reported_not_trapped():
 
 
 def fused_full_size_check(name, per_assignment=True):
-    """Both fusions (gathered gate/up, combine inside the down GEMM): the form bench.py times."""
+    """Both fusions at full size: the gathered gate/up (TMA row gathers on weight-major tiles,
+    cp.async on token-major ones) and the combine inside the down GEMM."""
     cfg = I.CONFIGS[name]
     host, dev = U.make_inputs(cfg)
     cap = O.capacity(cfg.T, cfg.E, cfg.k, cfg.capacity_factor, per_assignment)
