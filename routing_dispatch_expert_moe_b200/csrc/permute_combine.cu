@@ -7,18 +7,102 @@
 // handbook article (zicq.com), "MoE 的核心机制" (dispatch and aggregation are the real
 // bottleneck).
 //
-// Both kernels are pure data movement, bound by HBM bandwidth: one warp per token,
-// each lane moves 16-byte vectors so a warp instruction covers 512 contiguous bytes of
-// the hidden dimension.
-//   permute: x[t] is read once and written to each of its kept rows (k stores per load).
+// Both kernels are pure data movement, bound by HBM bandwidth, one warp per token.
+//   permute: x[t] is read once and written to each of its kept rows, by bulk copies
+//            through shared memory (or, for rows too long for the buffers, 16-byte vectors
+//            from registers, a warp instruction covering 512 contiguous bytes).
 //   combine: all k rows of a token are loaded before any is added (k independent loads in
 //            flight per lane), summed in fp32 in slot order, then the shared-expert row,
 //            then rounded to nearest even.
 #include "common.cuh"
 #include "row8.cuh"
+#include "tc_prims.cuh"
 
 namespace moe {
 namespace {
+
+// Permute by bulk copies.  A warp takes the tokens t0, t0 + nw, ...: lane 0 brings token
+// t's row into a shared-memory buffer with one bulk copy (global -> shared, completing on
+// the buffer's mbarrier), then lanes 0..k-1 each write it to one kept row of x_perm with
+// one bulk copy back (shared -> global).  Three buffers per warp: the load of the token
+// two ahead is issued once the stores of the token before have read their buffer, so a
+// warp keeps a load and up to two tokens' stores in flight without the SM issuing any
+// per-vector loads or stores.  Row bytes a multiple of 16.  Every wait is bounded; on a
+// timeout the warp stops and drains what it issued.
+// Four warps with three buffers each, two loads issued ahead (4 x 3 with one ahead and
+// 6 x 2 measured within 2% of it; this one was ahead of the per-vector copy on both the
+// 7168- and the 2048-wide rows).
+constexpr int kPermWarps = 4, kPermBufs = 3, kPermDepth = 2;   // depth: loads issued ahead
+constexpr int kPermHead = (8 * kPermBufs * kPermWarps + 4 + 127) / 128 * 128;  // mbarriers + abort flag
+static_assert(kPermDepth >= 1 && kPermDepth < kPermBufs, "a buffer is reloaded only after its stores have read it");
+
+__device__ __forceinline__ void bulk_load_row(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_store_row(void* dst, uint32_t src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+__global__ void __launch_bounds__(32 * kPermWarps)
+permute_bulk_kernel(const uint8_t* __restrict__ x, int T, int row_bytes, int row_pitch, int k,
+                    const int32_t* __restrict__ row_of, long long rows_max, uint8_t* __restrict__ x_perm, int* err) {
+  extern __shared__ __align__(128) uint8_t psm[];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const uint32_t bar0 = smem_u32(psm) + (uint32_t)(8 * kPermBufs * w);
+  const uint32_t buf0 = smem_u32(psm) + (uint32_t)kPermHead + (uint32_t)(row_pitch * kPermBufs * w);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(psm + 8 * kPermBufs * kPermWarps);
+  if (threadIdx.x == 0) *abort_flag = 0;
+  if (lane == 0) {
+    for (int b = 0; b < kPermBufs; ++b) mbar_init(bar0 + 8 * b, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const long long nw = (long long)gridDim.x * kPermWarps;
+  const long long t0 = (long long)blockIdx.x * kPermWarps + w;
+  const long long n_iter = t0 < T ? (T - t0 + nw - 1) / nw : 0;
+  int issued = 0;                                         // loads issued (iterations 0 .. issued - 1)
+  auto issue_load = [&](long long i) {
+    if (i < n_iter) {
+      if (lane == 0) {
+        const uint32_t b = (uint32_t)(i % kPermBufs);
+        mbar_expect_tx(bar0 + 8 * b, (uint32_t)row_bytes);
+        bulk_load_row(buf0 + b * (uint32_t)row_pitch, x + (t0 + i * nw) * row_bytes, (uint32_t)row_bytes, bar0 + 8 * b);
+      }
+      issued = (int)i + 1;
+    }
+  };
+  for (int j = 0; j < kPermDepth; ++j) issue_load(j);
+  long long i = 0;
+  for (; i < n_iter; ++i) {
+    const long long t = t0 + i * nw;
+    const uint32_t b = (uint32_t)(i % kPermBufs);
+    int r = -1;
+    if (lane < k) {
+      r = __ldg(row_of + t * k + lane);
+      if (r >= rows_max) { record_error(err, MOE_DEVERR_ROW); r = -1; }
+    }
+    const bool got = mbar_wait(bar0 + 8 * b, (uint32_t)((i / kPermBufs) & 1), abort_flag, err);
+    if (!__all_sync(0xffffffffu, got)) break;
+    if (r >= 0) bulk_store_row(x_perm + (long long)r * row_bytes, buf0 + b * (uint32_t)row_pitch, (uint32_t)row_bytes);
+    bulk_commit();                                        // every lane: an empty group where it stored nothing
+    bulk_wait_read<kPermBufs - kPermDepth>();             // the stores of token i + depth - bufs have read their buffer
+    __syncwarp();
+    issue_load(i + kPermDepth);                           // into that buffer
+  }
+  bulk_wait_all();                                        // the stores are done before the CTA exits
+  if (lane == 0)                                          // after a timeout: let every issued load land
+    for (long long j = i; j < issued; ++j)
+      mbar_wait_drain(bar0 + 8 * (uint32_t)(j % kPermBufs), (uint32_t)((j / kPermBufs) & 1), err);
+}
 
 template <int UNROLL>
 __global__ void __launch_bounds__(256)
@@ -192,7 +276,22 @@ moe_status launch_permute(const void* x, int dtype, int T, int d, int k, const i
                           long long rows_max, void* x_perm, cudaStream_t s) {
   if (T == 0) return MOE_OK;
   const int esz = dtype == MOE_F32 ? 4 : 2;
-  const int nvec = d * esz / 16;
+  const int row_bytes = d * esz;                         // a multiple of 16 (d % 8 == 0)
+  const int row_pitch = (row_bytes + 127) / 128 * 128;
+  const size_t smem = kPermHead + (size_t)kPermWarps * kPermBufs * row_pitch;
+  if (smem <= 232448) {
+    static std::atomic<int> configured[kMaxDevices];   // the limit once, at the largest size a launch may ask
+    const moe_status st = ensure_smem_limit(configured, permute_bulk_kernel, 232448);
+    if (st != MOE_OK) return st;
+    const int per_sm = (int)(232448 / (smem + 1024));
+    const long long ctas = (T + kPermWarps - 1) / kPermWarps;
+    const long long cap = (long long)num_sms() * (per_sm < 1 ? 1 : per_sm);
+    permute_bulk_kernel<<<(unsigned)(ctas < cap ? ctas : cap), 32 * kPermWarps, smem, s>>>(
+        static_cast<const uint8_t*>(x), T, row_bytes, row_pitch, k, row_of, rows_max,
+        static_cast<uint8_t*>(x_perm), err_ptr());
+    return check_launch();
+  }
+  const int nvec = row_bytes / 16;                       // rows too long for the buffers
   permute_kernel<4><<<grid_for_warps(T), 256, 0, s>>>(static_cast<const uint4*>(x), T, nvec, k, row_of,
                                                       rows_max, static_cast<uint4*>(x_perm), err_ptr());
   return check_launch();
