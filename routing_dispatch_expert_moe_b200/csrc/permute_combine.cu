@@ -25,10 +25,10 @@ namespace {
 // t's row into a shared-memory buffer with one bulk copy (global -> shared, completing on
 // the buffer's mbarrier), then lanes 0..k-1 each write it to one kept row of x_perm with
 // one bulk copy back (shared -> global).  Three buffers per warp: the load of the token
-// two ahead is issued once the stores of the token before have read their buffer, so a
-// warp keeps a load and up to two tokens' stores in flight without the SM issuing any
-// per-vector loads or stores.  Row bytes a multiple of 16.  Every wait is bounded; on a
-// timeout the warp stops and drains what it issued.
+// two ahead is issued once the stores of the token before have read their buffer (their
+// writes may still be in flight), so a warp keeps two loads and the latest stores in
+// flight without the SM issuing any per-vector loads or stores.  Row bytes a multiple of
+// 16.  Every wait is bounded; on a timeout the warp stops and drains what it issued.
 // Four warps with three buffers each, two loads issued ahead (4 x 3 with one ahead and
 // 6 x 2 measured within 2% of it; this one was ahead of the per-vector copy on both the
 // 7168- and the 2048-wide rows).
