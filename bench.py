@@ -45,13 +45,27 @@ GATE_UP_TRAFFIC = {
 }
 
 
-def peaks():
-    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+def peaks(path=None):
+    """The roofline denominators: MEASURED_PEAKS.json's figures where it has them (a number,
+    or an object with a numeric "value"), the fallback figures for any it lacks.  Returns
+    the figures and, per figure, "measured" or "fallback"."""
+    p = path or os.path.join(ROOT, "MEASURED_PEAKS.json")
+    d = None
     if os.path.exists(p):
-        with open(p) as f:
-            d = json.load(f)
-        return d, "measured"
-    return dict(FALLBACK_PEAKS), "fallback"
+        try:
+            with open(p) as f:
+                d = json.load(f)
+        except (OSError, ValueError):
+            d = None
+    out, src = {}, {}
+    for key, fb in FALLBACK_PEAKS.items():
+        v = d.get(key) if isinstance(d, dict) else None
+        if isinstance(v, dict):
+            v = v.get("value")
+        ok = isinstance(v, (int, float)) and not isinstance(v, bool) and v > 0
+        out[key] = float(v) if ok else fb
+        src[key] = "measured" if ok else "fallback"
+    return out, src
 
 
 def max_over_ranks(v: float, device=None) -> float:
@@ -447,10 +461,10 @@ def run_ours(args):
     t_tensor, t_hbm = flops / (pk["bf16_tflops"] * 1e12), gu_bytes / (pk["hbm_gbs"] * 1e9)
     if t_tensor >= t_hbm:
         roof = {"bound": "tensor", "achieved": round(flops / (gate_up_ms * 1e-3) / 1e12, 1),
-                "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "peak_source": f"{pk_src} bf16_tflops (burst)"}
+                "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "peak_source": f"{pk_src['bf16_tflops']} bf16_tflops (burst)"}
     else:
         roof = {"bound": "hbm", "achieved": round(gu_bytes / (gate_up_ms * 1e-3) / 1e9, 1),
-                "peak": pk["hbm_gbs"], "unit": "GB/s", "peak_source": f"{pk_src} hbm_gbs"}
+                "peak": pk["hbm_gbs"], "unit": "GB/s", "peak_source": f"{pk_src['hbm_gbs']} hbm_gbs"}
     roof["frac"] = round(roof["achieved"] / roof["peak"], 4)
     roof["algorithmic"] = {"flops": flops, "bytes": gu_bytes, "rows": A, "experts_with_rows": E_act,
                            "tensor_ms": round(t_tensor * 1e3, 4), "hbm_ms": round(t_hbm * 1e3, 4),
