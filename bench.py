@@ -458,10 +458,14 @@ def run_ours(args):
     gather = layer.dispatch_mode == "gather"
     gate_up_ms = stage_ms["timed_gate_up_gather" if gather else "timed_gate_up"]   # inside the timed region
     flops, gu_bytes = gate_up_work(cfg, A, E_act, gather)
-    t_tensor, t_hbm = flops / (pk["bf16_tflops"] * 1e12), gu_bytes / (pk["hbm_gbs"] * 1e9)
+    # the burst GEMM figure for a timed region well under a second, the sustained one (the
+    # power cap settles within about a second of dense work) for longer ones
+    tkey = "bf16_tflops_sustained" if total_ms > 1000.0 else "bf16_tflops"
+    t_tensor, t_hbm = flops / (pk[tkey] * 1e12), gu_bytes / (pk["hbm_gbs"] * 1e9)
     if t_tensor >= t_hbm:
         roof = {"bound": "tensor", "achieved": round(flops / (gate_up_ms * 1e-3) / 1e12, 1),
-                "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "peak_source": f"{pk_src['bf16_tflops']} bf16_tflops (burst)"}
+                "peak": pk[tkey], "unit": "TFLOP/s",
+                "peak_source": f"{pk_src[tkey]} {tkey}" + (" (burst)" if tkey == "bf16_tflops" else "")}
     else:
         roof = {"bound": "hbm", "achieved": round(gu_bytes / (gate_up_ms * 1e-3) / 1e9, 1),
                 "peak": pk["hbm_gbs"], "unit": "GB/s", "peak_source": f"{pk_src['hbm_gbs']} hbm_gbs"}
@@ -629,8 +633,8 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=300)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="c5_stress")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
