@@ -16,6 +16,7 @@
 // order (fp64); stage 2 sums the partials in a fixed lane-strided order followed by a
 // fixed butterfly, so the result does not depend on scheduling.
 #include "common.cuh"
+#include "tc_prims.cuh"
 
 namespace moe {
 namespace {
@@ -42,10 +43,14 @@ constexpr int kSub = kStatsThreads / 32;   // tokens per sub-chunk: one per warp
 // Every score is computed once.  Writes the CTA's P partials [E] and z2 partial.
 __global__ void __launch_bounds__(kStatsThreads, 2)
 stats_partial_kernel(const float* __restrict__ logits, int T, int E, int score, int tokens_per_cta,
-                     double* __restrict__ partP, double* __restrict__ partZ) {
+                     double* __restrict__ partP, double* __restrict__ partZ, int* err) {
   extern __shared__ float s_sc[];            // [kSub][E]
   __shared__ double s_inv[kSub];
   __shared__ double redz[kStatsThreads / 32];
+  __shared__ uint64_t s_bar[kSub];           // one row copy in flight per warp
+  // rows of a whole number of 16-byte pieces arrive by one bulk copy each: the sub-chunk's
+  // kSub rows are all in flight at once instead of a few loads per lane at a time
+  const bool bulk = (E & 3) == 0 && (reinterpret_cast<uintptr_t>(logits) & 15u) == 0;
   const unsigned lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int nwarps = kStatsThreads / 32;
@@ -56,17 +61,35 @@ stats_partial_kernel(const float* __restrict__ logits, int T, int E, int score, 
   double P[kStatsPer];
 #pragma unroll
   for (int q = 0; q < kStatsPer; ++q) P[q] = 0.0;
-  for (long long c0 = t_begin; c0 < t_end; c0 += kSub) {
+  if (threadIdx.x < kSub) mbar_init(smem_u32(&s_bar[threadIdx.x]), 1);
+  fence_mbar_init();
+  __syncthreads();
+  uint32_t phase = 0;
+  for (long long c0 = t_begin; c0 < t_end; c0 += kSub, phase ^= 1u) {
     const int n = (int)min((long long)kSub, t_end - c0);
     if (warp < n) {
       const float* row = logits + (c0 + warp) * E;
       float* srow = s_sc + warp * E;
       float mf = -INFINITY;
+      if (bulk) {
+        const uint32_t bar = smem_u32(&s_bar[warp]);
+        if (lane == 0) {
+          fence_proxy_async_smem();          // the previous sub-chunk's reads and writes of the row
+          mbar_expect_tx(bar, (uint32_t)E * 4u);
+          asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                       ::"r"(smem_u32(srow)), "l"(row), "r"((uint32_t)E * 4u), "r"(bar)
+                       : "memory");
+        }
+        mbar_wait_drain(bar, phase, err);    // bounded
 #pragma unroll 4
-      for (int e = lane; e < E; e += 32) {
-        const float l = __ldg(row + e);
-        srow[e] = l;
-        mf = fmaxf(mf, l);
+        for (int e = lane; e < E; e += 32) mf = fmaxf(mf, srow[e]);
+      } else {
+#pragma unroll 4
+        for (int e = lane; e < E; e += 32) {
+          const float l = __ldg(row + e);
+          srow[e] = l;
+          mf = fmaxf(mf, l);
+        }
       }
 #pragma unroll
       for (int o = 16; o; o >>= 1) mf = fmaxf(mf, __shfl_xor_sync(0xffffffffu, mf, o));
@@ -248,7 +271,7 @@ moe_status launch_router_stats(const float* logits, const int32_t* counts, const
   const size_t smem = (size_t)kSub * E * sizeof(float);    // up to 64 KB (E = 1024)
   moe_status st0 = ensure_smem_limit(configured, stats_partial_kernel, (size_t)kSub * 1024 * sizeof(float));
   if (st0 != MOE_OK) return st0;
-  stats_partial_kernel<<<parts, kStatsThreads, smem, s>>>(logits, T, E, score, tpc, pP, pZ);
+  stats_partial_kernel<<<parts, kStatsThreads, smem, s>>>(logits, T, E, score, tpc, pP, pZ, err_ptr());
   moe_status st = check_launch();
   if (st != MOE_OK) return st;
   stats_reduce_kernel<<<(E + 31) / 32, 256, 0, s>>>(pP, parts, E, pSum);
